@@ -1,0 +1,66 @@
+"""Numerics behind the prefill path's activation format (CPU only).
+
+The prefill path feeds activations to FP8 tensor cores.  The layer's
+tolerance (relative L2 <= 5e-3 against the exact layer) rules out a single
+e4m3 code per activation: three mantissa bits give a few percent error per
+element.  The reading taken is a two-term split with one shared fp32 scale
+per (row, 128-column block):
+
+    s = amax/448,  q_hi = e4m3(v/s),  q_lo = e4m3(v/s - q_hi),  v ~ s*(q_hi + q_lo)
+
+Because both terms share s, one accumulator takes both products.  This test
+measures one 35B-shaped expert (H = 2048, I = 512) three ways with the
+oracle's own e4m3 codec and numpy matmuls on the dequantised weights.
+"""
+import numpy as np
+import scipy.special
+import torch
+
+import moe_inputs as mi
+import oracle
+
+_DEC = np.array([oracle.e4m3_decode(c) for c in range(256)])
+
+
+def _enc(a):
+    return np.array([oracle.e4m3_encode(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def _single(v):
+    b = v.reshape(v.shape[0], -1, 128)
+    s = np.abs(b).max(axis=2, keepdims=True) / 448.0
+    s[s == 0] = 1.0
+    return (_DEC[_enc(b / s)] * s).reshape(v.shape)
+
+
+def _hilo(v):
+    b = v.reshape(v.shape[0], -1, 128)
+    s = np.abs(b).max(axis=2, keepdims=True) / 448.0
+    s[s == 0] = 1.0
+    hi = _DEC[_enc(b / s)]
+    lo = _DEC[_enc(b / s - hi)]
+    return ((hi + lo) * s).reshape(v.shape)
+
+
+def test_single_fp8_activations_fail_and_hilo_split_passes():
+    d = mi.QWEN36_35B_A3B
+    H, I = d.hidden, d.inter
+    slab, sc = mi.expert_slab(d, seed=0, e=0)
+    n13 = (2 * I // 128) * (H // 128)
+    dec = lambda q, s: (torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn)
+                        .to(torch.float64).numpy() * np.kron(s.astype(np.float64), np.ones((128, 128))))
+    W13 = dec(slab[: 2 * I * H].reshape(2 * I, H), sc[:n13].reshape(2 * I // 128, H // 128))
+    W2 = dec(slab[2 * I * H:].reshape(H, I), sc[n13:].reshape(H // 128, I // 128))
+    x = oracle.bf16_bits_to_f64(mi.make_x(d, 8, seed=0))
+
+    def layer(fx, fh):
+        gu = fx(x) @ W13.T
+        h = gu[:, :I] * scipy.special.expit(gu[:, :I]) * gu[:, I:]
+        return fh(h) @ W2.T
+
+    exact = layer(lambda v: v, lambda v: v)
+    rel = lambda y: np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    e_single = rel(layer(_single, _single))
+    e_hilo = rel(layer(_hilo, _hilo))
+    assert e_single > 5e-3          # misses the tolerance on its own
+    assert e_hilo < 2e-3            # leaves room for the bf16 output rounding
