@@ -1,0 +1,153 @@
+/*
+ * moe_ffn.h -- C ABI of the B200 (sm_100a) top-k mixture-of-experts FFN layer.
+ *
+ * The operation (one decode or prefill step of a Qwen3.5/3.6-style MoE FFN):
+ *
+ *   l[t,e]  = sum_h x[t,h] * Wr[e,h]  (+ bias[e])            router GEMV (bf16)
+ *   idx[t]  = the k largest l[t,:] (ties: lower expert first), by descending logit
+ *   w[t,r]  = exp(l[t,idx_r]) / sum_j exp(l[t,idx_j])         softmax over the k chosen
+ *   z[t]    = sum_h x[t,h] * g[h],  gs[t] = sigmoid(z[t])      shared-expert gate
+ *   E_e(x)  = W2_e ( silu(W13_e[:I] x) * W13_e[I:] x )         SwiGLU expert, FP8 weights
+ *   out[t]  = sum_r w[t,r] E_{idx_r}(x_t) + gs[t] E_shared(x_t) (+ residual[t]),
+ *             rounded once to bf16.
+ *
+ * Passages it follows: the "Qwen3.6-35B-A3B-FP8 on NVIDIA GB10" blueprint page
+ * (Kernels table: dense_gemv_bf16 router, moe_topk_softmax, gate_up and
+ * silu_down FP8 expert kernels with the shared expert fused, weighted-sum
+ * blend; Precision table: fp8/block128x128 weights against bf16 and f32
+ * activations, f32,i32 top-k outputs); the "colibri #1992" PR page (frame A2:
+ * the shared expert together with its gate; a warp per output row with 16-byte
+ * lane loads and the activation in shared memory for decode GEMVs); the
+ * "Neurarch Qwen3-8B" page (SwiGLU gate_proj/up_proj [I,H], down_proj [H,I]).
+ *
+ * Dimensions: H, I and Is must be multiples of 128; 1 <= k <= min(E, 32);
+ * E <= 1024.
+ *
+ * Layouts (all row-major, reduction dimension contiguous, device memory):
+ *   x, residual, out     bf16 [rows, H]
+ *   router_w             bf16 [E, H]
+ *   shared_gate          bf16 [H]
+ *   router_bias          fp32 [E]                       (nullable)
+ *   expert_w8            e4m3 bytes, E slabs of 3*I*H:  [W13 (2I x H) | W2 (H x I)];
+ *                        W13 holds the gate rows, then the up rows
+ *   expert_scales        fp32, E slabs of (2I/128)(H/128) + (H/128)(I/128):
+ *                        [s13 (2I/128 x H/128) | s2 (H/128 x I/128)];
+ *                        weight value = e4m3(code) * scale of its 128x128 block
+ *   shared_w             one slab of the same layout with Is in place of I
+ *   topk_idx / topk_w    int32 / fp32 [rows, k], descending weight
+ *   shared_gate_sig      fp32 [rows]
+ *
+ * Ownership and execution: the caller owns every buffer and the stream.  The
+ * library allocates no device memory; it uses the caller's workspace
+ * (moe_workspace_bytes) and keeps one host-side table of per-device
+ * properties.  Every call is asynchronous on `stream` (a cudaStream_t; NULL
+ * = the legacy default stream) and returns after enqueueing.  Device
+ * pointers must be 16-byte aligned.  `out` may alias `residual`; no other
+ * output may alias an input.  A workspace serves one stream at a time: calls
+ * that overlap on the device must use different workspaces.  A fresh
+ * workspace must be zero-filled once (moe_workspace_init) before its first
+ * use; the library leaves it reusable after every call it completes.
+ *
+ * Errors: every call returns a status (MOE_OK = 0, else a negative code).
+ * Argument errors are detected on the host before anything is enqueued.
+ * A CUDA error is sticky, as a lost device is in the pages' CUDA chain: after
+ * MOE_ECUDA every call returns MOE_ECUDA until moe_reset_status() (after
+ * which the workspace must be re-initialised).
+ */
+#ifndef MOE_FFN_H
+#define MOE_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_EINVAL -1        /* null pointer, misaligned pointer, rows < 0, bad path */
+#define MOE_EUNSUPPORTED -2  /* H, I or Is not a multiple of 128, k > E, k > 32, E > 1024 */
+#define MOE_EWORKSPACE -3    /* workspace smaller than moe_workspace_bytes(d, rows) */
+#define MOE_ECUDA -4         /* a CUDA launch or runtime error (sticky) */
+
+#define MOE_PATH_AUTO 0      /* decode kernels for rows <= MOE_DECODE_MAX_ROWS, else prefill */
+#define MOE_PATH_DECODE 1    /* warp-per-row FP8 GEMVs with expert dedup */
+#define MOE_PATH_PREFILL 2   /* token permute -> tcgen05 FP8 grouped GEMMs -> unpermute */
+#define MOE_DECODE_MAX_ROWS 64
+
+typedef struct moe_dims {
+    int32_t hidden;       /* H  */
+    int32_t n_experts;    /* E  */
+    int32_t top_k;        /* k  */
+    int32_t inter;        /* I  : routed expert intermediate size */
+    int32_t shared_inter; /* Is : shared expert intermediate size */
+} moe_dims;
+
+/* One expert's weights in the slab layout above (used for the shared expert). */
+typedef struct moe_fp8_expert {
+    const uint8_t *w8;    /* 3*Is*H e4m3 codes */
+    const float *scales;  /* (2Is/128)(H/128) + (H/128)(Is/128) fp32 scales */
+} moe_fp8_expert;
+
+/* Bytes of workspace needed by any call with rows <= max_rows on either path.
+ * Returns 0 for invalid or unsupported dims or max_rows < 0. */
+MOE_API size_t moe_workspace_bytes(const moe_dims *d, int32_t max_rows);
+
+/* Zero-fill a workspace on `stream` (needed once per fresh workspace). */
+MOE_API int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Router GEMV, shared-gate sigmoid and top-k softmax for `rows` rows of x.
+ * Outputs topk_idx [rows, k] (int32), topk_w [rows, k] (fp32, renormalised
+ * over the k chosen, descending) and shared_gate_sig [rows] (fp32).
+ * router_bias may be NULL.  rows == 0 is a no-op. */
+MOE_API int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows,
+                    const uint16_t *router_w, const float *router_bias,
+                    const uint16_t *shared_gate, int32_t *topk_idx, float *topk_w,
+                    float *shared_gate_sig, void *ws, size_t ws_bytes, void *stream);
+
+/* The whole layer step: out = sum_r w_r E_{idx_r}(x) + sigmoid(g.x) E_shared(x)
+ * (+ residual), bf16 [rows, H].  residual and router_bias may be NULL.
+ * Chooses the decode path for rows <= MOE_DECODE_MAX_ROWS, else prefill.
+ * rows == 0 is a no-op. */
+MOE_API int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows,
+                    const uint16_t *router_w, const uint8_t *expert_w8,
+                    const float *expert_scales, const moe_fp8_expert *shared_w,
+                    const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
+                    const float *router_bias, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_ffn_forward with an explicit path (MOE_PATH_*) and optional copies of
+ * the routing it used (each nullable): topk_idx [rows, k], topk_w [rows, k],
+ * shared_gate_sig [rows].  The decode path accepts any rows but is sized for
+ * rows <= MOE_DECODE_MAX_ROWS. */
+MOE_API int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows,
+                         const uint16_t *router_w, const uint8_t *expert_w8,
+                         const float *expert_scales, const moe_fp8_expert *shared_w,
+                         const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
+                         const float *router_bias, void *ws, size_t ws_bytes, void *stream,
+                         int32_t path, int32_t *topk_idx, float *topk_w,
+                         float *shared_gate_sig);
+
+/* Sticky status: MOE_OK, or MOE_ECUDA after a CUDA error. */
+MOE_API int moe_status(void);
+/* Clear the sticky status (also clears a pending CUDA error of this thread). */
+MOE_API void moe_reset_status(void);
+/* Static, human-readable text for a status code. */
+MOE_API const char *moe_status_string(int status);
+
+/* Host-side fault injection, after the pages' fake device loss: the n-th
+ * next call (n >= 1) fails with MOE_ECUDA before enqueueing anything, as if
+ * a launch had failed, and sets the sticky status.  n = 0 disarms.  Nothing
+ * runs on the device. */
+MOE_API void moe_debug_inject_fault(int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FFN_H */

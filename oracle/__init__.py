@@ -57,6 +57,7 @@ def _load():
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_quantize_blocks.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, P]
         lib.oracle_topk.argtypes = [P, ctypes.c_int32, ctypes.c_int32, P, P]
+        lib.oracle_router_topk.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, P, P, P, P, P, P, P]
         lib.oracle_expert_ffn.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, P, P]
         lib.oracle_moe_forward.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, P, P, P, P, P,
                                            P, P, P, P, P, P, P, P, P, ctypes.c_int32]
@@ -126,6 +127,24 @@ def topk(logits: np.ndarray, k: int):
     w = np.empty(k, dtype=np.float64)
     _check(_load().oracle_topk(_ptr(l), l.shape[0], k, _ptr(idx), _ptr(w)), "oracle_topk")
     return idx, w
+
+
+def router_topk(d, x, router_w, shared_gate, router_bias=None):
+    """Router step alone -> (logits float64 [rows, E], idx int32 [rows, k], w float64 [rows, k],
+    gate_sig float64 [rows])."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    rows = x.shape[0]
+    logits = np.empty((rows, d.n_experts), dtype=np.float64)
+    idx = np.empty((rows, d.top_k), dtype=np.int32)
+    w = np.empty((rows, d.top_k), dtype=np.float64)
+    gs = np.empty(rows, dtype=np.float64)
+    dims = _dims(d)
+    _check(_load().oracle_router_topk(
+        ctypes.byref(dims), _ptr(x), rows, _ptr(np.ascontiguousarray(router_w, dtype=np.uint16)),
+        _ptr(None if router_bias is None else np.ascontiguousarray(router_bias, dtype=np.float32)),
+        _ptr(np.ascontiguousarray(shared_gate, dtype=np.uint16)), _ptr(logits), _ptr(idx), _ptr(w),
+        _ptr(gs)), "oracle_router_topk")
+    return logits, idx, w, gs
 
 
 def expert_ffn(w8: np.ndarray, scales: np.ndarray, H: int, I: int, x: np.ndarray) -> np.ndarray:

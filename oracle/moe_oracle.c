@@ -219,6 +219,26 @@ int oracle_topk(const double *l, int32_t E, int32_t k, int32_t *idx, double *w)
     return 0;
 }
 
+/* Router step alone for `rows` rows: logits [rows, E], top-k idx/w [rows, k]
+ * and sigmoid(g . x) [rows], by the same definitions as the layer below. */
+int oracle_router_topk(const oracle_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                       const float *router_bias, const uint16_t *shared_gate, double *logits,
+                       int32_t *idx, double *w, double *gate_sig)
+{
+    if (!d || !x || !router_w || !shared_gate || !logits || !idx || !w || !gate_sig || rows < 0) return -1;
+    const int E = d->n_experts, K = d->top_k;
+    if (K < 1 || K > E) return -2;
+    for (int t = 0; t < rows; ++t) {
+        double z;
+        router_row(d, x + (int64_t)t * d->hidden, router_w, router_bias, shared_gate,
+                   logits + (int64_t)t * E, &z);
+        int st = oracle_topk(logits + (int64_t)t * E, E, K, idx + (int64_t)t * K, w + (int64_t)t * K);
+        if (st) return st;
+        gate_sig[t] = sigmoid(z);
+    }
+    return 0;
+}
+
 /* One SwiGLU expert on one row, from its slab [W13: 2I x H | W2: H x I]
  * (e4m3 codes) and scales [s13: 2I/128 x H/128 | s2: H/128 x I/128]:
  *   gu = W13 x;  h_j = silu(gu_j) * gu_{I+j};  y = W2 h. */

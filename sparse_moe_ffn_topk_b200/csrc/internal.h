@@ -1,0 +1,105 @@
+// internal.h -- host-side pieces shared by the C ABI and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe_ffn.h"
+
+namespace moe {
+
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;
+constexpr int kCounters = 1024;         // int32 counters at the head of the workspace
+constexpr int kCtrRouter = 0;           // last-arriver counter of the router kernel
+constexpr int kCtrBlend = 64;           // first of the down/blend per-chunk counters
+constexpr int kDownRowsPerItem = 32;    // output rows per down work item (blend chunk)
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Decode-path workspace, carved from the caller's buffer.
+struct DecodeLayout {
+    size_t counters, logits, topk_idx, topk_w, gsig, plan, h_routed, h_shared, yslot, total;
+};
+
+inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
+{
+    DecodeLayout L{};
+    const int64_t E = d.n_experts, K = d.top_k, H = d.hidden, I = d.inter, Is = d.shared_inter;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+    L.counters = take(sizeof(int32_t) * kCounters);
+    L.logits = take(sizeof(float) * rows * (E + 1));
+    L.topk_idx = take(sizeof(int32_t) * rows * K);
+    L.topk_w = take(sizeof(float) * rows * K);
+    L.gsig = take(sizeof(float) * rows);
+    // plan: n_active | active_expert[E] | active_off[E+1] | pair_list[rows*K]
+    L.plan = take(sizeof(int32_t) * (1 + E + (E + 1) + rows * K));
+    L.h_routed = take(sizeof(float) * rows * K * I);
+    L.h_shared = take(sizeof(float) * rows * Is);
+    L.yslot = take(sizeof(float) * rows * (K + 1) * H);
+    L.total = o;
+    return L;
+}
+
+// Device properties cached per device.
+struct DeviceInfo {
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    size_t max_smem_optin = 0;
+};
+const DeviceInfo &device_info();
+
+// ------------------------------------------------------------ decode path
+struct RouterLaunch {
+    const moe_dims *d;
+    const uint16_t *x;
+    int32_t rows;
+    const uint16_t *router_w;
+    const float *router_bias;
+    const uint16_t *shared_gate;
+    int32_t *topk_idx;
+    float *topk_w;
+    float *gsig;
+    float *logits;   // workspace
+    int32_t *counters;
+    int32_t *plan;   // nullptr: no plan
+};
+cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s);
+
+struct ExpertsLaunch {
+    const moe_dims *d;
+    const uint16_t *x;
+    int32_t rows;
+    const uint8_t *expert_w8;
+    const float *expert_scales;
+    const uint8_t *shared_w8;
+    const float *shared_scales;
+    const uint16_t *residual;
+    uint16_t *out;
+    const int32_t *topk_idx;
+    const float *topk_w;
+    const float *gsig;
+    const int32_t *plan;
+    float *h_routed;
+    float *h_shared;
+    float *yslot;
+    int32_t *counters;
+};
+cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s);
+
+// ------------------------------------------------------------ prefill path
+// Bytes of workspace for `rows` rows on either path.
+size_t workspace_bytes(const moe_dims &d, int64_t rows);
+// Whether the prefill path is built into this library.
+bool prefill_available();
+// The prefill path (router GEMM, permute, grouped FP8 GEMMs, unpermute).
+// Returns a MOE_* status; launch errors come back as MOE_ECUDA.
+int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                    const uint8_t *expert_w8, const float *expert_scales, const uint8_t *shared_w8,
+                    const float *shared_scales, const uint16_t *shared_gate, uint16_t *out,
+                    const uint16_t *residual, const float *router_bias, void *ws, cudaStream_t s,
+                    int32_t *topk_idx_out, float *topk_w_out, float *gsig_out);
+
+}  // namespace moe

@@ -1,0 +1,253 @@
+// moe_api.cu -- the C ABI declared in include/moe_ffn.h.
+//
+// Host side only: argument checks, workspace carving, path selection, the
+// sticky status and the host fault knob.  Every step of the layer runs in
+// the kernels of decode.cu and prefill.cu.
+#include <atomic>
+#include <mutex>
+
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+std::atomic<int> g_status{MOE_OK};
+std::atomic<int> g_fault_countdown{0};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+bool g_dev_ready[64] = {};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const moe_dims *d)
+{
+    if (!d) return MOE_EINVAL;
+    if (d->hidden <= 0 || d->n_experts <= 0 || d->top_k <= 0 || d->inter <= 0 || d->shared_inter <= 0)
+        return MOE_EUNSUPPORTED;
+    if (d->hidden % 128 || d->inter % 128 || d->shared_inter % 128) return MOE_EUNSUPPORTED;
+    if (d->top_k > d->n_experts || d->top_k > kMaxTopK || d->n_experts > kMaxExperts) return MOE_EUNSUPPORTED;
+    if (d->hidden / kDownRowsPerItem > kCounters - kCtrBlend) return MOE_EUNSUPPORTED;
+    return MOE_OK;
+}
+
+// Common entry: sticky status and the host fault knob.
+int enter()
+{
+    if (g_status.load() != MOE_OK) return MOE_ECUDA;
+    int n = g_fault_countdown.load();
+    while (n > 0) {
+        if (g_fault_countdown.compare_exchange_weak(n, n - 1)) {
+            if (n == 1) {
+                g_status.store(MOE_ECUDA);
+                return MOE_ECUDA;
+            }
+            break;
+        }
+    }
+    return MOE_OK;
+}
+
+int finish(cudaError_t e)
+{
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        g_status.store(MOE_ECUDA);
+        return MOE_ECUDA;
+    }
+    return MOE_OK;
+}
+
+}  // namespace
+
+const DeviceInfo &device_info()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_dev_ready[dev]) {
+        DeviceInfo &i = g_dev[dev];
+        cudaDeviceGetAttribute(&i.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&i.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&i.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+        int smem = 0;
+        cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        i.max_smem_optin = (size_t)smem;
+        if (i.sm_count <= 0) i.sm_count = 1;
+        g_dev_ready[dev] = true;
+    }
+    return g_dev[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_dims *d, int32_t max_rows)
+{
+    if (check_dims(d) != MOE_OK || max_rows < 0) return 0;
+    return workspace_bytes(*d, max_rows < 1 ? 1 : max_rows);
+}
+
+int moe_workspace_init(void *ws, size_t ws_bytes, void *stream)
+{
+    int st = enter();
+    if (st) return st;
+    if (!ws && ws_bytes) return MOE_EINVAL;
+    if (!ws_bytes) return MOE_OK;
+    return finish(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                    const float *router_bias, const uint16_t *shared_gate, int32_t *topk_idx,
+                    float *topk_w, float *shared_gate_sig, void *ws, size_t ws_bytes, void *stream)
+{
+    int st = check_dims(d);
+    if (st) return st;
+    if (rows < 0) return MOE_EINVAL;
+    if (!x || !router_w || !shared_gate || !topk_idx || !topk_w || !shared_gate_sig || !ws) return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(shared_gate) || !aligned16(ws) ||
+        (router_bias && !aligned16(router_bias)) || !aligned16(topk_idx) || !aligned16(topk_w) ||
+        !aligned16(shared_gate_sig))
+        return MOE_EINVAL;
+    if (ws_bytes < workspace_bytes(*d, rows < 1 ? 1 : rows)) return MOE_EWORKSPACE;
+    st = enter();
+    if (st) return st;
+    if (rows == 0) return MOE_OK;
+    const DecodeLayout L = decode_layout(*d, rows);
+    char *base = static_cast<char *>(ws);
+    RouterLaunch a;
+    a.d = d;
+    a.x = x;
+    a.rows = rows;
+    a.router_w = router_w;
+    a.router_bias = router_bias;
+    a.shared_gate = shared_gate;
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.gsig = shared_gate_sig;
+    a.logits = reinterpret_cast<float *>(base + L.logits);
+    a.counters = reinterpret_cast<int32_t *>(base + L.counters);
+    a.plan = nullptr;
+    return finish(launch_router_topk(a, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                         const uint8_t *expert_w8, const float *expert_scales,
+                         const moe_fp8_expert *shared_w, const uint16_t *shared_gate, uint16_t *out,
+                         const uint16_t *residual, const float *router_bias, void *ws, size_t ws_bytes,
+                         void *stream, int32_t path, int32_t *topk_idx_out, float *topk_w_out,
+                         float *shared_gate_sig_out)
+{
+    int st = check_dims(d);
+    if (st) return st;
+    if (rows < 0) return MOE_EINVAL;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_EINVAL;
+    if (!x || !router_w || !expert_w8 || !expert_scales || !shared_w || !shared_w->w8 ||
+        !shared_w->scales || !shared_gate || !out || !ws)
+        return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(expert_w8) || !aligned16(expert_scales) ||
+        !aligned16(shared_w->w8) || !aligned16(shared_w->scales) || !aligned16(shared_gate) ||
+        !aligned16(out) || !aligned16(ws) || (residual && !aligned16(residual)) ||
+        (router_bias && !aligned16(router_bias)) || (topk_idx_out && !aligned16(topk_idx_out)) ||
+        (topk_w_out && !aligned16(topk_w_out)) || (shared_gate_sig_out && !aligned16(shared_gate_sig_out)))
+        return MOE_EINVAL;
+    if (static_cast<const void *>(out) == static_cast<const void *>(x)) return MOE_EINVAL;
+    if (ws_bytes < workspace_bytes(*d, rows < 1 ? 1 : rows)) return MOE_EWORKSPACE;
+    st = enter();
+    if (st) return st;
+    if (rows == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (path == MOE_PATH_AUTO)
+        path = (rows <= MOE_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
+    if (path == MOE_PATH_PREFILL) {
+        int rc = prefill_forward(*d, x, rows, router_w, expert_w8, expert_scales, shared_w->w8,
+                                 shared_w->scales, shared_gate, out, residual, router_bias, ws, s,
+                                 topk_idx_out, topk_w_out, shared_gate_sig_out);
+        if (rc == MOE_ECUDA) g_status.store(MOE_ECUDA);
+        return rc;
+    }
+
+    const DecodeLayout L = decode_layout(*d, rows);
+    char *base = static_cast<char *>(ws);
+    int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
+    int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
+    float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
+    float *gs = shared_gate_sig_out ? shared_gate_sig_out : reinterpret_cast<float *>(base + L.gsig);
+    int32_t *plan = reinterpret_cast<int32_t *>(base + L.plan);
+
+    RouterLaunch ra;
+    ra.d = d;
+    ra.x = x;
+    ra.rows = rows;
+    ra.router_w = router_w;
+    ra.router_bias = router_bias;
+    ra.shared_gate = shared_gate;
+    ra.topk_idx = tidx;
+    ra.topk_w = tw;
+    ra.gsig = gs;
+    ra.logits = reinterpret_cast<float *>(base + L.logits);
+    ra.counters = counters;
+    ra.plan = plan;
+    cudaError_t e = launch_router_topk(ra, s);
+    if (e != cudaSuccess) return finish(e);
+
+    ExpertsLaunch ea;
+    ea.d = d;
+    ea.x = x;
+    ea.rows = rows;
+    ea.expert_w8 = expert_w8;
+    ea.expert_scales = expert_scales;
+    ea.shared_w8 = shared_w->w8;
+    ea.shared_scales = shared_w->scales;
+    ea.residual = residual;
+    ea.out = out;
+    ea.topk_idx = tidx;
+    ea.topk_w = tw;
+    ea.gsig = gs;
+    ea.plan = plan;
+    ea.h_routed = reinterpret_cast<float *>(base + L.h_routed);
+    ea.h_shared = reinterpret_cast<float *>(base + L.h_shared);
+    ea.yslot = reinterpret_cast<float *>(base + L.yslot);
+    ea.counters = counters;
+    return finish(launch_decode_experts(ea, s));
+}
+
+int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                    const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                    const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
+                    const float *router_bias, void *ws, size_t ws_bytes, void *stream)
+{
+    return moe_ffn_forward_path(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out,
+                                residual, router_bias, ws, ws_bytes, stream, MOE_PATH_AUTO, nullptr,
+                                nullptr, nullptr);
+}
+
+int moe_status(void) { return g_status.load(); }
+
+void moe_reset_status(void)
+{
+    cudaGetLastError();
+    g_status.store(MOE_OK);
+    g_fault_countdown.store(0);
+}
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument (null or misaligned pointer, negative rows, bad path)";
+    case MOE_EUNSUPPORTED: return "unsupported dimensions (H, I, Is multiples of 128; k <= min(E, 32); E <= 1024)";
+    case MOE_EWORKSPACE: return "workspace too small (see moe_workspace_bytes)";
+    case MOE_ECUDA: return "CUDA error (sticky until moe_reset_status)";
+    default: return "unknown status";
+    }
+}
+
+void moe_debug_inject_fault(int32_t n) { g_fault_countdown.store(n > 0 ? n : 0); }
+
+}  // extern "C"

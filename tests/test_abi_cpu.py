@@ -1,0 +1,109 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol ``include/*.h`` declares, and its host-side checks (dims, nulls,
+alignment, workspace size, the fault knob) answer without touching CUDA."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import moe_inputs as mi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+moe = pytest.importorskip("sparse_moe_ffn_topk_b200")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_moe_ffn_topk_b200 import build
+    build.build()
+    return moe.lib()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names |= set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert names, "no declarations found"
+    assert names == set(moe.EXPORTED) | (names - set(moe.EXPORTED))
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_binding_names_match_header():
+    assert set(moe.EXPORTED) == declared_symbols()
+
+
+def D(h=2048, e=256, k=8, i=512, s=512):
+    return moe.MoeDims(h, e, k, i, s)
+
+
+def test_workspace_bytes(L):
+    d = D()
+    a = moe.workspace_bytes(d, 1)
+    b = moe.workspace_bytes(d, 64)
+    assert 0 < a < b
+    assert moe.workspace_bytes(D(h=2000), 1) == 0          # not a multiple of 128
+    assert moe.workspace_bytes(D(k=33, e=64), 1) == 0      # k > 32
+    assert moe.workspace_bytes(D(k=9, e=8), 1) == 0        # k > E
+    assert moe.workspace_bytes(D(e=1025), 1) == 0          # E > 1024
+    assert moe.workspace_bytes(d, -1) == 0
+
+
+FAKE = 1 << 20  # an aligned, never dereferenced address
+
+
+def fwd(L, d, rows=1, x=FAKE, out=FAKE + 4096, ws=FAKE, ws_bytes=None, shared=True, path=0):
+    sh = moe.MoeFp8Expert(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE)) if shared else None
+    if ws_bytes is None:
+        ws_bytes = moe.workspace_bytes(d, max(rows, 1))
+    P = lambda a: ctypes.c_void_p(a) if a else None
+    return L.moe_ffn_forward_path(ctypes.byref(d), P(x), rows, P(FAKE), P(FAKE), P(FAKE),
+                                  ctypes.byref(sh) if sh else None, P(FAKE), P(out), None, None, P(ws),
+                                  ws_bytes, None, path, None, None, None)
+
+
+def test_argument_checks_on_host(L):
+    d = D()
+    assert fwd(L, d, x=0) == moe.MOE_EINVAL
+    assert fwd(L, d, x=FAKE + 2) == moe.MOE_EINVAL          # misaligned
+    assert fwd(L, d, shared=False) == moe.MOE_EINVAL
+    assert fwd(L, d, rows=-1) == moe.MOE_EINVAL
+    assert fwd(L, d, path=7) == moe.MOE_EINVAL
+    assert fwd(L, d, out=FAKE) == moe.MOE_EINVAL            # out aliases x
+    assert fwd(L, D(i=500)) == moe.MOE_EUNSUPPORTED
+    assert fwd(L, d, ws_bytes=16) == moe.MOE_EWORKSPACE
+    assert fwd(L, d, rows=0) == moe.MOE_OK                   # no-op, no CUDA call
+    assert L.moe_router_topk(ctypes.byref(d), None, 1, None, None, None, None, None, None, None, 0,
+                             None) == moe.MOE_EINVAL
+
+
+def test_fault_knob_is_sticky_until_reset(L):
+    d = D()
+    moe.reset_status()
+    moe.debug_inject_fault(2)
+    assert fwd(L, d, rows=0) == moe.MOE_OK        # first call passes (a no-op)
+    assert fwd(L, d, rows=0) == moe.MOE_ECUDA     # second call: the injected loss
+    assert moe.status() == moe.MOE_ECUDA
+    assert fwd(L, d, rows=0) == moe.MOE_ECUDA     # sticky
+    moe.reset_status()
+    assert moe.status() == moe.MOE_OK
+    assert fwd(L, d, rows=0) == moe.MOE_OK
+
+
+def test_status_strings(L):
+    for c in (0, -1, -2, -3, -4, -99):
+        assert isinstance(moe.status_string(c), str) and moe.status_string(c)
+
+
+def test_dims_match_input_generator():
+    for d in (mi.TINY, mi.QWEN36_35B_A3B, mi.QWEN35_397B_A17B):
+        assert moe.workspace_bytes(d, 1) > 0

@@ -1,0 +1,169 @@
+"""GPU parity of the decode path against the CPU oracle, through the C ABI.
+
+Covers the tiny workload, the Qwen3.6-35B-A3B-shaped layer at rows 1, 2, 8,
+16, 32, 64, and the Qwen3.5-397B-A17B-shaped layer at rows 1 and 32 (all at
+full size), plus odd shapes, residual, router bias, repeated calls on one
+workspace, batch invariance, rows = 0 and the router-only entry point.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+moe = pytest.importorskip("sparse_moe_ffn_topk_b200")
+
+
+@pytest.fixture(scope="session")
+def layer35():
+    return mi.make_layer(mi.QWEN36_35B_A3B, seed=0)
+
+
+@pytest.fixture(scope="session")
+def dev35(layer35):
+    return P.device_weights(layer35)
+
+
+def run_forward(case, dev=None, path=moe.MOE_PATH_AUTO, residual_inplace=False):
+    d = case.dims
+    dev = dev or P.device_weights(case.layer)
+    rows = case.x.shape[0]
+    x = P.bf16_tensor(case.x)
+    res = P.bf16_tensor(case.residual) if case.residual is not None else None
+    out = res if (residual_inplace and res is not None) else torch.empty(rows, d.hidden, dtype=torch.bfloat16,
+                                                                          device="cuda")
+    idx = torch.empty(rows, d.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(rows, d.top_k, dtype=torch.float32, device="cuda")
+    gs = torch.empty(rows, dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(d, rows)
+    moe.ffn_forward_path(d, x, dev["router_w"], dev["expert_w8"], dev["expert_scales"], dev["shared_w8"],
+                         dev["shared_scales"], dev["shared_gate"], out, ws, path=path, residual=res,
+                         router_bias=dev["router_bias"], topk_idx=idx, topk_w=w, shared_gate_sig=gs)
+    torch.cuda.synchronize()
+    return P.bf16_to_f64(out), idx.cpu().numpy(), w.cpu().numpy(), gs.cpu().numpy()
+
+
+def check(case, dev=None, **kw):
+    out, idx, w, gs = run_forward(case, dev, **kw)
+    _, oidx, ow, ogs = oracle.router_topk(case.dims, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    return P.compare_output(case, out, idx)
+
+
+def test_tiny():
+    d = mi.TINY
+    case = P.build_case(d, 4, all_experts=True)
+    check(case)
+
+
+@pytest.mark.parametrize("rows", [1, 2, 8, 16, 32, 64])
+def test_qwen36_35b_decode(rows, layer35, dev35):
+    case = P.build_case(mi.QWEN36_35B_A3B, rows, layer=layer35)
+    rel, mx = check(case, dev35)
+    assert rel < 5e-3
+
+
+@pytest.fixture(scope="session")
+def case397():
+    d = mi.QWEN35_397B_A17B
+    rw, g, _ = mi.make_router(d, 0)
+    need = set()
+    xs = {r: mi.make_x(d, r, seed=0, stream=r) for r in (1, 32)}
+    for r, x in xs.items():
+        lg, _, _, _ = oracle.router_topk(d, x, rw, g)
+        need |= P.needed_experts(lg, d.top_k)
+    layer = mi.make_layer(d, seed=0, experts=need)
+    return layer, P.device_weights(layer)
+
+
+@pytest.mark.parametrize("rows", [1, 32])
+def test_qwen35_397b_decode(rows, case397):
+    layer, dev = case397
+    case = P.build_case(mi.QWEN35_397B_A17B, rows, layer=layer)
+    check(case, dev)
+
+
+@pytest.mark.parametrize("dims,rows", [
+    (mi.LayerDims(hidden=384, n_experts=12, top_k=3, inter=256, shared_inter=128), 5),
+    (mi.LayerDims(hidden=640, n_experts=40, top_k=7, inter=384, shared_inter=640), 3),
+    (mi.LayerDims(hidden=256, n_experts=16, top_k=16, inter=128, shared_inter=128), 2),   # k = E
+    (mi.LayerDims(hidden=128, n_experts=1, top_k=1, inter=128, shared_inter=128), 1),     # one expert
+    (mi.LayerDims(hidden=8192, n_experts=4, top_k=2, inter=128, shared_inter=256), 3),    # two K segments
+    (mi.LayerDims(hidden=256, n_experts=33, top_k=5, inter=1152, shared_inter=128), 9),   # I > 1024
+])
+def test_odd_shapes(dims, rows):
+    case = P.build_case(dims, rows, all_experts=True)
+    check(case)
+
+
+def test_residual_and_router_bias():
+    d = mi.LayerDims(hidden=512, n_experts=32, top_k=4, inter=256, shared_inter=256)
+    case = P.build_case(d, 6, router_bias=True, all_experts=True, residual=True)
+    check(case)
+
+
+def test_residual_in_place():
+    d = mi.TINY
+    case = P.build_case(d, 4, all_experts=True, residual=True)
+    check(case, residual_inplace=True)
+
+
+def test_rows_64_max_decode_tile_then_rows_1_on_same_workspace(layer35, dev35):
+    """Counters left by one call must not disturb the next (different rows)."""
+    d = mi.QWEN36_35B_A3B
+    ws = moe.alloc_workspace(d, 64)
+    outs = []
+    for rows in (64, 1, 64):
+        case = P.build_case(d, rows, layer=layer35)
+        x = P.bf16_tensor(case.x)
+        out = torch.empty(rows, d.hidden, dtype=torch.bfloat16, device="cuda")
+        moe.ffn_forward(d, x, dev35["router_w"], dev35["expert_w8"], dev35["expert_scales"],
+                        dev35["shared_w8"], dev35["shared_scales"], dev35["shared_gate"], out, ws)
+        torch.cuda.synchronize()
+        outs.append(out.clone())
+    assert torch.equal(outs[0], outs[2])
+
+
+def test_batch_invariance_bitwise(layer35, dev35):
+    """Row r of an 8-row call equals a 1-row call on row r, bit for bit."""
+    d = mi.QWEN36_35B_A3B
+    case = P.build_case(d, 8, layer=layer35)
+    out8, idx8, w8, _ = run_forward(case, dev35)
+    for r in range(8):
+        one = P.Case(d, layer35, case.x[r:r + 1].copy(), case.logits[r:r + 1])
+        out1, idx1, w1, _ = run_forward(one, dev35)
+        assert np.array_equal(out1[0], out8[r])
+        assert np.array_equal(idx1[0], idx8[r]) and np.array_equal(w1[0], w8[r])
+
+
+def test_rows_zero_is_noop():
+    d = mi.TINY
+    L = mi.make_layer(d, seed=0)
+    dev = P.device_weights(L)
+    x = torch.empty(0, d.hidden, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((1, d.hidden), 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = moe.alloc_workspace(d, 1)
+    moe.ffn_forward(d, x, dev["router_w"], dev["expert_w8"], dev["expert_scales"], dev["shared_w8"],
+                    dev["shared_scales"], dev["shared_gate"], out, ws)
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+
+
+@pytest.mark.parametrize("dims,rows", [(mi.TINY, 4), (mi.QWEN36_35B_A3B, 64), (mi.QWEN35_397B_A17B, 32)])
+def test_router_topk_entry_point(dims, rows):
+    rw, g, _ = mi.make_router(dims, 0)
+    x = mi.make_x(dims, rows, seed=0, stream=rows)
+    logits, oidx, ow, ogs = oracle.router_topk(dims, x, rw, g)
+    idx = torch.empty(rows, dims.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(rows, dims.top_k, dtype=torch.float32, device="cuda")
+    gs = torch.empty(rows, dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(dims, rows)
+    moe.router_topk(dims, P.bf16_tensor(x), P.bf16_tensor(rw), P.bf16_tensor(g), idx, w, gs, ws)
+    torch.cuda.synchronize()
+    case = P.Case(dims, None, x, logits)
+    P.check_routing(case, idx.cpu().numpy(), w.cpu().numpy(), gs.cpu().numpy(), ow, ogs)
