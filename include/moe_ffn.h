@@ -75,6 +75,7 @@ extern "C" {
 #define MOE_EUNSUPPORTED -2  /* H, I or Is not a multiple of 128, k > E, k > 32, E > 1024 */
 #define MOE_EWORKSPACE -3    /* workspace smaller than moe_workspace_bytes(d, rows) */
 #define MOE_ECUDA -4         /* a CUDA launch or runtime error (sticky) */
+#define MOE_ETIMEOUT -5      /* a bounded wait inside a kernel ran out (device status word) */
 
 #define MOE_PATH_AUTO 0      /* decode kernels for rows <= MOE_DECODE_MAX_ROWS, else prefill */
 #define MOE_PATH_DECODE 1    /* warp-per-row FP8 GEMVs with expert dedup */
@@ -105,7 +106,7 @@ MOE_API int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
 /* Router GEMV, shared-gate sigmoid and top-k softmax for `rows` rows of x.
  * Outputs topk_idx [rows, k] (int32), topk_w [rows, k] (fp32, renormalised
  * over the k chosen, descending) and shared_gate_sig [rows] (fp32).
- * router_bias may be NULL.  rows == 0 is a no-op. */
+ * router_bias may be NULL.  rows == 0 is a no-op (pointers may then be NULL). */
 MOE_API int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows,
                     const uint16_t *router_w, const float *router_bias,
                     const uint16_t *shared_gate, int32_t *topk_idx, float *topk_w,
@@ -114,7 +115,7 @@ MOE_API int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows,
 /* The whole layer step: out = sum_r w_r E_{idx_r}(x) + sigmoid(g.x) E_shared(x)
  * (+ residual), bf16 [rows, H].  residual and router_bias may be NULL.
  * Chooses the decode path for rows <= MOE_DECODE_MAX_ROWS, else prefill.
- * rows == 0 is a no-op. */
+ * rows == 0 is a no-op (pointers may then be NULL). */
 MOE_API int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows,
                     const uint16_t *router_w, const uint8_t *expert_w8,
                     const float *expert_scales, const moe_fp8_expert *shared_w,
@@ -132,6 +133,37 @@ MOE_API int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t r
                          const float *router_bias, void *ws, size_t ws_bytes, void *stream,
                          int32_t path, int32_t *topk_idx, float *topk_w,
                          float *shared_gate_sig);
+
+/* Number of kernels one moe_ffn_forward_path call launches for these dims,
+ * rows and path (MOE_PATH_AUTO resolved as moe_ffn_forward does); 0 for
+ * invalid arguments or rows == 0. */
+MOE_API int32_t moe_kernel_launches(const moe_dims *d, int32_t rows, int32_t path);
+
+/* moe_ffn_forward_path for per-kernel timing: records events[0] on `stream`
+ * before the first kernel and events[j] after kernel j-1 (each a caller-owned
+ * cudaEvent_t created with timing enabled), and launches the kernels without
+ * programmatic dependent launch so that consecutive events bracket exactly
+ * one kernel.  n_events must be at least moe_kernel_launches(d, rows, path)
+ * + 1, else MOE_EINVAL.  Results are identical to moe_ffn_forward_path. */
+MOE_API int moe_ffn_forward_timed(const moe_dims *d, const uint16_t *x, int32_t rows,
+                          const uint16_t *router_w, const uint8_t *expert_w8,
+                          const float *expert_scales, const moe_fp8_expert *shared_w,
+                          const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
+                          const float *router_bias, void *ws, size_t ws_bytes, void *stream,
+                          int32_t path, void *const *events, int32_t n_events);
+
+/* Device-side status of a workspace: synchronises `stream`, then reads the
+ * status word the kernels keep in the workspace (MOE_OK, or MOE_ETIMEOUT if
+ * a bounded wait inside a kernel ran out; the outputs of that call are then
+ * incomplete and the workspace must be re-initialised).  Returns MOE_ECUDA
+ * if the copy itself fails. */
+MOE_API int moe_device_status(const void *ws, size_t ws_bytes, void *stream);
+
+/* Test hook for the bounded waits: launches one CTA that waits on an
+ * mbarrier nothing completes, gives up after limit_us microseconds (clamped
+ * to [1, 2000000]) and records MOE_ETIMEOUT in the workspace status word, so
+ * that moe_device_status reports it.  The GPU context stays usable. */
+MOE_API int moe_debug_wait_timeout(void *ws, size_t ws_bytes, int32_t limit_us, void *stream);
 
 /* Sticky status: MOE_OK, or MOE_ECUDA after a CUDA error. */
 MOE_API int moe_status(void);

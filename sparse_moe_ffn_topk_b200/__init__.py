@@ -32,6 +32,7 @@ MOE_EINVAL = -1
 MOE_EUNSUPPORTED = -2
 MOE_EWORKSPACE = -3
 MOE_ECUDA = -4
+MOE_ETIMEOUT = -5
 
 MOE_PATH_AUTO = 0
 MOE_PATH_DECODE = 1
@@ -40,7 +41,8 @@ MOE_DECODE_MAX_ROWS = 64
 
 EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe_ffn_forward",
             "moe_ffn_forward_path", "moe_status", "moe_reset_status", "moe_status_string",
-            "moe_debug_inject_fault")
+            "moe_debug_inject_fault", "moe_kernel_launches", "moe_ffn_forward_timed",
+            "moe_device_status", "moe_debug_wait_timeout")
 
 
 class MoeDims(ctypes.Structure):
@@ -83,6 +85,12 @@ def lib() -> ctypes.CDLL:
                                       ctypes.c_size_t, P]
         L.moe_ffn_forward_path.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P,
                                            P, ctypes.c_size_t, P, I32, P, P, P]
+        L.moe_kernel_launches.argtypes = [DP, I32, I32]
+        L.moe_kernel_launches.restype = I32
+        L.moe_ffn_forward_timed.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P,
+                                            P, ctypes.c_size_t, P, I32, ctypes.POINTER(ctypes.c_void_p), I32]
+        L.moe_device_status.argtypes = [P, ctypes.c_size_t, P]
+        L.moe_debug_wait_timeout.argtypes = [P, ctypes.c_size_t, I32, P]
         L.moe_status.argtypes = []
         L.moe_reset_status.argtypes = []
         L.moe_reset_status.restype = None
@@ -179,6 +187,35 @@ def ffn_forward_path(dims, x, router_w, expert_w8, expert_scales, shared_w8, sha
                                       ws.numel() * ws.element_size(), _stream(stream), int(path),
                                       _ptr(topk_idx), _ptr(topk_w), _ptr(shared_gate_sig)),
            "moe_ffn_forward_path")
+
+
+def kernel_launches(dims, rows: int, path=MOE_PATH_AUTO) -> int:
+    return int(lib().moe_kernel_launches(ctypes.byref(_dims(dims)), int(rows), int(path)))
+
+
+def ffn_forward_timed(dims, x, router_w, expert_w8, expert_scales, shared_w8, shared_scales, shared_gate,
+                      out, ws, events, path=MOE_PATH_AUTO, residual=None, router_bias=None, stream=None):
+    """Forward that records ``events`` (torch.cuda.Event(enable_timing=True), at least
+    kernel_launches()+1 of them) around each kernel it launches."""
+    d = _dims(dims)
+    sh = MoeFp8Expert(_ptr(shared_w8), _ptr(shared_scales))
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().moe_ffn_forward_timed(ctypes.byref(d), _ptr(x), _rows(x), _ptr(router_w), _ptr(expert_w8),
+                                       _ptr(expert_scales), ctypes.byref(sh), _ptr(shared_gate), _ptr(out),
+                                       _ptr(residual), _ptr(router_bias), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream), int(path), arr,
+                                       len(events)),
+           "moe_ffn_forward_timed")
+
+
+def device_status(ws, stream=None) -> int:
+    """Synchronises the stream and returns the workspace's device status word."""
+    return int(lib().moe_device_status(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def debug_wait_timeout(ws, limit_us: int, stream=None):
+    _check(lib().moe_debug_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us),
+                                        _stream(stream)), "moe_debug_wait_timeout")
 
 
 def status() -> int:

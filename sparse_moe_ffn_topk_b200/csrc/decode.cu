@@ -1,37 +1,82 @@
 // decode.cu -- decode path (rows <= a few dozen): weight-streaming GEMVs.
 //
-// Three launches chained with programmatic dependent launch:
-//   1. router_topk_kernel: bf16 router GEMV + shared-gate dot, one warp per
-//      router row with the row held in registers and the activation rows in
-//      shared memory; the last CTA to finish runs the top-k softmax and
-//      builds the per-expert row lists (expert dedup across rows).
-//   2. gate_up_kernel: for every (active expert, chunk of 16 gate/up row
-//      pairs) work item, a warp per row pair streams both FP8 rows with
-//      16-byte lane loads, applies the 128x128 block scales in registers and
-//      writes h = silu(gate) * up in fp32.
-//   3. down_blend_kernel: for every (active expert, 32 output rows) item, a
-//      warp per output row streams the FP8 down row against h (shared
-//      memory), scales by the routing weight (or the shared gate) and writes
-//      one partial per routed slot; the last item to finish a 32-row chunk
-//      blends the k partials in rank order plus the shared partial (plus the
-//      residual) and rounds once to bf16.
+// Three launches chained with programmatic dependent launch (PDL):
+//   1. router_topk_kernel: bf16 router GEMV + shared-gate dot.  Each CTA
+//      bulk-copies its slice of router rows into shared memory before it
+//      waits on the kernel that produced x, one warp per router row; the last
+//      CTA to finish runs the top-k softmax and builds the per-expert work
+//      table (expert dedup across rows).
+//   2. gate_up_kernel: persistent CTAs walk (expert, block of gate/up row
+//      pairs) items through a ring of shared-memory stages filled by bulk
+//      copies; shared-expert items come first and are fetched before the PDL
+//      wait, since they do not depend on routing.  A warp per row pair,
+//      block scales applied in registers, h = silu(gate) * up kept in fp32.
+//   3. down_blend_kernel: (expert, block of down rows) items, fetched
+//      through the same kind of ring; the weight blocks are fetched as soon
+//      as the CTA starts (routing is final by then) and only h waits for
+//      gate_up.  A warp per output row, one partial per routed slot scaled by
+//      its routing weight (or the shared gate); the last item to finish a row
+//      block blends the k partials in rank order plus the shared partial
+//      (plus the residual) and rounds once to bf16.
 //
-// The pages' kernels are the prior art: the GB10 blueprint's per-layer MoE
-// chain (router GEMV, top-k softmax, gate_up with the shared expert fused,
-// silu+down, weighted blend; fp8/block128x128 weights read against bf16 and
-// f32 activations) and the colibri PR's decode GEMV (one warp per output row,
-// 16 bytes per lane, the activation in shared memory).
+// Prior art on the pages: the GB10 blueprint's per-layer MoE chain (router
+// GEMV, top-k softmax, gate_up with the shared expert fused, silu+down,
+// weighted blend; fp8/block128x128 weights read against bf16 and f32
+// activations) and the colibri PR's decode GEMV (one warp per output row, 16
+// bytes a lane, the activation in shared memory).  Here the weight bytes
+// reach shared memory by bulk DMA instead of through registers, so the bytes
+// in flight per SM are bounded by shared memory, not by registers.
+//
+// Every wait is bounded (kWaitLimitNs); a wait that runs out records
+// MOE_ETIMEOUT in the workspace status word and the CTA leaves.
 #include <math.h>
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.h"
 
 namespace moe {
 
 // ------------------------------------------------------------------ helpers
+
+__device__ __forceinline__ void set_status(int32_t *counters, int32_t code)
+{
+    atomicCAS(&counters[kCtrStatus], 0, code);
+}
+
+// 8 e4m3 codes (two words) against 8 bf16 activations (16 bytes).
+__device__ __forceinline__ float dot8_e4m3_bf16(uint2 w, uint4 x)
+{
+    float2 f0 = e4m3x2_to_f32x2(static_cast<uint16_t>(w.x & 0xFFFFu));
+    float2 f1 = e4m3x2_to_f32x2(static_cast<uint16_t>(w.x >> 16));
+    float2 f2 = e4m3x2_to_f32x2(static_cast<uint16_t>(w.y & 0xFFFFu));
+    float2 f3 = e4m3x2_to_f32x2(static_cast<uint16_t>(w.y >> 16));
+    float a = f0.x * bf16_lo(x.x);
+    float b = f0.y * bf16_hi(x.x);
+    a = fmaf(f1.x, bf16_lo(x.y), a);
+    b = fmaf(f1.y, bf16_hi(x.y), b);
+    a = fmaf(f2.x, bf16_lo(x.z), a);
+    b = fmaf(f2.y, bf16_hi(x.z), b);
+    a = fmaf(f3.x, bf16_lo(x.w), a);
+    b = fmaf(f3.y, bf16_hi(x.w), b);
+    return a + b;
+}
+
+// 4 e4m3 codes (one word) against 4 fp32 values.
+__device__ __forceinline__ float dot4_e4m3_f32(uint32_t w, float4 h)
+{
+    float2 f0 = e4m3x2_to_f32x2(static_cast<uint16_t>(w & 0xFFFFu));
+    float2 f1 = e4m3x2_to_f32x2(static_cast<uint16_t>(w >> 16));
+    float a = f0.x * h.x;
+    float b = f0.y * h.y;
+    a = fmaf(f1.x, h.z, a);
+    b = fmaf(f1.y, h.w, b);
+    return a + b;
+}
 
 __device__ __forceinline__ float dot8_bf16(uint4 w, uint4 x)
 {
@@ -46,256 +91,307 @@ __device__ __forceinline__ float dot8_bf16(uint4 w, uint4 x)
     return a + b;
 }
 
-// 4 e4m3 codes (one word) against 4 bf16 activations (two words).
-__device__ __forceinline__ void fma4_e4m3_bf16(uint32_t w, uint32_t x01, uint32_t x23, float &a, float &b)
-{
-    float2 f0 = e4m3x2_to_f32x2(static_cast<uint16_t>(w & 0xFFFFu));
-    float2 f1 = e4m3x2_to_f32x2(static_cast<uint16_t>(w >> 16));
-    a = fmaf(f0.x, bf16_lo(x01), a);
-    b = fmaf(f0.y, bf16_hi(x01), b);
-    a = fmaf(f1.x, bf16_lo(x23), a);
-    b = fmaf(f1.y, bf16_hi(x23), b);
-}
+__host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
-// 16 e4m3 codes against 16 bf16 activations (two 16-byte words).
-__device__ __forceinline__ float dot16_e4m3_bf16(uint4 w, uint4 xa, uint4 xb)
-{
-    float a = 0.f, b = 0.f;
-    fma4_e4m3_bf16(w.x, xa.x, xa.y, a, b);
-    fma4_e4m3_bf16(w.y, xa.z, xa.w, a, b);
-    fma4_e4m3_bf16(w.z, xb.x, xb.y, a, b);
-    fma4_e4m3_bf16(w.w, xb.z, xb.w, a, b);
-    return a + b;
-}
-
-__device__ __forceinline__ void fma4_e4m3_f32(uint32_t w, float4 h, float &a, float &b)
-{
-    float2 f0 = e4m3x2_to_f32x2(static_cast<uint16_t>(w & 0xFFFFu));
-    float2 f1 = e4m3x2_to_f32x2(static_cast<uint16_t>(w >> 16));
-    a = fmaf(f0.x, h.x, a);
-    b = fmaf(f0.y, h.y, b);
-    a = fmaf(f1.x, h.z, a);
-    b = fmaf(f1.y, h.w, b);
-}
-
+// Order-preserving 32-bit key of a float (larger key = larger value).
 __device__ __forceinline__ uint32_t ordered_key(float f)
 {
-    uint32_t u = __float_as_uint(f);
+    const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 // ---------------------------------------------------------------- router
 
-constexpr int kRouterWarps = 16;  // router rows per CTA (one per warp)
-constexpr int kRouterTok = 8;     // activation rows staged per pass
+constexpr int kRouterMaxRows = 16;  // router rows per CTA (one per warp)
+constexpr int kRouterTok = 8;       // activation rows staged per pass
 
 struct RouterParams {
     const uint16_t *x;
     int rows, H, E, K;
+    int ld;            // logits row stride (floats, a multiple of 4)
+    int rows_per_cta;  // router rows (warps) per CTA
+    int group_tokens;  // activation rows per token group (gridDim.y groups)
     const uint16_t *wr;
     const float *bias;
     const uint16_t *g;
-    float *logits;
+    float *logits;     // [rows, ld]; column E holds the shared-gate logit
+    uint8_t *xq;       // x as hi/lo e4m3 rows [rows][2H] for the expert kernels
+    float *xsc;        // their scales [rows][H/128]
     int32_t *topk_idx;
     float *topk_w;
     float *gsig;
     int32_t *counters;
-    int32_t *plan;
+    int32_t *plan;     // nullptr: no plan
 };
 
-// Top-k of every row (warp per row), run by the last router CTA.  Logits are
-// compared as order-preserving 32-bit keys; 0 marks a taken (or absent)
-// expert and a NaN logit gets key 1, so every round selects a valid,
-// untaken expert even on non-finite input.  Equal keys go to the lower
-// expert index.
-__device__ void router_topk_rows(const RouterParams &p)
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int t = warp; t < p.rows; t += kRouterWarps) {
-        const float *lrow = p.logits + (size_t)t * (p.E + 1);
-        uint32_t v[kMaxExperts / kWarp];
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Top-k of one row (one warp) on order-preserving keys.  Lane L holds the
+// EPL experts L*EPL .. L*EPL+EPL-1.  Key 0 marks a taken (or absent) expert
+// and a NaN logit gets key 1, so every round picks a valid, untaken expert
+// even on non-finite input; equal keys go to the lower expert index.
+template <int EPL>
+__device__ void topk_row(const RouterParams &p, int t)
+{
+    const int lane = threadIdx.x & 31;
+    const float *lrow = p.logits + (size_t)t * p.ld;
+    uint32_t v[EPL];
 #pragma unroll
-        for (int i = 0; i < kMaxExperts / kWarp; ++i) {
-            const int e = lane + kWarp * i;
-            const float l = (e < p.E) ? __ldcg(lrow + e) : 0.f;
-            v[i] = (e < p.E) ? (isnan(l) ? 1u : max(ordered_key(l), 2u)) : 0u;
-        }
-        int my_e = 0;
-        float my_v = 0.f;
-        for (int r = 0; r < p.K; ++r) {
-            uint32_t bk = 0;
-            int be = 0x7FFFFFFF;
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane * EPL + i;
+        const float l = (e < p.E) ? __ldcg(lrow + e) : 0.f;
+        v[i] = (e < p.E) ? (isnan(l) ? 1u : max(ordered_key(l), 2u)) : 0u;
+    }
+    const float z = __ldcg(lrow + p.E);
+    int my_e = 0;
+    uint32_t my_k = 0;
+    for (int r = 0; r < p.K; ++r) {
+        uint32_t bk = 0;
+        int bi = 0;
 #pragma unroll
-            for (int i = 0; i < kMaxExperts / kWarp; ++i)
-                if (v[i] > bk) { bk = v[i]; be = lane + kWarp * i; }
-            const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, bk);
-            const int emin = (int)__reduce_min_sync(0xFFFFFFFFu, bk == kmax ? (uint32_t)be : 0x7FFFFFFFu);
+        for (int i = 0; i < EPL; ++i)
+            if (v[i] > bk) { bk = v[i]; bi = i; }
+        const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, bk);
+        const uint32_t cand = (bk == kmax) ? (uint32_t)(lane * EPL + bi) : 0x7FFFFFFFu;
+        const int emin = (int)__reduce_min_sync(0xFFFFFFFFu, cand);
+        if (lane == emin / EPL) {
 #pragma unroll
-            for (int i = 0; i < kMaxExperts / kWarp; ++i)
-                if (lane + kWarp * i == emin) v[i] = 0u;
-            if (lane == r) { my_e = emin; my_v = __ldcg(lrow + emin); }
+            for (int i = 0; i < EPL; ++i)
+                if (i == emin - lane * EPL) v[i] = 0u;
         }
-        const float top = __shfl_sync(0xFFFFFFFFu, my_v, 0);
-        const float ev = (lane < p.K) ? expf(my_v - top) : 0.f;
-        const float sum = warp_sum(ev);
-        if (lane < p.K) {
-            p.topk_idx[(size_t)t * p.K + lane] = my_e;
-            p.topk_w[(size_t)t * p.K + lane] = ev / sum;
-        }
-        if (lane == 0) p.gsig[t] = sigmoidf_(__ldcg(lrow + p.E));
+        if (lane == r) { my_e = emin; my_k = kmax; }
+    }
+    const float my_v = (my_k == 1u) ? __int_as_float(0x7FC00000) : key_value(my_k);
+    const float top = __shfl_sync(0xFFFFFFFFu, my_v, 0);
+    const float ev = (lane < p.K) ? expf(my_v - top) : 0.f;
+    const float sum = warp_sum(ev);
+    if (lane < p.K) {
+        p.topk_idx[(size_t)t * p.K + lane] = my_e;
+        p.topk_w[(size_t)t * p.K + lane] = ev / sum;
+    }
+    if (lane == 0) p.gsig[t] = sigmoidf_(z);
+}
+
+__device__ void topk_rows(const RouterParams &p, int t_begin, int t_end)
+{
+    const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int t = t_begin + warp; t < t_end; t += nwarps) {
+        if (p.E <= 32) topk_row<1>(p, t);
+        else if (p.E <= 64) topk_row<2>(p, t);
+        else if (p.E <= 128) topk_row<4>(p, t);
+        else if (p.E <= 256) topk_row<8>(p, t);
+        else if (p.E <= 512) topk_row<16>(p, t);
+        else topk_row<32>(p, t);
     }
 }
 
-// Per-expert lists of routed pairs (pair id = t*K + r), active experts in
-// ascending id, pairs within an expert in ascending pair id.
-__device__ void router_build_plan(const RouterParams &p, int *cnt, int *cursor)
+// Exclusive prefix sum over the block of one value per thread; returns the
+// block total in *total.  scratch: >= 32 ints of shared memory.
+__device__ int block_exclusive_scan(int v, int *scratch, int *total)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == kWarp - 1) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = (lane < nwarps) ? scratch[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < kWarp; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nwarps) scratch[lane] = wi - w;
+        if (lane == kWarp - 1) scratch[kWarp] = wi;
+    }
+    __syncthreads();
+    const int r = scratch[warp] + incl - v;
+    *total = scratch[kWarp];
+    __syncthreads();
+    return r;
+}
+
+// Work table of the expert kernels.  plan[0] = number of active routed
+// experts; descriptor u (kDescInts ints at plan + 4 + kDescInts*u) =
+// {expert, pairs routed to it, first index in the pair list, 0, the first
+// kDescPairs pair ids}; active experts in ascending id.  The pair list (at
+// plan + 4 + kDescInts*E) holds each expert's pair ids (t*K + r) together;
+// their order within an expert is immaterial (each pair is computed alone).
+__device__ void build_plan(const RouterParams &p, int *smem_i)
+{
     const int E = p.E, P = p.rows * p.K;
-    int32_t *n_active = p.plan;
-    int32_t *act_e = p.plan + 1;
-    int32_t *act_off = act_e + E;
-    int32_t *pairs = act_off + E + 1;
+    int *cnt = smem_i;             // [E]
+    int *cursor = smem_i + E;      // [E]
+    int *slot = smem_i + 2 * E;    // [E] active index of each expert
+    int *scratch = smem_i + 3 * E; // [33]
+    int32_t *desc = p.plan + 4;
+    int32_t *pairs = p.plan + 4 + kDescInts * E;
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < P; i += blockDim.x) atomicAdd(&cnt[__ldcg(p.topk_idx + i)], 1);
     __syncthreads();
-    if (warp == 0) {
-        int run = 0, nact = 0;
-        for (int e0 = 0; e0 < E; e0 += kWarp) {
-            const int e = e0 + lane;
-            const int c = (e < E) ? cnt[e] : 0;
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < kWarp; o <<= 1) {
-                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const int excl = run + incl - c;
-            const uint32_t act = __ballot_sync(0xFFFFFFFFu, c > 0);
-            const int apos = nact + __popc(act & ((1u << lane) - 1u));
-            if (c > 0) {
-                act_e[apos] = e;
-                act_off[apos] = excl;
-                cursor[e] = excl;
-            }
-            run += __shfl_sync(0xFFFFFFFFu, incl, kWarp - 1);
-            nact += __popc(act);
+    int run_off = 0, run_act = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        const int c = (e < E) ? cnt[e] : 0;
+        int tot_off, tot_act;
+        const int off = block_exclusive_scan(c, scratch, &tot_off);
+        const int act = block_exclusive_scan(c > 0 ? 1 : 0, scratch, &tot_act);
+        if (c > 0) {
+            const int u = run_act + act;
+            int32_t *dd = desc + kDescInts * u;
+            dd[0] = e;
+            dd[1] = c;
+            dd[2] = run_off + off;
+            dd[3] = 0;
+            cursor[e] = run_off + off;
+            slot[e] = u;
         }
-        if (lane == 0) {
-            act_off[nact] = run;
-            n_active[0] = nact;
-        }
-        __syncwarp();
-        for (int p0 = 0; p0 < P; p0 += kWarp) {
-            const int i = p0 + lane;
-            const int e = (i < P) ? __ldcg(p.topk_idx + i) : -1;
-            const uint32_t m = __match_any_sync(0xFFFFFFFFu, e);
-            const int rank = __popc(m & ((1u << lane) - 1u));
-            const int base = (i < P) ? cursor[e] : 0;
-            __syncwarp();
-            if (i < P) {
-                pairs[base + rank] = i;
-                if (lane == __ffs(m) - 1) cursor[e] = base + __popc(m);
-            }
-            __syncwarp();
-        }
+        run_off += tot_off;
+        run_act += tot_act;
+    }
+    if (threadIdx.x == 0) p.plan[0] = run_act;
+    __syncthreads();
+    for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        const int e = __ldcg(p.topk_idx + i);
+        const int pos = atomicAdd(&cursor[e], 1);
+        pairs[pos] = i;
+        const int local = pos - desc[kDescInts * slot[e] + 2];
+        if (local < kDescPairs) desc[kDescInts * slot[e] + 4 + local] = i;
     }
 }
 
-template <int KC>  // 16-byte bf16 chunks per lane per segment: segment = KC*256 columns
-__global__ void __launch_bounds__(kRouterWarps * kWarp) router_topk_kernel(RouterParams p)
+// grid = (router-row blocks, token groups).  Shared memory: [rows_per_cta
+// router rows, bf16][kRouterTok activation rows, bf16]; the last CTA reuses
+// it as plan scratch.
+__global__ void __launch_bounds__(kRouterMaxRows * kWarp) router_topk_kernel(RouterParams p)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_last;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bar_w, bar_x;
+    __shared__ int s_last, s_abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x * kRouterWarps + warp;  // rows 0..E-1: router; row E: shared gate
-    const bool active = row <= p.E;
-    const uint16_t *wrow = (row < p.E) ? p.wr + (size_t)row * p.H : p.g;
-    constexpr int kSeg = KC * 256;
-    const int nseg = (p.H + kSeg - 1) / kSeg;
+    const int row0 = blockIdx.x * p.rows_per_cta;
+    const int nrows = min(p.rows_per_cta, p.E + 1 - row0);   // rows of this CTA; the gate row is index E
+    const int nrouter = max(0, min(nrows, p.E - row0));      // of which rows of Wr
+    const int t_begin = blockIdx.y * p.group_tokens;
+    const int t_end = min(p.rows, t_begin + p.group_tokens);
+    const size_t rowb = (size_t)p.H * 2;
+    unsigned char *wsm = smem;
+    unsigned char *xs = smem + (size_t)p.rows_per_cta * rowb;
 
     // The router weights are layer constants: fetch them before waiting on
     // the kernel that produced x.
-    uint4 w[KC];
-#pragma unroll
-    for (int c = 0; c < KC; ++c) {
-        const int col = c * 256 + lane * 8;
-        w[c] = (active && col < p.H) ? ld_stream_v4(wrow + col) : make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        mbar_init(&bar_w, 1);
+        mbar_init(&bar_x, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar_w, (uint32_t)(nrows * rowb));
+        if (nrouter > 0) bulk_g2s(wsm, p.wr + (size_t)row0 * p.H, (uint32_t)(nrouter * rowb), &bar_w);
+        if (nrouter < nrows) bulk_g2s(wsm + nrouter * rowb, p.g, (uint32_t)rowb, &bar_w);
     }
-    const float b = (active && row < p.E && p.bias) ? p.bias[row] : 0.f;
+    const bool active = warp < nrows;
+    const float b = (active && row0 + warp < p.E && p.bias) ? p.bias[row0 + warp] : 0.f;
+    if (threadIdx.x == 0) MOE_TRACE(0, 0);
     pdl_wait();
     pdl_trigger();
+    __syncthreads();
+    if (!mbar_wait(&bar_w, 0, kWaitLimitNs)) s_abort = 1;
+    if (threadIdx.x == 0) MOE_TRACE(0, 1);
 
-    uint4 *xs = reinterpret_cast<uint4 *>(smem);
+    const uint4 *wrow = reinterpret_cast<const uint4 *>(wsm + warp * rowb);
+    const uint4 *xsv = reinterpret_cast<const uint4 *>(xs);
     const int hv = p.H / 8;
-    for (int t0 = 0; t0 < p.rows; t0 += kRouterTok) {
-        const int nt = min(kRouterTok, p.rows - t0);
+    int pass = 0;
+    for (int t0 = t_begin; t0 < t_end; t0 += kRouterTok, ++pass) {
+        const int nt = min(kRouterTok, t_end - t0);
+        __syncthreads();  // previous pass done with xs
+        if (threadIdx.x == 0) {
+            mbar_arrive_expect_tx(&bar_x, (uint32_t)(nt * rowb));
+            bulk_g2s(xs, p.x + (size_t)t0 * p.H, (uint32_t)(nt * rowb), &bar_x);
+        }
+        if (!mbar_wait(&bar_x, pass & 1, kWaitLimitNs)) s_abort = 1;
         __syncthreads();
-        const uint4 *xg = reinterpret_cast<const uint4 *>(p.x + (size_t)t0 * p.H);
-        for (int i = threadIdx.x; i < nt * hv; i += blockDim.x) xs[i] = xg[i];
-        __syncthreads();
-        if (!active) continue;
-        float acc[kRouterTok];
-#pragma unroll
-        for (int t = 0; t < kRouterTok; ++t) acc[t] = 0.f;
-        for (int s = 0; s < nseg; ++s) {
-            if (nseg > 1 && !(s == 0 && t0 == 0)) {
-#pragma unroll
-                for (int c = 0; c < KC; ++c) {
-                    const int col = s * kSeg + c * 256 + lane * 8;
-                    w[c] = (col < p.H) ? ld_stream_v4(wrow + col) : make_uint4(0, 0, 0, 0);
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < kRouterTok; ++t) {
-                if (t < nt) {
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        const int col = s * kSeg + c * 256 + lane * 8;
-                        if (col < p.H) acc[t] += dot8_bf16(w[c], xs[t * hv + col / 8]);
-                    }
-                }
+        if (s_abort) break;
+        if (blockIdx.x == 0 && p.xq) {
+            // the expert kernels' activation format: hi/lo e4m3, one scale per (row, 128 block)
+            const int hb = p.H / 128;
+            for (int u = warp; u < nt * hb; u += blockDim.x >> 5) {
+                const int t = u / hb, kb = u - t * hb;
+                const uint2 raw = reinterpret_cast<const uint2 *>(xs + (size_t)t * rowb)[kb * 32 + lane];
+                const float4 v = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+                const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                const float sc = amax > 0.f ? amax / 448.f : 1.f;
+                uint32_t hi, lo;
+                quant4_hilo(v, 1.f / sc, hi, lo);
+                uint32_t *dst = reinterpret_cast<uint32_t *>(p.xq + (size_t)(t0 + t) * 2 * p.H);
+                dst[kb * 32 + lane] = hi;
+                dst[p.H / 4 + kb * 32 + lane] = lo;
+                if (lane == 0) p.xsc[(size_t)(t0 + t) * hb + kb] = sc;
             }
         }
-#pragma unroll
-        for (int t = 0; t < kRouterTok; ++t) {
-            if (t < nt) {
-                const float v = warp_sum(acc[t]);
-                if (lane == 0) p.logits[(size_t)(t0 + t) * (p.E + 1) + row] = v + b;
-            }
+        if (!active) continue;
+        for (int t = 0; t < nt; ++t) {
+            float acc = 0.f;
+            for (int c = lane; c < hv; c += kWarp) acc += dot8_bf16(wrow[c], xsv[t * hv + c]);
+            acc = warp_sum(acc);
+            if (lane == 0) p.logits[(size_t)(t0 + t) * p.ld + row0 + warp] = acc + b;
         }
     }
-
-    // Last CTA to finish runs the top-k (no CTA waits for another).
     __syncthreads();
+    if (s_abort) {  // the same decision in every thread of the CTA
+        if (threadIdx.x == 0) set_status(p.counters, MOE_ETIMEOUT);
+        return;
+    }
+
+    // The last CTA of this token group runs its top-k; the last group to
+    // finish builds the work table (no CTA waits for another).
+    if (threadIdx.x == 0) MOE_TRACE(0, 2);
     if (threadIdx.x == 0) {
-        __threadfence();
-        const int prev = atomicAdd(&p.counters[kCtrRouter], 1);
+        const int prev = atomic_add_acq_rel_gpu(p.counters + kCtrRouterGroup + blockIdx.y, 1);
         s_last = (prev == (int)gridDim.x - 1);
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    router_topk_rows(p);
-    if (p.plan) {
-        __syncthreads();
-        int *cnt = reinterpret_cast<int *>(smem);
-        router_build_plan(p, cnt, cnt + p.E);
+    if (threadIdx.x == 0) MOE_TRACE(0, 3);
+    topk_rows(p, t_begin, t_end);
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(0, 4);
+    if (threadIdx.x == 0) {
+        p.counters[kCtrRouterGroup + blockIdx.y] = 0;
+        const int prev = atomic_add_acq_rel_gpu(p.counters + kCtrRouter, 1);
+        s_last = (prev == (int)gridDim.y - 1);
     }
     __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (p.plan) build_plan(p, reinterpret_cast<int *>(smem));
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(0, 5);
     if (threadIdx.x == 0) p.counters[kCtrRouter] = 0;
 }
 
-// -------------------------------------------------------------- gate_up
-
-constexpr int kGuWarps = 8;
-constexpr int kGuPairsPerWarp = 2;
-constexpr int kGuPairs = kGuWarps * kGuPairsPerWarp;  // row pairs per work item
-constexpr int kGuTok = 8;                             // activation rows staged per pass
+// ------------------------------------------------------- expert kernels
 
 struct ExpertParams {
     const uint16_t *x;
+    const uint8_t *xq;  // activations as hi/lo e4m3: [rows][hi: H | lo: H]
+    const float *xsc;   // their scales: [rows][H/128]
     int rows, H, E, K, I, Is;
     const uint8_t *w8;
     const float *sc;
@@ -310,357 +406,782 @@ struct ExpertParams {
     const uint16_t *residual;
     uint16_t *out;
     int32_t *counters;
+    int pairs;   // gate_up: gate/up row pairs per item (a multiple of 8, <= 32)
+    int drows;   // down: rows per item (a multiple of 16, <= 64)
+    int tok;     // activation / h rows staged with an item (<= kDescPairs)
+    int stages;  // ring depth
 };
 
-struct ItemView {
-    const uint8_t *slab;   // expert slab (codes)
-    const float *scales;   // expert scales
-    const int32_t *pairs;  // routed pair ids, or nullptr for the shared expert
-    int n;                 // rows routed to this expert
+// What a stage holds; written by the producer before the stage's "full"
+// arrival, read by the consumers after the phase completes.
+struct StageDesc {
+    const uint8_t *slab;
+    const float *scales;
+    const int32_t *pairs;  // all pair ids of the expert, or nullptr for the shared expert
+    int n;                 // rows routed to the expert
     int inter;             // I or Is
-    int chunk;
+    int first;             // first gate/up pair (gate_up) or first down row (down)
+    int rows[kDescPairs];  // pair ids (routed) or token rows (shared) staged with the item
+    float wt[kDescPairs];  // down: routing weight (or shared gate) of each staged slot
 };
 
-__device__ __forceinline__ ItemView item_view(const ExpertParams &p, int item, int nch_r, int n_active)
+__device__ __forceinline__ int expert_nscales(int H, int I)
 {
-    ItemView v;
-    const int32_t *act_e = p.plan + 1;
-    const int32_t *act_off = act_e + p.E;
-    const int32_t *pairs = act_off + p.E + 1;
-    if (item < n_active * nch_r) {
-        const int u = item / nch_r;
-        const int e = act_e[u];
-        v.chunk = item - u * nch_r;
-        v.inter = p.I;
-        v.slab = p.w8 + (size_t)e * 3 * p.I * p.H;
-        v.scales = p.sc + (size_t)e * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128));
-        v.pairs = pairs + act_off[u];
-        v.n = act_off[u + 1] - act_off[u];
-    } else {
-        v.chunk = item - n_active * nch_r;
-        v.inter = p.Is;
-        v.slab = p.sw8;
-        v.scales = p.ssc;
-        v.pairs = nullptr;
-        v.n = p.rows;
-    }
-    return v;
+    return (2 * I / 128) * (H / 128) + (H / 128) * (I / 128);
 }
 
-// Shared-memory layout of a staged bf16 activation row: 16-byte units of
-// the row are stored so that, for each 512-column chunk c and half j, lane L
-// reads unit (c, j, L) at position c*64 + j*32 + L (conflict-free).
-template <int KC>
-__global__ void __launch_bounds__(kGuWarps * kWarp) gate_up_kernel(ExpertParams p)
+// Item i: shared-expert items first (routing-independent), then the routed
+// experts in table order.
+__device__ __forceinline__ void describe(const ExpertParams &p, int item, int per_shared, int per_routed,
+                                         int block, const int4 *dsc, StageDesc &d)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    pdl_wait();
-    pdl_trigger();
-    const int n_active = p.plan[0];
-    const int nch_r = p.I / kGuPairs, nch_s = p.Is / kGuPairs;
-    const int n_items = n_active * nch_r + nch_s;
-    const int nck = (p.H + 511) / 512;   // 512-column chunks per row
-    const int row_units = nck * 64;      // staged 16-byte units per row
-    const int hb = p.H / 128;
-    constexpr int kSeg = KC * 512;
-    const int nseg = (p.H + kSeg - 1) / kSeg;
-    uint4 *xs = reinterpret_cast<uint4 *>(smem);
+    if (item < per_shared) {
+        d.slab = p.sw8;
+        d.scales = p.ssc;
+        d.pairs = nullptr;
+        d.n = p.rows;
+        d.inter = p.Is;
+        d.first = item * block;
+#pragma unroll
+        for (int i = 0; i < kDescPairs; ++i) d.rows[i] = i;
+    } else {
+        const int r = item - per_shared;
+        const int u = r / per_routed;
+        int4 h = dsc[0];
+        const int P = p.rows * p.K;
+        if (h.x < 0 || h.x >= p.E || h.y < 0 || h.z < 0 || h.z + h.y > P) h = make_int4(0, 0, 0, 0);
+        d.slab = p.w8 + (size_t)h.x * 3 * p.I * p.H;
+        d.scales = p.sc + (size_t)h.x * expert_nscales(p.H, p.I);
+        d.pairs = p.plan + 4 + kDescInts * p.E + h.z;
+        d.n = h.y;
+        d.inter = p.I;
+        d.first = (r - u * per_routed) * block;
+        const int4 a = dsc[1], b = dsc[2];
+        const int ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < kDescPairs; ++i) d.rows[i] = min(max(ids[i], 0), max(P - 1, 0));
+    }
+}
 
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const ItemView v = item_view(p, item, nch_r, n_active);
-        const int Iu = v.inter;
-        for (int tok0 = 0; tok0 < v.n; tok0 += kGuTok) {
-            const int nt = min(kGuTok, v.n - tok0);
-            __syncthreads();
-            for (int i = threadIdx.x; i < nt * (p.H / 8); i += blockDim.x) {
-                const int t = i / (p.H / 8), q = i - t * (p.H / 8);
-                const int tok = v.pairs ? v.pairs[tok0 + t] / p.K : tok0 + t;
-                const int c = q >> 6, r = q & 63;
-                xs[t * row_units + c * 64 + (r & 1) * 32 + (r >> 1)] =
-                    reinterpret_cast<const uint4 *>(p.x + (size_t)tok * p.H)[q];
-            }
-            __syncthreads();
-#pragma unroll 1
-            for (int qp = 0; qp < kGuPairsPerWarp; ++qp) {
-                const int j = v.chunk * kGuPairs + qp * kGuWarps + warp;  // gate row j, up row Iu + j
-                const uint8_t *rg = v.slab + (size_t)j * p.H;
-                const uint8_t *ru = v.slab + (size_t)(Iu + j) * p.H;
-                const float *sg = v.scales + (j / 128) * hb;
-                const float *su = v.scales + ((Iu + j) / 128) * hb;
-                float ag[kGuTok], au[kGuTok];
-#pragma unroll
-                for (int t = 0; t < kGuTok; ++t) ag[t] = au[t] = 0.f;
-                for (int s = 0; s < nseg; ++s) {
-                    uint4 wg[KC], wu[KC];
-                    float cg[KC], cu[KC];
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        const int col = s * kSeg + c * 512 + lane * 16;
-                        const bool in = col < p.H;
-                        wg[c] = in ? ld_stream_v4(rg + col) : make_uint4(0, 0, 0, 0);
-                        wu[c] = in ? ld_stream_v4(ru + col) : make_uint4(0, 0, 0, 0);
-                        cg[c] = in ? sg[col >> 7] : 0.f;
-                        cu[c] = in ? su[col >> 7] : 0.f;
-                    }
-#pragma unroll
-                    for (int t = 0; t < kGuTok; ++t) {
-                        if (t < nt) {
-#pragma unroll
-                            for (int c = 0; c < KC; ++c) {
-                                const int col = s * kSeg + c * 512 + lane * 16;
-                                if (col < p.H) {
-                                    const int cc = s * KC + c;
-                                    const uint4 xa = xs[t * row_units + cc * 64 + lane];
-                                    const uint4 xb = xs[t * row_units + cc * 64 + 32 + lane];
-                                    ag[t] = fmaf(cg[c], dot16_e4m3_bf16(wg[c], xa, xb), ag[t]);
-                                    au[t] = fmaf(cu[c], dot16_e4m3_bf16(wu[c], xa, xb), au[t]);
-                                }
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < kGuTok; ++t) {
-                    if (t < nt) {
-                        const float g = warp_sum(ag[t]);
-                        const float u = warp_sum(au[t]);
-                        if (lane == 0) {
-                            const float h = siluf_(g) * u;
-                            if (v.pairs)
-                                p.h_routed[(size_t)v.pairs[tok0 + t] * Iu + j] = h;
-                            else
-                                p.h_shared[(size_t)(tok0 + t) * Iu + j] = h;
-                        }
-                    }
-                }
-            }
+// The descriptor of a routed item (three 16-byte words), or zeros.
+__device__ __forceinline__ void load_desc(const ExpertParams &p, int item, int per_shared, int per_routed,
+                                          int n_items, int4 *dv)
+{
+    dv[0] = dv[1] = dv[2] = make_int4(0, 0, 0, 0);
+    if (item >= per_shared && item < n_items) {
+        const int4 *dp = reinterpret_cast<const int4 *>(p.plan + 4 + kDescInts * ((item - per_shared) / per_routed));
+        dv[0] = __ldcg(dp);
+        dv[1] = __ldcg(dp + 1);
+        dv[2] = __ldcg(dp + 2);
+    }
+}
+
+__device__ __forceinline__ int active_experts(const ExpertParams &p)
+{
+    // an earlier kernel of this call gave up: the work table is not valid
+    return __ldcg(p.counters + kCtrStatus) ? 0 : min(__ldcg(p.plan), p.E);
+}
+
+// Warp roles of the expert kernels: warps 0..7 compute (consumers), warp 8
+// is the producer.  Each stage has a "full" mbarrier (one producer arrival
+// plus the bulk-copy bytes) and an "empty" mbarrier (one arrival per
+// consumer warp).  The producer runs up to `stages` items ahead: it fetches
+// an item's descriptor, issues the bulk copies of its weight rows (one per
+// row, into rows padded by 16 bytes so that the tensor-core fragment loads
+// hit distinct banks) and activations, loads the block scales into the
+// stage and arrives.
+//
+// The consumers feed the e4m3 weights straight into mma.m16n8k32 as the A
+// operand and the hi/lo e4m3 activations as B (up to 8 rows in the 8
+// columns).  Within each 32-wide K chunk, lane t of a quad reads the 8
+// bytes [8t, 8t+8) of its two rows and of its activation column; the first
+// four bytes play the fragment's k = 4t..4t+3 and the next four k =
+// 16+4t..19+4t, for A and B alike, so the products pair up the same
+// columns.  Each 128-wide K block is summed by the tensor cores, then scaled
+// by its weight and activation block scales into fp32 registers; the K
+// blocks are spread over the warps and reduced through shared memory.
+constexpr int kConsumerWarps = 8;
+constexpr int kExpThreads = (kConsumerWarps + 1) * kWarp;
+constexpr int kConsumerThreads = kConsumerWarps * kWarp;
+constexpr int kMaxStages = 4;
+constexpr int kMaxTiles = 4;  // 16-row MMA tiles per item
+constexpr int kRowPad = 16;   // bytes of padding after each staged row
+
+// ------------------------------------------------------------- gate_up
+
+// Stage layout (WS = H + 16): [16*T weight rows: tile tau's rows 0..7 are
+// gate rows first+8tau.., rows 8..15 the matching up rows][tok x-hi rows]
+// [tok x-lo rows][x scales: tok * H/128][gate scales: H/128][up scales: H/128]
+struct GuLayout {
+    int WS, T, hb;
+    size_t xh, xl, xs, sw, bytes;
+};
+__device__ __forceinline__ GuLayout gu_layout(const ExpertParams &p)
+{
+    GuLayout L;
+    L.WS = p.H + kRowPad;
+    L.T = p.pairs / 8;
+    L.hb = p.H / 128;
+    L.xh = (size_t)16 * L.T * L.WS;
+    L.xl = L.xh + (size_t)p.tok * L.WS;
+    L.xs = L.xl + (size_t)p.tok * L.WS;
+    L.sw = L.xs + (size_t)p.tok * L.hb * 4;
+    L.bytes = align16(L.sw + (size_t)2 * L.hb * 4);
+    return L;
+}
+
+// Producer warp, all lanes: weights (and/or activations) of a stage.
+__device__ void gu_produce(const ExpertParams &p, const GuLayout &L, const StageDesc &d, unsigned char *st,
+                           uint64_t *bar, uint64_t pol, bool weights, bool acts)
+{
+    const int lane = threadIdx.x & 31;
+    const int nt = min(p.tok, d.n);
+    if (lane == 0) {
+        uint32_t bytes = 0;
+        if (weights) bytes += (uint32_t)(16 * L.T * p.H);
+        if (acts) bytes += (uint32_t)(2 * nt * p.H);
+        mbar_expect_tx(bar, bytes);
+    }
+    __syncwarp();
+    if (weights) {
+        for (int i = lane; i < 16 * L.T; i += kWarp) {
+            const int tau = i >> 4, r = i & 15;
+            const int src = r < 8 ? d.first + 8 * tau + r : d.inter + d.first + 8 * tau + r - 8;
+            bulk_g2s_stream(st + (size_t)i * L.WS, d.slab + (size_t)src * p.H, (uint32_t)p.H, bar, pol);
+        }
+        float *sw = reinterpret_cast<float *>(st + L.sw);
+        const float *sg = d.scales + (d.first / 128) * L.hb;
+        const float *su = d.scales + ((d.inter + d.first) / 128) * L.hb;
+        for (int i = lane; i < 2 * L.hb; i += kWarp) sw[i] = (i < L.hb) ? __ldg(sg + i) : __ldg(su + i - L.hb);
+    }
+    if (acts) {
+        for (int i = lane; i < 2 * nt; i += kWarp) {
+            const int t = i >> 1, lo = i & 1;
+            const int row = d.pairs ? d.rows[t] / p.K : d.rows[t];
+            bulk_g2s(st + (lo ? L.xl : L.xh) + (size_t)t * L.WS, p.xq + (size_t)row * 2 * p.H + (size_t)lo * p.H,
+                     (uint32_t)p.H, bar);
+        }
+        float *xs = reinterpret_cast<float *>(st + L.xs);
+        for (int i = lane; i < nt * L.hb; i += kWarp) {
+            const int t = i / L.hb;
+            const int row = d.pairs ? d.rows[t] / p.K : d.rows[t];
+            xs[i] = __ldcg(p.xsc + (size_t)row * L.hb + (i - t * L.hb));
         }
     }
+}
+
+__global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ StageDesc desc[kMaxStages];
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const GuLayout L = gu_layout(p);
+    const int per_shared = p.Is / p.pairs, per_routed = p.I / p.pairs;
+    const int S = p.stages;
+    float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [warp][tile][lane]
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(1, 0);
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------- producer
+        const uint64_t pol = policy_evict_first();
+        // Shared-expert weights and scales do not depend on routing: fetch
+        // them before waiting on the router.
+        for (int q = 0; q < S; ++q) {
+            const int item = blockIdx.x + q * gridDim.x;
+            if (item >= per_shared) break;
+            if (lane == 0) describe(p, item, per_shared, per_routed, p.pairs, nullptr, desc[q]);
+            __syncwarp();
+            gu_produce(p, L, desc[q], smem + q * L.bytes, &full[q], pol, true, false);
+        }
+        __syncwarp();
+        pdl_wait();
+        pdl_trigger();
+        if (lane == 0) MOE_TRACE(1, 1);
+        const int n_items = per_shared + active_experts(p) * per_routed;
+        int4 dv[3];
+        load_desc(p, blockIdx.x, per_shared, per_routed, n_items, dv);
+        for (int q = 0;; ++q) {
+            const int item = blockIdx.x + q * gridDim.x;
+            if (item >= n_items) break;
+            const int s = q % S;
+            int4 cur[3] = {dv[0], dv[1], dv[2]};
+            load_desc(p, item + gridDim.x, per_shared, per_routed, n_items, dv);  // the next item's, early
+            if (q >= S && !mbar_wait(&empty[s], ((q / S) - 1) & 1, kWaitLimitNs)) {
+                if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+                s_abort = 1;
+                break;
+            }
+            unsigned char *st = smem + s * L.bytes;
+            const bool prefetched = q < S && item < per_shared;
+            if (lane == 0) {
+                if (q >= S) fence_proxy_async_smem();  // consumers' generic accesses precede the copies
+                if (!prefetched) describe(p, item, per_shared, per_routed, p.pairs, cur, desc[s]);
+            }
+            __syncwarp();
+            gu_produce(p, L, desc[s], st, &full[s], pol, !prefetched, true);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------- consumers
+    pdl_wait();
+    pdl_trigger();
+    const int n_items = per_shared + active_experts(p) * per_routed;
+    const int g = lane >> 2, t = lane & 3;
+    for (int q = 0;; ++q) {
+        const int item = blockIdx.x + q * gridDim.x;
+        if (item >= n_items) break;
+        const int s = q % S;
+        unsigned char *st = smem + s * L.bytes;
+        if (!s_abort && !mbar_wait(&full[s], (q / S) & 1, kWaitLimitNs)) {
+            if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+            s_abort = 1;
+        }
+        named_barrier(1, kConsumerThreads);  // every consumer warp sees the same abort flag
+        if (q < 2 && threadIdx.x == 0) MOE_TRACE(1, 2 + 2 * q);
+        const bool skip = s_abort;  // keep the loop (and its barriers) uniform after a timeout
+        const StageDesc &d = desc[s];  // read in place; the producer rewrites it only after "empty"
+        const int Iu = d.inter;
+        const float *xsc = reinterpret_cast<const float *>(st + L.xs);
+        const float *swg = reinterpret_cast<const float *>(st + L.sw);
+        for (int tok0 = 0; tok0 < (skip ? 0 : d.n); tok0 += p.tok) {
+            const int nt = min(p.tok, d.n - tok0);
+            if (tok0 > 0) {  // more rows than a stage holds: restage the next ones in place
+                named_barrier(1, kConsumerThreads);
+                const int hv = p.H / 16;
+                for (int i = threadIdx.x; i < 2 * nt * hv; i += kConsumerThreads) {
+                    const int tr = i / (2 * hv), rem = i - tr * 2 * hv, lo = rem / hv, c = rem - lo * hv;
+                    const int row = d.pairs ? __ldcg(d.pairs + tok0 + tr) / p.K : tok0 + tr;
+                    reinterpret_cast<uint4 *>(st + (lo ? L.xl : L.xh) + (size_t)tr * L.WS)[c] =
+                        __ldcg(reinterpret_cast<const uint4 *>(p.xq + (size_t)row * 2 * p.H + (size_t)lo * p.H) + c);
+                }
+                for (int i = threadIdx.x; i < nt * L.hb; i += kConsumerThreads) {
+                    const int tr = i / L.hb;
+                    const int row = d.pairs ? __ldcg(d.pairs + tok0 + tr) / p.K : tok0 + tr;
+                    const_cast<float *>(xsc)[i] = __ldcg(p.xsc + (size_t)row * L.hb + (i - tr * L.hb));
+                }
+                named_barrier(1, kConsumerThreads);
+            }
+            float acc[kMaxTiles][4];
+#pragma unroll
+            for (int tau = 0; tau < kMaxTiles; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
+            const bool col_ok = g < nt;
+            for (int kb = warp; kb < L.hb; kb += kConsumerWarps) {
+                float tmp[kMaxTiles][4];
+#pragma unroll
+                for (int tau = 0; tau < kMaxTiles; ++tau) tmp[tau][0] = tmp[tau][1] = tmp[tau][2] = tmp[tau][3] = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int k0 = kb * 128 + c * 32 + 8 * t;
+                    uint2 bh = make_uint2(0, 0), bl = make_uint2(0, 0);
+                    if (col_ok) {
+                        bh = *reinterpret_cast<const uint2 *>(st + L.xh + (size_t)g * L.WS + k0);
+                        bl = *reinterpret_cast<const uint2 *>(st + L.xl + (size_t)g * L.WS + k0);
+                    }
+#pragma unroll
+                    for (int tau = 0; tau < kMaxTiles; ++tau) {
+                        if (tau < L.T) {
+                            const uint2 ra = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g) * L.WS + k0);
+                            const uint2 rb = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g + 8) * L.WS + k0);
+                            mma_e4m3_16832(tmp[tau], ra.x, rb.x, ra.y, rb.y, bh.x, bh.y);
+                            mma_e4m3_16832(tmp[tau], ra.x, rb.x, ra.y, rb.y, bl.x, bl.y);
+                        }
+                    }
+                }
+                const float sg = swg[kb], su = swg[L.hb + kb];
+                const float x0 = (2 * t < nt) ? xsc[(2 * t) * L.hb + kb] : 0.f;
+                const float x1 = (2 * t + 1 < nt) ? xsc[(2 * t + 1) * L.hb + kb] : 0.f;
+#pragma unroll
+                for (int tau = 0; tau < kMaxTiles; ++tau) {
+                    acc[tau][0] = fmaf(sg * x0, tmp[tau][0], acc[tau][0]);
+                    acc[tau][1] = fmaf(sg * x1, tmp[tau][1], acc[tau][1]);
+                    acc[tau][2] = fmaf(su * x0, tmp[tau][2], acc[tau][2]);
+                    acc[tau][3] = fmaf(su * x1, tmp[tau][3], acc[tau][3]);
+                }
+            }
+#pragma unroll
+            for (int tau = 0; tau < kMaxTiles; ++tau)
+                if (tau < L.T)
+                    red[(warp * kMaxTiles + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
+            named_barrier(1, kConsumerThreads);
+            // (tile, pair row g, column n) -> h
+            for (int i = threadIdx.x; i < 64 * L.T; i += kConsumerThreads) {
+                const int tau = i >> 6, gg = (i >> 3) & 7, n = i & 7;
+                if (n >= nt) continue;
+                const int src = gg * 4 + (n >> 1), comp = n & 1;
+                float gate = 0.f, up = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float4 v = red[(w * kMaxTiles + tau) * kWarp + src];
+                    gate += comp ? v.y : v.x;
+                    up += comp ? v.w : v.z;
+                }
+                const float h = siluf_(gate) * up;
+                const int j = d.first + 8 * tau + gg;
+                if (d.pairs) {
+                    const int pr = tok0 == 0 ? d.rows[n] : __ldcg(d.pairs + tok0 + n);
+                    p.h_routed[(size_t)pr * Iu + j] = h;
+                } else {
+                    p.h_shared[(size_t)(tok0 + n) * Iu + j] = h;
+                }
+            }
+            named_barrier(1, kConsumerThreads);  // red is free again
+        }
+        if (q < 2 && threadIdx.x == 0) MOE_TRACE(1, 3 + 2 * q);
+        __syncwarp();  // this warp is done with the stage and its descriptor
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (threadIdx.x == 0) MOE_TRACE(1, 6);
 }
 
 // ------------------------------------------------------------ down+blend
 
-constexpr int kDnWarps = 8;
-constexpr int kDnRowsPerWarp = kDownRowsPerItem / kDnWarps;  // 4
-constexpr int kDnSlots = 8;                                  // h rows staged per pass
-
-// Staged fp32 h rows: float4 units, for 512-column chunk c and quarter j,
-// lane L reads unit (c, j, L) at position c*128 + j*32 + L.
-template <int KC>
-__global__ void __launch_bounds__(kDnWarps * kWarp) down_blend_kernel(ExpertParams p)
+// Stage layout (WS = Imax + 16): [drows weight rows][tok raw h rows, fp32]
+// [tok h-hi rows][tok h-lo rows][h scales: tok * Imax/128][row-block scales:
+// Imax/128]
+struct DnLayout {
+    int WS, T, imax;
+    size_t hr, hh, hl, hs, sw, bytes;
+};
+__device__ __forceinline__ DnLayout dn_layout(const ExpertParams &p)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_last;
+    DnLayout L;
+    L.imax = max(p.I, p.Is);
+    L.WS = L.imax + kRowPad;
+    L.T = p.drows / 16;
+    L.hr = (size_t)p.drows * L.WS;
+    L.hh = L.hr + (size_t)p.tok * L.imax * 4;
+    L.hl = L.hh + (size_t)p.tok * L.WS;
+    L.hs = L.hl + (size_t)p.tok * L.WS;
+    L.sw = L.hs + (size_t)p.tok * (L.imax / 128) * 4;
+    L.bytes = align16(L.sw + (size_t)(L.imax / 128) * 4);
+    return L;
+}
+
+__device__ void dn_produce(const ExpertParams &p, const DnLayout &L, StageDesc &d, unsigned char *st,
+                           uint64_t *bar, uint64_t pol, bool weights, bool acts)
+{
+    const int lane = threadIdx.x & 31;
+    const int ns = min(p.tok, d.n);
+    if (lane == 0) {
+        uint32_t bytes = 0;
+        if (weights) bytes += (uint32_t)(p.drows * d.inter);
+        if (acts) bytes += (uint32_t)(ns * d.inter * 4);
+        mbar_expect_tx(bar, bytes);
+    }
+    __syncwarp();
+    if (weights) {
+        const uint8_t *w2 = d.slab + (size_t)2 * d.inter * p.H + (size_t)d.first * d.inter;
+        for (int i = lane; i < p.drows; i += kWarp)
+            bulk_g2s_stream(st + (size_t)i * L.WS, w2 + (size_t)i * d.inter, (uint32_t)d.inter, bar, pol);
+        const int ib = d.inter / 128;
+        float *sw = reinterpret_cast<float *>(st + L.sw);
+        const float *src = d.scales + (2 * d.inter / 128) * (p.H / 128) + (d.first / 128) * ib;
+        for (int i = lane; i < ib; i += kWarp) sw[i] = __ldg(src + i);
+        if (lane < ns) d.wt[lane] = d.pairs ? __ldcg(p.topk_w + d.rows[lane]) : __ldcg(p.gsig + lane);
+    }
+    if (acts) {
+        for (int i = lane; i < ns; i += kWarp) {
+            const float *src = d.pairs ? p.h_routed + (size_t)d.rows[i] * d.inter : p.h_shared + (size_t)i * d.inter;
+            bulk_g2s(st + L.hr + (size_t)i * L.imax * 4, src, (uint32_t)d.inter * 4, bar);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ StageDesc desc[kMaxStages];
+    __shared__ volatile int s_abort, s_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const DnLayout L = dn_layout(p);
+    const int per_block = p.H / p.drows;  // items per expert
+    const int S = p.stages;
+    float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [warp][tile][lane]
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(2, 0);
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------- producer
+        // The router has finished when this kernel starts (its predecessor
+        // waited for the router before letting this kernel launch), so the
+        // work table is final: fetch the first stages' down weights and
+        // scales now; only h waits for gate_up.
+        const uint64_t pol = policy_evict_first();
+        const int n_items = per_block + active_experts(p) * per_block;
+        int4 dv[3];
+        load_desc(p, blockIdx.x, per_block, per_block, n_items, dv);
+        for (int q = 0; q < S; ++q) {
+            const int item = blockIdx.x + q * gridDim.x;
+            if (item >= n_items) break;
+            int4 cur[3] = {dv[0], dv[1], dv[2]};
+            load_desc(p, item + gridDim.x, per_block, per_block, n_items, dv);
+            if (lane == 0) describe(p, item, per_block, per_block, p.drows, cur, desc[q]);
+            __syncwarp();
+            dn_produce(p, L, desc[q], smem + q * L.bytes, &full[q], pol, true, false);
+        }
+        __syncwarp();  // the lanes' stage writes precede lane 0's arrivals
+        pdl_wait();
+        pdl_trigger();
+        if (lane == 0) MOE_TRACE(2, 1);
+        for (int q = 0;; ++q) {
+            const int item = blockIdx.x + q * gridDim.x;
+            if (item >= n_items) break;
+            const int s = q % S;
+            unsigned char *st = smem + s * L.bytes;
+            if (q < S) {
+                dn_produce(p, L, desc[s], st, &full[s], pol, false, true);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[s]);
+                continue;
+            }
+            int4 cur[3] = {dv[0], dv[1], dv[2]};
+            load_desc(p, item + gridDim.x, per_block, per_block, n_items, dv);
+            if (!mbar_wait(&empty[s], ((q / S) - 1) & 1, kWaitLimitNs)) {
+                if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+                s_abort = 1;
+                break;
+            }
+            if (lane == 0) {
+                fence_proxy_async_smem();  // consumers' generic accesses precede the copies
+                describe(p, item, per_block, per_block, p.drows, cur, desc[s]);
+            }
+            __syncwarp();
+            dn_produce(p, L, desc[s], st, &full[s], pol, true, true);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------- consumers
     pdl_wait();
     pdl_trigger();
-    const int n_active = p.plan[0];
-    const int n_chunks = p.H / kDownRowsPerItem;
-    const int n_items = (n_active + 1) * n_chunks;
-    constexpr int kSeg = KC * 512;
-    float4 *hs = reinterpret_cast<float4 *>(smem);
-
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int u = item / n_chunks;       // expert-major: neighbouring items stream neighbouring rows
-        const int chunk = item - u * n_chunks;
-        const ItemView v = item_view(p, u < n_active ? u : n_active, 1, n_active);
-        const int Iu = v.inter;
-        const int nck = (Iu + 511) / 512;
-        const int row_units = nck * 128;
+    const int n_active = active_experts(p);
+    const int n_items = per_block + n_active * per_block;
+    const int g = lane >> 2, t = lane & 3;
+    for (int q = 0;; ++q) {
+        const int item = blockIdx.x + q * gridDim.x;
+        if (item >= n_items) break;
+        const int s = q % S;
+        unsigned char *st = smem + s * L.bytes;
+        if (!s_abort && !mbar_wait(&full[s], (q / S) & 1, kWaitLimitNs)) {
+            if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+            s_abort = 1;
+        }
+        named_barrier(1, kConsumerThreads);  // every consumer warp sees the same abort flag
+        if (q < 2 && threadIdx.x == 0) MOE_TRACE(2, 2 + 3 * q);
+        const bool skip = s_abort;  // keep the loop (and its barriers) uniform after a timeout
+        const StageDesc &d = desc[s];  // read in place; the producer rewrites it only after "empty"
+        const int Iu = d.inter;
         const int ib = Iu / 128;
-        const int nseg = (Iu + kSeg - 1) / kSeg;
-        const float *hsrc = v.pairs ? p.h_routed : p.h_shared;
-        for (int s0 = 0; s0 < v.n; s0 += kDnSlots) {
-            const int ns = min(kDnSlots, v.n - s0);
-            __syncthreads();
-            for (int i = threadIdx.x; i < ns * (Iu / 4); i += blockDim.x) {
-                const int sl = i / (Iu / 4), q = i - sl * (Iu / 4);
-                const int slot = v.pairs ? v.pairs[s0 + sl] : s0 + sl;
-                const int c = q >> 7, r = q & 127;
-                hs[sl * row_units + c * 128 + (r & 3) * 32 + (r >> 2)] =
-                    reinterpret_cast<const float4 *>(hsrc + (size_t)slot * Iu)[q];
-            }
-            __syncthreads();
-#pragma unroll 1
-            for (int rr = 0; rr < kDnRowsPerWarp; ++rr) {
-                const int n = chunk * kDownRowsPerItem + warp * kDnRowsPerWarp + rr;
-                const uint8_t *row = v.slab + (size_t)2 * Iu * p.H + (size_t)n * Iu;
-                const float *sc = v.scales + (2 * Iu / 128) * (p.H / 128) + (n / 128) * ib;
-                float acc[kDnSlots];
-#pragma unroll
-                for (int t = 0; t < kDnSlots; ++t) acc[t] = 0.f;
-                for (int s = 0; s < nseg; ++s) {
-                    uint4 w[KC];
-                    float cs[KC];
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        const int col = s * kSeg + c * 512 + lane * 16;
-                        const bool in = col < Iu;
-                        w[c] = in ? ld_stream_v4(row + col) : make_uint4(0, 0, 0, 0);
-                        cs[c] = in ? sc[col >> 7] : 0.f;
-                    }
-#pragma unroll
-                    for (int t = 0; t < kDnSlots; ++t) {
-                        if (t < ns) {
-#pragma unroll
-                            for (int c = 0; c < KC; ++c) {
-                                const int col = s * kSeg + c * 512 + lane * 16;
-                                if (col < Iu) {
-                                    const float4 *hr = hs + t * row_units + (s * KC + c) * 128 + lane;
-                                    float a = 0.f, b = 0.f;
-                                    fma4_e4m3_f32(w[c].x, hr[0], a, b);
-                                    fma4_e4m3_f32(w[c].y, hr[32], a, b);
-                                    fma4_e4m3_f32(w[c].z, hr[64], a, b);
-                                    fma4_e4m3_f32(w[c].w, hr[96], a, b);
-                                    acc[t] = fmaf(cs[c], a + b, acc[t]);
-                                }
-                            }
-                        }
-                    }
+        const float *sw = reinterpret_cast<const float *>(st + L.sw);
+        float *hsc = reinterpret_cast<float *>(st + L.hs);
+        for (int s0 = 0; s0 < (skip ? 0 : d.n); s0 += p.tok) {
+            const int ns = min(p.tok, d.n - s0);
+            if (s0 > 0) {  // more slots than a stage holds: restage raw h in place
+                named_barrier(1, kConsumerThreads);
+                float4 *hv = reinterpret_cast<float4 *>(st + L.hr);
+                const int iv = Iu / 4, rv = L.imax / 4;
+                for (int i = threadIdx.x; i < ns * iv; i += kConsumerThreads) {
+                    const int tr = i / iv;
+                    const float *src = d.pairs ? p.h_routed + (size_t)__ldcg(d.pairs + s0 + tr) * Iu
+                                               : p.h_shared + (size_t)(s0 + tr) * Iu;
+                    hv[tr * rv + (i - tr * iv)] = __ldcg(reinterpret_cast<const float4 *>(src) + (i - tr * iv));
                 }
+                named_barrier(1, kConsumerThreads);
+            }
+            // h -> hi/lo e4m3 with one scale per (slot, 128 block): a warp per block
+            for (int u = warp; u < ns * ib; u += kConsumerWarps) {
+                const int tr = u / ib, kb = u - tr * ib;
+                const float4 v = reinterpret_cast<const float4 *>(st + L.hr + (size_t)tr * L.imax * 4)[kb * 32 + lane];
+                const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                const float sc = amax > 0.f ? amax / 448.f : 1.f;
+                uint32_t hi, lo;
+                quant4_hilo(v, 1.f / sc, hi, lo);
+                reinterpret_cast<uint32_t *>(st + L.hh + (size_t)tr * L.WS)[kb * 32 + lane] = hi;
+                reinterpret_cast<uint32_t *>(st + L.hl + (size_t)tr * L.WS)[kb * 32 + lane] = lo;
+                if (lane == 0) hsc[tr * (L.imax / 128) + kb] = sc;
+            }
+            named_barrier(1, kConsumerThreads);
+            // (tile, K block) units over the warps
+            float acc[kMaxTiles][4];
 #pragma unroll
-                for (int t = 0; t < kDnSlots; ++t) {
-                    if (t < ns) {
-                        const float y = warp_sum(acc[t]);
-                        if (lane == 0) {
-                            int yrow;
-                            float wt;
-                            if (v.pairs) {
-                                yrow = v.pairs[s0 + t];
-                                wt = p.topk_w[yrow];
-                            } else {
-                                yrow = p.rows * p.K + s0 + t;
-                                wt = p.gsig[s0 + t];
-                            }
-                            p.yslot[(size_t)yrow * p.H + n] = wt * y;
-                        }
+            for (int tau = 0; tau < kMaxTiles; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
+            const bool col_ok = g < ns;
+            for (int u = warp; u < L.T * ib; u += kConsumerWarps) {
+                const int tau = u % L.T, kb = u / L.T;
+                float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int k0 = kb * 128 + c * 32 + 8 * t;
+                    uint2 bh = make_uint2(0, 0), bl = make_uint2(0, 0);
+                    if (col_ok) {
+                        bh = *reinterpret_cast<const uint2 *>(st + L.hh + (size_t)g * L.WS + k0);
+                        bl = *reinterpret_cast<const uint2 *>(st + L.hl + (size_t)g * L.WS + k0);
+                    }
+                    const uint2 ra = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g) * L.WS + k0);
+                    const uint2 rb = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g + 8) * L.WS + k0);
+                    mma_e4m3_16832(tmp, ra.x, rb.x, ra.y, rb.y, bh.x, bh.y);
+                    mma_e4m3_16832(tmp, ra.x, rb.x, ra.y, rb.y, bl.x, bl.y);
+                }
+                const float ws_ = sw[kb];
+                const float h0 = (2 * t < ns) ? hsc[(2 * t) * (L.imax / 128) + kb] : 0.f;
+                const float h1 = (2 * t + 1 < ns) ? hsc[(2 * t + 1) * (L.imax / 128) + kb] : 0.f;
+#pragma unroll
+                for (int tt = 0; tt < kMaxTiles; ++tt) {
+                    if (tt == tau) {
+                        acc[tt][0] = fmaf(ws_ * h0, tmp[0], acc[tt][0]);
+                        acc[tt][1] = fmaf(ws_ * h1, tmp[1], acc[tt][1]);
+                        acc[tt][2] = fmaf(ws_ * h0, tmp[2], acc[tt][2]);
+                        acc[tt][3] = fmaf(ws_ * h1, tmp[3], acc[tt][3]);
                     }
                 }
             }
+#pragma unroll
+            for (int tau = 0; tau < kMaxTiles; ++tau)
+                if (tau < L.T)
+                    red[(warp * kMaxTiles + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
+            named_barrier(1, kConsumerThreads);
+            // (output row, slot column) -> weighted partial
+            for (int i = threadIdx.x; i < 128 * L.T; i += kConsumerThreads) {
+                const int tau = i >> 7, r = (i >> 3) & 15, n = i & 7;
+                if (n >= ns) continue;
+                const int src = (r & 7) * 4 + (n >> 1), comp = (n & 1) + (r >= 8 ? 2 : 0);
+                float y = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float4 v = red[(w * kMaxTiles + tau) * kWarp + src];
+                    y += comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w;
+                }
+                const int row = d.first + 16 * tau + r;
+                int yrow;
+                float wt;
+                if (d.pairs) {
+                    yrow = s0 == 0 ? d.rows[n] : __ldcg(d.pairs + s0 + n);
+                    wt = s0 == 0 ? d.wt[n] : __ldcg(p.topk_w + yrow);
+                } else {
+                    yrow = p.rows * p.K + s0 + n;
+                    wt = s0 == 0 ? d.wt[n] : __ldcg(p.gsig + s0 + n);
+                }
+                p.yslot[(size_t)yrow * p.H + row] = wt * y;
+            }
+            named_barrier(1, kConsumerThreads);  // red and the h staging are free again
         }
-        // The last item to finish this 32-row chunk blends it.
-        __syncthreads();
+        if (q < 2 && threadIdx.x == 0) MOE_TRACE(2, 3 + 3 * q);
+        const int chunk = d.first / p.drows;
+        named_barrier(1, kConsumerThreads);  // every warp is done with the stage and its descriptor
+        if (lane == 0) mbar_arrive(&empty[s]);  // the producer may refill the stage
+        // Count the item; the last item of a row block blends it.
         if (threadIdx.x == 0) {
-            __threadfence();
-            const int prev = atomicAdd(&p.counters[kCtrBlend + chunk], 1);
-            s_last = (prev == n_active);  // n_active routed items + 1 shared item per chunk
+            const int prev = skip ? -1 : atomic_add_acq_rel_gpu(p.counters + kCtrBlend + chunk, 1);
+            s_last = (prev == n_active);  // n_active routed items + 1 shared item per block
         }
-        __syncthreads();
+        named_barrier(1, kConsumerThreads);
         if (s_last) {
             __threadfence();
-            const int n0 = chunk * kDownRowsPerItem;
-            for (int i = threadIdx.x; i < p.rows * kDownRowsPerItem; i += blockDim.x) {
-                const int t = i / kDownRowsPerItem;
-                const int n = n0 + (i - t * kDownRowsPerItem);
-                float acc = 0.f;
-                for (int r = 0; r < p.K; ++r) acc += __ldcg(p.yslot + (size_t)(t * p.K + r) * p.H + n);
-                acc += __ldcg(p.yslot + (size_t)(p.rows * p.K + t) * p.H + n);
-                if (p.residual) acc += bf16_bits_to_f32(p.residual[(size_t)t * p.H + n]);
-                p.out[(size_t)t * p.H + n] = f32_to_bf16_bits(acc);
+            const int n0 = chunk * p.drows;
+            for (int i = threadIdx.x; i < p.rows * p.drows; i += kConsumerThreads) {
+                const int tr = i / p.drows;
+                const int n = n0 + (i - tr * p.drows);
+                float a = 0.f;
+                for (int r = 0; r < p.K; ++r) a += __ldcg(p.yslot + (size_t)(tr * p.K + r) * p.H + n);
+                a += __ldcg(p.yslot + (size_t)(p.rows * p.K + tr) * p.H + n);
+                if (p.residual) a += bf16_bits_to_f32(p.residual[(size_t)tr * p.H + n]);
+                p.out[(size_t)tr * p.H + n] = f32_to_bf16_bits(a);
             }
             if (threadIdx.x == 0) p.counters[kCtrBlend + chunk] = 0;
         }
+        named_barrier(1, kConsumerThreads);  // s_last is read by all before the next item sets it
+        if (q < 2 && threadIdx.x == 0) MOE_TRACE(2, 4 + 3 * q);
     }
+    if (threadIdx.x == 0) MOE_TRACE(2, 8);
+}
+
+#ifdef MOE_PHASE_TRACE
+extern "C" __attribute__((visibility("default"))) int moe_trace_set(void *p)
+{
+    return (int)cudaMemcpyToSymbol(g_moe_trace, &p, sizeof(p));
+}
+#endif
+
+// ------------------------------------------------------------ wait probe
+
+// One thread waits on an mbarrier that expects an arrival nobody makes, with
+// the same bounded wait the kernels use, and records the timeout.
+__global__ void wait_probe_kernel(int32_t *counters, uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0, limit_ns)) set_status(counters, MOE_ETIMEOUT);
 }
 
 // ------------------------------------------------------------- launchers
 
 namespace {
 
-template <typename P>
-cudaError_t launch_ex(void (*kernel)(P), int grid, int block, size_t smem, cudaStream_t s, const P &p)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, p);
-}
-
-int pick_kc(int cols_per_chunk, int n)  // smallest of 1,2,4,8 chunks covering n columns, else 8
-{
-    const int need = (n + cols_per_chunk - 1) / cols_per_chunk;
-    if (need <= 1) return 1;
-    if (need <= 2) return 2;
-    if (need <= 4) return 4;
-    return 8;
-}
-
-struct KernelSlot {
-    int device = -1;  // device the entry was measured on
-    int blocks_per_sm = 1;
-};
-
 std::mutex g_mu;
 
+// Blocks per SM of a kernel at a dynamic shared-memory size, per device.  On
+// first use on a device the kernel's dynamic shared-memory limit is set to
+// the most the device allows (the attribute sets the limit, it does not
+// raise it, so it is set once and never lowered).
 template <typename P>
-int occupancy(void (*kernel)(P), int block, size_t smem, KernelSlot &slot)
+int occupancy(void (*kernel)(P), int block, size_t smem)
 {
+    struct Entry {
+        const void *fn;
+        int device;
+        size_t smem;
+        int blocks;
+    };
+    static std::vector<Entry> cache;
+    static std::vector<std::pair<const void *, int>> configured;
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lk(g_mu);
-    if (slot.device != dev) {
-        if (smem > 48 * 1024) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, block, smem) != cudaSuccess || b < 1) b = 1;
-        slot.blocks_per_sm = b;
-        slot.device = dev;
+    for (const Entry &e : cache)
+        if (e.fn == (const void *)kernel && e.device == dev && e.smem == smem) return e.blocks;
+    bool done = false;
+    for (const auto &c : configured) done |= (c.first == (const void *)kernel && c.second == dev);
+    if (!done) {
+        cudaFuncAttributes fa{};
+        cudaFuncGetAttributes(&fa, kernel);
+        const size_t optin = device_info().max_smem_optin;
+        if (optin > fa.sharedSizeBytes)
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(optin - fa.sharedSizeBytes));
+        configured.push_back({(const void *)kernel, dev});
     }
-    return slot.blocks_per_sm;
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, block, smem) != cudaSuccess) b = 0;
+    cache.push_back({(const void *)kernel, dev, smem, b});
+    return b;
 }
 
 }  // namespace
 
+DecodeShape decode_shape(const moe_dims &d, int64_t rows)
+{
+    DecodeShape s{};
+    const int H = d.hidden, I = d.inter, Is = d.shared_inter, E = d.n_experts;
+    const int imax = std::max(I, Is);
+    rows = std::max<int64_t>(rows, 1);
+    // router: rows_per_cta router rows (<= 32 KB) and kRouterTok activation rows per CTA
+    s.router_rows = std::max(4, std::min(kRouterMaxRows, 32768 / H));
+    s.router_groups = (int)std::min<int64_t>((rows + kRouterTok - 1) / kRouterTok, kMaxRouterGroups);
+    s.router_group_tokens = (int)((rows + s.router_groups - 1) / s.router_groups);
+    s.router_smem = std::max<size_t>((size_t)(s.router_rows + kRouterTok) * H * 2, (size_t)(3 * E + 33) * 4);
+    s.logits_ld = (E + 1 + 3) / 4 * 4;
+    // activation rows per item: the 8 MMA columns, fewer for wide rows
+    s.tok = (int)std::min<int64_t>({(int64_t)kDescPairs, rows, std::max(1, 16384 / H)});
+    // gate_up: 8..32 pairs (a power of two: divides I and Is), ~32 KB of weights per item
+    int pairs = 8;
+    while (pairs * 2 <= 32 && pairs * 2 * 2 * H <= 32768) pairs *= 2;
+    s.gu_pairs = pairs;
+    const size_t ws_g = (size_t)H + kRowPad;
+    const size_t gu_stage = align16(16 * (pairs / 8) * ws_g + 2 * s.tok * ws_g + (size_t)s.tok * (H / 128) * 4 +
+                                    (size_t)2 * (H / 128) * 4);
+    // down: 16..64 rows (a power of two: divides H and 128), ~32 KB of weights per item
+    int drows = 16;
+    while (drows * 2 <= 64 && drows * 2 * imax <= 32768) drows *= 2;
+    s.dn_rows = drows;
+    const size_t ws_d = (size_t)imax + kRowPad;
+    const size_t dn_stage = align16(drows * ws_d + (size_t)s.tok * imax * 4 + 2 * s.tok * ws_d +
+                                    (size_t)s.tok * (imax / 128) * 4 + (size_t)(imax / 128) * 4);
+    const size_t red = (size_t)kConsumerWarps * kMaxTiles * kWarp * 16;
+    // One gate_up and one down CTA share an SM when they fit (down fetches
+    // its weights while gate_up streams); else each has the SM alone.
+    const size_t budget = 224 * 1024 - 2048;
+    int gs = 3, ds = 3;
+    while (gs * gu_stage + red + ds * dn_stage + red > budget && (gs > 2 || ds > 2)) {
+        if (gs * gu_stage >= ds * dn_stage && gs > 2) --gs;
+        else if (ds > 2) --ds;
+        else --gs;
+    }
+    if (gs * gu_stage + red + ds * dn_stage + red > budget) {
+        gs = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - red) / gu_stage));
+        ds = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - red) / dn_stage));
+    }
+    s.gu_stages = gs;
+    s.dn_stages = ds;
+    s.gu_smem = gs * gu_stage + red;
+    s.dn_smem = ds * dn_stage + red;
+    return s;
+}
+
+cudaError_t launch_wait_probe(int32_t *counters, uint64_t limit_ns, cudaStream_t s)
+{
+    wait_probe_kernel<<<1, 32, 0, s>>>(counters, limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s)
 {
     const moe_dims &d = *a.d;
+    const DecodeShape sh = decode_shape(d, a.rows);
     RouterParams p;
     p.x = a.x;
     p.rows = a.rows;
     p.H = d.hidden;
     p.E = d.n_experts;
     p.K = d.top_k;
+    p.ld = sh.logits_ld;
+    p.rows_per_cta = sh.router_rows;
+    p.group_tokens = sh.router_group_tokens;
     p.wr = a.router_w;
     p.bias = a.router_bias;
     p.g = a.shared_gate;
     p.logits = a.logits;
+    p.xq = a.xq;
+    p.xsc = a.xsc;
     p.topk_idx = a.topk_idx;
     p.topk_w = a.topk_w;
     p.gsig = a.gsig;
     p.counters = a.counters;
     p.plan = a.plan;
-    const int grid = (d.n_experts + 1 + kRouterWarps - 1) / kRouterWarps;
-    const size_t xs = (size_t)kRouterTok * d.hidden * 2;
-    const size_t plan_smem = a.plan ? (size_t)2 * d.n_experts * sizeof(int) : 0;
-    const size_t smem = xs > plan_smem ? xs : plan_smem;
-    const int need = (d.hidden + 255) / 256;
-    void (*k)(RouterParams);
-    if (need <= 2) k = router_topk_kernel<2>;
-    else if (need <= 4) k = router_topk_kernel<4>;
-    else if (need <= 8) k = router_topk_kernel<8>;
-    else k = router_topk_kernel<16>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    return launch_ex(k, grid, kRouterWarps * kWarp, smem, s, p);
+    const dim3 grid((d.n_experts + 1 + sh.router_rows - 1) / sh.router_rows,
+                    (a.rows + sh.router_group_tokens - 1) / sh.router_group_tokens);
+    if (occupancy(router_topk_kernel, sh.router_rows * kWarp, sh.router_smem) < 1)
+        return cudaErrorInvalidConfiguration;
+    return launch_kernel(router_topk_kernel, grid, dim3(sh.router_rows * kWarp), sh.router_smem, s, p);
 }
-
-static KernelSlot g_gu_slots[9], g_dn_slots[9];
 
 cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
 {
     const moe_dims &d = *a.d;
     const DeviceInfo &di = device_info();
+    const DecodeShape sh = decode_shape(d, a.rows);
     ExpertParams p;
     p.x = a.x;
+    p.xq = a.xq;
+    p.xsc = a.xsc;
     p.rows = a.rows;
     p.H = d.hidden;
     p.E = d.n_experts;
@@ -680,32 +1201,29 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
     p.residual = a.residual;
     p.out = a.out;
     p.counters = a.counters;
-
+    p.tok = sh.tok;
+    p.pairs = sh.gu_pairs;
+    p.drows = sh.dn_rows;
     const int64_t max_active = std::min<int64_t>(d.n_experts, (int64_t)a.rows * d.top_k);
 
     // gate_up
     {
-        const int kc = pick_kc(512, d.hidden);
-        void (*k)(ExpertParams) = kc == 1 ? gate_up_kernel<1> : kc == 2 ? gate_up_kernel<2>
-                                : kc == 4 ? gate_up_kernel<4> : gate_up_kernel<8>;
-        const size_t smem = (size_t)kGuTok * ((d.hidden + 511) / 512) * 64 * 16;
-        const int bps = occupancy(k, kGuWarps * kWarp, smem, g_gu_slots[kc]);
-        const int64_t items = max_active * (d.inter / kGuPairs) + d.shared_inter / kGuPairs;
-        const int grid = (int)std::min<int64_t>(items, (int64_t)bps * di.sm_count);
-        cudaError_t e = launch_ex(k, grid, kGuWarps * kWarp, smem, s, p);
+        p.stages = sh.gu_stages;
+        const int bps = occupancy(gate_up_kernel, kExpThreads, sh.gu_smem);
+        if (bps < 1) return cudaErrorInvalidConfiguration;
+        const int64_t items = (int64_t)(d.shared_inter / sh.gu_pairs) + max_active * (d.inter / sh.gu_pairs);
+        const int grid = (int)std::min<int64_t>(items, (int64_t)di.sm_count);
+        cudaError_t e = launch_kernel(gate_up_kernel, dim3(grid), dim3(kExpThreads), sh.gu_smem, s, p);
         if (e != cudaSuccess) return e;
     }
     // down + blend
     {
-        const int imax = d.inter > d.shared_inter ? d.inter : d.shared_inter;
-        const int kc = pick_kc(512, imax);
-        void (*k)(ExpertParams) = kc == 1 ? down_blend_kernel<1> : kc == 2 ? down_blend_kernel<2>
-                                : kc == 4 ? down_blend_kernel<4> : down_blend_kernel<8>;
-        const size_t smem = (size_t)kDnSlots * ((imax + 511) / 512) * 128 * 16;
-        const int bps = occupancy(k, kDnWarps * kWarp, smem, g_dn_slots[kc]);
-        const int64_t items = (max_active + 1) * (d.hidden / kDownRowsPerItem);
-        const int grid = (int)std::min<int64_t>(items, (int64_t)bps * di.sm_count);
-        cudaError_t e = launch_ex(k, grid, kDnWarps * kWarp, smem, s, p);
+        p.stages = sh.dn_stages;
+        const int bps = occupancy(down_blend_kernel, kExpThreads, sh.dn_smem);
+        if (bps < 1) return cudaErrorInvalidConfiguration;
+        const int64_t items = (max_active + 1) * (d.hidden / sh.dn_rows);
+        const int grid = (int)std::min<int64_t>(items, (int64_t)di.sm_count);
+        cudaError_t e = launch_kernel(down_blend_kernel, dim3(grid), dim3(kExpThreads), sh.dn_smem, s, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -11,17 +11,33 @@ namespace moe {
 
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
-constexpr int kCounters = 1024;         // int32 counters at the head of the workspace
-constexpr int kCtrRouter = 0;           // last-arriver counter of the router kernel
-constexpr int kCtrBlend = 64;           // first of the down/blend per-chunk counters
-constexpr int kDownRowsPerItem = 32;    // output rows per down work item (blend chunk)
+constexpr int kCounters = 4096;         // int32 counters at the head of the workspace
+constexpr int kCtrRouter = 0;           // last-arriver counter over the router's token groups
+constexpr int kCtrStatus = 1;           // device status word: 0, or a MOE_* error a kernel recorded
+constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per token-group counters
+constexpr int kMaxRouterGroups = 1024;
+constexpr int kCtrBlend = 2048;         // first of the down/blend per-row-block counters
+constexpr int kMaxBlendBlocks = kCounters - kCtrBlend;
+constexpr int kDescInts = 12;           // per active expert: {e, n, first pair, 0}, pair ids [8]
+constexpr int kDescPairs = 8;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Decode-path workspace, carved from the caller's buffer.
 struct DecodeLayout {
-    size_t counters, logits, topk_idx, topk_w, gsig, plan, h_routed, h_shared, yslot, total;
+    size_t counters, logits, xq, xsc, topk_idx, topk_w, gsig, plan, h_routed, h_shared, yslot, total;
 };
+
+// Tile shapes of the decode kernels for given dims and rows.
+struct DecodeShape {
+    int router_rows, router_groups, router_group_tokens, logits_ld;
+    size_t router_smem;
+    int gu_pairs, tok, gu_stages;
+    size_t gu_smem;
+    int dn_rows, dn_stages;
+    size_t dn_smem;
+};
+DecodeShape decode_shape(const moe_dims &d, int64_t rows);
 
 inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
 {
@@ -30,12 +46,14 @@ inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
     L.counters = take(sizeof(int32_t) * kCounters);
-    L.logits = take(sizeof(float) * rows * (E + 1));
+    L.logits = take(sizeof(float) * rows * ((E + 1 + 3) / 4 * 4));
+    L.xq = take((size_t)rows * 2 * H);
+    L.xsc = take(sizeof(float) * rows * (H / 128));
     L.topk_idx = take(sizeof(int32_t) * rows * K);
     L.topk_w = take(sizeof(float) * rows * K);
     L.gsig = take(sizeof(float) * rows);
-    // plan: n_active | active_expert[E] | active_off[E+1] | pair_list[rows*K]
-    L.plan = take(sizeof(int32_t) * (1 + E + (E + 1) + rows * K));
+    // plan: header[4] | descriptor[E][kDescInts] | pair ids[rows*K]
+    L.plan = take(sizeof(int32_t) * (4 + kDescInts * E + rows * K));
     L.h_routed = take(sizeof(float) * rows * K * I);
     L.h_shared = take(sizeof(float) * rows * Is);
     L.yslot = take(sizeof(float) * rows * (K + 1) * H);
@@ -63,6 +81,8 @@ struct RouterLaunch {
     float *topk_w;
     float *gsig;
     float *logits;   // workspace
+    uint8_t *xq;     // workspace: x as hi/lo e4m3 (nullptr: not needed)
+    float *xsc;
     int32_t *counters;
     int32_t *plan;   // nullptr: no plan
 };
@@ -71,6 +91,8 @@ cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s);
 struct ExpertsLaunch {
     const moe_dims *d;
     const uint16_t *x;
+    const uint8_t *xq;
+    const float *xsc;
     int32_t rows;
     const uint8_t *expert_w8;
     const float *expert_scales;
@@ -88,12 +110,17 @@ struct ExpertsLaunch {
     int32_t *counters;
 };
 cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s);
+// One CTA waits on an mbarrier that nothing completes, for at most limit_ns,
+// then records MOE_ETIMEOUT in counters[kCtrStatus].
+cudaError_t launch_wait_probe(int32_t *counters, uint64_t limit_ns, cudaStream_t s);
 
 // ------------------------------------------------------------ prefill path
 // Bytes of workspace for `rows` rows on either path.
 size_t workspace_bytes(const moe_dims &d, int64_t rows);
 // Whether the prefill path is built into this library.
 bool prefill_available();
+// Kernels one prefill call launches.
+int prefill_kernel_launches(const moe_dims &d, int64_t rows);
 // The prefill path (router GEMM, permute, grouped FP8 GEMMs, unpermute).
 // Returns a MOE_* status; launch errors come back as MOE_ECUDA.
 int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const uint16_t *router_w,

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "launch.h"
 
 namespace moe {
 
@@ -28,7 +29,7 @@ int check_dims(const moe_dims *d)
         return MOE_EUNSUPPORTED;
     if (d->hidden % 128 || d->inter % 128 || d->shared_inter % 128) return MOE_EUNSUPPORTED;
     if (d->top_k > d->n_experts || d->top_k > kMaxTopK || d->n_experts > kMaxExperts) return MOE_EUNSUPPORTED;
-    if (d->hidden / kDownRowsPerItem > kCounters - kCtrBlend) return MOE_EUNSUPPORTED;
+    if (d->hidden / 8 > kMaxBlendBlocks) return MOE_EUNSUPPORTED;
     return MOE_OK;
 }
 
@@ -60,6 +61,21 @@ int finish(cudaError_t e)
 }
 
 }  // namespace
+
+TimingSession &timing_session()
+{
+    static thread_local TimingSession ts;
+    return ts;
+}
+
+int kernel_launches(const moe_dims &d, int32_t rows, int32_t path)
+{
+    if (rows <= 0) return 0;
+    if (path == MOE_PATH_AUTO)
+        path = (rows <= MOE_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
+    if (path == MOE_PATH_PREFILL) return prefill_kernel_launches(d, rows);
+    return 3;  // router_topk, gate_up, down_blend
+}
 
 const DeviceInfo &device_info()
 {
@@ -109,6 +125,7 @@ int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
     int st = check_dims(d);
     if (st) return st;
     if (rows < 0) return MOE_EINVAL;
+    if (rows == 0) return enter();  // a no-op: no pointer is read
     if (!x || !router_w || !shared_gate || !topk_idx || !topk_w || !shared_gate_sig || !ws) return MOE_EINVAL;
     if (!aligned16(x) || !aligned16(router_w) || !aligned16(shared_gate) || !aligned16(ws) ||
         (router_bias && !aligned16(router_bias)) || !aligned16(topk_idx) || !aligned16(topk_w) ||
@@ -131,6 +148,8 @@ int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
     a.topk_w = topk_w;
     a.gsig = shared_gate_sig;
     a.logits = reinterpret_cast<float *>(base + L.logits);
+    a.xq = nullptr;
+    a.xsc = nullptr;
     a.counters = reinterpret_cast<int32_t *>(base + L.counters);
     a.plan = nullptr;
     return finish(launch_router_topk(a, static_cast<cudaStream_t>(stream)));
@@ -147,6 +166,7 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     if (st) return st;
     if (rows < 0) return MOE_EINVAL;
     if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_EINVAL;
+    if (rows == 0) return enter();  // a no-op: no pointer is read
     if (!x || !router_w || !expert_w8 || !expert_scales || !shared_w || !shared_w->w8 ||
         !shared_w->scales || !shared_gate || !out || !ws)
         return MOE_EINVAL;
@@ -191,6 +211,8 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     ra.topk_w = tw;
     ra.gsig = gs;
     ra.logits = reinterpret_cast<float *>(base + L.logits);
+    ra.xq = reinterpret_cast<uint8_t *>(base + L.xq);
+    ra.xsc = reinterpret_cast<float *>(base + L.xsc);
     ra.counters = counters;
     ra.plan = plan;
     cudaError_t e = launch_router_topk(ra, s);
@@ -199,6 +221,8 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     ExpertsLaunch ea;
     ea.d = d;
     ea.x = x;
+    ea.xq = reinterpret_cast<const uint8_t *>(base + L.xq);
+    ea.xsc = reinterpret_cast<const float *>(base + L.xsc);
     ea.rows = rows;
     ea.expert_w8 = expert_w8;
     ea.expert_scales = expert_scales;
@@ -227,6 +251,64 @@ int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
                                 nullptr, nullptr);
 }
 
+int32_t moe_kernel_launches(const moe_dims *d, int32_t rows, int32_t path)
+{
+    if (check_dims(d) != MOE_OK || rows < 0) return 0;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return 0;
+    return kernel_launches(*d, rows, path);
+}
+
+int moe_ffn_forward_timed(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                          const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                          const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
+                          const float *router_bias, void *ws, size_t ws_bytes, void *stream, int32_t path,
+                          void *const *events, int32_t n_events)
+{
+    if (!events || check_dims(d) != MOE_OK || rows < 0) return !events ? MOE_EINVAL : check_dims(d);
+    const int need = kernel_launches(*d, rows, path);
+    if (n_events < need + 1) return MOE_EINVAL;
+    for (int i = 0; i < need + 1; ++i)
+        if (!events[i]) return MOE_EINVAL;
+    TimingSession &ts = timing_session();
+    ts.events = reinterpret_cast<cudaEvent_t *>(const_cast<void **>(events));
+    ts.n_events = need + 1;
+    ts.next = 0;
+    ts.overflow = false;
+    int rc = moe_ffn_forward_path(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out,
+                                  residual, router_bias, ws, ws_bytes, stream, path, nullptr, nullptr, nullptr);
+    const int recorded = ts.next;
+    ts = TimingSession{};
+    if (rc != MOE_OK || rows == 0) return rc;
+    if (recorded != need) return MOE_EINVAL;
+    return finish(cudaEventRecord(static_cast<cudaEvent_t>(events[need]), static_cast<cudaStream_t>(stream)));
+}
+
+int moe_device_status(const void *ws, size_t ws_bytes, void *stream)
+{
+    if (!ws || ws_bytes < sizeof(int32_t) * kCounters || !aligned16(ws)) return MOE_EINVAL;
+    int32_t v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&v, static_cast<const int32_t *>(ws) + kCtrStatus, sizeof v,
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        g_status.store(MOE_ECUDA);
+        return MOE_ECUDA;
+    }
+    return v;
+}
+
+int moe_debug_wait_timeout(void *ws, size_t ws_bytes, int32_t limit_us, void *stream)
+{
+    if (!ws || ws_bytes < sizeof(int32_t) * kCounters || !aligned16(ws)) return MOE_EINVAL;
+    int st = enter();
+    if (st) return st;
+    if (limit_us < 1) limit_us = 1;
+    if (limit_us > 2000000) limit_us = 2000000;
+    return finish(launch_wait_probe(static_cast<int32_t *>(ws), (uint64_t)limit_us * 1000ull,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
 int moe_status(void) { return g_status.load(); }
 
 void moe_reset_status(void)
@@ -244,6 +326,7 @@ const char *moe_status_string(int status)
     case MOE_EUNSUPPORTED: return "unsupported dimensions (H, I, Is multiples of 128; k <= min(E, 32); E <= 1024)";
     case MOE_EWORKSPACE: return "workspace too small (see moe_workspace_bytes)";
     case MOE_ECUDA: return "CUDA error (sticky until moe_reset_status)";
+    case MOE_ETIMEOUT: return "a bounded wait inside a kernel ran out (re-initialise the workspace)";
     default: return "unknown status";
     }
 }

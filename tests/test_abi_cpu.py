@@ -82,6 +82,7 @@ def test_argument_checks_on_host(L):
     assert fwd(L, D(i=500)) == moe.MOE_EUNSUPPORTED
     assert fwd(L, d, ws_bytes=16) == moe.MOE_EWORKSPACE
     assert fwd(L, d, rows=0) == moe.MOE_OK                   # no-op, no CUDA call
+    assert fwd(L, d, rows=0, x=0, out=0, ws=0) == moe.MOE_OK  # empty tensors have null pointers
     assert L.moe_router_topk(ctypes.byref(d), None, 1, None, None, None, None, None, None, None, 0,
                              None) == moe.MOE_EINVAL
 
