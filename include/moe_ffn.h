@@ -165,6 +165,29 @@ MOE_API int moe_device_status(const void *ws, size_t ws_bytes, void *stream);
  * that moe_device_status reports it.  The GPU context stays usable. */
 MOE_API int moe_debug_wait_timeout(void *ws, size_t ws_bytes, int32_t limit_us, void *stream);
 
+/* moe_ffn_forward for callers that cannot allocate device memory (their
+ * device memory belongs to a host application's allocator, or they must not
+ * take an allocation path mid-run).  No counterpart on the reference pages:
+ * it is a library-service entry point.  Instead of a caller workspace it
+ * uses a scratch array built into the library, moe_static_scratch_bytes()
+ * large (16 MiB), of which every GPU that loads the library holds one copy
+ * until the process exits.  Calls whose moe_workspace_bytes(d, rows) exceeds
+ * it fail with MOE_EWORKSPACE.  The call allocates nothing (no cudaMalloc,
+ * no allocating library routine); it clears the array's counters on `stream`
+ * before launching.  The first call on a device looks up the array's device
+ * address, so make it before any stream capture.  All calls on a device
+ * share the one array: calls that overlap on the GPU race and must not be
+ * issued (serialise them on one stream).  Arguments and results are those of
+ * moe_ffn_forward. */
+MOE_API int moe_ffn_forward_static(const moe_dims *d, const uint16_t *x, int32_t rows,
+                           const uint16_t *router_w, const uint8_t *expert_w8,
+                           const float *expert_scales, const moe_fp8_expert *shared_w,
+                           const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
+                           const float *router_bias, void *stream);
+
+/* Size in bytes of the scratch array moe_ffn_forward_static uses. */
+MOE_API size_t moe_static_scratch_bytes(void);
+
 /* Sticky status: MOE_OK, or MOE_ECUDA after a CUDA error. */
 MOE_API int moe_status(void);
 /* Clear the sticky status (also clears a pending CUDA error of this thread). */

@@ -42,7 +42,8 @@ MOE_DECODE_MAX_ROWS = 64
 EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe_ffn_forward",
             "moe_ffn_forward_path", "moe_status", "moe_reset_status", "moe_status_string",
             "moe_debug_inject_fault", "moe_kernel_launches", "moe_ffn_forward_timed",
-            "moe_device_status", "moe_debug_wait_timeout")
+            "moe_device_status", "moe_debug_wait_timeout", "moe_ffn_forward_static",
+            "moe_static_scratch_bytes")
 
 
 class MoeDims(ctypes.Structure):
@@ -91,6 +92,9 @@ def lib() -> ctypes.CDLL:
                                             P, ctypes.c_size_t, P, I32, ctypes.POINTER(ctypes.c_void_p), I32]
         L.moe_device_status.argtypes = [P, ctypes.c_size_t, P]
         L.moe_debug_wait_timeout.argtypes = [P, ctypes.c_size_t, I32, P]
+        L.moe_ffn_forward_static.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P, P]
+        L.moe_static_scratch_bytes.argtypes = []
+        L.moe_static_scratch_bytes.restype = ctypes.c_size_t
         L.moe_status.argtypes = []
         L.moe_reset_status.argtypes = []
         L.moe_reset_status.restype = None
@@ -216,6 +220,23 @@ def device_status(ws, stream=None) -> int:
 def debug_wait_timeout(ws, limit_us: int, stream=None):
     _check(lib().moe_debug_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us),
                                         _stream(stream)), "moe_debug_wait_timeout")
+
+
+def ffn_forward_static(dims, x, router_w, expert_w8, expert_scales, shared_w8, shared_scales, shared_gate,
+                       out, residual=None, router_bias=None, stream=None):
+    """ffn_forward without a workspace: uses the library's built-in scratch
+    array (static_scratch_bytes() large); allocates nothing.  Calls that would
+    overlap on the GPU must not be issued (they share the array)."""
+    d = _dims(dims)
+    sh = MoeFp8Expert(_ptr(shared_w8), _ptr(shared_scales))
+    _check(lib().moe_ffn_forward_static(ctypes.byref(d), _ptr(x), _rows(x), _ptr(router_w), _ptr(expert_w8),
+                                        _ptr(expert_scales), ctypes.byref(sh), _ptr(shared_gate), _ptr(out),
+                                        _ptr(residual), _ptr(router_bias), _stream(stream)),
+           "moe_ffn_forward_static")
+
+
+def static_scratch_bytes() -> int:
+    return int(lib().moe_static_scratch_bytes())
 
 
 def status() -> int:
