@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "internal.h"
 #include "moe_ffn.h"
 
 namespace moe {
@@ -227,6 +228,12 @@ __device__ __forceinline__ float warp_max(float v)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
     return v;
+}
+
+// Record a device-side error in the workspace status word (first one wins).
+__device__ __forceinline__ void set_status(int32_t *counters, int32_t code)
+{
+    atomicCAS(&counters[kCtrStatus], 0, code);
 }
 
 // Default bound on any wait inside a kernel (wall time).

@@ -43,11 +43,6 @@ namespace moe {
 
 // ------------------------------------------------------------------ helpers
 
-__device__ __forceinline__ void set_status(int32_t *counters, int32_t code)
-{
-    atomicCAS(&counters[kCtrStatus], 0, code);
-}
-
 // 8 e4m3 codes (two words) against 8 bf16 activations (16 bytes).
 __device__ __forceinline__ float dot8_e4m3_bf16(uint2 w, uint4 x)
 {

@@ -1,19 +1,741 @@
-// prefill.cu -- prefill path (rows above a few dozen).
+// prefill.cu -- prefill path (rows above a few dozen): token permute ->
+// expert-grouped FP8 GEMMs on the tcgen05 tensor cores -> unpermute + blend.
+//
+// Launch chain (programmatic dependent launch between every pair):
+//   1. router_topk_kernel (decode.cu): router GEMV, top-k per row, and the
+//      activations x as hi/lo e4m3 rows with one scale per (row, 128 block).
+//   2. count_kernel: rows routed to each expert; each (row, rank) pair's
+//      position within its expert.
+//   3. scan_kernel (one CTA): expert offsets and the table of 128-row M tiles
+//      (routed experts in order, then the shared expert over all rows).
+//   4. permute_kernel: gathers each pair's hi/lo x row and scales into its
+//      expert's contiguous rows; records its position and blend weight.
+//   5. gemm_kernel<GEMM1>: per M tile and 128-column block j of h,
+//      [gate_j | up_j] = A (hi+lo) x W13^T on tcgen05 (M=128, N=256, K=32 per
+//      instruction), each 128-wide K block promoted into fp32 registers with
+//      its row scale x block scale; epilogue h = silu(gate) * up, quantised
+//      to hi/lo e4m3 with one scale per (row, 128 block) for GEMM2.
+//   6. gemm_kernel<GEMM2>: y = h (hi+lo) x W2^T the same way; epilogue
+//      scales by the row's routing weight (or the shared gate) into one
+//      partial row per (row, slot).
+//   7. blend_kernel: out[t] = sum of its k partials in rank order + the
+//      shared partial (+ residual), rounded once to bf16.
+//
+// Rows space of the GEMMs: the T*k routed pairs sorted by expert, then the T
+// shared-expert rows in token order.
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
 #include "internal.h"
+#include "launch.h"
+#include "tcgen05.cuh"
 
 namespace moe {
 
-size_t workspace_bytes(const moe_dims &d, int64_t rows) { return decode_layout(d, rows).total; }
+constexpr int kBM = 128;     // rows per M tile
+constexpr int kBN = 256;     // accumulator columns per tile
+constexpr int kBK = 128;     // K bytes per stage (one scale block of e4m3)
+constexpr int kGemmStages = 3;
+constexpr int kGemmThreads = 320;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2..9: epilogue
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
+constexpr size_t kStageBytes = 2 * kBM * kBK + kBN * kBK;  // A hi, A lo, B
+constexpr size_t kGemmSmem = kGemmStages * kStageBytes + 1024 /* alignment slack */ + 4096 /* epilogue scratch */;
 
-bool prefill_available() { return false; }
+// ------------------------------------------------------------ layout
 
-int prefill_kernel_launches(const moe_dims &, int64_t) { return 0; }
+struct PrefillLayout {
+    size_t counters, logits, xq, xsc, topk_idx, topk_w, gsig, counts, offsets, rank, pos, mtiles, xp, xps, slot_w,
+        hq, hs, yslot, total;
+    int64_t routed, rows_total, max_mtiles;
+};
 
-int prefill_forward(const moe_dims &, const uint16_t *, int32_t, const uint16_t *, const uint8_t *,
-                    const float *, const uint8_t *, const float *, const uint16_t *, uint16_t *,
-                    const uint16_t *, const float *, void *, cudaStream_t, int32_t *, float *, float *)
+inline PrefillLayout prefill_layout(const moe_dims &d, int64_t T)
 {
-    return MOE_EUNSUPPORTED;
+    PrefillLayout L{};
+    const int64_t E = d.n_experts, K = d.top_k, H = d.hidden, I = d.inter, Is = d.shared_inter;
+    const int64_t imax = std::max(I, Is);
+    L.routed = T * K;
+    L.rows_total = T * K + T;
+    L.max_mtiles = (T * K + kBM - 1) / kBM + E + (T + kBM - 1) / kBM + 1;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 1024); return at; };
+    L.counters = take(sizeof(int32_t) * kCounters);
+    L.logits = take(sizeof(float) * T * ((E + 1 + 3) / 4 * 4));
+    const int64_t Tp = std::max<int64_t>(T, kBM);  // TMA boxes are 128 rows: tensors have at least that many
+    L.xq = take((size_t)Tp * 2 * H);
+    L.xsc = take(sizeof(float) * T * (H / 128));
+    L.topk_idx = take(sizeof(int32_t) * T * K);
+    L.topk_w = take(sizeof(float) * T * K);
+    L.gsig = take(sizeof(float) * T);
+    L.counts = take(sizeof(int32_t) * (E + 1));
+    L.offsets = take(sizeof(int32_t) * (E + 2));
+    L.rank = take(sizeof(int32_t) * T * K);
+    L.pos = take(sizeof(int32_t) * T * K);
+    L.mtiles = take(sizeof(int4) * (1 + L.max_mtiles));
+    L.xp = take((size_t)std::max<int64_t>(L.routed, kBM) * 2 * H);
+    L.xps = take(sizeof(float) * std::max<int64_t>(L.routed, 1) * (H / 128));
+    L.slot_w = take(sizeof(float) * L.rows_total);
+    L.hq = take((size_t)std::max<int64_t>(L.rows_total, kBM) * 2 * imax);
+    L.hs = take(sizeof(float) * L.rows_total * (imax / 128));
+    L.yslot = take(sizeof(float) * L.rows_total * H);
+    L.total = o;
+    return L;
+}
+
+size_t workspace_bytes(const moe_dims &d, int64_t rows)
+{
+    return std::max(decode_layout(d, rows).total, prefill_layout(d, rows).total);
+}
+
+bool prefill_available() { return true; }
+
+int prefill_kernel_launches(const moe_dims &, int64_t) { return 7; }
+
+// ------------------------------------------------------------ count / scan / permute
+
+struct PlanParams {
+    int T, E, K, H, I, Is;
+    const int32_t *topk_idx;
+    const float *topk_w;
+    const float *gsig;
+    int32_t *counts;   // [E]
+    int32_t *offsets;  // [E+1]
+    int32_t *rank;     // [T*K]
+    int32_t *pos;      // [T*K]
+    int4 *mtiles;      // [0].x = count; entries from [1]: {group, row0, rows, a_row0}
+    const uint8_t *xq;
+    const float *xsc;
+    uint8_t *xp;
+    float *xps;
+    float *slot_w;
+    int32_t *counters;
+};
+
+__global__ void __launch_bounds__(256) count_kernel(PlanParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int P = p.T * p.K;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P; i += gridDim.x * blockDim.x) {
+        int e = p.topk_idx[i];
+        e = min(max(e, 0), p.E - 1);
+        p.rank[i] = atomicAdd(&p.counts[e], 1);
+    }
+}
+
+__device__ int block_scan_excl(int v, int *scratch, int *total)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = (lane < nwarps) ? scratch[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nwarps) scratch[lane] = wi - w;
+        if (lane == 31) scratch[32] = wi;
+    }
+    __syncthreads();
+    const int r = scratch[warp] + incl - v;
+    *total = scratch[32];
+    __syncthreads();
+    return r;
+}
+
+// One CTA of 1024 threads: expert offsets and the M-tile table.
+__global__ void __launch_bounds__(1024) scan_kernel(PlanParams p)
+{
+    __shared__ int scratch[33];
+    pdl_wait();
+    pdl_trigger();
+    int run_rows = 0, run_tiles = 0;
+    for (int e0 = 0; e0 < p.E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        const int c = (e < p.E) ? p.counts[e] : 0;
+        const int mt = (c + kBM - 1) / kBM;
+        int tot_rows, tot_tiles;
+        const int off = block_scan_excl(c, scratch, &tot_rows) + run_rows;
+        const int toff = block_scan_excl(mt, scratch, &tot_tiles) + run_tiles;
+        if (e < p.E) {
+            p.offsets[e] = off;
+            for (int i = 0; i < mt; ++i)
+                p.mtiles[1 + toff + i] = make_int4(e, off + i * kBM, min(kBM, c - i * kBM), off + i * kBM);
+        }
+        run_rows += tot_rows;
+        run_tiles += tot_tiles;
+    }
+    if (threadIdx.x == 0) p.offsets[p.E] = run_rows;
+    // the shared expert: all T rows, in token order, after the routed rows
+    const int smt = (p.T + kBM - 1) / kBM;
+    for (int i = threadIdx.x; i < smt; i += blockDim.x)
+        p.mtiles[1 + run_tiles + i] = make_int4(p.E, p.T * p.K + i * kBM, min(kBM, p.T - i * kBM), i * kBM);
+    if (threadIdx.x == 0) p.mtiles[0] = make_int4(run_tiles + smt, run_tiles, 0, 0);
+}
+
+// A warp per routed pair (plus the shared rows' blend weights): the pair's
+// hi/lo x row and scales into its expert's rows.
+__global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int P = p.T * p.K;
+    const int hb = p.H / 128;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    for (int i = gw; i < P + p.T; i += nw) {
+        if (i >= P) {
+            if (lane == 0) p.slot_w[i] = p.gsig[i - P];
+            continue;
+        }
+        const int t = i / p.K;
+        const int e = min(max(p.topk_idx[i], 0), p.E - 1);
+        const int dst = p.offsets[e] + p.rank[i];
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.xq + (size_t)t * 2 * p.H);
+        uint4 *dv = reinterpret_cast<uint4 *>(p.xp + (size_t)dst * 2 * p.H);
+        for (int c = lane; c < p.H / 8; c += 32) dv[c] = src[c];
+        for (int c = lane; c < hb; c += 32) p.xps[(size_t)dst * hb + c] = p.xsc[(size_t)t * hb + c];
+        if (lane == 0) {
+            p.pos[i] = dst;
+            p.slot_w[dst] = p.topk_w[i];
+        }
+    }
+}
+
+// ------------------------------------------------------------ grouped GEMM
+
+struct GemmParams {
+    CUtensorMap a_routed;  // A rows of the routed groups (GEMM1: permuted x; GEMM2: h)
+    CUtensorMap a_shared;  // A rows of the shared group (GEMM1: x in token order; GEMM2: h)
+    CUtensorMap b_routed;  // 3D: (K bytes, rows, expert)
+    CUtensorMap b_shared;  // 3D with one expert
+    int H, E, I, Is;
+    int imax;
+    const int4 *mtiles;
+    const float *a_scales_routed;  // [rows][K/128]
+    const float *a_scales_shared;
+    int a_scales_ld;               // floats per row of the A scales
+    const float *w_scales;         // routed experts' scale slabs
+    const float *w_scales_shared;
+    uint8_t *hq;                   // GEMM1 out: [rows][2*imax] (hi | lo)
+    float *hs;                     // GEMM1 out: [rows][imax/128]
+    const float *slot_w;           // GEMM2: blend weight per row
+    float *yslot;                  // GEMM2 out: [rows][H]
+    int32_t *counters;
+    int max_ntiles;
+};
+
+// Per tile facts every role needs.
+struct TileInfo {
+    int group, row0, rows, a_row0, nt, kdim, ntiles;
+    bool shared_grp;
+};
+
+template <int MODE>
+__device__ __forceinline__ bool tile_info(const GemmParams &p, int n_mtiles, int t, TileInfo &ti)
+{
+    const int mt = t / p.max_ntiles;
+    ti.nt = t - mt * p.max_ntiles;
+    if (mt >= n_mtiles) return false;
+    const int4 m = __ldcg(p.mtiles + 1 + mt);
+    ti.group = m.x;
+    ti.row0 = m.y;
+    ti.rows = m.z;
+    ti.a_row0 = m.w;
+    ti.shared_grp = (m.x == p.E);
+    const int inter = ti.shared_grp ? p.Is : p.I;
+    if (MODE == 1) {
+        ti.kdim = p.H;
+        ti.ntiles = inter / 128;  // one 128-column block of h per tile
+    } else {
+        ti.kdim = inter;
+        ti.ntiles = p.H / kBN;
+    }
+    return true;
+}
+
+// MODE 1 (GEMM1): B tile = gate rows [128 nt, +128) and up rows [inter + 128 nt, +128) of W13.
+// MODE 2 (GEMM2): B tile = rows [256 nt, +256) of W2.
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], acc_full[2], acc_empty[2];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    float *epi_scratch = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes);  // [2][128] amax exchange
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kEpiThreads / 32);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_s, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&p.a_routed);
+        tma_prefetch_desc(&p.a_shared);
+        tma_prefetch_desc(&p.b_routed);
+        tma_prefetch_desc(&p.b_shared);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    pdl_wait();
+    pdl_trigger();
+    const int n_mtiles = __ldcg(p.mtiles).x;
+    const int n_tiles = n_mtiles * p.max_ntiles;
+
+    if (warp == 0) {
+        // --------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();  // weights stream once per M tile
+            const uint64_t pol_a = policy_evict_last();   // activations are re-read for every N tile
+            int it = 0;
+            for (int t = blockIdx.x; t < n_tiles && !s_abort; t += gridDim.x) {
+                TileInfo ti;
+                if (!tile_info<MODE>(p, n_mtiles, t, ti) || ti.nt >= ti.ntiles) continue;
+                const int nkb = ti.kdim / kBK;
+                const CUtensorMap *amap = ti.shared_grp ? &p.a_shared : &p.a_routed;
+                const CUtensorMap *bmap = ti.shared_grp ? &p.b_shared : &p.b_routed;
+                const int ez = ti.shared_grp ? 0 : ti.group;
+                const int inter = ti.shared_grp ? p.Is : p.I;
+                // A rows: GEMM1 reads x rows (permuted rows, or token rows for the
+                // shared group); GEMM2 reads h at the tile's rows of the row space.
+                const int arow = MODE == 1 ? ti.a_row0 : ti.row0;
+                const int lo_x = MODE == 1 ? p.H : p.imax;  // where the lo half of a row starts
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kGemmStages;
+                    if (it >= kGemmStages && !mbar_wait(&empty[s], ((it / kGemmStages) - 1) & 1, kWaitLimitNs)) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        break;
+                    }
+                    unsigned char *st = smem + s * kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)kStageBytes);
+                    // A: hi at x = kb*128, lo at x = kdim + kb*128 of the row
+                    tma_load_2d(st, amap, kb * kBK, arow, &full[s], pol_a);
+                    tma_load_2d(st + kBM * kBK, amap, lo_x + kb * kBK, arow, &full[s], pol_a);
+                    unsigned char *bt = st + 2 * kBM * kBK;
+                    if (MODE == 1) {
+                        tma_load_3d(bt, bmap, kb * kBK, ti.nt * 128, ez, &full[s], pol_w);
+                        tma_load_3d(bt + 128 * kBK, bmap, kb * kBK, inter + ti.nt * 128, ez, &full[s], pol_w);
+                    } else {
+                        tma_load_3d(bt, bmap, kb * kBK, ti.nt * kBN, ez, &full[s], pol_w);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_e4m3_f32(kBM, kBN);
+            int it = 0, acc_it = 0;
+            for (int t = blockIdx.x; t < n_tiles && !s_abort; t += gridDim.x) {
+                TileInfo ti;
+                if (!tile_info<MODE>(p, n_mtiles, t, ti) || ti.nt >= ti.ntiles) continue;
+                const int nkb = ti.kdim / kBK;
+                for (int kb = 0; kb < nkb; ++kb, ++it, ++acc_it) {
+                    const int s = it % kGemmStages;
+                    const int b = acc_it & 1;
+                    if (!mbar_wait(&full[s], (it / kGemmStages) & 1, kWaitLimitNs) ||
+                        (acc_it >= 2 && !mbar_wait(&acc_empty[b], ((acc_it >> 1) - 1) & 1, kWaitLimitNs))) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + s * kStageBytes);
+                    const uint32_t d = tmem_base + (uint32_t)(b * kBN);
+                    const uint32_t bsm = st + 2 * kBM * kBK;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {  // hi, then lo
+                        const uint32_t asm_ = st + part * kBM * kBK;
+#pragma unroll
+                        for (int k4 = 0; k4 < kBK / 32; ++k4)
+                            umma_f8f6f4(d, umma_desc_sw128(asm_ + k4 * 32), umma_desc_sw128(bsm + k4 * 32), idesc,
+                                        (part | k4) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);   // the stage may be refilled once these MMAs have read it
+                    umma_commit(&acc_full[b]);  // the K block's partial sum is ready
+                }
+            }
+        }
+    } else {
+        // --------------------------------------------------- epilogue (warps 2..9)
+        const int q = warp & 3;                   // TMEM lane quadrant of this warp
+        const int half = (warp - 2) >> 2;          // column half
+        const int r = q * 32 + lane;               // row within the tile
+        const int et = threadIdx.x - 64;           // 0..255
+        int acc_it = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+            TileInfo ti;
+            if (!tile_info<MODE>(p, n_mtiles, t, ti) || ti.nt >= ti.ntiles) continue;
+            const int nkb = ti.kdim / kBK;
+            const bool valid = r < ti.rows;
+            const int arow = (MODE == 1 ? ti.a_row0 : ti.row0) + r;  // row in the A tensor (and its scales)
+            const float *asc = (ti.shared_grp ? p.a_scales_shared : p.a_scales_routed) + (size_t)arow * p.a_scales_ld;
+            const int inter = ti.shared_grp ? p.Is : p.I;
+            const float *wsc;
+            int wld, wn0, wn1;  // scale rows of the tile's two column halves
+            if (MODE == 1) {
+                wsc = ti.shared_grp ? p.w_scales_shared
+                                    : p.w_scales + (size_t)ti.group * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128));
+                wld = p.H / 128;
+                wn0 = ti.nt;                 // gate block row
+                wn1 = inter / 128 + ti.nt;   // up block row
+            } else {
+                wsc = (ti.shared_grp ? p.w_scales_shared
+                                     : p.w_scales + (size_t)ti.group * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128))) +
+                      (2 * inter / 128) * (p.H / 128);
+                wld = inter / 128;
+                wn0 = ti.nt * 2;
+                wn1 = ti.nt * 2 + 1;
+            }
+            float tot[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) tot[i] = 0.f;
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb, ++acc_it) {
+                const int b = acc_it & 1;
+                const float sa = (valid && ok) ? __ldg(asc + kb) : 0.f;
+                const float s0 = __ldg(wsc + (size_t)wn0 * wld + kb), s1 = __ldg(wsc + (size_t)wn1 * wld + kb);
+                if (ok && !mbar_wait(&acc_full[b], (acc_it >> 1) & 1, kWaitLimitNs)) {
+                    set_status(p.counters, MOE_ETIMEOUT);
+                    s_abort = 1;
+                    ok = false;
+                }
+                if (!ok) continue;
+                tc_fence_after();
+                const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kBN);
+                // MODE 1: this thread's columns are [64 half, +64) (gate) and [128 + 64 half, +64) (up)
+                // MODE 2: [128 half, +128)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    int col;
+                    float sc;
+                    if (MODE == 1) {
+                        col = (c < 2) ? (64 * half + 32 * c) : (128 + 64 * half + 32 * (c - 2));
+                        sc = sa * ((c < 2) ? s0 : s1);
+                    } else {
+                        col = 128 * half + 32 * c;
+                        sc = sa * (half ? s1 : s0);
+                    }
+                    float v[32];
+                    tmem_ld_32x32(tbase + (uint32_t)col, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) tot[32 * c + i] = fmaf(sc, v[i], tot[32 * c + i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+            }
+            if (MODE == 1) {
+                // h = silu(gate) * up for this thread's 64 columns of the block
+                float amax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const float g = tot[i], u = tot[64 + i];
+                    const float hv = g / (1.f + __expf(-g)) * u;
+                    tot[i] = hv;
+                    amax = fmaxf(amax, fabsf(hv));
+                }
+                // both halves of the row's 128-column block share one scale
+                named_barrier(2, kEpiThreads);
+                epi_scratch[half * 128 + r] = amax;
+                named_barrier(2, kEpiThreads);
+                amax = fmaxf(epi_scratch[r], epi_scratch[128 + r]);
+                const float sc = amax > 0.f ? amax / 448.f : 1.f;
+                const float inv = 1.f / sc;
+                if (valid && ok) {
+                    const size_t grow = (size_t)ti.row0 + r;
+                    uint32_t *hi = reinterpret_cast<uint32_t *>(p.hq + grow * 2 * p.imax + ti.nt * 128 + 64 * half);
+                    uint32_t *lo = reinterpret_cast<uint32_t *>(p.hq + grow * 2 * p.imax + p.imax + ti.nt * 128 + 64 * half);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t h4, l4;
+                        quant4_hilo(make_float4(tot[4 * i], tot[4 * i + 1], tot[4 * i + 2], tot[4 * i + 3]), inv, h4, l4);
+                        hi[i] = h4;
+                        lo[i] = l4;
+                    }
+                    if (half == 0) p.hs[grow * (p.imax / 128) + ti.nt] = sc;
+                }
+            } else {
+                if (valid && ok) {
+                    const size_t grow = (size_t)ti.row0 + r;
+                    const float w = __ldg(p.slot_w + grow);
+                    float4 *y = reinterpret_cast<float4 *>(p.yslot + grow * p.H + ti.nt * kBN + 128 * half);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        y[i] = make_float4(w * tot[4 * i], w * tot[4 * i + 1], w * tot[4 * i + 2], w * tot[4 * i + 3]);
+                }
+            }
+            (void)et;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------ blend
+
+struct BlendParams {
+    int T, K, H;
+    const int32_t *pos;
+    const float *yslot;
+    const uint16_t *residual;
+    uint16_t *out;
+};
+
+// out[t] = sum_r yslot[pos(t, r)] (rank order) + yslot[T*K + t] (+ residual)
+__global__ void __launch_bounds__(256) blend_kernel(BlendParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int nv = p.H / 4;
+    const size_t total = (size_t)p.T * nv;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / nv), c = (int)(i - (size_t)t * nv);
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < p.K; ++r) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.yslot + (size_t)p.pos[t * p.K + r] * p.H) + c);
+            a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+        }
+        const float4 s = __ldcg(reinterpret_cast<const float4 *>(p.yslot + ((size_t)p.T * p.K + t) * p.H) + c);
+        a.x += s.x; a.y += s.y; a.z += s.z; a.w += s.w;
+        if (p.residual) {
+            const uint2 rv = reinterpret_cast<const uint2 *>(p.residual + (size_t)t * p.H)[c];
+            a.x += bf16_lo(rv.x); a.y += bf16_hi(rv.x); a.z += bf16_lo(rv.y); a.w += bf16_hi(rv.y);
+        }
+        uint2 o;
+        o.x = (uint32_t)f32_to_bf16_bits(a.x) | ((uint32_t)f32_to_bf16_bits(a.y) << 16);
+        o.y = (uint32_t)f32_to_bf16_bits(a.z) | ((uint32_t)f32_to_bf16_bits(a.w) << 16);
+        reinterpret_cast<uint2 *>(p.out + (size_t)t * p.H)[c] = o;
+    }
+}
+
+// ------------------------------------------------------------ host side
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// A byte tensor [outer][rows][inner] (inner contiguous) as a TMA map with
+// 128-byte-swizzled boxes of [128 bytes, box_rows, 1].
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t outer, uint64_t row_stride,
+              uint64_t outer_stride, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {inner, rows, outer};
+    const cuuint64_t strides[2] = {row_stride, outer_stride};
+    const cuuint32_t box[3] = {128, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const cuuint32_t rank = outer > 1 || outer_stride ? 3 : 2;
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename P>
+int gemm_occupancy_once(void (*kernel)(P))
+{
+    static std::mutex mu;
+    static std::vector<std::pair<const void *, int>> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    for (auto &d : done)
+        if (d.first == (const void *)kernel && d.second == dev) return 1;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) != cudaSuccess)
+        return 0;
+    done.push_back({(const void *)kernel, dev});
+    return 1;
+}
+
+}  // namespace
+
+int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                    const uint8_t *expert_w8, const float *expert_scales, const uint8_t *shared_w8,
+                    const float *shared_scales, const uint16_t *shared_gate, uint16_t *out,
+                    const uint16_t *residual, const float *router_bias, void *ws, cudaStream_t s,
+                    int32_t *topk_idx_out, float *topk_w_out, float *gsig_out)
+{
+    const int T = rows, E = d.n_experts, K = d.top_k, H = d.hidden, I = d.inter, Is = d.shared_inter;
+    const int imax = std::max(I, Is);
+    if (H % kBN || H % kBK) return MOE_EUNSUPPORTED;  // GEMM2 N tiles of 256 columns
+    const PrefillLayout L = prefill_layout(d, T);
+    char *base = static_cast<char *>(ws);
+    int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
+    int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
+    float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
+    float *gs = gsig_out ? gsig_out : reinterpret_cast<float *>(base + L.gsig);
+    uint8_t *xq = reinterpret_cast<uint8_t *>(base + L.xq);
+    float *xsc = reinterpret_cast<float *>(base + L.xsc);
+
+    cudaError_t e = cudaMemsetAsync(base + L.counts, 0, sizeof(int32_t) * (E + 1), s);
+    if (e != cudaSuccess) return MOE_ECUDA;
+
+    // 1. router + top-k + x in hi/lo e4m3
+    RouterLaunch ra;
+    ra.d = &d;
+    ra.x = x;
+    ra.rows = rows;
+    ra.router_w = router_w;
+    ra.router_bias = router_bias;
+    ra.shared_gate = shared_gate;
+    ra.topk_idx = tidx;
+    ra.topk_w = tw;
+    ra.gsig = gs;
+    ra.logits = reinterpret_cast<float *>(base + L.logits);
+    ra.xq = xq;
+    ra.xsc = xsc;
+    ra.counters = counters;
+    ra.plan = nullptr;
+    if ((e = launch_router_topk(ra, s)) != cudaSuccess) return MOE_ECUDA;
+
+    PlanParams pp;
+    pp.T = T;
+    pp.E = E;
+    pp.K = K;
+    pp.H = H;
+    pp.I = I;
+    pp.Is = Is;
+    pp.topk_idx = tidx;
+    pp.topk_w = tw;
+    pp.gsig = gs;
+    pp.counts = reinterpret_cast<int32_t *>(base + L.counts);
+    pp.offsets = reinterpret_cast<int32_t *>(base + L.offsets);
+    pp.rank = reinterpret_cast<int32_t *>(base + L.rank);
+    pp.pos = reinterpret_cast<int32_t *>(base + L.pos);
+    pp.mtiles = reinterpret_cast<int4 *>(base + L.mtiles);
+    pp.xq = xq;
+    pp.xsc = xsc;
+    pp.xp = reinterpret_cast<uint8_t *>(base + L.xp);
+    pp.xps = reinterpret_cast<float *>(base + L.xps);
+    pp.slot_w = reinterpret_cast<float *>(base + L.slot_w);
+    pp.counters = counters;
+    const DeviceInfo &di = device_info();
+    const int P = T * K;
+    // 2..4
+    if ((e = launch_kernel(count_kernel, dim3(std::max(1, std::min(4 * di.sm_count, (P + 255) / 256))), dim3(256),
+                           0, s, pp)) != cudaSuccess)
+        return MOE_ECUDA;
+    if ((e = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pp)) != cudaSuccess) return MOE_ECUDA;
+    if ((e = launch_kernel(permute_kernel, dim3(std::max(1, std::min(8 * di.sm_count, (P + T + 7) / 8))), dim3(256),
+                           0, s, pp)) != cudaSuccess)
+        return MOE_ECUDA;
+
+    // 5. GEMM1
+    GemmParams g{};
+    g.H = H;
+    g.E = E;
+    g.I = I;
+    g.Is = Is;
+    g.imax = imax;
+    g.mtiles = pp.mtiles;
+    g.w_scales = expert_scales;
+    g.w_scales_shared = shared_scales;
+    g.hq = reinterpret_cast<uint8_t *>(base + L.hq);
+    g.hs = reinterpret_cast<float *>(base + L.hs);
+    g.slot_w = pp.slot_w;
+    g.yslot = reinterpret_cast<float *>(base + L.yslot);
+    g.counters = counters;
+    const int64_t R = L.rows_total;
+    // A tensors are declared with at least 128 rows (their buffers are that
+    // large); rows past the valid ones are read but never stored.
+    bool ok = make_map(&g.a_routed, pp.xp, 2 * (uint64_t)H, (uint64_t)std::max<int64_t>(L.routed, kBM), 1,
+                       2 * (uint64_t)H, 0, kBM) &&
+              make_map(&g.a_shared, xq, 2 * (uint64_t)H, (uint64_t)std::max(T, kBM), 1, 2 * (uint64_t)H, 0, kBM) &&
+              make_map(&g.b_routed, expert_w8, (uint64_t)H, 2 * (uint64_t)I, (uint64_t)E, (uint64_t)H,
+                       3 * (uint64_t)I * H, 128) &&
+              make_map(&g.b_shared, shared_w8, (uint64_t)H, 2 * (uint64_t)Is, 1, (uint64_t)H, 3 * (uint64_t)Is * H, 128);
+    if (!ok) return MOE_ECUDA;
+    g.a_scales_routed = pp.xps;
+    g.a_scales_shared = xsc;
+    g.a_scales_ld = H / 128;
+    g.max_ntiles = imax / 128;
+    if (!gemm_occupancy_once(gemm_kernel<1>) || !gemm_occupancy_once(gemm_kernel<2>)) return MOE_ECUDA;
+    if ((e = launch_kernel(gemm_kernel<1>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g)) != cudaSuccess)
+        return MOE_ECUDA;
+
+    // 6. GEMM2
+    GemmParams g2 = g;
+    const uint64_t Rp = (uint64_t)std::max<int64_t>(R, kBM);
+    ok = make_map(&g2.a_routed, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, kBM) &&
+         make_map(&g2.a_shared, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, kBM) &&
+         make_map(&g2.b_routed, expert_w8 + (size_t)2 * I * H, (uint64_t)I, (uint64_t)H, (uint64_t)E, (uint64_t)I,
+                  3 * (uint64_t)I * H, kBN) &&
+         make_map(&g2.b_shared, shared_w8 + (size_t)2 * Is * H, (uint64_t)Is, (uint64_t)H, 1, (uint64_t)Is,
+                  3 * (uint64_t)Is * H, kBN);
+    if (!ok) return MOE_ECUDA;
+    g2.a_scales_routed = g.hs;
+    g2.a_scales_shared = g.hs;
+    g2.a_scales_ld = imax / 128;
+    g2.max_ntiles = H / kBN;
+    if ((e = launch_kernel(gemm_kernel<2>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g2)) != cudaSuccess)
+        return MOE_ECUDA;
+
+    // 7. blend
+    BlendParams bp;
+    bp.T = T;
+    bp.K = K;
+    bp.H = H;
+    bp.pos = pp.pos;
+    bp.yslot = g.yslot;
+    bp.residual = residual;
+    bp.out = out;
+    const size_t work = (size_t)T * (H / 4);
+    if ((e = launch_kernel(blend_kernel, dim3((unsigned)std::min<size_t>(8 * di.sm_count, (work + 255) / 256)),
+                           dim3(256), 0, s, bp)) != cudaSuccess)
+        return MOE_ECUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 }  // namespace moe

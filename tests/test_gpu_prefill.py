@@ -1,0 +1,78 @@
+"""GPU parity of the prefill path (token permute -> tcgen05 FP8 grouped GEMMs
+-> unpermute) against the CPU oracle, through the C ABI.
+
+Small shapes are checked on every row; the 4096-row Qwen3.6-35B-A3B-shaped
+prefill (router bias for uneven expert loads) is checked on its routing for
+every row and on the output of sampled rows, which the oracle computes one
+by one (rows are independent in the layer).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+moe = pytest.importorskip("sparse_moe_ffn_topk_b200")
+
+
+def run(case, path, dev=None):
+    d = case.dims
+    dev = dev or P.device_weights(case.layer)
+    rows = case.x.shape[0]
+    out = torch.empty(rows, d.hidden, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(rows, d.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(rows, d.top_k, dtype=torch.float32, device="cuda")
+    gs = torch.empty(rows, dtype=torch.float32, device="cuda")
+    ws = moe.alloc_workspace(d, rows)
+    res = P.bf16_tensor(case.residual) if case.residual is not None else None
+    moe.ffn_forward_path(d, P.bf16_tensor(case.x), dev["router_w"], dev["expert_w8"], dev["expert_scales"],
+                         dev["shared_w8"], dev["shared_scales"], dev["shared_gate"], out, ws, path=path,
+                         residual=res, router_bias=dev["router_bias"], topk_idx=idx, topk_w=w, shared_gate_sig=gs)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws) == moe.MOE_OK
+    return P.bf16_to_f64(out), idx.cpu().numpy(), w.cpu().numpy(), gs.cpu().numpy()
+
+
+@pytest.mark.parametrize("dims,rows,bias", [
+    (mi.TINY, 4, False),
+    (mi.TINY, 100, True),
+    (mi.LayerDims(hidden=512, n_experts=32, top_k=4, inter=256, shared_inter=256), 300, True),
+    (mi.LayerDims(hidden=256, n_experts=16, top_k=2, inter=128, shared_inter=256), 130, False),   # I != Is
+    (mi.LayerDims(hidden=768, n_experts=12, top_k=3, inter=384, shared_inter=128), 200, True),
+])
+def test_prefill_small_shapes(dims, rows, bias):
+    case = P.build_case(dims, rows, router_bias=bias, all_experts=True, residual=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL)
+    _, oidx, ow, ogs = oracle.router_topk(dims, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
+
+
+def test_auto_path_uses_prefill_above_64_rows():
+    d = mi.TINY
+    assert moe.kernel_launches(d, 64) == 3
+    assert moe.kernel_launches(d, 65) == 7
+    case = P.build_case(d, 65, all_experts=True)
+    out, idx, _, _ = run(case, moe.MOE_PATH_AUTO)
+    P.compare_output(case, out, idx)
+
+
+def test_qwen36_35b_prefill_4096_rows_sampled():
+    d = mi.QWEN36_35B_A3B
+    rows = 4096
+    case = P.build_case(d, rows, router_bias=True, all_experts=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    # loads are uneven (the router bias): the busiest expert gets many M tiles
+    counts = np.bincount(idx.ravel(), minlength=d.n_experts)
+    assert counts.max() > 4 * counts.mean()
+    sample = np.random.default_rng(0).choice(rows, 48, replace=False)
+    sub = P.Case(d, case.layer, case.x[sample].copy(), case.logits[sample])
+    P.compare_output(sub, out[sample], idx[sample])
