@@ -87,6 +87,33 @@ def algorithmic_bytes(d, rows: int, n_active: int, residual: bool = False) -> di
             "router_topk": rt, "gate_up": gu, "down_blend": dn}
 
 
+def prefill_flops(d, rows: int) -> dict:
+    """Algorithmic FLOPs of a prefill step (2 per multiply-add): router GEMV,
+    then per token k routed experts and the shared expert (gate_up 2I x H,
+    down H x I)."""
+    H, I, Is, E, k = d.hidden, d.inter, d.shared_inter, d.n_experts, d.top_k
+    g1 = rows * (k * 2 * (2 * I) * H + 2 * (2 * Is) * H)
+    g2 = rows * (k * 2 * I * H + 2 * Is * H)
+    rt = rows * (2 * E * H + 2 * H)
+    return {"total": g1 + g2 + rt, "gemm_gate_up": g1, "gemm_down": g2, "router_topk": rt}
+
+
+def prefill_bytes(d, rows: int, n_active: int) -> int:
+    """Bytes a prefill step must move: the touched weights once, x, out."""
+    return algorithmic_bytes(d, rows, n_active)["total"]
+
+
+def prefill_executed_flops(d, counts) -> dict:
+    """Tensor-core FLOPs the two GEMMs issue: every expert's rows padded to
+    128-row tiles, and each activation as two e4m3 terms (hi and lo)."""
+    H, I, Is = d.hidden, d.inter, d.shared_inter
+    tiles = sum((int(c) + 127) // 128 for c in counts)
+    ts = (int(sum(counts)) // d.top_k + 127) // 128
+    g1 = 2 * 2 * 128 * (tiles * 2 * I * H + ts * 2 * Is * H)
+    g2 = 2 * 2 * 128 * (tiles * I * H + ts * Is * H)
+    return {"gemm_gate_up": g1, "gemm_down": g2}
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons for one GPU."""
 
@@ -363,6 +390,93 @@ class DecodeBench:
         return counts
 
 
+class PrefillBench(DecodeBench):
+    """Prefill steps of the same layer: `rows` tokens, a per-expert router
+    bias, the prefill path (permute -> tcgen05 grouped GEMMs -> blend)."""
+
+    def __init__(self, dims, inst, bias, xs, rows):
+        super().__init__(dims, [inst], xs, rows)
+        self.bias = bias
+
+    def step(self, i, events=None):
+        w = self.insts[0]
+        x = self.xs[i % len(self.xs)]
+        out = self.outs[i % len(self.outs)]
+        args = (self.d, x, w["router_w"], w["expert_w8"], w["expert_scales"], w["shared_w8"], w["shared_scales"],
+                w["shared_gate"], out, self.ws)
+        if events is None:
+            self.moe.ffn_forward_path(*args, path=self.moe.MOE_PATH_PREFILL, router_bias=self.bias,
+                                      stream=self.stream)
+        else:
+            self.moe.ffn_forward_timed(*args, events=events, path=self.moe.MOE_PATH_PREFILL,
+                                       router_bias=self.bias, stream=self.stream)
+
+    def expert_counts(self):
+        torch, moe = self.torch, self.moe
+        idx = torch.empty(self.rows, self.d.top_k, dtype=torch.int32, device="cuda")
+        w = self.insts[0]
+        moe.ffn_forward_path(self.d, self.xs[0], w["router_w"], w["expert_w8"], w["expert_scales"],
+                             w["shared_w8"], w["shared_scales"], w["shared_gate"], self.outs[0], self.ws,
+                             path=moe.MOE_PATH_PREFILL, router_bias=self.bias, topk_idx=idx)
+        return torch.bincount(idx.flatten().long(), minlength=self.d.n_experts).cpu().tolist()
+
+
+PREFILL_KERNELS = ["router_topk", "scan", "permute", "gemm_gate_up", "gemm_down", "blend"]
+
+
+def prefill_leg(args, d, inst, dist: Dist, bus, hbm_peak, bf16_peak, peak_kind):
+    """The 4096-token prefill: whole-step and per-kernel times, TFLOP/s
+    against the FP8 dense peak (the measured bf16 GEMM peak x 2, the nominal
+    fp8:bf16 ratio of the part)."""
+    import torch
+
+    import moe_inputs as mi
+    rows = 4096
+    bias = torch.from_numpy(mi.make_router(d, args.seed, True)[2]).cuda()
+    xs = [torch.from_numpy(mi.make_x(d, rows, seed=args.seed + 3, stream=i).view("int16")).view(torch.bfloat16)
+          .cuda() for i in range(2)]
+    pb = PrefillBench(d, inst, bias, xs, rows)
+    counts = pb.expert_counts()
+    n_active = sum(1 for c in counts if c)
+    fl = prefill_flops(d, rows)
+    ex = prefill_executed_flops(d, counts)
+    fp8_peak = 2.0 * bf16_peak
+    kp = max(10, min(50, args.steps // 40))
+    sampler = ClockSampler(bus)
+    sampler.start()
+    ms, _ = pb.time_steps(kp, max(3, min(args.warmup, 5)), dist, sampler)
+    clocks = sampler.stop()
+    s = dist.max(ms / 1000.0)
+    step_s = s / kp
+    tflops = aggregate(kp * fl["total"], dist.world, s) / 1e12
+    res = {"workload": f"Qwen3.6-35B-A3B-shaped MoE FFN layer, prefill rows={rows}, per-expert router bias N(0,1)",
+           "rows": rows, "steps": kp, "us_per_layer": round(step_s * 1e6, 2),
+           "tokens_per_s": round(aggregate(kp * rows, dist.world, s), 1),
+           "tflops": round(tflops, 1), "fp8_peak_tflops": round(fp8_peak, 1),
+           "frac_of_fp8_peak": round(tflops / dist.world / fp8_peak, 4),
+           "hbm_gb_s": round(aggregate(kp * prefill_bytes(d, rows, n_active), dist.world, s) / 1e9, 1),
+           "flops_per_step": int(fl["total"]), "distinct_experts": n_active,
+           "max_expert_rows": int(max(counts)), "mean_expert_rows": round(sum(counts) / len(counts), 1),
+           "peak_source": f"{peak_kind} bf16 GEMM {bf16_peak} TFLOP/s (burst) x 2 (nominal fp8:bf16 ratio)",
+           "clocks": clocks,
+           "gpu_launches": int(pb.moe.kernel_launches(d, rows, pb.moe.MOE_PATH_PREFILL) * kp)}
+    if not args.no_extras:
+        per = pb.per_kernel_us(min(kp, 24), PREFILL_KERNELS, batch=8)
+        res["per_kernel_us"] = {k: round(v, 2) for k, v in per.items()}
+        dom = max(("gemm_gate_up", "gemm_down"), key=lambda k: per[k])
+        ach = fl[dom] / (per[dom] * 1e-6) / 1e12
+        exe = ex[dom] / (per[dom] * 1e-6) / 1e12
+        res["roofline"] = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                           "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4),
+                           "traffic": profiled_traffic(dom, "qwen36_35b_prefill_rows4096"),
+                           "algorithmic_flops_per_launch": int(fl[dom]),
+                           "executed_tflops": round(exe, 1), "executed_frac": round(exe / fp8_peak, 4),
+                           "note": "achieved counts the layer's own FLOPs; executed counts the MMAs issued "
+                                   "(128-row tile padding, and two e4m3 terms per activation)"}
+    del pb
+    return res
+
+
 def e2e_measure(dims, insts, rows: int, steps: int, dist: Dist, seed: int):
     """The same metric through the public call with host buffers: every step
     copies its x from pinned host memory and its output back to pinned host
@@ -433,7 +547,7 @@ def run_ours(args, dist: Dist):
 
     torch.cuda.set_device(dist.local)
     d = mi.QWEN36_35B_A3B
-    hbm_peak, _, peak_kind = peaks()
+    hbm_peak, bf16_peak, peak_kind = peaks()
     t0 = time.time()
     layer = mi.make_layer(d, seed=args.seed)
     gen_s = time.time() - t0
@@ -514,6 +628,12 @@ def run_ours(args, dist: Dist):
                             "hbm_frac_of_measured": round(gbs64 / dist.world / hbm_peak, 4),
                             "tokens_per_s": round(aggregate(k64 * r64, dist.world, s64), 1),
                             "distinct_experts_per_step": round(u64, 1), "steps": k64}
+
+    # ---- prefill, 4096 tokens
+    result["prefill"] = prefill_leg(args, d, insts[0], dist, bus, hbm_peak, bf16_peak, peak_kind)
+    p = result["prefill"]
+    print(f"[bench] prefill: {p['us_per_layer']:.1f} us/layer, {p['tflops']:.1f} TFLOP/s "
+          f"({100 * p['frac_of_fp8_peak']:.1f}% of fp8 peak)", file=sys.stderr, flush=True)
 
     # ---- end to end through the public call with host buffers
     ke = min(args.steps, 1000)

@@ -236,6 +236,21 @@ __device__ __forceinline__ void set_status(int32_t *counters, int32_t code)
     atomicCAS(&counters[kCtrStatus], 0, code);
 }
 
+// Order-preserving 32-bit key of a float (larger key = larger value).
+__device__ __forceinline__ uint32_t ordered_key(float f)
+{
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Router top-k key of a logit: larger is better; NaN ranks below every
+// number (key 1) and 0 marks an empty slot.
+__device__ __forceinline__ uint32_t topk_key(float l) { return isnan(l) ? 1u : max(ordered_key(l), 2u); }
+
 // Default bound on any wait inside a kernel (wall time).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 

@@ -88,16 +88,6 @@ __device__ __forceinline__ float dot8_bf16(uint4 w, uint4 x)
 
 __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
-// Order-preserving 32-bit key of a float (larger key = larger value).
-__device__ __forceinline__ uint32_t ordered_key(float f)
-{
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_value(uint32_t k)
-{
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
 
 // ---------------------------------------------------------------- router
 
@@ -120,7 +110,6 @@ struct RouterParams {
     float *topk_w;
     float *gsig;
     int32_t *counters;
-    int32_t *plan;     // nullptr: no plan
 };
 
 __device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v)
@@ -165,6 +154,7 @@ __device__ void topk_row(const RouterParams &p, int t)
         }
         if (lane == r) { my_e = emin; my_k = kmax; }
     }
+    if (threadIdx.x == 0) MOE_TRACE(0, 5);
     const float my_v = (my_k == 1u) ? __int_as_float(0x7FC00000) : key_value(my_k);
     const float top = __shfl_sync(0xFFFFFFFFu, my_v, 0);
     const float ev = (lane < p.K) ? expf(my_v - top) : 0.f;
@@ -174,6 +164,7 @@ __device__ void topk_row(const RouterParams &p, int t)
         p.topk_w[(size_t)t * p.K + lane] = ev / sum;
     }
     if (lane == 0) p.gsig[t] = sigmoidf_(z);
+    if (threadIdx.x == 0) MOE_TRACE(0, 6);
 }
 
 __device__ void topk_rows(const RouterParams &p, int t_begin, int t_end)
@@ -220,59 +211,8 @@ __device__ int block_exclusive_scan(int v, int *scratch, int *total)
     return r;
 }
 
-// Work table of the expert kernels.  plan[0] = number of active routed
-// experts; descriptor u (kDescInts ints at plan + 4 + kDescInts*u) =
-// {expert, pairs routed to it, first index in the pair list, 0, the first
-// kDescPairs pair ids}; active experts in ascending id.  The pair list (at
-// plan + 4 + kDescInts*E) holds each expert's pair ids (t*K + r) together;
-// their order within an expert is immaterial (each pair is computed alone).
-__device__ void build_plan(const RouterParams &p, int *smem_i)
-{
-    const int E = p.E, P = p.rows * p.K;
-    int *cnt = smem_i;             // [E]
-    int *cursor = smem_i + E;      // [E]
-    int *slot = smem_i + 2 * E;    // [E] active index of each expert
-    int *scratch = smem_i + 3 * E; // [33]
-    int32_t *desc = p.plan + 4;
-    int32_t *pairs = p.plan + 4 + kDescInts * E;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < P; i += blockDim.x) atomicAdd(&cnt[__ldcg(p.topk_idx + i)], 1);
-    __syncthreads();
-    int run_off = 0, run_act = 0;
-    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
-        const int e = e0 + threadIdx.x;
-        const int c = (e < E) ? cnt[e] : 0;
-        int tot_off, tot_act;
-        const int off = block_exclusive_scan(c, scratch, &tot_off);
-        const int act = block_exclusive_scan(c > 0 ? 1 : 0, scratch, &tot_act);
-        if (c > 0) {
-            const int u = run_act + act;
-            int32_t *dd = desc + kDescInts * u;
-            dd[0] = e;
-            dd[1] = c;
-            dd[2] = run_off + off;
-            dd[3] = 0;
-            cursor[e] = run_off + off;
-            slot[e] = u;
-        }
-        run_off += tot_off;
-        run_act += tot_act;
-    }
-    if (threadIdx.x == 0) p.plan[0] = run_act;
-    __syncthreads();
-    for (int i = threadIdx.x; i < P; i += blockDim.x) {
-        const int e = __ldcg(p.topk_idx + i);
-        const int pos = atomicAdd(&cursor[e], 1);
-        pairs[pos] = i;
-        const int local = pos - desc[kDescInts * slot[e] + 2];
-        if (local < kDescPairs) desc[kDescInts * slot[e] + 4 + local] = i;
-    }
-}
-
 // grid = (router-row blocks, token groups).  Shared memory: [rows_per_cta
-// router rows, bf16][kRouterTok activation rows, bf16]; the last CTA reuses
-// it as plan scratch.
+// router rows, bf16][kRouterTok activation rows, bf16].
 __global__ void __launch_bounds__(kRouterMaxRows * kWarp) router_topk_kernel(RouterParams p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -353,8 +293,8 @@ __global__ void __launch_bounds__(kRouterMaxRows * kWarp) router_topk_kernel(Rou
         return;
     }
 
-    // The last CTA of this token group runs its top-k; the last group to
-    // finish builds the work table (no CTA waits for another).
+    // The last CTA of this token group to finish runs the group's top-k (no
+    // CTA waits for another).
     if (threadIdx.x == 0) MOE_TRACE(0, 2);
     if (threadIdx.x == 0) {
         const int prev = atomic_add_acq_rel_gpu(p.counters + kCtrRouterGroup + blockIdx.y, 1);
@@ -367,18 +307,7 @@ __global__ void __launch_bounds__(kRouterMaxRows * kWarp) router_topk_kernel(Rou
     topk_rows(p, t_begin, t_end);
     __syncthreads();
     if (threadIdx.x == 0) MOE_TRACE(0, 4);
-    if (threadIdx.x == 0) {
-        p.counters[kCtrRouterGroup + blockIdx.y] = 0;
-        const int prev = atomic_add_acq_rel_gpu(p.counters + kCtrRouter, 1);
-        s_last = (prev == (int)gridDim.y - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (p.plan) build_plan(p, reinterpret_cast<int *>(smem));
-    __syncthreads();
-    if (threadIdx.x == 0) MOE_TRACE(0, 5);
-    if (threadIdx.x == 0) p.counters[kCtrRouter] = 0;
+    if (threadIdx.x == 0) p.counters[kCtrRouterGroup + blockIdx.y] = 0;
 }
 
 // ------------------------------------------------------- expert kernels
@@ -392,7 +321,7 @@ struct ExpertParams {
     const float *sc;
     const uint8_t *sw8;
     const float *ssc;
-    const int32_t *plan;
+    const int32_t *topk_idx;
     const float *topk_w;
     const float *gsig;
     float *h_routed;
@@ -425,10 +354,79 @@ __device__ __forceinline__ int expert_nscales(int H, int I)
     return (2 * I / 128) * (H / 128) + (H / 128) * (I / 128);
 }
 
+// The routing table of one expert CTA, built in its shared memory from
+// topk_idx: the active experts in ascending id, where each one's pairs
+// start in the pair list, and the pair ids (t*K + r) grouped by expert.
+// Every CTA builds the same table (the order of pairs within an expert may
+// differ between CTAs; each pair is computed on its own, so it does not
+// matter).
+struct LocalPlan {
+    int *cnt;       // [E] counts, then fill cursors
+    int *e_of;      // [min(E, P)] active expert ids
+    int *first_of;  // [min(E, P) + 1] each active expert's first pair slot
+    int *pairs;     // [P]
+    int *scratch;   // [kWarp + 1] scan scratch
+};
+
+__host__ __device__ __forceinline__ size_t plan_bytes(int E, int P)
+{
+    const int U = E < P ? E : P;
+    return align16(sizeof(int) * ((size_t)E + U + (U + 1) + P + (kWarp + 1)));
+}
+
+__device__ __forceinline__ LocalPlan plan_at(unsigned char *base, int E, int P)
+{
+    const int U = min(E, P);
+    LocalPlan lp;
+    lp.cnt = reinterpret_cast<int *>(base);
+    lp.e_of = lp.cnt + E;
+    lp.first_of = lp.e_of + U;
+    lp.pairs = lp.first_of + U + 1;
+    lp.scratch = lp.pairs + P;
+    return lp;
+}
+
+// All threads of the CTA.  Returns the number of active routed experts (0
+// if an earlier kernel of this call recorded an error: its outputs are not
+// valid).
+__device__ int build_local_plan(const ExpertParams &p, const LocalPlan &lp)
+{
+    const int E = p.E, P = p.rows * p.K;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) lp.cnt[e] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < P; i += blockDim.x)
+        atomicAdd(&lp.cnt[min(max(__ldcg(p.topk_idx + i), 0), E - 1)], 1);
+    __syncthreads();
+    int run_off = 0, run_act = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        const int c = (e < E) ? lp.cnt[e] : 0;
+        int tot_off, tot_act;
+        const int off = block_exclusive_scan(c, lp.scratch, &tot_off);
+        const int act = block_exclusive_scan(c > 0 ? 1 : 0, lp.scratch, &tot_act);
+        if (c > 0) {
+            lp.e_of[run_act + act] = e;
+            lp.first_of[run_act + act] = run_off + off;
+            lp.cnt[e] = run_off + off;
+        }
+        run_off += tot_off;
+        run_act += tot_act;
+    }
+    if (threadIdx.x == 0) lp.first_of[run_act] = run_off;
+    __syncthreads();
+    for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        const int e = min(max(__ldcg(p.topk_idx + i), 0), E - 1);
+        lp.pairs[atomicAdd(&lp.cnt[e], 1)] = i;
+    }
+    const int bad = __ldcg(p.counters + kCtrStatus);
+    __syncthreads();
+    return bad ? 0 : run_act;
+}
+
 // Item i: shared-expert items first (routing-independent), then the routed
 // experts in table order.
 __device__ __forceinline__ void describe(const ExpertParams &p, int item, int per_shared, int per_routed,
-                                         int block, const int4 *dsc, StageDesc &d)
+                                         int block, const LocalPlan *lp, StageDesc &d)
 {
     if (item < per_shared) {
         d.slab = p.sw8;
@@ -442,39 +440,16 @@ __device__ __forceinline__ void describe(const ExpertParams &p, int item, int pe
     } else {
         const int r = item - per_shared;
         const int u = r / per_routed;
-        int4 h = dsc[0];
-        const int P = p.rows * p.K;
-        if (h.x < 0 || h.x >= p.E || h.y < 0 || h.z < 0 || h.z + h.y > P) h = make_int4(0, 0, 0, 0);
-        d.slab = p.w8 + (size_t)h.x * 3 * p.I * p.H;
-        d.scales = p.sc + (size_t)h.x * expert_nscales(p.H, p.I);
-        d.pairs = p.plan + 4 + kDescInts * p.E + h.z;
-        d.n = h.y;
+        const int e = lp->e_of[u], f0 = lp->first_of[u];
+        d.slab = p.w8 + (size_t)e * 3 * p.I * p.H;
+        d.scales = p.sc + (size_t)e * expert_nscales(p.H, p.I);
+        d.pairs = lp->pairs + f0;
+        d.n = lp->first_of[u + 1] - f0;
         d.inter = p.I;
         d.first = (r - u * per_routed) * block;
-        const int4 a = dsc[1], b = dsc[2];
-        const int ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int i = 0; i < kDescPairs; ++i) d.rows[i] = min(max(ids[i], 0), max(P - 1, 0));
+        for (int i = 0; i < kDescPairs; ++i) d.rows[i] = i < d.n ? d.pairs[i] : 0;
     }
-}
-
-// The descriptor of a routed item (three 16-byte words), or zeros.
-__device__ __forceinline__ void load_desc(const ExpertParams &p, int item, int per_shared, int per_routed,
-                                          int n_items, int4 *dv)
-{
-    dv[0] = dv[1] = dv[2] = make_int4(0, 0, 0, 0);
-    if (item >= per_shared && item < n_items) {
-        const int4 *dp = reinterpret_cast<const int4 *>(p.plan + 4 + kDescInts * ((item - per_shared) / per_routed));
-        dv[0] = __ldcg(dp);
-        dv[1] = __ldcg(dp + 1);
-        dv[2] = __ldcg(dp + 2);
-    }
-}
-
-__device__ __forceinline__ int active_experts(const ExpertParams &p)
-{
-    // an earlier kernel of this call gave up: the work table is not valid
-    return __ldcg(p.counters + kCtrStatus) ? 0 : min(__ldcg(p.plan), p.E);
 }
 
 // Warp roles of the expert kernels: warps 0..7 compute (consumers), warp 8
@@ -501,6 +476,8 @@ constexpr int kConsumerThreads = kConsumerWarps * kWarp;
 constexpr int kMaxStages = 4;
 constexpr int kMaxTiles = 4;  // 16-row MMA tiles per item
 constexpr int kRowPad = 16;   // bytes of padding after each staged row
+// Cross-warp reduction area of an item with T 16-row MMA tiles.
+__host__ __device__ constexpr size_t red_bytes(int T) { return (size_t)kConsumerWarps * T * kWarp * 16; }
 
 // ------------------------------------------------------------- gate_up
 
@@ -576,6 +553,7 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
     const int per_shared = p.Is / p.pairs, per_routed = p.I / p.pairs;
     const int S = p.stages;
     float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [warp][tile][lane]
+    const LocalPlan lp = plan_at(smem + (size_t)S * L.bytes + red_bytes(L.T), p.E, p.rows * p.K);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -588,9 +566,8 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
     __syncthreads();
     if (threadIdx.x == 0) MOE_TRACE(1, 0);
 
+    const uint64_t pol = policy_evict_first();
     if (warp == kConsumerWarps) {
-        // ------------------------------------------------------- producer
-        const uint64_t pol = policy_evict_first();
         // Shared-expert weights and scales do not depend on routing: fetch
         // them before waiting on the router.
         for (int q = 0; q < S; ++q) {
@@ -601,18 +578,18 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
             gu_produce(p, L, desc[q], smem + q * L.bytes, &full[q], pol, true, false);
         }
         __syncwarp();
-        pdl_wait();
-        pdl_trigger();
-        if (lane == 0) MOE_TRACE(1, 1);
-        const int n_items = per_shared + active_experts(p) * per_routed;
-        int4 dv[3];
-        load_desc(p, blockIdx.x, per_shared, per_routed, n_items, dv);
+    }
+    pdl_wait();
+    pdl_trigger();
+    const int n_items = per_shared + build_local_plan(p, lp) * per_routed;
+    if (threadIdx.x == 0) MOE_TRACE(1, 1);
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------- producer
         for (int q = 0;; ++q) {
             const int item = blockIdx.x + q * gridDim.x;
             if (item >= n_items) break;
             const int s = q % S;
-            int4 cur[3] = {dv[0], dv[1], dv[2]};
-            load_desc(p, item + gridDim.x, per_shared, per_routed, n_items, dv);  // the next item's, early
             if (q >= S && !mbar_wait(&empty[s], ((q / S) - 1) & 1, kWaitLimitNs)) {
                 if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
                 s_abort = 1;
@@ -622,7 +599,7 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
             const bool prefetched = q < S && item < per_shared;
             if (lane == 0) {
                 if (q >= S) fence_proxy_async_smem();  // consumers' generic accesses precede the copies
-                if (!prefetched) describe(p, item, per_shared, per_routed, p.pairs, cur, desc[s]);
+                if (!prefetched) describe(p, item, per_shared, per_routed, p.pairs, &lp, desc[s]);
             }
             __syncwarp();
             gu_produce(p, L, desc[s], st, &full[s], pol, !prefetched, true);
@@ -633,9 +610,6 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
     }
 
     // ----------------------------------------------------------- consumers
-    pdl_wait();
-    pdl_trigger();
-    const int n_items = per_shared + active_experts(p) * per_routed;
     const int g = lane >> 2, t = lane & 3;
     for (int q = 0;; ++q) {
         const int item = blockIdx.x + q * gridDim.x;
@@ -660,13 +634,13 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
                 const int hv = p.H / 16;
                 for (int i = threadIdx.x; i < 2 * nt * hv; i += kConsumerThreads) {
                     const int tr = i / (2 * hv), rem = i - tr * 2 * hv, lo = rem / hv, c = rem - lo * hv;
-                    const int row = d.pairs ? __ldcg(d.pairs + tok0 + tr) / p.K : tok0 + tr;
+                    const int row = d.pairs ? d.pairs[tok0 + tr] / p.K : tok0 + tr;
                     reinterpret_cast<uint4 *>(st + (lo ? L.xl : L.xh) + (size_t)tr * L.WS)[c] =
                         __ldcg(reinterpret_cast<const uint4 *>(p.xq + (size_t)row * 2 * p.H + (size_t)lo * p.H) + c);
                 }
                 for (int i = threadIdx.x; i < nt * L.hb; i += kConsumerThreads) {
                     const int tr = i / L.hb;
-                    const int row = d.pairs ? __ldcg(d.pairs + tok0 + tr) / p.K : tok0 + tr;
+                    const int row = d.pairs ? d.pairs[tok0 + tr] / p.K : tok0 + tr;
                     const_cast<float *>(xsc)[i] = __ldcg(p.xsc + (size_t)row * L.hb + (i - tr * L.hb));
                 }
                 named_barrier(1, kConsumerThreads);
@@ -708,11 +682,13 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
                     acc[tau][3] = fmaf(su * x1, tmp[tau][3], acc[tau][3]);
                 }
             }
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(1, 7);
 #pragma unroll
             for (int tau = 0; tau < kMaxTiles; ++tau)
                 if (tau < L.T)
-                    red[(warp * kMaxTiles + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
+                    red[(warp * L.T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
             named_barrier(1, kConsumerThreads);
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(1, 8);
             // (tile, pair row g, column n) -> h
             for (int i = threadIdx.x; i < 64 * L.T; i += kConsumerThreads) {
                 const int tau = i >> 6, gg = (i >> 3) & 7, n = i & 7;
@@ -721,20 +697,22 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
                 float gate = 0.f, up = 0.f;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float4 v = red[(w * kMaxTiles + tau) * kWarp + src];
+                    const float4 v = red[(w * L.T + tau) * kWarp + src];
                     gate += comp ? v.y : v.x;
                     up += comp ? v.w : v.z;
                 }
                 const float h = siluf_(gate) * up;
                 const int j = d.first + 8 * tau + gg;
                 if (d.pairs) {
-                    const int pr = tok0 == 0 ? d.rows[n] : __ldcg(d.pairs + tok0 + n);
+                    const int pr = tok0 == 0 ? d.rows[n] : d.pairs[tok0 + n];
                     p.h_routed[(size_t)pr * Iu + j] = h;
                 } else {
                     p.h_shared[(size_t)(tok0 + n) * Iu + j] = h;
                 }
             }
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(1, 9);
             named_barrier(1, kConsumerThreads);  // red is free again
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(1, 10);
         }
         if (q < 2 && threadIdx.x == 0) MOE_TRACE(1, 3 + 2 * q);
         __syncwarp();  // this warp is done with the stage and its descriptor
@@ -808,6 +786,7 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
     const int per_block = p.H / p.drows;  // items per expert
     const int S = p.stages;
     float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [warp][tile][lane]
+    const LocalPlan lp = plan_at(smem + (size_t)S * L.bytes + red_bytes(L.T), p.E, p.rows * p.K);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -819,23 +798,20 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
     }
     __syncthreads();
     if (threadIdx.x == 0) MOE_TRACE(2, 0);
+    // The router has finished when this kernel starts (its predecessor
+    // waited for the router before letting this kernel launch), so the
+    // routing is final: build the table and fetch the first stages' down
+    // weights and scales now; only h waits for gate_up.
+    const int n_active = build_local_plan(p, lp);
+    const int n_items = per_block + n_active * per_block;
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------- producer
-        // The router has finished when this kernel starts (its predecessor
-        // waited for the router before letting this kernel launch), so the
-        // work table is final: fetch the first stages' down weights and
-        // scales now; only h waits for gate_up.
         const uint64_t pol = policy_evict_first();
-        const int n_items = per_block + active_experts(p) * per_block;
-        int4 dv[3];
-        load_desc(p, blockIdx.x, per_block, per_block, n_items, dv);
         for (int q = 0; q < S; ++q) {
             const int item = blockIdx.x + q * gridDim.x;
             if (item >= n_items) break;
-            int4 cur[3] = {dv[0], dv[1], dv[2]};
-            load_desc(p, item + gridDim.x, per_block, per_block, n_items, dv);
-            if (lane == 0) describe(p, item, per_block, per_block, p.drows, cur, desc[q]);
+            if (lane == 0) describe(p, item, per_block, per_block, p.drows, &lp, desc[q]);
             __syncwarp();
             dn_produce(p, L, desc[q], smem + q * L.bytes, &full[q], pol, true, false);
         }
@@ -854,8 +830,6 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
                 if (lane == 0) mbar_arrive(&full[s]);
                 continue;
             }
-            int4 cur[3] = {dv[0], dv[1], dv[2]};
-            load_desc(p, item + gridDim.x, per_block, per_block, n_items, dv);
             if (!mbar_wait(&empty[s], ((q / S) - 1) & 1, kWaitLimitNs)) {
                 if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
                 s_abort = 1;
@@ -863,7 +837,7 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
             }
             if (lane == 0) {
                 fence_proxy_async_smem();  // consumers' generic accesses precede the copies
-                describe(p, item, per_block, per_block, p.drows, cur, desc[s]);
+                describe(p, item, per_block, per_block, p.drows, &lp, desc[s]);
             }
             __syncwarp();
             dn_produce(p, L, desc[s], st, &full[s], pol, true, true);
@@ -876,8 +850,6 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
     // ----------------------------------------------------------- consumers
     pdl_wait();
     pdl_trigger();
-    const int n_active = active_experts(p);
-    const int n_items = per_block + n_active * per_block;
     const int g = lane >> 2, t = lane & 3;
     for (int q = 0;; ++q) {
         const int item = blockIdx.x + q * gridDim.x;
@@ -904,7 +876,7 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
                 const int iv = Iu / 4, rv = L.imax / 4;
                 for (int i = threadIdx.x; i < ns * iv; i += kConsumerThreads) {
                     const int tr = i / iv;
-                    const float *src = d.pairs ? p.h_routed + (size_t)__ldcg(d.pairs + s0 + tr) * Iu
+                    const float *src = d.pairs ? p.h_routed + (size_t)d.pairs[s0 + tr] * Iu
                                                : p.h_shared + (size_t)(s0 + tr) * Iu;
                     hv[tr * rv + (i - tr * iv)] = __ldcg(reinterpret_cast<const float4 *>(src) + (i - tr * iv));
                 }
@@ -960,7 +932,7 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
 #pragma unroll
             for (int tau = 0; tau < kMaxTiles; ++tau)
                 if (tau < L.T)
-                    red[(warp * kMaxTiles + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
+                    red[(warp * L.T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
             named_barrier(1, kConsumerThreads);
             // (output row, slot column) -> weighted partial
             for (int i = threadIdx.x; i < 128 * L.T; i += kConsumerThreads) {
@@ -970,14 +942,14 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
                 float y = 0.f;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float4 v = red[(w * kMaxTiles + tau) * kWarp + src];
+                    const float4 v = red[(w * L.T + tau) * kWarp + src];
                     y += comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w;
                 }
                 const int row = d.first + 16 * tau + r;
                 int yrow;
                 float wt;
                 if (d.pairs) {
-                    yrow = s0 == 0 ? d.rows[n] : __ldcg(d.pairs + s0 + n);
+                    yrow = s0 == 0 ? d.rows[n] : d.pairs[s0 + n];
                     wt = s0 == 0 ? d.wt[n] : __ldcg(p.topk_w + yrow);
                 } else {
                     yrow = p.rows * p.K + s0 + n;
@@ -1089,7 +1061,7 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
     const int imax = std::max(I, Is);
     rows = std::max<int64_t>(rows, 1);
     // router: rows_per_cta router rows (<= 32 KB) and kRouterTok activation rows per CTA
-    s.router_rows = std::max(4, std::min(kRouterMaxRows, 32768 / H));
+    s.router_rows = std::max(1, std::min(4, 32768 / H));
     s.router_groups = (int)std::min<int64_t>((rows + kRouterTok - 1) / kRouterTok, kMaxRouterGroups);
     s.router_group_tokens = (int)((rows + s.router_groups - 1) / s.router_groups);
     s.router_smem = std::max<size_t>((size_t)(s.router_rows + kRouterTok) * H * 2, (size_t)(3 * E + 33) * 4);
@@ -1110,24 +1082,26 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
     const size_t ws_d = (size_t)imax + kRowPad;
     const size_t dn_stage = align16(drows * ws_d + (size_t)s.tok * imax * 4 + 2 * s.tok * ws_d +
                                     (size_t)s.tok * (imax / 128) * 4 + (size_t)(imax / 128) * 4);
-    const size_t red = (size_t)kConsumerWarps * kMaxTiles * kWarp * 16;
+    const size_t plan = plan_bytes(E, (int)(rows * d.top_k));
+    const size_t gu_extra = red_bytes(pairs / 8) + plan, dn_extra = red_bytes(drows / 16) + plan;
     // One gate_up and one down CTA share an SM when they fit (down fetches
-    // its weights while gate_up streams); else each has the SM alone.
+    // its weights while gate_up streams); gate_up, with two thirds of the
+    // bytes, gets the deeper ring.  Else each has the SM alone.
     const size_t budget = 224 * 1024 - 2048;
-    int gs = 3, ds = 3;
-    while (gs * gu_stage + red + ds * dn_stage + red > budget && (gs > 2 || ds > 2)) {
-        if (gs * gu_stage >= ds * dn_stage && gs > 2) --gs;
-        else if (ds > 2) --ds;
-        else --gs;
-    }
-    if (gs * gu_stage + red + ds * dn_stage + red > budget) {
-        gs = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - red) / gu_stage));
-        ds = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - red) / dn_stage));
+    int gs = kMaxStages, ds = 3;
+    auto total = [&] { return gs * gu_stage + gu_extra + ds * dn_stage + dn_extra; };
+    while (total() > budget && ds > 2) --ds;
+    while (total() > budget && gs > 2) --gs;
+    while (total() > budget && ds > 1) --ds;
+    while (total() > budget && gs > 1) --gs;
+    if (total() > budget) {
+        gs = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - gu_extra) / gu_stage));
+        ds = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - dn_extra) / dn_stage));
     }
     s.gu_stages = gs;
     s.dn_stages = ds;
-    s.gu_smem = gs * gu_stage + red;
-    s.dn_smem = ds * dn_stage + red;
+    s.gu_smem = gs * gu_stage + gu_extra;
+    s.dn_smem = ds * dn_stage + dn_extra;
     return s;
 }
 
@@ -1160,7 +1134,6 @@ cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s)
     p.topk_w = a.topk_w;
     p.gsig = a.gsig;
     p.counters = a.counters;
-    p.plan = a.plan;
     const dim3 grid((d.n_experts + 1 + sh.router_rows - 1) / sh.router_rows,
                     (a.rows + sh.router_group_tokens - 1) / sh.router_group_tokens);
     if (occupancy(router_topk_kernel, sh.router_rows * kWarp, sh.router_smem) < 1)
@@ -1187,7 +1160,7 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
     p.sc = a.expert_scales;
     p.sw8 = a.shared_w8;
     p.ssc = a.shared_scales;
-    p.plan = a.plan;
+    p.topk_idx = a.topk_idx;
     p.topk_w = a.topk_w;
     p.gsig = a.gsig;
     p.h_routed = a.h_routed;

@@ -18,14 +18,13 @@ constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per toke
 constexpr int kMaxRouterGroups = 1024;
 constexpr int kCtrBlend = 2048;         // first of the down/blend per-row-block counters
 constexpr int kMaxBlendBlocks = kCounters - kCtrBlend;
-constexpr int kDescInts = 12;           // per active expert: {e, n, first pair, 0}, pair ids [8]
-constexpr int kDescPairs = 8;
+constexpr int kDescPairs = 8;           // pair ids a stage descriptor carries
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Decode-path workspace, carved from the caller's buffer.
 struct DecodeLayout {
-    size_t counters, logits, xq, xsc, topk_idx, topk_w, gsig, plan, h_routed, h_shared, yslot, total;
+    size_t counters, logits, xq, xsc, topk_idx, topk_w, gsig, h_routed, h_shared, yslot, total;
 };
 
 // Tile shapes of the decode kernels for given dims and rows.
@@ -52,8 +51,6 @@ inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
     L.topk_idx = take(sizeof(int32_t) * rows * K);
     L.topk_w = take(sizeof(float) * rows * K);
     L.gsig = take(sizeof(float) * rows);
-    // plan: header[4] | descriptor[E][kDescInts] | pair ids[rows*K]
-    L.plan = take(sizeof(int32_t) * (4 + kDescInts * E + rows * K));
     L.h_routed = take(sizeof(float) * rows * K * I);
     L.h_shared = take(sizeof(float) * rows * Is);
     L.yslot = take(sizeof(float) * rows * (K + 1) * H);
@@ -84,7 +81,6 @@ struct RouterLaunch {
     uint8_t *xq;     // workspace: x as hi/lo e4m3 (nullptr: not needed)
     float *xsc;
     int32_t *counters;
-    int32_t *plan;   // nullptr: no plan
 };
 cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s);
 
@@ -103,7 +99,6 @@ struct ExpertsLaunch {
     const int32_t *topk_idx;
     const float *topk_w;
     const float *gsig;
-    const int32_t *plan;
     float *h_routed;
     float *h_shared;
     float *yslot;

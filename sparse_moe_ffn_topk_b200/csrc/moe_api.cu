@@ -151,7 +151,6 @@ int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
     a.xq = nullptr;
     a.xsc = nullptr;
     a.counters = reinterpret_cast<int32_t *>(base + L.counters);
-    a.plan = nullptr;
     return finish(launch_router_topk(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -198,7 +197,6 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
     float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
     float *gs = shared_gate_sig_out ? shared_gate_sig_out : reinterpret_cast<float *>(base + L.gsig);
-    int32_t *plan = reinterpret_cast<int32_t *>(base + L.plan);
 
     RouterLaunch ra;
     ra.d = d;
@@ -214,7 +212,6 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     ra.xq = reinterpret_cast<uint8_t *>(base + L.xq);
     ra.xsc = reinterpret_cast<float *>(base + L.xsc);
     ra.counters = counters;
-    ra.plan = plan;
     cudaError_t e = launch_router_topk(ra, s);
     if (e != cudaSuccess) return finish(e);
 
@@ -233,7 +230,6 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     ea.topk_idx = tidx;
     ea.topk_w = tw;
     ea.gsig = gs;
-    ea.plan = plan;
     ea.h_routed = reinterpret_cast<float *>(base + L.h_routed);
     ea.h_shared = reinterpret_cast<float *>(base + L.h_shared);
     ea.yslot = reinterpret_cast<float *>(base + L.yslot);

@@ -2,23 +2,24 @@
 // expert-grouped FP8 GEMMs on the tcgen05 tensor cores -> unpermute + blend.
 //
 // Launch chain (programmatic dependent launch between every pair):
-//   1. router_topk_kernel (decode.cu): router GEMV, top-k per row, and the
-//      activations x as hi/lo e4m3 rows with one scale per (row, 128 block).
-//   2. count_kernel: rows routed to each expert; each (row, rank) pair's
-//      position within its expert.
-//   3. scan_kernel (one CTA): expert offsets and the table of 128-row M tiles
+//   1. router_tc_kernel: logits = x Wr^T (+ bias) and the shared-gate logit
+//      x g on tcgen05 (bf16, M=128 rows, N = experts), the top-k of each row
+//      straight from tensor memory, softmax over the k, and each (row, rank)
+//      pair's position within its expert (an atomic count per expert).
+//   2. scan_kernel (one CTA): expert offsets and the table of 128-row M tiles
 //      (routed experts in order, then the shared expert over all rows).
-//   4. permute_kernel: gathers each pair's hi/lo x row and scales into its
-//      expert's contiguous rows; records its position and blend weight.
-//   5. gemm_kernel<GEMM1>: per M tile and 128-column block j of h,
+//   3. permute_kernel: each pair's x row, quantised to hi/lo e4m3 with one
+//      scale per 128 block, into its expert's contiguous rows; then every
+//      row again in token order for the shared expert.
+//   4. gemm_kernel<GEMM1>: per M tile and 128-column block j of h,
 //      [gate_j | up_j] = A (hi+lo) x W13^T on tcgen05 (M=128, N=256, K=32 per
 //      instruction), each 128-wide K block promoted into fp32 registers with
 //      its row scale x block scale; epilogue h = silu(gate) * up, quantised
 //      to hi/lo e4m3 with one scale per (row, 128 block) for GEMM2.
-//   6. gemm_kernel<GEMM2>: y = h (hi+lo) x W2^T the same way; epilogue
+//   5. gemm_kernel<GEMM2>: y = h (hi+lo) x W2^T the same way; epilogue
 //      scales by the row's routing weight (or the shared gate) into one
 //      partial row per (row, slot).
-//   7. blend_kernel: out[t] = sum of its k partials in rank order + the
+//   6. blend_kernel: out[t] = sum of its k partials in rank order + the
 //      shared partial (+ residual), rounded once to bf16.
 //
 // Rows space of the GEMMs: the T*k routed pairs sorted by expert, then the T
@@ -46,8 +47,8 @@ constexpr size_t kGemmSmem = kGemmStages * kStageBytes + 1024 /* alignment slack
 // ------------------------------------------------------------ layout
 
 struct PrefillLayout {
-    size_t counters, logits, xq, xsc, topk_idx, topk_w, gsig, counts, offsets, rank, pos, mtiles, xp, xps, slot_w,
-        hq, hs, yslot, total;
+    size_t counters, topk_idx, topk_w, gsig, counts, offsets, rank, pos, mtiles, xp, xps, slot_w, hq, hs, yslot,
+        total;
     int64_t routed, rows_total, max_mtiles;
 };
 
@@ -62,10 +63,6 @@ inline PrefillLayout prefill_layout(const moe_dims &d, int64_t T)
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 1024); return at; };
     L.counters = take(sizeof(int32_t) * kCounters);
-    L.logits = take(sizeof(float) * T * ((E + 1 + 3) / 4 * 4));
-    const int64_t Tp = std::max<int64_t>(T, kBM);  // TMA boxes are 128 rows: tensors have at least that many
-    L.xq = take((size_t)Tp * 2 * H);
-    L.xsc = take(sizeof(float) * T * (H / 128));
     L.topk_idx = take(sizeof(int32_t) * T * K);
     L.topk_w = take(sizeof(float) * T * K);
     L.gsig = take(sizeof(float) * T);
@@ -74,8 +71,10 @@ inline PrefillLayout prefill_layout(const moe_dims &d, int64_t T)
     L.rank = take(sizeof(int32_t) * T * K);
     L.pos = take(sizeof(int32_t) * T * K);
     L.mtiles = take(sizeof(int4) * (1 + L.max_mtiles));
-    L.xp = take((size_t)std::max<int64_t>(L.routed, kBM) * 2 * H);
-    L.xps = take(sizeof(float) * std::max<int64_t>(L.routed, 1) * (H / 128));
+    // routed rows, then the T shared rows; TMA boxes are 128 rows, so each of
+    // the two tensors spans at least that many rows of the buffer
+    L.xp = take((size_t)(std::max<int64_t>(L.routed, kBM) + std::max<int64_t>(T, kBM)) * 2 * H);
+    L.xps = take(sizeof(float) * (L.routed + T) * (H / 128));
     L.slot_w = take(sizeof(float) * L.rows_total);
     L.hq = take((size_t)std::max<int64_t>(L.rows_total, kBM) * 2 * imax);
     L.hs = take(sizeof(float) * L.rows_total * (imax / 128));
@@ -91,7 +90,7 @@ size_t workspace_bytes(const moe_dims &d, int64_t rows)
 
 bool prefill_available() { return true; }
 
-int prefill_kernel_launches(const moe_dims &, int64_t) { return 7; }
+int prefill_kernel_launches(const moe_dims &, int64_t) { return 6; }
 
 // ------------------------------------------------------------ count / scan / permute
 
@@ -105,25 +104,13 @@ struct PlanParams {
     int32_t *rank;     // [T*K]
     int32_t *pos;      // [T*K]
     int4 *mtiles;      // [0].x = count; entries from [1]: {group, row0, rows, a_row0}
-    const uint8_t *xq;
-    const float *xsc;
+    const uint16_t *x; // [T][H] bf16
+    int xp_shared0;    // first xp row of the shared expert's rows (the routed rows span at least 128)
     uint8_t *xp;
     float *xps;
     float *slot_w;
     int32_t *counters;
 };
-
-__global__ void __launch_bounds__(256) count_kernel(PlanParams p)
-{
-    pdl_wait();
-    pdl_trigger();
-    const int P = p.T * p.K;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P; i += gridDim.x * blockDim.x) {
-        int e = p.topk_idx[i];
-        e = min(max(e, 0), p.E - 1);
-        p.rank[i] = atomicAdd(&p.counts[e], 1);
-    }
-}
 
 __device__ int block_scan_excl(int v, int *scratch, int *total)
 {
@@ -184,8 +171,10 @@ __global__ void __launch_bounds__(1024) scan_kernel(PlanParams p)
     if (threadIdx.x == 0) p.mtiles[0] = make_int4(run_tiles + smt, run_tiles, 0, 0);
 }
 
-// A warp per routed pair (plus the shared rows' blend weights): the pair's
-// hi/lo x row and scales into its expert's rows.
+// A warp per GEMM row: routed pair i < T*k takes its token's x row into its
+// expert's rows; row T*k + t takes token t's row for the shared expert.  Rows
+// are stored as hi/lo e4m3 (hi codes [H], then lo codes [H]) with one scale
+// per 128 block, amax / 448: x ~ s * (hi + lo).
 __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
 {
     pdl_wait();
@@ -196,21 +185,258 @@ __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
     for (int i = gw; i < P + p.T; i += nw) {
-        if (i >= P) {
-            if (lane == 0) p.slot_w[i] = p.gsig[i - P];
-            continue;
+        int t, dst, xrow;
+        if (i < P) {
+            t = i / p.K;
+            const int e = min(max(p.topk_idx[i], 0), p.E - 1);
+            dst = p.offsets[e] + p.rank[i];
+            xrow = dst;
+            if (lane == 0) {
+                p.pos[i] = dst;
+                p.slot_w[dst] = p.topk_w[i];
+            }
+        } else {
+            t = i - P;
+            dst = i;
+            xrow = p.xp_shared0 + t;
+            if (lane == 0) p.slot_w[i] = p.gsig[t];
         }
-        const int t = i / p.K;
-        const int e = min(max(p.topk_idx[i], 0), p.E - 1);
-        const int dst = p.offsets[e] + p.rank[i];
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.xq + (size_t)t * 2 * p.H);
-        uint4 *dv = reinterpret_cast<uint4 *>(p.xp + (size_t)dst * 2 * p.H);
-        for (int c = lane; c < p.H / 8; c += 32) dv[c] = src[c];
-        for (int c = lane; c < hb; c += 32) p.xps[(size_t)dst * hb + c] = p.xsc[(size_t)t * hb + c];
+        const uint2 *src = reinterpret_cast<const uint2 *>(p.x + (size_t)t * p.H);
+        uint32_t *dq = reinterpret_cast<uint32_t *>(p.xp + (size_t)xrow * 2 * p.H);
+        for (int kb = 0; kb < hb; ++kb) {
+            const uint2 raw = __ldg(src + kb * 32 + lane);
+            const float4 v = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+            const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            const float sc = amax > 0.f ? amax / 448.f : 1.f;
+            uint32_t hi, lo;
+            quant4_hilo(v, 1.f / sc, hi, lo);
+            dq[kb * 32 + lane] = hi;
+            dq[p.H / 4 + kb * 32 + lane] = lo;
+            if (lane == 0) p.xps[(size_t)dst * hb + kb] = sc;
+        }
+    }
+}
+
+// ------------------------------------------------------------ router on tcgen05
+
+constexpr int kRtBK = 128;                         // K bytes per stage: 64 bf16
+constexpr int kRtStages = 4;
+constexpr int kRtThreads = 192;                    // warp 0: TMA, warp 1: MMA + TMEM, warps 2..5: top-k
+constexpr int kRtChunk = 256;                      // experts per accumulator pass
+constexpr size_t kRtStageBytes = (size_t)kBM * kRtBK + (size_t)kRtChunk * kRtBK + 16 * kRtBK;  // x, Wr, g
+constexpr size_t kRtSmem = kRtStages * kRtStageBytes + 1024;
+
+struct RouterTcParams {
+    CUtensorMap x;    // [T][2H bytes], boxes of 128 rows
+    CUtensorMap wr;   // [E][2H bytes], boxes of nbox rows
+    CUtensorMap g;    // [1][2H bytes], boxes of 16 rows (rows past the first read as zero)
+    int T, E, K, H;
+    int nbox;         // rows of a router box / N of the expert MMA: min(256, E rounded up to 16)
+    const float *bias;
+    int32_t *topk_idx;
+    float *topk_w;
+    float *gsig;
+    int32_t *counts;  // [E], zero on entry
+    int32_t *rank;    // [T*K]
+    int32_t *counters;
+};
+
+template <int KM>
+__device__ __forceinline__ void topk_insert(uint32_t (&keys)[KM], int (&ids)[KM], uint32_t k, int e)
+{
+    if (k <= keys[KM - 1]) return;  // equal keys keep the lower expert first
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        if (k > keys[j]) {
+            const uint32_t tk = keys[j];
+            const int ti = ids[j];
+            keys[j] = k;
+            ids[j] = e;
+            k = tk;
+            e = ti;
+        }
+    }
+}
+
+// One CTA per 128-row tile of x (persistent over tiles).  The accumulator
+// holds one pass of up to 256 experts (TMEM columns [0, 256)) and the shared
+// gate logit (column 256); an epilogue thread owns one row and keeps its
+// running top-k in registers across passes.
+template <int KM>
+__global__ void __launch_bounds__(kRtThreads, 1) router_tc_kernel(const __grid_constant__ RouterTcParams p)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kRtStages], empty[kRtStages], acc_full, acc_empty;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kRtStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, 4);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_s, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&p.x);
+        tma_prefetch_desc(&p.wr);
+        tma_prefetch_desc(&p.g);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    pdl_wait();
+    pdl_trigger();
+    const int n_tiles = (p.T + kBM - 1) / kBM;
+    const int npass = (p.E + kRtChunk - 1) / kRtChunk;
+    const int nkb = 2 * p.H / kRtBK;
+    const uint32_t stage_tx = (uint32_t)(kBM * kRtBK + p.nbox * kRtBK + 16 * kRtBK);
+
+    if (warp == 0) {
         if (lane == 0) {
-            p.pos[i] = dst;
-            p.slot_w[dst] = p.topk_w[i];
+            const uint64_t pol = policy_evict_last();  // x and Wr are re-read by other tiles / passes
+            int it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !s_abort; tile += gridDim.x) {
+                for (int ps = 0; ps < npass && !s_abort; ++ps) {
+                    for (int kb = 0; kb < nkb; ++kb, ++it) {
+                        const int s = it % kRtStages;
+                        if (it >= kRtStages && !mbar_wait(&empty[s], ((it / kRtStages) - 1) & 1, kWaitLimitNs)) {
+                            set_status(p.counters, MOE_ETIMEOUT);
+                            s_abort = 1;
+                            break;
+                        }
+                        unsigned char *st = smem + s * kRtStageBytes;
+                        mbar_arrive_expect_tx(&full[s], stage_tx);
+                        tma_load_2d(st, &p.x, kb * kRtBK, tile * kBM, &full[s], pol);
+                        tma_load_2d(st + kBM * kRtBK, &p.wr, kb * kRtBK, ps * kRtChunk, &full[s], pol);
+                        tma_load_2d(st + (kBM + kRtChunk) * kRtBK, &p.g, kb * kRtBK, 0, &full[s], pol);
+                    }
+                }
+            }
         }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_e = idesc_bf16_f32(kBM, p.nbox);
+            const uint32_t id_g = idesc_bf16_f32(kBM, 16);
+            int it = 0, acc_it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !s_abort; tile += gridDim.x) {
+                for (int ps = 0; ps < npass && !s_abort; ++ps, ++acc_it) {
+                    if (acc_it >= 1 && !mbar_wait(&acc_empty, (acc_it - 1) & 1, kWaitLimitNs)) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int kb = 0; kb < nkb; ++kb, ++it) {
+                        const int s = it % kRtStages;
+                        if (!mbar_wait(&full[s], (it / kRtStages) & 1, kWaitLimitNs)) {
+                            set_status(p.counters, MOE_ETIMEOUT);
+                            s_abort = 1;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t st = smem_u32(smem + s * kRtStageBytes);
+                        const uint32_t bw = st + kBM * kRtBK, bg = st + (kBM + kRtChunk) * kRtBK;
+#pragma unroll
+                        for (int k4 = 0; k4 < kRtBK / 32; ++k4) {
+                            const uint64_t ad = umma_desc_sw128(st + k4 * 32);
+                            const uint32_t acc = (kb | k4) ? 1u : 0u;
+                            umma_bf16(tmem_base, ad, umma_desc_sw128(bw + k4 * 32), id_e, acc);
+                            if (ps == 0) umma_bf16(tmem_base + kRtChunk, ad, umma_desc_sw128(bg + k4 * 32), id_g, acc);
+                        }
+                        umma_commit(&empty[s]);
+                    }
+                    if (s_abort) break;
+                    umma_commit(&acc_full);
+                }
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int acc_it = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int t = tile * kBM + r;
+            uint32_t keys[KM];
+            int ids[KM];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                keys[j] = 0u;
+                ids[j] = 0;
+            }
+            float z = 0.f;
+            bool ok = true;
+            for (int ps = 0; ps < npass; ++ps, ++acc_it) {
+                if (!mbar_wait(&acc_full, acc_it & 1, kWaitLimitNs)) {
+                    set_status(p.counters, MOE_ETIMEOUT);
+                    s_abort = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
+                const int ncol = min(kRtChunk, p.E - ps * kRtChunk);
+                for (int c0 = 0; c0 < ncol; c0 += 32) {
+                    float v[32];
+                    tmem_ld_32x32(tb + (uint32_t)c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = ps * kRtChunk + c0 + i;
+                        if (c0 + i < ncol) {
+                            const float l = v[i] + (p.bias ? __ldg(p.bias + e) : 0.f);
+                            topk_insert<KM>(keys, ids, topk_key(l), e);
+                        }
+                    }
+                }
+                if (ps == 0) {
+                    float v[32];
+                    tmem_ld_32x32(tb + (uint32_t)kRtChunk, v);
+                    tmem_wait_ld();
+                    z = v[0];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty);
+            }
+            if (!ok) break;
+            if (t < p.T) {
+                const float top = (keys[0] == 1u) ? __int_as_float(0x7FC00000) : key_value(keys[0]);
+                float ev[KM], sum = 0.f;
+#pragma unroll
+                for (int j = 0; j < KM; ++j) {
+                    const float vj = (keys[j] == 1u) ? __int_as_float(0x7FC00000) : key_value(keys[j]);
+                    ev[j] = (j < p.K) ? expf(vj - top) : 0.f;
+                    sum += ev[j];
+                }
+#pragma unroll
+                for (int j = 0; j < KM; ++j) {
+                    if (j < p.K) {
+                        p.topk_idx[(size_t)t * p.K + j] = ids[j];
+                        p.topk_w[(size_t)t * p.K + j] = ev[j] / sum;
+                        p.rank[(size_t)t * p.K + j] = atomicAdd(&p.counts[ids[j]], 1);
+                    }
+                }
+                p.gsig[t] = sigmoidf_(z);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
     }
 }
 
@@ -584,7 +810,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, u
 }
 
 template <typename P>
-int gemm_occupancy_once(void (*kernel)(P))
+int gemm_occupancy_once(void (*kernel)(P), size_t smem = kGemmSmem)
 {
     static std::mutex mu;
     static std::vector<std::pair<const void *, int>> done;
@@ -593,10 +819,17 @@ int gemm_occupancy_once(void (*kernel)(P))
     std::lock_guard<std::mutex> lk(mu);
     for (auto &d : done)
         if (d.first == (const void *)kernel && d.second == dev) return 1;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return 0;
     done.push_back({(const void *)kernel, dev});
     return 1;
+}
+
+template <int KM>
+cudaError_t launch_router_tc(unsigned grid, const RouterTcParams &rp, cudaStream_t s)
+{
+    if (!gemm_occupancy_once(router_tc_kernel<KM>, kRtSmem)) return cudaErrorInvalidValue;
+    return launch_kernel(router_tc_kernel<KM>, dim3(grid), dim3(kRtThreads), kRtSmem, s, rp);
 }
 
 }  // namespace
@@ -616,29 +849,11 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
     float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
     float *gs = gsig_out ? gsig_out : reinterpret_cast<float *>(base + L.gsig);
-    uint8_t *xq = reinterpret_cast<uint8_t *>(base + L.xq);
-    float *xsc = reinterpret_cast<float *>(base + L.xsc);
+    const DeviceInfo &di = device_info();
+    const int P = T * K;
 
     cudaError_t e = cudaMemsetAsync(base + L.counts, 0, sizeof(int32_t) * (E + 1), s);
     if (e != cudaSuccess) return MOE_ECUDA;
-
-    // 1. router + top-k + x in hi/lo e4m3
-    RouterLaunch ra;
-    ra.d = &d;
-    ra.x = x;
-    ra.rows = rows;
-    ra.router_w = router_w;
-    ra.router_bias = router_bias;
-    ra.shared_gate = shared_gate;
-    ra.topk_idx = tidx;
-    ra.topk_w = tw;
-    ra.gsig = gs;
-    ra.logits = reinterpret_cast<float *>(base + L.logits);
-    ra.xq = xq;
-    ra.xsc = xsc;
-    ra.counters = counters;
-    ra.plan = nullptr;
-    if ((e = launch_router_topk(ra, s)) != cudaSuccess) return MOE_ECUDA;
 
     PlanParams pp;
     pp.T = T;
@@ -655,24 +870,46 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     pp.rank = reinterpret_cast<int32_t *>(base + L.rank);
     pp.pos = reinterpret_cast<int32_t *>(base + L.pos);
     pp.mtiles = reinterpret_cast<int4 *>(base + L.mtiles);
-    pp.xq = xq;
-    pp.xsc = xsc;
+    pp.x = x;
+    pp.xp_shared0 = std::max(P, kBM);
     pp.xp = reinterpret_cast<uint8_t *>(base + L.xp);
     pp.xps = reinterpret_cast<float *>(base + L.xps);
     pp.slot_w = reinterpret_cast<float *>(base + L.slot_w);
     pp.counters = counters;
-    const DeviceInfo &di = device_info();
-    const int P = T * K;
-    // 2..4
-    if ((e = launch_kernel(count_kernel, dim3(std::max(1, std::min(4 * di.sm_count, (P + 255) / 256))), dim3(256),
-                           0, s, pp)) != cudaSuccess)
+
+    // 1. router + top-k + per-expert ranks
+    RouterTcParams rp{};
+    rp.T = T;
+    rp.E = E;
+    rp.K = K;
+    rp.H = H;
+    rp.nbox = std::min(kRtChunk, (E + 15) / 16 * 16);
+    rp.bias = router_bias;
+    rp.topk_idx = tidx;
+    rp.topk_w = tw;
+    rp.gsig = gs;
+    rp.counts = pp.counts;
+    rp.rank = pp.rank;
+    rp.counters = counters;
+    if (!make_map(&rp.x, x, 2 * (uint64_t)H, (uint64_t)T, 1, 2 * (uint64_t)H, 0, kBM) ||
+        !make_map(&rp.wr, router_w, 2 * (uint64_t)H, (uint64_t)E, 1, 2 * (uint64_t)H, 0, (uint32_t)rp.nbox) ||
+        !make_map(&rp.g, shared_gate, 2 * (uint64_t)H, 1, 1, 2 * (uint64_t)H, 0, 16))
         return MOE_ECUDA;
+    const unsigned rt_grid = (unsigned)std::min<int64_t>(di.sm_count, (T + kBM - 1) / kBM);
+    if (K <= 2) e = launch_router_tc<2>(rt_grid, rp, s);
+    else if (K <= 4) e = launch_router_tc<4>(rt_grid, rp, s);
+    else if (K <= 8) e = launch_router_tc<8>(rt_grid, rp, s);
+    else if (K <= 16) e = launch_router_tc<16>(rt_grid, rp, s);
+    else e = launch_router_tc<32>(rt_grid, rp, s);
+    if (e != cudaSuccess) return MOE_ECUDA;
+
+    // 2, 3
     if ((e = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pp)) != cudaSuccess) return MOE_ECUDA;
     if ((e = launch_kernel(permute_kernel, dim3(std::max(1, std::min(8 * di.sm_count, (P + T + 7) / 8))), dim3(256),
                            0, s, pp)) != cudaSuccess)
         return MOE_ECUDA;
 
-    // 5. GEMM1
+    // 4. GEMM1
     GemmParams g{};
     g.H = H;
     g.E = E;
@@ -692,20 +929,21 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     // large); rows past the valid ones are read but never stored.
     bool ok = make_map(&g.a_routed, pp.xp, 2 * (uint64_t)H, (uint64_t)std::max<int64_t>(L.routed, kBM), 1,
                        2 * (uint64_t)H, 0, kBM) &&
-              make_map(&g.a_shared, xq, 2 * (uint64_t)H, (uint64_t)std::max(T, kBM), 1, 2 * (uint64_t)H, 0, kBM) &&
+              make_map(&g.a_shared, pp.xp + (size_t)pp.xp_shared0 * 2 * H, 2 * (uint64_t)H,
+                       (uint64_t)std::max(T, kBM), 1, 2 * (uint64_t)H, 0, kBM) &&
               make_map(&g.b_routed, expert_w8, (uint64_t)H, 2 * (uint64_t)I, (uint64_t)E, (uint64_t)H,
                        3 * (uint64_t)I * H, 128) &&
               make_map(&g.b_shared, shared_w8, (uint64_t)H, 2 * (uint64_t)Is, 1, (uint64_t)H, 3 * (uint64_t)Is * H, 128);
     if (!ok) return MOE_ECUDA;
     g.a_scales_routed = pp.xps;
-    g.a_scales_shared = xsc;
+    g.a_scales_shared = pp.xps + (size_t)P * (H / 128);
     g.a_scales_ld = H / 128;
     g.max_ntiles = imax / 128;
     if (!gemm_occupancy_once(gemm_kernel<1>) || !gemm_occupancy_once(gemm_kernel<2>)) return MOE_ECUDA;
     if ((e = launch_kernel(gemm_kernel<1>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g)) != cudaSuccess)
         return MOE_ECUDA;
 
-    // 6. GEMM2
+    // 5. GEMM2
     GemmParams g2 = g;
     const uint64_t Rp = (uint64_t)std::max<int64_t>(R, kBM);
     ok = make_map(&g2.a_routed, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, kBM) &&
@@ -722,7 +960,7 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     if ((e = launch_kernel(gemm_kernel<2>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g2)) != cudaSuccess)
         return MOE_ECUDA;
 
-    // 7. blend
+    // 6. blend
     BlendParams bp;
     bp.T = T;
     bp.K = K;

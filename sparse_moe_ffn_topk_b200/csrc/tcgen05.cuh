@@ -32,6 +32,27 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n)
            | ((uint32_t)(m >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor of kind::f16 with bf16 A and B (K-major) and an fp32
+// accumulator, for an M x N tile.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n)
+{
+    return (1u << 4)                        // D format: f32
+           | (1u << 7) | (1u << 10)         // A, B format: bf16
+           | ((uint32_t)(n >> 3) << 17)     // N / 8
+           | ((uint32_t)(m >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one K=16 step of bf16.
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(tmem_d), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one K=32 step of e4m3.
 __device__ __forceinline__ void umma_f8f6f4(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate)
