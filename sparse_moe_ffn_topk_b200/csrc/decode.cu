@@ -91,7 +91,7 @@ __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) &
 
 // ---------------------------------------------------------------- router
 
-constexpr int kRouterMaxRows = 16;  // router rows per CTA (one per warp)
+constexpr int kRouterMaxRows = 4;   // router rows per CTA (one per warp)
 constexpr int kRouterTok = 8;       // activation rows staged per pass
 
 struct RouterParams {
@@ -120,39 +120,61 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v)
 }
 
 // Top-k of one row (one warp) on order-preserving keys.  Lane L holds the
-// EPL experts L*EPL .. L*EPL+EPL-1.  Key 0 marks a taken (or absent) expert
-// and a NaN logit gets key 1, so every round picks a valid, untaken expert
-// even on non-finite input; equal keys go to the lower expert index.
+// EPL experts L*EPL .. L*EPL+EPL-1, sorted once by descending key (a stable
+// sort, so equal keys keep the lower expert first).  Each round takes the
+// best head across the warp; equal heads go to the lower lane, whose
+// experts all have lower indices, and the winning lane pops its head.  Key 0
+// marks an absent expert and a NaN logit gets key 1, so every round picks a
+// valid expert even on non-finite input.
 template <int EPL>
 __device__ void topk_row(const RouterParams &p, int t)
 {
     const int lane = threadIdx.x & 31;
     const float *lrow = p.logits + (size_t)t * p.ld;
     uint32_t v[EPL];
+    int id[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane * EPL + i;
         const float l = (e < p.E) ? __ldcg(lrow + e) : 0.f;
-        v[i] = (e < p.E) ? (isnan(l) ? 1u : max(ordered_key(l), 2u)) : 0u;
+        v[i] = (e < p.E) ? topk_key(l) : 0u;
+        id[i] = e;
     }
     const float z = __ldcg(lrow + p.E);
+    // odd-even transposition sort, descending; swaps only on a strict
+    // inequality, so it is stable
+#pragma unroll
+    for (int pass = 0; pass < EPL; ++pass) {
+#pragma unroll
+        for (int j = pass & 1; j + 1 < EPL; j += 2) {
+            if (v[j] < v[j + 1]) {
+                const uint32_t tv = v[j];
+                v[j] = v[j + 1];
+                v[j + 1] = tv;
+                const int ti = id[j];
+                id[j] = id[j + 1];
+                id[j + 1] = ti;
+            }
+        }
+    }
     int my_e = 0;
     uint32_t my_k = 0;
     for (int r = 0; r < p.K; ++r) {
-        uint32_t bk = 0;
-        int bi = 0;
+        const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, v[0]);
+        const int wl = __ffs(__ballot_sync(0xFFFFFFFFu, v[0] == kmax)) - 1;
+        const int ew = __shfl_sync(0xFFFFFFFFu, id[0], wl);
+        if (lane == wl) {
 #pragma unroll
-        for (int i = 0; i < EPL; ++i)
-            if (v[i] > bk) { bk = v[i]; bi = i; }
-        const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, bk);
-        const uint32_t cand = (bk == kmax) ? (uint32_t)(lane * EPL + bi) : 0x7FFFFFFFu;
-        const int emin = (int)__reduce_min_sync(0xFFFFFFFFu, cand);
-        if (lane == emin / EPL) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == emin - lane * EPL) v[i] = 0u;
+            for (int j = 0; j + 1 < EPL; ++j) {
+                v[j] = v[j + 1];
+                id[j] = id[j + 1];
+            }
+            v[EPL - 1] = 0u;
         }
-        if (lane == r) { my_e = emin; my_k = kmax; }
+        if (lane == r) {
+            my_e = ew;
+            my_k = kmax;
+        }
     }
     if (threadIdx.x == 0) MOE_TRACE(0, 5);
     const float my_v = (my_k == 1u) ? __int_as_float(0x7FC00000) : key_value(my_k);
@@ -474,7 +496,6 @@ constexpr int kConsumerWarps = 8;
 constexpr int kExpThreads = (kConsumerWarps + 1) * kWarp;
 constexpr int kConsumerThreads = kConsumerWarps * kWarp;
 constexpr int kMaxStages = 4;
-constexpr int kMaxTiles = 4;  // 16-row MMA tiles per item
 constexpr int kRowPad = 16;   // bytes of padding after each staged row
 // Cross-warp reduction area of an item with T 16-row MMA tiles.
 __host__ __device__ constexpr size_t red_bytes(int T) { return (size_t)kConsumerWarps * T * kWarp * 16; }
@@ -508,10 +529,14 @@ __device__ void gu_produce(const ExpertParams &p, const GuLayout &L, const Stage
 {
     const int lane = threadIdx.x & 31;
     const int nt = min(p.tok, d.n);
+    // Scale rows (H/128 floats) travel by bulk copy on the stage's barrier
+    // when they are whole 16-byte units; otherwise the lanes store them.
+    const uint32_t scb = (uint32_t)L.hb * 4;
+    const bool bsc = (scb % 16) == 0 && (smem_u32(st + L.sw) & 15) == 0 && (smem_u32(st + L.xs) & 15) == 0;
     if (lane == 0) {
         uint32_t bytes = 0;
-        if (weights) bytes += (uint32_t)(16 * L.T * p.H);
-        if (acts) bytes += (uint32_t)(2 * nt * p.H);
+        if (weights) bytes += (uint32_t)(16 * L.T * p.H) + (bsc ? 2 * scb : 0);
+        if (acts) bytes += (uint32_t)(2 * nt * p.H) + (bsc ? nt * scb : 0);
         mbar_expect_tx(bar, bytes);
     }
     __syncwarp();
@@ -524,7 +549,12 @@ __device__ void gu_produce(const ExpertParams &p, const GuLayout &L, const Stage
         float *sw = reinterpret_cast<float *>(st + L.sw);
         const float *sg = d.scales + (d.first / 128) * L.hb;
         const float *su = d.scales + ((d.inter + d.first) / 128) * L.hb;
-        for (int i = lane; i < 2 * L.hb; i += kWarp) sw[i] = (i < L.hb) ? __ldg(sg + i) : __ldg(su + i - L.hb);
+        if (bsc) {
+            if (lane == 0) bulk_g2s(sw, sg, scb, bar);
+            if (lane == 1) bulk_g2s(sw + L.hb, su, scb, bar);
+        } else {
+            for (int i = lane; i < 2 * L.hb; i += kWarp) sw[i] = (i < L.hb) ? __ldg(sg + i) : __ldg(su + i - L.hb);
+        }
     }
     if (acts) {
         for (int i = lane; i < 2 * nt; i += kWarp) {
@@ -534,15 +564,23 @@ __device__ void gu_produce(const ExpertParams &p, const GuLayout &L, const Stage
                      (uint32_t)p.H, bar);
         }
         float *xs = reinterpret_cast<float *>(st + L.xs);
-        for (int i = lane; i < nt * L.hb; i += kWarp) {
-            const int t = i / L.hb;
-            const int row = d.pairs ? d.rows[t] / p.K : d.rows[t];
-            xs[i] = __ldcg(p.xsc + (size_t)row * L.hb + (i - t * L.hb));
+        if (bsc) {
+            for (int t = lane; t < nt; t += kWarp) {
+                const int row = d.pairs ? d.rows[t] / p.K : d.rows[t];
+                bulk_g2s(xs + t * L.hb, p.xsc + (size_t)row * L.hb, scb, bar);
+            }
+        } else {
+            for (int i = lane; i < nt * L.hb; i += kWarp) {
+                const int t = i / L.hb;
+                const int row = d.pairs ? d.rows[t] / p.K : d.rows[t];
+                xs[i] = __ldcg(p.xsc + (size_t)row * L.hb + (i - t * L.hb));
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
+template <int T>
+__global__ void __launch_bounds__(kExpThreads, 2) gate_up_kernel(ExpertParams p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
@@ -645,48 +683,55 @@ __global__ void __launch_bounds__(kExpThreads) gate_up_kernel(ExpertParams p)
                 }
                 named_barrier(1, kConsumerThreads);
             }
-            float acc[kMaxTiles][4];
+            float acc[T][4];
 #pragma unroll
-            for (int tau = 0; tau < kMaxTiles; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
+            for (int tau = 0; tau < T; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
             const bool col_ok = g < nt;
             for (int kb = warp; kb < L.hb; kb += kConsumerWarps) {
-                float tmp[kMaxTiles][4];
-#pragma unroll
-                for (int tau = 0; tau < kMaxTiles; ++tau) tmp[tau][0] = tmp[tau][1] = tmp[tau][2] = tmp[tau][3] = 0.f;
+                // all fragments of the K block first, then the MMAs: hi and lo
+                // products on separate accumulator chains
+                uint2 bh[4], bl[4], ra[T][4], rb[T][4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int k0 = kb * 128 + c * 32 + 8 * t;
-                    uint2 bh = make_uint2(0, 0), bl = make_uint2(0, 0);
+                    bh[c] = bl[c] = make_uint2(0, 0);
                     if (col_ok) {
-                        bh = *reinterpret_cast<const uint2 *>(st + L.xh + (size_t)g * L.WS + k0);
-                        bl = *reinterpret_cast<const uint2 *>(st + L.xl + (size_t)g * L.WS + k0);
+                        bh[c] = *reinterpret_cast<const uint2 *>(st + L.xh + (size_t)g * L.WS + k0);
+                        bl[c] = *reinterpret_cast<const uint2 *>(st + L.xl + (size_t)g * L.WS + k0);
                     }
 #pragma unroll
-                    for (int tau = 0; tau < kMaxTiles; ++tau) {
-                        if (tau < L.T) {
-                            const uint2 ra = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g) * L.WS + k0);
-                            const uint2 rb = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g + 8) * L.WS + k0);
-                            mma_e4m3_16832(tmp[tau], ra.x, rb.x, ra.y, rb.y, bh.x, bh.y);
-                            mma_e4m3_16832(tmp[tau], ra.x, rb.x, ra.y, rb.y, bl.x, bl.y);
-                        }
+                    for (int tau = 0; tau < T; ++tau) {
+                        ra[tau][c] = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g) * L.WS + k0);
+                        rb[tau][c] = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g + 8) * L.WS + k0);
                     }
                 }
+                float th[T][4], tl[T][4];
+#pragma unroll
+                for (int tau = 0; tau < T; ++tau)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) th[tau][i] = tl[tau][i] = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int tau = 0; tau < T; ++tau) {
+                        mma_e4m3_16832(th[tau], ra[tau][c].x, rb[tau][c].x, ra[tau][c].y, rb[tau][c].y, bh[c].x, bh[c].y);
+                        mma_e4m3_16832(tl[tau], ra[tau][c].x, rb[tau][c].x, ra[tau][c].y, rb[tau][c].y, bl[c].x, bl[c].y);
+                    }
                 const float sg = swg[kb], su = swg[L.hb + kb];
                 const float x0 = (2 * t < nt) ? xsc[(2 * t) * L.hb + kb] : 0.f;
                 const float x1 = (2 * t + 1 < nt) ? xsc[(2 * t + 1) * L.hb + kb] : 0.f;
 #pragma unroll
-                for (int tau = 0; tau < kMaxTiles; ++tau) {
-                    acc[tau][0] = fmaf(sg * x0, tmp[tau][0], acc[tau][0]);
-                    acc[tau][1] = fmaf(sg * x1, tmp[tau][1], acc[tau][1]);
-                    acc[tau][2] = fmaf(su * x0, tmp[tau][2], acc[tau][2]);
-                    acc[tau][3] = fmaf(su * x1, tmp[tau][3], acc[tau][3]);
+                for (int tau = 0; tau < T; ++tau) {
+                    acc[tau][0] = fmaf(sg * x0, th[tau][0] + tl[tau][0], acc[tau][0]);
+                    acc[tau][1] = fmaf(sg * x1, th[tau][1] + tl[tau][1], acc[tau][1]);
+                    acc[tau][2] = fmaf(su * x0, th[tau][2] + tl[tau][2], acc[tau][2]);
+                    acc[tau][3] = fmaf(su * x1, th[tau][3] + tl[tau][3], acc[tau][3]);
                 }
             }
             if (q == 0 && threadIdx.x == 0) MOE_TRACE(1, 7);
 #pragma unroll
-            for (int tau = 0; tau < kMaxTiles; ++tau)
-                if (tau < L.T)
-                    red[(warp * L.T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
+            for (int tau = 0; tau < T; ++tau)
+                red[(warp * T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
             named_barrier(1, kConsumerThreads);
             if (q == 0 && threadIdx.x == 0) MOE_TRACE(1, 8);
             // (tile, pair row g, column n) -> h
@@ -750,9 +795,13 @@ __device__ void dn_produce(const ExpertParams &p, const DnLayout &L, StageDesc &
 {
     const int lane = threadIdx.x & 31;
     const int ns = min(p.tok, d.n);
+    // The row block's scales (I/128 floats) travel by bulk copy when they
+    // are a whole number of 16-byte units.
+    const int ib = d.inter / 128;
+    const bool bsc = (ib % 4) == 0 && ((p.H / 128) % 4) == 0 && (smem_u32(st + L.sw) & 15) == 0;
     if (lane == 0) {
         uint32_t bytes = 0;
-        if (weights) bytes += (uint32_t)(p.drows * d.inter);
+        if (weights) bytes += (uint32_t)(p.drows * d.inter) + (bsc ? (uint32_t)ib * 4 : 0);
         if (acts) bytes += (uint32_t)(ns * d.inter * 4);
         mbar_expect_tx(bar, bytes);
     }
@@ -761,10 +810,13 @@ __device__ void dn_produce(const ExpertParams &p, const DnLayout &L, StageDesc &
         const uint8_t *w2 = d.slab + (size_t)2 * d.inter * p.H + (size_t)d.first * d.inter;
         for (int i = lane; i < p.drows; i += kWarp)
             bulk_g2s_stream(st + (size_t)i * L.WS, w2 + (size_t)i * d.inter, (uint32_t)d.inter, bar, pol);
-        const int ib = d.inter / 128;
         float *sw = reinterpret_cast<float *>(st + L.sw);
         const float *src = d.scales + (2 * d.inter / 128) * (p.H / 128) + (d.first / 128) * ib;
-        for (int i = lane; i < ib; i += kWarp) sw[i] = __ldg(src + i);
+        if (bsc) {
+            if (lane == 0) bulk_g2s(sw, src, (uint32_t)ib * 4, bar);
+        } else {
+            for (int i = lane; i < ib; i += kWarp) sw[i] = __ldg(src + i);
+        }
         if (lane < ns) d.wt[lane] = d.pairs ? __ldcg(p.topk_w + d.rows[lane]) : __ldcg(p.gsig + lane);
     }
     if (acts) {
@@ -775,7 +827,8 @@ __device__ void dn_produce(const ExpertParams &p, const DnLayout &L, StageDesc &
     }
 }
 
-__global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
+template <int T>
+__global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
@@ -895,45 +948,52 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
                 if (lane == 0) hsc[tr * (L.imax / 128) + kb] = sc;
             }
             named_barrier(1, kConsumerThreads);
-            // (tile, K block) units over the warps
-            float acc[kMaxTiles][4];
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 9);
+            // (tile, K block) units over the warps; per unit all fragments first,
+            // then the MMAs, hi and lo products on separate accumulator chains
+            float acc[T][4];
 #pragma unroll
-            for (int tau = 0; tau < kMaxTiles; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
+            for (int tau = 0; tau < T; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
             const bool col_ok = g < ns;
-            for (int u = warp; u < L.T * ib; u += kConsumerWarps) {
-                const int tau = u % L.T, kb = u / L.T;
-                float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int u = warp; u < T * ib; u += kConsumerWarps) {
+                const int tau = u % T, kb = u / T;
+                uint2 bh[4], bl[4], ra[4], rb[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int k0 = kb * 128 + c * 32 + 8 * t;
-                    uint2 bh = make_uint2(0, 0), bl = make_uint2(0, 0);
+                    bh[c] = bl[c] = make_uint2(0, 0);
                     if (col_ok) {
-                        bh = *reinterpret_cast<const uint2 *>(st + L.hh + (size_t)g * L.WS + k0);
-                        bl = *reinterpret_cast<const uint2 *>(st + L.hl + (size_t)g * L.WS + k0);
+                        bh[c] = *reinterpret_cast<const uint2 *>(st + L.hh + (size_t)g * L.WS + k0);
+                        bl[c] = *reinterpret_cast<const uint2 *>(st + L.hl + (size_t)g * L.WS + k0);
                     }
-                    const uint2 ra = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g) * L.WS + k0);
-                    const uint2 rb = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g + 8) * L.WS + k0);
-                    mma_e4m3_16832(tmp, ra.x, rb.x, ra.y, rb.y, bh.x, bh.y);
-                    mma_e4m3_16832(tmp, ra.x, rb.x, ra.y, rb.y, bl.x, bl.y);
+                    ra[c] = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g) * L.WS + k0);
+                    rb[c] = *reinterpret_cast<const uint2 *>(st + (size_t)(16 * tau + g + 8) * L.WS + k0);
+                }
+                float th[4] = {0.f, 0.f, 0.f, 0.f}, tl[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    mma_e4m3_16832(th, ra[c].x, rb[c].x, ra[c].y, rb[c].y, bh[c].x, bh[c].y);
+                    mma_e4m3_16832(tl, ra[c].x, rb[c].x, ra[c].y, rb[c].y, bl[c].x, bl[c].y);
                 }
                 const float ws_ = sw[kb];
                 const float h0 = (2 * t < ns) ? hsc[(2 * t) * (L.imax / 128) + kb] : 0.f;
                 const float h1 = (2 * t + 1 < ns) ? hsc[(2 * t + 1) * (L.imax / 128) + kb] : 0.f;
 #pragma unroll
-                for (int tt = 0; tt < kMaxTiles; ++tt) {
+                for (int tt = 0; tt < T; ++tt) {
                     if (tt == tau) {
-                        acc[tt][0] = fmaf(ws_ * h0, tmp[0], acc[tt][0]);
-                        acc[tt][1] = fmaf(ws_ * h1, tmp[1], acc[tt][1]);
-                        acc[tt][2] = fmaf(ws_ * h0, tmp[2], acc[tt][2]);
-                        acc[tt][3] = fmaf(ws_ * h1, tmp[3], acc[tt][3]);
+                        acc[tt][0] = fmaf(ws_ * h0, th[0] + tl[0], acc[tt][0]);
+                        acc[tt][1] = fmaf(ws_ * h1, th[1] + tl[1], acc[tt][1]);
+                        acc[tt][2] = fmaf(ws_ * h0, th[2] + tl[2], acc[tt][2]);
+                        acc[tt][3] = fmaf(ws_ * h1, th[3] + tl[3], acc[tt][3]);
                     }
                 }
             }
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 10);
 #pragma unroll
-            for (int tau = 0; tau < kMaxTiles; ++tau)
-                if (tau < L.T)
-                    red[(warp * L.T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
+            for (int tau = 0; tau < T; ++tau)
+                red[(warp * T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
             named_barrier(1, kConsumerThreads);
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 11);
             // (output row, slot column) -> weighted partial
             for (int i = threadIdx.x; i < 128 * L.T; i += kConsumerThreads) {
                 const int tau = i >> 7, r = (i >> 3) & 15, n = i & 7;
@@ -957,6 +1017,7 @@ __global__ void __launch_bounds__(kExpThreads) down_blend_kernel(ExpertParams p)
                 }
                 p.yslot[(size_t)yrow * p.H + row] = wt * y;
             }
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 12);
             named_barrier(1, kConsumerThreads);  // red and the h staging are free again
         }
         if (q < 2 && threadIdx.x == 0) MOE_TRACE(2, 3 + 3 * q);
@@ -1044,6 +1105,9 @@ int occupancy(void (*kernel)(P), int block, size_t smem)
         if (optin > fa.sharedSizeBytes)
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(optin - fa.sharedSizeBytes));
+        // The largest shared-memory carveout, so that a gate_up and a down CTA
+        // (different kernels) can be resident on one SM together.
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         configured.push_back({(const void *)kernel, dev});
     }
     int b = 0;
@@ -1061,7 +1125,7 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
     const int imax = std::max(I, Is);
     rows = std::max<int64_t>(rows, 1);
     // router: rows_per_cta router rows (<= 32 KB) and kRouterTok activation rows per CTA
-    s.router_rows = std::max(1, std::min(4, 32768 / H));
+    s.router_rows = std::max(1, std::min(kRouterMaxRows, 32768 / H));
     s.router_groups = (int)std::min<int64_t>((rows + kRouterTok - 1) / kRouterTok, kMaxRouterGroups);
     s.router_group_tokens = (int)((rows + s.router_groups - 1) / s.router_groups);
     s.router_smem = std::max<size_t>((size_t)(s.router_rows + kRouterTok) * H * 2, (size_t)(3 * E + 33) * 4);
@@ -1177,21 +1241,27 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
     // gate_up
     {
         p.stages = sh.gu_stages;
-        const int bps = occupancy(gate_up_kernel, kExpThreads, sh.gu_smem);
+        void (*kern)(ExpertParams) = sh.gu_pairs == 8    ? gate_up_kernel<1>
+                                     : sh.gu_pairs == 16 ? gate_up_kernel<2>
+                                                         : gate_up_kernel<4>;
+        const int bps = occupancy(kern, kExpThreads, sh.gu_smem);
         if (bps < 1) return cudaErrorInvalidConfiguration;
         const int64_t items = (int64_t)(d.shared_inter / sh.gu_pairs) + max_active * (d.inter / sh.gu_pairs);
         const int grid = (int)std::min<int64_t>(items, (int64_t)di.sm_count);
-        cudaError_t e = launch_kernel(gate_up_kernel, dim3(grid), dim3(kExpThreads), sh.gu_smem, s, p);
+        cudaError_t e = launch_kernel(kern, dim3(grid), dim3(kExpThreads), sh.gu_smem, s, p);
         if (e != cudaSuccess) return e;
     }
     // down + blend
     {
         p.stages = sh.dn_stages;
-        const int bps = occupancy(down_blend_kernel, kExpThreads, sh.dn_smem);
+        void (*kern)(ExpertParams) = sh.dn_rows == 16   ? down_blend_kernel<1>
+                                     : sh.dn_rows == 32 ? down_blend_kernel<2>
+                                                        : down_blend_kernel<4>;
+        const int bps = occupancy(kern, kExpThreads, sh.dn_smem);
         if (bps < 1) return cudaErrorInvalidConfiguration;
         const int64_t items = (max_active + 1) * (d.hidden / sh.dn_rows);
         const int grid = (int)std::min<int64_t>(items, (int64_t)di.sm_count);
-        cudaError_t e = launch_kernel(down_blend_kernel, dim3(grid), dim3(kExpThreads), sh.dn_smem, s, p);
+        cudaError_t e = launch_kernel(kern, dim3(grid), dim3(kExpThreads), sh.dn_smem, s, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -42,7 +42,9 @@ constexpr int kGemmThreads = 320;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2..
 constexpr int kEpiThreads = 256;
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 constexpr size_t kStageBytes = 2 * kBM * kBK + kBN * kBK;  // A hi, A lo, B
-constexpr size_t kGemmSmem = kGemmStages * kStageBytes + 1024 /* alignment slack */ + 4096 /* epilogue scratch */;
+constexpr int kStgBytes = 32 * 80;  // per epilogue warp: 32 rows x 80 B staging for coalesced stores
+constexpr size_t kGemmSmem =
+    kGemmStages * kStageBytes + 1024 /* alignment slack */ + 4096 /* amax exchange */ + 8 * kStgBytes;
 
 // ------------------------------------------------------------ layout
 
@@ -618,6 +620,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const int half = (warp - 2) >> 2;          // column half
         const int r = q * 32 + lane;               // row within the tile
         const int et = threadIdx.x - 64;           // 0..255
+        unsigned char *stg = smem + kGemmStages * kStageBytes + 4096 + (size_t)(warp - 2) * kStgBytes;
         int acc_it = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
             TileInfo ti;
@@ -647,14 +650,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 128; ++i) tot[i] = 0.f;
             bool ok = true;
+            // scales one K block ahead, so their loads overlap the wait for the accumulator
+            float sa_n = valid ? __ldg(asc) : 0.f;
+            float s0_n = __ldg(wsc + (size_t)wn0 * wld), s1_n = __ldg(wsc + (size_t)wn1 * wld);
             for (int kb = 0; kb < nkb; ++kb, ++acc_it) {
                 const int b = acc_it & 1;
-                const float sa = (valid && ok) ? __ldg(asc + kb) : 0.f;
-                const float s0 = __ldg(wsc + (size_t)wn0 * wld + kb), s1 = __ldg(wsc + (size_t)wn1 * wld + kb);
-                if (ok && !mbar_wait(&acc_full[b], (acc_it >> 1) & 1, kWaitLimitNs)) {
-                    set_status(p.counters, MOE_ETIMEOUT);
-                    s_abort = 1;
-                    ok = false;
+                const float sa = sa_n, s0 = s0_n, s1 = s1_n;
+                if (kb + 1 < nkb) {
+                    sa_n = valid ? __ldg(asc + kb + 1) : 0.f;
+                    s0_n = __ldg(wsc + (size_t)wn0 * wld + kb + 1);
+                    s1_n = __ldg(wsc + (size_t)wn1 * wld + kb + 1);
+                }
+                if (ok) {
+                    // warp-uniform outcome: the TMEM loads below are warp-collective
+                    const bool w = mbar_wait(&acc_full[b], (acc_it >> 1) & 1, kWaitLimitNs);
+                    if (!__all_sync(0xFFFFFFFFu, w)) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        ok = false;
+                    }
                 }
                 if (!ok) continue;
                 tc_fence_after();
@@ -699,27 +713,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 amax = fmaxf(epi_scratch[r], epi_scratch[128 + r]);
                 const float sc = amax > 0.f ? amax / 448.f : 1.f;
                 const float inv = 1.f / sc;
-                if (valid && ok) {
-                    const size_t grow = (size_t)ti.row0 + r;
-                    uint32_t *hi = reinterpret_cast<uint32_t *>(p.hq + grow * 2 * p.imax + ti.nt * 128 + 64 * half);
-                    uint32_t *lo = reinterpret_cast<uint32_t *>(p.hq + grow * 2 * p.imax + p.imax + ti.nt * 128 + 64 * half);
+                if (ok) {
+                    // hi, then lo: this warp's 32 rows x 64 bytes go through its staging
+                    // buffer, then out as 64-byte row segments, 16 bytes per lane
+                    uint4 *srow = reinterpret_cast<uint4 *>(stg + lane * 80);
+                    for (int part = 0; part < 2; ++part) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        uint32_t h4, l4;
-                        quant4_hilo(make_float4(tot[4 * i], tot[4 * i + 1], tot[4 * i + 2], tot[4 * i + 3]), inv, h4, l4);
-                        hi[i] = h4;
-                        lo[i] = l4;
+                        for (int i = 0; i < 4; ++i) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int c = 16 * i + 4 * j;
+                                uint32_t h4, l4;
+                                quant4_hilo(make_float4(tot[c], tot[c + 1], tot[c + 2], tot[c + 3]), inv, h4, l4);
+                                w4[j] = part ? l4 : h4;
+                            }
+                            srow[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = 8 * i + (lane >> 2), ch = lane & 3;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * 80 + ch * 16);
+                            if (q * 32 + rr < ti.rows) {
+                                const size_t grow = (size_t)ti.row0 + q * 32 + rr;
+                                *reinterpret_cast<uint4 *>(p.hq + grow * 2 * p.imax + (part ? p.imax : 0) + ti.nt * 128 +
+                                                           64 * half + ch * 16) = v;
+                            }
+                        }
+                        __syncwarp();
                     }
-                    if (half == 0) p.hs[grow * (p.imax / 128) + ti.nt] = sc;
+                    if (valid && half == 0) p.hs[((size_t)ti.row0 + r) * (p.imax / 128) + ti.nt] = sc;
                 }
             } else {
-                if (valid && ok) {
-                    const size_t grow = (size_t)ti.row0 + r;
-                    const float w = __ldg(p.slot_w + grow);
-                    float4 *y = reinterpret_cast<float4 *>(p.yslot + grow * p.H + ti.nt * kBN + 128 * half);
+                if (ok) {
+                    // 16 columns at a time through the staging buffer (rows of 17
+                    // floats), then out as 64-byte row segments, 16 bytes per lane
+                    const float w = valid ? __ldg(p.slot_w + (size_t)ti.row0 + r) : 0.f;
+                    float *sf = reinterpret_cast<float *>(stg);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        y[i] = make_float4(w * tot[4 * i], w * tot[4 * i + 1], w * tot[4 * i + 2], w * tot[4 * i + 3]);
+                    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) sf[lane * 17 + j] = w * tot[16 * c + j];
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = 8 * i + (lane >> 2), ch = lane & 3;
+                            const float *src = sf + rr * 17 + ch * 4;
+                            const float4 v = make_float4(src[0], src[1], src[2], src[3]);
+                            if (q * 32 + rr < ti.rows) {
+                                const size_t grow = (size_t)ti.row0 + q * 32 + rr;
+                                *reinterpret_cast<float4 *>(p.yslot + grow * p.H + ti.nt * kBN + 128 * half + 16 * c +
+                                                            4 * ch) = v;
+                            }
+                        }
+                        __syncwarp();
+                    }
                 }
             }
             (void)et;
