@@ -38,6 +38,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "launch.h"
+#include "tcgen05.cuh"
 
 namespace moe {
 
@@ -356,6 +357,8 @@ struct ExpertParams {
     int drows;   // down: rows per item (a multiple of 16, <= 64)
     int tok;     // activation / h rows staged with an item (<= kDescPairs)
     int stages;  // ring depth
+    int ue;      // down by output block: experts per stage
+    int l2_w2;   // gate_up: prefetch the active experts' down weights into L2
 };
 
 // What a stage holds; written by the producer before the stage's "full"
@@ -579,6 +582,32 @@ __device__ void gu_produce(const ExpertParams &p, const GuLayout &L, const Stage
     }
 }
 
+// Warm L2 with the down weights of the active experts and of the shared
+// expert, 64 KB pieces spread over the CTAs (piece i goes to CTA i mod grid):
+// the down kernel then reads them from L2 instead of waiting on HBM.
+__device__ void prefetch_down_weights(const ExpertParams &p, const LocalPlan &lp, int n_active)
+{
+    const int lane = threadIdx.x & 31;
+    const size_t piece = 65536, per = (size_t)p.I * p.H, per_s = (size_t)p.Is * p.H;
+    const size_t pieces_r = (per + piece - 1) / piece, pieces_s = (per_s + piece - 1) / piece;
+    const size_t total = (size_t)n_active * pieces_r + pieces_s;
+    for (size_t i = blockIdx.x + (size_t)lane * gridDim.x; i < total; i += (size_t)gridDim.x * kWarp) {
+        const uint8_t *base;
+        size_t off, len;
+        if (i < (size_t)n_active * pieces_r) {
+            const size_t u = i / pieces_r;
+            off = (i - u * pieces_r) * piece;
+            len = per;
+            base = p.w8 + (size_t)lp.e_of[u] * 3 * p.I * p.H + (size_t)2 * p.I * p.H;
+        } else {
+            off = (i - (size_t)n_active * pieces_r) * piece;
+            len = per_s;
+            base = p.sw8 + (size_t)2 * p.Is * p.H;
+        }
+        prefetch_l2(base + off, (uint32_t)(len - off < piece ? len - off : piece));
+    }
+}
+
 template <int T>
 __global__ void __launch_bounds__(kExpThreads, 2) gate_up_kernel(ExpertParams p)
 {
@@ -619,9 +648,9 @@ __global__ void __launch_bounds__(kExpThreads, 2) gate_up_kernel(ExpertParams p)
     }
     pdl_wait();
     pdl_trigger();
-    const int n_items = per_shared + build_local_plan(p, lp) * per_routed;
+    const int n_active = build_local_plan(p, lp);
+    const int n_items = per_shared + n_active * per_routed;
     if (threadIdx.x == 0) MOE_TRACE(1, 1);
-
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------- producer
         for (int q = 0;; ++q) {
@@ -643,7 +672,9 @@ __global__ void __launch_bounds__(kExpThreads, 2) gate_up_kernel(ExpertParams p)
             gu_produce(p, L, desc[s], st, &full[s], pol, !prefetched, true);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
+            if (q == S - 1 && p.l2_w2) prefetch_down_weights(p, lp, n_active);  // after this CTA's first stages
         }
+        if (p.l2_w2 && n_items <= (int)blockIdx.x + (S - 1) * (int)gridDim.x) prefetch_down_weights(p, lp, n_active);
         return;
     }
 
@@ -768,6 +799,20 @@ __global__ void __launch_bounds__(kExpThreads, 2) gate_up_kernel(ExpertParams p)
 
 // ------------------------------------------------------------ down+blend
 
+// One K block's contribution to a down product, in the fixed arithmetic both
+// down kernels share: (weight scale x h scale) x (hi product + lo product),
+// each operation rounded on its own.  Components: rows g and g+8 of the
+// tile, columns 2t and 2t+1.
+__device__ __forceinline__ float4 down_partial(float ws, float h0, float h1, const float (&th)[4], const float (&tl)[4])
+{
+    const float a0 = __fmul_rn(ws, h0), a1 = __fmul_rn(ws, h1);
+    return make_float4(__fmul_rn(a0, __fadd_rn(th[0], tl[0])), __fmul_rn(a1, __fadd_rn(th[1], tl[1])),
+                       __fmul_rn(a0, __fadd_rn(th[2], tl[2])), __fmul_rn(a1, __fadd_rn(th[3], tl[3])));
+}
+
+// Reduction area of a down item: one float4 per lane for each (tile, K block).
+__host__ __device__ constexpr size_t dn_red_bytes(int T, int ib) { return (size_t)T * (ib > 8 ? ib : 8) * kWarp * 16; }
+
 // Stage layout (WS = Imax + 16): [drows weight rows][tok raw h rows, fp32]
 // [tok h-hi rows][tok h-lo rows][h scales: tok * Imax/128][row-block scales:
 // Imax/128]
@@ -838,8 +883,8 @@ __global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams
     const DnLayout L = dn_layout(p);
     const int per_block = p.H / p.drows;  // items per expert
     const int S = p.stages;
-    float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [warp][tile][lane]
-    const LocalPlan lp = plan_at(smem + (size_t)S * L.bytes + red_bytes(L.T), p.E, p.rows * p.K);
+    float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [tile][K block][lane]
+    const LocalPlan lp = plan_at(smem + (size_t)S * L.bytes + dn_red_bytes(L.T, L.imax / 128), p.E, p.rows * p.K);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -950,10 +995,10 @@ __global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams
             named_barrier(1, kConsumerThreads);
             if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 9);
             // (tile, K block) units over the warps; per unit all fragments first,
-            // then the MMAs, hi and lo products on separate accumulator chains
-            float acc[T][4];
-#pragma unroll
-            for (int tau = 0; tau < T; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.f;
+            // then the MMAs, hi and lo products on separate accumulator chains.
+            // Each unit's scaled partial goes to its own slot of `red`; the
+            // partials are then summed in K-block order, so that the result
+            // does not depend on how units were spread over warps.
             const bool col_ok = g < ns;
             for (int u = warp; u < T * ib; u += kConsumerWarps) {
                 const int tau = u % T, kb = u / T;
@@ -978,20 +1023,9 @@ __global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams
                 const float ws_ = sw[kb];
                 const float h0 = (2 * t < ns) ? hsc[(2 * t) * (L.imax / 128) + kb] : 0.f;
                 const float h1 = (2 * t + 1 < ns) ? hsc[(2 * t + 1) * (L.imax / 128) + kb] : 0.f;
-#pragma unroll
-                for (int tt = 0; tt < T; ++tt) {
-                    if (tt == tau) {
-                        acc[tt][0] = fmaf(ws_ * h0, th[0] + tl[0], acc[tt][0]);
-                        acc[tt][1] = fmaf(ws_ * h1, th[1] + tl[1], acc[tt][1]);
-                        acc[tt][2] = fmaf(ws_ * h0, th[2] + tl[2], acc[tt][2]);
-                        acc[tt][3] = fmaf(ws_ * h1, th[3] + tl[3], acc[tt][3]);
-                    }
-                }
+                red[(tau * ib + kb) * kWarp + lane] = down_partial(ws_, h0, h1, th, tl);
             }
             if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 10);
-#pragma unroll
-            for (int tau = 0; tau < T; ++tau)
-                red[(warp * T + tau) * kWarp + lane] = make_float4(acc[tau][0], acc[tau][1], acc[tau][2], acc[tau][3]);
             named_barrier(1, kConsumerThreads);
             if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 11);
             // (output row, slot column) -> weighted partial
@@ -1000,10 +1034,9 @@ __global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams
                 if (n >= ns) continue;
                 const int src = (r & 7) * 4 + (n >> 1), comp = (n & 1) + (r >= 8 ? 2 : 0);
                 float y = 0.f;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float4 v = red[(w * L.T + tau) * kWarp + src];
-                    y += comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w;
+                for (int kb = 0; kb < ib; ++kb) {
+                    const float4 v = red[(tau * ib + kb) * kWarp + src];
+                    y = __fadd_rn(y, comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w);
                 }
                 const int row = d.first + 16 * tau + r;
                 int yrow;
@@ -1015,7 +1048,7 @@ __global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams
                     yrow = p.rows * p.K + s0 + n;
                     wt = s0 == 0 ? d.wt[n] : __ldcg(p.gsig + s0 + n);
                 }
-                p.yslot[(size_t)yrow * p.H + row] = wt * y;
+                p.yslot[(size_t)yrow * p.H + row] = __fmul_rn(wt, y);
             }
             if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 12);
             named_barrier(1, kConsumerThreads);  // red and the h staging are free again
@@ -1046,6 +1079,306 @@ __global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams
         }
         named_barrier(1, kConsumerThreads);  // s_last is read by all before the next item sets it
         if (q < 2 && threadIdx.x == 0) MOE_TRACE(2, 4 + 3 * q);
+    }
+    if (threadIdx.x == 0) MOE_TRACE(2, 8);
+}
+
+// ------------------------------------------------------- down, few rows
+
+// For a few rows, the down product and blend by output block: a CTA item is
+// 16 output rows (one MMA tile) for every active expert and the shared
+// expert, so each output element is complete inside one CTA and is written
+// straight to `out` (no per-slot partials in HBM, no cross-CTA counting).
+// The item's experts are streamed through a two-stage ring `ue` at a time;
+// each expert's 16 x I block arrives by TMA in 128-byte-swizzled boxes of
+// 16 rows x 128 bytes (one box per 128-wide K block).  Every h row arrives
+// by bulk copy and is quantised once per CTA.  The arithmetic is the one the
+// item-based down kernel uses (down_partial, K blocks in order, rank-order
+// blend), so the two kernels give identical bits.
+struct DsLayout {
+    int WS, imax, ib, ibp, ue, S_all;
+    size_t sc, stage, hraw, hh, hl, hs, ys, wt, plan;
+};
+__host__ __device__ inline DsLayout ds_layout(int K, int I, int Is, int rows, int ue, int stages)
+{
+    DsLayout L;
+    L.imax = I > Is ? I : Is;
+    L.WS = L.imax + kRowPad;
+    L.ib = L.imax / 128;
+    L.ibp = (L.ib + 3) / 4 * 4;
+    L.ue = ue;
+    L.S_all = rows * K + rows;
+    L.sc = (size_t)ue * L.ib * 2048;
+    L.stage = (L.sc + (size_t)ue * L.ibp * 4 + 1023) / 1024 * 1024;
+    L.hraw = (size_t)stages * L.stage;
+    L.hh = L.hraw + (size_t)L.S_all * L.imax * 4;
+    L.hl = L.hh + (size_t)L.S_all * L.WS;
+    L.hs = L.hl + (size_t)L.S_all * L.WS;
+    L.ys = L.hs + align16((size_t)L.S_all * L.ib * 4);
+    L.wt = L.ys + (size_t)L.S_all * 16 * 4;
+    L.plan = L.wt + align16((size_t)L.S_all * 4);
+    return L;
+}
+
+struct DsParams {
+    CUtensorMap w2r;  // routed down weights: (I bytes, H rows, E experts), boxes 128 B x 16 rows
+    CUtensorMap w2s;  // shared expert's down weights: (Is bytes, H rows)
+    ExpertParams p;
+};
+
+// Byte offset of (row r, K byte k) of a 16-row box group laid out by TMA with
+// the 128-byte swizzle: box kb = k / 128 at kb * 2048; in a box, row r at
+// r * 128 with its 16-byte units permuted by r mod 8.
+__device__ __forceinline__ uint32_t sw128_off(int r, int k)
+{
+    const int kb = k >> 7, o = k & 127;
+    return (uint32_t)(kb * 2048 + r * 128 + ((((o >> 4) ^ (r & 7))) << 4) + (o & 15));
+}
+
+// Producer warp: W2 rows [16 rb, +16) of experts [u0, u0 + n) of the table
+// (index n_active is the shared expert) and their row-block scales.
+__device__ void ds_produce(const DsParams &P, const DsLayout &L, const LocalPlan &lp, int n_active, int rb, int u0,
+                           int n, unsigned char *st, uint64_t *bar, uint64_t pol)
+{
+    const ExpertParams &p = P.p;
+    const int lane = threadIdx.x & 31;
+    uint32_t bytes = 0;
+    for (int j = 0; j < n; ++j) {
+        const int ibu = ((u0 + j < n_active) ? p.I : p.Is) / 128;
+        bytes += (uint32_t)ibu * 2048 + (ibu % 4 == 0 ? (uint32_t)ibu * 4 : 0);
+    }
+    if (lane == 0) mbar_expect_tx(bar, bytes);
+    __syncwarp();
+    for (int i = lane; i < n * L.ib; i += kWarp) {
+        const int j = i / L.ib, kb = i - j * L.ib, u = u0 + j;
+        const bool sh = u >= n_active;
+        if (kb >= (sh ? p.Is : p.I) / 128) continue;
+        unsigned char *dst = st + ((size_t)j * L.ib + kb) * 2048;
+        if (sh) tma_load_2d(dst, &P.w2s, kb * 128, 16 * rb, bar, pol);
+        else tma_load_3d(dst, &P.w2r, kb * 128, 16 * rb, lp.e_of[u], bar, pol);
+    }
+    for (int j = lane; j < n; j += kWarp) {
+        const int u = u0 + j;
+        const bool sh = u >= n_active;
+        const int inter = sh ? p.Is : p.I, ibu = inter / 128;
+        const float *src = (sh ? p.ssc : p.sc + (size_t)lp.e_of[u] * expert_nscales(p.H, p.I)) +
+                           (2 * inter / 128) * (p.H / 128) + ((16 * rb) / 128) * ibu;
+        float *dst = reinterpret_cast<float *>(st + L.sc) + j * L.ibp;
+        if (ibu % 4 == 0) {
+            bulk_g2s(dst, src, (uint32_t)ibu * 4, bar);
+        } else {
+            for (int k = 0; k < ibu; ++k) dst[k] = __ldg(src + k);
+        }
+    }
+    __syncwarp();  // the lanes' scale stores precede the arrival
+    if (lane == 0) mbar_arrive(bar);
+}
+
+// Producer warp: every h row (routed slots, then the shared rows) into the
+// CTA's h area by bulk copy, completing `bar`.
+__device__ void ds_produce_h(const ExpertParams &p, const DsLayout &L, unsigned char *smem, uint64_t *bar)
+{
+    const int lane = threadIdx.x & 31;
+    const int PR = p.rows * p.K;
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(PR * p.I + p.rows * p.Is) * 4);
+    __syncwarp();
+    for (int sl = lane; sl < L.S_all; sl += kWarp) {
+        const bool sh = sl >= PR;
+        const float *src = sh ? p.h_shared + (size_t)(sl - PR) * p.Is : p.h_routed + (size_t)sl * p.I;
+        bulk_g2s(smem + L.hraw + (size_t)sl * L.imax * 4, src, (uint32_t)(sh ? p.Is : p.I) * 4, bar);
+    }
+}
+
+__global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid_constant__ DsParams P)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], hbar;
+    __shared__ volatile int s_abort;
+    const ExpertParams &p = P.p;
+    const int ue = p.ue, S = p.stages;
+    unsigned char *smem =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const DsLayout L = ds_layout(p.K, p.I, p.Is, p.rows, ue, S);
+    const LocalPlan lp = plan_at(smem + L.plan, p.E, p.rows * p.K);
+    const int PR = p.rows * p.K;
+    float *wt = reinterpret_cast<float *>(smem + L.wt);
+    float *ys = reinterpret_cast<float *>(smem + L.ys);
+    float *hs = reinterpret_cast<float *>(smem + L.hs);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        mbar_init(&hbar, 1);
+        fence_mbar_init();
+    }
+    if (warp == kConsumerWarps && lane == 0) {
+        tma_prefetch_desc(&P.w2r);
+        tma_prefetch_desc(&P.w2s);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(2, 0);
+    // The router finished before this kernel could launch: the routing is final.
+    const int n_active = build_local_plan(p, lp);
+    const int n_exp = n_active + 1;             // + the shared expert
+    const int chunks = (n_exp + ue - 1) / ue;   // stage loads per item
+    const int n_items = p.H / 16;
+    for (int i = threadIdx.x; i < L.S_all; i += blockDim.x)
+        wt[i] = i < PR ? __ldcg(p.topk_w + i) : __ldcg(p.gsig + i - PR);
+    __syncthreads();  // every thread wrote some of wt; the consumers read all of it
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------- producer
+        const uint64_t pol = policy_evict_first();
+        int q = 0;
+        bool h_done = false;
+        for (int item = blockIdx.x; item < n_items && !s_abort; item += gridDim.x) {
+            for (int c = 0; c < chunks; ++c, ++q) {
+                const int s = q % S;
+                if (q == S && !h_done) {  // the first stages are in flight: now h (after gate_up)
+                    h_done = true;
+                    pdl_wait();
+                    pdl_trigger();
+                    ds_produce_h(p, L, smem, &hbar);
+                }
+                if (q >= S && !mbar_wait(&empty[s], ((q / S) - 1) & 1, kWaitLimitNs)) {
+                    if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+                    s_abort = 1;
+                    break;
+                }
+                if (lane == 0 && q >= S) fence_proxy_async_smem();
+                __syncwarp();
+                ds_produce(P, L, lp, n_active, item, c * ue, min(ue, n_exp - c * ue), smem + (size_t)s * L.stage,
+                           &full[s], pol);
+            }
+        }
+        if (!h_done) {
+            pdl_wait();
+            pdl_trigger();
+            ds_produce_h(p, L, smem, &hbar);
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------- consumers
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x == 0) MOE_TRACE(2, 1);
+    if (!mbar_wait(&hbar, 0, kWaitLimitNs)) {
+        if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+        s_abort = 1;
+    }
+    // every h row -> hi/lo e4m3 with a scale per (slot, 128 block): a warp per block
+    {
+        const int units_r = PR * (p.I / 128), units = units_r + p.rows * (p.Is / 128);
+        for (int u = warp; u < units; u += kConsumerWarps) {
+            int sl, kb;
+            if (u < units_r) {
+                sl = u / (p.I / 128);
+                kb = u - sl * (p.I / 128);
+            } else {
+                const int w = u - units_r;
+                const int t = w / (p.Is / 128);
+                kb = w - t * (p.Is / 128);
+                sl = PR + t;
+            }
+            const float4 v = reinterpret_cast<const float4 *>(smem + L.hraw + (size_t)sl * L.imax * 4)[kb * 32 + lane];
+            const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            const float sc = amax > 0.f ? amax / 448.f : 1.f;
+            uint32_t hi, lo;
+            quant4_hilo(v, 1.f / sc, hi, lo);
+            reinterpret_cast<uint32_t *>(smem + L.hh + (size_t)sl * L.WS)[kb * 32 + lane] = hi;
+            reinterpret_cast<uint32_t *>(smem + L.hl + (size_t)sl * L.WS)[kb * 32 + lane] = lo;
+            if (lane == 0) hs[sl * L.ib + kb] = sc;
+        }
+    }
+    named_barrier(1, kConsumerThreads);
+    if (threadIdx.x == 0) MOE_TRACE(2, 2);
+    const int g = lane >> 2, t = lane & 3;
+    int q = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        for (int c = 0; c < chunks; ++c, ++q) {
+            const int s = q % S;
+            const unsigned char *st = smem + (size_t)s * L.stage;
+            if (!s_abort && !mbar_wait(&full[s], (q / S) & 1, kWaitLimitNs)) {
+                if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
+                s_abort = 1;
+            }
+            named_barrier(1, kConsumerThreads);  // every consumer warp sees the same abort flag
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 3);
+            const int n = s_abort ? 0 : min(ue, n_exp - c * ue);
+            for (int j = warp; j < n; j += kConsumerWarps) {
+                const int u = c * ue + j;
+                const bool sh = u >= n_active;
+                const int ibu = (sh ? p.Is : p.I) / 128;
+                const int f0 = sh ? 0 : lp.first_of[u];
+                const int ncol = sh ? p.rows : lp.first_of[u + 1] - f0;  // <= rows <= 8
+                const int sg = g < ncol ? (sh ? PR + g : lp.pairs[f0 + g]) : -1;
+                const int c0 = 2 * t < ncol ? (sh ? PR + 2 * t : lp.pairs[f0 + 2 * t]) : -1;
+                const int c1 = 2 * t + 1 < ncol ? (sh ? PR + 2 * t + 1 : lp.pairs[f0 + 2 * t + 1]) : -1;
+                const float *wsc = reinterpret_cast<const float *>(st + L.sc) + j * L.ibp;
+                const unsigned char *wj = st + (size_t)j * L.ib * 2048;
+                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int kb = 0; kb < ibu; ++kb) {
+                    uint2 bh[4], bl[4], ra[4], rb[4];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const int k0 = kb * 128 + cc * 32 + 8 * t;
+                        bh[cc] = bl[cc] = make_uint2(0, 0);
+                        if (sg >= 0) {
+                            bh[cc] = *reinterpret_cast<const uint2 *>(smem + L.hh + (size_t)sg * L.WS + k0);
+                            bl[cc] = *reinterpret_cast<const uint2 *>(smem + L.hl + (size_t)sg * L.WS + k0);
+                        }
+                        ra[cc] = *reinterpret_cast<const uint2 *>(wj + sw128_off(g, k0));
+                        rb[cc] = *reinterpret_cast<const uint2 *>(wj + sw128_off(g + 8, k0));
+                    }
+                    float th[4] = {0.f, 0.f, 0.f, 0.f}, tl[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        mma_e4m3_16832(th, ra[cc].x, rb[cc].x, ra[cc].y, rb[cc].y, bh[cc].x, bh[cc].y);
+                        mma_e4m3_16832(tl, ra[cc].x, rb[cc].x, ra[cc].y, rb[cc].y, bl[cc].x, bl[cc].y);
+                    }
+                    const float h0 = c0 >= 0 ? hs[c0 * L.ib + kb] : 0.f;
+                    const float h1 = c1 >= 0 ? hs[c1 * L.ib + kb] : 0.f;
+                    const float4 v = down_partial(wsc[kb], h0, h1, th, tl);
+                    y.x = __fadd_rn(y.x, v.x);
+                    y.y = __fadd_rn(y.y, v.y);
+                    y.z = __fadd_rn(y.z, v.z);
+                    y.w = __fadd_rn(y.w, v.w);
+                }
+                if (c0 >= 0) {
+                    ys[c0 * 16 + g] = y.x;
+                    ys[c0 * 16 + g + 8] = y.z;
+                }
+                if (c1 >= 0) {
+                    ys[c1 * 16 + g] = y.y;
+                    ys[c1 * 16 + g + 8] = y.w;
+                }
+            }
+            named_barrier(1, kConsumerThreads);  // the stage is consumed, ys is complete for these experts
+            if (q == 0 && threadIdx.x == 0) MOE_TRACE(2, 4);
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        // out[t][16 item + r]: the k weighted partials in rank order, then the
+        // shared expert's, then the residual; one bf16 rounding
+        if (!s_abort) {
+            for (int i = threadIdx.x; i < p.rows * 16; i += kConsumerThreads) {
+                const int tr = i >> 4, r = i & 15;
+                float a = 0.f;
+                for (int k = 0; k < p.K; ++k) {
+                    const int sl = tr * p.K + k;
+                    a = __fadd_rn(a, __fmul_rn(wt[sl], ys[sl * 16 + r]));
+                }
+                a = __fadd_rn(a, __fmul_rn(wt[PR + tr], ys[(PR + tr) * 16 + r]));
+                const size_t o = (size_t)tr * p.H + 16 * item + r;
+                if (p.residual) a = __fadd_rn(a, bf16_bits_to_f32(p.residual[o]));
+                p.out[o] = f32_to_bf16_bits(a);
+            }
+        }
+        named_barrier(1, kConsumerThreads);  // ys may be rewritten by the next item
     }
     if (threadIdx.x == 0) MOE_TRACE(2, 8);
 }
@@ -1132,40 +1465,84 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
     s.logits_ld = (E + 1 + 3) / 4 * 4;
     // activation rows per item: the 8 MMA columns, fewer for wide rows
     s.tok = (int)std::min<int64_t>({(int64_t)kDescPairs, rows, std::max(1, 16384 / H)});
-    // gate_up: 8..32 pairs (a power of two: divides I and Is), ~32 KB of weights per item
+    // gate_up: 8..32 pairs (a power of two: divides I and Is).  Items of
+    // ~32 KB of weights, grown to at most 64 KB while every SM still gets
+    // one: at small row counts a CTA's whole share is then in flight at once.
+    const int sms = std::max(1, device_info().sm_count);
+    const int64_t umax = std::min<int64_t>(E, rows * d.top_k);
+    auto gu_items = [&](int pr) { return (int64_t)(Is / pr) + umax * (I / pr); };
     int pairs = 8;
-    while (pairs * 2 <= 32 && pairs * 2 * 2 * H <= 32768) pairs *= 2;
+    while (pairs * 2 <= 32 && (pairs * 2 * 2 * H <= 32768 || (pairs * 2 * 2 * H <= 65536 && gu_items(pairs * 2) >= sms)))
+        pairs *= 2;
     s.gu_pairs = pairs;
     const size_t ws_g = (size_t)H + kRowPad;
     const size_t gu_stage = align16(16 * (pairs / 8) * ws_g + 2 * s.tok * ws_g + (size_t)s.tok * (H / 128) * 4 +
                                     (size_t)2 * (H / 128) * 4);
-    // down: 16..64 rows (a power of two: divides H and 128), ~32 KB of weights per item
-    int drows = 16;
-    while (drows * 2 <= 64 && drows * 2 * imax <= 32768) drows *= 2;
-    s.dn_rows = drows;
-    const size_t ws_d = (size_t)imax + kRowPad;
-    const size_t dn_stage = align16(drows * ws_d + (size_t)s.tok * imax * 4 + 2 * s.tok * ws_d +
-                                    (size_t)s.tok * (imax / 128) * 4 + (size_t)(imax / 128) * 4);
     const size_t plan = plan_bytes(E, (int)(rows * d.top_k));
-    const size_t gu_extra = red_bytes(pairs / 8) + plan, dn_extra = red_bytes(drows / 16) + plan;
+    const size_t gu_extra = red_bytes(pairs / 8) + plan;
+    const size_t ws_d = (size_t)imax + kRowPad;
     // One gate_up and one down CTA share an SM when they fit (down fetches
     // its weights while gate_up streams); gate_up, with two thirds of the
-    // bytes, gets the deeper ring.  Else each has the SM alone.
+    // bytes, gets the deeper ring; down takes smaller items (16..64 rows, a
+    // power of two dividing H, ~32 KB of weights) rather than fewer than
+    // two stages.  Else each has the SM alone.
     const size_t budget = 224 * 1024 - 2048;
-    int gs = kMaxStages, ds = 3;
-    auto total = [&] { return gs * gu_stage + gu_extra + ds * dn_stage + dn_extra; };
-    while (total() > budget && ds > 2) --ds;
-    while (total() > budget && gs > 2) --gs;
-    while (total() > budget && ds > 1) --ds;
-    while (total() > budget && gs > 1) --gs;
-    if (total() > budget) {
-        gs = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - gu_extra) / gu_stage));
-        ds = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - dn_extra) / dn_stage));
+    int drows_max = 16;
+    while (drows_max * 2 <= 64 && drows_max * 2 * imax <= 32768) drows_max *= 2;
+    const int64_t gu_per_cta = (gu_items(pairs) + sms - 1) / sms;
+    int gs = 1, ds = 1, drows = drows_max;
+    size_t dn_stage = 0, dn_extra = 0;
+    for (drows = drows_max;; drows /= 2) {
+        dn_stage = align16(drows * ws_d + (size_t)s.tok * imax * 4 + 2 * s.tok * ws_d +
+                           (size_t)s.tok * (imax / 128) * 4 + (size_t)(imax / 128) * 4);
+        dn_extra = dn_red_bytes(drows / 16, imax / 128) + plan;
+        const int64_t dn_per_cta = ((umax + 1) * (H / drows) + sms - 1) / sms;
+        auto total = [&] { return gs * gu_stage + gu_extra + ds * dn_stage + dn_extra; };
+        gs = (int)std::min<int64_t>(std::max<int64_t>(gu_per_cta, 2), kMaxStages);
+        ds = 2;
+        while (total() > budget && gs > 2) --gs;
+        if (total() <= budget) {
+            while (ds < std::min<int64_t>(kMaxStages, dn_per_cta) && total() + dn_stage <= budget) ++ds;
+            break;
+        }
+        if (drows == 16) {
+            while (total() > budget && ds > 1) --ds;
+            while (total() > budget && gs > 1) --gs;
+            if (total() > budget) {
+                gs = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - gu_extra) / gu_stage));
+                ds = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - dn_extra) / dn_stage));
+            }
+            break;
+        }
     }
+    s.dn_rows = drows;
     s.gu_stages = gs;
     s.dn_stages = ds;
     s.gu_smem = gs * gu_stage + gu_extra;
     s.dn_smem = ds * dn_stage + dn_extra;
+    s.ds_ue = 0;
+    // Few rows: the down product by output block (one CTA item = 16 output
+    // rows of every active expert, two stages of up to all of them), when it
+    // fits; gate_up then has the SM to itself and warms L2 with the down
+    // weights instead.
+    if (rows <= kDescPairs) {
+        const int u1 = (int)umax + 1;
+        for (int ue = u1; ue >= 1; --ue) {
+            const DsLayout Ls = ds_layout(d.top_k, I, Is, (int)rows, ue, 2);
+            const size_t need = Ls.plan + plan + 1024;  // + alignment slack (1024-byte TMA boxes)
+            if (need <= budget) {
+                s.ds_ue = ue;
+                s.dn_stages = 2;
+                s.dn_smem = need;
+                s.dn_rows = 16;
+                gs = (int)std::min<int64_t>(std::max<int64_t>(gu_per_cta, 1), kMaxStages);
+                while (gs > 1 && gs * gu_stage + gu_extra > budget) --gs;
+                s.gu_stages = gs;
+                s.gu_smem = gs * gu_stage + gu_extra;
+                break;
+            }
+        }
+    }
     return s;
 }
 
@@ -1241,6 +1618,8 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
     // gate_up
     {
         p.stages = sh.gu_stages;
+        p.ue = 0;
+        p.l2_w2 = sh.ds_ue > 0 ? 1 : 0;
         void (*kern)(ExpertParams) = sh.gu_pairs == 8    ? gate_up_kernel<1>
                                      : sh.gu_pairs == 16 ? gate_up_kernel<2>
                                                          : gate_up_kernel<4>;
@@ -1252,6 +1631,21 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
         if (e != cudaSuccess) return e;
     }
     // down + blend
+    if (sh.ds_ue > 0) {
+        p.stages = sh.dn_stages;
+        p.ue = sh.ds_ue;
+        DsParams dp;
+        dp.p = p;
+        const int H = d.hidden, I = d.inter, Is = d.shared_inter;
+        if (!make_map(&dp.w2r, a.expert_w8 + (size_t)2 * I * H, (uint64_t)I, (uint64_t)H, (uint64_t)d.n_experts,
+                      (uint64_t)I, 3 * (uint64_t)I * H, 16) ||
+            !make_map(&dp.w2s, a.shared_w8 + (size_t)2 * Is * H, (uint64_t)Is, (uint64_t)H, 1, (uint64_t)Is, 0, 16))
+            return cudaErrorInvalidValue;
+        const int bps = occupancy(down_small_kernel, kExpThreads, sh.dn_smem);
+        if (bps < 1) return cudaErrorInvalidConfiguration;
+        const int grid = std::min(d.hidden / 16, di.sm_count);
+        return launch_kernel(down_small_kernel, dim3(grid), dim3(kExpThreads), sh.dn_smem, s, dp);
+    }
     {
         p.stages = sh.dn_stages;
         void (*kern)(ExpertParams) = sh.dn_rows == 16   ? down_blend_kernel<1>

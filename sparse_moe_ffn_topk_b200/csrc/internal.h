@@ -35,6 +35,8 @@ struct DecodeShape {
     size_t gu_smem;
     int dn_rows, dn_stages;
     size_t dn_smem;
+    // down by output block (few rows): experts per stage; 0 = the item-based down kernel
+    int ds_ue;
 };
 DecodeShape decode_shape(const moe_dims &d, int64_t rows);
 

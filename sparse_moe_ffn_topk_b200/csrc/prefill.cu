@@ -821,8 +821,6 @@ __global__ void __launch_bounds__(256) blend_kernel(BlendParams p)
 
 // ------------------------------------------------------------ host side
 
-namespace {
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -857,6 +855,8 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, u
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <typename P>
 int gemm_occupancy_once(void (*kernel)(P), size_t smem = kGemmSmem)

@@ -134,6 +134,11 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// A byte tensor [outer][rows][inner] (inner contiguous) as a TMA map with
+// 128-byte-swizzled boxes of [128 bytes, box_rows, 1] (prefill.cu).
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t outer, uint64_t row_stride,
+              uint64_t outer_stride, uint32_t box_rows);
+
 __device__ __forceinline__ uint64_t policy_evict_last()
 {
     uint64_t p;
