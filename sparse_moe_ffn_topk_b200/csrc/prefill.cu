@@ -173,10 +173,23 @@ __global__ void __launch_bounds__(1024) scan_kernel(PlanParams p)
     if (threadIdx.x == 0) p.mtiles[0] = make_int4(run_tiles + smt, run_tiles, 0, 0);
 }
 
-// A warp per GEMM row: routed pair i < T*k takes its token's x row into its
-// expert's rows; row T*k + t takes token t's row for the shared expert.  Rows
-// are stored as hi/lo e4m3 (hi codes [H], then lo codes [H]) with one scale
-// per 128 block, amax / 448: x ~ s * (hi + lo).
+// A warp per token: its x row is quantised once to hi/lo e4m3 (hi codes [H],
+// then lo codes [H]) with one scale per 128 block, amax / 448 (x ~ s * (hi +
+// lo)), and written to each of its k expert rows and to its row of the
+// shared expert; each routed pair's position and blend weight are recorded.
+// Rows of up to kPermMaxBlocks * 128 elements keep their codes in
+// registers; wider rows quantise again for each destination.
+constexpr int kPermMaxBlocks = 32;
+
+__device__ __forceinline__ void permute_write(const PlanParams &p, int dst_row, int dst_scale, int kb, int lane,
+                                              uint32_t hi, uint32_t lo, float sc)
+{
+    uint32_t *dq = reinterpret_cast<uint32_t *>(p.xp + (size_t)dst_row * 2 * p.H);
+    dq[kb * 32 + lane] = hi;
+    dq[p.H / 4 + kb * 32 + lane] = lo;
+    if (lane == 0) p.xps[(size_t)dst_scale * (p.H / 128) + kb] = sc;
+}
+
 __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
 {
     pdl_wait();
@@ -186,35 +199,52 @@ __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
     const int hb = p.H / 128;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
-    for (int i = gw; i < P + p.T; i += nw) {
-        int t, dst, xrow;
-        if (i < P) {
-            t = i / p.K;
+    for (int t = gw; t < p.T; t += nw) {
+        // destinations: k routed rows, then the shared row
+        int dst[kMaxTopK + 1];
+        for (int r = 0; r < p.K; ++r) {
+            const int i = t * p.K + r;
             const int e = min(max(p.topk_idx[i], 0), p.E - 1);
-            dst = p.offsets[e] + p.rank[i];
-            xrow = dst;
+            dst[r] = p.offsets[e] + p.rank[i];
             if (lane == 0) {
-                p.pos[i] = dst;
-                p.slot_w[dst] = p.topk_w[i];
+                p.pos[i] = dst[r];
+                p.slot_w[dst[r]] = p.topk_w[i];
+            }
+        }
+        if (lane == 0) p.slot_w[P + t] = p.gsig[t];
+        const uint2 *src = reinterpret_cast<const uint2 *>(p.x + (size_t)t * p.H);
+        if (hb <= kPermMaxBlocks) {
+            uint32_t hi[kPermMaxBlocks], lo[kPermMaxBlocks];
+            float scv[kPermMaxBlocks];
+#pragma unroll
+            for (int kb = 0; kb < kPermMaxBlocks; ++kb) {
+                if (kb >= hb) break;
+                const uint2 raw = __ldg(src + kb * 32 + lane);
+                const float4 v = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+                const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                scv[kb] = amax > 0.f ? amax / 448.f : 1.f;
+                quant4_hilo(v, 1.f / scv[kb], hi[kb], lo[kb]);
+            }
+            for (int r = 0; r <= p.K; ++r) {
+                const int row = r < p.K ? dst[r] : p.xp_shared0 + t;
+                const int srow = r < p.K ? dst[r] : P + t;
+#pragma unroll
+                for (int kb = 0; kb < kPermMaxBlocks; ++kb) {
+                    if (kb >= hb) break;
+                    permute_write(p, row, srow, kb, lane, hi[kb], lo[kb], scv[kb]);
+                }
             }
         } else {
-            t = i - P;
-            dst = i;
-            xrow = p.xp_shared0 + t;
-            if (lane == 0) p.slot_w[i] = p.gsig[t];
-        }
-        const uint2 *src = reinterpret_cast<const uint2 *>(p.x + (size_t)t * p.H);
-        uint32_t *dq = reinterpret_cast<uint32_t *>(p.xp + (size_t)xrow * 2 * p.H);
-        for (int kb = 0; kb < hb; ++kb) {
-            const uint2 raw = __ldg(src + kb * 32 + lane);
-            const float4 v = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
-            const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-            const float sc = amax > 0.f ? amax / 448.f : 1.f;
-            uint32_t hi, lo;
-            quant4_hilo(v, 1.f / sc, hi, lo);
-            dq[kb * 32 + lane] = hi;
-            dq[p.H / 4 + kb * 32 + lane] = lo;
-            if (lane == 0) p.xps[(size_t)dst * hb + kb] = sc;
+            for (int kb = 0; kb < hb; ++kb) {
+                const uint2 raw = __ldg(src + kb * 32 + lane);
+                const float4 v = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+                const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                const float sc = amax > 0.f ? amax / 448.f : 1.f;
+                uint32_t h, l;
+                quant4_hilo(v, 1.f / sc, h, l);
+                for (int r = 0; r <= p.K; ++r)
+                    permute_write(p, r < p.K ? dst[r] : p.xp_shared0 + t, r < p.K ? dst[r] : P + t, kb, lane, h, l, sc);
+            }
         }
     }
 }
@@ -650,6 +680,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 128; ++i) tot[i] = 0.f;
             bool ok = true;
+            // the row's blend weight (GEMM2) is needed only at the tile's end: load it now
+            const float w_row = (MODE == 2 && valid) ? __ldg(p.slot_w + (size_t)ti.row0 + r) : 0.f;
             // scales one K block ahead, so their loads overlap the wait for the accumulator
             float sa_n = valid ? __ldg(asc) : 0.f;
             float s0_n = __ldg(wsc + (size_t)wn0 * wld), s1_n = __ldg(wsc + (size_t)wn1 * wld);
@@ -702,7 +734,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
                     const float g = tot[i], u = tot[64 + i];
-                    const float hv = g / (1.f + __expf(-g)) * u;
+                    const float hv = g * __frcp_rn(1.f + __expf(-g)) * u;
                     tot[i] = hv;
                     amax = fmaxf(amax, fabsf(hv));
                 }
@@ -714,21 +746,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 const float sc = amax > 0.f ? amax / 448.f : 1.f;
                 const float inv = 1.f / sc;
                 if (ok) {
-                    // hi, then lo: this warp's 32 rows x 64 bytes go through its staging
-                    // buffer, then out as 64-byte row segments, 16 bytes per lane
+                    // quantise once: hi words to the staging buffer, lo words kept in
+                    // the registers the up half of tot no longer needs; each part
+                    // leaves as 64-byte row segments, 16 bytes per lane
                     uint4 *srow = reinterpret_cast<uint4 *>(stg + lane * 80);
+                    uint32_t low[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int c = 16 * i + 4 * j;
+                            quant4_hilo(make_float4(tot[c], tot[c + 1], tot[c + 2], tot[c + 3]), inv, w4[j], low[4 * i + j]);
+                        }
+                        srow[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
                     for (int part = 0; part < 2; ++part) {
+                        if (part == 1) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int c = 16 * i + 4 * j;
-                                uint32_t h4, l4;
-                                quant4_hilo(make_float4(tot[c], tot[c + 1], tot[c + 2], tot[c + 3]), inv, h4, l4);
-                                w4[j] = part ? l4 : h4;
-                            }
-                            srow[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            for (int i = 0; i < 4; ++i) srow[i] = make_uint4(low[4 * i], low[4 * i + 1], low[4 * i + 2], low[4 * i + 3]);
                         }
                         __syncwarp();
 #pragma unroll
@@ -749,7 +785,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 if (ok) {
                     // 16 columns at a time through the staging buffer (rows of 17
                     // floats), then out as 64-byte row segments, 16 bytes per lane
-                    const float w = valid ? __ldg(p.slot_w + (size_t)ti.row0 + r) : 0.f;
+                    const float w = w_row;
                     float *sf = reinterpret_cast<float *>(stg);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -954,7 +990,7 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
 
     // 2, 3
     if ((e = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pp)) != cudaSuccess) return MOE_ECUDA;
-    if ((e = launch_kernel(permute_kernel, dim3(std::max(1, std::min(8 * di.sm_count, (P + T + 7) / 8))), dim3(256),
+    if ((e = launch_kernel(permute_kernel, dim3(std::max(1, std::min(8 * di.sm_count, (T + 7) / 8))), dim3(256),
                            0, s, pp)) != cudaSuccess)
         return MOE_ECUDA;
 
