@@ -38,13 +38,14 @@ constexpr int kBM = 128;     // rows per M tile
 constexpr int kBN = 256;     // accumulator columns per tile
 constexpr int kBK = 128;     // K bytes per stage (one scale block of e4m3)
 constexpr int kGemmStages = 3;
-constexpr int kGemmThreads = 320;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2..9: epilogue
-constexpr int kEpiThreads = 256;
+constexpr int kEpiWarps = 16;
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2..17: epilogue
+constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 accumulators
 constexpr size_t kStageBytes = 2 * kBM * kBK + kBN * kBK;  // A hi, A lo, B
-constexpr int kStgBytes = 32 * 80;  // per epilogue warp: 32 rows x 80 B staging for coalesced stores
+constexpr int kStgBytes = 32 * 48;  // per epilogue warp: 32 rows x 48 B staging for coalesced stores
 constexpr size_t kGemmSmem =
-    kGemmStages * kStageBytes + 1024 /* alignment slack */ + 4096 /* amax exchange */ + 8 * kStgBytes;
+    kGemmStages * kStageBytes + 1024 /* alignment slack */ + 4096 /* amax exchange */ + kEpiWarps * kStgBytes;
 
 // ------------------------------------------------------------ layout
 
@@ -301,9 +302,11 @@ __global__ void __launch_bounds__(kRtThreads, 1) router_tc_kernel(const __grid_c
     __shared__ __align__(8) uint64_t full[kRtStages], empty[kRtStages], acc_full, acc_empty;
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int s_abort;
+    __shared__ float s_bias[kMaxExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
 
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_bias[e] = p.bias ? __ldg(p.bias + e) : 0.f;
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int s = 0; s < kRtStages; ++s) {
@@ -423,14 +426,15 @@ __global__ void __launch_bounds__(kRtThreads, 1) router_tc_kernel(const __grid_c
                     float v[32];
                     tmem_ld_32x32(tb + (uint32_t)c0, v);
                     tmem_wait_ld();
+                    uint32_t kk[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < 32; ++i) {  // keys first (independent), then the inserts
                         const int e = ps * kRtChunk + c0 + i;
-                        if (c0 + i < ncol) {
-                            const float l = v[i] + (p.bias ? __ldg(p.bias + e) : 0.f);
-                            topk_insert<KM>(keys, ids, topk_key(l), e);
-                        }
+                        kk[i] = (c0 + i < ncol) ? topk_key(v[i] + s_bias[min(e, p.E - 1)]) : 0u;
                     }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (kk[i] > keys[KM - 1]) topk_insert<KM>(keys, ids, kk[i], ps * kRtChunk + c0 + i);
                 }
                 if (ps == 0) {
                     float v[32];
@@ -457,10 +461,23 @@ __global__ void __launch_bounds__(kRtThreads, 1) router_tc_kernel(const __grid_c
                     if (j < p.K) {
                         p.topk_idx[(size_t)t * p.K + j] = ids[j];
                         p.topk_w[(size_t)t * p.K + j] = ev[j] / sum;
-                        p.rank[(size_t)t * p.K + j] = atomicAdd(&p.counts[ids[j]], 1);
                     }
                 }
                 p.gsig[t] = sigmoidf_(z);
+            }
+            // each pair's rank within its expert: one atomic per group of lanes
+            // that picked the same expert at the same rank position
+            const unsigned live = __ballot_sync(0xFFFFFFFFu, t < p.T);
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                if (j < p.K && t < p.T) {
+                    const unsigned grp = __match_any_sync(live, ids[j]);
+                    const int leader = __ffs(grp) - 1;
+                    int base = 0;
+                    if (lane == leader) base = atomicAdd(&p.counts[ids[j]], __popc(grp));
+                    base = __shfl_sync(grp, base, leader);
+                    p.rank[(size_t)t * p.K + j] = base + __popc(grp & ((1u << lane) - 1));
+                }
             }
         }
     }
@@ -535,7 +552,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     __shared__ volatile int s_abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    float *epi_scratch = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes);  // [2][128] amax exchange
+    float *epi_scratch = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes);  // [4][128] amax exchange
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -645,12 +662,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             }
         }
     } else {
-        // --------------------------------------------------- epilogue (warps 2..9)
-        const int q = warp & 3;                   // TMEM lane quadrant of this warp
-        const int half = (warp - 2) >> 2;          // column half
+        // --------------------------------------------------- epilogue (warps 2..17)
+        // Warp w reads TMEM lanes 32 (w mod 4) .. +32 (its rows); the four warps
+        // of a lane quadrant split the columns in quarters.  GEMM1: quarter j
+        // holds gate columns [32 j, +32) and the matching up columns, so
+        // silu(gate) * up stays in the thread; GEMM2: columns [64 j, +64).
+        const int ew = warp - 2;
+        const int q = warp & 3;                    // TMEM lane quadrant of this warp
+        const int quarter = ew >> 2;               // column quarter
         const int r = q * 32 + lane;               // row within the tile
-        const int et = threadIdx.x - 64;           // 0..255
-        unsigned char *stg = smem + kGemmStages * kStageBytes + 4096 + (size_t)(warp - 2) * kStgBytes;
+        unsigned char *stg = smem + kGemmStages * kStageBytes + 4096 + (size_t)ew * kStgBytes;
         int acc_it = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
             TileInfo ti;
@@ -661,7 +682,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             const float *asc = (ti.shared_grp ? p.a_scales_shared : p.a_scales_routed) + (size_t)arow * p.a_scales_ld;
             const int inter = ti.shared_grp ? p.Is : p.I;
             const float *wsc;
-            int wld, wn0, wn1;  // scale rows of the tile's two column halves
+            int wld, wn0, wn1;  // the block-scale rows of this thread's columns (gate and up; or one)
             if (MODE == 1) {
                 wsc = ti.shared_grp ? p.w_scales_shared
                                     : p.w_scales + (size_t)ti.group * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128));
@@ -673,12 +694,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                                      : p.w_scales + (size_t)ti.group * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128))) +
                       (2 * inter / 128) * (p.H / 128);
                 wld = inter / 128;
-                wn0 = ti.nt * 2;
-                wn1 = ti.nt * 2 + 1;
+                wn0 = wn1 = ti.nt * 2 + (quarter >> 1);
             }
-            float tot[128];
+            float tot[64];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) tot[i] = 0.f;
+            for (int i = 0; i < 64; ++i) tot[i] = 0.f;
             bool ok = true;
             // the row's blend weight (GEMM2) is needed only at the tile's end: load it now
             const float w_row = (MODE == 2 && valid) ? __ldg(p.slot_w + (size_t)ti.row0 + r) : 0.f;
@@ -705,54 +725,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 if (!ok) continue;
                 tc_fence_after();
                 const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kBN);
-                // MODE 1: this thread's columns are [64 half, +64) (gate) and [128 + 64 half, +64) (up)
-                // MODE 2: [128 half, +128)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    int col;
-                    float sc;
-                    if (MODE == 1) {
-                        col = (c < 2) ? (64 * half + 32 * c) : (128 + 64 * half + 32 * (c - 2));
-                        sc = sa * ((c < 2) ? s0 : s1);
-                    } else {
-                        col = 128 * half + 32 * c;
-                        sc = sa * (half ? s1 : s0);
-                    }
-                    float v[32];
-                    tmem_ld_32x32(tbase + (uint32_t)col, v);
+                for (int c = 0; c < 4; ++c) {  // 16 columns at a time
+                    const int col = MODE == 1 ? ((c < 2) ? 32 * quarter + 16 * c : 128 + 32 * quarter + 16 * (c - 2))
+                                              : 64 * quarter + 16 * c;
+                    const float sc = sa * ((MODE == 1 && c >= 2) ? s1 : s0);
+                    float v[16];
+                    tmem_ld_32x16(tbase + (uint32_t)col, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) tot[32 * c + i] = fmaf(sc, v[i], tot[32 * c + i]);
+                    for (int i = 0; i < 16; ++i) tot[16 * c + i] = fmaf(sc, v[i], tot[16 * c + i]);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[b]);
             }
             if (MODE == 1) {
-                // h = silu(gate) * up for this thread's 64 columns of the block
+                // h = silu(gate) * up for this thread's 32 columns of the block
                 float amax = 0.f;
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float g = tot[i], u = tot[64 + i];
+                for (int i = 0; i < 32; ++i) {
+                    const float g = tot[i], u = tot[32 + i];
                     const float hv = g * __frcp_rn(1.f + __expf(-g)) * u;
                     tot[i] = hv;
                     amax = fmaxf(amax, fabsf(hv));
                 }
-                // both halves of the row's 128-column block share one scale
+                // the four quarters of the row's 128-column block share one scale
                 named_barrier(2, kEpiThreads);
-                epi_scratch[half * 128 + r] = amax;
+                epi_scratch[quarter * 128 + r] = amax;
                 named_barrier(2, kEpiThreads);
-                amax = fmaxf(epi_scratch[r], epi_scratch[128 + r]);
+                amax = fmaxf(fmaxf(epi_scratch[r], epi_scratch[128 + r]), fmaxf(epi_scratch[256 + r], epi_scratch[384 + r]));
                 const float sc = amax > 0.f ? amax / 448.f : 1.f;
                 const float inv = 1.f / sc;
                 if (ok) {
-                    // quantise once: hi words to the staging buffer, lo words kept in
-                    // the registers the up half of tot no longer needs; each part
-                    // leaves as 64-byte row segments, 16 bytes per lane
-                    uint4 *srow = reinterpret_cast<uint4 *>(stg + lane * 80);
-                    uint32_t low[16];
+                    // quantise once: hi words to the staging buffer, lo words in
+                    // registers; each part leaves as 32-byte row segments, 16 bytes
+                    // per lane
+                    uint4 *srow = reinterpret_cast<uint4 *>(stg + lane * 48);
+                    uint32_t low[8];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < 2; ++i) {
                         uint32_t w4[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
@@ -763,43 +775,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     }
                     for (int part = 0; part < 2; ++part) {
                         if (part == 1) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) srow[i] = make_uint4(low[4 * i], low[4 * i + 1], low[4 * i + 2], low[4 * i + 3]);
+                            srow[0] = make_uint4(low[0], low[1], low[2], low[3]);
+                            srow[1] = make_uint4(low[4], low[5], low[6], low[7]);
                         }
                         __syncwarp();
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int rr = 8 * i + (lane >> 2), ch = lane & 3;
-                            const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * 80 + ch * 16);
+                        for (int i = 0; i < 2; ++i) {
+                            const int rr = 16 * i + (lane >> 1), ch = lane & 1;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(stg + rr * 48 + ch * 16);
                             if (q * 32 + rr < ti.rows) {
                                 const size_t grow = (size_t)ti.row0 + q * 32 + rr;
                                 *reinterpret_cast<uint4 *>(p.hq + grow * 2 * p.imax + (part ? p.imax : 0) + ti.nt * 128 +
-                                                           64 * half + ch * 16) = v;
+                                                           32 * quarter + ch * 16) = v;
                             }
                         }
                         __syncwarp();
                     }
-                    if (valid && half == 0) p.hs[((size_t)ti.row0 + r) * (p.imax / 128) + ti.nt] = sc;
+                    if (valid && quarter == 0) p.hs[((size_t)ti.row0 + r) * (p.imax / 128) + ti.nt] = sc;
                 }
             } else {
                 if (ok) {
-                    // 16 columns at a time through the staging buffer (rows of 17
-                    // floats), then out as 64-byte row segments, 16 bytes per lane
-                    const float w = w_row;
+                    // 8 columns at a time through the staging buffer (rows of 9
+                    // floats), then out as 32-byte row segments, 16 bytes per lane
                     float *sf = reinterpret_cast<float *>(stg);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) sf[lane * 17 + j] = w * tot[16 * c + j];
+                        for (int j = 0; j < 8; ++j) sf[lane * 9 + j] = w_row * tot[8 * c + j];
                         __syncwarp();
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int rr = 8 * i + (lane >> 2), ch = lane & 3;
-                            const float *src = sf + rr * 17 + ch * 4;
+                        for (int i = 0; i < 2; ++i) {
+                            const int rr = 16 * i + (lane >> 1), ch = lane & 1;
+                            const float *src = sf + rr * 9 + ch * 4;
                             const float4 v = make_float4(src[0], src[1], src[2], src[3]);
                             if (q * 32 + rr < ti.rows) {
                                 const size_t grow = (size_t)ti.row0 + q * 32 + rr;
-                                *reinterpret_cast<float4 *>(p.yslot + grow * p.H + ti.nt * kBN + 128 * half + 16 * c +
+                                *reinterpret_cast<float4 *>(p.yslot + grow * p.H + ti.nt * kBN + 64 * quarter + 8 * c +
                                                             4 * ch) = v;
                             }
                         }
@@ -807,7 +818,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     }
                 }
             }
-            (void)et;
         }
     }
     tc_fence_before();
