@@ -57,6 +57,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true", help="skip the rows=64 and per-kernel legs")
+    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
+                    help="a small case for a profiler: a few eager layer calls on one weight copy, then exit")
+    ap.add_argument("--calls", type=int, default=4, help="layer calls of --profile")
     return ap.parse_args(argv)
 
 
@@ -701,8 +704,37 @@ def run_reference(args, dist: Dist):
     }
 
 
+def run_profile_case(args):
+    """A few eager calls of one workload (35B-shaped layer, one weight copy):
+    decode at rows = 1 on fresh x each call, or the 4096-token biased
+    prefill.  Small enough for a profiler to replay every kernel."""
+    import torch
+
+    import moe_inputs as mi
+    import sparse_moe_ffn_topk_b200 as moe
+    d = mi.QWEN36_35B_A3B
+    inst = make_instances(mi.make_layer(d, seed=args.seed), 1)[0]
+    if args.profile == "decode":
+        rows, bias, path = 1, None, moe.MOE_PATH_AUTO
+    else:
+        rows, path = 4096, moe.MOE_PATH_PREFILL
+        bias = torch.from_numpy(mi.make_router(d, args.seed, True)[2]).cuda()
+    ws = moe.alloc_workspace(d, rows)
+    out = torch.empty(rows, d.hidden, dtype=torch.bfloat16, device="cuda")
+    for i in range(args.calls):
+        x = torch.from_numpy(mi.make_x(d, rows, seed=args.seed + 5, stream=i).view("int16")).view(torch.bfloat16).cuda()
+        moe.ffn_forward_path(d, x, inst["router_w"], inst["expert_w8"], inst["expert_scales"], inst["shared_w8"],
+                             inst["shared_scales"], inst["shared_gate"], out, ws, path=path, router_bias=bias)
+    torch.cuda.synchronize()
+    st = moe.device_status(ws)
+    print(json.dumps({"profile": args.profile, "calls": args.calls, "rows": rows, "device_status": st}), flush=True)
+    return 0 if st == moe.MOE_OK else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.profile:
+        return run_profile_case(args)
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -1472,7 +1472,8 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
     const int64_t umax = std::min<int64_t>(E, rows * d.top_k);
     auto gu_items = [&](int pr) { return (int64_t)(Is / pr) + umax * (I / pr); };
     int pairs = 8;
-    while (pairs * 2 <= 32 && (pairs * 2 * 2 * H <= 32768 || (pairs * 2 * 2 * H <= 65536 && gu_items(pairs * 2) >= sms)))
+    while (pairs * 2 <= 32 &&
+           (pairs * 2 * 2 * H <= 32768 || (s.tok <= 2 && pairs * 2 * 2 * H <= 65536 && gu_items(pairs * 2) >= sms)))
         pairs *= 2;
     s.gu_pairs = pairs;
     const size_t ws_g = (size_t)H + kRowPad;
@@ -1501,6 +1502,7 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
         gs = (int)std::min<int64_t>(std::max<int64_t>(gu_per_cta, 2), kMaxStages);
         ds = 2;
         while (total() > budget && gs > 2) --gs;
+        if (total() > budget) ds = 1;  // fewer, larger down items beat more, smaller ones
         if (total() <= budget) {
             while (ds < std::min<int64_t>(kMaxStages, dn_per_cta) && total() + dn_stage <= budget) ++ds;
             break;
