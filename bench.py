@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
                     help="a small case for a profiler: a few eager layer calls on one weight copy, then exit")
     ap.add_argument("--calls", type=int, default=4, help="layer calls of --profile")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every decode workload (35B rows 1..64, 397B rows 1 and 32) and print one JSON line")
     return ap.parse_args(argv)
 
 
@@ -704,6 +706,41 @@ def run_reference(args, dist: Dist):
     }
 
 
+def run_sweep(args, dist: Dist):
+    """Decode at every row count of the workloads: 35B-A3B-shaped rows 1, 2,
+    8, 16, 32, 64 (16 weight copies) and 397B-A17B-shaped rows 1 and 32 (two
+    6.4 GB copies); CUDA events over CUDA-graph replays, as the headline."""
+    import torch
+
+    import moe_inputs as mi
+    torch.cuda.set_device(dist.local)
+    hbm_peak, _, peak_kind = peaks()
+    res = []
+    for dims, name, rows_list, n_inst in ((mi.QWEN36_35B_A3B, "Qwen3.6-35B-A3B-shaped", [1, 2, 8, 16, 32, 64], 16),
+                                          (mi.QWEN35_397B_A17B, "Qwen3.5-397B-A17B-shaped", [1, 32], 2)):
+        insts = make_instances(mi.make_layer(dims, seed=args.seed), n_inst)
+        for rows in rows_list:
+            xs = [torch.from_numpy(mi.make_x(dims, rows, seed=args.seed + 1, stream=1000 * rows + i).view("int16"))
+                  .view(torch.bfloat16).cuda() for i in range(16)]
+            b = DecodeBench(dims, insts, xs, rows)
+            u = statistics.mean(b.routing(16))
+            by = algorithmic_bytes(dims, rows, u)
+            k = max(50, min(args.steps, 4000 // rows))
+            ms, _ = b.time_steps(k, max(3, args.warmup), dist)
+            sec = dist.max(ms / 1000.0)
+            gbs = aggregate(k * by["total"], dist.world, sec) / 1e9
+            res.append({"workload": f"{name} decode rows={rows}", "us_per_layer": round(sec * 1e6 / k, 3),
+                        "gb_s": round(gbs, 1), "hbm_frac_of_measured": round(gbs / dist.world / hbm_peak, 4),
+                        "tokens_per_s": round(aggregate(k * rows, dist.world, sec), 1),
+                        "distinct_experts": round(u, 1), "bytes_per_step": int(by["total"]), "steps": k})
+            print(f"[sweep] {res[-1]['workload']}: {res[-1]['us_per_layer']} us, {gbs:.0f} GB/s", file=sys.stderr,
+                  flush=True)
+            del b
+        del insts
+        torch.cuda.empty_cache()
+    return {"sweep": res, "peak_source": f"{peak_kind} ({hbm_peak} GB/s copy)", "n_gpus": dist.world}
+
+
 def run_profile_case(args):
     """A few eager calls of one workload (35B-shaped layer, one weight copy):
     decode at rows = 1 on fresh x each call, or the 4096-token biased
@@ -745,7 +782,7 @@ def main(argv=None):
         return 0
     dist = Dist(args.gpus)
     try:
-        res = run_ours(args, dist)
+        res = run_sweep(args, dist) if args.sweep else run_ours(args, dist)
         if dist.rank == 0:
             print(json.dumps(res), flush=True)
     finally:

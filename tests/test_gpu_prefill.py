@@ -76,3 +76,28 @@ def test_qwen36_35b_prefill_4096_rows_sampled():
     sample = np.random.default_rng(0).choice(rows, 48, replace=False)
     sub = P.Case(d, case.layer, case.x[sample].copy(), case.logits[sample])
     P.compare_output(sub, out[sample], idx[sample])
+
+
+def test_prefill_router_more_than_256_experts():
+    # the router takes the experts in passes of 256 accumulator columns
+    d = mi.LayerDims(hidden=256, n_experts=300, top_k=5, inter=128, shared_inter=128)
+    case = P.build_case(d, 130, router_bias=True, residual=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
+
+
+def test_qwen35_397b_prefill_sampled():
+    # 512 experts (two router passes), top-10, I = Is = 1024, uneven loads
+    d = mi.QWEN35_397B_A17B
+    rows = 96
+    case = P.build_case(d, rows, router_bias=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    sample = np.random.default_rng(1).choice(rows, 16, replace=False)
+    sub = P.Case(d, case.layer, case.x[sample].copy(), case.logits[sample])
+    P.compare_output(sub, out[sample], idx[sample])
