@@ -609,7 +609,7 @@ __device__ void prefetch_down_weights(const ExpertParams &p, const LocalPlan &lp
 }
 
 template <int T>
-__global__ void __launch_bounds__(kExpThreads, 2) gate_up_kernel(ExpertParams p)
+__global__ void __launch_bounds__(kExpThreads, 1) gate_up_kernel(ExpertParams p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
@@ -873,7 +873,7 @@ __device__ void dn_produce(const ExpertParams &p, const DnLayout &L, StageDesc &
 }
 
 template <int T>
-__global__ void __launch_bounds__(kExpThreads, 2) down_blend_kernel(ExpertParams p)
+__global__ void __launch_bounds__(kExpThreads, 1) down_blend_kernel(ExpertParams p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
@@ -1465,59 +1465,45 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
     s.logits_ld = (E + 1 + 3) / 4 * 4;
     // activation rows per item: the 8 MMA columns, fewer for wide rows
     s.tok = (int)std::min<int64_t>({(int64_t)kDescPairs, rows, std::max(1, 16384 / H)});
-    // gate_up: 8..32 pairs (a power of two: divides I and Is).  Items of
-    // ~32 KB of weights, grown to at most 64 KB while every SM still gets
-    // one: at small row counts a CTA's whole share is then in flight at once.
+    // Each expert kernel has an SM to itself (measured: deeper rings of larger
+    // items beat sharing an SM between a gate_up and a down CTA).
+    const size_t budget = 224 * 1024 - 2048;
     const int sms = std::max(1, device_info().sm_count);
     const int64_t umax = std::min<int64_t>(E, rows * d.top_k);
+    const size_t plan = plan_bytes(E, (int)(rows * d.top_k));
+    const size_t ws_g = (size_t)H + kRowPad;
+    auto gu_stage_of = [&](int pr) {
+        return align16(16 * (pr / 8) * ws_g + 2 * s.tok * ws_g + (size_t)s.tok * (H / 128) * 4 + (size_t)2 * (H / 128) * 4);
+    };
     auto gu_items = [&](int pr) { return (int64_t)(Is / pr) + umax * (I / pr); };
+    // gate_up: 8..32 gate/up row pairs per item (a power of two: divides I and
+    // Is); grown while an item stays <= 64 KB of weights, two stages fit and
+    // every SM still gets an item
     int pairs = 8;
-    while (pairs * 2 <= 32 &&
-           (pairs * 2 * 2 * H <= 32768 || (s.tok <= 2 && pairs * 2 * 2 * H <= 65536 && gu_items(pairs * 2) >= sms)))
+    while (pairs * 2 <= 32 && pairs * 2 * 2 * H <= 65536 && gu_items(pairs * 2) >= sms &&
+           2 * gu_stage_of(pairs * 2) + red_bytes(pairs * 2 / 8) + plan <= budget)
         pairs *= 2;
     s.gu_pairs = pairs;
-    const size_t ws_g = (size_t)H + kRowPad;
-    const size_t gu_stage = align16(16 * (pairs / 8) * ws_g + 2 * s.tok * ws_g + (size_t)s.tok * (H / 128) * 4 +
-                                    (size_t)2 * (H / 128) * 4);
-    const size_t plan = plan_bytes(E, (int)(rows * d.top_k));
+    const size_t gu_stage = gu_stage_of(pairs);
     const size_t gu_extra = red_bytes(pairs / 8) + plan;
-    const size_t ws_d = (size_t)imax + kRowPad;
-    // One gate_up and one down CTA share an SM when they fit (down fetches
-    // its weights while gate_up streams); gate_up, with two thirds of the
-    // bytes, gets the deeper ring; down takes smaller items (16..64 rows, a
-    // power of two dividing H, ~32 KB of weights) rather than fewer than
-    // two stages.  Else each has the SM alone.
-    const size_t budget = 224 * 1024 - 2048;
-    int drows_max = 16;
-    while (drows_max * 2 <= 64 && drows_max * 2 * imax <= 32768) drows_max *= 2;
     const int64_t gu_per_cta = (gu_items(pairs) + sms - 1) / sms;
-    int gs = 1, ds = 1, drows = drows_max;
-    size_t dn_stage = 0, dn_extra = 0;
-    for (drows = drows_max;; drows /= 2) {
-        dn_stage = align16(drows * ws_d + (size_t)s.tok * imax * 4 + 2 * s.tok * ws_d +
-                           (size_t)s.tok * (imax / 128) * 4 + (size_t)(imax / 128) * 4);
-        dn_extra = dn_red_bytes(drows / 16, imax / 128) + plan;
-        const int64_t dn_per_cta = ((umax + 1) * (H / drows) + sms - 1) / sms;
-        auto total = [&] { return gs * gu_stage + gu_extra + ds * dn_stage + dn_extra; };
-        gs = (int)std::min<int64_t>(std::max<int64_t>(gu_per_cta, 2), kMaxStages);
-        ds = 2;
-        while (total() > budget && gs > 2) --gs;
-        if (total() > budget) ds = 1;  // fewer, larger down items beat more, smaller ones
-        if (total() <= budget) {
-            while (ds < std::min<int64_t>(kMaxStages, dn_per_cta) && total() + dn_stage <= budget) ++ds;
-            break;
-        }
-        if (drows == 16) {
-            while (total() > budget && ds > 1) --ds;
-            while (total() > budget && gs > 1) --gs;
-            if (total() > budget) {
-                gs = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - gu_extra) / gu_stage));
-                ds = (int)std::max<size_t>(1, std::min<size_t>(kMaxStages, (budget - dn_extra) / dn_stage));
-            }
-            break;
-        }
-    }
+    int gs = (int)std::min<int64_t>(std::max<int64_t>(gu_per_cta, 2), kMaxStages);
+    while (gs > 1 && gs * gu_stage + gu_extra > budget) --gs;
+    // down (item kernel): rows per item 16..64 (a power of two dividing H and
+    // 128), ~32 KB of weights; as many stages as fit
+    const size_t ws_d = (size_t)imax + kRowPad;
+    int drows = 16;
+    while (drows * 2 <= 64 && drows * 2 * imax <= 32768) drows *= 2;
+    const size_t dn_stage = align16(drows * ws_d + (size_t)s.tok * imax * 4 + 2 * s.tok * ws_d +
+                                    (size_t)s.tok * (imax / 128) * 4 + (size_t)(imax / 128) * 4);
+    const size_t dn_extra = dn_red_bytes(drows / 16, imax / 128) + plan;
+    const int64_t dn_per_cta = ((umax + 1) * (H / drows) + sms - 1) / sms;
+    int ds = (int)std::min<int64_t>(std::max<int64_t>(dn_per_cta, 2), kMaxStages);
+    while (ds > 1 && ds * dn_stage + dn_extra > budget) --ds;
     s.dn_rows = drows;
+    // gate_up warms L2 with the active experts' down weights when they take
+    // a small part of it
+    s.l2_w2 = (umax * (int64_t)I * H + (int64_t)Is * H) <= (int64_t)48 << 20;
     s.gu_stages = gs;
     s.dn_stages = ds;
     s.gu_smem = gs * gu_stage + gu_extra;
@@ -1537,10 +1523,7 @@ DecodeShape decode_shape(const moe_dims &d, int64_t rows)
                 s.dn_stages = 2;
                 s.dn_smem = need;
                 s.dn_rows = 16;
-                gs = (int)std::min<int64_t>(std::max<int64_t>(gu_per_cta, 1), kMaxStages);
-                while (gs > 1 && gs * gu_stage + gu_extra > budget) --gs;
-                s.gu_stages = gs;
-                s.gu_smem = gs * gu_stage + gu_extra;
+                s.l2_w2 = true;
                 break;
             }
         }
@@ -1621,7 +1604,7 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
     {
         p.stages = sh.gu_stages;
         p.ue = 0;
-        p.l2_w2 = sh.ds_ue > 0 ? 1 : 0;
+        p.l2_w2 = sh.l2_w2 ? 1 : 0;
         void (*kern)(ExpertParams) = sh.gu_pairs == 8    ? gate_up_kernel<1>
                                      : sh.gu_pairs == 16 ? gate_up_kernel<2>
                                                          : gate_up_kernel<4>;

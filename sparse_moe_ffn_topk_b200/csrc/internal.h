@@ -37,6 +37,8 @@ struct DecodeShape {
     size_t dn_smem;
     // down by output block (few rows): experts per stage; 0 = the item-based down kernel
     int ds_ue;
+    // gate_up prefetches the active experts' down weights into L2
+    bool l2_w2;
 };
 DecodeShape decode_shape(const moe_dims &d, int64_t rows);
 
