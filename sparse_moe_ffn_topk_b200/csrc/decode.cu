@@ -128,20 +128,19 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v)
 // marks an absent expert and a NaN logit gets key 1, so every round picks a
 // valid expert even on non-finite input.
 template <int EPL>
-__device__ void topk_row(const RouterParams &p, int t)
+__device__ void topk_select(const float *lrow, int E, int K, int32_t *out_idx, float *out_w, float *out_gsig)
 {
     const int lane = threadIdx.x & 31;
-    const float *lrow = p.logits + (size_t)t * p.ld;
     uint32_t v[EPL];
     int id[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane * EPL + i;
-        const float l = (e < p.E) ? __ldcg(lrow + e) : 0.f;
-        v[i] = (e < p.E) ? topk_key(l) : 0u;
+        const float l = (e < E) ? __ldcg(lrow + e) : 0.f;
+        v[i] = (e < E) ? topk_key(l) : 0u;
         id[i] = e;
     }
-    const float z = __ldcg(lrow + p.E);
+    const float z = __ldcg(lrow + E);
     // odd-even transposition sort, descending; swaps only on a strict
     // inequality, so it is stable
 #pragma unroll
@@ -160,7 +159,7 @@ __device__ void topk_row(const RouterParams &p, int t)
     }
     int my_e = 0;
     uint32_t my_k = 0;
-    for (int r = 0; r < p.K; ++r) {
+    for (int r = 0; r < K; ++r) {
         const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, v[0]);
         const int wl = __ffs(__ballot_sync(0xFFFFFFFFu, v[0] == kmax)) - 1;
         const int ew = __shfl_sync(0xFFFFFFFFu, id[0], wl);
@@ -180,14 +179,22 @@ __device__ void topk_row(const RouterParams &p, int t)
     if (threadIdx.x == 0) MOE_TRACE(0, 5);
     const float my_v = (my_k == 1u) ? __int_as_float(0x7FC00000) : key_value(my_k);
     const float top = __shfl_sync(0xFFFFFFFFu, my_v, 0);
-    const float ev = (lane < p.K) ? expf(my_v - top) : 0.f;
+    const float ev = (lane < K) ? expf(my_v - top) : 0.f;
     const float sum = warp_sum(ev);
-    if (lane < p.K) {
-        p.topk_idx[(size_t)t * p.K + lane] = my_e;
-        p.topk_w[(size_t)t * p.K + lane] = ev / sum;
+    if (lane < K) {
+        out_idx[lane] = my_e;
+        out_w[lane] = ev / sum;
     }
-    if (lane == 0) p.gsig[t] = sigmoidf_(z);
+    if (lane == 0) *out_gsig = sigmoidf_(z);
     if (threadIdx.x == 0) MOE_TRACE(0, 6);
+}
+
+// One row's top-k from the router's logits in the workspace (one warp).
+template <int EPL>
+__device__ void topk_row(const RouterParams &p, int t)
+{
+    topk_select<EPL>(p.logits + (size_t)t * p.ld, p.E, p.K, p.topk_idx + (size_t)t * p.K, p.topk_w + (size_t)t * p.K,
+                     p.gsig + t);
 }
 
 __device__ void topk_rows(const RouterParams &p, int t_begin, int t_end)
@@ -417,10 +424,11 @@ __device__ __forceinline__ LocalPlan plan_at(unsigned char *base, int E, int P)
 __device__ int build_local_plan(const ExpertParams &p, const LocalPlan &lp)
 {
     const int E = p.E, P = p.rows * p.K;
+    auto expert_of = [&](int i) { return __ldcg(p.topk_idx + i); };
     for (int e = threadIdx.x; e < E; e += blockDim.x) lp.cnt[e] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < P; i += blockDim.x)
-        atomicAdd(&lp.cnt[min(max(__ldcg(p.topk_idx + i), 0), E - 1)], 1);
+        atomicAdd(&lp.cnt[min(max(expert_of(i), 0), E - 1)], 1);
     __syncthreads();
     int run_off = 0, run_act = 0;
     for (int e0 = 0; e0 < E; e0 += blockDim.x) {
@@ -440,7 +448,7 @@ __device__ int build_local_plan(const ExpertParams &p, const LocalPlan &lp)
     if (threadIdx.x == 0) lp.first_of[run_act] = run_off;
     __syncthreads();
     for (int i = threadIdx.x; i < P; i += blockDim.x) {
-        const int e = min(max(__ldcg(p.topk_idx + i), 0), E - 1);
+        const int e = min(max(expert_of(i), 0), E - 1);
         lp.pairs[atomicAdd(&lp.cnt[e], 1)] = i;
     }
     const int bad = __ldcg(p.counters + kCtrStatus);
@@ -608,49 +616,39 @@ __device__ void prefetch_down_weights(const ExpertParams &p, const LocalPlan &lp
     }
 }
 
-template <int T>
-__global__ void __launch_bounds__(kExpThreads, 1) gate_up_kernel(ExpertParams p)
+// gate_up, producer warp: the weights of the first stages' shared-expert
+// items, which do not depend on routing (fetched before the routing exists).
+__device__ void gu_prefetch_shared(const ExpertParams &p, unsigned char *smem, uint64_t *full, StageDesc *desc)
 {
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
-    __shared__ StageDesc desc[kMaxStages];
-    __shared__ volatile int s_abort;
+    const int lane = threadIdx.x & 31;
+    const GuLayout L = gu_layout(p);
+    const int per_shared = p.Is / p.pairs, per_routed = p.I / p.pairs;
+    const uint64_t pol = policy_evict_first();
+    for (int q = 0; q < p.stages; ++q) {
+        const int item = blockIdx.x + q * gridDim.x;
+        if (item >= per_shared) break;
+        if (lane == 0) describe(p, item, per_shared, per_routed, p.pairs, nullptr, desc[q]);
+        __syncwarp();
+        gu_produce(p, L, desc[q], smem + q * L.bytes, &full[q], pol, true, false);
+    }
+    __syncwarp();
+}
+
+// gate_up's item loops, once the routing table lp (n_active routed experts)
+// exists: the producer warp fills the stage ring, the consumer warps compute
+// h into HBM.  Every thread of the CTA calls this; it returns when the
+// thread's role is done.
+template <int T>
+__device__ void gu_items(const ExpertParams &p, unsigned char *smem, uint64_t *full, uint64_t *empty, StageDesc *desc,
+                         volatile int &s_abort, const LocalPlan &lp, int n_active)
+{
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const GuLayout L = gu_layout(p);
     const int per_shared = p.Is / p.pairs, per_routed = p.I / p.pairs;
     const int S = p.stages;
     float4 *red = reinterpret_cast<float4 *>(smem + (size_t)S * L.bytes);  // [warp][tile][lane]
-    const LocalPlan lp = plan_at(smem + (size_t)S * L.bytes + red_bytes(L.T), p.E, p.rows * p.K);
-
-    if (threadIdx.x == 0) {
-        s_abort = 0;
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) MOE_TRACE(1, 0);
-
     const uint64_t pol = policy_evict_first();
-    if (warp == kConsumerWarps) {
-        // Shared-expert weights and scales do not depend on routing: fetch
-        // them before waiting on the router.
-        for (int q = 0; q < S; ++q) {
-            const int item = blockIdx.x + q * gridDim.x;
-            if (item >= per_shared) break;
-            if (lane == 0) describe(p, item, per_shared, per_routed, p.pairs, nullptr, desc[q]);
-            __syncwarp();
-            gu_produce(p, L, desc[q], smem + q * L.bytes, &full[q], pol, true, false);
-        }
-        __syncwarp();
-    }
-    pdl_wait();
-    pdl_trigger();
-    const int n_active = build_local_plan(p, lp);
     const int n_items = per_shared + n_active * per_routed;
-    if (threadIdx.x == 0) MOE_TRACE(1, 1);
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------- producer
         for (int q = 0;; ++q) {
@@ -794,6 +792,36 @@ __global__ void __launch_bounds__(kExpThreads, 1) gate_up_kernel(ExpertParams p)
         __syncwarp();  // this warp is done with the stage and its descriptor
         if (lane == 0) mbar_arrive(&empty[s]);
     }
+}
+
+template <int T>
+__global__ void __launch_bounds__(kExpThreads, 1) gate_up_kernel(ExpertParams p)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ StageDesc desc[kMaxStages];
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5;
+    const GuLayout L = gu_layout(p);
+    const int S = p.stages;
+    const LocalPlan lp = plan_at(smem + (size_t)S * L.bytes + red_bytes(L.T), p.E, p.rows * p.K);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(1, 0);
+    if (warp == kConsumerWarps) gu_prefetch_shared(p, smem, full, desc);
+    pdl_wait();
+    pdl_trigger();
+    const int n_active = build_local_plan(p, lp);
+    if (threadIdx.x == 0) MOE_TRACE(1, 1);
+    gu_items<T>(p, smem, full, empty, desc, s_abort, lp, n_active);
     if (threadIdx.x == 0) MOE_TRACE(1, 6);
 }
 
@@ -1189,47 +1217,25 @@ __device__ void ds_produce_h(const ExpertParams &p, const DsLayout &L, unsigned 
     }
 }
 
-__global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid_constant__ DsParams P)
+// The down-by-output-block item loops, once the routing table lp (n_active
+// routed experts) and the slot weights wt (routing weights, then the shared
+// gates: rows*K + rows floats) are in shared memory.  The producer warp
+// streams W2 tiles through the stage ring and then the h rows (after
+// gate_up: they wait for it here); the consumer warps quantise h once and
+// write out.  Every thread of the CTA calls this.
+__device__ void ds_items(const DsParams &P, unsigned char *smem, uint64_t *full, uint64_t *empty, uint64_t *hbar,
+                         volatile int &s_abort, const LocalPlan &lp, int n_active, const float *wt)
 {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], hbar;
-    __shared__ volatile int s_abort;
     const ExpertParams &p = P.p;
     const int ue = p.ue, S = p.stages;
-    unsigned char *smem =
-        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const DsLayout L = ds_layout(p.K, p.I, p.Is, p.rows, ue, S);
-    const LocalPlan lp = plan_at(smem + L.plan, p.E, p.rows * p.K);
     const int PR = p.rows * p.K;
-    float *wt = reinterpret_cast<float *>(smem + L.wt);
     float *ys = reinterpret_cast<float *>(smem + L.ys);
     float *hs = reinterpret_cast<float *>(smem + L.hs);
-
-    if (threadIdx.x == 0) {
-        s_abort = 0;
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        mbar_init(&hbar, 1);
-        fence_mbar_init();
-    }
-    if (warp == kConsumerWarps && lane == 0) {
-        tma_prefetch_desc(&P.w2r);
-        tma_prefetch_desc(&P.w2s);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) MOE_TRACE(2, 0);
-    // The router finished before this kernel could launch: the routing is final.
-    const int n_active = build_local_plan(p, lp);
     const int n_exp = n_active + 1;             // + the shared expert
     const int chunks = (n_exp + ue - 1) / ue;   // stage loads per item
     const int n_items = p.H / 16;
-    for (int i = threadIdx.x; i < L.S_all; i += blockDim.x)
-        wt[i] = i < PR ? __ldcg(p.topk_w + i) : __ldcg(p.gsig + i - PR);
-    __syncthreads();  // every thread wrote some of wt; the consumers read all of it
-
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------- producer
         const uint64_t pol = policy_evict_first();
@@ -1242,7 +1248,7 @@ __global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid
                     h_done = true;
                     pdl_wait();
                     pdl_trigger();
-                    ds_produce_h(p, L, smem, &hbar);
+                    ds_produce_h(p, L, smem, hbar);
                 }
                 if (q >= S && !mbar_wait(&empty[s], ((q / S) - 1) & 1, kWaitLimitNs)) {
                     if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
@@ -1258,7 +1264,7 @@ __global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid
         if (!h_done) {
             pdl_wait();
             pdl_trigger();
-            ds_produce_h(p, L, smem, &hbar);
+            ds_produce_h(p, L, smem, hbar);
         }
         return;
     }
@@ -1267,7 +1273,7 @@ __global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid
     pdl_wait();
     pdl_trigger();
     if (threadIdx.x == 0) MOE_TRACE(2, 1);
-    if (!mbar_wait(&hbar, 0, kWaitLimitNs)) {
+    if (!mbar_wait(hbar, 0, kWaitLimitNs)) {
         if (lane == 0) set_status(p.counters, MOE_ETIMEOUT);
         s_abort = 1;
     }
@@ -1380,6 +1386,43 @@ __global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid
         }
         named_barrier(1, kConsumerThreads);  // ys may be rewritten by the next item
     }
+}
+
+__global__ void __launch_bounds__(kExpThreads, 1) down_small_kernel(const __grid_constant__ DsParams P)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], hbar;
+    __shared__ volatile int s_abort;
+    const ExpertParams &p = P.p;
+    unsigned char *smem =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const DsLayout L = ds_layout(p.K, p.I, p.Is, p.rows, p.ue, p.stages);
+    const LocalPlan lp = plan_at(smem + L.plan, p.E, p.rows * p.K);
+    const int PR = p.rows * p.K;
+    float *wt = reinterpret_cast<float *>(smem + L.wt);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        mbar_init(&hbar, 1);
+        fence_mbar_init();
+    }
+    if (warp == kConsumerWarps && lane == 0) {
+        tma_prefetch_desc(&P.w2r);
+        tma_prefetch_desc(&P.w2s);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) MOE_TRACE(2, 0);
+    // The router finished before this kernel could launch: the routing is final.
+    const int n_active = build_local_plan(p, lp);
+    for (int i = threadIdx.x; i < L.S_all; i += blockDim.x)
+        wt[i] = i < PR ? __ldcg(p.topk_w + i) : __ldcg(p.gsig + i - PR);
+    __syncthreads();  // every thread wrote some of wt; the consumers read all of it
+    ds_items(P, smem, full, empty, &hbar, s_abort, lp, n_active, wt);
     if (threadIdx.x == 0) MOE_TRACE(2, 8);
 }
 
@@ -1645,5 +1688,6 @@ cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s)
     }
     return cudaSuccess;
 }
+
 
 }  // namespace moe

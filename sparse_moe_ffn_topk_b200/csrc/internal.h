@@ -109,6 +109,7 @@ struct ExpertsLaunch {
     int32_t *counters;
 };
 cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s);
+
 // One CTA waits on an mbarrier that nothing completes, for at most limit_ns,
 // then records MOE_ETIMEOUT in counters[kCtrStatus].
 cudaError_t launch_wait_probe(int32_t *counters, uint64_t limit_ns, cudaStream_t s);

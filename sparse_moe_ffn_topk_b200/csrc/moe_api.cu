@@ -74,7 +74,7 @@ int kernel_launches(const moe_dims &d, int32_t rows, int32_t path)
     if (path == MOE_PATH_AUTO)
         path = (rows <= MOE_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
     if (path == MOE_PATH_PREFILL) return prefill_kernel_launches(d, rows);
-    return 3;  // router_topk, gate_up, down_blend
+    return 3;  // router_topk, gate_up, down
 }
 
 const DeviceInfo &device_info()
@@ -212,8 +212,6 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     ra.xq = reinterpret_cast<uint8_t *>(base + L.xq);
     ra.xsc = reinterpret_cast<float *>(base + L.xsc);
     ra.counters = counters;
-    cudaError_t e = launch_router_topk(ra, s);
-    if (e != cudaSuccess) return finish(e);
 
     ExpertsLaunch ea;
     ea.d = d;
@@ -234,6 +232,8 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     ea.h_shared = reinterpret_cast<float *>(base + L.h_shared);
     ea.yslot = reinterpret_cast<float *>(base + L.yslot);
     ea.counters = counters;
+    cudaError_t e = launch_router_topk(ra, s);
+    if (e != cudaSuccess) return finish(e);
     return finish(launch_decode_experts(ea, s));
 }
 
