@@ -508,19 +508,33 @@ def e2e_measure(dims, insts, rows: int, steps: int, dist: Dist, seed: int):
 
     with torch.cuda.stream(s):
         for i in range(5):
-            one(i)
+            one(i)  # eager: sets up kernel attributes
+    torch.cuda.synchronize()
+    # The steps are replayed from CUDA graphs (as a serving loop would run
+    # them); every step in a graph still copies its x from pinned host memory
+    # and its output back to pinned host memory.
+    chunk = 250
+    graphs = []
+    for first in range(0, steps, chunk):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for j in range(first, min(steps, first + chunk)):
+                one(j)
+        graphs.append(g)
+    graphs[0].replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
     with torch.cuda.stream(s):
         e0.record(s)
-        for i in range(steps):
-            one(i)
+        for g in graphs:
+            g.replay()
         e1.record(s)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     dist.barrier()
+    del graphs
     return ms, 2 * rows * dims.hidden, 2 * rows * dims.hidden
 
 
@@ -646,7 +660,9 @@ def run_ours(args, dist: Dist):
     es = dist.max(ems / 1000.0)
     result["e2e"] = {"value": round(aggregate(ke * by1["total"], dist.world, es) / 1e9, 2), "unit": "GB/s",
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                     "us_per_layer": round(es * 1e6 / ke, 3), "steps": ke}
+                     "us_per_layer": round(es * 1e6 / ke, 3), "steps": ke,
+                     "timing": "CUDA-graph replays of the public call; each step copies x from pinned host "
+                               "memory and out back to pinned host memory inside the timed region"}
 
     # ---- the CPU oracle on this host (rank 0, N = 1 only)
     if dist.world == 1:
