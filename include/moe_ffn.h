@@ -78,7 +78,7 @@ extern "C" {
 #define MOE_ETIMEOUT -5      /* a bounded wait inside a kernel ran out (device status word) */
 
 #define MOE_PATH_AUTO 0      /* decode kernels for rows <= MOE_DECODE_MAX_ROWS, else prefill */
-#define MOE_PATH_DECODE 1    /* warp-per-row FP8 GEMVs with expert dedup */
+#define MOE_PATH_DECODE 1    /* FP8 weight-streaming GEMVs (16-row tensor-core tiles) with expert dedup */
 #define MOE_PATH_PREFILL 2   /* token permute -> tcgen05 FP8 grouped GEMMs -> unpermute */
 #define MOE_DECODE_MAX_ROWS 64
 

@@ -3,21 +3,27 @@
 // Three launches chained with programmatic dependent launch (PDL):
 //   1. router_topk_kernel: bf16 router GEMV + shared-gate dot.  Each CTA
 //      bulk-copies its slice of router rows into shared memory before it
-//      waits on the kernel that produced x, one warp per router row; the last
-//      CTA to finish runs the top-k softmax and builds the per-expert work
-//      table (expert dedup across rows).
-//   2. gate_up_kernel: persistent CTAs walk (expert, block of gate/up row
-//      pairs) items through a ring of shared-memory stages filled by bulk
-//      copies; shared-expert items come first and are fetched before the PDL
-//      wait, since they do not depend on routing.  A warp per row pair,
-//      block scales applied in registers, h = silu(gate) * up kept in fp32.
-//   3. down_blend_kernel: (expert, block of down rows) items, fetched
-//      through the same kind of ring; the weight blocks are fetched as soon
-//      as the CTA starts (routing is final by then) and only h waits for
-//      gate_up.  A warp per output row, one partial per routed slot scaled by
-//      its routing weight (or the shared gate); the last item to finish a row
-//      block blends the k partials in rank order plus the shared partial
-//      (plus the residual) and rounds once to bf16.
+//      waits on the kernel that produced x, one warp per router row; the row
+//      block 0 CTA also writes x as hi/lo e4m3 rows; the last CTA of each
+//      token group runs the group's top-k softmax.
+//   2. gate_up_kernel: every CTA first builds the per-expert routing table
+//      (expert dedup across rows) in its shared memory from the top-k.
+//      Persistent CTAs then walk (expert, block of gate/up row pairs) items
+//      through a ring of shared-memory stages filled by bulk copies;
+//      shared-expert items come first and are fetched before the PDL wait,
+//      since they do not depend on routing.  The e4m3 weight bytes feed
+//      mma.m16n8k32 directly, block scales are applied per 128-wide K block
+//      in registers, h = silu(gate) * up is kept in fp32.
+//   3. The down product and blend, one of two kernels:
+//      down_small_kernel (few rows): a CTA item is 16 output rows of every
+//      active expert and the shared expert (W2 tiles by TMA), so each output
+//      row is complete in one CTA and written straight to out;
+//      down_blend_kernel (otherwise): (expert, block of down rows) items
+//      through the same kind of ring as gate_up; one partial per routed slot
+//      scaled by its routing weight (or the shared gate); the last item to
+//      finish a row block blends the k partials in rank order plus the
+//      shared partial (plus the residual) and rounds once to bf16.
+//      Both use one arithmetic, so their results are identical bits.
 //
 // Prior art on the pages: the GB10 blueprint's per-layer MoE chain (router
 // GEMV, top-k softmax, gate_up with the shared expert fused, silu+down,

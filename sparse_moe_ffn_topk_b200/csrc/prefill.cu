@@ -536,7 +536,7 @@ __device__ __forceinline__ bool tile_info(const GemmParams &p, int n_mtiles, int
         ti.ntiles = inter / 128;  // one 128-column block of h per tile
     } else {
         ti.kdim = inter;
-        ti.ntiles = p.H / kBN;
+        ti.ntiles = (p.H + kBN - 1) / kBN;  // the last tile is half empty when H is an odd multiple of 128
     }
     return true;
 }
@@ -694,7 +694,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                                      : p.w_scales + (size_t)ti.group * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128))) +
                       (2 * inter / 128) * (p.H / 128);
                 wld = inter / 128;
-                wn0 = wn1 = ti.nt * 2 + (quarter >> 1);
+                // a column quarter past H (the empty half of a last tile) keeps a
+                // valid scale row; its results are not stored
+                wn0 = wn1 = min(ti.nt * 2 + (quarter >> 1), p.H / 128 - 1);
             }
             float tot[64];
 #pragma unroll
@@ -794,7 +796,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     if (valid && quarter == 0) p.hs[((size_t)ti.row0 + r) * (p.imax / 128) + ti.nt] = sc;
                 }
             } else {
-                if (ok) {
+                if (ok && ti.nt * kBN + 64 * quarter < p.H) {
                     // 8 columns at a time through the staging buffer (rows of 9
                     // floats), then out as 32-byte row segments, 16 bytes per lane
                     float *sf = reinterpret_cast<float *>(stg);
@@ -937,7 +939,7 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
 {
     const int T = rows, E = d.n_experts, K = d.top_k, H = d.hidden, I = d.inter, Is = d.shared_inter;
     const int imax = std::max(I, Is);
-    if (H % kBN || H % kBK) return MOE_EUNSUPPORTED;  // GEMM2 N tiles of 256 columns
+    if (H % kBK) return MOE_EUNSUPPORTED;
     const PrefillLayout L = prefill_layout(d, T);
     char *base = static_cast<char *>(ws);
     int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
@@ -1051,7 +1053,7 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     g2.a_scales_routed = g.hs;
     g2.a_scales_shared = g.hs;
     g2.a_scales_ld = imax / 128;
-    g2.max_ntiles = H / kBN;
+    g2.max_ntiles = (H + kBN - 1) / kBN;
     if ((e = launch_kernel(gemm_kernel<2>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g2)) != cudaSuccess)
         return MOE_ECUDA;
 

@@ -101,3 +101,17 @@ def test_qwen35_397b_prefill_sampled():
     sample = np.random.default_rng(1).choice(rows, 16, replace=False)
     sub = P.Case(d, case.layer, case.x[sample].copy(), case.logits[sample])
     P.compare_output(sub, out[sample], idx[sample])
+
+
+@pytest.mark.parametrize("dims,rows", [
+    (mi.LayerDims(hidden=384, n_experts=12, top_k=3, inter=256, shared_inter=128), 150),
+    (mi.LayerDims(hidden=640, n_experts=20, top_k=4, inter=128, shared_inter=256), 100),
+])
+def test_prefill_hidden_odd_multiple_of_128(dims, rows):
+    # H/128 odd: the down GEMM's last 256-column tile is half empty; AUTO picks prefill above 64 rows
+    case = P.build_case(dims, rows, router_bias=True, all_experts=True, residual=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_AUTO)
+    _, oidx, ow, ogs = oracle.router_topk(dims, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
