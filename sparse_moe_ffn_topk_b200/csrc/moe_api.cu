@@ -72,7 +72,7 @@ int kernel_launches(const moe_dims &d, int32_t rows, int32_t path)
 {
     if (rows <= 0) return 0;
     if (path == MOE_PATH_AUTO)
-        path = (rows <= MOE_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
+        path = (rows <= MOE_AUTO_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
     if (path == MOE_PATH_PREFILL) return prefill_kernel_launches(d, rows);
     return 3;  // router_topk, gate_up, down
 }
@@ -182,7 +182,7 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     if (rows == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (path == MOE_PATH_AUTO)
-        path = (rows <= MOE_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
+        path = (rows <= MOE_AUTO_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
     if (path == MOE_PATH_PREFILL) {
         int rc = prefill_forward(*d, x, rows, router_w, expert_w8, expert_scales, shared_w->w8,
                                  shared_w->scales, shared_gate, out, residual, router_bias, ws, s,

@@ -28,7 +28,7 @@ def dev35(layer35):
     return P.device_weights(layer35)
 
 
-def run_forward(case, dev=None, path=moe.MOE_PATH_AUTO, residual_inplace=False):
+def run_forward(case, dev=None, path=moe.MOE_PATH_DECODE, residual_inplace=False):
     d = case.dims
     dev = dev or P.device_weights(case.layer)
     rows = case.x.shape[0]
@@ -113,18 +113,22 @@ def test_residual_in_place():
     check(case, residual_inplace=True)
 
 
-def test_rows_64_max_decode_tile_then_rows_1_on_same_workspace(layer35, dev35):
-    """Counters left by one call must not disturb the next (different rows)."""
+@pytest.mark.parametrize("path", ["decode", "auto"])
+def test_rows_64_max_decode_tile_then_rows_1_on_same_workspace(layer35, dev35, path):
+    """Counters left by one call must not disturb the next (different rows;
+    through AUTO, 64 rows take the prefill path and 1 row the decode path)."""
     d = mi.QWEN36_35B_A3B
     ws = moe.alloc_workspace(d, 64)
+    pcode = moe.MOE_PATH_DECODE if path == "decode" else moe.MOE_PATH_AUTO
     outs = []
     for rows in (64, 1, 64):
         case = P.build_case(d, rows, layer=layer35)
         x = P.bf16_tensor(case.x)
         out = torch.empty(rows, d.hidden, dtype=torch.bfloat16, device="cuda")
-        moe.ffn_forward(d, x, dev35["router_w"], dev35["expert_w8"], dev35["expert_scales"],
-                        dev35["shared_w8"], dev35["shared_scales"], dev35["shared_gate"], out, ws)
+        moe.ffn_forward_path(d, x, dev35["router_w"], dev35["expert_w8"], dev35["expert_scales"],
+                             dev35["shared_w8"], dev35["shared_scales"], dev35["shared_gate"], out, ws, path=pcode)
         torch.cuda.synchronize()
+        assert moe.device_status(ws) == moe.MOE_OK
         outs.append(out.clone())
     assert torch.equal(outs[0], outs[2])
 

@@ -53,12 +53,24 @@ def test_prefill_small_shapes(dims, rows, bias):
     P.compare_output(case, out, idx)
 
 
-def test_auto_path_uses_prefill_above_64_rows():
+def test_auto_path_switch():
     d = mi.TINY
-    assert moe.kernel_launches(d, 64) == 3
-    assert moe.kernel_launches(d, 65) == 6
-    case = P.build_case(d, 65, all_experts=True)
+    assert moe.MOE_AUTO_DECODE_MAX_ROWS == 12
+    assert moe.kernel_launches(d, 12) == 3
+    assert moe.kernel_launches(d, 13) == 6
+    case = P.build_case(d, 13, all_experts=True)
     out, idx, _, _ = run(case, moe.MOE_PATH_AUTO)
+    P.compare_output(case, out, idx)
+
+
+@pytest.mark.parametrize("rows", [16, 32, 64])
+def test_qwen36_35b_auto_prefill_at_decode_row_counts(rows):
+    # AUTO takes the grouped-GEMM path from 13 rows on: every row against the oracle
+    d = mi.QWEN36_35B_A3B
+    case = P.build_case(d, rows)
+    out, idx, w, gs = run(case, moe.MOE_PATH_AUTO)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate)
+    P.check_routing(case, idx, w, gs, ow, ogs)
     P.compare_output(case, out, idx)
 
 
