@@ -279,11 +279,12 @@ def make_instances(layer, n: int):
 
 
 class DecodeBench:
-    def __init__(self, dims, insts, xs, rows):
+    def __init__(self, dims, insts, xs, rows, path=None):
         import torch
 
         import sparse_moe_ffn_topk_b200 as moe
         self.moe, self.torch = moe, torch
+        self.path = moe.MOE_PATH_AUTO if path is None else path
         self.d, self.insts, self.xs, self.rows = dims, insts, xs, rows
         self.outs = [torch.empty(rows, dims.hidden, dtype=torch.bfloat16, device="cuda") for _ in range(len(xs))]
         self.ws = moe.alloc_workspace(dims, rows)
@@ -296,9 +297,9 @@ class DecodeBench:
         args = (self.d, x, w["router_w"], w["expert_w8"], w["expert_scales"], w["shared_w8"], w["shared_scales"],
                 w["shared_gate"], out, self.ws)
         if events is None:
-            self.moe.ffn_forward(*args, stream=self.stream)
+            self.moe.ffn_forward_path(*args, path=self.path, stream=self.stream)
         else:
-            self.moe.ffn_forward_timed(*args, events=events, stream=self.stream)
+            self.moe.ffn_forward_timed(*args, events=events, path=self.path, stream=self.stream)
 
     def graph(self, first: int, count: int, events=None):
         torch = self.torch
@@ -646,7 +647,8 @@ def run_ours(args, dist: Dist):
         result["rows64"] = {"us_per_layer": round(s64 * 1e6 / k64, 3), "gb_s": round(gbs64, 1),
                             "hbm_frac_of_measured": round(gbs64 / dist.world / hbm_peak, 4),
                             "tokens_per_s": round(aggregate(k64 * r64, dist.world, s64), 1),
-                            "distinct_experts_per_step": round(u64, 1), "steps": k64}
+                            "distinct_experts_per_step": round(u64, 1), "steps": k64,
+                            "kernels": "decode" if moe.kernel_launches(d, r64) == 3 else "prefill"}
 
     # ---- prefill, 4096 tokens
     result["prefill"] = prefill_leg(args, d, insts[0], dist, bus, hbm_peak, bf16_peak, peak_kind)
@@ -729,6 +731,7 @@ def run_sweep(args, dist: Dist):
     import torch
 
     import moe_inputs as mi
+    import sparse_moe_ffn_topk_b200 as moe
     torch.cuda.set_device(dist.local)
     hbm_peak, _, peak_kind = peaks()
     res = []
@@ -738,20 +741,28 @@ def run_sweep(args, dist: Dist):
         for rows in rows_list:
             xs = [torch.from_numpy(mi.make_x(dims, rows, seed=args.seed + 1, stream=1000 * rows + i).view("int16"))
                   .view(torch.bfloat16).cuda() for i in range(16)]
-            b = DecodeBench(dims, insts, xs, rows)
-            u = statistics.mean(b.routing(16))
-            by = algorithmic_bytes(dims, rows, u)
-            k = max(50, min(args.steps, 4000 // rows))
-            ms, _ = b.time_steps(k, max(3, args.warmup), dist)
-            sec = dist.max(ms / 1000.0)
-            gbs = aggregate(k * by["total"], dist.world, sec) / 1e9
-            res.append({"workload": f"{name} decode rows={rows}", "us_per_layer": round(sec * 1e6 / k, 3),
-                        "gb_s": round(gbs, 1), "hbm_frac_of_measured": round(gbs / dist.world / hbm_peak, 4),
-                        "tokens_per_s": round(aggregate(k * rows, dist.world, sec), 1),
-                        "distinct_experts": round(u, 1), "bytes_per_step": int(by["total"]), "steps": k})
-            print(f"[sweep] {res[-1]['workload']}: {res[-1]['us_per_layer']} us, {gbs:.0f} GB/s", file=sys.stderr,
-                  flush=True)
-            del b
+            # AUTO (what a caller gets), and the decode kernels forced where AUTO
+            # takes the grouped-GEMM path, to show the switch point
+            paths = [("auto", moe.MOE_PATH_AUTO)]
+            if rows > moe.MOE_AUTO_DECODE_MAX_ROWS:
+                paths.append(("decode", moe.MOE_PATH_DECODE))
+            for pname, pcode in paths:
+                b = DecodeBench(dims, insts, xs, rows, path=pcode)
+                u = statistics.mean(b.routing(16))
+                by = algorithmic_bytes(dims, rows, u)
+                k = max(50, min(args.steps, 4000 // rows))
+                ms, _ = b.time_steps(k, max(3, args.warmup), dist)
+                sec = dist.max(ms / 1000.0)
+                gbs = aggregate(k * by["total"], dist.world, sec) / 1e9
+                kern = "decode" if moe.kernel_launches(dims, rows, pcode) == 3 else "prefill"
+                res.append({"workload": f"{name} decode rows={rows}", "path": pname, "kernels": kern,
+                            "us_per_layer": round(sec * 1e6 / k, 3),
+                            "gb_s": round(gbs, 1), "hbm_frac_of_measured": round(gbs / dist.world / hbm_peak, 4),
+                            "tokens_per_s": round(aggregate(k * rows, dist.world, sec), 1),
+                            "distinct_experts": round(u, 1), "bytes_per_step": int(by["total"]), "steps": k})
+                print(f"[sweep] {res[-1]['workload']} {pname} ({kern}): {res[-1]['us_per_layer']} us, "
+                      f"{gbs:.0f} GB/s", file=sys.stderr, flush=True)
+                del b
         del insts
         torch.cuda.empty_cache()
     return {"sweep": res, "peak_source": f"{peak_kind} ({hbm_peak} GB/s copy)", "n_gpus": dist.world}
