@@ -57,8 +57,10 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true", help="skip the rows=64 and per-kernel legs")
-    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
-                    help="a small case for a profiler: a few eager layer calls on one weight copy, then exit")
+    ap.add_argument("--profile", choices=["decode", "prefill", "narrow"], default=None,
+                    help="a small case for a profiler: a few eager layer calls on one weight copy, then exit "
+                         "(decode: rows=1; prefill: 4096 biased rows; narrow: the narrow grouped GEMMs at --rows)")
+    ap.add_argument("--rows", type=int, default=64, help="rows of --profile narrow")
     ap.add_argument("--calls", type=int, default=4, help="layer calls of --profile")
     ap.add_argument("--sweep", action="store_true",
                     help="time every decode workload (35B rows 1..64, 397B rows 1 and 32) and print one JSON line")
@@ -363,7 +365,7 @@ class DecodeBench:
         Steps are enqueued eagerly behind a GPU sleep, so that the stream is
         full before the GPU reaches them and each event interval is GPU time."""
         torch = self.torch
-        nk = self.moe.kernel_launches(self.d, self.rows)
+        nk = self.moe.kernel_launches(self.d, self.rows, self.path)
         per = []
         done = 0
         while done < steps:
@@ -725,28 +727,32 @@ def run_reference(args, dist: Dist):
 
 
 def run_sweep(args, dist: Dist):
-    """Decode at every row count of the workloads: 35B-A3B-shaped rows 1, 2,
-    8, 16, 32, 64 (16 weight copies) and 397B-A17B-shaped rows 1 and 32 (two
-    6.4 GB copies); CUDA events over CUDA-graph replays, as the headline."""
+    """Every row count of the decode workloads (35B-A3B-shaped rows 1, 2, 8,
+    16, 32, 64, with 128 and 256 beside them; 397B-A17B-shaped rows 1 and 32)
+    on each path that takes it: the decode kernels (up to 64 rows), the
+    grouped GEMMs with 128-row token tiles, and the narrow grouped GEMMs;
+    each line says whether it is the path MOE_PATH_AUTO takes.  CUDA events
+    over CUDA-graph replays, 16 rotating weight copies (35B) or two (397B)."""
     import torch
 
     import moe_inputs as mi
     import sparse_moe_ffn_topk_b200 as moe
     torch.cuda.set_device(dist.local)
     hbm_peak, _, peak_kind = peaks()
+    names = {moe.MOE_PATH_DECODE: "decode", moe.MOE_PATH_PREFILL: "grouped", moe.MOE_PATH_PREFILL_NARROW: "narrow"}
     res = []
-    for dims, name, rows_list, n_inst in ((mi.QWEN36_35B_A3B, "Qwen3.6-35B-A3B-shaped", [1, 2, 8, 16, 32, 64], 16),
+    for dims, name, rows_list, n_inst in ((mi.QWEN36_35B_A3B, "Qwen3.6-35B-A3B-shaped",
+                                           [1, 2, 8, 16, 32, 64, 128, 256], 16),
                                           (mi.QWEN35_397B_A17B, "Qwen3.5-397B-A17B-shaped", [1, 32], 2)):
         insts = make_instances(mi.make_layer(dims, seed=args.seed), n_inst)
         for rows in rows_list:
             xs = [torch.from_numpy(mi.make_x(dims, rows, seed=args.seed + 1, stream=1000 * rows + i).view("int16"))
                   .view(torch.bfloat16).cuda() for i in range(16)]
-            # AUTO (what a caller gets), and the decode kernels forced where AUTO
-            # takes the grouped-GEMM path, to show the switch point
-            paths = [("auto", moe.MOE_PATH_AUTO)]
-            if rows > moe.MOE_AUTO_DECODE_MAX_ROWS:
-                paths.append(("decode", moe.MOE_PATH_DECODE))
-            for pname, pcode in paths:
+            auto = moe.auto_path(dims, rows)
+            paths = [moe.MOE_PATH_PREFILL, moe.MOE_PATH_PREFILL_NARROW]
+            if rows <= 64:
+                paths.insert(0, moe.MOE_PATH_DECODE)
+            for pcode in paths:
                 b = DecodeBench(dims, insts, xs, rows, path=pcode)
                 u = statistics.mean(b.routing(16))
                 by = algorithmic_bytes(dims, rows, u)
@@ -754,14 +760,13 @@ def run_sweep(args, dist: Dist):
                 ms, _ = b.time_steps(k, max(3, args.warmup), dist)
                 sec = dist.max(ms / 1000.0)
                 gbs = aggregate(k * by["total"], dist.world, sec) / 1e9
-                kern = "decode" if moe.kernel_launches(dims, rows, pcode) == 3 else "prefill"
-                res.append({"workload": f"{name} decode rows={rows}", "path": pname, "kernels": kern,
+                res.append({"workload": f"{name} rows={rows}", "path": names[pcode], "auto": pcode == auto,
                             "us_per_layer": round(sec * 1e6 / k, 3),
                             "gb_s": round(gbs, 1), "hbm_frac_of_measured": round(gbs / dist.world / hbm_peak, 4),
                             "tokens_per_s": round(aggregate(k * rows, dist.world, sec), 1),
                             "distinct_experts": round(u, 1), "bytes_per_step": int(by["total"]), "steps": k})
-                print(f"[sweep] {res[-1]['workload']} {pname} ({kern}): {res[-1]['us_per_layer']} us, "
-                      f"{gbs:.0f} GB/s", file=sys.stderr, flush=True)
+                print(f"[sweep] {res[-1]['workload']} {names[pcode]}{' (auto)' if pcode == auto else ''}: "
+                      f"{res[-1]['us_per_layer']} us, {gbs:.0f} GB/s", file=sys.stderr, flush=True)
                 del b
         del insts
         torch.cuda.empty_cache()
@@ -770,8 +775,9 @@ def run_sweep(args, dist: Dist):
 
 def run_profile_case(args):
     """A few eager calls of one workload (35B-shaped layer, one weight copy):
-    decode at rows = 1 on fresh x each call, or the 4096-token biased
-    prefill.  Small enough for a profiler to replay every kernel."""
+    decode at rows = 1 on fresh x each call, the 4096-token biased prefill, or
+    the narrow grouped GEMMs at --rows rows.  Small enough for a profiler to
+    replay every kernel."""
     import torch
 
     import moe_inputs as mi
@@ -780,6 +786,8 @@ def run_profile_case(args):
     inst = make_instances(mi.make_layer(d, seed=args.seed), 1)[0]
     if args.profile == "decode":
         rows, bias, path = 1, None, moe.MOE_PATH_AUTO
+    elif args.profile == "narrow":
+        rows, bias, path = args.rows, None, moe.MOE_PATH_PREFILL_NARROW
     else:
         rows, path = 4096, moe.MOE_PATH_PREFILL
         bias = torch.from_numpy(mi.make_router(d, args.seed, True)[2]).cuda()

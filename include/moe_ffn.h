@@ -80,6 +80,9 @@ extern "C" {
 #define MOE_PATH_AUTO 0      /* decode kernels for rows <= MOE_AUTO_DECODE_MAX_ROWS, else prefill */
 #define MOE_PATH_DECODE 1    /* FP8 weight-streaming GEMVs (16-row tensor-core tiles) with expert dedup */
 #define MOE_PATH_PREFILL 2   /* token permute -> tcgen05 FP8 grouped GEMMs -> unpermute */
+#define MOE_PATH_PREFILL_NARROW 3  /* the same pipeline with the grouped GEMMs tiled as 128 weight rows (the
+                                     MMA's M) x up to 32 rows of one expert (its N): for few rows per expert;
+                                     MOE_EUNSUPPORTED when H, I or Is exceeds 4096 */
 #define MOE_DECODE_MAX_ROWS 64       /* the decode path's tiles are sized for at most this many rows */
 #define MOE_AUTO_DECODE_MAX_ROWS 12  /* MOE_PATH_AUTO's switch to the prefill path (the two paths
                                         measured equal between 8 and 16 rows of a 35B-A3B-shaped
@@ -141,6 +144,11 @@ MOE_API int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t r
  * rows and path (MOE_PATH_AUTO resolved as moe_ffn_forward does); 0 for
  * invalid arguments or rows == 0. */
 MOE_API int32_t moe_kernel_launches(const moe_dims *d, int32_t rows, int32_t path);
+
+/* The path (MOE_PATH_DECODE, MOE_PATH_PREFILL or MOE_PATH_PREFILL_NARROW) that
+ * moe_ffn_forward and MOE_PATH_AUTO take for these dims and rows; host only,
+ * no device call; MOE_EINVAL for invalid dims or rows < 0. */
+MOE_API int32_t moe_auto_path(const moe_dims *d, int32_t rows);
 
 /* moe_ffn_forward_path for per-kernel timing: records events[0] on `stream`
  * before the first kernel and events[j] after kernel j-1 (each a caller-owned

@@ -37,12 +37,13 @@ MOE_ETIMEOUT = -5
 MOE_PATH_AUTO = 0
 MOE_PATH_DECODE = 1
 MOE_PATH_PREFILL = 2
+MOE_PATH_PREFILL_NARROW = 3
 MOE_DECODE_MAX_ROWS = 64
 MOE_AUTO_DECODE_MAX_ROWS = 12
 
 EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe_ffn_forward",
             "moe_ffn_forward_path", "moe_status", "moe_reset_status", "moe_status_string",
-            "moe_debug_inject_fault", "moe_kernel_launches", "moe_ffn_forward_timed",
+            "moe_debug_inject_fault", "moe_kernel_launches", "moe_auto_path", "moe_ffn_forward_timed",
             "moe_device_status", "moe_debug_wait_timeout", "moe_ffn_forward_static",
             "moe_static_scratch_bytes")
 
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
                                            P, ctypes.c_size_t, P, I32, P, P, P]
         L.moe_kernel_launches.argtypes = [DP, I32, I32]
         L.moe_kernel_launches.restype = I32
+        L.moe_auto_path.argtypes = [DP, I32]
+        L.moe_auto_path.restype = I32
         L.moe_ffn_forward_timed.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P,
                                             P, ctypes.c_size_t, P, I32, ctypes.POINTER(ctypes.c_void_p), I32]
         L.moe_device_status.argtypes = [P, ctypes.c_size_t, P]
@@ -198,12 +201,20 @@ def kernel_launches(dims, rows: int, path=MOE_PATH_AUTO) -> int:
     return int(lib().moe_kernel_launches(ctypes.byref(_dims(dims)), int(rows), int(path)))
 
 
+def auto_path(dims, rows: int) -> int:
+    """The MOE_PATH_* that MOE_PATH_AUTO takes for these dims and rows."""
+    return int(lib().moe_auto_path(ctypes.byref(_dims(dims)), int(rows)))
+
+
 def ffn_forward_timed(dims, x, router_w, expert_w8, expert_scales, shared_w8, shared_scales, shared_gate,
                       out, ws, events, path=MOE_PATH_AUTO, residual=None, router_bias=None, stream=None):
     """Forward that records ``events`` (torch.cuda.Event(enable_timing=True), at least
     kernel_launches()+1 of them) around each kernel it launches."""
     d = _dims(dims)
     sh = MoeFp8Expert(_ptr(shared_w8), _ptr(shared_scales))
+    for e in events:
+        if not e.cuda_event:  # torch creates an event's handle on its first record
+            e.record(stream if stream is not None else torch.cuda.current_stream())
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(lib().moe_ffn_forward_timed(ctypes.byref(d), _ptr(x), _rows(x), _ptr(router_w), _ptr(expert_w8),
                                        _ptr(expert_scales), ctypes.byref(sh), _ptr(shared_gate), _ptr(out),

@@ -127,6 +127,9 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
                     const uint8_t *expert_w8, const float *expert_scales, const uint8_t *shared_w8,
                     const float *shared_scales, const uint16_t *shared_gate, uint16_t *out,
                     const uint16_t *residual, const float *router_bias, void *ws, cudaStream_t s,
-                    int32_t *topk_idx_out, float *topk_w_out, float *gsig_out);
+                    int32_t *topk_idx_out, float *topk_w_out, float *gsig_out, bool narrow);
+// Whether the narrow grouped GEMMs (weight rows as M, up to 32 rows of a group
+// as N) take these dims.
+bool narrow_supported(const moe_dims &d);
 
 }  // namespace moe

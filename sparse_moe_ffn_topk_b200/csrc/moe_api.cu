@@ -68,12 +68,25 @@ TimingSession &timing_session()
     return ts;
 }
 
+bool valid_path(int32_t path)
+{
+    return path == MOE_PATH_AUTO || path == MOE_PATH_DECODE || path == MOE_PATH_PREFILL ||
+           path == MOE_PATH_PREFILL_NARROW;
+}
+
+// MOE_PATH_AUTO's choice for a row count.
+int32_t resolve_path(const moe_dims &d, int32_t rows, int32_t path)
+{
+    if (path != MOE_PATH_AUTO) return path;
+    if (rows <= MOE_AUTO_DECODE_MAX_ROWS || !prefill_available()) return MOE_PATH_DECODE;
+    return MOE_PATH_PREFILL;
+}
+
 int kernel_launches(const moe_dims &d, int32_t rows, int32_t path)
 {
     if (rows <= 0) return 0;
-    if (path == MOE_PATH_AUTO)
-        path = (rows <= MOE_AUTO_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
-    if (path == MOE_PATH_PREFILL) return prefill_kernel_launches(d, rows);
+    path = resolve_path(d, rows, path);
+    if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_NARROW) return prefill_kernel_launches(d, rows);
     return 3;  // router_topk, gate_up, down
 }
 
@@ -164,7 +177,7 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     int st = check_dims(d);
     if (st) return st;
     if (rows < 0) return MOE_EINVAL;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_EINVAL;
+    if (!valid_path(path)) return MOE_EINVAL;
     if (rows == 0) return enter();  // a no-op: no pointer is read
     if (!x || !router_w || !expert_w8 || !expert_scales || !shared_w || !shared_w->w8 ||
         !shared_w->scales || !shared_gate || !out || !ws)
@@ -181,12 +194,11 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     if (st) return st;
     if (rows == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (path == MOE_PATH_AUTO)
-        path = (rows <= MOE_AUTO_DECODE_MAX_ROWS || !prefill_available()) ? MOE_PATH_DECODE : MOE_PATH_PREFILL;
-    if (path == MOE_PATH_PREFILL) {
+    path = resolve_path(*d, rows, path);
+    if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_NARROW) {
         int rc = prefill_forward(*d, x, rows, router_w, expert_w8, expert_scales, shared_w->w8,
                                  shared_w->scales, shared_gate, out, residual, router_bias, ws, s,
-                                 topk_idx_out, topk_w_out, shared_gate_sig_out);
+                                 topk_idx_out, topk_w_out, shared_gate_sig_out, path == MOE_PATH_PREFILL_NARROW);
         if (rc == MOE_ECUDA) g_status.store(MOE_ECUDA);
         return rc;
     }
@@ -247,10 +259,16 @@ int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
                                 nullptr, nullptr);
 }
 
+int32_t moe_auto_path(const moe_dims *d, int32_t rows)
+{
+    if (check_dims(d) != MOE_OK || rows < 0) return MOE_EINVAL;
+    return resolve_path(*d, rows, MOE_PATH_AUTO);
+}
+
 int32_t moe_kernel_launches(const moe_dims *d, int32_t rows, int32_t path)
 {
     if (check_dims(d) != MOE_OK || rows < 0) return 0;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return 0;
+    if (!valid_path(path)) return 0;
     return kernel_launches(*d, rows, path);
 }
 

@@ -37,6 +37,8 @@ namespace moe {
 constexpr int kBM = 128;     // rows per M tile
 constexpr int kBN = 256;     // accumulator columns per tile
 constexpr int kBK = 128;     // K bytes per stage (one scale block of e4m3)
+constexpr int kNT = 32;      // token rows per item of the narrow grouped GEMM (its MMA's N)
+constexpr int kNtMaxKb = 32; // K blocks per item its scale table holds (K <= 4096)
 constexpr int kGemmStages = 3;
 constexpr int kEpiWarps = 16;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2..17: epilogue
@@ -50,8 +52,8 @@ constexpr size_t kGemmSmem =
 // ------------------------------------------------------------ layout
 
 struct PrefillLayout {
-    size_t counters, topk_idx, topk_w, gsig, counts, offsets, rank, pos, mtiles, xp, xps, slot_w, hq, hs, yslot,
-        total;
+    size_t counters, logits, topk_idx, topk_w, gsig, counts, offsets, rank, pos, mtiles, xp, xps, slot_w, hq, hs,
+        yslot, total;
     int64_t routed, rows_total, max_mtiles;
 };
 
@@ -62,10 +64,14 @@ inline PrefillLayout prefill_layout(const moe_dims &d, int64_t T)
     const int64_t imax = std::max(I, Is);
     L.routed = T * K;
     L.rows_total = T * K + T;
-    L.max_mtiles = (T * K + kBM - 1) / kBM + E + (T + kBM - 1) / kBM + 1;
+    // group tiles of kNT rows (the narrow GEMMs) outnumber those of kBM rows
+    L.max_mtiles = (T * K + kNT - 1) / kNT + E + (T + kNT - 1) / kNT + 1;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 1024); return at; };
     L.counters = take(sizeof(int32_t) * kCounters);
+    // up to MOE_DECODE_MAX_ROWS rows the decode path's router (spread over
+    // many CTAs) computes the routing; it needs fp32 logits rows
+    L.logits = take(T <= MOE_DECODE_MAX_ROWS ? sizeof(float) * T * ((E + 1 + 3) / 4 * 4) : 0);
     L.topk_idx = take(sizeof(int32_t) * T * K);
     L.topk_w = take(sizeof(float) * T * K);
     L.gsig = take(sizeof(float) * T);
@@ -95,6 +101,14 @@ bool prefill_available() { return true; }
 
 int prefill_kernel_launches(const moe_dims &, int64_t) { return 6; }
 
+// The narrow GEMMs keep a K block's activation scales of every item in
+// shared memory: K (H for GEMM1, the intermediate sizes for GEMM2) up to
+// 128 * kNtMaxKb.
+bool narrow_supported(const moe_dims &d)
+{
+    return d.hidden <= 128 * kNtMaxKb && d.inter <= 128 * kNtMaxKb && d.shared_inter <= 128 * kNtMaxKb;
+}
+
 // ------------------------------------------------------------ count / scan / permute
 
 struct PlanParams {
@@ -107,6 +121,8 @@ struct PlanParams {
     int32_t *rank;     // [T*K]
     int32_t *pos;      // [T*K]
     int4 *mtiles;      // [0].x = count; entries from [1]: {group, row0, rows, a_row0}
+    int tile_rows;     // rows per group tile: kBM, or kNT for the narrow GEMMs
+    int count_in_scan; // counts and ranks not given by the router: scan_kernel derives them
     const uint16_t *x; // [T][H] bf16
     int xp_shared0;    // first xp row of the shared expert's rows (the routed rows span at least 128)
     uint8_t *xp;
@@ -144,33 +160,46 @@ __device__ int block_scan_excl(int v, int *scratch, int *total)
     return r;
 }
 
-// One CTA of 1024 threads: expert offsets and the M-tile table.
+// One CTA of 1024 threads: expert offsets and the table of group tiles
+// (after each pair's rank within its expert, when the router gave none).
 __global__ void __launch_bounds__(1024) scan_kernel(PlanParams p)
 {
     __shared__ int scratch[33];
+    __shared__ int s_cnt[kMaxExperts];
     pdl_wait();
     pdl_trigger();
+    if (p.count_in_scan) {
+        for (int e = threadIdx.x; e < p.E; e += blockDim.x) s_cnt[e] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < p.T * p.K; i += blockDim.x) {
+            const int e = min(max(p.topk_idx[i], 0), p.E - 1);
+            p.rank[i] = atomicAdd(&s_cnt[e], 1);
+        }
+        __syncthreads();
+    }
     int run_rows = 0, run_tiles = 0;
     for (int e0 = 0; e0 < p.E; e0 += blockDim.x) {
         const int e = e0 + threadIdx.x;
-        const int c = (e < p.E) ? p.counts[e] : 0;
-        const int mt = (c + kBM - 1) / kBM;
+        const int c = (e < p.E) ? (p.count_in_scan ? s_cnt[e] : p.counts[e]) : 0;
+        const int mt = (c + p.tile_rows - 1) / p.tile_rows;
         int tot_rows, tot_tiles;
         const int off = block_scan_excl(c, scratch, &tot_rows) + run_rows;
         const int toff = block_scan_excl(mt, scratch, &tot_tiles) + run_tiles;
         if (e < p.E) {
             p.offsets[e] = off;
             for (int i = 0; i < mt; ++i)
-                p.mtiles[1 + toff + i] = make_int4(e, off + i * kBM, min(kBM, c - i * kBM), off + i * kBM);
+                p.mtiles[1 + toff + i] =
+                    make_int4(e, off + i * p.tile_rows, min(p.tile_rows, c - i * p.tile_rows), off + i * p.tile_rows);
         }
         run_rows += tot_rows;
         run_tiles += tot_tiles;
     }
     if (threadIdx.x == 0) p.offsets[p.E] = run_rows;
     // the shared expert: all T rows, in token order, after the routed rows
-    const int smt = (p.T + kBM - 1) / kBM;
+    const int tr = p.tile_rows;
+    const int smt = (p.T + tr - 1) / tr;
     for (int i = threadIdx.x; i < smt; i += blockDim.x)
-        p.mtiles[1 + run_tiles + i] = make_int4(p.E, p.T * p.K + i * kBM, min(kBM, p.T - i * kBM), i * kBM);
+        p.mtiles[1 + run_tiles + i] = make_int4(p.E, p.T * p.K + i * tr, min(tr, p.T - i * tr), i * tr);
     if (threadIdx.x == 0) p.mtiles[0] = make_int4(run_tiles + smt, run_tiles, 0, 0);
 }
 
@@ -830,6 +859,409 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
 }
 
+// ------------------------------------------------------------ narrow grouped GEMM
+//
+// For a few rows per expert the 128-row token tiles above are mostly padding.
+// Here the roles swap: the MMA's M is 128 weight rows (one 128-row scale
+// block of W13 or W2) and its N covers up to 32 rows of one group, so an item
+// streams one weight block once, whatever the group's row count.  The hi and
+// lo codes of the tile's rows are stacked as one 64-row B operand: one MMA
+// (M = 128, N = 64, K = 32) computes both terms into neighbouring accumulator
+// columns, and the weight tile is read from shared memory once per K step.
+// D[weight row][token] lands in TMEM with one lane per weight row; an
+// epilogue thread owns a weight row (an h column in GEMM1, an output column
+// in GEMM2) for all 32 tokens and, per 128-wide K block, adds
+// (activation scale x weight scale) x (hi + lo) in K-block order.
+
+constexpr int kNtEpiWarps = 4;                      // one per TMEM lane quadrant
+constexpr int kNtThreads = 64 + 32 * kNtEpiWarps;   // warp 0: TMA, warp 1: MMA + TMEM, warps 2..5: epilogue
+constexpr int kNtN = 2 * kNT;                       // MMA N: the tile's hi rows, then its lo rows
+constexpr uint32_t kNtTmemCols = 512;
+constexpr int kWB = 128;                            // weight rows per item (one scale block)
+constexpr int kNtPre = kNtMaxKb * kNT / (32 * kNtEpiWarps);  // activation scales per epilogue thread and item
+
+// TMEM columns per accumulator buffer (GEMM1: gate | up) and buffers.
+template <int MODE>
+__host__ __device__ constexpr int nt_acc_stride()
+{
+    return MODE == 1 ? 2 * kNtN : kNtN;
+}
+template <int MODE>
+__host__ __device__ constexpr int nt_acc_bufs()
+{
+    return (int)kNtTmemCols / nt_acc_stride<MODE>();
+}
+template <int MODE>
+__host__ __device__ constexpr size_t nt_stage_bytes()
+{
+    return (MODE == 1 ? 2 : 1) * (size_t)kWB * kBK + 2 * (size_t)kNT * kBK;  // weights (gate, up), rows hi, lo
+}
+template <int MODE>
+__host__ __device__ constexpr int nt_stages()
+{
+    return MODE == 1 ? 5 : 8;
+}
+template <int MODE>
+__host__ __device__ constexpr size_t nt_smem()
+{
+    return nt_stages<MODE>() * nt_stage_bytes<MODE>() + 1024;
+}
+
+struct NtItem {
+    int group, row0, rows, a_row0, nb, kdim, inter;
+    bool shared_grp;
+};
+
+// Item t = (group tile t / max_ntiles, weight block t % max_ntiles).
+template <int MODE>
+__device__ __forceinline__ bool nt_item(const GemmParams &p, int n_mtiles, int t, NtItem &ti)
+{
+    const int mt = t / p.max_ntiles;
+    ti.nb = t - mt * p.max_ntiles;
+    if (mt >= n_mtiles) return false;
+    const int4 m = __ldcg(p.mtiles + 1 + mt);
+    ti.group = m.x;
+    ti.row0 = m.y;
+    ti.rows = m.z;
+    ti.a_row0 = m.w;
+    ti.shared_grp = (m.x == p.E);
+    ti.inter = ti.shared_grp ? p.Is : p.I;
+    if (MODE == 1) {
+        ti.kdim = p.H;
+        return ti.nb < ti.inter / kWB;  // 128-column blocks of h
+    }
+    ti.kdim = ti.inter;
+    return true;                        // max_ntiles = H / 128 output blocks
+}
+
+// The first valid item at or after t, in steps of the grid (n_items if none).
+template <int MODE>
+__device__ __forceinline__ int nt_next(const GemmParams &p, int n_mtiles, int n_items, int t, NtItem &ti)
+{
+    while (t < n_items && !nt_item<MODE>(p, n_mtiles, t, ti)) t += gridDim.x;
+    return t;
+}
+
+// One epilogue thread's share of an item's scale tables (activation scales
+// [K block][row], the two weight-scale rows, GEMM2's blend weights), loaded
+// into registers while the previous item is computed.
+struct NtPre {
+    float sx[kNtPre];
+    float sw, wr;
+};
+
+template <int MODE>
+__device__ __forceinline__ void nt_prefetch(const GemmParams &p, const NtItem &ti, int et, NtPre &pr)
+{
+    const int nkb = ti.kdim / kBK;
+    const int arow0 = MODE == 1 ? ti.a_row0 : ti.row0;
+    const float *asc = (ti.shared_grp ? p.a_scales_shared : p.a_scales_routed) + (size_t)arow0 * p.a_scales_ld;
+    const float *wsc = ti.shared_grp
+                           ? p.w_scales_shared
+                           : p.w_scales + (size_t)ti.group * ((2 * p.I / 128) * (p.H / 128) + (p.H / 128) * (p.I / 128));
+    int wld, wn0, wn1;
+    if (MODE == 1) {
+        wld = p.H / 128;
+        wn0 = ti.nb;                    // gate block row
+        wn1 = ti.inter / 128 + ti.nb;   // up block row
+    } else {
+        wsc += (size_t)(2 * ti.inter / 128) * (p.H / 128);
+        wld = ti.inter / 128;
+        wn0 = wn1 = ti.nb;
+    }
+    const int j = et % kNT;  // this thread's row of the table
+#pragma unroll
+    for (int m = 0; m < kNtPre; ++m) {
+        const int kb = (et + 32 * kNtEpiWarps * m) / kNT;
+        pr.sx[m] = (kb < nkb && j < ti.rows) ? __ldg(asc + (size_t)j * p.a_scales_ld + kb) : 0.f;
+    }
+    pr.sw = et < nkb ? __ldg(wsc + (size_t)wn0 * wld + et)
+                     : (et < 2 * nkb ? __ldg(wsc + (size_t)wn1 * wld + et - nkb) : 0.f);
+    pr.wr = (MODE == 2 && et < ti.rows) ? __ldg(p.slot_w + (size_t)ti.row0 + et) : 0.f;
+}
+
+// MODE 1: item = h columns [128 nb, +128) of up to 32 rows: W13 gate rows
+// [128 nb, +128) and up rows [inter + 128 nb, +128) against x; epilogue
+// h = silu(gate) * up, quantised to hi/lo e4m3 with one scale per (row, 128
+// block), in the layout gemm_kernel<1> writes.  MODE 2: item = output
+// columns [128 nb, +128): W2 rows against h; epilogue x the row's blend
+// weight into its partial row.
+template <int MODE>
+__global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_constant__ GemmParams p)
+{
+    constexpr int kStages = nt_stages<MODE>();
+    constexpr uint32_t kSt = (uint32_t)nt_stage_bytes<MODE>();
+    constexpr uint32_t kAB = (MODE == 1 ? 2 : 1) * kWB * kBK;  // weight bytes of a stage
+    constexpr int kAccStride = nt_acc_stride<MODE>(), kAccBufs = nt_acc_bufs<MODE>();
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], acc_full[kAccBufs], acc_empty[kAccBufs];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ volatile int s_abort;
+    __shared__ __align__(16) float s_sx[kNtMaxKb * kNT];  // [kb][row]: the item's activation scales
+    __shared__ float s_sw[2 * kNtMaxKb];                  // the item's weight scales: gate row, up row
+    __shared__ float s_wrow[kNT];                         // GEMM2: blend weight per row
+    __shared__ float s_amax[4][kNT];                      // GEMM1: per-warp |h| maxima per row
+    __shared__ float s_inv[kNT], s_scl[kNT];
+    __shared__ __align__(16) uint8_t s_hq[2][kNT][kWB];   // GEMM1: h codes (hi, lo) staged for row stores
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kNtEpiWarps);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_s, kNtTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&p.a_routed);
+        tma_prefetch_desc(&p.a_shared);
+        tma_prefetch_desc(&p.b_routed);
+        tma_prefetch_desc(&p.b_shared);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    pdl_wait();
+    pdl_trigger();
+    const int n_mtiles = __ldcg(p.mtiles).x;
+    const int n_items = n_mtiles * p.max_ntiles;
+
+    if (warp == 0) {
+        // --------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();  // each weight block streams once per group tile
+            const uint64_t pol_a = policy_evict_last();   // a tile's rows are read for every weight block
+            int it = 0;
+            for (int t = blockIdx.x; t < n_items && !s_abort; t += gridDim.x) {
+                NtItem ti;
+                if (!nt_item<MODE>(p, n_mtiles, t, ti)) continue;
+                const int nkb = ti.kdim / kBK;
+                const CUtensorMap *amap = ti.shared_grp ? &p.a_shared : &p.a_routed;
+                const CUtensorMap *wmap = ti.shared_grp ? &p.b_shared : &p.b_routed;
+                const int ez = ti.shared_grp ? 0 : ti.group;
+                const int arow = MODE == 1 ? ti.a_row0 : ti.row0;
+                const int lo_x = MODE == 1 ? p.H : p.imax;  // where the lo half of an activation row starts
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kWaitLimitNs)) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        break;
+                    }
+                    unsigned char *st = smem + (size_t)s * kSt;
+                    mbar_arrive_expect_tx(&full[s], kSt);
+                    tma_load_3d(st, wmap, kb * kBK, ti.nb * kWB, ez, &full[s], pol_w);
+                    if (MODE == 1) tma_load_3d(st + kWB * kBK, wmap, kb * kBK, ti.inter + ti.nb * kWB, ez, &full[s], pol_w);
+                    // hi rows, then lo rows: together the 64-row B operand
+                    tma_load_2d(st + kAB, amap, kb * kBK, arow, &full[s], pol_a);
+                    tma_load_2d(st + kAB + kNT * kBK, amap, lo_x + kb * kBK, arow, &full[s], pol_a);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_e4m3_f32(kWB, kNtN);
+            int it = 0, acc_it = 0;
+            for (int t = blockIdx.x; t < n_items && !s_abort; t += gridDim.x) {
+                NtItem ti;
+                if (!nt_item<MODE>(p, n_mtiles, t, ti)) continue;
+                const int nkb = ti.kdim / kBK;
+                for (int kb = 0; kb < nkb; ++kb, ++it, ++acc_it) {
+                    const int s = it % kStages;
+                    const int b = acc_it % kAccBufs;
+                    if (!mbar_wait(&full[s], (it / kStages) & 1, kWaitLimitNs) ||
+                        (acc_it >= kAccBufs && !mbar_wait(&acc_empty[b], ((acc_it / kAccBufs) - 1) & 1, kWaitLimitNs))) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + (size_t)s * kSt);
+                    const uint32_t bsm = st + kAB;
+                    const uint32_t d = tmem_base + (uint32_t)(b * kAccStride);
+#pragma unroll
+                    for (int k4 = 0; k4 < kBK / 32; ++k4) {
+                        const uint32_t acc = k4 ? 1u : 0u;
+                        umma_f8f6f4(d, umma_desc_sw128(st + k4 * 32), umma_desc_sw128(bsm + k4 * 32), idesc, acc);
+                        if (MODE == 1)
+                            umma_f8f6f4(d + kNtN, umma_desc_sw128(st + kWB * kBK + k4 * 32), umma_desc_sw128(bsm + k4 * 32),
+                                        idesc, acc);
+                    }
+                    umma_commit(&empty[s]);
+                    umma_commit(&acc_full[b]);
+                }
+            }
+        }
+    } else {
+        // --------------------------------------------------- epilogue (warps 2..5)
+        const int q = warp & 3;        // TMEM lane quadrant
+        const int r = q * 32 + lane;   // weight row within the block
+        const int et = threadIdx.x - 64;
+        int acc_it = 0;
+        bool ok = true;
+        NtItem cur;
+        int t = nt_next<MODE>(p, n_mtiles, n_items, blockIdx.x, cur);
+        NtPre pre;
+        if (t < n_items) nt_prefetch<MODE>(p, cur, et, pre);
+        while (t < n_items) {
+            NtItem nxt;
+            const int tn = nt_next<MODE>(p, n_mtiles, n_items, t + gridDim.x, nxt);
+            const int nkb = cur.kdim / kBK;
+            // the item's scale tables into shared memory, then the next item's loads
+            named_barrier(1, 32 * kNtEpiWarps);
+#pragma unroll
+            for (int m = 0; m < kNtPre; ++m) {
+                const int i = et + 32 * kNtEpiWarps * m;
+                if (i < nkb * kNT) s_sx[i] = pre.sx[m];
+            }
+            if (et < 2 * nkb) s_sw[et] = pre.sw;
+            if (MODE == 2 && et < kNT) s_wrow[et] = pre.wr;
+            named_barrier(1, 32 * kNtEpiWarps);
+            if (tn < n_items) nt_prefetch<MODE>(p, nxt, et, pre);
+
+            float g[kNT], u[kNT];  // GEMM2 uses g only
+#pragma unroll
+            for (int j = 0; j < kNT; ++j) g[j] = u[j] = 0.f;
+            for (int kb = 0; kb < nkb; ++kb, ++acc_it) {
+                const int b = acc_it % kAccBufs;
+                if (ok) {
+                    const bool w = mbar_wait(&acc_full[b], (acc_it / kAccBufs) & 1, kWaitLimitNs);
+                    if (!__all_sync(0xFFFFFFFFu, w)) {
+                        set_status(p.counters, MOE_ETIMEOUT);
+                        s_abort = 1;
+                        ok = false;
+                    }
+                }
+                if (!ok) continue;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kAccStride);
+                const float sw0 = s_sw[kb], sw1 = s_sw[nkb + kb];
+                const float4 *sx4 = reinterpret_cast<const float4 *>(s_sx + kb * kNT);
+                if (MODE == 1) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {  // rows [16 h, +16)
+                        float gh[16], gl[16], uh[16], ul[16];
+                        tmem_ld_32x16(tb + 16 * h, gh);
+                        tmem_ld_32x16(tb + kNT + 16 * h, gl);
+                        tmem_ld_32x16(tb + kNtN + 16 * h, uh);
+                        tmem_ld_32x16(tb + kNtN + kNT + 16 * h, ul);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const float4 sx = sx4[4 * h + j4];
+                            const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const int i = 4 * j4 + c, j = 16 * h + i;
+                                g[j] = fmaf(sxa[c] * sw0, gh[i] + gl[i], g[j]);
+                                u[j] = fmaf(sxa[c] * sw1, uh[i] + ul[i], u[j]);
+                            }
+                        }
+                    }
+                } else {
+                    float vh[kNT], vl[kNT];
+                    tmem_ld_32x32(tb, vh);
+                    tmem_ld_32x32(tb + kNT, vl);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j4 = 0; j4 < kNT / 4; ++j4) {
+                        const float4 sx = sx4[j4];
+                        const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int j = 4 * j4 + c;
+                            g[j] = fmaf(sxa[c] * sw0, vh[j] + vl[j], g[j]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+            }
+            if (MODE == 1) {
+                // h = silu(gate) * up; the 128 columns of the block share one
+                // scale per row: max |h| over the warp by recursive halving
+                // (lane j ends with row j's maximum), then over the 4 warps
+                float m[kNT];
+#pragma unroll
+                for (int j = 0; j < kNT; ++j) {
+                    const float hv = g[j] * __frcp_rn(1.f + __expf(-g[j])) * u[j];
+                    g[j] = hv;
+                    m[j] = fabsf(hv);
+                }
+#pragma unroll
+                for (int w = kNT / 2; w >= 1; w >>= 1) {
+                    const bool upper = (lane & w) != 0;
+#pragma unroll
+                    for (int i = 0; i < w; ++i) {
+                        const float send = upper ? m[i] : m[i + w];
+                        const float keep = upper ? m[i + w] : m[i];
+                        m[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, w));
+                    }
+                }
+                s_amax[q][lane] = m[0];
+                named_barrier(1, 32 * kNtEpiWarps);
+                if (q == 0) {
+                    const float a = fmaxf(fmaxf(s_amax[0][lane], s_amax[1][lane]), fmaxf(s_amax[2][lane], s_amax[3][lane]));
+                    const float sc = a > 0.f ? a / 448.f : 1.f;
+                    s_scl[lane] = sc;
+                    s_inv[lane] = 1.f / sc;
+                }
+                named_barrier(1, 32 * kNtEpiWarps);
+#pragma unroll
+                for (int j = 0; j < kNT; j += 2) {
+                    const float a = g[j] * s_inv[j], c = g[j + 1] * s_inv[j + 1];
+                    const uint16_t hh = f32x2_to_e4m3x2(a, c);
+                    const float2 f = e4m3x2_to_f32x2(hh);
+                    const uint16_t ll = f32x2_to_e4m3x2(a - f.x, c - f.y);
+                    s_hq[0][j][r] = (uint8_t)(hh & 0xFF);
+                    s_hq[0][j + 1][r] = (uint8_t)(hh >> 8);
+                    s_hq[1][j][r] = (uint8_t)(ll & 0xFF);
+                    s_hq[1][j + 1][r] = (uint8_t)(ll >> 8);
+                }
+                named_barrier(1, 32 * kNtEpiWarps);
+                // rows of 128 codes out as 16-byte pieces
+                for (int i = et; i < 2 * kNT * (kWB / 16); i += 32 * kNtEpiWarps) {
+                    const int part = i / (kNT * (kWB / 16));
+                    const int j = (i / (kWB / 16)) % kNT, ch = i % (kWB / 16);
+                    if (j < cur.rows)
+                        *reinterpret_cast<uint4 *>(p.hq + ((size_t)cur.row0 + j) * 2 * p.imax + (part ? p.imax : 0) +
+                                                   cur.nb * kWB + ch * 16) =
+                            *reinterpret_cast<const uint4 *>(&s_hq[part][j][ch * 16]);
+                }
+                if (q == 0 && lane < cur.rows) p.hs[((size_t)cur.row0 + lane) * (p.imax / 128) + cur.nb] = s_scl[lane];
+            } else if (ok) {
+                // a warp stores 32 consecutive floats of each row's partial row
+                float *dst = p.yslot + (size_t)cur.row0 * p.H + cur.nb * kWB + r;
+#pragma unroll
+                for (int j = 0; j < kNT; ++j)
+                    if (j < cur.rows) dst[(size_t)j * p.H] = s_wrow[j] * g[j];
+            }
+            t = tn;
+            cur = nxt;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kNtTmemCols);
+    }
+}
+
 // ------------------------------------------------------------ blend
 
 struct BlendParams {
@@ -935,11 +1367,12 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
                     const uint8_t *expert_w8, const float *expert_scales, const uint8_t *shared_w8,
                     const float *shared_scales, const uint16_t *shared_gate, uint16_t *out,
                     const uint16_t *residual, const float *router_bias, void *ws, cudaStream_t s,
-                    int32_t *topk_idx_out, float *topk_w_out, float *gsig_out)
+                    int32_t *topk_idx_out, float *topk_w_out, float *gsig_out, bool narrow)
 {
     const int T = rows, E = d.n_experts, K = d.top_k, H = d.hidden, I = d.inter, Is = d.shared_inter;
     const int imax = std::max(I, Is);
     if (H % kBK) return MOE_EUNSUPPORTED;
+    if (narrow && !narrow_supported(d)) return MOE_EUNSUPPORTED;
     const PrefillLayout L = prefill_layout(d, T);
     char *base = static_cast<char *>(ws);
     int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
@@ -949,8 +1382,12 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     const DeviceInfo &di = device_info();
     const int P = T * K;
 
-    cudaError_t e = cudaMemsetAsync(base + L.counts, 0, sizeof(int32_t) * (E + 1), s);
-    if (e != cudaSuccess) return MOE_ECUDA;
+    // few rows: the decode router over many CTAs; else the tcgen05 router,
+    // which also counts each expert's rows
+    const bool small_router = T <= MOE_DECODE_MAX_ROWS;
+    cudaError_t e = cudaSuccess;
+    if (!small_router && (e = cudaMemsetAsync(base + L.counts, 0, sizeof(int32_t) * (E + 1), s)) != cudaSuccess)
+        return MOE_ECUDA;
 
     PlanParams pp;
     pp.T = T;
@@ -967,6 +1404,8 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     pp.rank = reinterpret_cast<int32_t *>(base + L.rank);
     pp.pos = reinterpret_cast<int32_t *>(base + L.pos);
     pp.mtiles = reinterpret_cast<int4 *>(base + L.mtiles);
+    pp.tile_rows = narrow ? kNT : kBM;
+    pp.count_in_scan = small_router ? 1 : 0;
     pp.x = x;
     pp.xp_shared0 = std::max(P, kBM);
     pp.xp = reinterpret_cast<uint8_t *>(base + L.xp);
@@ -974,31 +1413,49 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     pp.slot_w = reinterpret_cast<float *>(base + L.slot_w);
     pp.counters = counters;
 
-    // 1. router + top-k + per-expert ranks
-    RouterTcParams rp{};
-    rp.T = T;
-    rp.E = E;
-    rp.K = K;
-    rp.H = H;
-    rp.nbox = std::min(kRtChunk, (E + 15) / 16 * 16);
-    rp.bias = router_bias;
-    rp.topk_idx = tidx;
-    rp.topk_w = tw;
-    rp.gsig = gs;
-    rp.counts = pp.counts;
-    rp.rank = pp.rank;
-    rp.counters = counters;
-    if (!make_map(&rp.x, x, 2 * (uint64_t)H, (uint64_t)T, 1, 2 * (uint64_t)H, 0, kBM) ||
-        !make_map(&rp.wr, router_w, 2 * (uint64_t)H, (uint64_t)E, 1, 2 * (uint64_t)H, 0, (uint32_t)rp.nbox) ||
-        !make_map(&rp.g, shared_gate, 2 * (uint64_t)H, 1, 1, 2 * (uint64_t)H, 0, 16))
-        return MOE_ECUDA;
-    const unsigned rt_grid = (unsigned)std::min<int64_t>(di.sm_count, (T + kBM - 1) / kBM);
-    if (K <= 2) e = launch_router_tc<2>(rt_grid, rp, s);
-    else if (K <= 4) e = launch_router_tc<4>(rt_grid, rp, s);
-    else if (K <= 8) e = launch_router_tc<8>(rt_grid, rp, s);
-    else if (K <= 16) e = launch_router_tc<16>(rt_grid, rp, s);
-    else e = launch_router_tc<32>(rt_grid, rp, s);
-    if (e != cudaSuccess) return MOE_ECUDA;
+    // 1. router + top-k (+ per-expert ranks)
+    if (small_router) {
+        RouterLaunch ra{};
+        ra.d = &d;
+        ra.x = x;
+        ra.rows = T;
+        ra.router_w = router_w;
+        ra.router_bias = router_bias;
+        ra.shared_gate = shared_gate;
+        ra.topk_idx = tidx;
+        ra.topk_w = tw;
+        ra.gsig = gs;
+        ra.logits = reinterpret_cast<float *>(base + L.logits);
+        ra.xq = nullptr;  // the permute kernel quantises x
+        ra.xsc = nullptr;
+        ra.counters = counters;
+        if (launch_router_topk(ra, s) != cudaSuccess) return MOE_ECUDA;
+    } else {
+        RouterTcParams rp{};
+        rp.T = T;
+        rp.E = E;
+        rp.K = K;
+        rp.H = H;
+        rp.nbox = std::min(kRtChunk, (E + 15) / 16 * 16);
+        rp.bias = router_bias;
+        rp.topk_idx = tidx;
+        rp.topk_w = tw;
+        rp.gsig = gs;
+        rp.counts = pp.counts;
+        rp.rank = pp.rank;
+        rp.counters = counters;
+        if (!make_map(&rp.x, x, 2 * (uint64_t)H, (uint64_t)T, 1, 2 * (uint64_t)H, 0, kBM) ||
+            !make_map(&rp.wr, router_w, 2 * (uint64_t)H, (uint64_t)E, 1, 2 * (uint64_t)H, 0, (uint32_t)rp.nbox) ||
+            !make_map(&rp.g, shared_gate, 2 * (uint64_t)H, 1, 1, 2 * (uint64_t)H, 0, 16))
+            return MOE_ECUDA;
+        const unsigned rt_grid = (unsigned)std::min<int64_t>(di.sm_count, (T + kBM - 1) / kBM);
+        if (K <= 2) e = launch_router_tc<2>(rt_grid, rp, s);
+        else if (K <= 4) e = launch_router_tc<4>(rt_grid, rp, s);
+        else if (K <= 8) e = launch_router_tc<8>(rt_grid, rp, s);
+        else if (K <= 16) e = launch_router_tc<16>(rt_grid, rp, s);
+        else e = launch_router_tc<32>(rt_grid, rp, s);
+        if (e != cudaSuccess) return MOE_ECUDA;
+    }
 
     // 2, 3
     if ((e = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pp)) != cudaSuccess) return MOE_ECUDA;
@@ -1023,11 +1480,13 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     g.counters = counters;
     const int64_t R = L.rows_total;
     // A tensors are declared with at least 128 rows (their buffers are that
-    // large); rows past the valid ones are read but never stored.
+    // large); rows past the valid ones are read but never stored.  The narrow
+    // GEMMs read activation boxes of kNT rows.
+    const uint32_t abox = narrow ? kNT : kBM;
     bool ok = make_map(&g.a_routed, pp.xp, 2 * (uint64_t)H, (uint64_t)std::max<int64_t>(L.routed, kBM), 1,
-                       2 * (uint64_t)H, 0, kBM) &&
+                       2 * (uint64_t)H, 0, abox) &&
               make_map(&g.a_shared, pp.xp + (size_t)pp.xp_shared0 * 2 * H, 2 * (uint64_t)H,
-                       (uint64_t)std::max(T, kBM), 1, 2 * (uint64_t)H, 0, kBM) &&
+                       (uint64_t)std::max(T, kBM), 1, 2 * (uint64_t)H, 0, abox) &&
               make_map(&g.b_routed, expert_w8, (uint64_t)H, 2 * (uint64_t)I, (uint64_t)E, (uint64_t)H,
                        3 * (uint64_t)I * H, 128) &&
               make_map(&g.b_shared, shared_w8, (uint64_t)H, 2 * (uint64_t)Is, 1, (uint64_t)H, 3 * (uint64_t)Is * H, 128);
@@ -1036,26 +1495,39 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     g.a_scales_shared = pp.xps + (size_t)P * (H / 128);
     g.a_scales_ld = H / 128;
     g.max_ntiles = imax / 128;
-    if (!gemm_occupancy_once(gemm_kernel<1>) || !gemm_occupancy_once(gemm_kernel<2>)) return MOE_ECUDA;
-    if ((e = launch_kernel(gemm_kernel<1>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g)) != cudaSuccess)
-        return MOE_ECUDA;
+    if (narrow) {
+        if (!gemm_occupancy_once(gemm_nt_kernel<1>, nt_smem<1>()) ||
+            !gemm_occupancy_once(gemm_nt_kernel<2>, nt_smem<2>()))
+            return MOE_ECUDA;
+        e = launch_kernel(gemm_nt_kernel<1>, dim3(di.sm_count), dim3(kNtThreads), nt_smem<1>(), s, g);
+    } else {
+        if (!gemm_occupancy_once(gemm_kernel<1>) || !gemm_occupancy_once(gemm_kernel<2>)) return MOE_ECUDA;
+        e = launch_kernel(gemm_kernel<1>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g);
+    }
+    if (e != cudaSuccess) return MOE_ECUDA;
 
     // 5. GEMM2
     GemmParams g2 = g;
     const uint64_t Rp = (uint64_t)std::max<int64_t>(R, kBM);
-    ok = make_map(&g2.a_routed, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, kBM) &&
-         make_map(&g2.a_shared, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, kBM) &&
+    const uint32_t wbox = narrow ? kWB : kBN;  // W2 rows per box: one 128-row block, or a 256-column tile
+    ok = make_map(&g2.a_routed, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, abox) &&
+         make_map(&g2.a_shared, g.hq, 2 * (uint64_t)imax, Rp, 1, 2 * (uint64_t)imax, 0, abox) &&
          make_map(&g2.b_routed, expert_w8 + (size_t)2 * I * H, (uint64_t)I, (uint64_t)H, (uint64_t)E, (uint64_t)I,
-                  3 * (uint64_t)I * H, kBN) &&
+                  3 * (uint64_t)I * H, wbox) &&
          make_map(&g2.b_shared, shared_w8 + (size_t)2 * Is * H, (uint64_t)Is, (uint64_t)H, 1, (uint64_t)Is,
-                  3 * (uint64_t)Is * H, kBN);
+                  3 * (uint64_t)Is * H, wbox);
     if (!ok) return MOE_ECUDA;
     g2.a_scales_routed = g.hs;
     g2.a_scales_shared = g.hs;
     g2.a_scales_ld = imax / 128;
-    g2.max_ntiles = (H + kBN - 1) / kBN;
-    if ((e = launch_kernel(gemm_kernel<2>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g2)) != cudaSuccess)
-        return MOE_ECUDA;
+    if (narrow) {
+        g2.max_ntiles = H / kWB;
+        e = launch_kernel(gemm_nt_kernel<2>, dim3(di.sm_count), dim3(kNtThreads), nt_smem<2>(), s, g2);
+    } else {
+        g2.max_ntiles = (H + kBN - 1) / kBN;
+        e = launch_kernel(gemm_kernel<2>, dim3(di.sm_count), dim3(kGemmThreads), kGemmSmem, s, g2);
+    }
+    if (e != cudaSuccess) return MOE_ECUDA;
 
     // 6. blend
     BlendParams bp;

@@ -87,6 +87,23 @@ def test_argument_checks_on_host(L):
                              None) == moe.MOE_EINVAL
 
 
+def test_paths_and_launch_counts(L):
+    d = D()
+    assert moe.kernel_launches(d, 0) == 0
+    assert moe.kernel_launches(d, moe.MOE_AUTO_DECODE_MAX_ROWS) == 3
+    assert moe.kernel_launches(d, moe.MOE_AUTO_DECODE_MAX_ROWS + 1) == 6
+    for path, n in ((moe.MOE_PATH_DECODE, 3), (moe.MOE_PATH_PREFILL, 6), (moe.MOE_PATH_PREFILL_NARROW, 6)):
+        assert moe.kernel_launches(d, 5, path) == n
+    assert moe.kernel_launches(d, 5, 4) == 0                  # no such path
+    assert moe.auto_path(d, 1) == moe.MOE_PATH_DECODE
+    assert moe.auto_path(d, 4096) == moe.MOE_PATH_PREFILL
+    assert moe.auto_path(d, -1) == moe.MOE_EINVAL
+    # the narrow GEMMs hold at most 64 K blocks of scales per item: refused
+    # on the host before any device call
+    assert fwd(L, D(h=8320), path=moe.MOE_PATH_PREFILL_NARROW) == moe.MOE_EUNSUPPORTED
+    assert fwd(L, D(i=8320), path=moe.MOE_PATH_PREFILL_NARROW) == moe.MOE_EUNSUPPORTED
+
+
 def test_fault_knob_is_sticky_until_reset(L):
     d = D()
     moe.reset_status()

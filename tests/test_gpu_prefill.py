@@ -1,5 +1,6 @@
 """GPU parity of the prefill path (token permute -> tcgen05 FP8 grouped GEMMs
--> unpermute) against the CPU oracle, through the C ABI.
+-> unpermute), with 128-row token tiles and with the narrow tiling (128
+weight rows x up to 32 token rows), against the CPU oracle, through the C ABI.
 
 Small shapes are checked on every row; the 4096-row Qwen3.6-35B-A3B-shaped
 prefill (router bias for uneven expert loads) is checked on its routing for
@@ -127,3 +128,55 @@ def test_prefill_hidden_odd_multiple_of_128(dims, rows):
                                           router_bias=case.layer.router_bias)
     P.check_routing(case, idx, w, gs, ow, ogs)
     P.compare_output(case, out, idx)
+
+
+# ---------------------------------------------------------------- narrow grouped GEMMs
+# Weight rows as the MMA's M (128) and up to 32 rows of one group as its N.
+
+@pytest.mark.parametrize("dims,rows,bias", [
+    (mi.TINY, 4, False),
+    (mi.TINY, 300, True),     # several 32-row tiles per group, uneven loads
+    (mi.LayerDims(hidden=512, n_experts=32, top_k=4, inter=256, shared_inter=256), 70, True),
+    (mi.LayerDims(hidden=256, n_experts=16, top_k=2, inter=128, shared_inter=256), 45, False),   # I != Is
+    (mi.LayerDims(hidden=384, n_experts=12, top_k=3, inter=256, shared_inter=128), 33, True),    # H/128 odd
+    (mi.LayerDims(hidden=640, n_experts=20, top_k=4, inter=384, shared_inter=128), 17, False),
+])
+def test_narrow_small_shapes(dims, rows, bias):
+    case = P.build_case(dims, rows, router_bias=bias, all_experts=True, residual=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL_NARROW)
+    _, oidx, ow, ogs = oracle.router_topk(dims, case.x, case.layer.router_w, case.layer.shared_gate,
+                                          router_bias=case.layer.router_bias)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
+
+
+@pytest.mark.parametrize("rows", [1, 2, 8, 16, 32, 64])
+def test_qwen36_35b_narrow(rows):
+    d = mi.QWEN36_35B_A3B
+    case = P.build_case(d, rows)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL_NARROW)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
+
+
+def test_qwen35_397b_narrow_rows_32():
+    d = mi.QWEN35_397B_A17B
+    case = P.build_case(d, 32)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL_NARROW)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
+
+
+def test_narrow_matches_wide_tiles_on_the_same_routing():
+    # both tilings compute each (row, column) with the same per-K-block
+    # promotion; only the tensor cores' summation inside a K block may differ
+    d = mi.LayerDims(hidden=512, n_experts=32, top_k=4, inter=256, shared_inter=256)
+    case = P.build_case(d, 150, router_bias=True, all_experts=True)
+    dev = P.device_weights(case.layer)
+    a, ia, _, _ = run(case, moe.MOE_PATH_PREFILL, dev)
+    b, ib, _, _ = run(case, moe.MOE_PATH_PREFILL_NARROW, dev)
+    assert np.array_equal(ia, ib)
+    rel = np.linalg.norm(a - b) / np.linalg.norm(a)
+    assert rel < 2e-3, rel
