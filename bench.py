@@ -650,7 +650,8 @@ def run_ours(args, dist: Dist):
                             "hbm_frac_of_measured": round(gbs64 / dist.world / hbm_peak, 4),
                             "tokens_per_s": round(aggregate(k64 * r64, dist.world, s64), 1),
                             "distinct_experts_per_step": round(u64, 1), "steps": k64,
-                            "kernels": "decode" if moe.kernel_launches(d, r64) == 3 else "prefill"}
+                            "kernels": {moe.MOE_PATH_DECODE: "decode", moe.MOE_PATH_PREFILL: "grouped",
+                                        moe.MOE_PATH_PREFILL_NARROW: "narrow"}[moe.auto_path(d, r64)]}
 
     # ---- prefill, 4096 tokens
     result["prefill"] = prefill_leg(args, d, insts[0], dist, bus, hbm_peak, bf16_peak, peak_kind)
@@ -728,7 +729,8 @@ def run_reference(args, dist: Dist):
 
 def run_sweep(args, dist: Dist):
     """Every row count of the decode workloads (35B-A3B-shaped rows 1, 2, 8,
-    16, 32, 64, with 128 and 256 beside them; 397B-A17B-shaped rows 1 and 32)
+    16, 32, 64, with 4 and 128 to 1024 beside them; 397B-A17B-shaped rows 1
+    and 32, with 4 and 256)
     on each path that takes it: the decode kernels (up to 64 rows), the
     grouped GEMMs with 128-row token tiles, and the narrow grouped GEMMs;
     each line says whether it is the path MOE_PATH_AUTO takes.  CUDA events
@@ -742,8 +744,8 @@ def run_sweep(args, dist: Dist):
     names = {moe.MOE_PATH_DECODE: "decode", moe.MOE_PATH_PREFILL: "grouped", moe.MOE_PATH_PREFILL_NARROW: "narrow"}
     res = []
     for dims, name, rows_list, n_inst in ((mi.QWEN36_35B_A3B, "Qwen3.6-35B-A3B-shaped",
-                                           [1, 2, 8, 16, 32, 64, 128, 256], 16),
-                                          (mi.QWEN35_397B_A17B, "Qwen3.5-397B-A17B-shaped", [1, 32], 2)):
+                                           [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024], 16),
+                                          (mi.QWEN35_397B_A17B, "Qwen3.5-397B-A17B-shaped", [1, 4, 32, 256], 2)):
         insts = make_instances(mi.make_layer(dims, seed=args.seed), n_inst)
         for rows in rows_list:
             xs = [torch.from_numpy(mi.make_x(dims, rows, seed=args.seed + 1, stream=1000 * rows + i).view("int16"))

@@ -77,16 +77,19 @@ extern "C" {
 #define MOE_ECUDA -4         /* a CUDA launch or runtime error (sticky) */
 #define MOE_ETIMEOUT -5      /* a bounded wait inside a kernel ran out (device status word) */
 
-#define MOE_PATH_AUTO 0      /* decode kernels for rows <= MOE_AUTO_DECODE_MAX_ROWS, else prefill */
+#define MOE_PATH_AUTO 0      /* by rows: MOE_AUTO_DECODE_MAX_ROWS, MOE_AUTO_NARROW_MAX_PAIRS below */
 #define MOE_PATH_DECODE 1    /* FP8 weight-streaming GEMVs (16-row tensor-core tiles) with expert dedup */
 #define MOE_PATH_PREFILL 2   /* token permute -> tcgen05 FP8 grouped GEMMs -> unpermute */
 #define MOE_PATH_PREFILL_NARROW 3  /* the same pipeline with the grouped GEMMs tiled as 128 weight rows (the
                                      MMA's M) x up to 32 rows of one expert (its N): for few rows per expert;
                                      MOE_EUNSUPPORTED when H, I or Is exceeds 4096 */
 #define MOE_DECODE_MAX_ROWS 64       /* the decode path's tiles are sized for at most this many rows */
-#define MOE_AUTO_DECODE_MAX_ROWS 12  /* MOE_PATH_AUTO's switch to the prefill path (the two paths
-                                        measured equal between 8 and 16 rows of a 35B-A3B-shaped
-                                        layer on B200; above, the grouped GEMMs are faster) */
+#define MOE_AUTO_DECODE_MAX_ROWS 3    /* MOE_PATH_AUTO: the decode kernels up to this many rows; then the
+                                         narrow grouped GEMMs while rows * k <= MOE_AUTO_NARROW_MAX_PAIRS * E
+                                         (an expert's average routed rows), then the 128-row token tiles;
+                                         the switch points were measured on B200 with every path timed on
+                                         the 35B-A3B- and 397B-A17B-shaped layers */
+#define MOE_AUTO_NARROW_MAX_PAIRS 16
 
 typedef struct moe_dims {
     int32_t hidden;       /* H  */
@@ -120,7 +123,7 @@ MOE_API int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows,
 
 /* The whole layer step: out = sum_r w_r E_{idx_r}(x) + sigmoid(g.x) E_shared(x)
  * (+ residual), bf16 [rows, H].  residual and router_bias may be NULL.
- * Chooses the decode path for rows <= MOE_AUTO_DECODE_MAX_ROWS, else prefill.
+ * Chooses the path by rows, as MOE_PATH_AUTO describes (moe_auto_path tells which).
  * rows == 0 is a no-op (pointers may then be NULL). */
 MOE_API int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows,
                     const uint16_t *router_w, const uint8_t *expert_w8,

@@ -74,11 +74,15 @@ bool valid_path(int32_t path)
            path == MOE_PATH_PREFILL_NARROW;
 }
 
-// MOE_PATH_AUTO's choice for a row count.
+// MOE_PATH_AUTO's choice for a row count: the decode kernels for a few
+// rows, the narrow grouped GEMMs while an expert averages at most
+// MOE_AUTO_NARROW_MAX_PAIRS routed rows, the 128-row token tiles above.
 int32_t resolve_path(const moe_dims &d, int32_t rows, int32_t path)
 {
     if (path != MOE_PATH_AUTO) return path;
     if (rows <= MOE_AUTO_DECODE_MAX_ROWS || !prefill_available()) return MOE_PATH_DECODE;
+    if (narrow_supported(d) && (int64_t)rows * d.top_k <= (int64_t)MOE_AUTO_NARROW_MAX_PAIRS * d.n_experts)
+        return MOE_PATH_PREFILL_NARROW;
     return MOE_PATH_PREFILL;
 }
 

@@ -871,10 +871,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 // D[weight row][token] lands in TMEM with one lane per weight row; an
 // epilogue thread owns a weight row (an h column in GEMM1, an output column
 // in GEMM2) for all 32 tokens and, per 128-wide K block, adds
-// (activation scale x weight scale) x (hi + lo) in K-block order.
+// (activation scale x weight scale) x (hi + lo) in K-block order.  Two
+// epilogue warpgroups take the items in turn, so that one group's item tail
+// (GEMM1: silu, the per-row scale, quantisation and the h stores) overlaps
+// the other group's accumulation.
 
-constexpr int kNtEpiWarps = 4;                      // one per TMEM lane quadrant
-constexpr int kNtThreads = 64 + 32 * kNtEpiWarps;   // warp 0: TMA, warp 1: MMA + TMEM, warps 2..5: epilogue
+constexpr int kNtEpiWarps = 4;                      // per group: one per TMEM lane quadrant
+constexpr int kNtEpiGroups = 2;
+constexpr int kNtThreads = 64 + 32 * kNtEpiWarps * kNtEpiGroups;  // warp 0: TMA, warp 1: MMA + TMEM, 2..9: epilogue
 constexpr int kNtN = 2 * kNT;                       // MMA N: the tile's hi rows, then its lo rows
 constexpr uint32_t kNtTmemCols = 512;
 constexpr int kWB = 128;                            // weight rows per item (one scale block)
@@ -995,14 +999,23 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
     constexpr int kAccStride = nt_acc_stride<MODE>(), kAccBufs = nt_acc_bufs<MODE>();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages], acc_full[kAccBufs], acc_empty[kAccBufs];
+    // phase s completes once the group owning item s has received all of
+    // its accumulators; the owner of item s + 1 waits for it before its
+    // first accumulator wait, so no waiter on acc_full runs more than one
+    // phase ahead of the barrier (a parity wait two phases ahead would pass
+    // at once)
+    __shared__ __align__(8) uint64_t handoff;
     __shared__ uint32_t tmem_base_s;
     __shared__ volatile int s_abort;
-    __shared__ __align__(16) float s_sx[kNtMaxKb * kNT];  // [kb][row]: the item's activation scales
-    __shared__ float s_sw[2 * kNtMaxKb];                  // the item's weight scales: gate row, up row
-    __shared__ float s_wrow[kNT];                         // GEMM2: blend weight per row
-    __shared__ float s_amax[4][kNT];                      // GEMM1: per-warp |h| maxima per row
-    __shared__ float s_inv[kNT], s_scl[kNT];
-    __shared__ __align__(16) uint8_t s_hq[2][kNT][kWB];   // GEMM1: h codes (hi, lo) staged for row stores
+    // per epilogue group: the item's tables and staging
+    __shared__ __align__(16) float s_sx[kNtEpiGroups][kNtMaxKb * kNT];  // [kb][row]: activation scales
+    __shared__ float s_sw[kNtEpiGroups][2 * kNtMaxKb];                  // weight scales: gate row, up row
+    __shared__ float s_wrow[kNtEpiGroups][MODE == 2 ? kNT : 1];         // GEMM2: blend weight per row
+    __shared__ float s_inv[kNtEpiGroups][kNT], s_scl[kNtEpiGroups][kNT];
+    // GEMM1: h codes (hi, lo) staged for row stores; its first 512 bytes
+    // also carry the per-warp |h| maxima, which are read before the codes
+    // are written
+    __shared__ __align__(16) uint8_t s_hq[kNtEpiGroups][2][kNT][kWB];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
 
@@ -1014,8 +1027,9 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
         }
         for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kNtEpiWarps);
+            mbar_init(&acc_empty[b], kNtEpiWarps);  // the four warps of the group that owns the item
         }
+        mbar_init(&handoff, kNtEpiWarps);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -1106,35 +1120,58 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
             }
         }
     } else {
-        // --------------------------------------------------- epilogue (warps 2..5)
+        // --------------------------------------------------- epilogue (warps 2..9)
+        // Group eg takes the items at even (eg = 0) or odd (eg = 1) places of
+        // this CTA's sequence and skips the other group's K blocks.
+        const int eg = (warp - 2) / kNtEpiWarps;
         const int q = warp & 3;        // TMEM lane quadrant
         const int r = q * 32 + lane;   // weight row within the block
-        const int et = threadIdx.x - 64;
+        const int et = (warp - 2 - eg * kNtEpiWarps) * 32 + lane;
+        const int bar = 1 + eg;        // the group's named barrier
+        constexpr int kGT = 32 * kNtEpiWarps;
+        float *sx_tab = s_sx[eg];
+        float *sw_tab = s_sw[eg];
+        float(*amax_tab)[kNT] = reinterpret_cast<float(*)[kNT]>(&s_hq[eg][0][0][0]);
         int acc_it = 0;
+        int seq = eg;  // place of `cur` in this CTA's item sequence
         bool ok = true;
         NtItem cur;
         int t = nt_next<MODE>(p, n_mtiles, n_items, blockIdx.x, cur);
+        if (eg == 1 && t < n_items) {
+            acc_it += cur.kdim / kBK;
+            t = nt_next<MODE>(p, n_mtiles, n_items, t + gridDim.x, cur);
+        }
         NtPre pre;
         if (t < n_items) nt_prefetch<MODE>(p, cur, et, pre);
         while (t < n_items) {
-            NtItem nxt;
-            const int tn = nt_next<MODE>(p, n_mtiles, n_items, t + gridDim.x, nxt);
+            // the other group's item, then this group's next one
+            NtItem mid, nxt;
+            const int tm = nt_next<MODE>(p, n_mtiles, n_items, t + gridDim.x, mid);
+            const int tn = tm < n_items ? nt_next<MODE>(p, n_mtiles, n_items, tm + gridDim.x, nxt) : n_items;
             const int nkb = cur.kdim / kBK;
             // the item's scale tables into shared memory, then the next item's loads
-            named_barrier(1, 32 * kNtEpiWarps);
+            named_barrier(bar, kGT);
 #pragma unroll
             for (int m = 0; m < kNtPre; ++m) {
-                const int i = et + 32 * kNtEpiWarps * m;
-                if (i < nkb * kNT) s_sx[i] = pre.sx[m];
+                const int i = et + kGT * m;
+                if (i < nkb * kNT) sx_tab[i] = pre.sx[m];
             }
-            if (et < 2 * nkb) s_sw[et] = pre.sw;
-            if (MODE == 2 && et < kNT) s_wrow[et] = pre.wr;
-            named_barrier(1, 32 * kNtEpiWarps);
+            if (et < 2 * nkb) sw_tab[et] = pre.sw;
+            if (MODE == 2 && et < kNT) s_wrow[eg][et] = pre.wr;
+            named_barrier(bar, kGT);
             if (tn < n_items) nt_prefetch<MODE>(p, nxt, et, pre);
 
             float g[kNT], u[kNT];  // GEMM2 uses g only
 #pragma unroll
             for (int j = 0; j < kNT; ++j) g[j] = u[j] = 0.f;
+            if (ok && seq > 0) {
+                const bool w = mbar_wait(&handoff, (seq - 1) & 1, kWaitLimitNs);
+                if (!__all_sync(0xFFFFFFFFu, w)) {
+                    set_status(p.counters, MOE_ETIMEOUT);
+                    s_abort = 1;
+                    ok = false;
+                }
+            }
             for (int kb = 0; kb < nkb; ++kb, ++acc_it) {
                 const int b = acc_it % kAccBufs;
                 if (ok) {
@@ -1148,16 +1185,35 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                 if (!ok) continue;
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kAccStride);
-                const float sw0 = s_sw[kb], sw1 = s_sw[nkb + kb];
-                const float4 *sx4 = reinterpret_cast<const float4 *>(s_sx + kb * kNT);
+                const float sw0 = sw_tab[kb], sw1 = sw_tab[nkb + kb];
+                const float4 *sx4 = reinterpret_cast<const float4 *>(sx_tab + kb * kNT);
                 if (MODE == 1) {
 #pragma unroll
+                    for (int h = 0; h < kNT / 8; ++h) {  // rows [8 h, +8)
+                        float gh[8], gl[8], uh[8], ul[8];
+                        tmem_ld_32x8(tb + 8 * h, gh);
+                        tmem_ld_32x8(tb + kNT + 8 * h, gl);
+                        tmem_ld_32x8(tb + kNtN + 8 * h, uh);
+                        tmem_ld_32x8(tb + kNtN + kNT + 8 * h, ul);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j4 = 0; j4 < 2; ++j4) {
+                            const float4 sx = sx4[2 * h + j4];
+                            const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const int i = 4 * j4 + c, j = 8 * h + i;
+                                g[j] = fmaf(sxa[c] * sw0, gh[i] + gl[i], g[j]);
+                                u[j] = fmaf(sxa[c] * sw1, uh[i] + ul[i], u[j]);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
                     for (int h = 0; h < 2; ++h) {  // rows [16 h, +16)
-                        float gh[16], gl[16], uh[16], ul[16];
-                        tmem_ld_32x16(tb + 16 * h, gh);
-                        tmem_ld_32x16(tb + kNT + 16 * h, gl);
-                        tmem_ld_32x16(tb + kNtN + 16 * h, uh);
-                        tmem_ld_32x16(tb + kNtN + kNT + 16 * h, ul);
+                        float vh[16], vl[16];
+                        tmem_ld_32x16(tb + 16 * h, vh);
+                        tmem_ld_32x16(tb + kNT + 16 * h, vl);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j4 = 0; j4 < 4; ++j4) {
@@ -1166,24 +1222,8 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
 #pragma unroll
                             for (int c = 0; c < 4; ++c) {
                                 const int i = 4 * j4 + c, j = 16 * h + i;
-                                g[j] = fmaf(sxa[c] * sw0, gh[i] + gl[i], g[j]);
-                                u[j] = fmaf(sxa[c] * sw1, uh[i] + ul[i], u[j]);
+                                g[j] = fmaf(sxa[c] * sw0, vh[i] + vl[i], g[j]);
                             }
-                        }
-                    }
-                } else {
-                    float vh[kNT], vl[kNT];
-                    tmem_ld_32x32(tb, vh);
-                    tmem_ld_32x32(tb + kNT, vl);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j4 = 0; j4 < kNT / 4; ++j4) {
-                        const float4 sx = sx4[j4];
-                        const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int j = 4 * j4 + c;
-                            g[j] = fmaf(sxa[c] * sw0, vh[j] + vl[j], g[j]);
                         }
                     }
                 }
@@ -1191,6 +1231,8 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[b]);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&handoff);  // this item's accumulators are all received
             if (MODE == 1) {
                 // h = silu(gate) * up; the 128 columns of the block share one
                 // scale per row: max |h| over the warp by recursive halving
@@ -1212,44 +1254,47 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                         m[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, w));
                     }
                 }
-                s_amax[q][lane] = m[0];
-                named_barrier(1, 32 * kNtEpiWarps);
+                amax_tab[q][lane] = m[0];
+                named_barrier(bar, kGT);
                 if (q == 0) {
-                    const float a = fmaxf(fmaxf(s_amax[0][lane], s_amax[1][lane]), fmaxf(s_amax[2][lane], s_amax[3][lane]));
+                    const float a = fmaxf(fmaxf(amax_tab[0][lane], amax_tab[1][lane]),
+                                          fmaxf(amax_tab[2][lane], amax_tab[3][lane]));
                     const float sc = a > 0.f ? a / 448.f : 1.f;
-                    s_scl[lane] = sc;
-                    s_inv[lane] = 1.f / sc;
+                    s_scl[eg][lane] = sc;
+                    s_inv[eg][lane] = 1.f / sc;
                 }
-                named_barrier(1, 32 * kNtEpiWarps);
+                named_barrier(bar, kGT);
 #pragma unroll
                 for (int j = 0; j < kNT; j += 2) {
-                    const float a = g[j] * s_inv[j], c = g[j + 1] * s_inv[j + 1];
+                    const float a = g[j] * s_inv[eg][j], c = g[j + 1] * s_inv[eg][j + 1];
                     const uint16_t hh = f32x2_to_e4m3x2(a, c);
                     const float2 f = e4m3x2_to_f32x2(hh);
                     const uint16_t ll = f32x2_to_e4m3x2(a - f.x, c - f.y);
-                    s_hq[0][j][r] = (uint8_t)(hh & 0xFF);
-                    s_hq[0][j + 1][r] = (uint8_t)(hh >> 8);
-                    s_hq[1][j][r] = (uint8_t)(ll & 0xFF);
-                    s_hq[1][j + 1][r] = (uint8_t)(ll >> 8);
+                    s_hq[eg][0][j][r] = (uint8_t)(hh & 0xFF);
+                    s_hq[eg][0][j + 1][r] = (uint8_t)(hh >> 8);
+                    s_hq[eg][1][j][r] = (uint8_t)(ll & 0xFF);
+                    s_hq[eg][1][j + 1][r] = (uint8_t)(ll >> 8);
                 }
-                named_barrier(1, 32 * kNtEpiWarps);
+                named_barrier(bar, kGT);
                 // rows of 128 codes out as 16-byte pieces
-                for (int i = et; i < 2 * kNT * (kWB / 16); i += 32 * kNtEpiWarps) {
+                for (int i = et; i < 2 * kNT * (kWB / 16); i += kGT) {
                     const int part = i / (kNT * (kWB / 16));
                     const int j = (i / (kWB / 16)) % kNT, ch = i % (kWB / 16);
                     if (j < cur.rows)
                         *reinterpret_cast<uint4 *>(p.hq + ((size_t)cur.row0 + j) * 2 * p.imax + (part ? p.imax : 0) +
                                                    cur.nb * kWB + ch * 16) =
-                            *reinterpret_cast<const uint4 *>(&s_hq[part][j][ch * 16]);
+                            *reinterpret_cast<const uint4 *>(&s_hq[eg][part][j][ch * 16]);
                 }
-                if (q == 0 && lane < cur.rows) p.hs[((size_t)cur.row0 + lane) * (p.imax / 128) + cur.nb] = s_scl[lane];
+                if (q == 0 && lane < cur.rows) p.hs[((size_t)cur.row0 + lane) * (p.imax / 128) + cur.nb] = s_scl[eg][lane];
             } else if (ok) {
                 // a warp stores 32 consecutive floats of each row's partial row
                 float *dst = p.yslot + (size_t)cur.row0 * p.H + cur.nb * kWB + r;
 #pragma unroll
                 for (int j = 0; j < kNT; ++j)
-                    if (j < cur.rows) dst[(size_t)j * p.H] = s_wrow[j] * g[j];
+                    if (j < cur.rows) dst[(size_t)j * p.H] = s_wrow[eg][j] * g[j];
             }
+            if (tm < n_items) acc_it += mid.kdim / kBK;  // the other group's K blocks
+            seq += 2;
             t = tn;
             cur = nxt;
         }

@@ -122,6 +122,17 @@ __device__ __forceinline__ void tmem_ld_32x16(uint32_t taddr, float (&v)[16])
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 8 columns of 32-bit words from tensor memory.
+__device__ __forceinline__ void tmem_ld_32x8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // TMA tiled loads (no multicast), completing on an mbarrier.  The tensor map
 // is a kernel parameter (__grid_constant__).  x must be a multiple of 16
 // bytes.

@@ -96,6 +96,11 @@ def test_paths_and_launch_counts(L):
         assert moe.kernel_launches(d, 5, path) == n
     assert moe.kernel_launches(d, 5, 4) == 0                  # no such path
     assert moe.auto_path(d, 1) == moe.MOE_PATH_DECODE
+    assert moe.auto_path(d, moe.MOE_AUTO_DECODE_MAX_ROWS + 1) == moe.MOE_PATH_PREFILL_NARROW
+    narrow_max = moe.MOE_AUTO_NARROW_MAX_PAIRS * 256 // 8          # rows * k <= pairs * E
+    assert moe.auto_path(d, narrow_max) == moe.MOE_PATH_PREFILL_NARROW
+    assert moe.auto_path(d, narrow_max + 1) == moe.MOE_PATH_PREFILL
+    assert moe.auto_path(D(h=8192), 64) == moe.MOE_PATH_PREFILL  # beyond the narrow GEMMs' K
     assert moe.auto_path(d, 4096) == moe.MOE_PATH_PREFILL
     assert moe.auto_path(d, -1) == moe.MOE_EINVAL
     # the narrow GEMMs hold at most 64 K blocks of scales per item: refused

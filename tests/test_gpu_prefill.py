@@ -56,17 +56,19 @@ def test_prefill_small_shapes(dims, rows, bias):
 
 def test_auto_path_switch():
     d = mi.TINY
-    assert moe.MOE_AUTO_DECODE_MAX_ROWS == 12
-    assert moe.kernel_launches(d, 12) == 3
-    assert moe.kernel_launches(d, 13) == 6
-    case = P.build_case(d, 13, all_experts=True)
-    out, idx, _, _ = run(case, moe.MOE_PATH_AUTO)
-    P.compare_output(case, out, idx)
+    assert moe.auto_path(d, moe.MOE_AUTO_DECODE_MAX_ROWS) == moe.MOE_PATH_DECODE
+    assert moe.auto_path(d, moe.MOE_AUTO_DECODE_MAX_ROWS + 1) == moe.MOE_PATH_PREFILL_NARROW
+    big = moe.MOE_AUTO_NARROW_MAX_PAIRS * d.n_experts // d.top_k + 1
+    assert moe.auto_path(d, big) == moe.MOE_PATH_PREFILL
+    for rows in (moe.MOE_AUTO_DECODE_MAX_ROWS + 1, big):
+        case = P.build_case(d, rows, all_experts=True)
+        out, idx, _, _ = run(case, moe.MOE_PATH_AUTO)
+        P.compare_output(case, out, idx)
 
 
 @pytest.mark.parametrize("rows", [16, 32, 64])
-def test_qwen36_35b_auto_prefill_at_decode_row_counts(rows):
-    # AUTO takes the grouped-GEMM path from 13 rows on: every row against the oracle
+def test_qwen36_35b_auto_at_multi_row_decode_counts(rows):
+    # every row against the oracle, on the path AUTO takes
     d = mi.QWEN36_35B_A3B
     case = P.build_case(d, rows)
     out, idx, w, gs = run(case, moe.MOE_PATH_AUTO)
