@@ -123,6 +123,7 @@ struct PlanParams {
     int4 *mtiles;      // [0].x = count; entries from [1]: {group, row0, rows, a_row0}
     int tile_rows;     // rows per group tile: kBM, or kNT for the narrow GEMMs
     int count_in_scan; // counts and ranks not given by the router: scan_kernel derives them
+    int perm_split;    // permute_kernel: warps per token (its k + 1 destinations split between them)
     const uint16_t *x; // [T][H] bf16
     int xp_shared0;    // first xp row of the shared expert's rows (the routed rows span at least 128)
     uint8_t *xp;
@@ -203,12 +204,15 @@ __global__ void __launch_bounds__(1024) scan_kernel(PlanParams p)
     if (threadIdx.x == 0) p.mtiles[0] = make_int4(run_tiles + smt, run_tiles, 0, 0);
 }
 
-// A warp per token: its x row is quantised once to hi/lo e4m3 (hi codes [H],
-// then lo codes [H]) with one scale per 128 block, amax / 448 (x ~ s * (hi +
-// lo)), and written to each of its k expert rows and to its row of the
-// shared expert; each routed pair's position and blend weight are recorded.
-// Rows of up to kPermMaxBlocks * 128 elements keep their codes in
-// registers; wider rows quantise again for each destination.
+// A token's x row is quantised to hi/lo e4m3 (hi codes [H], then lo codes
+// [H]) with one scale per 128 block, amax / 448 (x ~ s * (hi + lo)), and
+// written to each of its k expert rows and to its row of the shared expert;
+// each routed pair's position and blend weight are recorded.  A warp takes
+// one token and perm_split-th of its k + 1 destinations (few tokens: one
+// destination per warp, so that the writes spread over many warps; many
+// tokens: all of them, quantising once).  Rows of up to kPermMaxBlocks * 128
+// elements keep their codes in registers; wider rows quantise again for each
+// destination.
 constexpr int kPermMaxBlocks = 32;
 
 __device__ __forceinline__ void permute_write(const PlanParams &p, int dst_row, int dst_scale, int kb, int lane,
@@ -227,21 +231,33 @@ __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
     const int lane = threadIdx.x & 31;
     const int P = p.T * p.K;
     const int hb = p.H / 128;
+    const int D = p.K + 1;  // destinations of a token: its k routed rows, then its shared row
+    const int ns = p.perm_split;
+    const int dpw = (D + ns - 1) / ns;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
-    for (int t = gw; t < p.T; t += nw) {
-        // destinations: k routed rows, then the shared row
-        int dst[kMaxTopK + 1];
-        for (int r = 0; r < p.K; ++r) {
-            const int i = t * p.K + r;
-            const int e = min(max(p.topk_idx[i], 0), p.E - 1);
-            dst[r] = p.offsets[e] + p.rank[i];
-            if (lane == 0) {
-                p.pos[i] = dst[r];
-                p.slot_w[dst[r]] = p.topk_w[i];
+    for (int w = gw; w < p.T * ns; w += nw) {
+        const int t = w / ns;
+        const int d0 = (w - t * ns) * dpw, nd = min(D, d0 + dpw) - d0;
+        if (nd <= 0) continue;
+        // this warp's destinations: rows of xp and of its scales
+        int row[kMaxTopK + 1], srow[kMaxTopK + 1];
+        for (int c = 0; c < nd; ++c) {
+            const int r = d0 + c;
+            if (r < p.K) {
+                const int i = t * p.K + r;
+                const int e = min(max(p.topk_idx[i], 0), p.E - 1);
+                row[c] = srow[c] = p.offsets[e] + p.rank[i];
+                if (lane == 0) {
+                    p.pos[i] = row[c];
+                    p.slot_w[row[c]] = p.topk_w[i];
+                }
+            } else {
+                row[c] = p.xp_shared0 + t;
+                srow[c] = P + t;
+                if (lane == 0) p.slot_w[P + t] = p.gsig[t];
             }
         }
-        if (lane == 0) p.slot_w[P + t] = p.gsig[t];
         const uint2 *src = reinterpret_cast<const uint2 *>(p.x + (size_t)t * p.H);
         if (hb <= kPermMaxBlocks) {
             uint32_t hi[kPermMaxBlocks], lo[kPermMaxBlocks];
@@ -255,13 +271,11 @@ __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
                 scv[kb] = amax > 0.f ? amax / 448.f : 1.f;
                 quant4_hilo(v, 1.f / scv[kb], hi[kb], lo[kb]);
             }
-            for (int r = 0; r <= p.K; ++r) {
-                const int row = r < p.K ? dst[r] : p.xp_shared0 + t;
-                const int srow = r < p.K ? dst[r] : P + t;
+            for (int c = 0; c < nd; ++c) {
 #pragma unroll
                 for (int kb = 0; kb < kPermMaxBlocks; ++kb) {
                     if (kb >= hb) break;
-                    permute_write(p, row, srow, kb, lane, hi[kb], lo[kb], scv[kb]);
+                    permute_write(p, row[c], srow[c], kb, lane, hi[kb], lo[kb], scv[kb]);
                 }
             }
         } else {
@@ -272,8 +286,7 @@ __global__ void __launch_bounds__(256) permute_kernel(PlanParams p)
                 const float sc = amax > 0.f ? amax / 448.f : 1.f;
                 uint32_t h, l;
                 quant4_hilo(v, 1.f / sc, h, l);
-                for (int r = 0; r <= p.K; ++r)
-                    permute_write(p, r < p.K ? dst[r] : p.xp_shared0 + t, r < p.K ? dst[r] : P + t, kb, lane, h, l, sc);
+                for (int c = 0; c < nd; ++c) permute_write(p, row[c], srow[c], kb, lane, h, l, sc);
             }
         }
     }
@@ -884,11 +897,13 @@ constexpr uint32_t kNtTmemCols = 512;
 constexpr int kWB = 128;                            // weight rows per item (one scale block)
 constexpr int kNtPre = kNtMaxKb * kNT / (32 * kNtEpiWarps);  // activation scales per epilogue thread and item
 
-// TMEM columns per accumulator buffer (GEMM1: gate | up) and buffers.
+// An item reads two 128-row weight blocks (GEMM1: the gate block and its up
+// block; GEMM2: two neighbouring W2 blocks, the second absent past H), each
+// into its own accumulator: TMEM columns per buffer, and buffers.
 template <int MODE>
 __host__ __device__ constexpr int nt_acc_stride()
 {
-    return MODE == 1 ? 2 * kNtN : kNtN;
+    return 2 * kNtN;
 }
 template <int MODE>
 __host__ __device__ constexpr int nt_acc_bufs()
@@ -898,12 +913,12 @@ __host__ __device__ constexpr int nt_acc_bufs()
 template <int MODE>
 __host__ __device__ constexpr size_t nt_stage_bytes()
 {
-    return (MODE == 1 ? 2 : 1) * (size_t)kWB * kBK + 2 * (size_t)kNT * kBK;  // weights (gate, up), rows hi, lo
+    return 2 * (size_t)kWB * kBK + 2 * (size_t)kNT * kBK;  // two weight blocks, then the rows' hi and lo codes
 }
 template <int MODE>
 __host__ __device__ constexpr int nt_stages()
 {
-    return MODE == 1 ? 5 : 8;
+    return 5;
 }
 template <int MODE>
 __host__ __device__ constexpr size_t nt_smem()
@@ -935,7 +950,15 @@ __device__ __forceinline__ bool nt_item(const GemmParams &p, int n_mtiles, int t
         return ti.nb < ti.inter / kWB;  // 128-column blocks of h
     }
     ti.kdim = ti.inter;
-    return true;                        // max_ntiles = H / 128 output blocks
+    return true;                        // max_ntiles = (H / 128 + 1) / 2 pairs of output blocks
+}
+
+// Weight blocks of an item: GEMM1 two (gate, up); GEMM2 two, or one for the
+// last pair when H / 128 is odd.
+template <int MODE>
+__device__ __forceinline__ int nt_blocks(const GemmParams &p, const NtItem &ti)
+{
+    return MODE == 1 ? 2 : min(2, p.H / kWB - 2 * ti.nb);
 }
 
 // The first valid item at or after t, in steps of the grid (n_items if none).
@@ -971,7 +994,8 @@ __device__ __forceinline__ void nt_prefetch(const GemmParams &p, const NtItem &t
     } else {
         wsc += (size_t)(2 * ti.inter / 128) * (p.H / 128);
         wld = ti.inter / 128;
-        wn0 = wn1 = ti.nb;
+        wn0 = 2 * ti.nb;                              // the pair's output blocks
+        wn1 = min(2 * ti.nb + 1, p.H / 128 - 1);      // (a valid row when the second is absent)
     }
     const int j = et % kNT;  // this thread's row of the table
 #pragma unroll
@@ -988,14 +1012,14 @@ __device__ __forceinline__ void nt_prefetch(const GemmParams &p, const NtItem &t
 // [128 nb, +128) and up rows [inter + 128 nb, +128) against x; epilogue
 // h = silu(gate) * up, quantised to hi/lo e4m3 with one scale per (row, 128
 // block), in the layout gemm_kernel<1> writes.  MODE 2: item = output
-// columns [128 nb, +128): W2 rows against h; epilogue x the row's blend
+// columns [256 nb, +256): W2 rows against h; epilogue x the row's blend
 // weight into its partial row.
 template <int MODE>
 __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_constant__ GemmParams p)
 {
     constexpr int kStages = nt_stages<MODE>();
     constexpr uint32_t kSt = (uint32_t)nt_stage_bytes<MODE>();
-    constexpr uint32_t kAB = (MODE == 1 ? 2 : 1) * kWB * kBK;  // weight bytes of a stage
+    constexpr uint32_t kAB = 2 * kWB * kBK;  // weight bytes of a stage (two blocks)
     constexpr int kAccStride = nt_acc_stride<MODE>(), kAccBufs = nt_acc_bufs<MODE>();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages], acc_full[kAccBufs], acc_empty[kAccBufs];
@@ -1067,6 +1091,10 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                 const int ez = ti.shared_grp ? 0 : ti.group;
                 const int arow = MODE == 1 ? ti.a_row0 : ti.row0;
                 const int lo_x = MODE == 1 ? p.H : p.imax;  // where the lo half of an activation row starts
+                const int nblk = nt_blocks<MODE>(p, ti);
+                // weight rows of the two blocks: gate and up (GEMM1), or a pair of W2 blocks
+                const int y0 = MODE == 1 ? ti.nb * kWB : 2 * ti.nb * kWB;
+                const int y1 = MODE == 1 ? ti.inter + ti.nb * kWB : y0 + kWB;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % kStages;
                     if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kWaitLimitNs)) {
@@ -1075,9 +1103,9 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                         break;
                     }
                     unsigned char *st = smem + (size_t)s * kSt;
-                    mbar_arrive_expect_tx(&full[s], kSt);
-                    tma_load_3d(st, wmap, kb * kBK, ti.nb * kWB, ez, &full[s], pol_w);
-                    if (MODE == 1) tma_load_3d(st + kWB * kBK, wmap, kb * kBK, ti.inter + ti.nb * kWB, ez, &full[s], pol_w);
+                    mbar_arrive_expect_tx(&full[s], kSt - (2 - nblk) * kWB * kBK);
+                    tma_load_3d(st, wmap, kb * kBK, y0, ez, &full[s], pol_w);
+                    if (nblk == 2) tma_load_3d(st + kWB * kBK, wmap, kb * kBK, y1, ez, &full[s], pol_w);
                     // hi rows, then lo rows: together the 64-row B operand
                     tma_load_2d(st + kAB, amap, kb * kBK, arow, &full[s], pol_a);
                     tma_load_2d(st + kAB + kNT * kBK, amap, lo_x + kb * kBK, arow, &full[s], pol_a);
@@ -1093,6 +1121,7 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                 NtItem ti;
                 if (!nt_item<MODE>(p, n_mtiles, t, ti)) continue;
                 const int nkb = ti.kdim / kBK;
+                const int nblk = nt_blocks<MODE>(p, ti);
                 for (int kb = 0; kb < nkb; ++kb, ++it, ++acc_it) {
                     const int s = it % kStages;
                     const int b = acc_it % kAccBufs;
@@ -1110,7 +1139,7 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                     for (int k4 = 0; k4 < kBK / 32; ++k4) {
                         const uint32_t acc = k4 ? 1u : 0u;
                         umma_f8f6f4(d, umma_desc_sw128(st + k4 * 32), umma_desc_sw128(bsm + k4 * 32), idesc, acc);
-                        if (MODE == 1)
+                        if (nblk == 2)
                             umma_f8f6f4(d + kNtN, umma_desc_sw128(st + kWB * kBK + k4 * 32), umma_desc_sw128(bsm + k4 * 32),
                                         idesc, acc);
                     }
@@ -1161,7 +1190,7 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
             named_barrier(bar, kGT);
             if (tn < n_items) nt_prefetch<MODE>(p, nxt, et, pre);
 
-            float g[kNT], u[kNT];  // GEMM2 uses g only
+            float g[kNT], u[kNT];  // the two blocks' sums
 #pragma unroll
             for (int j = 0; j < kNT; ++j) g[j] = u[j] = 0.f;
             if (ok && seq > 0) {
@@ -1187,43 +1216,25 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                 const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kAccStride);
                 const float sw0 = sw_tab[kb], sw1 = sw_tab[nkb + kb];
                 const float4 *sx4 = reinterpret_cast<const float4 *>(sx_tab + kb * kNT);
-                if (MODE == 1) {
+                // the two blocks' accumulators (GEMM1 gate and up; GEMM2 the pair
+                // of output blocks), 8 rows at a time
 #pragma unroll
-                    for (int h = 0; h < kNT / 8; ++h) {  // rows [8 h, +8)
-                        float gh[8], gl[8], uh[8], ul[8];
-                        tmem_ld_32x8(tb + 8 * h, gh);
-                        tmem_ld_32x8(tb + kNT + 8 * h, gl);
-                        tmem_ld_32x8(tb + kNtN + 8 * h, uh);
-                        tmem_ld_32x8(tb + kNtN + kNT + 8 * h, ul);
-                        tmem_wait_ld();
+                for (int h = 0; h < kNT / 8; ++h) {  // rows [8 h, +8)
+                    float gh[8], gl[8], uh[8], ul[8];
+                    tmem_ld_32x8(tb + 8 * h, gh);
+                    tmem_ld_32x8(tb + kNT + 8 * h, gl);
+                    tmem_ld_32x8(tb + kNtN + 8 * h, uh);
+                    tmem_ld_32x8(tb + kNtN + kNT + 8 * h, ul);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int j4 = 0; j4 < 2; ++j4) {
-                            const float4 sx = sx4[2 * h + j4];
-                            const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
+                    for (int j4 = 0; j4 < 2; ++j4) {
+                        const float4 sx = sx4[2 * h + j4];
+                        const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
 #pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const int i = 4 * j4 + c, j = 8 * h + i;
-                                g[j] = fmaf(sxa[c] * sw0, gh[i] + gl[i], g[j]);
-                                u[j] = fmaf(sxa[c] * sw1, uh[i] + ul[i], u[j]);
-                            }
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {  // rows [16 h, +16)
-                        float vh[16], vl[16];
-                        tmem_ld_32x16(tb + 16 * h, vh);
-                        tmem_ld_32x16(tb + kNT + 16 * h, vl);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j4 = 0; j4 < 4; ++j4) {
-                            const float4 sx = sx4[4 * h + j4];
-                            const float sxa[4] = {sx.x, sx.y, sx.z, sx.w};
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const int i = 4 * j4 + c, j = 16 * h + i;
-                                g[j] = fmaf(sxa[c] * sw0, vh[i] + vl[i], g[j]);
-                            }
+                        for (int c = 0; c < 4; ++c) {
+                            const int i = 4 * j4 + c, j = 8 * h + i;
+                            g[j] = fmaf(sxa[c] * sw0, gh[i] + gl[i], g[j]);
+                            u[j] = fmaf(sxa[c] * sw1, uh[i] + ul[i], u[j]);
                         }
                     }
                 }
@@ -1287,11 +1298,16 @@ __global__ void __launch_bounds__(kNtThreads, 1) gemm_nt_kernel(const __grid_con
                 }
                 if (q == 0 && lane < cur.rows) p.hs[((size_t)cur.row0 + lane) * (p.imax / 128) + cur.nb] = s_scl[eg][lane];
             } else if (ok) {
-                // a warp stores 32 consecutive floats of each row's partial row
-                float *dst = p.yslot + (size_t)cur.row0 * p.H + cur.nb * kWB + r;
+                // a warp stores 32 consecutive floats of each row's partial row, per block
+                const bool two = nt_blocks<MODE>(p, cur) == 2;
+                float *dst = p.yslot + (size_t)cur.row0 * p.H + 2 * cur.nb * kWB + r;
 #pragma unroll
-                for (int j = 0; j < kNT; ++j)
-                    if (j < cur.rows) dst[(size_t)j * p.H] = s_wrow[eg][j] * g[j];
+                for (int j = 0; j < kNT; ++j) {
+                    if (j < cur.rows) {
+                        dst[(size_t)j * p.H] = s_wrow[eg][j] * g[j];
+                        if (two) dst[(size_t)j * p.H + kWB] = s_wrow[eg][j] * u[j];
+                    }
+                }
             }
             if (tm < n_items) acc_it += mid.kdim / kBK;  // the other group's K blocks
             seq += 2;
@@ -1504,8 +1520,11 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
 
     // 2, 3
     if ((e = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, pp)) != cudaSuccess) return MOE_ECUDA;
-    if ((e = launch_kernel(permute_kernel, dim3(std::max(1, std::min(8 * di.sm_count, (T + 7) / 8))), dim3(256),
-                           0, s, pp)) != cudaSuccess)
+    // few tokens: a warp per destination row, so that ~32 warps per SM write
+    pp.perm_split = T >= 1024 ? 1 : std::min(K + 1, std::max(1, (32 * di.sm_count + T - 1) / T));
+    const int perm_warps = T * pp.perm_split;
+    if ((e = launch_kernel(permute_kernel, dim3(std::max(1, std::min(8 * di.sm_count, (perm_warps + 7) / 8))),
+                           dim3(256), 0, s, pp)) != cudaSuccess)
         return MOE_ECUDA;
 
     // 4. GEMM1
@@ -1566,7 +1585,7 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
     g2.a_scales_shared = g.hs;
     g2.a_scales_ld = imax / 128;
     if (narrow) {
-        g2.max_ntiles = H / kWB;
+        g2.max_ntiles = (H / kWB + 1) / 2;  // pairs of 128-row W2 blocks
         e = launch_kernel(gemm_nt_kernel<2>, dim3(di.sm_count), dim3(kNtThreads), nt_smem<2>(), s, g2);
     } else {
         g2.max_ntiles = (H + kBN - 1) / kBN;
