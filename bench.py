@@ -194,7 +194,9 @@ def source_hash(paths) -> str:
 
 def profiled_traffic(kernel: str, workload_tag: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel source (else None).  The summary names the source
+    files the kernel is built from (`source_files:`, paths under the package's
+    csrc/; all of csrc/ when absent) and their hash at capture time."""
     prof = os.path.join(ROOT, "profiles", f"{kernel}_{workload_tag}.md")
     if not os.path.exists(prof):
         return None
@@ -203,9 +205,11 @@ def profiled_traffic(kernel: str, workload_tag: str):
     h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
     if not m or not h:
         return None
-    srcs = sorted(os.path.join(ROOT, "sparse_moe_ffn_topk_b200", "csrc", f)
-                  for f in os.listdir(os.path.join(ROOT, "sparse_moe_ffn_topk_b200", "csrc")))
-    if h.group(1) != source_hash(srcs):
+    csrc = os.path.join(ROOT, "sparse_moe_ffn_topk_b200", "csrc")
+    f = re.search(r"source_files:\s*(.+)", txt)
+    names = f.group(1).split() if f else os.listdir(csrc)
+    srcs = sorted(os.path.join(csrc, n) for n in names)
+    if not all(os.path.exists(q) for q in srcs) or h.group(1) != source_hash(srcs):
         return None
     return float(m.group(1))
 
