@@ -89,7 +89,7 @@ extern "C" {
                                          (an expert's average routed rows), then the 128-row token tiles;
                                          the switch points were measured on B200 with every path timed on
                                          the 35B-A3B- and 397B-A17B-shaped layers */
-#define MOE_AUTO_NARROW_MAX_PAIRS 16
+#define MOE_AUTO_NARROW_MAX_PAIRS 32
 
 typedef struct moe_dims {
     int32_t hidden;       /* H  */

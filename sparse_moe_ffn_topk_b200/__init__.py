@@ -40,7 +40,7 @@ MOE_PATH_PREFILL = 2
 MOE_PATH_PREFILL_NARROW = 3
 MOE_DECODE_MAX_ROWS = 64
 MOE_AUTO_DECODE_MAX_ROWS = 3
-MOE_AUTO_NARROW_MAX_PAIRS = 16
+MOE_AUTO_NARROW_MAX_PAIRS = 32
 
 EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe_ffn_forward",
             "moe_ffn_forward_path", "moe_status", "moe_reset_status", "moe_status_string",

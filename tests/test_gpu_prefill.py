@@ -123,9 +123,9 @@ def test_qwen35_397b_prefill_sampled():
     (mi.LayerDims(hidden=640, n_experts=20, top_k=4, inter=128, shared_inter=256), 100),
 ])
 def test_prefill_hidden_odd_multiple_of_128(dims, rows):
-    # H/128 odd: the down GEMM's last 256-column tile is half empty; AUTO takes the 128-row tiles here
+    # H/128 odd: the down GEMM's last 256-column tile is half empty
     case = P.build_case(dims, rows, router_bias=True, all_experts=True, residual=True)
-    out, idx, w, gs = run(case, moe.MOE_PATH_AUTO)
+    out, idx, w, gs = run(case, moe.MOE_PATH_PREFILL)
     _, oidx, ow, ogs = oracle.router_topk(dims, case.x, case.layer.router_w, case.layer.shared_gate,
                                           router_bias=case.layer.router_bias)
     P.check_routing(case, idx, w, gs, ow, ogs)
