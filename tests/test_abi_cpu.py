@@ -38,6 +38,14 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), n
 
 
+def test_binding_constants_match_header():
+    src = open(os.path.join(ROOT, "include", "moe_ffn.h")).read()
+    defs = dict(re.findall(r"#define\s+(MOE_[A-Z0-9_]+)\s+(-?\d+)", src))
+    assert len(defs) >= 12
+    for name, value in defs.items():
+        assert getattr(moe, name) == int(value), name
+
+
 def test_binding_names_match_header():
     assert set(moe.EXPORTED) == declared_symbols()
 
