@@ -15,6 +15,11 @@
   expert(x) + expert_shared(x)/2; the routed result equals the dense,
   all-experts evaluation masked to the top-k; a hand-derived case with
   exact dyadic outputs.
+- the shared-expert gate: hand cases with g . x = +2, -2, -2.5, 3.5 against
+  scipy's logistic function (a flipped sign or a dot product with another
+  vector fails), and random gate vectors against numpy's float64 dot.
+- the router-only entry equals the layer's own routing (logits, experts,
+  weights, gate) on the tiny and 35B-A3B-shaped layers.
 """
 import math
 
@@ -375,3 +380,107 @@ def test_oracle_reproduces_its_tiny_regression_record():
     with open(os.path.join(here, "golden", "tiny_seed0.json")) as f:
         stored = json.load(f)
     assert make_golden.tiny_record(0) == stored
+
+
+# ------------------------------------------------------- shared-expert gate
+
+def _gate_case(gate_entries):
+    """H = I = Is = 128, E = 2, k = 1, one row x = e_0 + 2 e_1 (exact bf16).
+
+    Router rows give logits [1, 0], so expert 0 is chosen with weight 1.
+    Every 128x128 block holds a 112, so its scale is 0.25 and the entries
+    used are exact codes.  Expert 0: gate_0 = 112 x_0, up_0 = 0.25 x_1 = 0.5,
+    h_0 = silu(112) * 0.5 = 56, y_0 = 0.5 * 56 = 28.  Shared expert: gate_0 =
+    112 x_0, up_0 = 0.5 x_1 = 1, h_0 = 112, y_1 = 0.25 * 112 = 28.  So
+    out = [28, sigmoid(z) * 28, 0, ...] with z = g . x set by the gate
+    vector's first two entries.
+    """
+    H = I = 128
+    d = mi.LayerDims(hidden=H, n_experts=2, top_k=1, inter=I, shared_inter=I)
+    x = np.zeros((1, H), dtype=np.float32)
+    x[0, 0], x[0, 1] = 1.0, 2.0
+    rw = np.zeros((2, H), dtype=np.float32)
+    rw[0, 0] = 1.0
+    g = np.zeros(H, dtype=np.float32)
+    g[0], g[1] = gate_entries
+
+    def slab(up_val, y_row, y_val):
+        w13 = np.zeros((2 * I, H), dtype=np.float32)
+        w2 = np.zeros((H, I), dtype=np.float32)
+        w13[0, 0] = 112.0
+        w13[I + 0, 1] = up_val
+        w13[2 * I - 1, H - 1] = 112.0     # sets every W13 block's scale to 0.25
+        w2[y_row, 0] = y_val
+        w2[H - 1, I - 1] = 112.0          # and the W2 block's
+        return _slab_from_fp32(w13, w2)
+
+    e0 = slab(0.25, 0, 0.5)
+    e1 = slab(0.0, 2, 112.0)              # never chosen
+    sh = slab(0.5, 1, 0.25)
+    w8 = np.stack([e0[0], e1[0]])
+    sc = np.stack([e0[1], e1[1]])
+    return d, _bf16(x), _bf16(rw), w8, sc, sh[0], sh[1], _bf16(g)
+
+
+@pytest.mark.parametrize("entries,z", [((1.0, 0.5), 2.0), ((0.0, -1.0), -2.0), ((-3.0, 0.25), -2.5),
+                                       ((0.5, 1.5), 3.5)])
+def test_shared_gate_sigmoid_at_nonzero_z(entries, z):
+    """sigmoid(g . x) with g . x != 0, against scipy's logistic function: a
+    flipped sign (sigmoid(-z)), a dropped factor or a dot product with
+    another vector (the router row gives 1 here) fails."""
+    d, x, rw, w8, sc, sw8, ssc, g = _gate_case(entries)
+    r = oracle.moe_forward(d, x, rw, w8, sc, sw8, ssc, g)
+    want = scipy.special.expit(z)
+    assert r.idx[0].tolist() == [0] and r.w[0].tolist() == [1.0]
+    assert abs(r.gate_sig[0] - want) <= 1e-15
+    assert abs(r.gate_sig[0] - scipy.special.expit(-z)) > 0.1      # the sign matters here
+    assert r.out[0, 0] == 28.0
+    assert abs(r.out[0, 1] - want * 28.0) <= 1e-13
+    assert np.all(r.out[0, 2:] == 0.0)
+    _, _, _, gs = oracle.router_topk(d, x, rw, g)
+    assert abs(gs[0] - want) <= 1e-15
+
+
+def test_shared_gate_against_numpy_dot():
+    """Random gate vectors (tiny layer, 4 rows): the oracle's gate equals
+    scipy.expit of numpy's float64 dot product of the bf16-decoded x and g."""
+    d = mi.TINY
+    L = mi.make_layer(d, seed=3)
+    x = mi.make_x(d, 4, seed=3)
+    g = mi._bf16_bits(torch.randn(d.hidden, generator=torch.Generator().manual_seed(11)) * 0.05)
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    gd = torch.from_numpy(g.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    z = xd @ gd
+    assert np.all(np.abs(z) > 0.05)
+    r = oracle.moe_forward(d, x, L.router_w, L.expert_w8, L.expert_scales, L.shared_w8,
+                           L.shared_scales, g)
+    assert np.allclose(r.gate_sig, scipy.special.expit(z), rtol=0, atol=1e-14)
+
+
+def _router_vs_forward(d, L, x, bias=None):
+    lg, idx, w, gs = oracle.router_topk(d, x, L.router_w, L.shared_gate, router_bias=bias)
+    r = oracle.moe_forward(d, x, L.router_w, L.expert_w8, L.expert_scales, L.shared_w8,
+                           L.shared_scales, L.shared_gate, router_bias=bias)
+    assert np.array_equal(lg, r.logits)
+    assert np.array_equal(idx, r.idx)
+    assert np.array_equal(w, r.w)
+    assert np.array_equal(gs, r.gate_sig)
+
+
+def test_router_entry_equals_forward_routing_tiny():
+    """The router-only entry (the reference routing of every GPU test) gives
+    the same logits, experts, weights and gate as the layer's own routing."""
+    d = mi.TINY
+    L = mi.make_layer(d, seed=0, router_bias=True)
+    x = mi.make_x(d, 6, seed=0)
+    _router_vs_forward(d, L, x)
+    _router_vs_forward(d, L, x, L.router_bias)
+
+
+def test_router_entry_equals_forward_routing_35b():
+    d = mi.QWEN36_35B_A3B
+    x = mi.make_x(d, 2, seed=0, stream=2)
+    rw, g, _ = mi.make_router(d, 0)
+    lg, idx, _, _ = oracle.router_topk(d, x, rw, g)
+    L = mi.make_layer(d, seed=0, experts=set(idx.ravel().tolist()))
+    _router_vs_forward(d, L, x)
