@@ -113,18 +113,31 @@ MOE_API size_t moe_workspace_bytes(const moe_dims *d, int32_t max_rows);
 MOE_API int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Router GEMV, shared-gate sigmoid and top-k softmax for `rows` rows of x.
+ * Defined by the "Qwen3.6-35B-A3B-FP8 on NVIDIA GB10" blueprint page, Kernels
+ * table (the router as a bf16 dense GEMV, gemv::dense_gemv_bf16, feeding
+ * moe_topk::moe_topk_softmax) and its Precision table (top-k node output
+ * f32,i32); the shared-expert gate after the "colibri #1992" PR page, frame
+ * A2.  Arithmetic: bf16 x and router rows, fp32 products and sums.
  * Outputs topk_idx [rows, k] (int32), topk_w [rows, k] (fp32, renormalised
  * over the k chosen, descending) and shared_gate_sig [rows] (fp32).
- * router_bias may be NULL.  rows == 0 is a no-op (pointers may then be NULL). */
+ * router_bias may be NULL.  rows == 0 is a no-op (pointers may then be NULL).
+ * Errors: MOE_EINVAL (null or misaligned pointer, rows < 0), MOE_EUNSUPPORTED
+ * (dims), MOE_EWORKSPACE (ws_bytes < moe_workspace_bytes(d, rows)), MOE_ECUDA. */
 MOE_API int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows,
                     const uint16_t *router_w, const float *router_bias,
                     const uint16_t *shared_gate, int32_t *topk_idx, float *topk_w,
                     float *shared_gate_sig, void *ws, size_t ws_bytes, void *stream);
 
 /* The whole layer step: out = sum_r w_r E_{idx_r}(x) + sigmoid(g.x) E_shared(x)
- * (+ residual), bf16 [rows, H].  residual and router_bias may be NULL.
- * Chooses the path by rows, as MOE_PATH_AUTO describes (moe_auto_path tells which).
- * rows == 0 is a no-op (pointers may then be NULL). */
+ * (+ residual), bf16 [rows, H].  Defined by the "Qwen3.6-35B-A3B-FP8 on
+ * NVIDIA GB10" blueprint page, Kernels table (router GEMV, top-k softmax,
+ * FP8 gate/up with the shared expert, SiLU and down, weighted-sum blend) and
+ * Precision table (fp8 block128x128 weights against bf16 activations for
+ * gate/up and f32 activations for down); the SwiGLU form after the
+ * "Neurarch Qwen3-8B" page (swiglu block).  residual and router_bias may be
+ * NULL.  Chooses the path by rows, as MOE_PATH_AUTO describes (moe_auto_path
+ * tells which).  rows == 0 is a no-op (pointers may then be NULL).
+ * Errors: as moe_router_topk, plus MOE_EINVAL when out aliases x. */
 MOE_API int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows,
                     const uint16_t *router_w, const uint8_t *expert_w8,
                     const float *expert_scales, const moe_fp8_expert *shared_w,
@@ -186,18 +199,34 @@ MOE_API int moe_debug_wait_timeout(void *ws, size_t ws_bytes, int32_t limit_us, 
  * uses a scratch array built into the library, moe_static_scratch_bytes()
  * large (16 MiB), of which every GPU that loads the library holds one copy
  * until the process exits.  Calls whose moe_workspace_bytes(d, rows) exceeds
- * it fail with MOE_EWORKSPACE.  The call allocates nothing (no cudaMalloc,
- * no allocating library routine); it clears the array's counters on `stream`
- * before launching.  The first call on a device looks up the array's device
- * address, so make it before any stream capture.  All calls on a device
- * share the one array: calls that overlap on the GPU race and must not be
- * issued (serialise them on one stream).  Arguments and results are those of
- * moe_ffn_forward. */
+ * it fail with MOE_EWORKSPACE before anything is enqueued.  The call
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library
+ * routine); it clears the array's counters on `stream` before launching,
+ * all but the status word (see moe_static_device_status).  The first call
+ * on a device (and the first after its context was re-created) looks up the
+ * array's device address, so make it before any stream capture.  All calls
+ * on a device share the one array: calls that overlap on the GPU race and
+ * must not be issued (serialise them on one stream).  Arguments, results and
+ * host-side errors are those of moe_ffn_forward; a failed address lookup or
+ * clear returns MOE_ECUDA and sets the sticky status. */
 MOE_API int moe_ffn_forward_static(const moe_dims *d, const uint16_t *x, int32_t rows,
                            const uint16_t *router_w, const uint8_t *expert_w8,
                            const float *expert_scales, const moe_fp8_expert *shared_w,
                            const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual,
                            const float *router_bias, void *stream);
+
+/* Device-side status of moe_ffn_forward_static's scratch array (no
+ * counterpart on the reference pages): synchronises `stream`, then reads the
+ * array's status word.  MOE_OK, or MOE_ETIMEOUT if a bounded wait inside a
+ * kernel of an earlier static call ran out (the outputs of that call are
+ * incomplete).  A non-OK word stays set across static calls until this
+ * function reports it, and is cleared once reported.  Returns MOE_ECUDA
+ * (sticky) if the read itself fails. */
+MOE_API int moe_static_device_status(void *stream);
+
+/* Test hook: moe_debug_wait_timeout against the static scratch array, so
+ * that moe_static_device_status reports MOE_ETIMEOUT. */
+MOE_API int moe_debug_wait_timeout_static(int32_t limit_us, void *stream);
 
 /* Size in bytes of the scratch array moe_ffn_forward_static uses. */
 MOE_API size_t moe_static_scratch_bytes(void);

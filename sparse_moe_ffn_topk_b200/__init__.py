@@ -46,7 +46,7 @@ EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe
             "moe_ffn_forward_path", "moe_status", "moe_reset_status", "moe_status_string",
             "moe_debug_inject_fault", "moe_kernel_launches", "moe_auto_path", "moe_ffn_forward_timed",
             "moe_device_status", "moe_debug_wait_timeout", "moe_ffn_forward_static",
-            "moe_static_scratch_bytes")
+            "moe_static_scratch_bytes", "moe_static_device_status", "moe_debug_wait_timeout_static")
 
 
 class MoeDims(ctypes.Structure):
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_forward_static.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P, P]
         L.moe_static_scratch_bytes.argtypes = []
         L.moe_static_scratch_bytes.restype = ctypes.c_size_t
+        L.moe_static_device_status.argtypes = [P]
+        L.moe_debug_wait_timeout_static.argtypes = [I32, P]
         L.moe_status.argtypes = []
         L.moe_reset_status.argtypes = []
         L.moe_reset_status.restype = None
@@ -250,6 +252,17 @@ def ffn_forward_static(dims, x, router_w, expert_w8, expert_scales, shared_w8, s
 
 def static_scratch_bytes() -> int:
     return int(lib().moe_static_scratch_bytes())
+
+
+def static_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (then clears, if set) the status
+    word of the scratch array that ffn_forward_static uses."""
+    return int(lib().moe_static_device_status(_stream(stream)))
+
+
+def debug_wait_timeout_static(limit_us: int, stream=None):
+    _check(lib().moe_debug_wait_timeout_static(int(limit_us), _stream(stream)),
+           "moe_debug_wait_timeout_static")
 
 
 def status() -> int:

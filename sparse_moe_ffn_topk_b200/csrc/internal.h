@@ -62,6 +62,27 @@ inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
     return L;
 }
 
+// ------------------------------------------------------------ C ABI plumbing
+// Sticky status gate of every entry: MOE_ECUDA after an earlier CUDA error or
+// when the host fault knob fires, else MOE_OK.
+int enter();
+// MOE_OK, or MOE_ECUDA (and the sticky status set) if `e` or the thread's
+// last CUDA error is an error.
+int finish(cudaError_t e);
+// Host-side argument checks of a forward call, apart from the workspace.
+int check_forward_args(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                       const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                       const uint16_t *shared_gate, const uint16_t *out, const uint16_t *residual,
+                       const float *router_bias, int32_t path, const int32_t *topk_idx_out,
+                       const float *topk_w_out, const float *shared_gate_sig_out);
+// The layer step on a checked workspace of at least workspace_bytes(d, rows)
+// bytes, after enter() returned MOE_OK.
+int run_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual, const float *router_bias,
+                void *ws, void *stream, int32_t path, int32_t *topk_idx_out, float *topk_w_out,
+                float *shared_gate_sig_out);
+
 // Device properties cached per device.
 struct DeviceInfo {
     int sm_count = 0;

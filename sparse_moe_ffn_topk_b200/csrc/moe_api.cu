@@ -33,6 +33,8 @@ int check_dims(const moe_dims *d)
     return MOE_OK;
 }
 
+}  // namespace
+
 // Common entry: sticky status and the host fault knob.
 int enter()
 {
@@ -59,8 +61,6 @@ int finish(cudaError_t e)
     }
     return MOE_OK;
 }
-
-}  // namespace
 
 TimingSession &timing_session()
 {
@@ -112,6 +112,95 @@ const DeviceInfo &device_info()
         g_dev_ready[dev] = true;
     }
     return g_dev[dev];
+}
+
+// Argument checks of a forward call that need no workspace (host only).
+int check_forward_args(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                       const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                       const uint16_t *shared_gate, const uint16_t *out, const uint16_t *residual,
+                       const float *router_bias, int32_t path, const int32_t *topk_idx_out,
+                       const float *topk_w_out, const float *shared_gate_sig_out)
+{
+    int st = check_dims(d);
+    if (st) return st;
+    if (rows < 0) return MOE_EINVAL;
+    if (!valid_path(path)) return MOE_EINVAL;
+    if (rows == 0) return MOE_OK;
+    if (!x || !router_w || !expert_w8 || !expert_scales || !shared_w || !shared_w->w8 ||
+        !shared_w->scales || !shared_gate || !out)
+        return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(expert_w8) || !aligned16(expert_scales) ||
+        !aligned16(shared_w->w8) || !aligned16(shared_w->scales) || !aligned16(shared_gate) ||
+        !aligned16(out) || (residual && !aligned16(residual)) ||
+        (router_bias && !aligned16(router_bias)) || (topk_idx_out && !aligned16(topk_idx_out)) ||
+        (topk_w_out && !aligned16(topk_w_out)) || (shared_gate_sig_out && !aligned16(shared_gate_sig_out)))
+        return MOE_EINVAL;
+    if (static_cast<const void *>(out) == static_cast<const void *>(x)) return MOE_EINVAL;
+    return MOE_OK;
+}
+
+// The layer step on a checked, large-enough workspace, after enter().
+int run_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual, const float *router_bias,
+                void *ws, void *stream, int32_t path, int32_t *topk_idx_out, float *topk_w_out,
+                float *shared_gate_sig_out)
+{
+    if (rows == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    path = resolve_path(*d, rows, path);
+    if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_NARROW) {
+        int rc = prefill_forward(*d, x, rows, router_w, expert_w8, expert_scales, shared_w->w8,
+                                 shared_w->scales, shared_gate, out, residual, router_bias, ws, s,
+                                 topk_idx_out, topk_w_out, shared_gate_sig_out, path == MOE_PATH_PREFILL_NARROW);
+        if (rc == MOE_ECUDA) g_status.store(MOE_ECUDA);
+        return rc;
+    }
+
+    const DecodeLayout L = decode_layout(*d, rows);
+    char *base = static_cast<char *>(ws);
+    int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
+    int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
+    float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
+    float *gs = shared_gate_sig_out ? shared_gate_sig_out : reinterpret_cast<float *>(base + L.gsig);
+
+    RouterLaunch ra;
+    ra.d = d;
+    ra.x = x;
+    ra.rows = rows;
+    ra.router_w = router_w;
+    ra.router_bias = router_bias;
+    ra.shared_gate = shared_gate;
+    ra.topk_idx = tidx;
+    ra.topk_w = tw;
+    ra.gsig = gs;
+    ra.logits = reinterpret_cast<float *>(base + L.logits);
+    ra.xq = reinterpret_cast<uint8_t *>(base + L.xq);
+    ra.xsc = reinterpret_cast<float *>(base + L.xsc);
+    ra.counters = counters;
+
+    ExpertsLaunch ea;
+    ea.d = d;
+    ea.x = x;
+    ea.xq = reinterpret_cast<const uint8_t *>(base + L.xq);
+    ea.xsc = reinterpret_cast<const float *>(base + L.xsc);
+    ea.rows = rows;
+    ea.expert_w8 = expert_w8;
+    ea.expert_scales = expert_scales;
+    ea.shared_w8 = shared_w->w8;
+    ea.shared_scales = shared_w->scales;
+    ea.residual = residual;
+    ea.out = out;
+    ea.topk_idx = tidx;
+    ea.topk_w = tw;
+    ea.gsig = gs;
+    ea.h_routed = reinterpret_cast<float *>(base + L.h_routed);
+    ea.h_shared = reinterpret_cast<float *>(base + L.h_shared);
+    ea.yslot = reinterpret_cast<float *>(base + L.yslot);
+    ea.counters = counters;
+    cudaError_t e = launch_router_topk(ra, s);
+    if (e != cudaSuccess) return finish(e);
+    return finish(launch_decode_experts(ea, s));
 }
 
 }  // namespace moe
@@ -178,79 +267,16 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
                          void *stream, int32_t path, int32_t *topk_idx_out, float *topk_w_out,
                          float *shared_gate_sig_out)
 {
-    int st = check_dims(d);
+    int st = check_forward_args(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out,
+                                residual, router_bias, path, topk_idx_out, topk_w_out, shared_gate_sig_out);
     if (st) return st;
-    if (rows < 0) return MOE_EINVAL;
-    if (!valid_path(path)) return MOE_EINVAL;
     if (rows == 0) return enter();  // a no-op: no pointer is read
-    if (!x || !router_w || !expert_w8 || !expert_scales || !shared_w || !shared_w->w8 ||
-        !shared_w->scales || !shared_gate || !out || !ws)
-        return MOE_EINVAL;
-    if (!aligned16(x) || !aligned16(router_w) || !aligned16(expert_w8) || !aligned16(expert_scales) ||
-        !aligned16(shared_w->w8) || !aligned16(shared_w->scales) || !aligned16(shared_gate) ||
-        !aligned16(out) || !aligned16(ws) || (residual && !aligned16(residual)) ||
-        (router_bias && !aligned16(router_bias)) || (topk_idx_out && !aligned16(topk_idx_out)) ||
-        (topk_w_out && !aligned16(topk_w_out)) || (shared_gate_sig_out && !aligned16(shared_gate_sig_out)))
-        return MOE_EINVAL;
-    if (static_cast<const void *>(out) == static_cast<const void *>(x)) return MOE_EINVAL;
-    if (ws_bytes < workspace_bytes(*d, rows < 1 ? 1 : rows)) return MOE_EWORKSPACE;
+    if (!ws || !aligned16(ws)) return MOE_EINVAL;
+    if (ws_bytes < workspace_bytes(*d, rows)) return MOE_EWORKSPACE;
     st = enter();
     if (st) return st;
-    if (rows == 0) return MOE_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    path = resolve_path(*d, rows, path);
-    if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_NARROW) {
-        int rc = prefill_forward(*d, x, rows, router_w, expert_w8, expert_scales, shared_w->w8,
-                                 shared_w->scales, shared_gate, out, residual, router_bias, ws, s,
-                                 topk_idx_out, topk_w_out, shared_gate_sig_out, path == MOE_PATH_PREFILL_NARROW);
-        if (rc == MOE_ECUDA) g_status.store(MOE_ECUDA);
-        return rc;
-    }
-
-    const DecodeLayout L = decode_layout(*d, rows);
-    char *base = static_cast<char *>(ws);
-    int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
-    int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
-    float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
-    float *gs = shared_gate_sig_out ? shared_gate_sig_out : reinterpret_cast<float *>(base + L.gsig);
-
-    RouterLaunch ra;
-    ra.d = d;
-    ra.x = x;
-    ra.rows = rows;
-    ra.router_w = router_w;
-    ra.router_bias = router_bias;
-    ra.shared_gate = shared_gate;
-    ra.topk_idx = tidx;
-    ra.topk_w = tw;
-    ra.gsig = gs;
-    ra.logits = reinterpret_cast<float *>(base + L.logits);
-    ra.xq = reinterpret_cast<uint8_t *>(base + L.xq);
-    ra.xsc = reinterpret_cast<float *>(base + L.xsc);
-    ra.counters = counters;
-
-    ExpertsLaunch ea;
-    ea.d = d;
-    ea.x = x;
-    ea.xq = reinterpret_cast<const uint8_t *>(base + L.xq);
-    ea.xsc = reinterpret_cast<const float *>(base + L.xsc);
-    ea.rows = rows;
-    ea.expert_w8 = expert_w8;
-    ea.expert_scales = expert_scales;
-    ea.shared_w8 = shared_w->w8;
-    ea.shared_scales = shared_w->scales;
-    ea.residual = residual;
-    ea.out = out;
-    ea.topk_idx = tidx;
-    ea.topk_w = tw;
-    ea.gsig = gs;
-    ea.h_routed = reinterpret_cast<float *>(base + L.h_routed);
-    ea.h_shared = reinterpret_cast<float *>(base + L.h_shared);
-    ea.yslot = reinterpret_cast<float *>(base + L.yslot);
-    ea.counters = counters;
-    cudaError_t e = launch_router_topk(ra, s);
-    if (e != cudaSuccess) return finish(e);
-    return finish(launch_decode_experts(ea, s));
+    return run_forward(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out, residual,
+                       router_bias, ws, stream, path, topk_idx_out, topk_w_out, shared_gate_sig_out);
 }
 
 int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,

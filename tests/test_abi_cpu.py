@@ -138,3 +138,53 @@ def test_status_strings(L):
 def test_dims_match_input_generator():
     for d in (mi.TINY, mi.QWEN36_35B_A3B, mi.QWEN35_397B_A17B):
         assert moe.workspace_bytes(d, 1) > 0
+
+
+# ------------------------------------------------------------ the static entry
+
+def static_fwd(L, d, rows=1, x=FAKE, out=FAKE + 4096, shared=True):
+    sh = moe.MoeFp8Expert(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE)) if shared else None
+    P = lambda a: ctypes.c_void_p(a) if a else None
+    return L.moe_ffn_forward_static(ctypes.byref(d) if d is not None else None, P(x), rows, P(FAKE), P(FAKE),
+                                    P(FAKE), ctypes.byref(sh) if sh else None, P(FAKE), P(out), None, None,
+                                    None)
+
+
+def test_static_scratch_size_matches_header(L):
+    src = open(os.path.join(ROOT, "include", "moe_ffn.h")).read()
+    assert "16 MiB" in src
+    assert moe.static_scratch_bytes() == 16 << 20
+
+
+def test_static_entry_rejects_on_host_before_any_device_call(L):
+    """Every rejection below returns before the scratch address is looked up
+    or anything is enqueued (this machine has no GPU: a device call would
+    fail with MOE_ECUDA instead)."""
+    moe.reset_status()
+    d = D()
+    assert static_fwd(L, None) == moe.MOE_EINVAL                   # null dims
+    assert static_fwd(L, d, rows=-1) == moe.MOE_EINVAL
+    assert static_fwd(L, d, x=0) == moe.MOE_EINVAL
+    assert static_fwd(L, d, x=FAKE + 8) == moe.MOE_EINVAL          # misaligned
+    assert static_fwd(L, d, shared=False) == moe.MOE_EINVAL
+    assert static_fwd(L, d, out=FAKE) == moe.MOE_EINVAL            # out aliases x
+    assert static_fwd(L, D(i=500)) == moe.MOE_EUNSUPPORTED
+    assert static_fwd(L, d, rows=0) == moe.MOE_OK                  # a no-op
+    assert static_fwd(L, d, rows=0, x=0, out=0) == moe.MOE_OK
+    big = mi.QWEN35_397B_A17B
+    dd = moe.MoeDims(big.hidden, big.n_experts, big.top_k, big.inter, big.shared_inter)
+    assert moe.workspace_bytes(dd, 128) > moe.static_scratch_bytes()
+    assert static_fwd(L, dd, rows=128) == moe.MOE_EWORKSPACE       # beyond the scratch array
+    assert moe.status() == moe.MOE_OK                              # nothing above touched CUDA
+
+
+def test_static_entry_respects_sticky_status_and_fault_knob(L):
+    d = D()
+    moe.reset_status()
+    moe.debug_inject_fault(1)
+    assert static_fwd(L, d) == moe.MOE_ECUDA       # the knob fires before anything is enqueued
+    assert moe.status() == moe.MOE_ECUDA
+    assert static_fwd(L, d) == moe.MOE_ECUDA       # sticky
+    assert L.moe_static_device_status(None) == moe.MOE_ECUDA
+    moe.reset_status()
+    assert moe.status() == moe.MOE_OK

@@ -70,3 +70,22 @@ def test_static_scratch_rejects_shapes_beyond_its_size():
     with pytest.raises(moe.MoeError) as e:
         moe.ffn_forward_static(d, x, dummyb, dummy8, dummyf, dummy8, dummyf, dummyb, out)
     assert e.value.status == moe.MOE_EWORKSPACE
+
+
+def test_static_timeout_is_reported_and_not_erased_by_the_next_call():
+    """A bounded wait that runs out on the scratch array (a 2 ms wait on an
+    mbarrier nothing completes) shows up as MOE_ETIMEOUT through
+    moe_static_device_status, even after another static call, and is
+    reported once."""
+    d = mi.TINY
+    dev, xs = _inputs(d, 4, seed=6)
+    assert moe.static_device_status() == moe.MOE_OK
+    moe.debug_wait_timeout_static(2000)
+    out = torch.empty(4, d.hidden, dtype=torch.bfloat16, device="cuda")
+    moe.ffn_forward_static(d, xs[0], dev["router_w"], dev["expert_w8"], dev["expert_scales"], dev["shared_w8"],
+                           dev["shared_scales"], dev["shared_gate"], out)
+    assert moe.static_device_status() == moe.MOE_ETIMEOUT
+    assert moe.static_device_status() == moe.MOE_OK
+    assert moe.status() == moe.MOE_OK
+    ref, got = _run_both(d, dev, xs[1])        # the array still serves correct calls
+    _check_close(ref, got)
