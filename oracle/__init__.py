@@ -61,6 +61,7 @@ def _load():
         lib.oracle_expert_ffn.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, P, P]
         lib.oracle_moe_forward.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, P, P, P, P, P,
                                            P, P, P, P, P, P, P, P, P, ctypes.c_int32]
+        lib.oracle_rmsnorm.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
         lib.oracle_moe_forward_dense.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, P, P,
                                                  P, P, P, P, P, P, P, P, P, P, ctypes.c_int32]
         _lib = lib
@@ -155,6 +156,30 @@ def expert_ffn(w8: np.ndarray, scales: np.ndarray, H: int, I: int, x: np.ndarray
                                      _ptr(np.ascontiguousarray(scales, dtype=np.float32)),
                                      H, I, _ptr(x), _ptr(y)), "oracle_expert_ffn")
     return y
+
+
+def rmsnorm(resid: np.ndarray, norm_w: np.ndarray, eps: float):
+    """RMSNorm of each row of the residual stream (bf16 bits [rows, H]) times
+    the norm weight (bf16 bits [H]) -> (x float64 [rows, H] before rounding,
+    x as bf16 bits)."""
+    r = np.ascontiguousarray(resid, dtype=np.uint16)
+    rows, H = r.shape
+    xd = np.empty((rows, H), dtype=np.float64)
+    xb = np.empty((rows, H), dtype=np.uint16)
+    _check(_load().oracle_rmsnorm(H, rows, _ptr(r), _ptr(np.ascontiguousarray(norm_w, dtype=np.uint16)),
+                                  float(eps), _ptr(xd), _ptr(xb)), "oracle_rmsnorm")
+    return xd, xb
+
+
+def moe_forward_norm(d, resid, norm_w, eps, router_w, expert_w8, expert_scales, shared_w8, shared_scales,
+                     shared_gate, router_bias=None, forced_idx=None, want_logits=True,
+                     nthreads: int | None = None) -> ForwardResult:
+    """The layer behind its RMSNorm: x = bf16(rmsnorm(resid) * norm_w), out =
+    resid + layer(x), in double before the output rounding."""
+    _, xb = rmsnorm(resid, norm_w, eps)
+    return moe_forward(d, xb, router_w, expert_w8, expert_scales, shared_w8, shared_scales, shared_gate,
+                       residual=resid, router_bias=router_bias, forced_idx=forced_idx, want_logits=want_logits,
+                       nthreads=nthreads)
 
 
 @dataclass

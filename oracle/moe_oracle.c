@@ -172,6 +172,37 @@ static double dq(const uint8_t *q, const float *s, int64_t cols, int64_t r, int6
     return oracle_e4m3_decode(q[r * cols + c]) * (double)s[(r / 128) * (cols / 128) + (c / 128)];
 }
 
+/* ------------------------------------------------------------- RMSNorm */
+
+/* The norm in front of the MoE block ("Qwen3.6-35B-A3B-FP8 on NVIDIA GB10"
+ * blueprint page, Kernels table: norm::rms_norm and
+ * norm::residual_add_rms_norm, whose bf16 output feeds the router GEMV;
+ * "Neurarch Qwen3-8B" page: RMSNorm over the hidden size before each SwiGLU
+ * block).  For each row r of the residual stream (bf16 [rows, H]):
+ *   ms = sum_h r_h^2 / H,  inv = 1 / sqrt(ms + eps),  x_h = (r_h * inv) * w_h,
+ * in double; xd (nullable) receives x before rounding, x_bf16 the nearest
+ * bf16 (ties to even) of each x_h. */
+int oracle_rmsnorm(int32_t H, int32_t rows, const uint16_t *resid, const uint16_t *norm_w, double eps,
+                   double *xd, uint16_t *x_bf16)
+{
+    if (H <= 0 || rows < 0 || !resid || !norm_w || !x_bf16 || !(eps >= 0.0)) return -1;
+    for (int t = 0; t < rows; ++t) {
+        const uint16_t *r = resid + (int64_t)t * H;
+        double ss = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double v = oracle_bf16_to_f64(r[h]);
+            ss += v * v;
+        }
+        double inv = 1.0 / sqrt(ss / (double)H + eps);
+        for (int h = 0; h < H; ++h) {
+            double v = (oracle_bf16_to_f64(r[h]) * inv) * oracle_bf16_to_f64(norm_w[h]);
+            if (xd) xd[(int64_t)t * H + h] = v;
+            x_bf16[(int64_t)t * H + h] = oracle_f64_to_bf16(v);
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------ the layer */
 
 static double sigmoid(double a) { return 1.0 / (1.0 + exp(-a)); }

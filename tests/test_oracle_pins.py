@@ -484,3 +484,48 @@ def test_router_entry_equals_forward_routing_35b():
     lg, idx, _, _ = oracle.router_topk(d, x, rw, g)
     L = mi.make_layer(d, seed=0, experts=set(idx.ravel().tolist()))
     _router_vs_forward(d, L, x)
+
+
+# ------------------------------------------------------------------ RMSNorm
+
+def _bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_rmsnorm_hand_cases():
+    """Cases with exact results: a row of 2s has mean square 4, so with eps = 0
+    x = w exactly and with eps = 12 x = 2 w / 4 = w / 2 exactly (an eps added after
+    the root, or a mean over H - 1, fails); a row (8, 0, ..., 0) of H = 128
+    has mean square 1/2, so x_0 = 8 sqrt(2) w_0, whose nearest bf16 is 11.3125."""
+    H = 128
+    w = _bf16_bits(np.linspace(-3.0, 3.0, H))
+    wd = oracle.bf16_bits_to_f64(w)
+    r = _bf16_bits(np.full((2, H), 2.0))
+    r[1] = _bf16_bits(np.full(H, -2.0))
+    xd, xb = oracle.rmsnorm(r, w, 0.0)
+    assert np.array_equal(xd[0], wd) and np.array_equal(xd[1], -wd)
+    assert np.array_equal(xb[0], w)
+    xd, _ = oracle.rmsnorm(r[:1], w, 12.0)
+    assert np.array_equal(xd[0], wd / 2.0)
+    one = _bf16_bits(np.ones(H))
+    r2 = np.zeros((1, H), dtype=np.uint16)
+    r2[0, 0] = _bf16_bits([8.0])[0]
+    xd, xb = oracle.rmsnorm(r2, one, 0.0)
+    assert abs(xd[0, 0] - 8.0 * math.sqrt(2.0)) <= 1e-14
+    assert oracle.bf16_to_f64(int(xb[0, 0])) == 11.3125
+    assert np.all(xd[0, 1:] == 0.0)
+
+
+def test_rmsnorm_matches_torch_float64():
+    """Random residual rows against torch's rms_norm in float64 (a library
+    routine)."""
+    H, rows, eps = 384, 5, 1e-6
+    g = torch.Generator().manual_seed(3)
+    r = _bf16_bits((torch.randn(rows, H, generator=g) * 3.0).numpy())
+    w = _bf16_bits((1.0 + 0.1 * torch.randn(H, generator=g)).numpy())
+    xd, xb = oracle.rmsnorm(r, w, eps)
+    rt = torch.from_numpy(oracle.bf16_bits_to_f64(r))
+    wt = torch.from_numpy(oracle.bf16_bits_to_f64(w))
+    ref = torch.nn.functional.rms_norm(rt, (H,), weight=wt, eps=eps).numpy()
+    assert np.allclose(xd, ref, rtol=1e-14, atol=0.0)
+    assert np.array_equal(xb, oracle.round_to_bf16(xd))
