@@ -45,6 +45,11 @@ WORKLOAD = "Qwen3.6-35B-A3B-shaped MoE FFN layer, decode rows=1"
 N_INSTANCES = 16
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+# The arithmetic each leg computes in.
+DECODE_DTYPE = ("fp8e4m3 weights (fp32 block scales) x bf16 x for gate/up and x fp32 h for down, "
+                "exact products, fp32 accumulate")
+GROUPED_DTYPE = ("fp8e4m3 weights (fp32 block scales) x activations as two e4m3 terms (hi + lo, fp32 scale "
+                 "per 128 block), fp32 accumulate")
 
 
 # ----------------------------------------------------------------- helpers
@@ -90,7 +95,8 @@ def algorithmic_bytes(d, rows: int, n_active: int, residual: bool = False) -> di
     dn = (n_active * (I * H + 4 * (H // 128) * (I // 128)) + Is * H + 4 * (H // 128) * (Is // 128)
           + 4 * rows * (k * I + Is) + 2 * rows * H)
     rt = router + 2 * rows * H + rows * (8 * k + 4)
-    return {"total": n_active * exp_b + sh_b + router + act, "experts": n_active * exp_b + sh_b,
+    total = n_active * exp_b + sh_b + router + act
+    return {"total": total, "experts": n_active * exp_b + sh_b, "decode_step": total,
             "router_topk": rt, "gate_up": gu, "down_blend": dn}
 
 
@@ -465,7 +471,7 @@ def prefill_leg(args, d, inst, dist: Dist, bus, hbm_peak, bf16_peak, peak_kind):
            "rows": rows, "steps": kp, "us_per_layer": round(step_s * 1e6, 2),
            "tokens_per_s": round(aggregate(kp * rows, dist.world, s), 1),
            "tflops": round(tflops, 1), "fp8_peak_tflops": round(fp8_peak, 1),
-           "frac_of_fp8_peak": round(tflops / dist.world / fp8_peak, 4),
+           "frac_of_fp8_peak": round(tflops / dist.world / fp8_peak, 4), "dtype": GROUPED_DTYPE,
            "hbm_gb_s": round(aggregate(kp * prefill_bytes(d, rows, n_active), dist.world, s) / 1e9, 1),
            "flops_per_step": int(fl["total"]), "distinct_experts": n_active,
            "max_expert_rows": int(max(counts)), "mean_expert_rows": round(sum(counts) / len(counts), 1),
@@ -545,6 +551,19 @@ def e2e_measure(dims, insts, rows: int, steps: int, dist: Dist, seed: int):
     return ms, 2 * rows * dims.hidden, 2 * rows * dims.hidden
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def cpu_oracle_leg(dims, layer, rows: int, seed: int, budget_s: float = 12.0, max_steps: int = 40):
     """The CPU oracle, as it stands, on a bounded sample of the workload:
     consecutive rows=`rows` layer steps on fresh x until the time budget."""
@@ -584,7 +603,7 @@ def run_ours(args, dist: Dist):
         bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
     except Exception:
         pass
-    names = ["router_topk", "gate_up", "down_blend"]
+    names = ["decode_step"]
 
     def x_set(rows, n):
         return [torch.from_numpy(mi.make_x(d, rows, seed=args.seed + 1, stream=1000 * rows + i).view("int16"))
@@ -610,7 +629,7 @@ def run_ours(args, dist: Dist):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_s * 1000.0 / args.steps, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8e4m3-weights x bf16-activations, fp32 accumulate", "data": "synthetic (seeded)",
+        "dtype": DECODE_DTYPE, "data": "synthetic (seeded)",
         "config": {"workload": WORKLOAD, "hidden": d.hidden, "experts": d.n_experts, "top_k": d.top_k,
                    "inter": d.inter, "shared_inter": d.shared_inter, "rows": rows,
                    "l2": f"inputs larger than L2: {N_INSTANCES} rotating weight instances "
@@ -654,6 +673,7 @@ def run_ours(args, dist: Dist):
                             "hbm_frac_of_measured": round(gbs64 / dist.world / hbm_peak, 4),
                             "tokens_per_s": round(aggregate(k64 * r64, dist.world, s64), 1),
                             "distinct_experts_per_step": round(u64, 1), "steps": k64,
+                            "dtype": GROUPED_DTYPE if moe.auto_path(d, r64) != moe.MOE_PATH_DECODE else DECODE_DTYPE,
                             "kernels": {moe.MOE_PATH_DECODE: "decode", moe.MOE_PATH_PREFILL: "grouped",
                                         moe.MOE_PATH_PREFILL_NARROW: "narrow"}[moe.auto_path(d, r64)]}
 
@@ -678,9 +698,19 @@ def run_ours(args, dist: Dist):
         steps, secs, cores, na = cpu_oracle_leg(d, layer, rows, args.seed)
         byc = algorithmic_bytes(d, rows, statistics.mean(na))
         result["cpu_baseline"] = {"value": round(steps * byc["total"] / secs / 1e9, 4), "unit": "GB/s",
-                                  "cores": cores, "kind": "oracle",
+                                  "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+                                  "host_threads": os.cpu_count(),
                                   "sample": f"{steps} layer steps at rows={rows} (fresh x each), "
                                             f"{secs:.1f} s, {secs / steps * 1e3:.1f} ms/layer"}
+        if not args.no_extras:
+            # the oracle threaded over rows, at 64 rows
+            s64n, s64t, c64, na64 = cpu_oracle_leg(d, layer, 64, args.seed, budget_s=10.0, max_steps=4)
+            by64c = algorithmic_bytes(d, 64, statistics.mean(na64))
+            result["cpu_baseline"]["rows64"] = {
+                "value": round(s64n * by64c["total"] / s64t / 1e9, 4), "unit": "GB/s", "threads": c64,
+                "ms_per_layer": round(s64t / s64n * 1e3, 1),
+                "tokens_per_s": round(s64n * 64 / s64t, 1),
+                "sample": f"{s64n} layer steps at rows=64 (fresh x each), {s64t:.1f} s"}
     del b1
     return result
 

@@ -78,12 +78,12 @@ extern "C" {
 #define MOE_ETIMEOUT -5      /* a bounded wait inside a kernel ran out (device status word) */
 
 #define MOE_PATH_AUTO 0      /* by rows: MOE_AUTO_DECODE_MAX_ROWS, MOE_AUTO_NARROW_MAX_PAIRS below */
-#define MOE_PATH_DECODE 1    /* FP8 weight-streaming GEMVs (16-row tensor-core tiles) with expert dedup */
+#define MOE_PATH_DECODE 1    /* one persistent kernel per MOE_DECODE_MAX_ROWS rows: bf16 x and f32 h against FP8 weights */
 #define MOE_PATH_PREFILL 2   /* token permute -> tcgen05 FP8 grouped GEMMs -> unpermute */
 #define MOE_PATH_PREFILL_NARROW 3  /* the same pipeline with the grouped GEMMs tiled as 128 weight rows (the
                                      MMA's M) x up to 32 rows of one expert (its N): for few rows per expert;
                                      MOE_EUNSUPPORTED when H, I or Is exceeds 4096 */
-#define MOE_DECODE_MAX_ROWS 64       /* the decode path's tiles are sized for at most this many rows */
+#define MOE_DECODE_MAX_ROWS 4        /* rows per decode-step launch; more rows run as several launches */
 #define MOE_AUTO_DECODE_MAX_ROWS 3    /* MOE_PATH_AUTO: the decode kernels up to this many rows; then the
                                          narrow grouped GEMMs while rows * k <= MOE_AUTO_NARROW_MAX_PAIRS * E
                                          (an expert's average routed rows), then the 128-row token tiles;
@@ -155,6 +155,29 @@ MOE_API int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t r
                          const float *router_bias, void *ws, size_t ws_bytes, void *stream,
                          int32_t path, int32_t *topk_idx, float *topk_w,
                          float *shared_gate_sig);
+
+/* The layer behind its RMSNorm, with the residual join:
+ *   x   = bf16( (resid / sqrt(mean_h resid^2 + eps)) * norm_w ),
+ *   out = resid + [sum_r w_r E_{idx_r}(x) + sigmoid(g.x) E_shared(x)],  rounded once to bf16.
+ * After the "Qwen3.6-35B-A3B-FP8 on NVIDIA GB10" blueprint page, Kernels table
+ * (norm::rms_norm / norm::residual_add_rms_norm: the bf16 norm output feeds
+ * the router GEMV of the MoE block) and the "Neurarch Qwen3-8B" page (an
+ * RMSNorm over the hidden size before each SwiGLU block).  The mean square,
+ * the scaling and the product with norm_w are computed in double and
+ * rounded once to bf16.  On the decode path the norm runs inside the one
+ * decode-step kernel, so a stack of layers is one launch per layer; on the
+ * grouped-GEMM paths a norm kernel runs first.  resid bf16 [rows, H],
+ * norm_w bf16 [H], eps >= 0 (the pages give none; Qwen models use 1e-6);
+ * out may alias resid (an in-place update of the residual stream).  path is
+ * a MOE_PATH_* (MOE_PATH_AUTO as moe_ffn_forward chooses).  Workspace:
+ * moe_workspace_bytes(d, rows).  Errors as moe_ffn_forward, MOE_EINVAL also
+ * for a null or misaligned norm_w or eps < 0. */
+MOE_API int moe_ffn_forward_norm(const moe_dims *d, const uint16_t *resid, int32_t rows,
+                         const uint16_t *norm_w, float eps, const uint16_t *router_w,
+                         const uint8_t *expert_w8, const float *expert_scales,
+                         const moe_fp8_expert *shared_w, const uint16_t *shared_gate, uint16_t *out,
+                         const float *router_bias, void *ws, size_t ws_bytes, void *stream,
+                         int32_t path);
 
 /* Number of kernels one moe_ffn_forward_path call launches for these dims,
  * rows and path (MOE_PATH_AUTO resolved as moe_ffn_forward does); 0 for

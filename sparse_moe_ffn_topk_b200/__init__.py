@@ -38,7 +38,7 @@ MOE_PATH_AUTO = 0
 MOE_PATH_DECODE = 1
 MOE_PATH_PREFILL = 2
 MOE_PATH_PREFILL_NARROW = 3
-MOE_DECODE_MAX_ROWS = 64
+MOE_DECODE_MAX_ROWS = 4
 MOE_AUTO_DECODE_MAX_ROWS = 3
 MOE_AUTO_NARROW_MAX_PAIRS = 32
 
@@ -46,7 +46,8 @@ EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe
             "moe_ffn_forward_path", "moe_status", "moe_reset_status", "moe_status_string",
             "moe_debug_inject_fault", "moe_kernel_launches", "moe_auto_path", "moe_ffn_forward_timed",
             "moe_device_status", "moe_debug_wait_timeout", "moe_ffn_forward_static",
-            "moe_static_scratch_bytes", "moe_static_device_status", "moe_debug_wait_timeout_static")
+            "moe_static_scratch_bytes", "moe_static_device_status", "moe_debug_wait_timeout_static",
+            "moe_ffn_forward_norm")
 
 
 class MoeDims(ctypes.Structure):
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
                                       ctypes.c_size_t, P]
         L.moe_ffn_forward_path.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P,
                                            P, ctypes.c_size_t, P, I32, P, P, P]
+        L.moe_ffn_forward_norm.argtypes = [DP, P, I32, P, ctypes.c_float, P, P, P, ctypes.POINTER(MoeFp8Expert), P,
+                                           P, P, P, ctypes.c_size_t, P, I32]
         L.moe_kernel_launches.argtypes = [DP, I32, I32]
         L.moe_kernel_launches.restype = I32
         L.moe_auto_path.argtypes = [DP, I32]
@@ -200,6 +203,18 @@ def ffn_forward_path(dims, x, router_w, expert_w8, expert_scales, shared_w8, sha
            "moe_ffn_forward_path")
 
 
+def ffn_forward_norm(dims, resid, norm_w, eps, router_w, expert_w8, expert_scales, shared_w8, shared_scales,
+                     shared_gate, out, ws, router_bias=None, path=MOE_PATH_AUTO, stream=None):
+    """out = resid + layer(bf16(rmsnorm(resid) * norm_w)); out may be resid."""
+    d = _dims(dims)
+    sh = MoeFp8Expert(_ptr(shared_w8), _ptr(shared_scales))
+    _check(lib().moe_ffn_forward_norm(ctypes.byref(d), _ptr(resid), _rows(resid), _ptr(norm_w), float(eps),
+                                      _ptr(router_w), _ptr(expert_w8), _ptr(expert_scales), ctypes.byref(sh),
+                                      _ptr(shared_gate), _ptr(out), _ptr(router_bias), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream), int(path)),
+           "moe_ffn_forward_norm")
+
+
 def kernel_launches(dims, rows: int, path=MOE_PATH_AUTO) -> int:
     return int(lib().moe_kernel_launches(ctypes.byref(_dims(dims)), int(rows), int(path)))
 
@@ -290,7 +305,7 @@ class MoeLayer:
     and optionally router_bias [E] fp32.
     """
 
-    def __init__(self, dims, weights: dict, max_rows: int = MOE_DECODE_MAX_ROWS, device="cuda"):
+    def __init__(self, dims, weights: dict, max_rows: int = 64, device="cuda"):
         self.dims = _dims(dims)
         self.device = torch.device(device)
         self.w = {k: (v.to(self.device).contiguous() if v is not None else None) for k, v in weights.items()}

@@ -237,6 +237,32 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
+// Nearest bf16 of a double, ties to even, rounded once from the double (not
+// through float): for |v| in the normal bf16 range the double's fraction is
+// rounded at its 8th significant bit; below it, at the subnormal step 2^-133.
+__device__ __forceinline__ uint16_t f64_to_bf16_rn(double v)
+{
+    unsigned long long u = (unsigned long long)__double_as_longlong(v);
+    const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
+    unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
+    if (a >= 0x7FF0000000000000ull) return f32_to_bf16_bits((float)v);  // inf, NaN
+    if (a >= 0x3810000000000000ull) {                                     // >= 2^-126
+        a += 0x00000FFFFFFFFFFFull + ((a >> 45) & 1ull);
+        a &= ~0x00001FFFFFFFFFFFull;
+        const float f = (float)__longlong_as_double((long long)a);        // exact, or inf past the range
+        return (uint16_t)(sign | (uint16_t)(__float_as_uint(f) >> 16));
+    }
+    const double m = rint(__longlong_as_double((long long)a) * 0x1p133);  // subnormal steps, ties to even
+    return (uint16_t)(sign | (uint16_t)m);
+}
+
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Record a device-side error in the workspace status word (first one wins).
 __device__ __forceinline__ void set_status(int32_t *counters, int32_t code)
 {

@@ -1,0 +1,1203 @@
+// decode_step.cu -- the decode step (up to kStepMaxRows rows) as one
+// persistent kernel, at the arithmetic the pages give for this path.
+//
+// The pages' decode chain ("Qwen3.6-35B-A3B-FP8 on NVIDIA GB10" blueprint
+// page, Kernels table) is a router GEMV, a top-k softmax, the FP8 gate/up
+// product with the shared expert fused, SiLU and the down product, and a
+// weighted blend; its Precision table reads the fp8 block128x128 weights
+// against bf16 activations for gate/up and against f32 activations for down.
+// The "colibri #1992" PR page gives the decode GEMV's shape: a warp per
+// output row, 16 bytes a lane, the activation in shared memory.
+//
+// Here one CTA per SM runs the whole step with two grid-wide barriers:
+//
+//   P0  (before the programmatic-dependent-launch wait: weights only)
+//       the producer warp starts TMA copies of this CTA's router rows and of
+//       its shared-expert gate/up rows;
+//   P1  x -> shared memory as f16 with one power-of-two scale per
+//       (row, 128 block); the CTA's router rows (and the gate vector) against
+//       bf16 x in fp32 -> logits in the workspace;          grid barrier 1
+//   P2  every CTA takes the top-k of every row from the logits (no CTA
+//       waits for a designated one), builds the same list of distinct
+//       experts, and walks its share of gate/up units (8 gate + 8 up rows
+//       of one expert): h = silu(gate) * up in fp32 -> workspace; the
+//       producer keeps the ring full, the down rows of the active experts
+//       following the gate/up rows;                          grid barrier 2
+//   P3  h -> shared memory as three f16 terms per value (they sum exactly
+//       to the fp32 h) with one power-of-two scale per (slot, 128 block);
+//       the CTA's output rows: each expert's down product, then the blend
+//       in rank order (+ shared expert * sigmoid gate, + residual), one
+//       rounding to bf16.
+//
+// Tensor cores without narrowing the activations: the products run on
+// mma.m16n8k16 with f16 operands and fp32 accumulation.  Every e4m3 weight
+// is exactly an f16 value; a bf16 activation times a power of two is exactly
+// an f16 value (8 significant bits) unless it lies more than 2^31 below its
+// block's largest magnitude; an fp32 h is exactly the sum of three f16 terms
+// under the same condition (2^31 below the block maximum, else the error is
+// below 2^-39 of that maximum).  Products of f16 values are exact in fp32,
+// so the arithmetic is the pages': bf16 x times fp8 weights and f32 h times
+// fp8 weights, accumulated in fp32; each 128-wide K block's sum is then
+// scaled by its weight block scale and the activation's power of two.
+//
+// Weight tiles arrive by 4-D TMA boxes [K windows of 128 bytes][8 rows][128
+// bytes] with the 128-byte swizzle, which makes the fragment reads below free
+// of bank conflicts: lane (g, q) reads row g's 16-byte chunks 2q and 2q+1 of
+// each window, and the swizzle spreads rows 2p and 2p+1 over all 8 chunks.
+// The K order inside a window is permuted the same way for the weights and
+// the activations (a dot product does not depend on the order of its terms):
+// in MMA step s of a window, lane quad q holds bytes 32q + 4s .. 32q + 4s + 3.
+//
+// Every wait is bounded (kWaitLimitNs): a wait that runs out records
+// MOE_ETIMEOUT in the workspace status word; the CTA waits (bounded) for its
+// copies in flight and leaves.
+#include <math.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "launch.h"
+#include "tcgen05.cuh"
+#include "topk.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kSlot = 16384;           // ring slot bytes
+constexpr int kMaxNt = 8;              // output 8-row tiles per CTA
+constexpr uint32_t kSmemCap = 232448;  // dynamic shared memory per block (B200 opt-in)
+
+// ------------------------------------------------------------ device helpers
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two)
+{
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// D += A * B: m16n8k16, f16 operands, fp32 accumulator.
+//   a0: row g, k 2q..2q+1     a1: row g+8, k 2q..     a2: row g, k 2q+8..   a3: row g+8, k 2q+8..
+//   b0: col g, k 2q..2q+1     b1: col g, k 2q+8..
+//   d0, d1: row g, cols 2q, 2q+1      d2, d3: row g+8, cols 2q, 2q+1
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                            uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+        : "memory");
+}
+
+// The power of two that brings a block's largest magnitude into [2^14, 2^15)
+// (so that every value fits f16 with its bits intact), as its exponent,
+// clamped so that 2^s and 2^-s are normal floats.
+__device__ __forceinline__ int block_shift(float amax)
+{
+    if (!(amax > 0.f) || !isfinite(amax)) return 0;
+    const int be = (int)((__float_as_uint(amax) >> 23) & 0xFFu);  // 0 for a subnormal
+    return max(-100, min(100, 141 - be));
+}
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }
+
+__device__ __forceinline__ int atomic_add_release_gpu(int32_t *p, int v)
+{
+    int old;
+    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// A bounded wait, taken by lane 0 for the whole warp, for item q in ring
+// slot s: the result is the same in every lane and the warp is converged
+// again afterwards, as the mma.sync.aligned instructions that follow require.
+//
+// A warp's items are not consecutive in the ring (each warp takes its own
+// units), so a warp can reach item q while its slot still holds an older
+// item; a parity wait alone would then see the phase two back (same parity)
+// completed.  The producer writes q into the slot's tag after arming the
+// slot's barrier for q, which it does only once the slot's previous item was
+// consumed: once the tag reads q, phase q / ns is the barrier's current (or
+// just completed) phase and the parity wait is exact.
+__device__ __forceinline__ bool wait_item(const volatile int32_t *tag, uint64_t *full, int s, int q, int ns)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) {
+        if (tag[s] != q) {
+            const uint64_t t0 = globaltimer_ns();
+            while (tag[s] != q) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if (ok) ok = mbar_wait(&full[s], (uint32_t)((q / ns) & 1), kWaitLimitNs);
+    }
+    ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
+// The router items' wait (their slots' first use): lane 0 for the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, kWaitLimitNs);
+    ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
+// A wait that ran out: MOE_ETIMEOUT in the status word, and where this CTA
+// gave up (the first time) in its diagnostic word: kind << 24 | item.
+//   kind 1 router rows, 2 gate/up item (consumer), 3 down item (consumer),
+//   4 producer before grid barrier 2, 5 producer after it, 6 grid barrier 1,
+//   7 grid barrier 2.
+__device__ __forceinline__ void gave_up(int32_t *counters, int kind, int item)
+{
+    set_status(counters, MOE_ETIMEOUT);
+    atomicCAS(&counters[kCtrStepDiag + blockIdx.x], 0, (kind << 24) | (item & 0xFFFFFF));
+}
+
+// Progress markers of a development build (-DMOE_STEP_TRACE): per (CTA,
+// warp) the last point reached, stage << 24 | item.  Nothing in the library
+// build.
+#ifdef MOE_STEP_TRACE
+#define STEP_MARK(stage, item)                                                                              \
+    do {                                                                                                    \
+        if ((threadIdx.x & 31) == 0)                                                                        \
+            ((volatile int32_t *)p.counters)[kCtrStepDiag + 256 + blockIdx.x * 16 + (threadIdx.x >> 5)] =   \
+                ((stage) << 24) | ((item) & 0xFFFFFF);                                                      \
+    } while (0)
+// the words of a slot's full and empty barriers when a wait ran out
+#define STEP_SNAP(slot)                                                                                     \
+    do {                                                                                                    \
+        unsigned long long f_, e_;                                                                          \
+        asm volatile("ld.shared.b64 %0, [%1];" : "=l"(f_) : "r"(smem_u32(&full[slot])));                   \
+        asm volatile("ld.shared.b64 %0, [%1];" : "=l"(e_) : "r"(smem_u32(&empty[slot])));                  \
+        int32_t *d_ = p.counters + kCtrStepDiag + 1024 + blockIdx.x * 4;                                    \
+        if (atomicCAS(d_, 0, (int)(f_ & 0xFFFFFFFF)) == 0) {                                                \
+            d_[1] = (int)(f_ >> 32);                                                                        \
+            d_[2] = (int)(e_ & 0xFFFFFFFF);                                                                 \
+            d_[3] = (int)(e_ >> 32);                                                                        \
+        }                                                                                                   \
+    } while (0)
+#define STEP_CONSUMED(item)                                                                                 \
+    do {                                                                                                    \
+        if ((threadIdx.x & 31) == 0 && (item) < 64)                                                         \
+            atomicOr((unsigned *)&p.counters[kCtrStepDiag + 256 + blockIdx.x * 16 + 10 + ((item) >> 5)],     \
+                     1u << ((item) & 31));                                                                  \
+    } while (0)
+#else
+#define STEP_MARK(stage, item) \
+    do {                       \
+    } while (0)
+#define STEP_SNAP(slot) \
+    do {                \
+    } while (0)
+#define STEP_CONSUMED(item) \
+    do {                    \
+    } while (0)
+#endif
+
+// ------------------------------------------------------------ parameters
+
+struct StepParams {
+    CUtensorMap w13;   // routed W13: (128 B, 2I rows, H/128 windows, E), boxes {128, 8, gu_wp, 1}
+    CUtensorMap w13s;  // shared W13: (128 B, 2Is rows, H/128 windows, 1)
+    CUtensorMap w2;    // routed W2: (128 B, H rows, I/128 windows, E), boxes {128, 8, dn_wp, 1}
+    CUtensorMap w2s;   // shared W2: (128 B, H rows, Is/128 windows, 1), boxes {128, 8, dn_wp_s, 1}
+    const uint16_t *x;
+    const uint16_t *router_w;
+    const uint16_t *shared_gate;
+    const uint16_t *residual;
+    const float *router_bias;
+    const float *scales;   // routed experts' block scales, E slabs
+    const float *sscales;  // the shared expert's
+    const uint16_t *norm_w;  // RMSNorm weight [H], or null: x is the layer input as given
+    double eps;
+    uint16_t *out;
+    int32_t *topk_idx;  // routing outputs [rows][K], [rows][K], [rows] (written by CTA 0)
+    float *topk_w;
+    float *gsig;
+    float *logits;      // workspace [rows][ld]
+    float *h;           // workspace [rows * (K + 1)][imax]
+    int32_t *counters;  // workspace counters (grid barrier, exit, status)
+    int rows, H, E, K, I, Is, ld, imax;
+    int ns;              // ring slots
+    int gu_wp, gu_pieces;               // gate/up: K windows per piece, pieces
+    int dn_wp, dn_pieces, dn_wp_s, dn_pieces_s, dn_epi;  // down: windows/pieces (routed, shared), experts per item
+    int nt_max;          // output 8-row tiles per CTA, at most
+    int rr_per_item;     // router rows per ring item
+    // shared-memory offsets (from the 1024-aligned base)
+    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar;
+    int x_stride;        // halves per x row in shared memory (f16 and bf16 copies)
+    int t_stride;        // halves per h term row in shared memory
+};
+
+// Small shared-memory block: routing and plan.
+struct StepSmall {
+    int32_t idx[kStepMaxRows * kMaxTopK];
+    float w[kStepMaxRows * kMaxTopK];
+    int32_t loc[kStepMaxRows * kMaxTopK];  // index of idx in the list of distinct experts
+    float gs[kStepMaxRows];
+    uint32_t mask[kMaxExperts / 32];
+    int32_t list[kStepMaxRows * kMaxTopK];  // distinct routed experts, ascending
+    int32_t tag[16];                        // ring slot -> the item last issued into it (-1: none)
+    double red[kStepWarps * kStepMaxRows];  // RMSNorm: per-warp sums of squares
+    double inv[kStepMaxRows];               // RMSNorm: 1 / sqrt(mean square + eps) per row
+    int32_t n_list;
+    int32_t abort;
+    int32_t pad[2];
+};
+
+__host__ __device__ inline int n_router_rows(int E, int G, int c)
+{
+    return (int)(((int64_t)(c + 1) * (E + 1)) / G - ((int64_t)c * (E + 1)) / G);
+}
+__host__ __device__ inline int first_router_row(int E, int G, int c) { return (int)(((int64_t)c * (E + 1)) / G); }
+__host__ __device__ inline int first_tile(int n8, int G, int c) { return (int)(((int64_t)c * n8) / G); }
+
+// ------------------------------------------------------------ item sequence
+//
+// Every thread of a CTA enumerates the same item sequence:
+//   router items  (rr_per_item router rows each; the gate vector is row E)
+//   gate/up items (local unit l = 0.., unit u = c + l*G; pieces p)
+//   down items    (groups of dn_epi experts of the down list [shared,
+//                  routed ascending]; the shared expert alone; pieces p)
+// Item q lives in ring slot q % ns.
+
+struct Item {
+    int kind;    // 0 router, 1 gate/up, 2 down
+    int a, b, p; // router: first local row, row count; gate/up: unit, local unit index; down: group, -
+};
+
+struct Seq {
+    int n_router, n_units_local, n_gu, n_groups, n_dn, total;
+};
+
+__device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt)
+{
+    const int G = gridDim.x, c = blockIdx.x;
+    Seq s;
+    const int nr = n_router_rows(p.E, G, c);
+    s.n_router = (nr + p.rr_per_item - 1) / p.rr_per_item;
+    const int units = p.Is / 8 + U * (p.I / 8);
+    s.n_units_local = units > c ? (units - 1 - c) / G + 1 : 0;
+    s.n_gu = s.n_units_local * p.gu_pieces;
+    s.n_groups = nt > 0 ? 1 + (U + p.dn_epi - 1) / p.dn_epi : 0;
+    s.n_dn = nt > 0 ? p.dn_pieces_s + (s.n_groups - 1) * p.dn_pieces : 0;
+    s.total = s.n_router + s.n_gu + s.n_dn;
+    return s;
+}
+
+__device__ __forceinline__ Item item_at(const StepParams &p, const Seq &s, int q)
+{
+    Item it;
+    if (q < s.n_router) {
+        it.kind = 0;
+        it.a = q * p.rr_per_item;
+        it.b = 0;
+        it.p = 0;
+        return it;
+    }
+    q -= s.n_router;
+    if (q < s.n_gu) {
+        it.kind = 1;
+        const int l = q / p.gu_pieces;
+        it.b = l;
+        it.a = blockIdx.x + l * gridDim.x;
+        it.p = q - l * p.gu_pieces;
+        return it;
+    }
+    q -= s.n_gu;
+    it.kind = 2;
+    it.b = 0;
+    if (q < p.dn_pieces_s) {
+        it.a = 0;
+        it.p = q;
+    } else {
+        q -= p.dn_pieces_s;
+        it.a = 1 + q / p.dn_pieces;
+        it.p = q - (it.a - 1) * p.dn_pieces;
+    }
+    return it;
+}
+
+// Gate/up unit u -> (shared?, expert, first gate row j).
+__device__ __forceinline__ void unit_of(const StepParams &p, const StepSmall &sm, int u, bool &shared, int &e, int &j)
+{
+    const int us = p.Is / 8;
+    if (u < us) {
+        shared = true;
+        e = 0;
+        j = u * 8;
+    } else {
+        shared = false;
+        const int per = p.I / 8;
+        const int ue = (u - us) / per;
+        e = sm.list[ue];
+        j = (u - us - ue * per) * 8;
+    }
+}
+
+// Experts of down group gi: the shared expert alone (gi = 0), else list
+// entries [(gi-1)*epi, min(U, gi*epi)).
+__device__ __forceinline__ int group_size(const StepParams &p, int U, int gi)
+{
+    return gi == 0 ? 1 : min(p.dn_epi, U - (gi - 1) * p.dn_epi);
+}
+
+// ------------------------------------------------------------ producer
+
+__device__ __forceinline__ uint32_t item_bytes(const StepParams &p, const Item &it, int nr_total, int nt, int U)
+{
+    if (it.kind == 0) return (uint32_t)min(p.rr_per_item, nr_total - it.a) * (uint32_t)p.H * 2u;
+    if (it.kind == 1) return (uint32_t)p.gu_wp * 2048u;
+    const int ne = group_size(p, U, it.a);
+    return (uint32_t)ne * (uint32_t)nt * (uint32_t)(it.a == 0 ? p.dn_wp_s : p.dn_wp) * 1024u;
+}
+
+__device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t slot, uint64_t *full,
+                           int r0, int nr_total, int tile0, int nt, int U, uint64_t pol)
+{
+    mbar_arrive_expect_tx(full, item_bytes(p, it, nr_total, nt, U));
+    if (it.kind == 0) {
+        // router rows r0 + it.a ..; row E (the gate vector) comes from shared_gate
+        const int n = min(p.rr_per_item, nr_total - it.a);
+        const int first = r0 + it.a;
+        const int nw = max(0, min(n, p.E - first));  // rows of router_w
+        const uint32_t rowb = (uint32_t)p.H * 2u;
+        if (nw > 0) {
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                             slot),
+                         "l"(p.router_w + (size_t)first * p.H), "r"(nw * rowb), "r"(smem_u32(full))
+                         : "memory");
+        }
+        if (nw < n) {
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                             slot + nw * rowb),
+                         "l"(p.shared_gate), "r"(rowb), "r"(smem_u32(full))
+                         : "memory");
+        }
+        return;
+    }
+    if (it.kind == 1) {
+        bool shared;
+        int e, j;
+        unit_of(p, sm, it.a, shared, e, j);
+        const CUtensorMap *m = shared ? &p.w13s : &p.w13;
+        const int Iu = shared ? p.Is : p.I;
+        const int w0 = it.p * p.gu_wp;
+        tma_load_4d(slot, m, 0, j, w0, e, full, pol);
+        tma_load_4d(slot + (uint32_t)p.gu_wp * 1024u, m, 0, Iu + j, w0, e, full, pol);
+        return;
+    }
+    const int ne = group_size(p, U, it.a);
+    const int wp = it.a == 0 ? p.dn_wp_s : p.dn_wp;
+    const CUtensorMap *m = it.a == 0 ? &p.w2s : &p.w2;
+    const uint32_t box = (uint32_t)wp * 1024u;
+    for (int x = 0; x < ne; ++x) {
+        const int e = it.a == 0 ? 0 : sm.list[(it.a - 1) * p.dn_epi + x];
+        for (int i = 0; i < nt; ++i)
+            tma_load_4d(slot + (uint32_t)(x * nt + i) * box, m, 0, (tile0 + i) * 8, it.p * wp, e, full, pol);
+    }
+}
+
+// ------------------------------------------------------------ the kernel
+
+__global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __grid_constant__ StepParams p)
+{
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *sbase = smem_raw + (base - raw);
+    StepSmall &sm = *reinterpret_cast<StepSmall *>(sbase + p.o_sm);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sbase + p.o_bar);
+    uint64_t *empty = full + p.ns;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int rows = p.rows, H = p.H, E = p.E, K = p.K;
+    const int hb = H / 128;
+    const int nr_total = n_router_rows(E, G, c);
+    const int r0 = first_router_row(E, G, c);
+    const int n8 = H / 8;
+    const int tile0 = first_tile(n8, G, c);
+    const int nt = first_tile(n8, G, c + 1) - tile0;
+    const bool producer = warp == kStepWarps;
+    volatile int32_t *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.ns; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            sm.tag[s] = -1;
+        }
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- P0
+    // The producer issues the items that depend only on weights: router
+    // rows, then the shared expert's gate/up units (the first local units).
+    int q_issued = 0;
+    const uint64_t pol = policy_evict_first();
+    if (producer && lane == 0) {
+        tma_prefetch_desc(&p.w13);
+        tma_prefetch_desc(&p.w13s);
+        tma_prefetch_desc(&p.w2);
+        tma_prefetch_desc(&p.w2s);
+        const Seq s0 = make_seq(p, 0, 0);  // U = 0: router and shared-expert items only
+        for (; q_issued < s0.total && q_issued < p.ns; ++q_issued) {
+            const Item it = item_at(p, s0, q_issued);
+            issue_item(p, sm, it, base + (uint32_t)q_issued * kSlot, &full[q_issued], r0, nr_total, tile0, nt, 0, pol);
+            ((volatile int32_t *)sm.tag)[q_issued] = q_issued;
+        }
+    }
+
+    pdl_wait();  // x and the workspace may be written by the previous kernel
+
+    // ---------------------------------------------------------------- P1
+    if (!producer) {
+        // x (bf16) -> shared memory: the rows as given, or the RMSNorm of the
+        // residual rows (in double, rounded once to bf16, as the norm's
+        // definition reads)
+        uint16_t *xb = reinterpret_cast<uint16_t *>(sbase + p.o_xb);
+        const int ct = threadIdx.x;  // 0 .. kStepWarps*32 - 1
+        if (p.norm_w) {
+            for (int t = 0; t < rows; ++t) {
+                double ss = 0.0;
+                for (int h = ct; h < H; h += kStepWarps * kWarp) {
+                    const double v = (double)bf16_bits_to_f32(p.x[(size_t)t * H + h]);
+                    ss = fma(v, v, ss);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+                if (lane == 0) sm.red[warp * kStepMaxRows + t] = ss;
+            }
+            named_barrier(1, kStepWarps * kWarp);
+            if (ct < rows) {
+                double tot = 0.0;
+                for (int w = 0; w < kStepWarps; ++w) tot += sm.red[w * kStepMaxRows + ct];
+                sm.inv[ct] = 1.0 / sqrt(tot / (double)H + p.eps);
+            }
+            named_barrier(1, kStepWarps * kWarp);
+            for (int i = ct; i < rows * H; i += kStepWarps * kWarp) {
+                const int t = i / H, h = i - t * H;
+                const double v = ((double)bf16_bits_to_f32(p.x[(size_t)t * H + h]) * sm.inv[t]) *
+                                 (double)bf16_bits_to_f32(p.norm_w[h]);
+                xb[(size_t)t * p.x_stride + h] = f64_to_bf16_rn(v);
+            }
+        } else {
+            for (int i = ct; i < rows * (H / 8); i += kStepWarps * kWarp) {
+                const int t = i / (H / 8), ch = i - t * (H / 8);
+                *reinterpret_cast<uint4 *>(xb + (size_t)t * p.x_stride + ch * 8) =
+                    __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)t * H) + ch);
+            }
+        }
+        named_barrier(1, kStepWarps * kWarp);
+        // x -> f16 * 2^shift per (row, 128 block)
+        uint16_t *xs = reinterpret_cast<uint16_t *>(sbase + p.o_uni);
+        float *xfac = reinterpret_cast<float *>(sbase + p.o_xfac);
+        for (int u = warp; u < rows * hb; u += kStepWarps) {
+            const int t = u / hb, kb = u - t * hb;
+            const uint2 raw2 = *reinterpret_cast<const uint2 *>(xb + (size_t)t * p.x_stride + kb * 128 + lane * 4);
+            const float v0 = bf16_lo(raw2.x), v1 = bf16_hi(raw2.x), v2 = bf16_lo(raw2.y), v3 = bf16_hi(raw2.y);
+            const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
+            const int sh = block_shift(amax);
+            const float f = pow2f(sh);
+            uint2 o;
+            o.x = f32x2_to_f16x2(v0 * f, v1 * f);
+            o.y = f32x2_to_f16x2(v2 * f, v3 * f);
+            *reinterpret_cast<uint2 *>(xs + (size_t)t * p.x_stride + kb * 128 + lane * 4) = o;
+            if (lane == 0) xfac[t * hb + kb] = pow2f(-sh);
+        }
+        // router rows (router items 0 .. n_router-1 in slots 0 ..)
+        const Seq s0 = make_seq(p, 0, 0);
+        for (int ri = 0; ri < s0.n_router; ++ri) {
+            if (!warp_wait(&full[ri], 0)) {
+                if (lane == 0) {
+                    gave_up(p.counters, 1, ri);
+                    *abort = 1;
+                }
+                break;
+            }
+            const int first = ri * p.rr_per_item;
+            const int n = min(p.rr_per_item, nr_total - first);
+            for (int rr = warp; rr < n; rr += kStepWarps) {
+                const int e = r0 + first + rr;
+                const uint4 *wrow = reinterpret_cast<const uint4 *>(sbase + (size_t)ri * kSlot + (size_t)rr * H * 2);
+                float acc[kStepMaxRows];
+#pragma unroll
+                for (int t = 0; t < kStepMaxRows; ++t) acc[t] = 0.f;
+                for (int ch = lane; ch < H / 8; ch += kWarp) {
+                    const uint4 w8 = wrow[ch];
+#pragma unroll
+                    for (int t = 0; t < kStepMaxRows; ++t) {
+                        if (t < rows) {
+                            const uint4 xv = *reinterpret_cast<const uint4 *>(xb + (size_t)t * p.x_stride + ch * 8);
+                            float a = bf16_lo(w8.x) * bf16_lo(xv.x);
+                            float b = bf16_hi(w8.x) * bf16_hi(xv.x);
+                            a = fmaf(bf16_lo(w8.y), bf16_lo(xv.y), a);
+                            b = fmaf(bf16_hi(w8.y), bf16_hi(xv.y), b);
+                            a = fmaf(bf16_lo(w8.z), bf16_lo(xv.z), a);
+                            b = fmaf(bf16_hi(w8.z), bf16_hi(xv.z), b);
+                            a = fmaf(bf16_lo(w8.w), bf16_lo(xv.w), a);
+                            b = fmaf(bf16_hi(w8.w), bf16_hi(xv.w), b);
+                            acc[t] += a + b;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < kStepMaxRows; ++t) {
+                    if (t < rows) {
+                        const float v = warp_sum(acc[t]);
+                        if (lane == 0) p.logits[(size_t)t * p.ld + e] = v + ((e < E && p.router_bias) ? p.router_bias[e] : 0.f);
+                    }
+                }
+            }
+        }
+        __threadfence();
+        named_barrier(1, kStepWarps * kWarp);
+        if (threadIdx.x == 0) {
+            // the router slots are free again
+            for (int ri = 0; ri < s0.n_router; ++ri) mbar_arrive(&empty[ri]);
+            bool ok = !*abort;
+            if (ok) {
+                atomic_add_release_gpu(p.counters + kCtrStepBar, 1);
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_gpu(p.counters + kCtrStepBar) < G) {
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        gave_up(p.counters, 6, 0);
+                        *abort = 1;
+                        break;
+                    }
+                }
+            }
+        }
+        named_barrier(1, kStepWarps * kWarp);
+        // ------------------------------------------------------------ P2
+        // top-k of every row, in every CTA
+        if (!*abort && warp < rows) {
+            const float *lrow = p.logits + (size_t)warp * p.ld;
+            int32_t *oi = sm.idx + warp * K;
+            float *ow = sm.w + warp * K;
+            float *og = sm.gs + warp;
+            if (E <= 32) topk_select<1>(lrow, E, K, oi, ow, og);
+            else if (E <= 64) topk_select<2>(lrow, E, K, oi, ow, og);
+            else if (E <= 128) topk_select<4>(lrow, E, K, oi, ow, og);
+            else if (E <= 256) topk_select<8>(lrow, E, K, oi, ow, og);
+            else if (E <= 512) topk_select<16>(lrow, E, K, oi, ow, og);
+            else topk_select<32>(lrow, E, K, oi, ow, og);
+        }
+        named_barrier(1, kStepWarps * kWarp);
+        if (!*abort && warp == 0) {
+            // distinct routed experts, ascending, and each pair's place in the list
+            for (int i = lane; i < kMaxExperts / 32; i += kWarp) sm.mask[i] = 0u;
+            __syncwarp();
+            for (int i = lane; i < rows * K; i += kWarp) atomicOr(&sm.mask[sm.idx[i] >> 5], 1u << (sm.idx[i] & 31));
+            __syncwarp();
+            const int nwords = (E + 31) / 32;
+            int before = 0;
+            for (int w0 = 0; w0 < nwords; w0 += kWarp) {
+                const int wi = w0 + lane;
+                const uint32_t m = wi < nwords ? sm.mask[wi] : 0u;
+                const int cnt = __popc(m);
+                int incl = cnt;
+#pragma unroll
+                for (int o = 1; o < kWarp; o <<= 1) {
+                    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                int pos = before + incl - cnt;
+                uint32_t mm = m;
+                while (mm) {
+                    const int b = __ffs(mm) - 1;
+                    sm.list[pos++] = wi * 32 + b;
+                    mm &= mm - 1;
+                }
+                before += __shfl_sync(0xFFFFFFFFu, incl, kWarp - 1);
+            }
+            if (lane == 0) sm.n_list = before;
+            __syncwarp();
+            for (int i = lane; i < rows * K; i += kWarp) {
+                const int e = sm.idx[i];
+                int pos = 0;
+                for (int wi = 0; wi < (e >> 5); ++wi) pos += __popc(sm.mask[wi]);
+                pos += __popc(sm.mask[e >> 5] & ((1u << (e & 31)) - 1u));
+                sm.loc[i] = pos;
+            }
+            if (c == 0) {
+                for (int i = lane; i < rows * K; i += kWarp) {
+                    p.topk_idx[i] = sm.idx[i];
+                    p.topk_w[i] = sm.w[i];
+                }
+                if (lane < rows) p.gsig[lane] = sm.gs[lane];
+            }
+        }
+    }
+    __syncthreads();  // the plan is ready (all 288 threads)
+    const int U = *abort ? 0 : sm.n_list;
+    const Seq seq = make_seq(p, U, nt);
+
+    if (producer) {
+        // ---------------------------------------------------------- producer
+        // Phase A, before grid barrier 2: issue while the slot's previous
+        // item is a router or gate/up item (down items are consumed only
+        // after the barrier, so their slots cannot be waited for here).
+        if (lane == 0) {
+            int q = q_issued;
+            for (; q < seq.total && !*abort; ++q) {
+                const int s = q % p.ns;
+                STEP_MARK(10, q);
+                if (q >= p.ns) {
+                    if (item_at(p, seq, q - p.ns).kind == 2) break;
+                    if (!mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
+                        STEP_SNAP(s);
+                        gave_up(p.counters, 4, q);
+                        *abort = 1;
+                        break;
+                    }
+                    fence_proxy_async_smem();
+                }
+                issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt,
+                           U, pol);
+                ((volatile int32_t *)sm.tag)[s] = q;
+            }
+            q_issued = q;
+        }
+        __syncwarp();
+        named_barrier(2, kStepThreads);  // gate/up of this CTA done
+        named_barrier(2, kStepThreads);  // grid barrier 2 passed
+        if (lane == 0) {
+            // Phase B: the rest, as the down items are consumed.
+            int q = q_issued;
+            for (; q < seq.total && !*abort; ++q) {
+                const int s = q % p.ns;
+                if (q >= p.ns) {
+                    if (!mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
+                        gave_up(p.counters, 5, q);
+                        *abort = 1;
+                        break;
+                    }
+                    fence_proxy_async_smem();
+                }
+                issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt,
+                           U, pol);
+                ((volatile int32_t *)sm.tag)[s] = q;
+            }
+            q_issued = q;
+            // every issued copy lands before the CTA may leave
+            for (int qq = max(0, q_issued - p.ns); qq < q_issued; ++qq)
+                mbar_wait(&full[qq % p.ns], (qq / p.ns) & 1, kWaitLimitNs);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int g = lane >> 2, qd = lane & 3;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(sbase + p.o_uni);
+    const float *xfac = reinterpret_cast<const float *>(sbase + p.o_xfac);
+
+    // gate/up units: local unit l -> warp l % kStepWarps, its pieces in order
+    {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int q = seq.n_router; q < seq.n_router + seq.n_gu && !*abort; ++q) {
+            const Item it = item_at(p, seq, q);
+            if (it.b % kStepWarps != warp) continue;
+            const int s = q % p.ns;
+            STEP_MARK(2, q);
+            if (!wait_item(sm.tag, full, s, q, p.ns)) {
+                if (lane == 0) {
+                    STEP_SNAP(s);
+                    gave_up(p.counters, 2, q);
+                    *abort = 1;
+                }
+                break;
+            }
+            STEP_MARK(3, q);
+            bool shared;
+            int e, j;
+            unit_of(p, sm, it.a, shared, e, j);
+            const int Iu = shared ? p.Is : p.I;
+            const float *sc = shared ? p.sscales : p.scales + (size_t)e * ((size_t)(2 * Iu / 128) * hb + (size_t)hb * (Iu / 128));
+            const float *sg_row = sc + (size_t)(j / 128) * hb;
+            const float *su_row = sc + (size_t)((Iu + j) / 128) * hb;
+            if (it.p == 0) acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            const uint32_t sl = base + (uint32_t)s * kSlot;
+            const uint32_t gate_base = sl + (uint32_t)g * 128u;
+            const uint32_t up_base = sl + (uint32_t)p.gu_wp * 1024u + (uint32_t)g * 128u;
+            const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
+            const bool xrow = g < rows;
+            const uint32_t xaddr = smem_u32(xs) + (uint32_t)(g * p.x_stride * 2);
+            for (int w = 0; w < p.gu_wp; ++w) {
+                const int W = it.p * p.gu_wp + w;
+                if (W >= hb) break;
+                const uint4 ga0 = lds128(gate_base + w * 1024u + c0), ga1 = lds128(gate_base + w * 1024u + c1);
+                const uint4 ua0 = lds128(up_base + w * 1024u + c0), ua1 = lds128(up_base + w * 1024u + c1);
+                uint4 xb[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    xb[i] = xrow ? lds128(xaddr + (uint32_t)((W * 128 + 32 * qd + 8 * i) * 2)) : make_uint4(0, 0, 0, 0);
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int st = 0; st < 8; ++st) {
+                    const uint32_t gw = word_of(st < 4 ? ga0 : ga1, st & 3);
+                    const uint32_t uw = word_of(st < 4 ? ua0 : ua1, st & 3);
+                    const uint32_t b0 = word_of(xb[st >> 1], (st & 1) * 2);
+                    const uint32_t b1 = word_of(xb[st >> 1], (st & 1) * 2 + 1);
+                    mma_f16_16816(d, e4m3x2_to_f16x2(gw), e4m3x2_to_f16x2(uw), e4m3x2_to_f16x2(gw >> 16),
+                                  e4m3x2_to_f16x2(uw >> 16), b0, b1);
+                }
+                const float sgw = __ldg(sg_row + W), suw = __ldg(su_row + W);
+                const int t0 = 2 * qd, t1 = 2 * qd + 1;
+                const float f0 = t0 < rows ? xfac[t0 * hb + W] : 0.f;
+                const float f1 = t1 < rows ? xfac[t1 * hb + W] : 0.f;
+                acc[0] = fmaf(sgw * f0, d[0], acc[0]);
+                acc[1] = fmaf(sgw * f1, d[1], acc[1]);
+                acc[2] = fmaf(suw * f0, d[2], acc[2]);
+                acc[3] = fmaf(suw * f1, d[3], acc[3]);
+            }
+            STEP_MARK(4, q);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            STEP_MARK(5, q);
+            STEP_CONSUMED(q);
+            if (it.p == p.gu_pieces - 1) {
+                // h = silu(gate) * up for rows 2q, 2q+1 routed to this expert
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const int t = 2 * qd + k2;
+                    if (t >= rows) continue;
+                    int slot = -1;
+                    if (shared) {
+                        slot = rows * K + t;
+                    } else {
+                        for (int r = 0; r < K; ++r)
+                            if (sm.idx[t * K + r] == e) slot = t * K + r;
+                    }
+                    if (slot < 0) continue;
+                    const float gt = acc[k2], up = acc[2 + k2];
+                    p.h[(size_t)slot * p.imax + j + g] = siluf_(gt) * up;
+                }
+            }
+        }
+    }
+    STEP_MARK(6, 0);
+    __threadfence();
+    named_barrier(2, kStepThreads);  // gate/up of this CTA done (producer included)
+    if (threadIdx.x == 0) {
+        bool ok = !*abort;
+        if (ok) {
+            atomic_add_release_gpu(p.counters + kCtrStepBar, 1);
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(p.counters + kCtrStepBar) < 2 * G) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    gave_up(p.counters, 7, 0);
+                    *abort = 1;
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if (ok) {
+            // every CTA has passed both barriers once the exit count is full:
+            // the last one resets the counters for the next call
+            if (atomic_add_acq_rel_gpu(p.counters + kCtrStepExit, 1) == G - 1) {
+                p.counters[kCtrStepBar] = 0;
+                p.counters[kCtrStepExit] = 0;
+            }
+        }
+    }
+    named_barrier(2, kStepThreads);
+    pdl_trigger();
+    if (*abort || nt == 0) return;
+
+    // ---------------------------------------------------------------- P3
+    // h -> three f16 terms per value, scaled by a power of two per (slot, block)
+    const int nslots = rows * (K + 1);
+    const int ib = p.imax / 128;
+    uint16_t *terms = xs;  // the x region is free now
+    float *hfac = reinterpret_cast<float *>(sbase + p.o_hfac);
+    for (int u = warp; u < nslots * ib; u += kStepWarps) {
+        const int sl = u / ib, kb = u - sl * ib;
+        const int Iu = sl >= rows * K ? p.Is : p.I;
+        if (kb * 128 >= Iu) continue;
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane);
+        const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        const int sh = block_shift(amax);
+        const float f = pow2f(sh);
+        const float a[4] = {v.x * f, v.y * f, v.z * f, v.w * f};
+        uint32_t t0[2], t1[2], t2[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float x0 = a[2 * i], x1 = a[2 * i + 1];
+            const __half2 h0 = __floats2half2_rn(x0, x1);
+            const float2 r0 = __half22float2(h0);
+            const float y0 = x0 - r0.x, y1 = x1 - r0.y;
+            const __half2 h1 = __floats2half2_rn(y0, y1);
+            const float2 r1 = __half22float2(h1);
+            const __half2 h2 = __floats2half2_rn(y0 - r1.x, y1 - r1.y);
+            t0[i] = *reinterpret_cast<const uint32_t *>(&h0);
+            t1[i] = *reinterpret_cast<const uint32_t *>(&h1);
+            t2[i] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        uint16_t *row = terms + (size_t)sl * 3 * p.t_stride + kb * 128 + lane * 4;
+        *reinterpret_cast<uint2 *>(row) = make_uint2(t0[0], t0[1]);
+        *reinterpret_cast<uint2 *>(row + p.t_stride) = make_uint2(t1[0], t1[1]);
+        *reinterpret_cast<uint2 *>(row + 2 * p.t_stride) = make_uint2(t2[0], t2[1]);
+        if (lane == 0) hfac[sl * ib + kb] = pow2f(-sh);
+    }
+    named_barrier(1, kStepWarps * kWarp);
+
+    // down items: group gi -> warp gi % kStepWarps; per expert of the group,
+    // per output tile, accumulate over windows and pieces
+    float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);   // [U + 1][rows][nt_max * 8]
+    float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 128;  // [16][8]
+    const int yrow = p.nt_max * 8;
+    {
+        float acc[kStepMaxExpertsPerItem][kMaxNt][4];
+        for (int q = seq.n_router + seq.n_gu; q < seq.total && !*abort; ++q) {
+            const Item it = item_at(p, seq, q);
+            if (it.a % kStepWarps != warp) continue;
+            const int s = q % p.ns;
+            if (!wait_item(sm.tag, full, s, q, p.ns)) {
+                if (lane == 0) {
+                    gave_up(p.counters, 3, q);
+                    *abort = 1;
+                }
+                break;
+            }
+            const bool shared = it.a == 0;
+            const int ne = group_size(p, U, it.a);
+            const int wp = shared ? p.dn_wp_s : p.dn_wp;
+            const int pieces = shared ? p.dn_pieces_s : p.dn_pieces;
+            const int Iu = shared ? p.Is : p.I;
+            const int ibu = Iu / 128;
+            const uint32_t sl = base + (uint32_t)s * kSlot;
+            if (it.p == 0) {
+#pragma unroll
+                for (int x = 0; x < kStepMaxExpertsPerItem; ++x)
+#pragma unroll
+                    for (int i = 0; i < kMaxNt; ++i) acc[x][i][0] = acc[x][i][1] = acc[x][i][2] = acc[x][i][3] = 0.f;
+            }
+#pragma unroll
+            for (int x = 0; x < kStepMaxExpertsPerItem; ++x) {
+                if (x >= ne) break;
+                const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
+                const int e = shared ? 0 : sm.list[li];
+                // A rows m = 3t + j: row t's slot for this expert, term j
+                int slot_lo = -1, slot_hi = -1;
+                {
+                    const int m0 = g, m1 = g + 8;
+                    const int tlo = m0 / 3, thi = m1 / 3;
+                    if (tlo < rows) {
+                        if (shared) slot_lo = rows * K + tlo;
+                        else for (int r = 0; r < K; ++r) if (sm.idx[tlo * K + r] == e) slot_lo = tlo * K + r;
+                    }
+                    if (thi < rows) {
+                        if (shared) slot_hi = rows * K + thi;
+                        else for (int r = 0; r < K; ++r) if (sm.idx[thi * K + r] == e) slot_hi = thi * K + r;
+                    }
+                }
+                const int jlo = g % 3, jhi = (g + 8) % 3;
+                const uint32_t alo = slot_lo >= 0 ? smem_u32(terms + ((size_t)slot_lo * 3 + jlo) * p.t_stride) : 0u;
+                const uint32_t ahi = slot_hi >= 0 ? smem_u32(terms + ((size_t)slot_hi * 3 + jhi) * p.t_stride) : 0u;
+                const float *s2 = (shared ? p.sscales : p.scales + (size_t)e * ((size_t)(2 * Iu / 128) * hb + (size_t)hb * ibu)) +
+                                  (size_t)(2 * Iu / 128) * hb;
+                const uint32_t ebase = sl + (uint32_t)(x * nt) * (uint32_t)wp * 1024u + (uint32_t)g * 128u;
+                const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
+                for (int w = 0; w < wp; ++w) {
+                    const int W = it.p * wp + w;
+                    if (W >= ibu) break;
+                    uint4 al[4], ah[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t off = (uint32_t)((W * 128 + 32 * qd + 8 * i) * 2);
+                        al[i] = slot_lo >= 0 ? lds128(alo + off) : make_uint4(0, 0, 0, 0);
+                        ah[i] = slot_hi >= 0 ? lds128(ahi + off) : make_uint4(0, 0, 0, 0);
+                    }
+                    const float flo = slot_lo >= 0 ? hfac[slot_lo * ib + W] : 0.f;
+                    const float fhi = slot_hi >= 0 ? hfac[slot_hi * ib + W] : 0.f;
+#pragma unroll
+                    for (int i = 0; i < kMaxNt; ++i) {
+                        if (i >= nt) break;
+                        const uint32_t tb = ebase + (uint32_t)i * (uint32_t)wp * 1024u + (uint32_t)w * 1024u;
+                        const uint4 wb0 = lds128(tb + c0), wb1 = lds128(tb + c1);
+                        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int st = 0; st < 8; ++st) {
+                            const uint32_t ww = word_of(st < 4 ? wb0 : wb1, st & 3);
+                            const uint32_t a0 = word_of(al[st >> 1], (st & 1) * 2);
+                            const uint32_t a2 = word_of(al[st >> 1], (st & 1) * 2 + 1);
+                            const uint32_t a1 = word_of(ah[st >> 1], (st & 1) * 2);
+                            const uint32_t a3 = word_of(ah[st >> 1], (st & 1) * 2 + 1);
+                            mma_f16_16816(d, a0, a1, a2, a3, e4m3x2_to_f16x2(ww), e4m3x2_to_f16x2(ww >> 16));
+                        }
+                        const int nrow = (tile0 + i) * 8;
+                        const float sw = __ldg(s2 + (size_t)(nrow / 128) * ibu + W);
+                        acc[x][i][0] = fmaf(sw * flo, d[0], acc[x][i][0]);
+                        acc[x][i][1] = fmaf(sw * flo, d[1], acc[x][i][1]);
+                        acc[x][i][2] = fmaf(sw * fhi, d[2], acc[x][i][2]);
+                        acc[x][i][3] = fmaf(sw * fhi, d[3], acc[x][i][3]);
+                    }
+                }
+                if (it.p == pieces - 1) {
+                    // y[t][n] = sum of row t's three term rows, into the down buffer
+                    const int de = shared ? 0 : 1 + li;
+#pragma unroll
+                    for (int i = 0; i < kMaxNt; ++i) {
+                        if (i >= nt) break;
+                        scr[g * 8 + 2 * qd] = acc[x][i][0];
+                        scr[g * 8 + 2 * qd + 1] = acc[x][i][1];
+                        scr[(g + 8) * 8 + 2 * qd] = acc[x][i][2];
+                        scr[(g + 8) * 8 + 2 * qd + 1] = acc[x][i][3];
+                        __syncwarp();
+                        const int t = lane >> 3, n = lane & 7;
+                        if (t < rows) {
+                            const float y = (scr[(3 * t) * 8 + n] + scr[(3 * t + 1) * 8 + n]) + scr[(3 * t + 2) * 8 + n];
+                            ybuf[((size_t)de * rows + t) * yrow + i * 8 + n] = y;
+                        }
+                        __syncwarp();
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+    }
+    named_barrier(1, kStepWarps * kWarp);
+    if (*abort) return;
+
+    // blend: rank order, then the shared expert, then the residual; one rounding
+    for (int u = threadIdx.x; u < rows * nt * 8; u += kStepWarps * kWarp) {
+        const int t = u / (nt * 8), nn = u - t * (nt * 8);
+        float acc = 0.f;
+        for (int r = 0; r < K; ++r) acc = fmaf(sm.w[t * K + r], ybuf[((size_t)(1 + sm.loc[t * K + r]) * rows + t) * yrow + nn], acc);
+        acc = fmaf(sm.gs[t], ybuf[(size_t)t * yrow + nn], acc);
+        const size_t o = (size_t)t * H + (size_t)tile0 * 8 + nn;
+        if (p.residual) acc += bf16_bits_to_f32(p.residual[o]);
+        p.out[o] = f32_to_bf16_bits(acc);
+    }
+}
+
+// ------------------------------------------------------------ host side
+
+std::mutex g_mu;
+
+bool configured_for(int dev)
+{
+    static bool done[64] = {};
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev < 0 || dev >= 64) return false;
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(decode_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap) !=
+            cudaSuccess)
+            return false;
+        done[dev] = true;
+    }
+    return true;
+}
+
+// A byte tensor [outer][rows][windows of 128 bytes] as a 4-D TMA map over
+// (128 bytes, rows, windows, outer) with 128-byte-swizzled boxes
+// {128, 8, box_windows, 1}: a box lands as [window][8 rows][128 bytes].
+bool make_map_rows_windows(CUtensorMap *m, const void *base, uint64_t rows, uint64_t kbytes, uint64_t outer,
+                           uint64_t outer_stride, uint32_t box_windows)
+{
+    using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeFn>(nullptr);
+        return reinterpret_cast<EncodeFn>(f);
+    }();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {128, rows, kbytes / 128, outer};
+    const cuuint64_t strides[3] = {kbytes, 128, outer_stride ? outer_stride : rows * kbytes};
+    const cuuint32_t box[4] = {128, 8, box_windows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int pieces_for(int windows, int max_wp, int *wp)
+{
+    const int n = (windows + max_wp - 1) / max_wp;
+    *wp = (windows + n - 1) / n;
+    return n;
+}
+
+}  // namespace
+
+StepShape step_shape(const moe_dims &d, int rows, int sms)
+{
+    StepShape s{};
+    const int H = d.hidden, I = d.inter, Is = d.shared_inter, K = d.top_k;
+    const int imax = std::max(I, Is);
+    const int G = std::max(1, sms);
+    s.grid = G;
+    s.gu_pieces = pieces_for(H / 128, 8, &s.gu_wp);  // 8 + 8 rows x <= 1024 bytes
+    const int n8 = H / 8;
+    s.nt_max = (n8 + G - 1) / G;
+    const int max_wp_dn = std::max(1, kSlot / (s.nt_max * 1024));
+    s.dn_pieces = pieces_for(I / 128, max_wp_dn, &s.dn_wp);
+    s.dn_pieces_s = pieces_for(Is / 128, max_wp_dn, &s.dn_wp_s);
+    s.dn_epi = s.dn_pieces == 1 ? std::max(1, std::min(kStepMaxExpertsPerItem, kSlot / (s.nt_max * s.dn_wp * 1024)))
+                                : 1;
+    s.rr_per_item = std::max(1, kSlot / (2 * H));
+    // shared memory, after the ring
+    const int nslots = rows * (K + 1);
+    s.x_stride = H + 8;
+    s.t_stride = imax + 8;
+    const size_t xbytes = (size_t)rows * s.x_stride * 2;
+    const size_t tbytes = (size_t)nslots * 3 * s.t_stride * 2;
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 16); return (uint32_t)at; };
+    const uint32_t uni = take(std::max(2 * xbytes, tbytes));  // [f16 x | bf16 x] in P1-P2, h terms in P3
+    const uint32_t xfac = take((size_t)rows * (H / 128) * 4);
+    const uint32_t hfac = take((size_t)nslots * (imax / 128) * 4);
+    const int umax = std::min(d.n_experts, rows * K);
+    const uint32_t y = take((size_t)(umax + 1) * rows * s.nt_max * 8 * 4);
+    const uint32_t scr = take((size_t)kStepWarps * 128 * 4);
+    const uint32_t smo = take(sizeof(StepSmall));
+    const size_t tail = o;
+    // ring slots: whatever is left, up to 16
+    const size_t avail = (size_t)kSmemCap - 1024 - tail - 16 * 2 * 8;
+    s.ns = (int)std::min<size_t>(16, avail / kSlot);
+    const uint32_t ring = (uint32_t)s.ns * kSlot;
+    s.o_uni = ring + uni;
+    s.o_xb = ring + uni + (uint32_t)xbytes;
+    s.o_xfac = ring + xfac;
+    s.o_hfac = ring + hfac;
+    s.o_y = ring + y;
+    s.o_scr = ring + scr;
+    s.o_sm = ring + smo;
+    s.o_bar = (uint32_t)align_up(ring + tail, 8);
+    s.smem = s.o_bar + 2 * 8 * s.ns + 1024;
+    // the router items all sit in the ring before the first slot is reused
+    const int rr_max = (d.n_experts + 1 + G - 1) / G;
+    const int router_items = (rr_max + s.rr_per_item - 1) / s.rr_per_item;
+    s.ok = s.ns >= 2 && s.ns > router_items && s.nt_max <= kMaxNt && s.smem <= kSmemCap && 2 * H <= kSlot;
+    return s;
+}
+
+int step_rows_per_launch(const moe_dims &d, int sms)
+{
+    for (int r = kStepMaxRows; r >= 1; --r) {
+        const StepShape s = step_shape(d, r, sms);
+        if (s.ok && s.ns >= 4) return r;
+    }
+    return step_shape(d, 1, sms).ok ? 1 : 0;
+}
+
+cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
+{
+    const moe_dims &d = *a.d;
+    const DeviceInfo &di = device_info();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!configured_for(dev)) return cudaErrorInvalidConfiguration;
+    const StepShape sh = step_shape(d, a.rows, di.sm_count);
+    if (!sh.ok || a.rows < 1 || a.rows > kStepMaxRows) return cudaErrorInvalidConfiguration;
+    const int H = d.hidden, I = d.inter, Is = d.shared_inter, E = d.n_experts;
+    StepParams p;
+    if (!make_map_rows_windows(&p.w13, a.expert_w8, 2 * (uint64_t)I, (uint64_t)H, (uint64_t)E, 3 * (uint64_t)I * H,
+                               (uint32_t)sh.gu_wp) ||
+        !make_map_rows_windows(&p.w13s, a.shared_w8, 2 * (uint64_t)Is, (uint64_t)H, 1, 0, (uint32_t)sh.gu_wp) ||
+        !make_map_rows_windows(&p.w2, a.expert_w8 + (size_t)2 * I * H, (uint64_t)H, (uint64_t)I, (uint64_t)E,
+                               3 * (uint64_t)I * H, (uint32_t)sh.dn_wp) ||
+        !make_map_rows_windows(&p.w2s, a.shared_w8 + (size_t)2 * Is * H, (uint64_t)H, (uint64_t)Is, 1, 0,
+                               (uint32_t)sh.dn_wp_s))
+        return cudaErrorInvalidValue;
+    p.x = a.x;
+    p.router_w = a.router_w;
+    p.shared_gate = a.shared_gate;
+    p.residual = a.residual;
+    p.router_bias = a.router_bias;
+    p.scales = a.expert_scales;
+    p.sscales = a.shared_scales;
+    p.norm_w = a.norm_w;
+    p.eps = a.eps;
+    p.out = a.out;
+    p.topk_idx = a.topk_idx;
+    p.topk_w = a.topk_w;
+    p.gsig = a.gsig;
+    p.logits = a.logits;
+    p.h = a.h;
+    p.counters = a.counters;
+    p.rows = a.rows;
+    p.H = H;
+    p.E = E;
+    p.K = d.top_k;
+    p.I = I;
+    p.Is = Is;
+    p.ld = a.logits_ld;
+    p.imax = std::max(I, Is);
+    p.ns = sh.ns;
+    p.gu_wp = sh.gu_wp;
+    p.gu_pieces = sh.gu_pieces;
+    p.dn_wp = sh.dn_wp;
+    p.dn_pieces = sh.dn_pieces;
+    p.dn_wp_s = sh.dn_wp_s;
+    p.dn_pieces_s = sh.dn_pieces_s;
+    p.dn_epi = sh.dn_epi;
+    p.nt_max = sh.nt_max;
+    p.rr_per_item = sh.rr_per_item;
+    p.o_uni = sh.o_uni;
+    p.o_xb = sh.o_xb;
+    p.o_xfac = sh.o_xfac;
+    p.o_hfac = sh.o_hfac;
+    p.o_y = sh.o_y;
+    p.o_scr = sh.o_scr;
+    p.o_sm = sh.o_sm;
+    p.o_bar = sh.o_bar;
+    p.x_stride = sh.x_stride;
+    p.t_stride = sh.t_stride;
+    return launch_kernel(decode_step_kernel, dim3(sh.grid), dim3(kStepThreads), sh.smem, st, p);
+}
+
+}  // namespace moe

@@ -16,48 +16,42 @@ constexpr int kCtrRouter = 0;           // last-arriver counter over the router'
 constexpr int kCtrStatus = 1;           // device status word: 0, or a MOE_* error a kernel recorded
 constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per token-group counters
 constexpr int kMaxRouterGroups = 1024;
-constexpr int kCtrBlend = 2048;         // first of the down/blend per-row-block counters
-constexpr int kMaxBlendBlocks = kCounters - kCtrBlend;
-constexpr int kDescPairs = 8;           // pair ids a stage descriptor carries
+constexpr int kCtrStepBar = 8;          // decode step kernel: grid-barrier arrivals
+constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs past the last barrier
+constexpr int kCtrStepDiag = 2048;      // decode step kernel: per CTA, where a wait ran out (0: none)
+constexpr int kMaxBlendBlocks = 2048;   // H / 8 limit
+constexpr int kSmallRouterRows = 64;    // the grouped-GEMM path routes up to this many rows with the router kernel
+
+// The decode step kernel (decode_step.cu).
+constexpr int kStepMaxRows = 4;           // rows per launch; more rows run as several launches
+constexpr int kStepWarps = 8;             // consumer warps; plus one producer warp
+constexpr int kStepThreads = (kStepWarps + 1) * 32;
+constexpr int kStepMaxExpertsPerItem = 2; // down experts per ring item
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Decode-path workspace, carved from the caller's buffer.
+// Decode-path workspace, carved from the caller's buffer: the router's
+// logits and routing for all rows; h for one decode-step launch.
 struct DecodeLayout {
-    size_t counters, logits, xq, xsc, topk_idx, topk_w, gsig, h_routed, h_shared, yslot, total;
+    size_t counters, logits, topk_idx, topk_w, gsig, h, total;
+    int ld;
 };
-
-// Tile shapes of the decode kernels for given dims and rows.
-struct DecodeShape {
-    int router_rows, router_groups, router_group_tokens, logits_ld;
-    size_t router_smem;
-    int gu_pairs, tok, gu_stages;
-    size_t gu_smem;
-    int dn_rows, dn_stages;
-    size_t dn_smem;
-    // down by output block (few rows): experts per stage; 0 = the item-based down kernel
-    int ds_ue;
-    // gate_up prefetches the active experts' down weights into L2
-    bool l2_w2;
-};
-DecodeShape decode_shape(const moe_dims &d, int64_t rows);
 
 inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
 {
     DecodeLayout L{};
-    const int64_t E = d.n_experts, K = d.top_k, H = d.hidden, I = d.inter, Is = d.shared_inter;
+    const int64_t E = d.n_experts, K = d.top_k, I = d.inter, Is = d.shared_inter;
+    const int64_t imax = I > Is ? I : Is;
+    const int64_t hrows = rows < kStepMaxRows ? rows : kStepMaxRows;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+    L.ld = (int)((E + 1 + 3) / 4 * 4);
     L.counters = take(sizeof(int32_t) * kCounters);
-    L.logits = take(sizeof(float) * rows * ((E + 1 + 3) / 4 * 4));
-    L.xq = take((size_t)rows * 2 * H);
-    L.xsc = take(sizeof(float) * rows * (H / 128));
+    L.logits = take(sizeof(float) * rows * L.ld);
     L.topk_idx = take(sizeof(int32_t) * rows * K);
     L.topk_w = take(sizeof(float) * rows * K);
     L.gsig = take(sizeof(float) * rows);
-    L.h_routed = take(sizeof(float) * rows * K * I);
-    L.h_shared = take(sizeof(float) * rows * Is);
-    L.yslot = take(sizeof(float) * rows * (K + 1) * H);
+    L.h = take(sizeof(float) * hrows * (K + 1) * imax);
     L.total = o;
     return L;
 }
@@ -74,14 +68,14 @@ int check_forward_args(const moe_dims *d, const uint16_t *x, int32_t rows, const
                        const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
                        const uint16_t *shared_gate, const uint16_t *out, const uint16_t *residual,
                        const float *router_bias, int32_t path, const int32_t *topk_idx_out,
-                       const float *topk_w_out, const float *shared_gate_sig_out);
+                       const float *topk_w_out, const float *shared_gate_sig_out, bool out_may_alias_x);
 // The layer step on a checked workspace of at least workspace_bytes(d, rows)
 // bytes, after enter() returned MOE_OK.
 int run_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
                 const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
                 const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual, const float *router_bias,
                 void *ws, void *stream, int32_t path, int32_t *topk_idx_out, float *topk_w_out,
-                float *shared_gate_sig_out);
+                float *shared_gate_sig_out, const uint16_t *norm_w, double eps);
 
 // Device properties cached per device.
 struct DeviceInfo {
@@ -103,41 +97,60 @@ struct RouterLaunch {
     float *topk_w;
     float *gsig;
     float *logits;   // workspace
-    uint8_t *xq;     // workspace: x as hi/lo e4m3 (nullptr: not needed)
-    float *xsc;
     int32_t *counters;
 };
 cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s);
 
-struct ExpertsLaunch {
+// Shape of one decode-step launch (rows <= kStepMaxRows).
+struct StepShape {
+    bool ok;
+    int grid, ns, gu_wp, gu_pieces, dn_wp, dn_pieces, dn_wp_s, dn_pieces_s, dn_epi, nt_max, rr_per_item;
+    int x_stride, t_stride;
+    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar;
+    size_t smem;
+};
+StepShape step_shape(const moe_dims &d, int rows, int sms);
+// Rows one decode-step launch takes for these dims (0: the dims do not fit).
+int step_rows_per_launch(const moe_dims &d, int sms);
+
+struct StepLaunch {
     const moe_dims *d;
-    const uint16_t *x;
-    const uint8_t *xq;
-    const float *xsc;
+    const uint16_t *x;       // the layer input, or the residual rows when norm_w is set
+    const uint16_t *norm_w;  // null, or the RMSNorm weight: x = bf16(rmsnorm(x) * norm_w)
+    double eps;
     int32_t rows;
+    const uint16_t *router_w;
+    const float *router_bias;
+    const uint16_t *shared_gate;
     const uint8_t *expert_w8;
     const float *expert_scales;
     const uint8_t *shared_w8;
     const float *shared_scales;
     const uint16_t *residual;
     uint16_t *out;
-    const int32_t *topk_idx;
-    const float *topk_w;
-    const float *gsig;
-    float *h_routed;
-    float *h_shared;
-    float *yslot;
+    int32_t *topk_idx;
+    float *topk_w;
+    float *gsig;
+    float *logits;
+    int logits_ld;
+    float *h;
     int32_t *counters;
 };
-cudaError_t launch_decode_experts(const ExpertsLaunch &a, cudaStream_t s);
+cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t s);
+
+// x = bf16(rmsnorm(resid) * norm_w) for `rows` rows (one CTA per row).
+cudaError_t launch_rmsnorm(const uint16_t *resid, const uint16_t *norm_w, double eps, int H, int rows, uint16_t *x,
+                           cudaStream_t s);
 
 // One CTA waits on an mbarrier that nothing completes, for at most limit_ns,
 // then records MOE_ETIMEOUT in counters[kCtrStatus].
 cudaError_t launch_wait_probe(int32_t *counters, uint64_t limit_ns, cudaStream_t s);
 
 // ------------------------------------------------------------ prefill path
-// Bytes of workspace for `rows` rows on either path.
+// Bytes of workspace for `rows` rows on either path (with or without the norm).
 size_t workspace_bytes(const moe_dims &d, int64_t rows);
+// Offset of the normed-x buffer [rows][H] bf16 (the norm entry on the grouped path).
+size_t norm_buffer_offset(const moe_dims &d, int64_t rows);
 // Whether the prefill path is built into this library.
 bool prefill_available();
 // Kernels one prefill call launches.

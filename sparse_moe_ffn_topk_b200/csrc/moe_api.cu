@@ -3,6 +3,7 @@
 // Host side only: argument checks, workspace carving, path selection, the
 // sticky status and the host fault knob.  Every step of the layer runs in
 // the kernels of decode.cu and prefill.cu.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -91,7 +92,8 @@ int kernel_launches(const moe_dims &d, int32_t rows, int32_t path)
     if (rows <= 0) return 0;
     path = resolve_path(d, rows, path);
     if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_NARROW) return prefill_kernel_launches(d, rows);
-    return 3;  // router_topk, gate_up, down
+    const int per = step_rows_per_launch(d, device_info().sm_count);
+    return per > 0 ? (rows + per - 1) / per : 0;  // one decode-step launch per `per` rows
 }
 
 const DeviceInfo &device_info()
@@ -108,7 +110,7 @@ const DeviceInfo &device_info()
         int smem = 0;
         cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         i.max_smem_optin = (size_t)smem;
-        if (i.sm_count <= 0) i.sm_count = 1;
+        if (i.sm_count <= 0) i.sm_count = 148;  // no device to ask (host-only queries): a B200's count
         g_dev_ready[dev] = true;
     }
     return g_dev[dev];
@@ -119,7 +121,7 @@ int check_forward_args(const moe_dims *d, const uint16_t *x, int32_t rows, const
                        const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
                        const uint16_t *shared_gate, const uint16_t *out, const uint16_t *residual,
                        const float *router_bias, int32_t path, const int32_t *topk_idx_out,
-                       const float *topk_w_out, const float *shared_gate_sig_out)
+                       const float *topk_w_out, const float *shared_gate_sig_out, bool out_may_alias_x)
 {
     int st = check_dims(d);
     if (st) return st;
@@ -135,7 +137,7 @@ int check_forward_args(const moe_dims *d, const uint16_t *x, int32_t rows, const
         (router_bias && !aligned16(router_bias)) || (topk_idx_out && !aligned16(topk_idx_out)) ||
         (topk_w_out && !aligned16(topk_w_out)) || (shared_gate_sig_out && !aligned16(shared_gate_sig_out)))
         return MOE_EINVAL;
-    if (static_cast<const void *>(out) == static_cast<const void *>(x)) return MOE_EINVAL;
+    if (!out_may_alias_x && static_cast<const void *>(out) == static_cast<const void *>(x)) return MOE_EINVAL;
     return MOE_OK;
 }
 
@@ -144,12 +146,19 @@ int run_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16
                 const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
                 const uint16_t *shared_gate, uint16_t *out, const uint16_t *residual, const float *router_bias,
                 void *ws, void *stream, int32_t path, int32_t *topk_idx_out, float *topk_w_out,
-                float *shared_gate_sig_out)
+                float *shared_gate_sig_out, const uint16_t *norm_w, double eps)
 {
     if (rows == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     path = resolve_path(*d, rows, path);
     if (path == MOE_PATH_PREFILL || path == MOE_PATH_PREFILL_NARROW) {
+        if (norm_w) {
+            // the norm as its own kernel; the layer reads its output, the residual is the input rows
+            uint16_t *xn = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + norm_buffer_offset(*d, rows));
+            if (launch_rmsnorm(x, norm_w, eps, d->hidden, rows, xn, s) != cudaSuccess) return finish(cudaGetLastError());
+            residual = x;
+            x = xn;
+        }
         int rc = prefill_forward(*d, x, rows, router_w, expert_w8, expert_scales, shared_w->w8,
                                  shared_w->scales, shared_gate, out, residual, router_bias, ws, s,
                                  topk_idx_out, topk_w_out, shared_gate_sig_out, path == MOE_PATH_PREFILL_NARROW);
@@ -159,48 +168,39 @@ int run_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16
 
     const DecodeLayout L = decode_layout(*d, rows);
     char *base = static_cast<char *>(ws);
-    int32_t *counters = reinterpret_cast<int32_t *>(base + L.counters);
     int32_t *tidx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(base + L.topk_idx);
     float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.topk_w);
     float *gs = shared_gate_sig_out ? shared_gate_sig_out : reinterpret_cast<float *>(base + L.gsig);
-
-    RouterLaunch ra;
-    ra.d = d;
-    ra.x = x;
-    ra.rows = rows;
-    ra.router_w = router_w;
-    ra.router_bias = router_bias;
-    ra.shared_gate = shared_gate;
-    ra.topk_idx = tidx;
-    ra.topk_w = tw;
-    ra.gsig = gs;
-    ra.logits = reinterpret_cast<float *>(base + L.logits);
-    ra.xq = reinterpret_cast<uint8_t *>(base + L.xq);
-    ra.xsc = reinterpret_cast<float *>(base + L.xsc);
-    ra.counters = counters;
-
-    ExpertsLaunch ea;
-    ea.d = d;
-    ea.x = x;
-    ea.xq = reinterpret_cast<const uint8_t *>(base + L.xq);
-    ea.xsc = reinterpret_cast<const float *>(base + L.xsc);
-    ea.rows = rows;
-    ea.expert_w8 = expert_w8;
-    ea.expert_scales = expert_scales;
-    ea.shared_w8 = shared_w->w8;
-    ea.shared_scales = shared_w->scales;
-    ea.residual = residual;
-    ea.out = out;
-    ea.topk_idx = tidx;
-    ea.topk_w = tw;
-    ea.gsig = gs;
-    ea.h_routed = reinterpret_cast<float *>(base + L.h_routed);
-    ea.h_shared = reinterpret_cast<float *>(base + L.h_shared);
-    ea.yslot = reinterpret_cast<float *>(base + L.yslot);
-    ea.counters = counters;
-    cudaError_t e = launch_router_topk(ra, s);
-    if (e != cudaSuccess) return finish(e);
-    return finish(launch_decode_experts(ea, s));
+    const int per = step_rows_per_launch(*d, device_info().sm_count);
+    if (per < 1) return MOE_EUNSUPPORTED;
+    const int H = d->hidden, K = d->top_k;
+    for (int r0 = 0; r0 < rows; r0 += per) {
+        StepLaunch a;
+        a.d = d;
+        a.rows = std::min(per, rows - r0);
+        a.x = x + (size_t)r0 * H;
+        a.norm_w = norm_w;
+        a.eps = eps;
+        a.router_w = router_w;
+        a.router_bias = router_bias;
+        a.shared_gate = shared_gate;
+        a.expert_w8 = expert_w8;
+        a.expert_scales = expert_scales;
+        a.shared_w8 = shared_w->w8;
+        a.shared_scales = shared_w->scales;
+        a.residual = norm_w ? a.x : residual ? residual + (size_t)r0 * H : nullptr;
+        a.out = out + (size_t)r0 * H;
+        a.topk_idx = tidx + (size_t)r0 * K;
+        a.topk_w = tw + (size_t)r0 * K;
+        a.gsig = gs + r0;
+        a.logits = reinterpret_cast<float *>(base + L.logits);
+        a.logits_ld = L.ld;
+        a.h = reinterpret_cast<float *>(base + L.h);
+        a.counters = reinterpret_cast<int32_t *>(base + L.counters);
+        const cudaError_t e = launch_decode_step(a, s);
+        if (e != cudaSuccess) return finish(e);
+    }
+    return finish(cudaSuccess);
 }
 
 }  // namespace moe
@@ -254,8 +254,6 @@ int moe_router_topk(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
     a.topk_w = topk_w;
     a.gsig = shared_gate_sig;
     a.logits = reinterpret_cast<float *>(base + L.logits);
-    a.xq = nullptr;
-    a.xsc = nullptr;
     a.counters = reinterpret_cast<int32_t *>(base + L.counters);
     return finish(launch_router_topk(a, static_cast<cudaStream_t>(stream)));
 }
@@ -268,7 +266,7 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
                          float *shared_gate_sig_out)
 {
     int st = check_forward_args(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out,
-                                residual, router_bias, path, topk_idx_out, topk_w_out, shared_gate_sig_out);
+                                residual, router_bias, path, topk_idx_out, topk_w_out, shared_gate_sig_out, false);
     if (st) return st;
     if (rows == 0) return enter();  // a no-op: no pointer is read
     if (!ws || !aligned16(ws)) return MOE_EINVAL;
@@ -276,7 +274,24 @@ int moe_ffn_forward_path(const moe_dims *d, const uint16_t *x, int32_t rows, con
     st = enter();
     if (st) return st;
     return run_forward(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out, residual,
-                       router_bias, ws, stream, path, topk_idx_out, topk_w_out, shared_gate_sig_out);
+                       router_bias, ws, stream, path, topk_idx_out, topk_w_out, shared_gate_sig_out, nullptr, 0.0);
+}
+
+int moe_ffn_forward_norm(const moe_dims *d, const uint16_t *resid, int32_t rows, const uint16_t *norm_w, float eps,
+                         const uint16_t *router_w, const uint8_t *expert_w8, const float *expert_scales,
+                         const moe_fp8_expert *shared_w, const uint16_t *shared_gate, uint16_t *out,
+                         const float *router_bias, void *ws, size_t ws_bytes, void *stream, int32_t path)
+{
+    int st = check_forward_args(d, resid, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out,
+                                nullptr, router_bias, path, nullptr, nullptr, nullptr, true);
+    if (st) return st;
+    if (rows == 0) return enter();  // a no-op: no pointer is read
+    if (!norm_w || !aligned16(norm_w) || !(eps >= 0.f) || !ws || !aligned16(ws)) return MOE_EINVAL;
+    if (ws_bytes < workspace_bytes(*d, rows)) return MOE_EWORKSPACE;
+    st = enter();
+    if (st) return st;
+    return run_forward(d, resid, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out, nullptr,
+                       router_bias, ws, stream, path, nullptr, nullptr, nullptr, norm_w, (double)eps);
 }
 
 int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,

@@ -69,9 +69,9 @@ inline PrefillLayout prefill_layout(const moe_dims &d, int64_t T)
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 1024); return at; };
     L.counters = take(sizeof(int32_t) * kCounters);
-    // up to MOE_DECODE_MAX_ROWS rows the decode path's router (spread over
+    // up to kSmallRouterRows rows the decode path's router (spread over
     // many CTAs) computes the routing; it needs fp32 logits rows
-    L.logits = take(T <= MOE_DECODE_MAX_ROWS ? sizeof(float) * T * ((E + 1 + 3) / 4 * 4) : 0);
+    L.logits = take(T <= kSmallRouterRows ? sizeof(float) * T * ((E + 1 + 3) / 4 * 4) : 0);
     L.topk_idx = take(sizeof(int32_t) * T * K);
     L.topk_w = take(sizeof(float) * T * K);
     L.gsig = take(sizeof(float) * T);
@@ -92,9 +92,14 @@ inline PrefillLayout prefill_layout(const moe_dims &d, int64_t T)
     return L;
 }
 
+size_t norm_buffer_offset(const moe_dims &d, int64_t rows)
+{
+    return align_up(std::max(decode_layout(d, rows).total, prefill_layout(d, rows).total), 256);
+}
+
 size_t workspace_bytes(const moe_dims &d, int64_t rows)
 {
-    return std::max(decode_layout(d, rows).total, prefill_layout(d, rows).total);
+    return norm_buffer_offset(d, rows) + align_up((size_t)rows * d.hidden * 2, 256);
 }
 
 bool prefill_available() { return true; }
@@ -1445,7 +1450,7 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
 
     // few rows: the decode router over many CTAs; else the tcgen05 router,
     // which also counts each expert's rows
-    const bool small_router = T <= MOE_DECODE_MAX_ROWS;
+    const bool small_router = T <= kSmallRouterRows;
     cudaError_t e = cudaSuccess;
     if (!small_router && (e = cudaMemsetAsync(base + L.counts, 0, sizeof(int32_t) * (E + 1), s)) != cudaSuccess)
         return MOE_ECUDA;
@@ -1487,8 +1492,6 @@ int prefill_forward(const moe_dims &d, const uint16_t *x, int32_t rows, const ui
         ra.topk_w = tw;
         ra.gsig = gs;
         ra.logits = reinterpret_cast<float *>(base + L.logits);
-        ra.xq = nullptr;  // the permute kernel quantises x
-        ra.xsc = nullptr;
         ra.counters = counters;
         if (launch_router_topk(ra, s) != cudaSuccess) return MOE_ECUDA;
     } else {

@@ -100,7 +100,7 @@ MOE_API int moe_ffn_forward_static(const moe_dims *d, const uint16_t *x, int32_t
                                    const uint16_t *residual, const float *router_bias, void *stream)
 {
     int st = check_forward_args(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out,
-                                residual, router_bias, MOE_PATH_AUTO, nullptr, nullptr, nullptr);
+                                residual, router_bias, MOE_PATH_AUTO, nullptr, nullptr, nullptr, false);
     if (st) return st;
     if (rows == 0) return enter();  // a no-op: no pointer is read
     const size_t need = moe_workspace_bytes(d, rows);
@@ -121,7 +121,7 @@ MOE_API int moe_ffn_forward_static(const moe_dims *d, const uint16_t *x, int32_t
         e = cudaMemsetAsync(ctr + kCtrStatus + 1, 0, sizeof(int32_t) * (kCounters - kCtrStatus - 1), s);
     if (e != cudaSuccess) return cuda_failed(e);
     return run_forward(d, x, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate, out, residual,
-                       router_bias, ws, stream, MOE_PATH_AUTO, nullptr, nullptr, nullptr);
+                       router_bias, ws, stream, MOE_PATH_AUTO, nullptr, nullptr, nullptr, nullptr, 0.0);
 }
 
 MOE_API int moe_static_device_status(void *stream)

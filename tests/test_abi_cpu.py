@@ -98,10 +98,11 @@ def test_argument_checks_on_host(L):
 def test_paths_and_launch_counts(L):
     d = D()
     assert moe.kernel_launches(d, 0) == 0
-    assert moe.kernel_launches(d, moe.MOE_AUTO_DECODE_MAX_ROWS) == 3
+    assert moe.kernel_launches(d, moe.MOE_AUTO_DECODE_MAX_ROWS) == 1     # one decode-step kernel
     assert moe.kernel_launches(d, moe.MOE_AUTO_DECODE_MAX_ROWS + 1) == 6
-    for path, n in ((moe.MOE_PATH_DECODE, 3), (moe.MOE_PATH_PREFILL, 6), (moe.MOE_PATH_PREFILL_NARROW, 6)):
-        assert moe.kernel_launches(d, 5, path) == n
+    for path, n in ((moe.MOE_PATH_DECODE, 2), (moe.MOE_PATH_PREFILL, 6), (moe.MOE_PATH_PREFILL_NARROW, 6)):
+        assert moe.kernel_launches(d, 5, path) == n                        # decode: 4 rows per launch
+    assert moe.kernel_launches(d, 64, moe.MOE_PATH_DECODE) == 64 // moe.MOE_DECODE_MAX_ROWS
     assert moe.kernel_launches(d, 5, 4) == 0                  # no such path
     assert moe.auto_path(d, 1) == moe.MOE_PATH_DECODE
     assert moe.auto_path(d, moe.MOE_AUTO_DECODE_MAX_ROWS + 1) == moe.MOE_PATH_PREFILL_NARROW
