@@ -408,6 +408,24 @@ class DecodeBench:
         return counts
 
 
+class ChainBench(DecodeBench):
+    """A stack of layers behind their RMSNorms: step i runs layer i mod L on
+    the one residual stream r in place, r <- r + layer(bf16(rmsnorm(r) * w)),
+    so every step reads the previous step's output (one launch per layer on
+    the decode path, chained by programmatic dependent launch)."""
+
+    def __init__(self, dims, insts, norm_ws, resid, rows):
+        super().__init__(dims, insts, [resid], rows)
+        self.norm_ws = norm_ws
+        self.r = resid
+
+    def step(self, i, events=None):
+        w = self.insts[i % len(self.insts)]
+        self.moe.ffn_forward_norm(self.d, self.r, self.norm_ws[i % len(self.norm_ws)], 1e-6, w["router_w"],
+                                  w["expert_w8"], w["expert_scales"], w["shared_w8"], w["shared_scales"],
+                                  w["shared_gate"], self.r, self.ws, stream=self.stream)
+
+
 class PrefillBench(DecodeBench):
     """Prefill steps of the same layer: `rows` tokens, a per-expert router
     bias, the prefill path (permute -> tcgen05 grouped GEMMs -> blend)."""
@@ -676,6 +694,25 @@ def run_ours(args, dist: Dist):
                             "dtype": GROUPED_DTYPE if moe.auto_path(d, r64) != moe.MOE_PATH_DECODE else DECODE_DTYPE,
                             "kernels": {moe.MOE_PATH_DECODE: "decode", moe.MOE_PATH_PREFILL: "grouped",
                                         moe.MOE_PATH_PREFILL_NARROW: "narrow"}[moe.auto_path(d, r64)]}
+
+    # ---- a chain of layers behind their norms (rows = 1): one launch per layer
+    if not args.no_extras:
+        g = torch.Generator().manual_seed(args.seed + 7)
+        nws = [(1.0 + 0.1 * torch.randn(d.hidden, generator=g)).to(torch.bfloat16).cuda()
+               for _ in range(N_INSTANCES)]
+        r0 = torch.from_numpy(mi.make_residual(d, rows, seed=args.seed, stream=77).view("int16")).view(
+            torch.bfloat16).cuda()
+        cb = ChainBench(d, insts, nws, r0, rows)
+        kc = args.steps
+        msc, _ = cb.time_steps(kc, args.warmup, dist)
+        sc = dist.max(msc / 1000.0)
+        result["chain"] = {"layers": N_INSTANCES, "steps": kc, "us_per_layer": round(sc * 1e6 / kc, 3),
+                           "gb_s": round(aggregate(kc * by1["total"], dist.world, sc) / 1e9, 1),
+                           "hbm_frac_of_measured": round(aggregate(kc * by1["total"], dist.world, sc) / 1e9
+                                                         / dist.world / hbm_peak, 4),
+                           "what": "each step: r <- r + layer_l(bf16(rmsnorm(r) * w_l)) in place, l = step mod "
+                                   f"{N_INSTANCES}; the norm runs inside the decode-step kernel"}
+        del cb
 
     # ---- prefill, 4096 tokens
     result["prefill"] = prefill_leg(args, d, insts[0], dist, bus, hbm_peak, bf16_peak, peak_kind)

@@ -237,13 +237,37 @@ __device__ __forceinline__ void gave_up(int32_t *counters, int kind, int item)
     } while (0)
 #endif
 
+// Phase timestamps of a development build (-DMOE_STEP_TRACE): thread 0 of
+// each CTA (lane 0 of warp 0 for the per-warp points) records %globaltimer
+// at numbered points of the step.
+#ifdef MOE_STEP_TRACE
+__device__ unsigned long long g_step_trace[256 * 16];
+__device__ unsigned long long g_item_trace[256 * 64 * 6];  // per CTA, item: landed, done, issued, [issue start, after expect_tx, after 1st TMA]
+#define ITEM_T(q, which)                                                                        \
+    do {                                                                                        \
+        if ((threadIdx.x & 31) == 0 && (q) < 64)                                                \
+            g_item_trace[(blockIdx.x * 64 + (q)) * 6 + (which)] = globaltimer_ns();             \
+    } while (0)
+#define STEP_T(i)                                                                          \
+    do {                                                                                   \
+        if (threadIdx.x == 0) g_step_trace[blockIdx.x * 16 + (i)] = globaltimer_ns();      \
+    } while (0)
+#else
+#define STEP_T(i) \
+    do {          \
+    } while (0)
+#define ITEM_T(q, which) \
+    do {                 \
+    } while (0)
+#endif
+
 // ------------------------------------------------------------ parameters
 
 struct StepParams {
     CUtensorMap w13;   // routed W13: (128 B, 2I rows, H/128 windows, E), boxes {128, 8, gu_wp, 1}
     CUtensorMap w13s;  // shared W13: (128 B, 2Is rows, H/128 windows, 1)
-    CUtensorMap w2;    // routed W2: (128 B, H rows, I/128 windows, E), boxes {128, 8, dn_wp, 1}
-    CUtensorMap w2s;   // shared W2: (128 B, H rows, Is/128 windows, 1), boxes {128, 8, dn_wp_s, 1}
+    CUtensorMap w2;    // routed W2: (128 B, H rows, I/128 windows, E), boxes {128, 8, I/128, 1}
+    CUtensorMap w2s;   // shared W2: (128 B, H rows, Is/128 windows, 1), boxes {128, 8, Is/128, 1}
     const uint16_t *x;
     const uint16_t *router_w;
     const uint16_t *shared_gate;
@@ -263,11 +287,12 @@ struct StepParams {
     int rows, H, E, K, I, Is, ld, imax;
     int ns;              // ring slots
     int gu_wp, gu_pieces;               // gate/up: K windows per piece, pieces
-    int dn_wp, dn_pieces, dn_wp_s, dn_pieces_s, dn_epi;  // down: windows/pieces (routed, shared), experts per item
+    int dn_tpi, dn_tpi_s, dn_epi;  // down: output tiles per item (routed, shared), routed experts per item
     int nt_max;          // output 8-row tiles per CTA, at most
     int rr_per_item;     // router rows per ring item
     // shared-memory offsets (from the 1024-aligned base)
-    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar;
+    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_part;
+    int max_units;       // gate/up units per CTA, at most (rows of the scale table)
     int x_stride;        // halves per x row in shared memory (f16 and bf16 copies)
     int t_stride;        // halves per h term row in shared memory
 };
@@ -281,6 +306,7 @@ struct StepSmall {
     uint32_t mask[kMaxExperts / 32];
     int32_t list[kStepMaxRows * kMaxTopK];  // distinct routed experts, ascending
     int32_t tag[16];                        // ring slot -> the item last issued into it (-1: none)
+    int32_t unit_done[kStepWarps];          // split mode: pieces finished per local unit
     double red[kStepWarps * kStepMaxRows];  // RMSNorm: per-warp sums of squares
     double inv[kStepMaxRows];               // RMSNorm: 1 / sqrt(mean square + eps) per row
     int32_t n_list;
@@ -310,9 +336,12 @@ struct Item {
 };
 
 struct Seq {
-    int n_router, n_units_local, n_gu, n_groups, n_dn, total;
+    int n_router, n_units_local, n_gu, n_tc_s, n_tc_r, n_groups_r, n_dn, total;
 };
 
+// Down items: per group of experts (the shared expert alone, then groups of
+// dn_epi routed experts of the list), per chunk of dn_tpi output tiles of
+// this CTA, the full K of the down rows (one TMA box per expert and tile).
 __device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt)
 {
     const int G = gridDim.x, c = blockIdx.x;
@@ -322,12 +351,17 @@ __device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt)
     const int units = p.Is / 8 + U * (p.I / 8);
     s.n_units_local = units > c ? (units - 1 - c) / G + 1 : 0;
     s.n_gu = s.n_units_local * p.gu_pieces;
-    s.n_groups = nt > 0 ? 1 + (U + p.dn_epi - 1) / p.dn_epi : 0;
-    s.n_dn = nt > 0 ? p.dn_pieces_s + (s.n_groups - 1) * p.dn_pieces : 0;
+    s.n_tc_s = nt > 0 ? (nt + p.dn_tpi_s - 1) / p.dn_tpi_s : 0;
+    s.n_tc_r = nt > 0 ? (nt + p.dn_tpi - 1) / p.dn_tpi : 0;
+    s.n_groups_r = (U + p.dn_epi - 1) / p.dn_epi;
+    s.n_dn = s.n_tc_s + s.n_groups_r * s.n_tc_r;
     s.total = s.n_router + s.n_gu + s.n_dn;
     return s;
 }
 
+// kind 0 router: a = first local router row; kind 1 gate/up: a = unit, b =
+// local unit, p = piece; kind 2 down: a = group (0 shared), p = tile chunk,
+// b = the down item's index (its warp is b % kStepWarps).
 __device__ __forceinline__ Item item_at(const StepParams &p, const Seq &s, int q)
 {
     Item it;
@@ -349,14 +383,15 @@ __device__ __forceinline__ Item item_at(const StepParams &p, const Seq &s, int q
     }
     q -= s.n_gu;
     it.kind = 2;
-    it.b = 0;
-    if (q < p.dn_pieces_s) {
+    it.b = q;
+    if (q < s.n_tc_s) {
         it.a = 0;
         it.p = q;
     } else {
-        q -= p.dn_pieces_s;
-        it.a = 1 + q / p.dn_pieces;
-        it.p = q - (it.a - 1) * p.dn_pieces;
+        q -= s.n_tc_s;
+        const int g = q / s.n_tc_r;
+        it.a = 1 + g;
+        it.p = q - g * s.n_tc_r;
     }
     return it;
 }
@@ -392,13 +427,17 @@ __device__ __forceinline__ uint32_t item_bytes(const StepParams &p, const Item &
     if (it.kind == 0) return (uint32_t)min(p.rr_per_item, nr_total - it.a) * (uint32_t)p.H * 2u;
     if (it.kind == 1) return (uint32_t)p.gu_wp * 2048u;
     const int ne = group_size(p, U, it.a);
-    return (uint32_t)ne * (uint32_t)nt * (uint32_t)(it.a == 0 ? p.dn_wp_s : p.dn_wp) * 1024u;
+    const int tpi = it.a == 0 ? p.dn_tpi_s : p.dn_tpi;
+    const int ntile = min(tpi, nt - it.p * tpi);
+    return (uint32_t)ne * (uint32_t)ntile * 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);
 }
 
 __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t slot, uint64_t *full,
-                           int r0, int nr_total, int tile0, int nt, int U, uint64_t pol)
+                           int r0, int nr_total, int tile0, int nt, int U, uint64_t pol, int qdbg = 0)
 {
+    ITEM_T(qdbg, 3);
     mbar_arrive_expect_tx(full, item_bytes(p, it, nr_total, nt, U));
+    ITEM_T(qdbg, 4);
     if (it.kind == 0) {
         // router rows r0 + it.a ..; row E (the gate vector) comes from shared_gate
         const int n = min(p.rr_per_item, nr_total - it.a);
@@ -427,17 +466,19 @@ __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item 
         const int Iu = shared ? p.Is : p.I;
         const int w0 = it.p * p.gu_wp;
         tma_load_4d(slot, m, 0, j, w0, e, full, pol);
+        ITEM_T(qdbg, 5);
         tma_load_4d(slot + (uint32_t)p.gu_wp * 1024u, m, 0, Iu + j, w0, e, full, pol);
         return;
     }
     const int ne = group_size(p, U, it.a);
-    const int wp = it.a == 0 ? p.dn_wp_s : p.dn_wp;
+    const int tpi = it.a == 0 ? p.dn_tpi_s : p.dn_tpi;
+    const int ntile = min(tpi, nt - it.p * tpi);
     const CUtensorMap *m = it.a == 0 ? &p.w2s : &p.w2;
-    const uint32_t box = (uint32_t)wp * 1024u;
+    const uint32_t box = 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);
     for (int x = 0; x < ne; ++x) {
         const int e = it.a == 0 ? 0 : sm.list[(it.a - 1) * p.dn_epi + x];
-        for (int i = 0; i < nt; ++i)
-            tma_load_4d(slot + (uint32_t)(x * nt + i) * box, m, 0, (tile0 + i) * 8, it.p * wp, e, full, pol);
+        for (int i = 0; i < ntile; ++i)
+            tma_load_4d(slot + (uint32_t)(x * tpi + i) * box, m, 0, (tile0 + it.p * tpi + i) * 8, 0, e, full, pol);
     }
 }
 
@@ -470,30 +511,37 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             mbar_init(&empty[s], 1);
             sm.tag[s] = -1;
         }
+        for (int u = 0; u < kStepWarps; ++u) sm.unit_done[u] = 0;
         sm.abort = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
+    STEP_T(0);
     // ---------------------------------------------------------------- P0
     // The producer issues the items that depend only on weights: router
     // rows, then the shared expert's gate/up units (the first local units).
-    int q_issued = 0;
     const uint64_t pol = policy_evict_first();
-    if (producer && lane == 0) {
-        tma_prefetch_desc(&p.w13);
-        tma_prefetch_desc(&p.w13s);
-        tma_prefetch_desc(&p.w2);
-        tma_prefetch_desc(&p.w2s);
-        const Seq s0 = make_seq(p, 0, 0);  // U = 0: router and shared-expert items only
-        for (; q_issued < s0.total && q_issued < p.ns; ++q_issued) {
-            const Item it = item_at(p, s0, q_issued);
-            issue_item(p, sm, it, base + (uint32_t)q_issued * kSlot, &full[q_issued], r0, nr_total, tile0, nt, 0, pol);
-            ((volatile int32_t *)sm.tag)[q_issued] = q_issued;
+    const Seq s0 = make_seq(p, 0, 0);  // U = 0: router and shared-expert items only (a prefix of the full sequence)
+    const int p0_count = min(s0.total, p.ns);
+    if (producer) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.w13);
+            tma_prefetch_desc(&p.w13s);
+            tma_prefetch_desc(&p.w2);
+            tma_prefetch_desc(&p.w2s);
+        }
+        // the lanes issue in parallel: lane l takes items l, l + 32, ...
+        for (int q = lane; q < p0_count; q += kWarp) {
+            issue_item(p, sm, item_at(p, s0, q), base + (uint32_t)q * kSlot, &full[q], r0, nr_total, tile0, nt, 0,
+                       pol, q);
+            ((volatile int32_t *)sm.tag)[q] = q;
+            ITEM_T(q, 2);
         }
     }
 
     pdl_wait();  // x and the workspace may be written by the previous kernel
+    STEP_T(1);
 
     // ---------------------------------------------------------------- P1
     if (!producer) {
@@ -550,8 +598,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             *reinterpret_cast<uint2 *>(xs + (size_t)t * p.x_stride + kb * 128 + lane * 4) = o;
             if (lane == 0) xfac[t * hb + kb] = pow2f(-sh);
         }
+        STEP_T(2);  // x staged
         // router rows (router items 0 .. n_router-1 in slots 0 ..)
-        const Seq s0 = make_seq(p, 0, 0);
         for (int ri = 0; ri < s0.n_router; ++ri) {
             if (!warp_wait(&full[ri], 0)) {
                 if (lane == 0) {
@@ -597,6 +645,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         }
         __threadfence();
         named_barrier(1, kStepWarps * kWarp);
+        STEP_T(3);  // router rows done
         if (threadIdx.x == 0) {
             // the router slots are free again
             for (int ri = 0; ri < s0.n_router; ++ri) mbar_arrive(&empty[ri]);
@@ -614,9 +663,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             }
         }
         named_barrier(1, kStepWarps * kWarp);
+        STEP_T(4);  // grid barrier 1 passed
         // ------------------------------------------------------------ P2
         // top-k of every row, in every CTA
         if (!*abort && warp < rows) {
+            if (warp == 0) STEP_T(12);
             const float *lrow = p.logits + (size_t)warp * p.ld;
             int32_t *oi = sm.idx + warp * K;
             float *ow = sm.w + warp * K;
@@ -627,6 +678,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             else if (E <= 256) topk_select<8>(lrow, E, K, oi, ow, og);
             else if (E <= 512) topk_select<16>(lrow, E, K, oi, ow, og);
             else topk_select<32>(lrow, E, K, oi, ow, og);
+            if (warp == 0) STEP_T(13);
         }
         named_barrier(1, kStepWarps * kWarp);
         if (!*abort && warp == 0) {
@@ -658,6 +710,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             }
             if (lane == 0) sm.n_list = before;
             __syncwarp();
+            STEP_T(14);
             for (int i = lane; i < rows * K; i += kWarp) {
                 const int e = sm.idx[i];
                 int pos = 0;
@@ -675,59 +728,62 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         }
     }
     __syncthreads();  // the plan is ready (all 288 threads)
+    STEP_T(5);
     const int U = *abort ? 0 : sm.n_list;
     const Seq seq = make_seq(p, U, nt);
 
     if (producer) {
         // ---------------------------------------------------------- producer
-        // Phase A, before grid barrier 2: issue while the slot's previous
-        // item is a router or gate/up item (down items are consumed only
-        // after the barrier, so their slots cannot be waited for here).
-        if (lane == 0) {
-            int q = q_issued;
-            for (; q < seq.total && !*abort; ++q) {
+        // The lanes issue in parallel, lane l the items l, l + 32, ... in
+        // order; item q reuses ring slot q % ns once the slot's previous item
+        // (q - ns) was consumed.  Phase A, before grid barrier 2: items whose
+        // slot last held a router or gate/up item (down items are consumed
+        // only after the barrier, so their slots cannot be waited for here).
+        int q = lane;
+        while (q < p0_count) q += kWarp;  // issued in P0
+        for (int phase = 0; phase < 2; ++phase) {
+            for (; q < seq.total && !*abort; q += kWarp) {
                 const int s = q % p.ns;
-                STEP_MARK(10, q);
                 if (q >= p.ns) {
-                    if (item_at(p, seq, q - p.ns).kind == 2) break;
-                    if (!mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
+                    if (phase == 0 && item_at(p, seq, q - p.ns).kind == 2) break;
+                    // The slot's previous item (q - ns) belongs to another lane:
+                    // wait until it is issued (its tag), which proves that the
+                    // item before it in the slot was consumed; the parity wait
+                    // for its consumption is then exact (a lane running ahead
+                    // would otherwise see the phase two back completed).
+                    bool issued = ((volatile int32_t *)sm.tag)[s] == q - p.ns;
+                    if (!issued) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (!(issued = ((volatile int32_t *)sm.tag)[s] == q - p.ns))
+                            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+                    }
+                    if (!issued || !mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
                         STEP_SNAP(s);
-                        gave_up(p.counters, 4, q);
+                        gave_up(p.counters, 4 + phase, q);
                         *abort = 1;
                         break;
                     }
                     fence_proxy_async_smem();
                 }
                 issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt,
-                           U, pol);
+                           U, pol, q);
                 ((volatile int32_t *)sm.tag)[s] = q;
+                ITEM_T(q, 2);
             }
-            q_issued = q;
+            if (phase == 0) {
+                __syncwarp();
+                named_barrier(2, kStepThreads);  // gate/up of this CTA done
+                named_barrier(2, kStepThreads);  // grid barrier 2 passed
+            }
         }
+        // every issued copy lands before the CTA may leave: the last item
+        // issued into each slot (all of them were consumed on the normal path)
         __syncwarp();
-        named_barrier(2, kStepThreads);  // gate/up of this CTA done
-        named_barrier(2, kStepThreads);  // grid barrier 2 passed
         if (lane == 0) {
-            // Phase B: the rest, as the down items are consumed.
-            int q = q_issued;
-            for (; q < seq.total && !*abort; ++q) {
-                const int s = q % p.ns;
-                if (q >= p.ns) {
-                    if (!mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
-                        gave_up(p.counters, 5, q);
-                        *abort = 1;
-                        break;
-                    }
-                    fence_proxy_async_smem();
-                }
-                issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt,
-                           U, pol);
-                ((volatile int32_t *)sm.tag)[s] = q;
+            for (int sl = 0; sl < p.ns; ++sl) {
+                const int t = ((volatile int32_t *)sm.tag)[sl];
+                if (t >= 0) mbar_wait(&full[sl], (t / p.ns) & 1, kWaitLimitNs);
             }
-            q_issued = q;
-            // every issued copy lands before the CTA may leave
-            for (int qq = max(0, q_issued - p.ns); qq < q_issued; ++qq)
-                mbar_wait(&full[qq % p.ns], (qq / p.ns) & 1, kWaitLimitNs);
         }
         return;
     }
@@ -737,12 +793,66 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     uint16_t *xs = reinterpret_cast<uint16_t *>(sbase + p.o_uni);
     const float *xfac = reinterpret_cast<const float *>(sbase + p.o_xfac);
 
-    // gate/up units: local unit l -> warp l % kStepWarps, its pieces in order
+    // Block scales of this CTA's work into shared memory, one round trip for
+    // all of them (the weight copies are in flight meanwhile): per local
+    // gate/up unit its gate and up row blocks [2][H/128]; per down expert
+    // (shared first, then the routed list) the row blocks of this CTA's
+    // output rows [2][Iu/128].
+    float *gsc = reinterpret_cast<float *>(sbase + p.o_gsc);
+    float *dsc = reinterpret_cast<float *>(sbase + p.o_dsc);
+    const int ibm = p.imax / 128;
+    const int rb0 = (tile0 * 8) / 128;
     {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int ng = seq.n_units_local * 2 * hb;
+        const int nd = nt > 0 ? (U + 1) * 2 * ibm : 0;
+        for (int i = threadIdx.x; i < ng + nd; i += kStepWarps * kWarp) {
+            if (i < ng) {
+                const int l = i / (2 * hb), rem = i - l * 2 * hb, half = rem / hb, W = rem - half * hb;
+                bool shared;
+                int e, j;
+                unit_of(p, sm, c + l * G, shared, e, j);
+                const int Iu = shared ? p.Is : p.I;
+                const float *sc = shared ? p.sscales
+                                         : p.scales + (size_t)e * ((size_t)(2 * Iu / 128) * hb + (size_t)hb * (Iu / 128));
+                gsc[i] = __ldg(sc + (size_t)((half ? Iu + j : j) / 128) * hb + W);
+            } else {
+                const int k = i - ng;
+                const int de = k / (2 * ibm), rem = k - de * 2 * ibm, rb = rem / ibm, W = rem - rb * ibm;
+                const bool shared = de == 0;
+                const int e = shared ? 0 : sm.list[de - 1];
+                const int Iu = shared ? p.Is : p.I;
+                const int ibu = Iu / 128;
+                float v = 0.f;
+                if (W < ibu && rb0 + rb < H / 128) {
+                    const float *s2 = (shared ? p.sscales
+                                              : p.scales + (size_t)e * ((size_t)(2 * Iu / 128) * hb + (size_t)hb * ibu)) +
+                                      (size_t)(2 * Iu / 128) * hb;
+                    v = __ldg(s2 + (size_t)(rb0 + rb) * ibu + W);
+                }
+                dsc[k] = v;
+            }
+        }
+        named_barrier(1, kStepWarps * kWarp);
+    }
+
+    // gate/up items.  With at least as many local units as warps, unit l
+    // goes to warp l % kStepWarps, which takes its K pieces in order and keeps
+    // the sums in registers.  With fewer (split mode), the items go round
+    // robin over the warps; each piece's partial sums go to shared memory
+    // and the warp that finishes a unit's last piece adds the pieces in
+    // piece order and runs the unit's epilogue.
+    {
+        const bool split = seq.n_units_local < kStepWarps;
+        float *part = reinterpret_cast<float *>(sbase + p.o_part);  // [unit][piece][32 lanes][4]
+        const int t0 = 2 * qd, t1 = 2 * qd + 1;
+        // acc: one piece's sums (from zero); tot: the pieces added in piece
+        // order, the same in both modes (a row's bits must not depend on the
+        // other rows of the call)
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
         for (int q = seq.n_router; q < seq.n_router + seq.n_gu && !*abort; ++q) {
             const Item it = item_at(p, seq, q);
-            if (it.b % kStepWarps != warp) continue;
+            const int owner = split ? (q - seq.n_router) % kStepWarps : it.b % kStepWarps;
+            if (owner != warp) continue;
             const int s = q % p.ns;
             STEP_MARK(2, q);
             if (!wait_item(sm.tag, full, s, q, p.ns)) {
@@ -754,54 +864,86 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 break;
             }
             STEP_MARK(3, q);
+            ITEM_T(q, 0);
+            if (threadIdx.x == 0 && q == seq.n_router) STEP_T(6);  // warp 0's first gate/up item landed
             bool shared;
             int e, j;
             unit_of(p, sm, it.a, shared, e, j);
-            const int Iu = shared ? p.Is : p.I;
-            const float *sc = shared ? p.sscales : p.scales + (size_t)e * ((size_t)(2 * Iu / 128) * hb + (size_t)hb * (Iu / 128));
-            const float *sg_row = sc + (size_t)(j / 128) * hb;
-            const float *su_row = sc + (size_t)((Iu + j) / 128) * hb;
-            if (it.p == 0) acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            const float *sg_row = gsc + (size_t)it.b * 2 * hb;
+            const float *su_row = sg_row + hb;
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
             const uint32_t sl = base + (uint32_t)s * kSlot;
             const uint32_t gate_base = sl + (uint32_t)g * 128u;
             const uint32_t up_base = sl + (uint32_t)p.gu_wp * 1024u + (uint32_t)g * 128u;
             const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
             const bool xrow = g < rows;
             const uint32_t xaddr = smem_u32(xs) + (uint32_t)(g * p.x_stride * 2);
+            // one window per iteration: 8 MMA steps on two accumulators
+            // (even and odd steps)
             for (int w = 0; w < p.gu_wp; ++w) {
                 const int W = it.p * p.gu_wp + w;
                 if (W >= hb) break;
-                const uint4 ga0 = lds128(gate_base + w * 1024u + c0), ga1 = lds128(gate_base + w * 1024u + c1);
-                const uint4 ua0 = lds128(up_base + w * 1024u + c0), ua1 = lds128(up_base + w * 1024u + c1);
+                const uint32_t wo = (uint32_t)w * 1024u;
+                const uint4 ga0 = lds128(gate_base + wo + c0), ga1 = lds128(gate_base + wo + c1);
+                const uint4 ua0 = lds128(up_base + wo + c0), ua1 = lds128(up_base + wo + c1);
                 uint4 xb[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     xb[i] = xrow ? lds128(xaddr + (uint32_t)((W * 128 + 32 * qd + 8 * i) * 2)) : make_uint4(0, 0, 0, 0);
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
                 for (int st = 0; st < 8; ++st) {
                     const uint32_t gw = word_of(st < 4 ? ga0 : ga1, st & 3);
                     const uint32_t uw = word_of(st < 4 ? ua0 : ua1, st & 3);
                     const uint32_t b0 = word_of(xb[st >> 1], (st & 1) * 2);
                     const uint32_t b1 = word_of(xb[st >> 1], (st & 1) * 2 + 1);
-                    mma_f16_16816(d, e4m3x2_to_f16x2(gw), e4m3x2_to_f16x2(uw), e4m3x2_to_f16x2(gw >> 16),
+                    mma_f16_16816(d[st & 1], e4m3x2_to_f16x2(gw), e4m3x2_to_f16x2(uw), e4m3x2_to_f16x2(gw >> 16),
                                   e4m3x2_to_f16x2(uw >> 16), b0, b1);
                 }
-                const float sgw = __ldg(sg_row + W), suw = __ldg(su_row + W);
-                const int t0 = 2 * qd, t1 = 2 * qd + 1;
+                const float sgw = sg_row[W], suw = su_row[W];
                 const float f0 = t0 < rows ? xfac[t0 * hb + W] : 0.f;
                 const float f1 = t1 < rows ? xfac[t1 * hb + W] : 0.f;
-                acc[0] = fmaf(sgw * f0, d[0], acc[0]);
-                acc[1] = fmaf(sgw * f1, d[1], acc[1]);
-                acc[2] = fmaf(suw * f0, d[2], acc[2]);
-                acc[3] = fmaf(suw * f1, d[3], acc[3]);
+                acc[0] = fmaf(sgw * f0, d[0][0] + d[1][0], acc[0]);
+                acc[1] = fmaf(sgw * f1, d[0][1] + d[1][1], acc[1]);
+                acc[2] = fmaf(suw * f0, d[0][2] + d[1][2], acc[2]);
+                acc[3] = fmaf(suw * f1, d[0][3] + d[1][3], acc[3]);
             }
             STEP_MARK(4, q);
+            ITEM_T(q, 1);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
             STEP_MARK(5, q);
             STEP_CONSUMED(q);
-            if (it.p == p.gu_pieces - 1) {
+            bool last = it.p == p.gu_pieces - 1;
+            if (!split || p.gu_pieces == 1) {
+                if (it.p == 0) tot[0] = tot[1] = tot[2] = tot[3] = 0.f;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) tot[r] += acc[r];
+            } else {
+                // this piece's sums to shared memory; the last piece of the unit adds them in order
+                float *pp = part + (((size_t)it.b * p.gu_pieces + it.p) * kWarp + lane) * 4;
+                pp[0] = acc[0];
+                pp[1] = acc[1];
+                pp[2] = acc[2];
+                pp[3] = acc[3];
+                __threadfence_block();
+                __syncwarp();
+                int prev = 0;
+                if (lane == 0) prev = atomicAdd(&sm.unit_done[it.b], 1);
+                prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+                last = prev == p.gu_pieces - 1;
+                if (last) {
+                    __threadfence_block();
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) tot[r] = 0.f;
+                    for (int pc = 0; pc < p.gu_pieces; ++pc) {
+                        const float *src = part + (((size_t)it.b * p.gu_pieces + pc) * kWarp + lane) * 4;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) tot[r] += ((volatile const float *)src)[r];
+                    }
+                }
+            }
+            if (last) {
                 // h = silu(gate) * up for rows 2q, 2q+1 routed to this expert
 #pragma unroll
                 for (int k2 = 0; k2 < 2; ++k2) {
@@ -815,13 +957,14 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                             if (sm.idx[t * K + r] == e) slot = t * K + r;
                     }
                     if (slot < 0) continue;
-                    const float gt = acc[k2], up = acc[2 + k2];
+                    const float gt = tot[k2], up = tot[2 + k2];
                     p.h[(size_t)slot * p.imax + j + g] = siluf_(gt) * up;
                 }
             }
         }
     }
     STEP_MARK(6, 0);
+    STEP_T(7);  // warp 0's gate/up items done
     __threadfence();
     named_barrier(2, kStepThreads);  // gate/up of this CTA done (producer included)
     if (threadIdx.x == 0) {
@@ -848,6 +991,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         }
     }
     named_barrier(2, kStepThreads);
+    STEP_T(8);  // grid barrier 2 passed
     pdl_trigger();
     if (*abort || nt == 0) return;
 
@@ -857,156 +1001,189 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const int ib = p.imax / 128;
     uint16_t *terms = xs;  // the x region is free now
     float *hfac = reinterpret_cast<float *>(sbase + p.o_hfac);
-    for (int u = warp; u < nslots * ib; u += kStepWarps) {
-        const int sl = u / ib, kb = u - sl * ib;
-        const int Iu = sl >= rows * K ? p.Is : p.I;
-        if (kb * 128 >= Iu) continue;
-        const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane);
-        const float amax = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        const int sh = block_shift(amax);
-        const float f = pow2f(sh);
-        const float a[4] = {v.x * f, v.y * f, v.z * f, v.w * f};
-        uint32_t t0[2], t1[2], t2[2];
+    {
+        // every (slot, block) pair of h: one warp each, in batches of 8 per
+        // warp with all eight loads in flight before any is used
+        constexpr int kBatch = 8;
+        const int n_items = nslots * ib;
+        for (int u0 = warp; u0 < n_items; u0 += kStepWarps * kBatch) {
+            float4 v[kBatch];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float x0 = a[2 * i], x1 = a[2 * i + 1];
-            const __half2 h0 = __floats2half2_rn(x0, x1);
-            const float2 r0 = __half22float2(h0);
-            const float y0 = x0 - r0.x, y1 = x1 - r0.y;
-            const __half2 h1 = __floats2half2_rn(y0, y1);
-            const float2 r1 = __half22float2(h1);
-            const __half2 h2 = __floats2half2_rn(y0 - r1.x, y1 - r1.y);
-            t0[i] = *reinterpret_cast<const uint32_t *>(&h0);
-            t1[i] = *reinterpret_cast<const uint32_t *>(&h1);
-            t2[i] = *reinterpret_cast<const uint32_t *>(&h2);
+            for (int k = 0; k < kBatch; ++k) {
+                const int u = u0 + k * kStepWarps;
+                const int sl = u / ib, kb = u - sl * ib;
+                const int Iu = sl >= rows * K ? p.Is : p.I;
+                v[k] = (u < n_items && kb * 128 < Iu)
+                           ? __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const int u = u0 + k * kStepWarps;
+                const int sl = u / ib, kb = u - sl * ib;
+                const int Iu = sl >= rows * K ? p.Is : p.I;
+                if (u >= n_items || kb * 128 >= Iu) continue;
+                const float amax =
+                    warp_max(fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
+                const int sh = block_shift(amax);
+                const float f = pow2f(sh);
+                const float a[4] = {v[k].x * f, v[k].y * f, v[k].z * f, v[k].w * f};
+                uint32_t t0[2], t1[2], t2[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float x0 = a[2 * i], x1 = a[2 * i + 1];
+                    const __half2 h0 = __floats2half2_rn(x0, x1);
+                    const float2 r0 = __half22float2(h0);
+                    const float y0 = x0 - r0.x, y1 = x1 - r0.y;
+                    const __half2 h1 = __floats2half2_rn(y0, y1);
+                    const float2 r1 = __half22float2(h1);
+                    const __half2 h2 = __floats2half2_rn(y0 - r1.x, y1 - r1.y);
+                    t0[i] = *reinterpret_cast<const uint32_t *>(&h0);
+                    t1[i] = *reinterpret_cast<const uint32_t *>(&h1);
+                    t2[i] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                uint16_t *row = terms + (size_t)sl * 3 * p.t_stride + kb * 128 + lane * 4;
+                *reinterpret_cast<uint2 *>(row) = make_uint2(t0[0], t0[1]);
+                *reinterpret_cast<uint2 *>(row + p.t_stride) = make_uint2(t1[0], t1[1]);
+                *reinterpret_cast<uint2 *>(row + 2 * p.t_stride) = make_uint2(t2[0], t2[1]);
+                if (lane == 0) hfac[sl * ib + kb] = pow2f(-sh);
+            }
         }
-        uint16_t *row = terms + (size_t)sl * 3 * p.t_stride + kb * 128 + lane * 4;
-        *reinterpret_cast<uint2 *>(row) = make_uint2(t0[0], t0[1]);
-        *reinterpret_cast<uint2 *>(row + p.t_stride) = make_uint2(t1[0], t1[1]);
-        *reinterpret_cast<uint2 *>(row + 2 * p.t_stride) = make_uint2(t2[0], t2[1]);
-        if (lane == 0) hfac[sl * ib + kb] = pow2f(-sh);
     }
     named_barrier(1, kStepWarps * kWarp);
-
-    // down items: group gi -> warp gi % kStepWarps; per expert of the group,
-    // per output tile, accumulate over windows and pieces
+    STEP_T(9);  // h staged as terms
+    // down items, round robin over the warps: per expert of the item's group,
+    // per output tile of its chunk (two at a time, each as two MMA chains),
+    // the full K; the result goes straight to the down buffer
     float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);   // [U + 1][rows][nt_max * 8]
     float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 128;  // [16][8]
     const int yrow = p.nt_max * 8;
-    {
-        float acc[kStepMaxExpertsPerItem][kMaxNt][4];
-        for (int q = seq.n_router + seq.n_gu; q < seq.total && !*abort; ++q) {
-            const Item it = item_at(p, seq, q);
-            if (it.a % kStepWarps != warp) continue;
-            const int s = q % p.ns;
-            if (!wait_item(sm.tag, full, s, q, p.ns)) {
-                if (lane == 0) {
-                    gave_up(p.counters, 3, q);
-                    *abort = 1;
-                }
-                break;
+    for (int q = seq.n_router + seq.n_gu; q < seq.total && !*abort; ++q) {
+        const Item it = item_at(p, seq, q);
+        if (it.b % kStepWarps != warp) continue;
+        const int s = q % p.ns;
+        if (!wait_item(sm.tag, full, s, q, p.ns)) {
+            if (lane == 0) {
+                gave_up(p.counters, 3, q);
+                *abort = 1;
             }
-            const bool shared = it.a == 0;
-            const int ne = group_size(p, U, it.a);
-            const int wp = shared ? p.dn_wp_s : p.dn_wp;
-            const int pieces = shared ? p.dn_pieces_s : p.dn_pieces;
-            const int Iu = shared ? p.Is : p.I;
-            const int ibu = Iu / 128;
-            const uint32_t sl = base + (uint32_t)s * kSlot;
-            if (it.p == 0) {
-#pragma unroll
-                for (int x = 0; x < kStepMaxExpertsPerItem; ++x)
-#pragma unroll
-                    for (int i = 0; i < kMaxNt; ++i) acc[x][i][0] = acc[x][i][1] = acc[x][i][2] = acc[x][i][3] = 0.f;
-            }
-#pragma unroll
-            for (int x = 0; x < kStepMaxExpertsPerItem; ++x) {
-                if (x >= ne) break;
-                const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
-                const int e = shared ? 0 : sm.list[li];
-                // A rows m = 3t + j: row t's slot for this expert, term j
-                int slot_lo = -1, slot_hi = -1;
-                {
-                    const int m0 = g, m1 = g + 8;
-                    const int tlo = m0 / 3, thi = m1 / 3;
-                    if (tlo < rows) {
-                        if (shared) slot_lo = rows * K + tlo;
-                        else for (int r = 0; r < K; ++r) if (sm.idx[tlo * K + r] == e) slot_lo = tlo * K + r;
-                    }
-                    if (thi < rows) {
-                        if (shared) slot_hi = rows * K + thi;
-                        else for (int r = 0; r < K; ++r) if (sm.idx[thi * K + r] == e) slot_hi = thi * K + r;
-                    }
+            break;
+        }
+        ITEM_T(q, 0);
+        const bool shared = it.a == 0;
+        const int ne = group_size(p, U, it.a);
+        const int Iu = shared ? p.Is : p.I;
+        const int ibu = Iu / 128;
+        const int tpi = shared ? p.dn_tpi_s : p.dn_tpi;
+        const int tfirst = it.p * tpi;                 // first tile of the chunk (local)
+        const int ntile = min(tpi, nt - tfirst);
+        const uint32_t box = 8u * (uint32_t)Iu;        // bytes of one expert's tile box
+        const uint32_t sl = base + (uint32_t)s * kSlot;
+        const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
+        for (int x = 0; x < ne; ++x) {
+            const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
+            const int e = shared ? 0 : sm.list[li];
+            const int de = shared ? 0 : 1 + li;
+            // A rows m = 3t + j: row t's slot for this expert, term j
+            int slot_lo = -1, slot_hi = -1;
+            {
+                const int tlo = g / 3, thi = (g + 8) / 3;
+                if (tlo < rows) {
+                    if (shared) slot_lo = rows * K + tlo;
+                    else for (int r = 0; r < K; ++r) if (sm.idx[tlo * K + r] == e) slot_lo = tlo * K + r;
                 }
-                const int jlo = g % 3, jhi = (g + 8) % 3;
-                const uint32_t alo = slot_lo >= 0 ? smem_u32(terms + ((size_t)slot_lo * 3 + jlo) * p.t_stride) : 0u;
-                const uint32_t ahi = slot_hi >= 0 ? smem_u32(terms + ((size_t)slot_hi * 3 + jhi) * p.t_stride) : 0u;
-                const float *s2 = (shared ? p.sscales : p.scales + (size_t)e * ((size_t)(2 * Iu / 128) * hb + (size_t)hb * ibu)) +
-                                  (size_t)(2 * Iu / 128) * hb;
-                const uint32_t ebase = sl + (uint32_t)(x * nt) * (uint32_t)wp * 1024u + (uint32_t)g * 128u;
-                const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
-                for (int w = 0; w < wp; ++w) {
-                    const int W = it.p * wp + w;
-                    if (W >= ibu) break;
+                if (thi < rows) {
+                    if (shared) slot_hi = rows * K + thi;
+                    else for (int r = 0; r < K; ++r) if (sm.idx[thi * K + r] == e) slot_hi = thi * K + r;
+                }
+            }
+            const int jlo = g % 3, jhi = (g + 8) % 3;
+            const uint32_t alo = slot_lo >= 0 ? smem_u32(terms + ((size_t)slot_lo * 3 + jlo) * p.t_stride) : 0u;
+            const uint32_t ahi = slot_hi >= 0 ? smem_u32(terms + ((size_t)slot_hi * 3 + jhi) * p.t_stride) : 0u;
+            const float *s2 = dsc + (size_t)de * 2 * ibm;
+            const uint32_t ebase = sl + (uint32_t)(x * tpi) * box + (uint32_t)g * 128u;
+            for (int i0 = 0; i0 < ntile; i0 += 2) {
+                const bool two = i0 + 1 < ntile;
+                float acc[2][4];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
+                for (int w = 0; w < ibu; ++w) {
                     uint4 al[4], ah[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const uint32_t off = (uint32_t)((W * 128 + 32 * qd + 8 * i) * 2);
+                        const uint32_t off = (uint32_t)((w * 128 + 32 * qd + 8 * i) * 2);
                         al[i] = slot_lo >= 0 ? lds128(alo + off) : make_uint4(0, 0, 0, 0);
                         ah[i] = slot_hi >= 0 ? lds128(ahi + off) : make_uint4(0, 0, 0, 0);
                     }
-                    const float flo = slot_lo >= 0 ? hfac[slot_lo * ib + W] : 0.f;
-                    const float fhi = slot_hi >= 0 ? hfac[slot_hi * ib + W] : 0.f;
+                    uint4 wb[2][2];
 #pragma unroll
-                    for (int i = 0; i < kMaxNt; ++i) {
-                        if (i >= nt) break;
-                        const uint32_t tb = ebase + (uint32_t)i * (uint32_t)wp * 1024u + (uint32_t)w * 1024u;
-                        const uint4 wb0 = lds128(tb + c0), wb1 = lds128(tb + c1);
-                        float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int k = 0; k < 2; ++k) {
+                        const bool on = k == 0 || two;
+                        const uint32_t tb = ebase + (uint32_t)(i0 + k) * box + (uint32_t)w * 1024u;
+                        wb[k][0] = on ? lds128(tb + c0) : make_uint4(0, 0, 0, 0);
+                        wb[k][1] = on ? lds128(tb + c1) : make_uint4(0, 0, 0, 0);
+                    }
+                    // every MMA step on its own accumulator, then a fixed-order add tree
+                    float d[2][8][4];
 #pragma unroll
-                        for (int st = 0; st < 8; ++st) {
-                            const uint32_t ww = word_of(st < 4 ? wb0 : wb1, st & 3);
-                            const uint32_t a0 = word_of(al[st >> 1], (st & 1) * 2);
-                            const uint32_t a2 = word_of(al[st >> 1], (st & 1) * 2 + 1);
-                            const uint32_t a1 = word_of(ah[st >> 1], (st & 1) * 2);
-                            const uint32_t a3 = word_of(ah[st >> 1], (st & 1) * 2 + 1);
-                            mma_f16_16816(d, a0, a1, a2, a3, e4m3x2_to_f16x2(ww), e4m3x2_to_f16x2(ww >> 16));
+                    for (int k = 0; k < 2; ++k)
+#pragma unroll
+                        for (int st = 0; st < 8; ++st) d[k][st][0] = d[k][st][1] = d[k][st][2] = d[k][st][3] = 0.f;
+#pragma unroll
+                    for (int st = 0; st < 8; ++st) {
+                        const uint32_t a0 = word_of(al[st >> 1], (st & 1) * 2);
+                        const uint32_t a2 = word_of(al[st >> 1], (st & 1) * 2 + 1);
+                        const uint32_t a1 = word_of(ah[st >> 1], (st & 1) * 2);
+                        const uint32_t a3 = word_of(ah[st >> 1], (st & 1) * 2 + 1);
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            const uint32_t ww = word_of(wb[k][st >> 2], st & 3);
+                            mma_f16_16816(d[k][st], a0, a1, a2, a3, e4m3x2_to_f16x2(ww), e4m3x2_to_f16x2(ww >> 16));
                         }
-                        const int nrow = (tile0 + i) * 8;
-                        const float sw = __ldg(s2 + (size_t)(nrow / 128) * ibu + W);
-                        acc[x][i][0] = fmaf(sw * flo, d[0], acc[x][i][0]);
-                        acc[x][i][1] = fmaf(sw * flo, d[1], acc[x][i][1]);
-                        acc[x][i][2] = fmaf(sw * fhi, d[2], acc[x][i][2]);
-                        acc[x][i][3] = fmaf(sw * fhi, d[3], acc[x][i][3]);
+                    }
+                    const float flo = slot_lo >= 0 ? hfac[slot_lo * ib + w] : 0.f;
+                    const float fhi = slot_hi >= 0 ? hfac[slot_hi * ib + w] : 0.f;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        float sum[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            sum[r] = ((d[k][0][r] + d[k][1][r]) + (d[k][2][r] + d[k][3][r])) +
+                                     ((d[k][4][r] + d[k][5][r]) + (d[k][6][r] + d[k][7][r]));
+                        const int nrow = (tile0 + tfirst + i0 + k) * 8;
+                        const float sw = s2[(nrow / 128 - rb0) * ibm + w];
+                        acc[k][0] = fmaf(sw * flo, sum[0], acc[k][0]);
+                        acc[k][1] = fmaf(sw * flo, sum[1], acc[k][1]);
+                        acc[k][2] = fmaf(sw * fhi, sum[2], acc[k][2]);
+                        acc[k][3] = fmaf(sw * fhi, sum[3], acc[k][3]);
                     }
                 }
-                if (it.p == pieces - 1) {
-                    // y[t][n] = sum of row t's three term rows, into the down buffer
-                    const int de = shared ? 0 : 1 + li;
+                // y[t][n] = the sum of row t's three term rows, into the down buffer
 #pragma unroll
-                    for (int i = 0; i < kMaxNt; ++i) {
-                        if (i >= nt) break;
-                        scr[g * 8 + 2 * qd] = acc[x][i][0];
-                        scr[g * 8 + 2 * qd + 1] = acc[x][i][1];
-                        scr[(g + 8) * 8 + 2 * qd] = acc[x][i][2];
-                        scr[(g + 8) * 8 + 2 * qd + 1] = acc[x][i][3];
-                        __syncwarp();
-                        const int t = lane >> 3, n = lane & 7;
-                        if (t < rows) {
-                            const float y = (scr[(3 * t) * 8 + n] + scr[(3 * t + 1) * 8 + n]) + scr[(3 * t + 2) * 8 + n];
-                            ybuf[((size_t)de * rows + t) * yrow + i * 8 + n] = y;
-                        }
-                        __syncwarp();
+                for (int k = 0; k < 2; ++k) {
+                    if (k == 1 && !two) break;
+                    scr[g * 8 + 2 * qd] = acc[k][0];
+                    scr[g * 8 + 2 * qd + 1] = acc[k][1];
+                    scr[(g + 8) * 8 + 2 * qd] = acc[k][2];
+                    scr[(g + 8) * 8 + 2 * qd + 1] = acc[k][3];
+                    __syncwarp();
+                    const int t = lane >> 3, n = lane & 7;
+                    if (t < rows) {
+                        const float y = (scr[(3 * t) * 8 + n] + scr[(3 * t + 1) * 8 + n]) + scr[(3 * t + 2) * 8 + n];
+                        ybuf[((size_t)de * rows + t) * yrow + (tfirst + i0 + k) * 8 + n] = y;
                     }
+                    __syncwarp();
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
         }
+        ITEM_T(q, 1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
     }
     named_barrier(1, kStepWarps * kWarp);
     if (*abort) return;
 
+    STEP_T(10);  // down items done
     // blend: rank order, then the shared expert, then the residual; one rounding
     for (int u = threadIdx.x; u < rows * nt * 8; u += kStepWarps * kWarp) {
         const int t = u / (nt * 8), nn = u - t * (nt * 8);
@@ -1017,6 +1194,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         if (p.residual) acc += bf16_bits_to_f32(p.residual[o]);
         p.out[o] = f32_to_bf16_bits(acc);
     }
+    STEP_T(11);
 }
 
 // ------------------------------------------------------------ host side
@@ -1083,11 +1261,10 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     s.gu_pieces = pieces_for(H / 128, 8, &s.gu_wp);  // 8 + 8 rows x <= 1024 bytes
     const int n8 = H / 8;
     s.nt_max = (n8 + G - 1) / G;
-    const int max_wp_dn = std::max(1, kSlot / (s.nt_max * 1024));
-    s.dn_pieces = pieces_for(I / 128, max_wp_dn, &s.dn_wp);
-    s.dn_pieces_s = pieces_for(Is / 128, max_wp_dn, &s.dn_wp_s);
-    s.dn_epi = s.dn_pieces == 1 ? std::max(1, std::min(kStepMaxExpertsPerItem, kSlot / (s.nt_max * s.dn_wp * 1024)))
-                                : 1;
+    // down items: the full K of one or two output tiles per expert
+    s.dn_tpi = 2 * 8 * I <= kSlot ? 2 : 1;
+    s.dn_tpi_s = 2 * 8 * Is <= kSlot ? 2 : 1;
+    s.dn_epi = 1;  // one expert per down item: more items for the warps
     s.rr_per_item = std::max(1, kSlot / (2 * H));
     // shared memory, after the ring
     const int nslots = rows * (K + 1);
@@ -1103,6 +1280,13 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     const int umax = std::min(d.n_experts, rows * K);
     const uint32_t y = take((size_t)(umax + 1) * rows * s.nt_max * 8 * 4);
     const uint32_t scr = take((size_t)kStepWarps * 128 * 4);
+    const int64_t units_max = Is / 8 + (int64_t)umax * (I / 8);
+    s.max_units = (int)((units_max + G - 1) / G);
+    const uint32_t gsc = take((size_t)s.max_units * 2 * (H / 128) * 4);
+    const uint32_t dsc = take((size_t)(umax + 1) * 2 * (imax / 128) * 4);
+    // split mode (fewer local units than warps): per unit and piece, 32 lanes x 4 sums
+    const int split_units = std::min(s.max_units, kStepWarps - 1);
+    const uint32_t part = take((size_t)split_units * s.gu_pieces * kWarp * 4 * 4);
     const uint32_t smo = take(sizeof(StepSmall));
     const size_t tail = o;
     // ring slots: whatever is left, up to 16
@@ -1115,13 +1299,17 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     s.o_hfac = ring + hfac;
     s.o_y = ring + y;
     s.o_scr = ring + scr;
+    s.o_gsc = ring + gsc;
+    s.o_dsc = ring + dsc;
+    s.o_part = ring + part;
     s.o_sm = ring + smo;
     s.o_bar = (uint32_t)align_up(ring + tail, 8);
     s.smem = s.o_bar + 2 * 8 * s.ns + 1024;
     // the router items all sit in the ring before the first slot is reused
     const int rr_max = (d.n_experts + 1 + G - 1) / G;
     const int router_items = (rr_max + s.rr_per_item - 1) / s.rr_per_item;
-    s.ok = s.ns >= 2 && s.ns > router_items && s.nt_max <= kMaxNt && s.smem <= kSmemCap && 2 * H <= kSlot;
+    s.ok = s.ns >= 2 && s.ns > router_items && s.nt_max <= kMaxNt && s.smem <= kSmemCap && 2 * H <= kSlot &&
+           8 * I <= kSlot && 8 * Is <= kSlot;
     return s;
 }
 
@@ -1149,9 +1337,9 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
                                (uint32_t)sh.gu_wp) ||
         !make_map_rows_windows(&p.w13s, a.shared_w8, 2 * (uint64_t)Is, (uint64_t)H, 1, 0, (uint32_t)sh.gu_wp) ||
         !make_map_rows_windows(&p.w2, a.expert_w8 + (size_t)2 * I * H, (uint64_t)H, (uint64_t)I, (uint64_t)E,
-                               3 * (uint64_t)I * H, (uint32_t)sh.dn_wp) ||
+                               3 * (uint64_t)I * H, (uint32_t)(I / 128)) ||
         !make_map_rows_windows(&p.w2s, a.shared_w8 + (size_t)2 * Is * H, (uint64_t)H, (uint64_t)Is, 1, 0,
-                               (uint32_t)sh.dn_wp_s))
+                               (uint32_t)(Is / 128)))
         return cudaErrorInvalidValue;
     p.x = a.x;
     p.router_w = a.router_w;
@@ -1180,10 +1368,8 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.ns = sh.ns;
     p.gu_wp = sh.gu_wp;
     p.gu_pieces = sh.gu_pieces;
-    p.dn_wp = sh.dn_wp;
-    p.dn_pieces = sh.dn_pieces;
-    p.dn_wp_s = sh.dn_wp_s;
-    p.dn_pieces_s = sh.dn_pieces_s;
+    p.dn_tpi = sh.dn_tpi;
+    p.dn_tpi_s = sh.dn_tpi_s;
     p.dn_epi = sh.dn_epi;
     p.nt_max = sh.nt_max;
     p.rr_per_item = sh.rr_per_item;
@@ -1193,6 +1379,10 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.o_hfac = sh.o_hfac;
     p.o_y = sh.o_y;
     p.o_scr = sh.o_scr;
+    p.o_gsc = sh.o_gsc;
+    p.o_dsc = sh.o_dsc;
+    p.o_part = sh.o_part;
+    p.max_units = sh.max_units;
     p.o_sm = sh.o_sm;
     p.o_bar = sh.o_bar;
     p.x_stride = sh.x_stride;
@@ -1201,3 +1391,21 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
 }
 
 }  // namespace moe
+
+#ifdef MOE_STEP_TRACE
+extern "C" MOE_API int moe_debug_item_trace(void *host, void *stream)
+{
+    cudaError_t e = cudaMemcpyFromSymbolAsync(host, moe::g_item_trace, sizeof(moe::g_item_trace), 0,
+                                              cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? 0 : -4;
+}
+
+extern "C" MOE_API int moe_debug_step_trace(void *host, void *stream)
+{
+    cudaError_t e = cudaMemcpyFromSymbolAsync(host, moe::g_step_trace, sizeof(moe::g_step_trace), 0,
+                                              cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? 0 : -4;
+}
+#endif

@@ -104,9 +104,10 @@ cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s);
 // Shape of one decode-step launch (rows <= kStepMaxRows).
 struct StepShape {
     bool ok;
-    int grid, ns, gu_wp, gu_pieces, dn_wp, dn_pieces, dn_wp_s, dn_pieces_s, dn_epi, nt_max, rr_per_item;
+    int grid, ns, gu_wp, gu_pieces, dn_tpi, dn_tpi_s, dn_epi, nt_max, rr_per_item;
     int x_stride, t_stride;
-    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar;
+    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_part;
+    int max_units;
     size_t smem;
 };
 StepShape step_shape(const moe_dims &d, int rows, int sms);
