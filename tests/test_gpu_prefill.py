@@ -77,7 +77,10 @@ def test_qwen36_35b_auto_at_multi_row_decode_counts(rows):
     P.compare_output(case, out, idx)
 
 
-def test_qwen36_35b_prefill_4096_rows_sampled():
+def test_qwen36_35b_prefill_4096_rows_every_row():
+    """The 4096-token prefill workload (per-expert router bias: uneven loads,
+    the busiest expert over twenty 128-row tiles, every expert's last tile
+    ragged), every output element of every row against the oracle."""
     d = mi.QWEN36_35B_A3B
     rows = 4096
     case = P.build_case(d, rows, router_bias=True, all_experts=True)
@@ -85,12 +88,23 @@ def test_qwen36_35b_prefill_4096_rows_sampled():
     _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate,
                                           router_bias=case.layer.router_bias)
     P.check_routing(case, idx, w, gs, ow, ogs)
-    # loads are uneven (the router bias): the busiest expert gets many M tiles
     counts = np.bincount(idx.ravel(), minlength=d.n_experts)
-    assert counts.max() > 4 * counts.mean()
-    sample = np.random.default_rng(0).choice(rows, 48, replace=False)
-    sub = P.Case(d, case.layer, case.x[sample].copy(), case.logits[sample])
-    P.compare_output(sub, out[sample], idx[sample])
+    assert counts.max() > 16 * 128 and counts.max() > 4 * counts.mean()
+    assert np.count_nonzero(counts % 128) > 100          # ragged last tiles
+    P.compare_output(case, out, idx)
+
+
+@pytest.mark.parametrize("rows", [128, 512, 1024])
+def test_qwen36_35b_auto_every_row(rows):
+    """The 35B layer at 128, 512 and 1024 rows through AUTO (the narrow
+    grouped GEMMs there), every row against the oracle."""
+    d = mi.QWEN36_35B_A3B
+    assert moe.auto_path(d, rows) == moe.MOE_PATH_PREFILL_NARROW
+    case = P.build_case(d, rows, all_experts=True)
+    out, idx, w, gs = run(case, moe.MOE_PATH_AUTO)
+    _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
 
 
 def test_prefill_router_more_than_256_experts():
@@ -104,7 +118,7 @@ def test_prefill_router_more_than_256_experts():
     P.compare_output(case, out, idx)
 
 
-def test_qwen35_397b_prefill_sampled():
+def test_qwen35_397b_prefill_every_row():
     # 512 experts (two router passes), top-10, I = Is = 1024, uneven loads
     d = mi.QWEN35_397B_A17B
     rows = 96
@@ -113,9 +127,7 @@ def test_qwen35_397b_prefill_sampled():
     _, oidx, ow, ogs = oracle.router_topk(d, case.x, case.layer.router_w, case.layer.shared_gate,
                                           router_bias=case.layer.router_bias)
     P.check_routing(case, idx, w, gs, ow, ogs)
-    sample = np.random.default_rng(1).choice(rows, 16, replace=False)
-    sub = P.Case(d, case.layer, case.x[sample].copy(), case.logits[sample])
-    P.compare_output(sub, out[sample], idx[sample])
+    P.compare_output(case, out, idx)
 
 
 @pytest.mark.parametrize("dims,rows", [
