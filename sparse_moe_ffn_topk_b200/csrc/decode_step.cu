@@ -68,20 +68,40 @@ namespace {
 
 constexpr int kSlot = 16384;           // ring slot bytes
 constexpr int kMaxNt = 8;              // output 8-row tiles per CTA
+constexpr int kGuRows = 32;            // gate (and up) rows of one gate/up unit: M = 64 of the MMA
+constexpr uint32_t kGuWindow = 8192;   // one 128-byte K window of a unit's 64 rows
+// The gate/up MMAs are issued by lane 0 of warps kIssuer0 .. kIssuer0 +
+// kIssuers - 1 (an issuing thread is the bottleneck of MMAs this small, so
+// several take the items in turn); they spin while they wait, on SM
+// sub-partitions other than the producer's (warp % 4 == 0).
+constexpr int kIssuer0 = 5;
+constexpr int kIssuers = 3;
+constexpr int kEpiWaiter = 32;         // the epilogue's waiting thread (warp 1, lane 0)
 constexpr uint32_t kSmemCap = 232448;  // dynamic shared memory per block (B200 opt-in)
 
 // ------------------------------------------------------------ device helpers
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two)
+// Four e4m3 bytes -> two f16x2 registers (bytes 0,1 and bytes 2,3); exact,
+// every e4m3 value is an f16 value.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi)
 {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2; cvt.rn.f16x2.e4m3x2 %0, l; cvt.rn.f16x2.e4m3x2 %1, h; }"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
-__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi)
+// Two fp32 -> two e5m2 (round to nearest even, saturating), lo in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e5m2x2(float lo, float hi)
 {
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
+    uint16_t r;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 e5m2x2_to_f32x2(uint32_t two)
+{
+    uint32_t h;
+    asm("{ .reg .b16 l, u; mov.b32 {l, u}, %1; cvt.rn.f16x2.e5m2x2 %0, l; }" : "=r"(h) : "r"(two));
+    return __half22float2(*reinterpret_cast<__half2 *>(&h));
 }
 
 // D += A * B: m16n8k16, f16 operands, fp32 accumulator.
@@ -91,23 +111,26 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi)
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                               uint32_t b0, uint32_t b1)
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                            int c4, uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "l"(policy)
+        : "memory");
 }
 
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
@@ -173,6 +196,17 @@ __device__ __forceinline__ bool wait_item(const volatile int32_t *tag, uint64_t 
     ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
     __syncwarp();
     return ok;
+}
+
+// wait_item for one thread (the gate/up MMA issuer).
+__device__ __forceinline__ bool wait_item_lane(const volatile int32_t *tag, uint64_t *full, int s, int q, int ns)
+{
+    if (tag[s] != q) {
+        const uint64_t t0 = globaltimer_ns();
+        while (tag[s] != q)
+            if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return mbar_wait_spin(&full[s], (uint32_t)((q / ns) & 1), kWaitLimitNs);
 }
 
 // The router items' wait (their slots' first use): lane 0 for the warp.
@@ -248,6 +282,10 @@ __device__ unsigned long long g_item_trace[256 * 64 * 6];  // per CTA, item: lan
         if ((threadIdx.x & 31) == 0 && (q) < 64)                                                \
             g_item_trace[(blockIdx.x * 64 + (q)) * 6 + (which)] = globaltimer_ns();             \
     } while (0)
+#define ITEM_TL(q, which)                                                                       \
+    do {                                                                                        \
+        if ((q) < 64) g_item_trace[(blockIdx.x * 64 + (q)) * 6 + (which)] = globaltimer_ns();   \
+    } while (0)
 #define STEP_T(i)                                                                          \
     do {                                                                                   \
         if (threadIdx.x == 0) g_step_trace[blockIdx.x * 16 + (i)] = globaltimer_ns();      \
@@ -259,13 +297,47 @@ __device__ unsigned long long g_item_trace[256 * 64 * 6];  // per CTA, item: lan
 #define ITEM_T(q, which) \
     do {                 \
     } while (0)
+#define ITEM_TL(q, which) \
+    do {                  \
+    } while (0)
 #endif
+
+// One gate/up unit row's sums (this lane's tensor-memory lane of buffer
+// tb): per row t of x, the K windows in order, each window's three term
+// columns added first, times the window's weight block scale and the row's
+// x scale.  NB = the accumulator columns of a window.
+template <int NB>
+__device__ __forceinline__ void gu_row_sums(uint32_t tb, int hb, int rows, const float *srow, const float *xfac,
+                                            float (&acc)[kStepMaxRows])
+{
+    constexpr int kWpl = 32 / NB;                             // K windows per 32-column load
+    constexpr int kTmax = NB == 8 ? 2 : kStepMaxRows;         // rows whose terms fit in NB columns
+#pragma unroll
+    for (int t = 0; t < kStepMaxRows; ++t) acc[t] = 0.f;
+    for (int W0 = 0; W0 < hb; W0 += kWpl) {
+        float v[32];
+        tmem_ld_32x32(tb + (uint32_t)(W0 * NB), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int wi = 0; wi < kWpl; ++wi) {
+            const int W = W0 + wi;
+            if (W >= hb) break;
+            const float sw = srow[W];
+#pragma unroll
+            for (int t = 0; t < kTmax; ++t) {
+                if (t >= rows) break;
+                const float g = (v[wi * NB + 3 * t] + v[wi * NB + 3 * t + 1]) + v[wi * NB + 3 * t + 2];
+                acc[t] = fmaf(sw * xfac[t * hb + W], g, acc[t]);
+            }
+        }
+    }
+}
 
 // ------------------------------------------------------------ parameters
 
 struct StepParams {
-    CUtensorMap w13;   // routed W13: (128 B, 2I rows, H/128 windows, E), boxes {128, 8, gu_wp, 1}
-    CUtensorMap w13s;  // shared W13: (128 B, 2Is rows, H/128 windows, 1)
+    CUtensorMap w13;   // routed W13: (128 B, I rows, gate|up, H/128 windows, E), boxes {128, 32, 2, gu_wp, 1}
+    CUtensorMap w13s;  // shared W13: (128 B, Is rows, gate|up, H/128 windows, 1), the same boxes
     CUtensorMap w2;    // routed W2: (128 B, H rows, I/128 windows, E), boxes {128, 8, I/128, 1}
     CUtensorMap w2s;   // shared W2: (128 B, H rows, Is/128 windows, 1), boxes {128, 8, Is/128, 1}
     const uint16_t *x;
@@ -283,6 +355,7 @@ struct StepParams {
     float *gsig;
     float *logits;      // workspace [rows][ld]
     float *h;           // workspace [rows * (K + 1)][imax]
+    uint32_t *hmax;     // workspace [rows * (K + 1)][imax / 128]: largest |h| of each block (fp32 bits)
     int32_t *counters;  // workspace counters (grid barrier, exit, status)
     int rows, H, E, K, I, Is, ld, imax;
     int ns;              // ring slots
@@ -291,7 +364,12 @@ struct StepParams {
     int nt_max;          // output 8-row tiles per CTA, at most
     int rr_per_item;     // router rows per ring item
     // shared-memory offsets (from the 1024-aligned base)
-    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_part;
+    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_cand;
+    uint32_t o_xB;       // x as e5m2 terms: per K window a [nb rows][128 B] operand tile (128-byte swizzle)
+    int nb;              // gate/up MMA N: 3 terms per row, 8 or 16
+    int nbuf, tbuf;      // gate/up accumulator buffers in tensor memory, columns of each (H/128 * nb)
+    int tcols;           // tensor-memory columns allocated
+    int cand2;           // two-stage top-k: chunk candidates [rows][chunks][K] keys, then experts, at o_cand
     int max_units;       // gate/up units per CTA, at most (rows of the scale table)
     int x_stride;        // halves per x row in shared memory (f16 and bf16 copies)
     int t_stride;        // halves per h term row in shared memory
@@ -306,7 +384,9 @@ struct StepSmall {
     uint32_t mask[kMaxExperts / 32];
     int32_t list[kStepMaxRows * kMaxTopK];  // distinct routed experts, ascending
     int32_t tag[16];                        // ring slot -> the item last issued into it (-1: none)
-    int32_t unit_done[kStepWarps];          // split mode: pieces finished per local unit
+    float xch[32 * kStepMaxRows];           // gate/up epilogue: the up rows' sums per row of x
+    uint32_t tmem;                          // tensor-memory base of this CTA's accumulators
+    int32_t gu_stop;                        // gate/up epilogue: leave the unit loop (written by its waiter)
     double red[kStepWarps * kStepMaxRows];  // RMSNorm: per-warp sums of squares
     double inv[kStepMaxRows];               // RMSNorm: 1 / sqrt(mean square + eps) per row
     int32_t n_list;
@@ -348,7 +428,7 @@ __device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt)
     Seq s;
     const int nr = n_router_rows(p.E, G, c);
     s.n_router = (nr + p.rr_per_item - 1) / p.rr_per_item;
-    const int units = p.Is / 8 + U * (p.I / 8);
+    const int units = p.Is / kGuRows + U * (p.I / kGuRows);
     s.n_units_local = units > c ? (units - 1 - c) / G + 1 : 0;
     s.n_gu = s.n_units_local * p.gu_pieces;
     s.n_tc_s = nt > 0 ? (nt + p.dn_tpi_s - 1) / p.dn_tpi_s : 0;
@@ -399,17 +479,17 @@ __device__ __forceinline__ Item item_at(const StepParams &p, const Seq &s, int q
 // Gate/up unit u -> (shared?, expert, first gate row j).
 __device__ __forceinline__ void unit_of(const StepParams &p, const StepSmall &sm, int u, bool &shared, int &e, int &j)
 {
-    const int us = p.Is / 8;
+    const int us = p.Is / kGuRows;
     if (u < us) {
         shared = true;
         e = 0;
-        j = u * 8;
+        j = u * kGuRows;
     } else {
         shared = false;
-        const int per = p.I / 8;
+        const int per = p.I / kGuRows;
         const int ue = (u - us) / per;
         e = sm.list[ue];
-        j = (u - us - ue * per) * 8;
+        j = (u - us - ue * per) * kGuRows;
     }
 }
 
@@ -425,7 +505,7 @@ __device__ __forceinline__ int group_size(const StepParams &p, int U, int gi)
 __device__ __forceinline__ uint32_t item_bytes(const StepParams &p, const Item &it, int nr_total, int nt, int U)
 {
     if (it.kind == 0) return (uint32_t)min(p.rr_per_item, nr_total - it.a) * (uint32_t)p.H * 2u;
-    if (it.kind == 1) return (uint32_t)p.gu_wp * 2048u;
+    if (it.kind == 1) return (uint32_t)p.gu_wp * kGuWindow;  // a whole box, also past the last window (zeros)
     const int ne = group_size(p, U, it.a);
     const int tpi = it.a == 0 ? p.dn_tpi_s : p.dn_tpi;
     const int ntile = min(tpi, nt - it.p * tpi);
@@ -435,9 +515,9 @@ __device__ __forceinline__ uint32_t item_bytes(const StepParams &p, const Item &
 __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t slot, uint64_t *full,
                            int r0, int nr_total, int tile0, int nt, int U, uint64_t pol, int qdbg = 0)
 {
-    ITEM_T(qdbg, 3);
+    ITEM_TL(qdbg, 3);
     mbar_arrive_expect_tx(full, item_bytes(p, it, nr_total, nt, U));
-    ITEM_T(qdbg, 4);
+    ITEM_TL(qdbg, 4);
     if (it.kind == 0) {
         // router rows r0 + it.a ..; row E (the gate vector) comes from shared_gate
         const int n = min(p.rr_per_item, nr_total - it.a);
@@ -459,15 +539,13 @@ __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item 
         return;
     }
     if (it.kind == 1) {
+        // one box: per K window, the unit's 32 gate rows then its 32 up
+        // rows, a 64-row operand tile of the 128-byte swizzle layout
         bool shared;
         int e, j;
         unit_of(p, sm, it.a, shared, e, j);
-        const CUtensorMap *m = shared ? &p.w13s : &p.w13;
-        const int Iu = shared ? p.Is : p.I;
-        const int w0 = it.p * p.gu_wp;
-        tma_load_4d(slot, m, 0, j, w0, e, full, pol);
-        ITEM_T(qdbg, 5);
-        tma_load_4d(slot + (uint32_t)p.gu_wp * 1024u, m, 0, Iu + j, w0, e, full, pol);
+        tma_load_5d(slot, shared ? &p.w13s : &p.w13, 0, j, 0, it.p * p.gu_wp, e, full, pol);
+        ITEM_TL(qdbg, 5);
         return;
     }
     const int ne = group_size(p, U, it.a);
@@ -490,9 +568,15 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sbase = smem_raw + (base - raw);
+    // 16 bytes of shared memory at a shared-window address (an ordinary load:
+    // the compiler may schedule it, but not across the barrier waits)
+    auto lds128 = [=](uint32_t a) { return *reinterpret_cast<const uint4 *>(sbase + (a - base)); };
     StepSmall &sm = *reinterpret_cast<StepSmall *>(sbase + p.o_sm);
     uint64_t *full = reinterpret_cast<uint64_t *>(sbase + p.o_bar);
     uint64_t *empty = full + p.ns;
+    uint64_t *tfull = empty + p.ns;  // [2] a unit's gate/up MMAs done (tcgen05.commit)
+    uint64_t *tfree = tfull + 2;     // [2] its accumulators read (the 4 epilogue warps)
+    uint64_t *tdone = tfree + 2;     // every MMA of this CTA done
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
     const int rows = p.rows, H = p.H, E = p.E, K = p.K;
@@ -511,11 +595,22 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             mbar_init(&empty[s], 1);
             sm.tag[s] = -1;
         }
-        for (int u = 0; u < kStepWarps; ++u) sm.unit_done[u] = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], kIssuers);
+            mbar_init(&tfree[b], 4);
+        }
+        mbar_init(tdone, kIssuers);
         sm.abort = 0;
         fence_mbar_init();
     }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem, (uint32_t)p.tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
 
     STEP_T(0);
     // ---------------------------------------------------------------- P0
@@ -582,22 +677,47 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             }
         }
         named_barrier(1, kStepWarps * kWarp);
-        // x -> f16 * 2^shift per (row, 128 block)
-        uint16_t *xs = reinterpret_cast<uint16_t *>(sbase + p.o_uni);
+        // x -> three e5m2 terms per value, the B operand of the gate/up
+        // products: per (row, 128 block) a power of two puts the block's
+        // largest magnitude in [2^14, 2^15), and t1 = e5m2(x'),
+        // t2 = e5m2(x' - t1), t3 = e5m2(x' - t1 - t2) (differences exact in
+        // fp32) sum exactly to x' for every value within 2^23 of that
+        // maximum.  Term j of row t is operand row 3t + j; K window W is a
+        // [nb rows][128 B] tile with the 128-byte swizzle (16-byte chunk c of
+        // row n at chunk c ^ (n % 8) of the row).
+        unsigned char *xB = sbase + p.o_xB;
         float *xfac = reinterpret_cast<float *>(sbase + p.o_xfac);
         for (int u = warp; u < rows * hb; u += kStepWarps) {
             const int t = u / hb, kb = u - t * hb;
             const uint2 raw2 = *reinterpret_cast<const uint2 *>(xb + (size_t)t * p.x_stride + kb * 128 + lane * 4);
-            const float v0 = bf16_lo(raw2.x), v1 = bf16_hi(raw2.x), v2 = bf16_lo(raw2.y), v3 = bf16_hi(raw2.y);
-            const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
+            const float v[4] = {bf16_lo(raw2.x), bf16_hi(raw2.x), bf16_lo(raw2.y), bf16_hi(raw2.y)};
+            const float amax = warp_max(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
             const int sh = block_shift(amax);
             const float f = pow2f(sh);
-            uint2 o;
-            o.x = f32x2_to_f16x2(v0 * f, v1 * f);
-            o.y = f32x2_to_f16x2(v2 * f, v3 * f);
-            *reinterpret_cast<uint2 *>(xs + (size_t)t * p.x_stride + kb * 128 + lane * 4) = o;
+            uint32_t tw[3] = {0u, 0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float x0 = v[2 * i] * f, x1 = v[2 * i + 1] * f;
+                const uint32_t c1 = f32x2_to_e5m2x2(x0, x1);
+                const float2 d1 = e5m2x2_to_f32x2(c1);
+                const float y0 = x0 - d1.x, y1 = x1 - d1.y;
+                const uint32_t c2 = f32x2_to_e5m2x2(y0, y1);
+                const float2 d2 = e5m2x2_to_f32x2(c2);
+                const uint32_t c3 = f32x2_to_e5m2x2(y0 - d2.x, y1 - d2.y);
+                tw[0] |= c1 << (16 * i);
+                tw[1] |= c2 << (16 * i);
+                tw[2] |= c3 << (16 * i);
+            }
+#pragma unroll
+            for (int jt = 0; jt < 3; ++jt) {
+                const int n = 3 * t + jt;
+                const uint32_t off = (uint32_t)(kb * p.nb * 128 + (n >> 3) * 1024 + (n & 7) * 128) +
+                                     (uint32_t)((((lane >> 2) ^ (n & 7)) * 16) + (lane & 3) * 4);
+                *reinterpret_cast<uint32_t *>(xB + off) = tw[jt];
+            }
             if (lane == 0) xfac[t * hb + kb] = pow2f(-sh);
         }
+        fence_proxy_async_smem();  // the tensor cores read the terms through the async proxy
         STEP_T(2);  // x staged
         // router rows (router items 0 .. n_router-1 in slots 0 ..)
         for (int ri = 0; ri < s0.n_router; ++ri) {
@@ -643,6 +763,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 }
             }
         }
+        // the block maxima of h start at zero (P2 raises them after grid barrier 1)
+        if (c == 0)
+            for (int i = threadIdx.x; i < rows * (K + 1) * (p.imax / 128); i += kStepWarps * kWarp) p.hmax[i] = 0u;
         __threadfence();
         named_barrier(1, kStepWarps * kWarp);
         STEP_T(3);  // router rows done
@@ -665,9 +788,35 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         named_barrier(1, kStepWarps * kWarp);
         STEP_T(4);  // grid barrier 1 passed
         // ------------------------------------------------------------ P2
-        // top-k of every row, in every CTA
-        if (!*abort && warp < rows) {
-            if (warp == 0) STEP_T(12);
+        // top-k of every row, in every CTA: in two stages over all warps
+        // (the k best of each chunk of 32 experts, then of the chunks'
+        // candidates), or one warp per row
+        if (warp == 0) STEP_T(12);
+        const int nch = (E + kWarp - 1) / kWarp;
+        if (!*abort && p.cand2) {
+            uint32_t *ckey = reinterpret_cast<uint32_t *>(sbase + p.o_cand);
+            int32_t *cid = reinterpret_cast<int32_t *>(ckey + rows * nch * K);
+            for (int task = warp; task < rows * nch; task += kStepWarps) {
+                const int t = task / nch, ch = task - t * nch;
+                topk_chunk(p.logits + (size_t)t * p.ld, E, K, ch, ckey + task * K, cid + task * K);
+            }
+            named_barrier(1, kStepWarps * kWarp);
+            if (warp < rows) {
+                const int n = nch * K;
+                const uint32_t *rk = ckey + warp * n;
+                const int32_t *ri = cid + warp * n;
+                const float *lrow = p.logits + (size_t)warp * p.ld;
+                int32_t *oi = sm.idx + warp * K;
+                float *ow = sm.w + warp * K;
+                float *og = sm.gs + warp;
+                if (n <= kWarp) topk_merge<1>(rk, ri, n, lrow, E, K, oi, ow, og);
+                else if (n <= 2 * kWarp) topk_merge<2>(rk, ri, n, lrow, E, K, oi, ow, og);
+                else if (n <= 4 * kWarp) topk_merge<4>(rk, ri, n, lrow, E, K, oi, ow, og);
+                else if (n <= 8 * kWarp) topk_merge<8>(rk, ri, n, lrow, E, K, oi, ow, og);
+                else topk_merge<16>(rk, ri, n, lrow, E, K, oi, ow, og);
+            }
+            if (warp == 0) STEP_T(13);
+        } else if (!*abort && warp < rows) {
             const float *lrow = p.logits + (size_t)warp * p.ld;
             int32_t *oi = sm.idx + warp * K;
             float *ow = sm.w + warp * K;
@@ -681,8 +830,40 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             if (warp == 0) STEP_T(13);
         }
         named_barrier(1, kStepWarps * kWarp);
-        if (!*abort && warp == 0) {
-            // distinct routed experts, ascending, and each pair's place in the list
+        if (!*abort && warp == 0 && rows * K <= kWarp) {
+            // distinct routed experts, ascending, and each pair's place in the
+            // list: lane i holds pair i as (expert << 5 | i); a bitonic sort
+            // across the warp orders the pairs by expert, the first pair of
+            // each expert marks a list entry
+            const int n = rows * K;
+            uint32_t key = lane < n ? ((uint32_t)sm.idx[lane] << 5) | (uint32_t)lane : 0xFFFFFFFFu;
+#pragma unroll
+            for (int k2 = 2; k2 <= kWarp; k2 <<= 1) {
+#pragma unroll
+                for (int j = k2 >> 1; j > 0; j >>= 1) {
+                    const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, key, j);
+                    key = (((lane & j) == 0) == ((lane & k2) == 0)) ? min(key, o) : max(key, o);
+                }
+            }
+            const uint32_t prev = __shfl_up_sync(0xFFFFFFFFu, key, 1);
+            const bool valid = lane < n;
+            const bool first = valid && (lane == 0 || (prev >> 5) != (key >> 5));
+            const uint32_t firsts = __ballot_sync(0xFFFFFFFFu, first);
+            const int pos = __popc(firsts & (0xFFFFFFFFu >> (31 - lane))) - 1;
+            if (first) sm.list[pos] = (int32_t)(key >> 5);
+            if (valid) sm.loc[key & 31u] = pos;
+            if (lane == 0) sm.n_list = __popc(firsts);
+            __syncwarp();
+            STEP_T(14);
+            if (c == 0) {
+                for (int i = lane; i < rows * K; i += kWarp) {
+                    p.topk_idx[i] = sm.idx[i];
+                    p.topk_w[i] = sm.w[i];
+                }
+                if (lane < rows) p.gsig[lane] = sm.gs[lane];
+            }
+        } else if (!*abort && warp == 0) {
+            // the same for more pairs than lanes, through a bitmask of experts
             for (int i = lane; i < kMaxExperts / 32; i += kWarp) sm.mask[i] = 0u;
             __syncwarp();
             for (int i = lane; i < rows * K; i += kWarp) atomicOr(&sm.mask[sm.idx[i] >> 5], 1u << (sm.idx[i] & 31));
@@ -741,6 +922,16 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         // only after the barrier, so their slots cannot be waited for here).
         int q = lane;
         while (q < p0_count) q += kWarp;  // issued in P0
+        // first the items that take a slot for the first time: no lane waits,
+        // so none holds up the others' issue (lanes of a warp that spin in
+        // different places are scheduled one path at a time)
+        for (; q < min(p.ns, seq.total) && !*abort; q += kWarp) {
+            issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)q * kSlot, &full[q], r0, nr_total, tile0, nt, U,
+                       pol, q);
+            ((volatile int32_t *)sm.tag)[q] = q;
+            ITEM_TL(q, 2);
+        }
+        __syncwarp();
         for (int phase = 0; phase < 2; ++phase) {
             for (; q < seq.total && !*abort; q += kWarp) {
                 const int s = q % p.ns;
@@ -768,10 +959,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt,
                            U, pol, q);
                 ((volatile int32_t *)sm.tag)[s] = q;
-                ITEM_T(q, 2);
+                ITEM_TL(q, 2);
             }
             if (phase == 0) {
                 __syncwarp();
+                ITEM_T(63, 3);
                 named_barrier(2, kStepThreads);  // gate/up of this CTA done
                 named_barrier(2, kStepThreads);  // grid barrier 2 passed
             }
@@ -835,138 +1027,152 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         named_barrier(1, kStepWarps * kWarp);
     }
 
-    // gate/up items.  With at least as many local units as warps, unit l
-    // goes to warp l % kStepWarps, which takes its K pieces in order and keeps
-    // the sums in registers.  With fewer (split mode), the items go round
-    // robin over the warps; each piece's partial sums go to shared memory
-    // and the warp that finishes a unit's last piece adds the pieces in
-    // piece order and runs the unit's epilogue.
+    // gate/up on the tensor cores.  Three issuing threads take, per local unit, the MMAs
+    // of its items as their copies land: A = the unit's 32 gate and 32 up
+    // rows of one K window (e4m3), B = the x terms (e5m2), K = 32 an
+    // instruction, one fp32 accumulator of nb columns per K window (each
+    // window has its own block scales); it commits them to the slot's empty
+    // barrier, so the producer may refill the slot once they are done, and
+    // after the unit's last item to the unit's accumulator buffer.  Warps
+    // 0-3 then read the buffer (unit row m sits in tensor-memory lane
+    // m % 16 + 32 (m / 16)), add each row of x's three term columns, scale
+    // and add the K windows in order, and write h = silu(gate) * up.  With
+    // two buffers the next unit's MMAs run during an epilogue.
     {
-        const bool split = seq.n_units_local < kStepWarps;
-        float *part = reinterpret_cast<float *>(sbase + p.o_part);  // [unit][piece][32 lanes][4]
-        const int t0 = 2 * qd, t1 = 2 * qd + 1;
-        // acc: one piece's sums (from zero); tot: the pieces added in piece
-        // order, the same in both modes (a row's bits must not depend on the
-        // other rows of the call)
-        float acc[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int q = seq.n_router; q < seq.n_router + seq.n_gu && !*abort; ++q) {
-            const Item it = item_at(p, seq, q);
-            const int owner = split ? (q - seq.n_router) % kStepWarps : it.b % kStepWarps;
-            if (owner != warp) continue;
-            const int s = q % p.ns;
-            STEP_MARK(2, q);
-            if (!wait_item(sm.tag, full, s, q, p.ns)) {
-                if (lane == 0) {
-                    STEP_SNAP(s);
-                    gave_up(p.counters, 2, q);
-                    *abort = 1;
-                }
-                break;
-            }
-            STEP_MARK(3, q);
-            ITEM_T(q, 0);
-            if (threadIdx.x == 0 && q == seq.n_router) STEP_T(6);  // warp 0's first gate/up item landed
-            bool shared;
-            int e, j;
-            unit_of(p, sm, it.a, shared, e, j);
-            const float *sg_row = gsc + (size_t)it.b * 2 * hb;
-            const float *su_row = sg_row + hb;
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-            const uint32_t sl = base + (uint32_t)s * kSlot;
-            const uint32_t gate_base = sl + (uint32_t)g * 128u;
-            const uint32_t up_base = sl + (uint32_t)p.gu_wp * 1024u + (uint32_t)g * 128u;
-            const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
-            const bool xrow = g < rows;
-            const uint32_t xaddr = smem_u32(xs) + (uint32_t)(g * p.x_stride * 2);
-            // one window per iteration: 8 MMA steps on two accumulators
-            // (even and odd steps)
-            for (int w = 0; w < p.gu_wp; ++w) {
-                const int W = it.p * p.gu_wp + w;
-                if (W >= hb) break;
-                const uint32_t wo = (uint32_t)w * 1024u;
-                const uint4 ga0 = lds128(gate_base + wo + c0), ga1 = lds128(gate_base + wo + c1);
-                const uint4 ua0 = lds128(up_base + wo + c0), ua1 = lds128(up_base + wo + c1);
-                uint4 xb[4];
+        const uint32_t xb_u32 = base + p.o_xB;
+        if (warp >= kIssuer0 && warp < kIssuer0 + kIssuers) {
+            if (lane == 0) {
+                const int me = warp - kIssuer0;
+                const uint32_t idesc = idesc_e4m3_e5m2_f32(2 * kGuRows, p.nb);
+                for (int l = 0; l < seq.n_units_local && !*abort; ++l) {
+                    const int b = l % p.nbuf, kk = l / p.nbuf;
+                    if (kk >= 1 && !mbar_wait_spin(&tfree[b], (uint32_t)((kk - 1) & 1), kWaitLimitNs)) {
+                        gave_up(p.counters, 8, l);
+                        *abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t dbase = tmem + (uint32_t)(b * p.tbuf);
+                    bool ok = true;
+                    for (int pc = me; pc < p.gu_pieces; pc += kIssuers) {
+                        const int q = seq.n_router + l * p.gu_pieces + pc;
+                        const int s = q % p.ns;
+                        STEP_MARK(2, q);
+                        if (!wait_item_lane(sm.tag, full, s, q, p.ns)) {
+                            STEP_SNAP(s);
+                            gave_up(p.counters, 2, q);
+                            *abort = 1;
+                            ok = false;
+                            break;
+                        }
+                        ITEM_T(q, 0);
+                        if (q == seq.n_router) STEP_T(6);  // the first gate/up item landed
+                        tc_fence_after();
+                        const uint32_t sl = base + (uint32_t)s * kSlot;
+                        for (int wl = 0; wl < p.gu_wp; ++wl) {
+                            const int W = pc * p.gu_wp + wl;
+                            if (W >= hb) break;
+                            const uint32_t a0 = sl + (uint32_t)wl * kGuWindow;
+                            const uint32_t b0 = xb_u32 + (uint32_t)(W * p.nb * 128);
+                            const uint32_t d = dbase + (uint32_t)(W * p.nb);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    xb[i] = xrow ? lds128(xaddr + (uint32_t)((W * 128 + 32 * qd + 8 * i) * 2)) : make_uint4(0, 0, 0, 0);
-                float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int st = 0; st < 8; ++st) {
-                    const uint32_t gw = word_of(st < 4 ? ga0 : ga1, st & 3);
-                    const uint32_t uw = word_of(st < 4 ? ua0 : ua1, st & 3);
-                    const uint32_t b0 = word_of(xb[st >> 1], (st & 1) * 2);
-                    const uint32_t b1 = word_of(xb[st >> 1], (st & 1) * 2 + 1);
-                    mma_f16_16816(d[st & 1], e4m3x2_to_f16x2(gw), e4m3x2_to_f16x2(uw), e4m3x2_to_f16x2(gw >> 16),
-                                  e4m3x2_to_f16x2(uw >> 16), b0, b1);
+                            for (int k4 = 0; k4 < 4; ++k4)
+                                umma_f8f6f4(d, umma_desc_sw128(a0 + 32 * k4), umma_desc_sw128(b0 + 32 * k4), idesc,
+                                            k4 > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&empty[s]);
+                        ITEM_T(q, 1);
+                    }
+                    if (!ok) break;
+                    umma_commit(&tfull[b]);
                 }
-                const float sgw = sg_row[W], suw = su_row[W];
-                const float f0 = t0 < rows ? xfac[t0 * hb + W] : 0.f;
-                const float f1 = t1 < rows ? xfac[t1 * hb + W] : 0.f;
-                acc[0] = fmaf(sgw * f0, d[0][0] + d[1][0], acc[0]);
-                acc[1] = fmaf(sgw * f1, d[0][1] + d[1][1], acc[1]);
-                acc[2] = fmaf(suw * f0, d[0][2] + d[1][2], acc[2]);
-                acc[3] = fmaf(suw * f1, d[0][3] + d[1][3], acc[3]);
+                umma_commit(tdone);  // also with nothing issued: the barrier then completes at once
             }
-            STEP_MARK(4, q);
-            ITEM_T(q, 1);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-            STEP_MARK(5, q);
-            STEP_CONSUMED(q);
-            bool last = it.p == p.gu_pieces - 1;
-            if (!split || p.gu_pieces == 1) {
-                if (it.p == 0) tot[0] = tot[1] = tot[2] = tot[3] = 0.f;
+        } else if (warp < 4) {
+            const int m = lane + 16 * warp;  // the unit row of this lane (lanes 0-15)
+            const bool gate = warp < 2;
+            // one thread waits for each unit and tells the four warps through
+            // a flag only it writes, so that they leave the loop together
+            // (the loop holds named barriers)
+            for (int l = 0; l < seq.n_units_local; ++l) {
+                const int b = l % p.nbuf, kk = l / p.nbuf;
+                if (threadIdx.x == kEpiWaiter) {
+                    const bool ok = !*abort && mbar_wait_spin(&tfull[b], (uint32_t)(kk & 1), kWaitLimitNs);
+                    if (!ok) {
+                        if (!*abort) gave_up(p.counters, 9, l);
+                        *abort = 1;
+                    }
+                    sm.gu_stop = ok ? 0 : 1;
+                }
+                named_barrier(3, 4 * kWarp);
+                if (sm.gu_stop) break;
+                tc_fence_after();
+                bool shared;
+                int e, j;
+                unit_of(p, sm, c + l * G, shared, e, j);
+                const float *srow = gsc + (size_t)l * 2 * hb + (gate ? 0 : hb);
+                float acc[kStepMaxRows];
+                const uint32_t tb = tmem + (uint32_t)(b * p.tbuf) + ((uint32_t)(32 * warp) << 16);
+                if (p.nb == 8) gu_row_sums<8>(tb, hb, rows, srow, xfac, acc);
+                else gu_row_sums<16>(tb, hb, rows, srow, xfac, acc);
+                // the up rows' sums to the gate rows' lanes
+                if (!gate && lane < 16) {
 #pragma unroll
-                for (int r = 0; r < 4; ++r) tot[r] += acc[r];
-            } else {
-                // this piece's sums to shared memory; the last piece of the unit adds them in order
-                float *pp = part + (((size_t)it.b * p.gu_pieces + it.p) * kWarp + lane) * 4;
-                pp[0] = acc[0];
-                pp[1] = acc[1];
-                pp[2] = acc[2];
-                pp[3] = acc[3];
-                __threadfence_block();
-                __syncwarp();
-                int prev = 0;
-                if (lane == 0) prev = atomicAdd(&sm.unit_done[it.b], 1);
-                prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-                last = prev == p.gu_pieces - 1;
-                if (last) {
-                    __threadfence_block();
+                    for (int t = 0; t < kStepMaxRows; ++t) sm.xch[(m - kGuRows) * kStepMaxRows + t] = acc[t];
+                }
+                tc_fence_before();
+                named_barrier(3, 4 * kWarp);
+                if (gate) {
+                    // h = silu(gate) * up for the rows routed to this expert
+                    // (lanes 0-15), and the largest |h| of the warp's 16 into
+                    // the block maximum (one atomic a warp and row)
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) tot[r] = 0.f;
-                    for (int pc = 0; pc < p.gu_pieces; ++pc) {
-                        const float *src = part + (((size_t)it.b * p.gu_pieces + pc) * kWarp + lane) * 4;
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) tot[r] += ((volatile const float *)src)[r];
+                    for (int t = 0; t < kStepMaxRows; ++t) {
+                        if (t >= rows) continue;
+                        int slot = -1;
+                        if (shared) {
+                            slot = rows * K + t;
+                        } else {
+                            for (int r = 0; r < K; ++r)
+                                if (sm.idx[t * K + r] == e) slot = t * K + r;
+                        }
+                        if (slot < 0) continue;  // the same in every lane
+                        float hv = 0.f;
+                        if (lane < 16) {
+                            hv = siluf_(acc[t]) * sm.xch[m * kStepMaxRows + t];
+                            p.h[(size_t)slot * p.imax + j + m] = hv;
+                        }
+                        const float mx = warp_max(fabsf(hv));
+                        if (lane == 0)
+                            atomicMax(p.hmax + (size_t)slot * (p.imax / 128) + j / 128, __float_as_uint(mx));
                     }
                 }
+                named_barrier(3, 4 * kWarp);  // the exchange slots are free again
+                if (lane == 0) mbar_arrive(&tfree[b]);
             }
-            if (last) {
-                // h = silu(gate) * up for rows 2q, 2q+1 routed to this expert
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                    const int t = 2 * qd + k2;
-                    if (t >= rows) continue;
-                    int slot = -1;
-                    if (shared) {
-                        slot = rows * K + t;
-                    } else {
-                        for (int r = 0; r < K; ++r)
-                            if (sm.idx[t * K + r] == e) slot = t * K + r;
-                    }
-                    if (slot < 0) continue;
-                    const float gt = tot[k2], up = tot[2 + k2];
-                    p.h[(size_t)slot * p.imax + j + g] = siluf_(gt) * up;
-                }
+        }
+        // every MMA done and every accumulator read: the tensor memory goes
+        // back before anything below can leave early
+        tc_fence_before();
+        if (warp < 4 || (warp >= kIssuer0 && warp < kIssuer0 + kIssuers)) named_barrier(4, (4 + kIssuers) * kWarp);
+        if (warp == 0) {
+            tc_fence_after();
+            if (lane == 0 && !mbar_wait(tdone, 0, kWaitLimitNs)) {
+                gave_up(p.counters, 10, 0);
+                *abort = 1;
             }
+            __syncwarp();
+            tmem_dealloc(tmem, (uint32_t)p.tcols);
         }
     }
     STEP_MARK(6, 0);
     STEP_T(7);  // warp 0's gate/up items done
+    ITEM_T(55 + warp, 3);
     __threadfence();
+    ITEM_T(55 + warp, 4);
     named_barrier(2, kStepThreads);  // gate/up of this CTA done (producer included)
+    STEP_T(15);  // all gate/up items of this CTA done
     if (threadIdx.x == 0) {
         bool ok = !*abort;
         if (ok) {
@@ -996,26 +1202,29 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     if (*abort || nt == 0) return;
 
     // ---------------------------------------------------------------- P3
-    // h -> three f16 terms per value, scaled by a power of two per (slot, block)
+    // h -> three f16 terms per value, scaled by a power of two per (slot,
+    // block) from the block's largest |h| (gathered during P2)
     const int nslots = rows * (K + 1);
     const int ib = p.imax / 128;
     uint16_t *terms = xs;  // the x region is free now
     float *hfac = reinterpret_cast<float *>(sbase + p.o_hfac);
     {
         // every (slot, block) pair of h: one warp each, in batches of 8 per
-        // warp with all eight loads in flight before any is used
+        // warp with all loads in flight before any is used
         constexpr int kBatch = 8;
         const int n_items = nslots * ib;
         for (int u0 = warp; u0 < n_items; u0 += kStepWarps * kBatch) {
             float4 v[kBatch];
+            uint32_t mx[kBatch];
 #pragma unroll
             for (int k = 0; k < kBatch; ++k) {
                 const int u = u0 + k * kStepWarps;
                 const int sl = u / ib, kb = u - sl * ib;
                 const int Iu = sl >= rows * K ? p.Is : p.I;
-                v[k] = (u < n_items && kb * 128 < Iu)
-                           ? __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                const bool on = u < n_items && kb * 128 < Iu;
+                v[k] = on ? __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                mx[k] = on ? __ldcg(p.hmax + u) : 0u;
             }
 #pragma unroll
             for (int k = 0; k < kBatch; ++k) {
@@ -1023,9 +1232,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 const int sl = u / ib, kb = u - sl * ib;
                 const int Iu = sl >= rows * K ? p.Is : p.I;
                 if (u >= n_items || kb * 128 >= Iu) continue;
-                const float amax =
-                    warp_max(fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
-                const int sh = block_shift(amax);
+                const int sh = block_shift(__uint_as_float(mx[k]));
                 const float f = pow2f(sh);
                 const float a[4] = {v[k].x * f, v[k].y * f, v[k].z * f, v[k].w * f};
                 uint32_t t0[2], t1[2], t2[2];
@@ -1052,15 +1259,20 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     }
     named_barrier(1, kStepWarps * kWarp);
     STEP_T(9);  // h staged as terms
-    // down items, round robin over the warps: per expert of the item's group,
-    // per output tile of its chunk (two at a time, each as two MMA chains),
-    // the full K; the result goes straight to the down buffer
+    // down items, round robin over the warps (item b to warp b % 8): per
+    // expert of the item, per pair of output tiles, the full K.  A = the 16
+    // weight rows of the two tiles (rows g of the first tile in MMA rows 0-7,
+    // of the second in 8-15), B = the h terms, column 3t + j = term j of row t
+    // (two MMAs per step above 8 columns); each lane's four accumulator
+    // chains take every fourth MMA step of a window.
     float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);   // [U + 1][rows][nt_max * 8]
-    float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 128;  // [16][8]
+    float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 256;  // [16 rows][16 columns]
     const int yrow = p.nt_max * 8;
-    for (int q = seq.n_router + seq.n_gu; q < seq.total && !*abort; ++q) {
+    const int ncol = 3 * rows;
+    const int nblk = ncol > 8 ? 2 : 1;
+    for (int b = warp; b < seq.n_dn && !*abort; b += kStepWarps) {
+        const int q = seq.n_router + seq.n_gu + b;
         const Item it = item_at(p, seq, q);
-        if (it.b % kStepWarps != warp) continue;
         const int s = q % p.ns;
         if (!wait_item(sm.tag, full, s, q, p.ns)) {
             if (lane == 0) {
@@ -1084,96 +1296,104 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
             const int e = shared ? 0 : sm.list[li];
             const int de = shared ? 0 : 1 + li;
-            // A rows m = 3t + j: row t's slot for this expert, term j
-            int slot_lo = -1, slot_hi = -1;
-            {
-                const int tlo = g / 3, thi = (g + 8) / 3;
-                if (tlo < rows) {
-                    if (shared) slot_lo = rows * K + tlo;
-                    else for (int r = 0; r < K; ++r) if (sm.idx[tlo * K + r] == e) slot_lo = tlo * K + r;
-                }
-                if (thi < rows) {
-                    if (shared) slot_hi = rows * K + thi;
-                    else for (int r = 0; r < K; ++r) if (sm.idx[thi * K + r] == e) slot_hi = thi * K + r;
+            // slot of row t for this expert (-1: row t does not route to it)
+            auto slot_of = [&](int t) {
+                if (t >= rows) return -1;
+                if (shared) return rows * K + t;
+                int r_ = -1;
+                for (int r = 0; r < K; ++r)
+                    if (sm.idx[t * K + r] == e) r_ = t * K + r;
+                return r_;
+            };
+            // B column g of each column block, and the slots of the lane's D columns 2q, 2q+1
+            uint32_t baddr[2];
+            int bslot[2], dslot[2][2];
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const int cb = nb * 8 + g;
+                bslot[nb] = cb < ncol ? slot_of(cb / 3) : -1;
+                baddr[nb] = bslot[nb] >= 0 ? smem_u32(terms + ((size_t)bslot[nb] * 3 + cb % 3) * p.t_stride) : 0u;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int cd = nb * 8 + 2 * qd + cc;
+                    dslot[nb][cc] = cd < ncol ? slot_of(cd / 3) : -1;
                 }
             }
-            const int jlo = g % 3, jhi = (g + 8) % 3;
-            const uint32_t alo = slot_lo >= 0 ? smem_u32(terms + ((size_t)slot_lo * 3 + jlo) * p.t_stride) : 0u;
-            const uint32_t ahi = slot_hi >= 0 ? smem_u32(terms + ((size_t)slot_hi * 3 + jhi) * p.t_stride) : 0u;
             const float *s2 = dsc + (size_t)de * 2 * ibm;
             const uint32_t ebase = sl + (uint32_t)(x * tpi) * box + (uint32_t)g * 128u;
             for (int i0 = 0; i0 < ntile; i0 += 2) {
                 const bool two = i0 + 1 < ntile;
+                const int row0 = (tile0 + tfirst + i0) * 8, row1 = row0 + 8;
                 float acc[2][4];
 #pragma unroll
-                for (int k = 0; k < 2; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
+                for (int nb = 0; nb < 2; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
                 for (int w = 0; w < ibu; ++w) {
-                    uint4 al[4], ah[4];
+                    const uint32_t t0b = ebase + (uint32_t)i0 * box + (uint32_t)w * 1024u;
+                    const uint32_t t1b = t0b + box;
+                    const uint4 w0l = lds128(t0b + c0), w0h = lds128(t0b + c1);
+                    const uint4 w1l = two ? lds128(t1b + c0) : make_uint4(0, 0, 0, 0);
+                    const uint4 w1h = two ? lds128(t1b + c1) : make_uint4(0, 0, 0, 0);
+                    uint4 bv[2][4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t off = (uint32_t)((w * 128 + 32 * qd + 8 * i) * 2);
-                        al[i] = slot_lo >= 0 ? lds128(alo + off) : make_uint4(0, 0, 0, 0);
-                        ah[i] = slot_hi >= 0 ? lds128(ahi + off) : make_uint4(0, 0, 0, 0);
-                    }
-                    uint4 wb[2][2];
+                    for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const bool on = k == 0 || two;
-                        const uint32_t tb = ebase + (uint32_t)(i0 + k) * box + (uint32_t)w * 1024u;
-                        wb[k][0] = on ? lds128(tb + c0) : make_uint4(0, 0, 0, 0);
-                        wb[k][1] = on ? lds128(tb + c1) : make_uint4(0, 0, 0, 0);
-                    }
-                    // every MMA step on its own accumulator, then a fixed-order add tree
-                    float d[2][8][4];
+                        for (int i = 0; i < 4; ++i)
+                            bv[nb][i] = (nb < nblk && bslot[nb] >= 0)
+                                            ? lds128(baddr[nb] + (uint32_t)((w * 128 + 32 * qd + 8 * i) * 2))
+                                            : make_uint4(0, 0, 0, 0);
+                    float d[2][4][4];
 #pragma unroll
-                    for (int k = 0; k < 2; ++k)
+                    for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-                        for (int st = 0; st < 8; ++st) d[k][st][0] = d[k][st][1] = d[k][st][2] = d[k][st][3] = 0.f;
+                        for (int ch = 0; ch < 4; ++ch) d[nb][ch][0] = d[nb][ch][1] = d[nb][ch][2] = d[nb][ch][3] = 0.f;
 #pragma unroll
                     for (int st = 0; st < 8; ++st) {
-                        const uint32_t a0 = word_of(al[st >> 1], (st & 1) * 2);
-                        const uint32_t a2 = word_of(al[st >> 1], (st & 1) * 2 + 1);
-                        const uint32_t a1 = word_of(ah[st >> 1], (st & 1) * 2);
-                        const uint32_t a3 = word_of(ah[st >> 1], (st & 1) * 2 + 1);
+                        const uint32_t x0 = word_of(st < 4 ? w0l : w0h, st & 3);
+                        const uint32_t x1 = word_of(st < 4 ? w1l : w1h, st & 3);
+                        uint32_t a0, a1, a2, a3;
+                        e4m3x4_to_f16x2x2(x0, a0, a2);
+                        e4m3x4_to_f16x2x2(x1, a1, a3);
 #pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            const uint32_t ww = word_of(wb[k][st >> 2], st & 3);
-                            mma_f16_16816(d[k][st], a0, a1, a2, a3, e4m3x2_to_f16x2(ww), e4m3x2_to_f16x2(ww >> 16));
+                        for (int nb = 0; nb < 2; ++nb) {
+                            if (nb < nblk)
+                                mma_f16_16816(d[nb][st & 3], a0, a1, a2, a3, word_of(bv[nb][st >> 1], (st & 1) * 2),
+                                              word_of(bv[nb][st >> 1], (st & 1) * 2 + 1));
                         }
                     }
-                    const float flo = slot_lo >= 0 ? hfac[slot_lo * ib + w] : 0.f;
-                    const float fhi = slot_hi >= 0 ? hfac[slot_hi * ib + w] : 0.f;
+                    const float sw0 = s2[(row0 / 128 - rb0) * ibm + w];
+                    const float sw1 = two ? s2[(row1 / 128 - rb0) * ibm + w] : 0.f;
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
+                    for (int nb = 0; nb < 2; ++nb) {
+                        if (nb >= nblk) continue;
+                        const float f0 = dslot[nb][0] >= 0 ? hfac[dslot[nb][0] * ib + w] : 0.f;
+                        const float f1 = dslot[nb][1] >= 0 ? hfac[dslot[nb][1] * ib + w] : 0.f;
                         float sum[4];
 #pragma unroll
                         for (int r = 0; r < 4; ++r)
-                            sum[r] = ((d[k][0][r] + d[k][1][r]) + (d[k][2][r] + d[k][3][r])) +
-                                     ((d[k][4][r] + d[k][5][r]) + (d[k][6][r] + d[k][7][r]));
-                        const int nrow = (tile0 + tfirst + i0 + k) * 8;
-                        const float sw = s2[(nrow / 128 - rb0) * ibm + w];
-                        acc[k][0] = fmaf(sw * flo, sum[0], acc[k][0]);
-                        acc[k][1] = fmaf(sw * flo, sum[1], acc[k][1]);
-                        acc[k][2] = fmaf(sw * fhi, sum[2], acc[k][2]);
-                        acc[k][3] = fmaf(sw * fhi, sum[3], acc[k][3]);
+                            sum[r] = (d[nb][0][r] + d[nb][1][r]) + (d[nb][2][r] + d[nb][3][r]);
+                        acc[nb][0] = fmaf(sw0 * f0, sum[0], acc[nb][0]);
+                        acc[nb][1] = fmaf(sw0 * f1, sum[1], acc[nb][1]);
+                        acc[nb][2] = fmaf(sw1 * f0, sum[2], acc[nb][2]);
+                        acc[nb][3] = fmaf(sw1 * f1, sum[3], acc[nb][3]);
                     }
                 }
-                // y[t][n] = the sum of row t's three term rows, into the down buffer
+                // y[t][n] = (term 0 + term 1) + term 2 of row t, into the down buffer
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    if (k == 1 && !two) break;
-                    scr[g * 8 + 2 * qd] = acc[k][0];
-                    scr[g * 8 + 2 * qd + 1] = acc[k][1];
-                    scr[(g + 8) * 8 + 2 * qd] = acc[k][2];
-                    scr[(g + 8) * 8 + 2 * qd + 1] = acc[k][3];
-                    __syncwarp();
-                    const int t = lane >> 3, n = lane & 7;
-                    if (t < rows) {
-                        const float y = (scr[(3 * t) * 8 + n] + scr[(3 * t + 1) * 8 + n]) + scr[(3 * t + 2) * 8 + n];
-                        ybuf[((size_t)de * rows + t) * yrow + (tfirst + i0 + k) * 8 + n] = y;
-                    }
-                    __syncwarp();
+                for (int nb = 0; nb < 2; ++nb) {
+                    if (nb >= nblk) continue;
+                    scr[g * 16 + nb * 8 + 2 * qd] = acc[nb][0];
+                    scr[g * 16 + nb * 8 + 2 * qd + 1] = acc[nb][1];
+                    scr[(g + 8) * 16 + nb * 8 + 2 * qd] = acc[nb][2];
+                    scr[(g + 8) * 16 + nb * 8 + 2 * qd + 1] = acc[nb][3];
                 }
+                __syncwarp();
+                for (int u = lane; u < rows * 16; u += kWarp) {
+                    const int t = u >> 4, r = u & 15;
+                    if (r >= 8 && !two) continue;
+                    const float y = (scr[r * 16 + 3 * t] + scr[r * 16 + 3 * t + 1]) + scr[r * 16 + 3 * t + 2];
+                    ybuf[((size_t)de * rows + t) * yrow + (tfirst + i0 + (r >> 3)) * 8 + (r & 7)] = y;
+                }
+                __syncwarp();
             }
         }
         ITEM_T(q, 1);
@@ -1215,11 +1435,39 @@ bool configured_for(int dev)
     return true;
 }
 
+// W13 of one expert slab [gate rows | up rows][windows of 128 bytes] (inter
+// rows each) as a 5-D TMA map over (128 bytes, rows, gate|up, windows,
+// experts) with 128-byte-swizzled boxes {128, 32, 2, box_windows, 1}: a box
+// lands as [window][gate 32 rows, up 32 rows][128 bytes].
+bool make_map_gate_up(CUtensorMap *m, const void *base, uint64_t inter, uint64_t kbytes, uint64_t experts,
+                      uint64_t expert_stride, uint32_t box_windows)
+{
+    using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeFn>(nullptr);
+        return reinterpret_cast<EncodeFn>(f);
+    }();
+    if (!fn) return false;
+    const cuuint64_t dims[5] = {128, inter, 2, kbytes / 128, experts};
+    const cuuint64_t strides[4] = {kbytes, inter * kbytes, 128, expert_stride ? expert_stride : 3 * inter * kbytes};
+    const cuuint32_t box[5] = {128, (cuuint32_t)kGuRows, 2, box_windows, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A byte tensor [outer][rows][windows of 128 bytes] as a 4-D TMA map over
 // (128 bytes, rows, windows, outer) with 128-byte-swizzled boxes
-// {128, 8, box_windows, 1}: a box lands as [window][8 rows][128 bytes].
+// {128, box_rows, box_windows, 1}: a box lands as [window][box_rows][128 bytes].
 bool make_map_rows_windows(CUtensorMap *m, const void *base, uint64_t rows, uint64_t kbytes, uint64_t outer,
-                           uint64_t outer_stride, uint32_t box_windows)
+                           uint64_t outer_stride, uint32_t box_windows, uint32_t box_rows = 8)
 {
     using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -1235,18 +1483,11 @@ bool make_map_rows_windows(CUtensorMap *m, const void *base, uint64_t rows, uint
     if (!fn) return false;
     const cuuint64_t dims[4] = {128, rows, kbytes / 128, outer};
     const cuuint64_t strides[3] = {kbytes, 128, outer_stride ? outer_stride : rows * kbytes};
-    const cuuint32_t box[4] = {128, 8, box_windows, 1};
+    const cuuint32_t box[4] = {128, box_rows, box_windows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int pieces_for(int windows, int max_wp, int *wp)
-{
-    const int n = (windows + max_wp - 1) / max_wp;
-    *wp = (windows + n - 1) / n;
-    return n;
 }
 
 }  // namespace
@@ -1258,7 +1499,20 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     const int imax = std::max(I, Is);
     const int G = std::max(1, sms);
     s.grid = G;
-    s.gu_pieces = pieces_for(H / 128, 8, &s.gu_wp);  // 8 + 8 rows x <= 1024 bytes
+    // gate/up items: two K windows of a unit's 64 rows (16 KB)
+    s.gu_wp = 2;
+    s.gu_pieces = (H / 128 + s.gu_wp - 1) / s.gu_wp;
+    // gate/up MMA N: three x terms per row, in 8 or 16 columns; one
+    // accumulator of nb columns per K window, two buffers when they fit in
+    // the 512 columns of tensor memory
+    s.nb = 3 * rows <= 8 ? 8 : 16;
+    s.tbuf = (H / 128) * s.nb;
+    s.nbuf = 2 * s.tbuf <= 512 ? 2 : 1;
+    {
+        const int need = (s.nbuf - 1) * s.tbuf + (s.tbuf + 31) / 32 * 32;  // loads take 32 columns at a time
+        s.tcols = 32;
+        while (s.tcols < need) s.tcols *= 2;
+    }
     const int n8 = H / 8;
     s.nt_max = (n8 + G - 1) / G;
     // down items: the full K of one or two output tiles per expert
@@ -1274,42 +1528,47 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     const size_t tbytes = (size_t)nslots * 3 * s.t_stride * 2;
     size_t o = 0;
     auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 16); return (uint32_t)at; };
-    const uint32_t uni = take(std::max(2 * xbytes, tbytes));  // [f16 x | bf16 x] in P1-P2, h terms in P3
+    const size_t xBbytes = (size_t)(H / 128) * s.nb * 128;
+    const uint32_t uni = take(std::max(xBbytes + xbytes, tbytes));  // [x terms | bf16 x] in P1-P2, h terms in P3
     const uint32_t xfac = take((size_t)rows * (H / 128) * 4);
     const uint32_t hfac = take((size_t)nslots * (imax / 128) * 4);
     const int umax = std::min(d.n_experts, rows * K);
     const uint32_t y = take((size_t)(umax + 1) * rows * s.nt_max * 8 * 4);
-    const uint32_t scr = take((size_t)kStepWarps * 128 * 4);
-    const int64_t units_max = Is / 8 + (int64_t)umax * (I / 8);
+    const uint32_t scr = take((size_t)kStepWarps * 256 * 4);
+    const int64_t units_max = Is / kGuRows + (int64_t)umax * (I / kGuRows);
     s.max_units = (int)((units_max + G - 1) / G);
     const uint32_t gsc = take((size_t)s.max_units * 2 * (H / 128) * 4);
     const uint32_t dsc = take((size_t)(umax + 1) * 2 * (imax / 128) * 4);
-    // split mode (fewer local units than warps): per unit and piece, 32 lanes x 4 sums
-    const int split_units = std::min(s.max_units, kStepWarps - 1);
-    const uint32_t part = take((size_t)split_units * s.gu_pieces * kWarp * 4 * 4);
+    // two-stage top-k: more than one chunk of 32 experts, at most 16
+    // candidates a lane in the second stage
+    const int nch = (d.n_experts + kWarp - 1) / kWarp;
+    s.cand2 = nch > 1 && nch * K <= 16 * kWarp;
+    const uint32_t cand = take(s.cand2 ? (size_t)rows * nch * K * 8 : 0);
     const uint32_t smo = take(sizeof(StepSmall));
     const size_t tail = o;
     // ring slots: whatever is left, up to 16
-    const size_t avail = (size_t)kSmemCap - 1024 - tail - 16 * 2 * 8;
+    const size_t avail = (size_t)kSmemCap - 1024 - tail - (16 * 2 + 5) * 8;
     s.ns = (int)std::min<size_t>(16, avail / kSlot);
     const uint32_t ring = (uint32_t)s.ns * kSlot;
-    s.o_uni = ring + uni;
-    s.o_xb = ring + uni + (uint32_t)xbytes;
+    s.o_uni = ring + uni;  // 1024-aligned: the ring is a multiple of 16 KB and uni comes first
+    s.o_xB = ring + uni;
+    s.o_xb = ring + uni + (uint32_t)xBbytes;
     s.o_xfac = ring + xfac;
     s.o_hfac = ring + hfac;
     s.o_y = ring + y;
     s.o_scr = ring + scr;
     s.o_gsc = ring + gsc;
     s.o_dsc = ring + dsc;
-    s.o_part = ring + part;
+    s.o_cand = ring + cand;
     s.o_sm = ring + smo;
     s.o_bar = (uint32_t)align_up(ring + tail, 8);
-    s.smem = s.o_bar + 2 * 8 * s.ns + 1024;
+    s.smem = s.o_bar + (2 * s.ns + 5) * 8 + 1024;
     // the router items all sit in the ring before the first slot is reused
     const int rr_max = (d.n_experts + 1 + G - 1) / G;
     const int router_items = (rr_max + s.rr_per_item - 1) / s.rr_per_item;
     s.ok = s.ns >= 2 && s.ns > router_items && s.nt_max <= kMaxNt && s.smem <= kSmemCap && 2 * H <= kSlot &&
-           8 * I <= kSlot && 8 * Is <= kSlot;
+           8 * I <= kSlot && 8 * Is <= kSlot && 3 * rows <= 16 && s.tbuf <= 512 && I % kGuRows == 0 &&
+           Is % kGuRows == 0;
     return s;
 }
 
@@ -1333,9 +1592,9 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     if (!sh.ok || a.rows < 1 || a.rows > kStepMaxRows) return cudaErrorInvalidConfiguration;
     const int H = d.hidden, I = d.inter, Is = d.shared_inter, E = d.n_experts;
     StepParams p;
-    if (!make_map_rows_windows(&p.w13, a.expert_w8, 2 * (uint64_t)I, (uint64_t)H, (uint64_t)E, 3 * (uint64_t)I * H,
-                               (uint32_t)sh.gu_wp) ||
-        !make_map_rows_windows(&p.w13s, a.shared_w8, 2 * (uint64_t)Is, (uint64_t)H, 1, 0, (uint32_t)sh.gu_wp) ||
+    if (!make_map_gate_up(&p.w13, a.expert_w8, (uint64_t)I, (uint64_t)H, (uint64_t)E, 3 * (uint64_t)I * H,
+                          (uint32_t)sh.gu_wp) ||
+        !make_map_gate_up(&p.w13s, a.shared_w8, (uint64_t)Is, (uint64_t)H, 1, 0, (uint32_t)sh.gu_wp) ||
         !make_map_rows_windows(&p.w2, a.expert_w8 + (size_t)2 * I * H, (uint64_t)H, (uint64_t)I, (uint64_t)E,
                                3 * (uint64_t)I * H, (uint32_t)(I / 128)) ||
         !make_map_rows_windows(&p.w2s, a.shared_w8 + (size_t)2 * Is * H, (uint64_t)H, (uint64_t)Is, 1, 0,
@@ -1356,6 +1615,7 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.gsig = a.gsig;
     p.logits = a.logits;
     p.h = a.h;
+    p.hmax = a.hmax;
     p.counters = a.counters;
     p.rows = a.rows;
     p.H = H;
@@ -1381,7 +1641,13 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.o_scr = sh.o_scr;
     p.o_gsc = sh.o_gsc;
     p.o_dsc = sh.o_dsc;
-    p.o_part = sh.o_part;
+    p.o_xB = sh.o_xB;
+    p.nb = sh.nb;
+    p.nbuf = sh.nbuf;
+    p.tbuf = sh.tbuf;
+    p.tcols = sh.tcols;
+    p.o_cand = sh.o_cand;
+    p.cand2 = sh.cand2 ? 1 : 0;
     p.max_units = sh.max_units;
     p.o_sm = sh.o_sm;
     p.o_bar = sh.o_bar;

@@ -33,7 +33,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Decode-path workspace, carved from the caller's buffer: the router's
 // logits and routing for all rows; h for one decode-step launch.
 struct DecodeLayout {
-    size_t counters, logits, topk_idx, topk_w, gsig, h, total;
+    size_t counters, logits, topk_idx, topk_w, gsig, h, hmax, total;
     int ld;
 };
 
@@ -52,6 +52,7 @@ inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
     L.topk_w = take(sizeof(float) * rows * K);
     L.gsig = take(sizeof(float) * rows);
     L.h = take(sizeof(float) * hrows * (K + 1) * imax);
+    L.hmax = take(sizeof(uint32_t) * hrows * (K + 1) * (imax / 128));
     L.total = o;
     return L;
 }
@@ -106,7 +107,9 @@ struct StepShape {
     bool ok;
     int grid, ns, gu_wp, gu_pieces, dn_tpi, dn_tpi_s, dn_epi, nt_max, rr_per_item;
     int x_stride, t_stride;
-    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_part;
+    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_cand, o_xB;
+    int nb, nbuf, tbuf, tcols;
+    bool cand2;
     int max_units;
     size_t smem;
 };
@@ -135,6 +138,7 @@ struct StepLaunch {
     float *logits;
     int logits_ld;
     float *h;
+    uint32_t *hmax;  // per (slot, 128 block) the largest |h| as fp32 bits
     int32_t *counters;
 };
 cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t s);

@@ -32,6 +32,16 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n)
            | ((uint32_t)(m >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor of kind::f8f6f4 with e4m3 A, e5m2 B (both K-major)
+// and an fp32 accumulator, for an M x N tile.
+__host__ __device__ constexpr uint32_t idesc_e4m3_e5m2_f32(int m, int n)
+{
+    return (1u << 4)                        // D format: f32
+           | (0u << 7) | (1u << 10)         // A format: e4m3, B format: e5m2
+           | ((uint32_t)(n >> 3) << 17)     // N / 8
+           | ((uint32_t)(m >> 4) << 24);    // M / 16
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B (K-major) and an fp32
 // accumulator, for an M x N tile.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n)

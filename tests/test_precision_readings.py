@@ -64,3 +64,32 @@ def test_single_fp8_activations_fail_and_hilo_split_passes():
     e_hilo = rel(layer(_hilo, _hilo))
     assert e_single > 5e-3          # misses the tolerance on its own
     assert e_hilo < 2e-3            # leaves room for the bf16 output rounding
+
+
+def _e5m2(a):
+    import ml_dtypes
+    return np.asarray(a, dtype=np.float32).astype(ml_dtypes.float8_e5m2).astype(np.float64)
+
+
+def test_bf16_splits_exactly_into_three_e5m2_terms():
+    """The decode step feeds x to the tensor cores as three e5m2 terms per value
+    after a power-of-two scale that puts the block's largest magnitude in
+    [2^14, 2^15): t1 = e5m2(x'), t2 = e5m2(x' - t1), t3 = e5m2(x' - t1 - t2),
+    each difference taken in fp32 as the kernel does.  Every bf16 value with
+    x' >= 2^-9 (within 2^23 of the block maximum) is then exactly t1 + t2 + t3;
+    below that the sum is within 2^-17 of x', i.e. under 2^-31 of the block
+    maximum.  Checked over every positive bf16 pattern in [2^-24, 2^15) (the
+    split is odd in x, and scaling by a power of two is exact)."""
+    bits = np.arange(0x3380, 0x4700, dtype=np.uint32)  # bf16 patterns from 2^-24 up to 2^15
+    xs = (bits << 16).view(np.float32).astype(np.float64)
+    xs = xs[xs < 2.0 ** 15]
+    t1 = _e5m2(xs)
+    r1 = (xs.astype(np.float32) - t1.astype(np.float32)).astype(np.float64)
+    t2 = _e5m2(r1)
+    r2 = (r1.astype(np.float32) - t2.astype(np.float32)).astype(np.float64)
+    t3 = _e5m2(r2)
+    err = np.abs(t1 + t2 + t3 - xs)
+    big = xs >= 2.0 ** -9
+    assert np.all(err[big] == 0.0)
+    assert np.all(err[~big] <= 2.0 ** -17)
+    assert np.any(err[~big] > 0.0)  # the bound is reached: the floor is real
