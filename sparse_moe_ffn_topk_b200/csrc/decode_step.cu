@@ -72,10 +72,10 @@ constexpr int kGuRows = 32;            // gate (and up) rows of one gate/up unit
 constexpr uint32_t kGuWindow = 8192;   // one 128-byte K window of a unit's 64 rows
 // The gate/up MMAs are issued by lane 0 of warps kIssuer0 .. kIssuer0 +
 // kIssuers - 1 (an issuing thread is the bottleneck of MMAs this small, so
-// several take the items in turn); they spin while they wait, on SM
-// sub-partitions other than the producer's (warp % 4 == 0).
-constexpr int kIssuer0 = 5;
-constexpr int kIssuers = 3;
+// several take the items in turn; not the epilogue warps, which the
+// issuers wait for when the accumulator buffers run out).
+constexpr int kIssuer0 = 4;
+constexpr int kIssuers = 4;
 constexpr int kEpiWaiter = 32;         // the epilogue's waiting thread (warp 1, lane 0)
 constexpr uint32_t kSmemCap = 232448;  // dynamic shared memory per block (B200 opt-in)
 
@@ -159,6 +159,10 @@ __device__ __forceinline__ int atomic_add_release_gpu(int32_t *p, int v)
     int old;
     asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
+}
+__device__ __forceinline__ void red_release_gpu(int32_t *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
 {
@@ -422,11 +426,10 @@ struct Seq {
 // Down items: per group of experts (the shared expert alone, then groups of
 // dn_epi routed experts of the list), per chunk of dn_tpi output tiles of
 // this CTA, the full K of the down rows (one TMA box per expert and tile).
-__device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt)
+__device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt, int nr)
 {
     const int G = gridDim.x, c = blockIdx.x;
     Seq s;
-    const int nr = n_router_rows(p.E, G, c);
     s.n_router = (nr + p.rr_per_item - 1) / p.rr_per_item;
     const int units = p.Is / kGuRows + U * (p.I / kGuRows);
     s.n_units_local = units > c ? (units - 1 - c) / G + 1 : 0;
@@ -512,11 +515,16 @@ __device__ __forceinline__ uint32_t item_bytes(const StepParams &p, const Item &
     return (uint32_t)ne * (uint32_t)ntile * 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);
 }
 
-__device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t slot, uint64_t *full,
-                           int r0, int nr_total, int tile0, int nt, int U, uint64_t pol, int qdbg = 0)
+// Issue item `it` into ring slot `slot`.  With go == false the same code
+// runs without arming the barrier or copying anything (it brings the
+// instructions into the cache ahead of their first real use).
+__device__ __noinline__ void issue_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t slot,
+                                        uint64_t *full, int r0, int nr_total, int tile0, int nt, int U, uint64_t pol,
+                                        int qdbg = 0, bool go = true)
 {
     ITEM_TL(qdbg, 3);
-    mbar_arrive_expect_tx(full, item_bytes(p, it, nr_total, nt, U));
+    const uint32_t bytes = item_bytes(p, it, nr_total, nt, U);
+    if (go) mbar_arrive_expect_tx(full, bytes);
     ITEM_TL(qdbg, 4);
     if (it.kind == 0) {
         // router rows r0 + it.a ..; row E (the gate vector) comes from shared_gate
@@ -524,13 +532,13 @@ __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item 
         const int first = r0 + it.a;
         const int nw = max(0, min(n, p.E - first));  // rows of router_w
         const uint32_t rowb = (uint32_t)p.H * 2u;
-        if (nw > 0) {
+        if (go && nw > 0) {
             asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                              slot),
                          "l"(p.router_w + (size_t)first * p.H), "r"(nw * rowb), "r"(smem_u32(full))
                          : "memory");
         }
-        if (nw < n) {
+        if (go && nw < n) {
             asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                              slot + nw * rowb),
                          "l"(p.shared_gate), "r"(rowb), "r"(smem_u32(full))
@@ -544,7 +552,7 @@ __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item 
         bool shared;
         int e, j;
         unit_of(p, sm, it.a, shared, e, j);
-        tma_load_5d(slot, shared ? &p.w13s : &p.w13, 0, j, 0, it.p * p.gu_wp, e, full, pol);
+        if (go) tma_load_5d(slot, shared ? &p.w13s : &p.w13, 0, j, 0, it.p * p.gu_wp, e, full, pol);
         ITEM_TL(qdbg, 5);
         return;
     }
@@ -555,8 +563,246 @@ __device__ void issue_item(const StepParams &p, const StepSmall &sm, const Item 
     const uint32_t box = 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);
     for (int x = 0; x < ne; ++x) {
         const int e = it.a == 0 ? 0 : sm.list[(it.a - 1) * p.dn_epi + x];
-        for (int i = 0; i < ntile; ++i)
+        for (int i = 0; i < ntile && go; ++i)
             tma_load_4d(slot + (uint32_t)(x * tpi + i) * box, m, 0, (tile0 + it.p * tpi + i) * 8, 0, e, full, pol);
+    }
+}
+
+// The gate/up item of local unit l, K piece pc into `slot` (one 5-D box);
+// with go == false nothing is armed or copied (instruction-cache warm-up).
+__device__ __noinline__ void issue_gu(const StepParams &p, const StepSmall &sm, int l, int pc, uint32_t slot,
+                                      uint64_t *full, uint64_t pol, bool go)
+{
+    bool shared;
+    int e, j;
+    unit_of(p, sm, blockIdx.x + l * gridDim.x, shared, e, j);
+    if (go) {
+        mbar_arrive_expect_tx(full, (uint32_t)p.gu_wp * kGuWindow);
+        tma_load_5d(slot, shared ? &p.w13s : &p.w13, 0, j, 0, pc * p.gu_wp, e, full, pol);
+    }
+}
+
+// The down item's expert: wait until all its gate/up units are counted
+// (every lane polls with acquire semantics, bounded), then its slots of h ->
+// three f16 terms per value, scaled by a power of two per (slot, 128 block)
+// from the block's largest |h| (gathered during P2), all loads of a slot in
+// flight before any is used.  False if the wait ran out.
+__device__ __forceinline__ bool stage_expert_h(const StepParams &p, const StepSmall &sm, const Item &it, int U,
+                                               uint16_t *terms, float *hfac, int ib)
+{
+    const int lane = threadIdx.x & 31;
+    const int rows = p.rows, K = p.K;
+    const bool shared = it.a == 0;
+    const int li = shared ? -1 : (it.a - 1) * p.dn_epi;  // one expert a down item
+    const int e = shared ? 0 : sm.list[li];
+    const int de = shared ? 0 : 1 + li;
+    const int need = (shared ? p.Is : p.I) / kGuRows;
+    const int32_t *ready = p.counters + kCtrStepReady + de;
+    if (ld_acquire_gpu(ready) < need) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(ready) < need)
+            if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    __syncwarp();
+    const int Iu = shared ? p.Is : p.I;
+    const int ibu = Iu / 128;
+    for (int t = 0; t < rows; ++t) {
+        int sl = -1;
+        if (shared) {
+            sl = rows * K + t;
+        } else {
+            for (int r = 0; r < K; ++r)
+                if (sm.idx[t * K + r] == e) sl = t * K + r;
+        }
+        if (sl < 0) continue;  // the same in every lane
+        for (int kb0 = 0; kb0 < ibu; kb0 += 8) {
+            float4 v[8];
+            uint32_t mx[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int kb = kb0 + k;
+                v[k] = kb < ibu ? __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                mx[k] = kb < ibu ? __ldcg(p.hmax + sl * ib + kb) : 0u;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int kb = kb0 + k;
+                if (kb >= ibu) break;
+                const int sh = block_shift(__uint_as_float(mx[k]));
+                const float f = pow2f(sh);
+                const float a[4] = {v[k].x * f, v[k].y * f, v[k].z * f, v[k].w * f};
+                uint32_t t0[2], t1[2], t2[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float x0 = a[2 * i], x1 = a[2 * i + 1];
+                    const __half2 h0 = __floats2half2_rn(x0, x1);
+                    const float2 r0 = __half22float2(h0);
+                    const float y0 = x0 - r0.x, y1 = x1 - r0.y;
+                    const __half2 h1 = __floats2half2_rn(y0, y1);
+                    const float2 r1 = __half22float2(h1);
+                    const __half2 h2 = __floats2half2_rn(y0 - r1.x, y1 - r1.y);
+                    t0[i] = *reinterpret_cast<const uint32_t *>(&h0);
+                    t1[i] = *reinterpret_cast<const uint32_t *>(&h1);
+                    t2[i] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                uint16_t *row = terms + (size_t)sl * 3 * p.t_stride + kb * 128 + lane * 4;
+                *reinterpret_cast<uint2 *>(row) = make_uint2(t0[0], t0[1]);
+                *reinterpret_cast<uint2 *>(row + p.t_stride) = make_uint2(t1[0], t1[1]);
+                *reinterpret_cast<uint2 *>(row + 2 * p.t_stride) = make_uint2(t2[0], t2[1]);
+                if (lane == 0) hfac[sl * ib + kb] = pow2f(-sh);
+            }
+        }
+    }
+    __syncwarp();
+    return true;
+}
+
+// The K windows of one pair of output tiles for a down item: per window 8
+// MMA steps (A = the tiles' weight rows, B = the h-term columns of NBLK
+// column blocks) on four accumulator chains, then the window's scales (the
+// weight block scale of each tile's rows, the h factor of each column's
+// slot).  acc[nb][0..1]: the first tile's row g at this lane's two columns,
+// acc[nb][2..3]: the second tile's.
+template <int NBLK>
+__device__ __forceinline__ void down_windows(unsigned char *sbase, uint32_t base, uint32_t t0base, uint32_t box,
+                                             bool two, int ibu, const uint32_t (&baddr)[2], const int (&bslot)[2],
+                                             const int (&dslot)[2][2], uint32_t c0, uint32_t c1, int qd,
+                                             const float *s2a, const float *s2b, const float *hfac, int ib,
+                                             float (&acc)[2][4])
+{
+    auto lds128 = [=](uint32_t a) { return *reinterpret_cast<const uint4 *>(sbase + (a - base)); };
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+#pragma unroll 2
+    for (int w = 0; w < ibu; ++w) {
+        const uint32_t t0b = t0base + (uint32_t)w * 1024u;
+        const uint32_t t1b = t0b + box;
+        const uint4 w0l = lds128(t0b + c0), w0h = lds128(t0b + c1);
+        const uint4 w1l = two ? lds128(t1b + c0) : make_uint4(0, 0, 0, 0);
+        const uint4 w1h = two ? lds128(t1b + c1) : make_uint4(0, 0, 0, 0);
+        uint4 bv[NBLK][4];
+#pragma unroll
+        for (int nb = 0; nb < NBLK; ++nb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                bv[nb][i] = bslot[nb] >= 0 ? lds128(baddr[nb] + (uint32_t)((w * 128 + 32 * qd + 8 * i) * 2))
+                                           : make_uint4(0, 0, 0, 0);
+        float d[NBLK][4][4];
+#pragma unroll
+        for (int nb = 0; nb < NBLK; ++nb)
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) d[nb][ch][0] = d[nb][ch][1] = d[nb][ch][2] = d[nb][ch][3] = 0.f;
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+            const uint32_t x0 = word_of(st < 4 ? w0l : w0h, st & 3);
+            const uint32_t x1 = word_of(st < 4 ? w1l : w1h, st & 3);
+            uint32_t a0, a1, a2, a3;
+            e4m3x4_to_f16x2x2(x0, a0, a2);
+            e4m3x4_to_f16x2x2(x1, a1, a3);
+#pragma unroll
+            for (int nb = 0; nb < NBLK; ++nb)
+                mma_f16_16816(d[nb][st & 3], a0, a1, a2, a3, word_of(bv[nb][st >> 1], (st & 1) * 2),
+                              word_of(bv[nb][st >> 1], (st & 1) * 2 + 1));
+        }
+        const float sw0 = s2a[w];
+        const float sw1 = two ? s2b[w] : 0.f;
+#pragma unroll
+        for (int nb = 0; nb < NBLK; ++nb) {
+            const float f0 = dslot[nb][0] >= 0 ? hfac[dslot[nb][0] * ib + w] : 0.f;
+            const float f1 = dslot[nb][1] >= 0 ? hfac[dslot[nb][1] * ib + w] : 0.f;
+            float sum[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sum[r] = (d[nb][0][r] + d[nb][1][r]) + (d[nb][2][r] + d[nb][3][r]);
+            acc[nb][0] = fmaf(sw0 * f0, sum[0], acc[nb][0]);
+            acc[nb][1] = fmaf(sw0 * f1, sum[1], acc[nb][1]);
+            acc[nb][2] = fmaf(sw1 * f0, sum[2], acc[nb][2]);
+            acc[nb][3] = fmaf(sw1 * f1, sum[3], acc[nb][3]);
+        }
+    }
+}
+
+// One down item: per expert of the item, per pair of output tiles, the full
+// K.  A = the 16 weight rows of the two tiles (rows g of the first tile in
+// MMA rows 0-7, of the second in 8-15), B = the h terms, column 3t + j = term
+// j of row t (two MMAs per step above 8 columns); each lane's four
+// accumulator chains take every fourth MMA step of a window.  The result
+// goes to the down buffer (with go == false it does not).
+__device__ __forceinline__ void down_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t sl,
+                                       unsigned char *sbase, uint32_t base, int U, int rows, int K, int nt, int tile0,
+                                       int rb0, int ibm, int ib, const uint16_t *terms, const float *hfac,
+                                       const float *dsc, float *ybuf, float *scr, bool go)
+{
+    const int lane = threadIdx.x & 31, g = lane >> 2, qd = lane & 3;
+    const int yrow = p.nt_max * 8;
+    const int ncol = 3 * rows;
+    const int nblk = ncol > 8 ? 2 : 1;
+    const bool shared = it.a == 0;
+    const int ne = group_size(p, U, it.a);
+    const int Iu = shared ? p.Is : p.I;
+    const int ibu = Iu / 128;
+    const int tpi = shared ? p.dn_tpi_s : p.dn_tpi;
+    const int tfirst = it.p * tpi;                 // first tile of the chunk (local)
+    const int ntile = min(tpi, nt - tfirst);
+    const uint32_t box = 8u * (uint32_t)Iu;        // bytes of one expert's tile box
+    const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
+    for (int x = 0; x < ne; ++x) {
+        const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
+        const int e = shared ? 0 : sm.list[li];
+        const int de = shared ? 0 : 1 + li;
+        // slot of row t for this expert (-1: row t does not route to it)
+        auto slot_of = [&](int t) {
+            if (t >= rows) return -1;
+            if (shared) return rows * K + t;
+            int r_ = -1;
+            for (int r = 0; r < K; ++r)
+                if (sm.idx[t * K + r] == e) r_ = t * K + r;
+            return r_;
+        };
+        // B column g of each column block, and the slots of the lane's D columns 2q, 2q+1
+        uint32_t baddr[2];
+        int bslot[2], dslot[2][2];
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+            const int cb = nb * 8 + g;
+            bslot[nb] = cb < ncol ? slot_of(cb / 3) : -1;
+            baddr[nb] = bslot[nb] >= 0 ? smem_u32(terms + ((size_t)bslot[nb] * 3 + cb % 3) * p.t_stride) : 0u;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int cd = nb * 8 + 2 * qd + cc;
+                dslot[nb][cc] = cd < ncol ? slot_of(cd / 3) : -1;
+            }
+        }
+        const float *s2 = dsc + (size_t)de * 2 * ibm;
+        const uint32_t ebase = sl + (uint32_t)(x * tpi) * box + (uint32_t)g * 128u;
+        for (int i0 = 0; i0 < ntile; i0 += 2) {
+            const bool two = i0 + 1 < ntile;
+            const int row0 = (tile0 + tfirst + i0) * 8, row1 = row0 + 8;
+            float acc[2][4];
+            if (nblk == 1)
+                down_windows<1>(sbase, base, ebase + (uint32_t)i0 * box, box, two, ibu, baddr, bslot, dslot, c0, c1,
+                                qd, s2 + (row0 / 128 - rb0) * ibm, s2 + (row1 / 128 - rb0) * ibm, hfac, ib, acc);
+            else
+                down_windows<2>(sbase, base, ebase + (uint32_t)i0 * box, box, two, ibu, baddr, bslot, dslot, c0, c1,
+                                qd, s2 + (row0 / 128 - rb0) * ibm, s2 + (row1 / 128 - rb0) * ibm, hfac, ib, acc);
+            // y[t][n] = (term 0 + term 1) + term 2 of row t, into the down buffer
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                if (nb >= nblk) continue;
+                scr[g * 16 + nb * 8 + 2 * qd] = acc[nb][0];
+                scr[g * 16 + nb * 8 + 2 * qd + 1] = acc[nb][1];
+                scr[(g + 8) * 16 + nb * 8 + 2 * qd] = acc[nb][2];
+                scr[(g + 8) * 16 + nb * 8 + 2 * qd + 1] = acc[nb][3];
+            }
+            __syncwarp();
+            for (int u = lane; u < rows * 16; u += kWarp) {
+                const int t = u >> 4, r = u & 15;
+                if (r >= 8 && !two) continue;
+                const float y = (scr[r * 16 + 3 * t] + scr[r * 16 + 3 * t + 1]) + scr[r * 16 + 3 * t + 2];
+                if (go) ybuf[((size_t)de * rows + t) * yrow + (tfirst + i0 + (r >> 3)) * 8 + (r & 7)] = y;
+            }
+            __syncwarp();
+        }
     }
 }
 
@@ -568,9 +814,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char *sbase = smem_raw + (base - raw);
-    // 16 bytes of shared memory at a shared-window address (an ordinary load:
-    // the compiler may schedule it, but not across the barrier waits)
-    auto lds128 = [=](uint32_t a) { return *reinterpret_cast<const uint4 *>(sbase + (a - base)); };
     StepSmall &sm = *reinterpret_cast<StepSmall *>(sbase + p.o_sm);
     uint64_t *full = reinterpret_cast<uint64_t *>(sbase + p.o_bar);
     uint64_t *empty = full + p.ns;
@@ -617,7 +860,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     // The producer issues the items that depend only on weights: router
     // rows, then the shared expert's gate/up units (the first local units).
     const uint64_t pol = policy_evict_first();
-    const Seq s0 = make_seq(p, 0, 0);  // U = 0: router and shared-expert items only (a prefix of the full sequence)
+    const Seq s0 = make_seq(p, 0, 0, nr_total);  // U = 0: router and shared-expert items only (a prefix of the full sequence)
     const int p0_count = min(s0.total, p.ns);
     if (producer) {
         if (lane == 0) {
@@ -635,6 +878,23 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         }
     }
 
+    // Each producer lane's first item after the plan, if a gate/up item in
+    // a fresh slot (its unit and piece do not depend on the routing), and
+    // the issue paths run once without issuing, so that the first wave after
+    // the plan neither divides nor waits for instruction fetches (the
+    // distinct-expert list is not built yet: no coordinate is used).
+    int fq = lane;
+    while (fq < p0_count) fq += kWarp;
+    const int fg = fq - s0.n_router;
+    const int fl = fg >= 0 ? fg / p.gu_pieces : 0, fpc = fg >= 0 ? fg - fl * p.gu_pieces : 0;
+    if (producer && lane == 0) {
+        const int Uw = min(rows * K, E);
+        const Seq sw = make_seq(p, Uw, nt, nr_total);
+        if (sw.n_gu > 0) issue_gu(p, sm, 0, 0, base, &full[0], pol, false);
+        if (sw.n_dn > 0)
+            issue_item(p, sm, item_at(p, sw, sw.n_router + sw.n_gu), base, &full[0], r0, nr_total, tile0, nt, Uw,
+                       pol, 0, false);
+    }
     pdl_wait();  // x and the workspace may be written by the previous kernel
     STEP_T(1);
 
@@ -763,10 +1023,14 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 }
             }
         }
-        // the block maxima of h start at zero (P2 raises them after grid barrier 1)
-        if (c == 0)
+        // the block maxima of h and the per-expert unit counts start at zero
+        // (P2 raises them after the grid barrier)
+        if (c == 0) {
             for (int i = threadIdx.x; i < rows * (K + 1) * (p.imax / 128); i += kStepWarps * kWarp) p.hmax[i] = 0u;
-        __threadfence();
+            for (int i = threadIdx.x; i <= rows * K; i += kStepWarps * kWarp) p.counters[kCtrStepReady + i] = 0;
+        }
+        // the logits and the zeros are ordered before thread 0's release
+        // through the CTA barrier (its fence is cumulative)
         named_barrier(1, kStepWarps * kWarp);
         STEP_T(3);  // router rows done
         if (threadIdx.x == 0) {
@@ -774,14 +1038,24 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             for (int ri = 0; ri < s0.n_router; ++ri) mbar_arrive(&empty[ri]);
             bool ok = !*abort;
             if (ok) {
+                __threadfence();
                 atomic_add_release_gpu(p.counters + kCtrStepBar, 1);
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_gpu(p.counters + kCtrStepBar) < G) {
                     if (globaltimer_ns() - t0 > kWaitLimitNs) {
                         gave_up(p.counters, 6, 0);
                         *abort = 1;
+                        ok = false;
                         break;
                     }
+                }
+            }
+            if (ok) {
+                // every CTA has passed the barrier once the exit count is
+                // full: the last one resets both for the next call
+                if (atomic_add_acq_rel_gpu(p.counters + kCtrStepExit, 1) == G - 1) {
+                    p.counters[kCtrStepBar] = 0;
+                    p.counters[kCtrStepExit] = 0;
                 }
             }
         }
@@ -911,20 +1185,24 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     __syncthreads();  // the plan is ready (all 288 threads)
     STEP_T(5);
     const int U = *abort ? 0 : sm.n_list;
-    const Seq seq = make_seq(p, U, nt);
+    const Seq seq = make_seq(p, U, nt, nr_total);
 
     if (producer) {
         // ---------------------------------------------------------- producer
         // The lanes issue in parallel, lane l the items l, l + 32, ... in
         // order; item q reuses ring slot q % ns once the slot's previous item
-        // (q - ns) was consumed.  Phase A, before grid barrier 2: items whose
-        // slot last held a router or gate/up item (down items are consumed
-        // only after the barrier, so their slots cannot be waited for here).
-        int q = lane;
-        while (q < p0_count) q += kWarp;  // issued in P0
+        // (q - ns) was consumed.
+        int q = fq;  // items before it were issued in P0
         // first the items that take a slot for the first time: no lane waits,
         // so none holds up the others' issue (lanes of a warp that spin in
-        // different places are scheduled one path at a time)
+        // different places are scheduled one path at a time); a lane's first
+        // one, when a gate/up item, straight from what P0 worked out
+        if (q < min(p.ns, seq.total) && fg >= 0 && fg < seq.n_gu && !*abort) {
+            issue_gu(p, sm, fl, fpc, base + (uint32_t)q * kSlot, &full[q], pol, true);
+            ((volatile int32_t *)sm.tag)[q] = q;
+            ITEM_TL(q, 2);
+            q += kWarp;
+        }
         for (; q < min(p.ns, seq.total) && !*abort; q += kWarp) {
             issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)q * kSlot, &full[q], r0, nr_total, tile0, nt, U,
                        pol, q);
@@ -932,41 +1210,32 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             ITEM_TL(q, 2);
         }
         __syncwarp();
-        for (int phase = 0; phase < 2; ++phase) {
-            for (; q < seq.total && !*abort; q += kWarp) {
-                const int s = q % p.ns;
-                if (q >= p.ns) {
-                    if (phase == 0 && item_at(p, seq, q - p.ns).kind == 2) break;
-                    // The slot's previous item (q - ns) belongs to another lane:
-                    // wait until it is issued (its tag), which proves that the
-                    // item before it in the slot was consumed; the parity wait
-                    // for its consumption is then exact (a lane running ahead
-                    // would otherwise see the phase two back completed).
-                    bool issued = ((volatile int32_t *)sm.tag)[s] == q - p.ns;
-                    if (!issued) {
-                        const uint64_t t0 = globaltimer_ns();
-                        while (!(issued = ((volatile int32_t *)sm.tag)[s] == q - p.ns))
-                            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-                    }
-                    if (!issued || !mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
-                        STEP_SNAP(s);
-                        gave_up(p.counters, 4 + phase, q);
-                        *abort = 1;
-                        break;
-                    }
-                    fence_proxy_async_smem();
+        for (; q < seq.total && !*abort; q += kWarp) {
+            const int s = q % p.ns;
+            if (q >= p.ns) {
+                // The slot's previous item (q - ns) belongs to another lane:
+                // wait until it is issued (its tag), which proves that the
+                // item before it in the slot was consumed; the parity wait
+                // for its consumption is then exact (a lane running ahead
+                // would otherwise see the phase two back completed).
+                bool issued = ((volatile int32_t *)sm.tag)[s] == q - p.ns;
+                if (!issued) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!(issued = ((volatile int32_t *)sm.tag)[s] == q - p.ns))
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
                 }
-                issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt,
-                           U, pol, q);
-                ((volatile int32_t *)sm.tag)[s] = q;
-                ITEM_TL(q, 2);
+                if (!issued || !mbar_wait(&empty[s], ((q / p.ns) - 1) & 1, kWaitLimitNs)) {
+                    STEP_SNAP(s);
+                    gave_up(p.counters, 4, q);
+                    *abort = 1;
+                    break;
+                }
+                fence_proxy_async_smem();
             }
-            if (phase == 0) {
-                __syncwarp();
-                ITEM_T(63, 3);
-                named_barrier(2, kStepThreads);  // gate/up of this CTA done
-                named_barrier(2, kStepThreads);  // grid barrier 2 passed
-            }
+            issue_item(p, sm, item_at(p, seq, q), base + (uint32_t)s * kSlot, &full[s], r0, nr_total, tile0, nt, U,
+                       pol, q);
+            ((volatile int32_t *)sm.tag)[s] = q;
+            ITEM_TL(q, 2);
         }
         // every issued copy lands before the CTA may leave: the last item
         // issued into each slot (all of them were consumed on the normal path)
@@ -981,7 +1250,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     }
 
     // ---------------------------------------------------------------- consumers
-    const int g = lane >> 2, qd = lane & 3;
     uint16_t *xs = reinterpret_cast<uint16_t *>(sbase + p.o_uni);
     const float *xfac = reinterpret_cast<const float *>(sbase + p.o_xfac);
 
@@ -1027,7 +1295,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         named_barrier(1, kStepWarps * kWarp);
     }
 
-    // gate/up on the tensor cores.  Three issuing threads take, per local unit, the MMAs
+    // gate/up on the tensor cores.  Four issuing threads take, per local unit, the MMAs
     // of its items as their copies land: A = the unit's 32 gate and 32 up
     // rows of one K window (e4m3), B = the x terms (e5m2), K = 32 an
     // instruction, one fp32 accumulator of nb columns per K window (each
@@ -1150,6 +1418,15 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 }
                 named_barrier(3, 4 * kWarp);  // the exchange slots are free again
                 if (lane == 0) mbar_arrive(&tfree[b]);
+                if (threadIdx.x == kEpiWaiter) {
+                    // this unit's h (both warps' writes, ordered by the CTA
+                    // barrier above) before its count for the expert: the down
+                    // items of every CTA wait for their expert's full count
+                    const int u = c + l * G, us = p.Is / kGuRows;
+                    const int de = u < us ? 0 : 1 + (u - us) / (p.I / kGuRows);
+                    __threadfence();
+                    red_release_gpu(p.counters + kCtrStepReady + de, 1);
+                }
             }
         }
         // every MMA done and every accumulator read: the tensor memory goes
@@ -1166,114 +1443,40 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             tmem_dealloc(tmem, (uint32_t)p.tcols);
         }
     }
+    // P3's buffers
+    const int ib = p.imax / 128;
+    uint16_t *terms = xs;  // the x region, once the gate/up MMAs are done
+    float *hfac = reinterpret_cast<float *>(sbase + p.o_hfac);
+    float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);   // [U + 1][rows][nt_max * 8]
+    float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 256;  // [16 rows][16 columns]
     STEP_MARK(6, 0);
     STEP_T(7);  // warp 0's gate/up items done
     ITEM_T(55 + warp, 3);
-    __threadfence();
-    ITEM_T(55 + warp, 4);
-    named_barrier(2, kStepThreads);  // gate/up of this CTA done (producer included)
-    STEP_T(15);  // all gate/up items of this CTA done
-    if (threadIdx.x == 0) {
-        bool ok = !*abort;
-        if (ok) {
-            atomic_add_release_gpu(p.counters + kCtrStepBar, 1);
-            const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_gpu(p.counters + kCtrStepBar) < 2 * G) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    gave_up(p.counters, 7, 0);
-                    *abort = 1;
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        if (ok) {
-            // every CTA has passed both barriers once the exit count is full:
-            // the last one resets the counters for the next call
-            if (atomic_add_acq_rel_gpu(p.counters + kCtrStepExit, 1) == G - 1) {
-                p.counters[kCtrStepBar] = 0;
-                p.counters[kCtrStepExit] = 0;
-            }
-        }
-    }
-    named_barrier(2, kStepThreads);
-    STEP_T(8);  // grid barrier 2 passed
-    pdl_trigger();
+    pdl_trigger();  // this CTA's weight reads are all issued: the next kernel may start
     if (*abort || nt == 0) return;
 
     // ---------------------------------------------------------------- P3
-    // h -> three f16 terms per value, scaled by a power of two per (slot,
-    // block) from the block's largest |h| (gathered during P2)
-    const int nslots = rows * (K + 1);
-    const int ib = p.imax / 128;
-    uint16_t *terms = xs;  // the x region is free now
-    float *hfac = reinterpret_cast<float *>(sbase + p.o_hfac);
-    {
-        // every (slot, block) pair of h: one warp each, in batches of 8 per
-        // warp with all loads in flight before any is used
-        constexpr int kBatch = 8;
-        const int n_items = nslots * ib;
-        for (int u0 = warp; u0 < n_items; u0 += kStepWarps * kBatch) {
-            float4 v[kBatch];
-            uint32_t mx[kBatch];
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-                const int u = u0 + k * kStepWarps;
-                const int sl = u / ib, kb = u - sl * ib;
-                const int Iu = sl >= rows * K ? p.Is : p.I;
-                const bool on = u < n_items && kb * 128 < Iu;
-                v[k] = on ? __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                mx[k] = on ? __ldcg(p.hmax + u) : 0u;
-            }
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-                const int u = u0 + k * kStepWarps;
-                const int sl = u / ib, kb = u - sl * ib;
-                const int Iu = sl >= rows * K ? p.Is : p.I;
-                if (u >= n_items || kb * 128 >= Iu) continue;
-                const int sh = block_shift(__uint_as_float(mx[k]));
-                const float f = pow2f(sh);
-                const float a[4] = {v[k].x * f, v[k].y * f, v[k].z * f, v[k].w * f};
-                uint32_t t0[2], t1[2], t2[2];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float x0 = a[2 * i], x1 = a[2 * i + 1];
-                    const __half2 h0 = __floats2half2_rn(x0, x1);
-                    const float2 r0 = __half22float2(h0);
-                    const float y0 = x0 - r0.x, y1 = x1 - r0.y;
-                    const __half2 h1 = __floats2half2_rn(y0, y1);
-                    const float2 r1 = __half22float2(h1);
-                    const __half2 h2 = __floats2half2_rn(y0 - r1.x, y1 - r1.y);
-                    t0[i] = *reinterpret_cast<const uint32_t *>(&h0);
-                    t1[i] = *reinterpret_cast<const uint32_t *>(&h1);
-                    t2[i] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                uint16_t *row = terms + (size_t)sl * 3 * p.t_stride + kb * 128 + lane * 4;
-                *reinterpret_cast<uint2 *>(row) = make_uint2(t0[0], t0[1]);
-                *reinterpret_cast<uint2 *>(row + p.t_stride) = make_uint2(t1[0], t1[1]);
-                *reinterpret_cast<uint2 *>(row + 2 * p.t_stride) = make_uint2(t2[0], t2[1]);
-                if (lane == 0) hfac[sl * ib + kb] = pow2f(-sh);
-            }
-        }
-    }
-    named_barrier(1, kStepWarps * kWarp);
-    STEP_T(9);  // h staged as terms
+    // no grid barrier: each down item waits until its expert's gate/up units
+    // (in whichever CTAs) are all counted, stages that expert's slots of h as
+    // terms, then runs
     // down items, round robin over the warps (item b to warp b % 8): per
     // expert of the item, per pair of output tiles, the full K.  A = the 16
     // weight rows of the two tiles (rows g of the first tile in MMA rows 0-7,
     // of the second in 8-15), B = the h terms, column 3t + j = term j of row t
     // (two MMAs per step above 8 columns); each lane's four accumulator
     // chains take every fourth MMA step of a window.
-    float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);   // [U + 1][rows][nt_max * 8]
-    float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 256;  // [16 rows][16 columns]
-    const int yrow = p.nt_max * 8;
-    const int ncol = 3 * rows;
-    const int nblk = ncol > 8 ? 2 : 1;
     for (int b = warp; b < seq.n_dn && !*abort; b += kStepWarps) {
         const int q = seq.n_router + seq.n_gu + b;
         const Item it = item_at(p, seq, q);
         const int s = q % p.ns;
+        if (!stage_expert_h(p, sm, it, U, terms, hfac, ib)) {
+            if (lane == 0) {
+                gave_up(p.counters, 11, q);
+                *abort = 1;
+            }
+            break;
+        }
+        if (warp == 0 && b == 0) STEP_T(9);  // warp 0's first expert staged
         if (!wait_item(sm.tag, full, s, q, p.ns)) {
             if (lane == 0) {
                 gave_up(p.counters, 3, q);
@@ -1282,120 +1485,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             break;
         }
         ITEM_T(q, 0);
-        const bool shared = it.a == 0;
-        const int ne = group_size(p, U, it.a);
-        const int Iu = shared ? p.Is : p.I;
-        const int ibu = Iu / 128;
-        const int tpi = shared ? p.dn_tpi_s : p.dn_tpi;
-        const int tfirst = it.p * tpi;                 // first tile of the chunk (local)
-        const int ntile = min(tpi, nt - tfirst);
-        const uint32_t box = 8u * (uint32_t)Iu;        // bytes of one expert's tile box
-        const uint32_t sl = base + (uint32_t)s * kSlot;
-        const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
-        for (int x = 0; x < ne; ++x) {
-            const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
-            const int e = shared ? 0 : sm.list[li];
-            const int de = shared ? 0 : 1 + li;
-            // slot of row t for this expert (-1: row t does not route to it)
-            auto slot_of = [&](int t) {
-                if (t >= rows) return -1;
-                if (shared) return rows * K + t;
-                int r_ = -1;
-                for (int r = 0; r < K; ++r)
-                    if (sm.idx[t * K + r] == e) r_ = t * K + r;
-                return r_;
-            };
-            // B column g of each column block, and the slots of the lane's D columns 2q, 2q+1
-            uint32_t baddr[2];
-            int bslot[2], dslot[2][2];
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                const int cb = nb * 8 + g;
-                bslot[nb] = cb < ncol ? slot_of(cb / 3) : -1;
-                baddr[nb] = bslot[nb] >= 0 ? smem_u32(terms + ((size_t)bslot[nb] * 3 + cb % 3) * p.t_stride) : 0u;
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int cd = nb * 8 + 2 * qd + cc;
-                    dslot[nb][cc] = cd < ncol ? slot_of(cd / 3) : -1;
-                }
-            }
-            const float *s2 = dsc + (size_t)de * 2 * ibm;
-            const uint32_t ebase = sl + (uint32_t)(x * tpi) * box + (uint32_t)g * 128u;
-            for (int i0 = 0; i0 < ntile; i0 += 2) {
-                const bool two = i0 + 1 < ntile;
-                const int row0 = (tile0 + tfirst + i0) * 8, row1 = row0 + 8;
-                float acc[2][4];
-#pragma unroll
-                for (int nb = 0; nb < 2; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-                for (int w = 0; w < ibu; ++w) {
-                    const uint32_t t0b = ebase + (uint32_t)i0 * box + (uint32_t)w * 1024u;
-                    const uint32_t t1b = t0b + box;
-                    const uint4 w0l = lds128(t0b + c0), w0h = lds128(t0b + c1);
-                    const uint4 w1l = two ? lds128(t1b + c0) : make_uint4(0, 0, 0, 0);
-                    const uint4 w1h = two ? lds128(t1b + c1) : make_uint4(0, 0, 0, 0);
-                    uint4 bv[2][4];
-#pragma unroll
-                    for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            bv[nb][i] = (nb < nblk && bslot[nb] >= 0)
-                                            ? lds128(baddr[nb] + (uint32_t)((w * 128 + 32 * qd + 8 * i) * 2))
-                                            : make_uint4(0, 0, 0, 0);
-                    float d[2][4][4];
-#pragma unroll
-                    for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) d[nb][ch][0] = d[nb][ch][1] = d[nb][ch][2] = d[nb][ch][3] = 0.f;
-#pragma unroll
-                    for (int st = 0; st < 8; ++st) {
-                        const uint32_t x0 = word_of(st < 4 ? w0l : w0h, st & 3);
-                        const uint32_t x1 = word_of(st < 4 ? w1l : w1h, st & 3);
-                        uint32_t a0, a1, a2, a3;
-                        e4m3x4_to_f16x2x2(x0, a0, a2);
-                        e4m3x4_to_f16x2x2(x1, a1, a3);
-#pragma unroll
-                        for (int nb = 0; nb < 2; ++nb) {
-                            if (nb < nblk)
-                                mma_f16_16816(d[nb][st & 3], a0, a1, a2, a3, word_of(bv[nb][st >> 1], (st & 1) * 2),
-                                              word_of(bv[nb][st >> 1], (st & 1) * 2 + 1));
-                        }
-                    }
-                    const float sw0 = s2[(row0 / 128 - rb0) * ibm + w];
-                    const float sw1 = two ? s2[(row1 / 128 - rb0) * ibm + w] : 0.f;
-#pragma unroll
-                    for (int nb = 0; nb < 2; ++nb) {
-                        if (nb >= nblk) continue;
-                        const float f0 = dslot[nb][0] >= 0 ? hfac[dslot[nb][0] * ib + w] : 0.f;
-                        const float f1 = dslot[nb][1] >= 0 ? hfac[dslot[nb][1] * ib + w] : 0.f;
-                        float sum[4];
-#pragma unroll
-                        for (int r = 0; r < 4; ++r)
-                            sum[r] = (d[nb][0][r] + d[nb][1][r]) + (d[nb][2][r] + d[nb][3][r]);
-                        acc[nb][0] = fmaf(sw0 * f0, sum[0], acc[nb][0]);
-                        acc[nb][1] = fmaf(sw0 * f1, sum[1], acc[nb][1]);
-                        acc[nb][2] = fmaf(sw1 * f0, sum[2], acc[nb][2]);
-                        acc[nb][3] = fmaf(sw1 * f1, sum[3], acc[nb][3]);
-                    }
-                }
-                // y[t][n] = (term 0 + term 1) + term 2 of row t, into the down buffer
-#pragma unroll
-                for (int nb = 0; nb < 2; ++nb) {
-                    if (nb >= nblk) continue;
-                    scr[g * 16 + nb * 8 + 2 * qd] = acc[nb][0];
-                    scr[g * 16 + nb * 8 + 2 * qd + 1] = acc[nb][1];
-                    scr[(g + 8) * 16 + nb * 8 + 2 * qd] = acc[nb][2];
-                    scr[(g + 8) * 16 + nb * 8 + 2 * qd + 1] = acc[nb][3];
-                }
-                __syncwarp();
-                for (int u = lane; u < rows * 16; u += kWarp) {
-                    const int t = u >> 4, r = u & 15;
-                    if (r >= 8 && !two) continue;
-                    const float y = (scr[r * 16 + 3 * t] + scr[r * 16 + 3 * t + 1]) + scr[r * 16 + 3 * t + 2];
-                    ybuf[((size_t)de * rows + t) * yrow + (tfirst + i0 + (r >> 3)) * 8 + (r & 7)] = y;
-                }
-                __syncwarp();
-            }
-        }
+        down_item(p, sm, it, base + (uint32_t)s * kSlot, sbase, base, U, rows, K, nt, tile0, rb0, ibm, ib, terms, hfac,
+                  dsc, ybuf, scr, true);
         ITEM_T(q, 1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -1405,6 +1496,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
 
     STEP_T(10);  // down items done
     // blend: rank order, then the shared expert, then the residual; one rounding
+    const int yrow = p.nt_max * 8;
     for (int u = threadIdx.x; u < rows * nt * 8; u += kStepWarps * kWarp) {
         const int t = u / (nt * 8), nn = u - t * (nt * 8);
         float acc = 0.f;

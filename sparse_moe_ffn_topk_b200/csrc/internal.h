@@ -17,7 +17,8 @@ constexpr int kCtrStatus = 1;           // device status word: 0, or a MOE_* err
 constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per token-group counters
 constexpr int kMaxRouterGroups = 1024;
 constexpr int kCtrStepBar = 8;          // decode step kernel: grid-barrier arrivals
-constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs past the last barrier
+constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs past the grid barrier
+constexpr int kCtrStepReady = 16;       // decode step kernel: per down expert (shared, then the routed list), units done
 constexpr int kCtrStepDiag = 2048;      // decode step kernel: per CTA, where a wait ran out (0: none)
 constexpr int kMaxBlendBlocks = 2048;   // H / 8 limit
 constexpr int kSmallRouterRows = 64;    // the grouped-GEMM path routes up to this many rows with the router kernel
