@@ -9,44 +9,46 @@
 // The "colibri #1992" PR page gives the decode GEMV's shape: a warp per
 // output row, 16 bytes a lane, the activation in shared memory.
 //
-// Here one CTA per SM runs the whole step with two grid-wide barriers:
+// Here one CTA per SM (eight consumer warps and a producer warp that keeps a
+// ring of 16 KB shared-memory slots filled by TMA) runs the whole step with
+// one grid-wide barrier:
 //
 //   P0  (before the programmatic-dependent-launch wait: weights only)
-//       the producer warp starts TMA copies of this CTA's router rows and of
-//       its shared-expert gate/up rows;
-//   P1  x -> shared memory as f16 with one power-of-two scale per
-//       (row, 128 block); the CTA's router rows (and the gate vector) against
-//       bf16 x in fp32 -> logits in the workspace;          grid barrier 1
-//   P2  every CTA takes the top-k of every row from the logits (no CTA
-//       waits for a designated one), builds the same list of distinct
-//       experts, and walks its share of gate/up units (8 gate + 8 up rows
-//       of one expert): h = silu(gate) * up in fp32 -> workspace; the
-//       producer keeps the ring full, the down rows of the active experts
-//       following the gate/up rows;                          grid barrier 2
-//   P3  h -> shared memory as three f16 terms per value (they sum exactly
-//       to the fp32 h) with one power-of-two scale per (slot, 128 block);
-//       the CTA's output rows: each expert's down product, then the blend
-//       in rank order (+ shared expert * sigmoid gate, + residual), one
-//       rounding to bf16.
+//       the producer starts the copies of this CTA's router rows and of its
+//       shared-expert gate/up rows;
+//   P1  x -> shared memory (bf16, and as three e5m2 terms per value with one
+//       power-of-two scale per (row, 128 block): the gate/up MMAs' B
+//       operand); the CTA's router rows (and the gate vector) against bf16 x
+//       in fp32 -> logits in the workspace;                  grid barrier 1
+//   P2  every CTA takes the top-k of every row from the logits (two stages
+//       over all warps; no CTA waits for a designated one), builds the same
+//       list of distinct experts, and runs its share of gate/up units (32
+//       gate + 32 up rows of one expert) on tcgen05: A = the e4m3 weight rows
+//       from the ring, B = the x terms, fp32 accumulators in tensor memory;
+//       the epilogue writes h = silu(gate) * up to the workspace as eight
+//       e5m2 terms per value (one power of two per 32 values, laid out as
+//       the down MMAs' B registers) and counts the unit for its expert;
+//   P3  no second grid barrier: each down item (one expert, this CTA's one
+//       or two 8-row output tiles, the full K) waits until its expert's
+//       units are all counted, bulk-copies the expert's h terms, and runs
+//       mma.sync m16n8k32 (A = the weight rows through ldmatrix, B = the h
+//       terms); then the blend in rank order (+ shared expert * sigmoid
+//       gate, + residual), one rounding to bf16.
 //
-// Tensor cores without narrowing the activations: the products run on
-// mma.m16n8k16 with f16 operands and fp32 accumulation.  Every e4m3 weight
-// is exactly an f16 value; a bf16 activation times a power of two is exactly
-// an f16 value (8 significant bits) unless it lies more than 2^31 below its
-// block's largest magnitude; an fp32 h is exactly the sum of three f16 terms
-// under the same condition (2^31 below the block maximum, else the error is
-// below 2^-39 of that maximum).  Products of f16 values are exact in fp32,
-// so the arithmetic is the pages': bf16 x times fp8 weights and f32 h times
-// fp8 weights, accumulated in fp32; each 128-wide K block's sum is then
-// scaled by its weight block scale and the activation's power of two.
+// The pages' arithmetic without narrowing the activations: a bf16 value
+// times a power of two that brings its block maximum into [2^14, 2^15) is
+// exactly the sum of three e5m2 terms unless it lies more than 2^23 below
+// that maximum; an fp32 h is exactly the sum of eight e5m2 terms within 2^7
+// of its block maximum and within 2^-31 of that maximum below.  Products of
+// e4m3 and e5m2 values are exact, the tensor cores accumulate in fp32, and
+// each block's sum is scaled by its weight block scale and the activation's
+// power of two: bf16 x times fp8 weights and f32 h times fp8 weights,
+// accumulated in fp32.
 //
-// Weight tiles arrive by 4-D TMA boxes [K windows of 128 bytes][8 rows][128
-// bytes] with the 128-byte swizzle, which makes the fragment reads below free
-// of bank conflicts: lane (g, q) reads row g's 16-byte chunks 2q and 2q+1 of
-// each window, and the swizzle spreads rows 2p and 2p+1 over all 8 chunks.
-// The K order inside a window is permuted the same way for the weights and
-// the activations (a dot product does not depend on the order of its terms):
-// in MMA step s of a window, lane quad q holds bytes 32q + 4s .. 32q + 4s + 3.
+// Weight tiles arrive by 5-D TMA boxes with the 128-byte swizzle (gate/up:
+// [K window][32 gate, 32 up rows][128 bytes]; down: [K window][tile][8
+// rows][128 bytes]); the same layout is the tcgen05 operand and the ldmatrix
+// source (16-byte chunk c of row r at c xor (r % 8)).
 //
 // Every wait is bounded (kWaitLimitNs): a wait that runs out records
 // MOE_ETIMEOUT in the workspace status word; the CTA waits (bounded) for its
@@ -81,15 +83,6 @@ constexpr uint32_t kSmemCap = 232448;  // dynamic shared memory per block (B200 
 
 // ------------------------------------------------------------ device helpers
 
-// Four e4m3 bytes -> two f16x2 registers (bytes 0,1 and bytes 2,3); exact,
-// every e4m3 value is an f16 value.
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi)
-{
-    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2; cvt.rn.f16x2.e4m3x2 %0, l; cvt.rn.f16x2.e4m3x2 %1, h; }"
-        : "=r"(lo), "=r"(hi)
-        : "r"(w));
-}
-
 // Two fp32 -> two e5m2 (round to nearest even, saturating), lo in the low byte.
 __device__ __forceinline__ uint32_t f32x2_to_e5m2x2(float lo, float hi)
 {
@@ -104,24 +97,6 @@ __device__ __forceinline__ float2 e5m2x2_to_f32x2(uint32_t two)
     return __half22float2(*reinterpret_cast<__half2 *>(&h));
 }
 
-// D += A * B: m16n8k16, f16 operands, fp32 accumulator.
-//   a0: row g, k 2q..2q+1     a1: row g+8, k 2q..     a2: row g, k 2q+8..   a3: row g+8, k 2q+8..
-//   b0: col g, k 2q..2q+1     b1: col g, k 2q+8..
-//   d0, d1: row g, cols 2q, 2q+1      d2, d3: row g+8, cols 2q, 2q+1
-__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                              uint32_t b0, uint32_t b1)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
-{
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
                                             int c4, uint64_t *bar, uint64_t policy)
 {
@@ -133,19 +108,8 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
-                                            uint64_t *bar, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
-        : "memory");
-}
-
-// The power of two that brings a block's largest magnitude into [2^14, 2^15)
-// (so that every value fits f16 with its bits intact), as its exponent,
-// clamped so that 2^s and 2^-s are normal floats.
+// The power of two that brings a block's largest magnitude into [2^14, 2^15),
+// as its exponent, clamped so that 2^s and 2^-s are normal floats.
 __device__ __forceinline__ int block_shift(float amax)
 {
     if (!(amax > 0.f) || !isfinite(amax)) return 0;
@@ -294,7 +258,14 @@ __device__ unsigned long long g_item_trace[256 * 64 * 6];  // per CTA, item: lan
     do {                                                                                   \
         if (threadIdx.x == 0) g_step_trace[blockIdx.x * 16 + (i)] = globaltimer_ns();      \
     } while (0)
+#define STEP_TL(i)                                                  \
+    do {                                                            \
+        g_step_trace[blockIdx.x * 16 + (i)] = globaltimer_ns();     \
+    } while (0)
 #else
+#define STEP_TL(i) \
+    do {           \
+    } while (0)
 #define STEP_T(i) \
     do {          \
     } while (0)
@@ -358,8 +329,8 @@ struct StepParams {
     float *topk_w;
     float *gsig;
     float *logits;      // workspace [rows][ld]
-    float *h;           // workspace [rows * (K + 1)][imax]
-    uint32_t *hmax;     // workspace [rows * (K + 1)][imax / 128]: largest |h| of each block (fp32 bits)
+    unsigned char *hterm;  // workspace [rows * (K + 1)][imax / 32][256]: h as e5m2 terms in the down MMAs' B layout
+    float *hsc;            // workspace [rows * (K + 1)][imax / 32]: the power of two of each chunk of terms
     int32_t *counters;  // workspace counters (grid barrier, exit, status)
     int rows, H, E, K, I, Is, ld, imax;
     int ns;              // ring slots
@@ -368,7 +339,8 @@ struct StepParams {
     int nt_max;          // output 8-row tiles per CTA, at most
     int rr_per_item;     // router rows per ring item
     // shared-memory offsets (from the 1024-aligned base)
-    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_cand;
+    uint32_t o_uni, o_xb, o_xfac, o_y, o_sm, o_bar, o_gsc, o_dsc, o_cand;
+    int rdy;             // ints between two experts' unit counters (each on its own 128-byte line when it fits)
     uint32_t o_xB;       // x as e5m2 terms: per K window a [nb rows][128 B] operand tile (128-byte swizzle)
     int nb;              // gate/up MMA N: 3 terms per row, 8 or 16
     int nbuf, tbuf;      // gate/up accumulator buffers in tensor memory, columns of each (H/128 * nb)
@@ -376,7 +348,6 @@ struct StepParams {
     int cand2;           // two-stage top-k: chunk candidates [rows][chunks][K] keys, then experts, at o_cand
     int max_units;       // gate/up units per CTA, at most (rows of the scale table)
     int x_stride;        // halves per x row in shared memory (f16 and bf16 copies)
-    int t_stride;        // halves per h term row in shared memory
 };
 
 // Small shared-memory block: routing and plan.
@@ -389,8 +360,10 @@ struct StepSmall {
     int32_t list[kStepMaxRows * kMaxTopK];  // distinct routed experts, ascending
     int32_t tag[16];                        // ring slot -> the item last issued into it (-1: none)
     float xch[32 * kStepMaxRows];           // gate/up epilogue: the up rows' sums per row of x
+    float hmx[2 * kStepMaxRows];            // gate/up epilogue: each gate warp's largest |h| per row of x
     uint32_t tmem;                          // tensor-memory base of this CTA's accumulators
     int32_t gu_stop;                        // gate/up epilogue: leave the unit loop (written by its waiter)
+    int32_t dn_next;                        // down phase: the next item to claim
     double red[kStepWarps * kStepMaxRows];  // RMSNorm: per-warp sums of squares
     double inv[kStepMaxRows];               // RMSNorm: 1 / sqrt(mean square + eps) per row
     int32_t n_list;
@@ -496,23 +469,14 @@ __device__ __forceinline__ void unit_of(const StepParams &p, const StepSmall &sm
     }
 }
 
-// Experts of down group gi: the shared expert alone (gi = 0), else list
-// entries [(gi-1)*epi, min(U, gi*epi)).
-__device__ __forceinline__ int group_size(const StepParams &p, int U, int gi)
-{
-    return gi == 0 ? 1 : min(p.dn_epi, U - (gi - 1) * p.dn_epi);
-}
-
 // ------------------------------------------------------------ producer
 
 __device__ __forceinline__ uint32_t item_bytes(const StepParams &p, const Item &it, int nr_total, int nt, int U)
 {
     if (it.kind == 0) return (uint32_t)min(p.rr_per_item, nr_total - it.a) * (uint32_t)p.H * 2u;
     if (it.kind == 1) return (uint32_t)p.gu_wp * kGuWindow;  // a whole box, also past the last window (zeros)
-    const int ne = group_size(p, U, it.a);
     const int tpi = it.a == 0 ? p.dn_tpi_s : p.dn_tpi;
-    const int ntile = min(tpi, nt - it.p * tpi);
-    return (uint32_t)ne * (uint32_t)ntile * 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);
+    return (uint32_t)tpi * 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);  // a whole box (tiles past H: zeros)
 }
 
 // Issue item `it` into ring slot `slot`.  With go == false the same code
@@ -556,16 +520,11 @@ __device__ __noinline__ void issue_item(const StepParams &p, const StepSmall &sm
         ITEM_TL(qdbg, 5);
         return;
     }
-    const int ne = group_size(p, U, it.a);
+    // one box: per K window, the item's output tiles (8 rows each) of its
+    // expert's W2, [window][tile][8 rows][128 B]
     const int tpi = it.a == 0 ? p.dn_tpi_s : p.dn_tpi;
-    const int ntile = min(tpi, nt - it.p * tpi);
-    const CUtensorMap *m = it.a == 0 ? &p.w2s : &p.w2;
-    const uint32_t box = 8u * (uint32_t)(it.a == 0 ? p.Is : p.I);
-    for (int x = 0; x < ne; ++x) {
-        const int e = it.a == 0 ? 0 : sm.list[(it.a - 1) * p.dn_epi + x];
-        for (int i = 0; i < ntile && go; ++i)
-            tma_load_4d(slot + (uint32_t)(x * tpi + i) * box, m, 0, (tile0 + it.p * tpi + i) * 8, 0, e, full, pol);
-    }
+    const int e = it.a == 0 ? 0 : sm.list[(it.a - 1) * p.dn_epi];
+    if (go) tma_load_5d(slot, it.a == 0 ? &p.w2s : &p.w2, 0, 0, tile0 + it.p * tpi, 0, e, full, pol);
 }
 
 // The gate/up item of local unit l, K piece pc into `slot` (one 5-D box);
@@ -582,13 +541,13 @@ __device__ __noinline__ void issue_gu(const StepParams &p, const StepSmall &sm, 
     }
 }
 
-// The down item's expert: wait until all its gate/up units are counted
-// (every lane polls with acquire semantics, bounded), then its slots of h ->
-// three f16 terms per value, scaled by a power of two per (slot, 128 block)
-// from the block's largest |h| (gathered during P2), all loads of a slot in
-// flight before any is used.  False if the wait ran out.
-__device__ __forceinline__ bool stage_expert_h(const StepParams &p, const StepSmall &sm, const Item &it, int U,
-                                               uint16_t *terms, float *hfac, int ib)
+// A down item's expert: wait until all of its gate/up units (in whichever
+// CTAs) are counted (lane 0 polls with acquire semantics, bounded; the warp
+// barrier then orders the lanes' reads of h after the counted writes).
+// sl[t] = the slot of h of row t of x routed to the expert (-1: not routed),
+// bit t of *routed set for those rows.  False if the wait ran out.
+__device__ __forceinline__ bool wait_expert(const StepParams &p, const StepSmall &sm, const Item &it,
+                                            int (&sl)[kStepMaxRows], uint32_t *routed)
 {
     const int lane = threadIdx.x & 31;
     const int rows = p.rows, K = p.K;
@@ -597,211 +556,224 @@ __device__ __forceinline__ bool stage_expert_h(const StepParams &p, const StepSm
     const int e = shared ? 0 : sm.list[li];
     const int de = shared ? 0 : 1 + li;
     const int need = (shared ? p.Is : p.I) / kGuRows;
-    const int32_t *ready = p.counters + kCtrStepReady + de;
-    if (ld_acquire_gpu(ready) < need) {
+    const int32_t *ready = p.counters + kCtrStepReady + de * p.rdy;
+    int ok = 1;
+    if (lane == 0 && ld_acquire_gpu(ready) < need) {
         const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(ready) < need)
-            if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    }
-    __syncwarp();
-    const int Iu = shared ? p.Is : p.I;
-    const int ibu = Iu / 128;
-    for (int t = 0; t < rows; ++t) {
-        int sl = -1;
-        if (shared) {
-            sl = rows * K + t;
-        } else {
-            for (int r = 0; r < K; ++r)
-                if (sm.idx[t * K + r] == e) sl = t * K + r;
-        }
-        if (sl < 0) continue;  // the same in every lane
-        for (int kb0 = 0; kb0 < ibu; kb0 += 8) {
-            float4 v[8];
-            uint32_t mx[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int kb = kb0 + k;
-                v[k] = kb < ibu ? __ldcg(reinterpret_cast<const float4 *>(p.h + (size_t)sl * p.imax + kb * 128) + lane)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                mx[k] = kb < ibu ? __ldcg(p.hmax + sl * ib + kb) : 0u;
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int kb = kb0 + k;
-                if (kb >= ibu) break;
-                const int sh = block_shift(__uint_as_float(mx[k]));
-                const float f = pow2f(sh);
-                const float a[4] = {v[k].x * f, v[k].y * f, v[k].z * f, v[k].w * f};
-                uint32_t t0[2], t1[2], t2[2];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float x0 = a[2 * i], x1 = a[2 * i + 1];
-                    const __half2 h0 = __floats2half2_rn(x0, x1);
-                    const float2 r0 = __half22float2(h0);
-                    const float y0 = x0 - r0.x, y1 = x1 - r0.y;
-                    const __half2 h1 = __floats2half2_rn(y0, y1);
-                    const float2 r1 = __half22float2(h1);
-                    const __half2 h2 = __floats2half2_rn(y0 - r1.x, y1 - r1.y);
-                    t0[i] = *reinterpret_cast<const uint32_t *>(&h0);
-                    t1[i] = *reinterpret_cast<const uint32_t *>(&h1);
-                    t2[i] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                uint16_t *row = terms + (size_t)sl * 3 * p.t_stride + kb * 128 + lane * 4;
-                *reinterpret_cast<uint2 *>(row) = make_uint2(t0[0], t0[1]);
-                *reinterpret_cast<uint2 *>(row + p.t_stride) = make_uint2(t1[0], t1[1]);
-                *reinterpret_cast<uint2 *>(row + 2 * p.t_stride) = make_uint2(t2[0], t2[1]);
-                if (lane == 0) hfac[sl * ib + kb] = pow2f(-sh);
+        while (ld_acquire_gpu(ready) < need) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                ok = 0;
+                break;
             }
         }
     }
-    __syncwarp();
+    if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) return false;
+    uint32_t m = 0;
+#pragma unroll
+    for (int t = 0; t < kStepMaxRows; ++t) {
+        sl[t] = -1;
+        if (t < rows) {
+            if (shared) {
+                sl[t] = rows * K + t;
+            } else {
+                for (int r = 0; r < K; ++r)
+                    if (sm.idx[t * K + r] == e) sl[t] = t * K + r;
+            }
+            if (sl[t] >= 0) m |= 1u << t;
+        }
+    }
+    *routed = m;
     return true;
 }
 
-// The K windows of one pair of output tiles for a down item: per window 8
-// MMA steps (A = the tiles' weight rows, B = the h-term columns of NBLK
-// column blocks) on four accumulator chains, then the window's scales (the
-// weight block scale of each tile's rows, the h factor of each column's
-// slot).  acc[nb][0..1]: the first tile's row g at this lane's two columns,
-// acc[nb][2..3]: the second tile's.
-template <int NBLK>
-__device__ __forceinline__ void down_windows(unsigned char *sbase, uint32_t base, uint32_t t0base, uint32_t box,
-                                             bool two, int ibu, const uint32_t (&baddr)[2], const int (&bslot)[2],
-                                             const int (&dslot)[2][2], uint32_t c0, uint32_t c1, int qd,
-                                             const float *s2a, const float *s2b, const float *hfac, int ib,
-                                             float (&acc)[2][4])
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&a)[4])
 {
-    auto lds128 = [=](uint32_t a) { return *reinterpret_cast<const uint4 *>(sbase + (a - base)); };
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-#pragma unroll 2
-    for (int w = 0; w < ibu; ++w) {
-        const uint32_t t0b = t0base + (uint32_t)w * 1024u;
-        const uint32_t t1b = t0b + box;
-        const uint4 w0l = lds128(t0b + c0), w0h = lds128(t0b + c1);
-        const uint4 w1l = two ? lds128(t1b + c0) : make_uint4(0, 0, 0, 0);
-        const uint4 w1h = two ? lds128(t1b + c1) : make_uint4(0, 0, 0, 0);
-        uint4 bv[NBLK][4];
-#pragma unroll
-        for (int nb = 0; nb < NBLK; ++nb)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                bv[nb][i] = bslot[nb] >= 0 ? lds128(baddr[nb] + (uint32_t)((w * 128 + 32 * qd + 8 * i) * 2))
-                                           : make_uint4(0, 0, 0, 0);
-        float d[NBLK][4][4];
-#pragma unroll
-        for (int nb = 0; nb < NBLK; ++nb)
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) d[nb][ch][0] = d[nb][ch][1] = d[nb][ch][2] = d[nb][ch][3] = 0.f;
-#pragma unroll
-        for (int st = 0; st < 8; ++st) {
-            const uint32_t x0 = word_of(st < 4 ? w0l : w0h, st & 3);
-            const uint32_t x1 = word_of(st < 4 ? w1l : w1h, st & 3);
-            uint32_t a0, a1, a2, a3;
-            e4m3x4_to_f16x2x2(x0, a0, a2);
-            e4m3x4_to_f16x2x2(x1, a1, a3);
-#pragma unroll
-            for (int nb = 0; nb < NBLK; ++nb)
-                mma_f16_16816(d[nb][st & 3], a0, a1, a2, a3, word_of(bv[nb][st >> 1], (st & 1) * 2),
-                              word_of(bv[nb][st >> 1], (st & 1) * 2 + 1));
-        }
-        const float sw0 = s2a[w];
-        const float sw1 = two ? s2b[w] : 0.f;
-#pragma unroll
-        for (int nb = 0; nb < NBLK; ++nb) {
-            const float f0 = dslot[nb][0] >= 0 ? hfac[dslot[nb][0] * ib + w] : 0.f;
-            const float f1 = dslot[nb][1] >= 0 ? hfac[dslot[nb][1] * ib + w] : 0.f;
-            float sum[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) sum[r] = (d[nb][0][r] + d[nb][1][r]) + (d[nb][2][r] + d[nb][3][r]);
-            acc[nb][0] = fmaf(sw0 * f0, sum[0], acc[nb][0]);
-            acc[nb][1] = fmaf(sw0 * f1, sum[1], acc[nb][1]);
-            acc[nb][2] = fmaf(sw1 * f0, sum[2], acc[nb][2]);
-            acc[nb][3] = fmaf(sw1 * f1, sum[3], acc[nb][3]);
-        }
-    }
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(addr));
 }
 
-// One down item: per expert of the item, per pair of output tiles, the full
-// K.  A = the 16 weight rows of the two tiles (rows g of the first tile in
-// MMA rows 0-7, of the second in 8-15), B = the h terms, column 3t + j = term
-// j of row t (two MMAs per step above 8 columns); each lane's four
-// accumulator chains take every fourth MMA step of a window.  The result
-// goes to the down buffer (with go == false it does not).
-__device__ __forceinline__ void down_item(const StepParams &p, const StepSmall &sm, const Item &it, uint32_t sl,
-                                       unsigned char *sbase, uint32_t base, int U, int rows, int K, int nt, int tile0,
-                                       int rb0, int ibm, int ib, const uint16_t *terms, const float *hfac,
-                                       const float *dsc, float *ybuf, float *scr, bool go)
+// D = A * B for one K chunk of 32: A 16 x 32 e4m3 (row major), B 32 x 8 e5m2
+// (column major), fp32 accumulation from zero.
+__device__ __forceinline__ void mma_e4m3_e5m2_16832(float (&d)[4], const uint32_t (&a)[4], uint2 b)
 {
-    const int lane = threadIdx.x & 31, g = lane >> 2, qd = lane & 3;
-    const int yrow = p.nt_max * 8;
-    const int ncol = 3 * rows;
-    const int nblk = ncol > 8 ? 2 : 1;
-    const bool shared = it.a == 0;
-    const int ne = group_size(p, U, it.a);
-    const int Iu = shared ? p.Is : p.I;
-    const int ibu = Iu / 128;
-    const int tpi = shared ? p.dn_tpi_s : p.dn_tpi;
-    const int tfirst = it.p * tpi;                 // first tile of the chunk (local)
-    const int ntile = min(tpi, nt - tfirst);
-    const uint32_t box = 8u * (uint32_t)Iu;        // bytes of one expert's tile box
-    const uint32_t c0 = (uint32_t)(((2 * qd) ^ g) * 16), c1 = (uint32_t)(((2 * qd + 1) ^ g) * 16);
-    for (int x = 0; x < ne; ++x) {
-        const int li = shared ? -1 : (it.a - 1) * p.dn_epi + x;  // index in the routed list
-        const int e = shared ? 0 : sm.list[li];
-        const int de = shared ? 0 : 1 + li;
-        // slot of row t for this expert (-1: row t does not route to it)
-        auto slot_of = [&](int t) {
-            if (t >= rows) return -1;
-            if (shared) return rows * K + t;
-            int r_ = -1;
-            for (int r = 0; r < K; ++r)
-                if (sm.idx[t * K + r] == e) r_ = t * K + r;
-            return r_;
-        };
-        // B column g of each column block, and the slots of the lane's D columns 2q, 2q+1
-        uint32_t baddr[2];
-        int bslot[2], dslot[2][2];
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e5m2.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y), "f"(0.f));
+}
+
+// One down item, by one warp, on the tensor cores (mma.sync): per K chunk of
+// 32, A = the item's weight rows (its two 8-row output tiles as MMA rows 0-7
+// and 8-15; with one tile a copy of it) straight from the TMA slot through
+// ldmatrix (the 128-byte swizzle: 16-byte chunk c of row r sits at c xor
+// (r % 8)), B = the eight e5m2 terms of h of a row of x routed to the expert
+// (column j = term j), as the gate/up epilogue laid them out (lane l's eight
+// bytes of a chunk are its two B registers), brought into the warp's buffer
+// bbuf (16 chunks) by one bulk copy a round.  Each chunk's D, its eight term
+// columns added, times the window's weight block scale and the chunk's power
+// of two of h, into a running sum per row; the four lanes of a row then add
+// their sums.  Products are exact (e4m3 x e5m2); sums fp32.  *bphase: the
+// parity of bbar's next phase.  False if a copy's wait ran out.
+template <int R>
+__device__ __forceinline__ bool down_item_mma(const StepParams &p, uint32_t slot_u32, int tpi, int ibu, int tl0,
+                                              int nt, int tile0, int rb0, const float *s2e, int ibm, float *yb,
+                                              int yrow, const int (&sl)[kStepMaxRows], uint32_t routed,
+                                              unsigned char *bbuf, uint64_t *bbar, uint32_t *bphase)
+{
+    const int lane = threadIdx.x & 31, g = lane >> 2;
+    const int nch = ibu * 4;         // K chunks of 32
+    const int ntc = p.imax / 32;     // chunks of a slot of h terms
+    // this lane's ldmatrix row: matrix lane / 8 (0: rows 0-7, K 0-15; 1: rows
+    // 8-15; 2, 3: K 16-31), row lane % 8 of it
+    const int mi = lane >> 3, rr = lane & 7;
+    const uint32_t abase = slot_u32 + (uint32_t)((tpi == 2 ? (mi & 1) : 0) * 1024 + rr * 128);
+    const int tlB = min(tl0 + 1, nt - 1);
+    const float *s2a = s2e + min(1, ((tile0 + tl0) * 8) / 128 - rb0) * ibm;
+    const float *s2b = s2e + min(1, ((tile0 + tlB) * 8) / 128 - rb0) * ibm;
+    const uint32_t bb = smem_u32(bbuf) + (uint32_t)lane * 8;
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-            const int cb = nb * 8 + g;
-            bslot[nb] = cb < ncol ? slot_of(cb / 3) : -1;
-            baddr[nb] = bslot[nb] >= 0 ? smem_u32(terms + ((size_t)bslot[nb] * 3 + cb % 3) * p.t_stride) : 0u;
+    for (int t = 0; t < R; ++t) {
+        if (!((routed >> t) & 1u)) continue;  // the same in every lane
+        // four independent sums per tile row (chunk i into sums i % 4), added
+        // in a fixed order at the end
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c0 = 0; c0 < nch; c0 += 16) {
+            const int n = min(16, nch - c0);
+            if (lane == 0) {
+                fence_proxy_async_smem();  // the lanes' reads of the last round (ordered by the warp barrier)
+                mbar_arrive_expect_tx(bbar, (uint32_t)n * 256);
+                bulk_g2s(bbuf, p.hterm + ((size_t)sl[t] * ntc + c0) * 256, (uint32_t)n * 256, bbar);
+            }
+            const float hs = lane < n ? __ldcg(p.hsc + (size_t)sl[t] * ntc + c0 + lane) : 0.f;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_spin(bbar, *bphase, kWaitLimitNs) ? 1 : 0;
+            *bphase ^= 1u;
+            ITEM_T(40 + (threadIdx.x >> 5), 4);  // trace: the warp's last copy of h terms landed
+            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) return false;
+            // a window (four chunks) at a time: n is a multiple of 4
+            for (int i0 = 0; i0 < n; i0 += 4) {
+                const int w = (c0 + i0) >> 2;
+                uint32_t a[4][4];
+                uint2 b[4];
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int cd = nb * 8 + 2 * qd + cc;
-                dslot[nb][cc] = cd < ncol ? slot_of(cd / 3) : -1;
+                for (int kc = 0; kc < 4; ++kc) {
+                    ldmatrix_x4(abase + (uint32_t)(w * tpi * 1024) + ((uint32_t)((2 * kc + (mi >> 1)) ^ rr) << 4),
+                                a[kc]);
+                    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                 : "=r"(b[kc].x), "=r"(b[kc].y)
+                                 : "r"(bb + (uint32_t)(i0 + kc) * 256));
+                }
+                float d[4][4];
+#pragma unroll
+                for (int kc = 0; kc < 4; ++kc) mma_e4m3_e5m2_16832(d[kc], a[kc], b[kc]);
+                const float sa = s2a[w], sb = s2b[w];
+#pragma unroll
+                for (int kc = 0; kc < 4; ++kc) {
+                    const float f = __shfl_sync(0xFFFFFFFFu, hs, i0 + kc);
+                    acc0[kc] = fmaf(sa * f, d[kc][0] + d[kc][1], acc0[kc]);
+                    acc1[kc] = fmaf(sb * f, d[kc][2] + d[kc][3], acc1[kc]);
+                }
+            }
+            __syncwarp();  // the buffer is free for the next round
+        }
+        float v0 = (acc0[0] + acc0[1]) + (acc0[2] + acc0[3]);
+        float v1 = (acc1[0] + acc1[1]) + (acc1[2] + acc1[3]);
+        v0 += __shfl_xor_sync(0xFFFFFFFFu, v0, 1);
+        v0 += __shfl_xor_sync(0xFFFFFFFFu, v0, 2);
+        v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, 1);
+        v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, 2);
+        if ((lane & 3) == 0) {
+            if (tl0 < nt) yb[(size_t)t * yrow + tl0 * 8 + g] = v0;
+            if (tpi == 2 && tl0 + 1 < nt) yb[(size_t)t * yrow + (tl0 + 1) * 8 + g] = v1;
+        }
+    }
+    return true;
+}
+
+// P3, by each consumer warp: down items claimed one at a time in item order
+// (warps arrive as they finish gate/up); each waits until its
+// expert's gate/up units (in whichever CTAs) are all counted and for its
+// weight rows, then multiplies them by the expert's h terms on the tensor
+// cores (mma.sync, one warp an item) into the down buffer.
+__device__ __forceinline__ void down_phase(const StepParams &p, StepSmall &sm, unsigned char *sbase, uint32_t base,
+                                           uint64_t *full, uint64_t *empty, uint64_t *tdone, uint64_t *bbars,
+                                           const Seq &seq, int nt, int tile0, int rb0, int ibm, const float *dsc,
+                                           float *ybuf, volatile int32_t *abort)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = p.rows;
+    {
+        const int yrow = p.nt_max * 8;
+        // the warp's buffer of h terms (in the x-term region: first every
+        // gate/up MMA, which reads the x terms, must be done)
+        unsigned char *bbuf = sbase + p.o_uni + (size_t)warp * 16 * 256;
+        uint64_t *bbar = &bbars[warp];
+        uint32_t bphase = 0;
+        {
+            int okd = 1;
+            if (lane == 0) okd = mbar_wait(tdone, 0, kWaitLimitNs) ? 1 : 0;
+            if (!__shfl_sync(0xFFFFFFFFu, okd, 0)) {
+                if (lane == 0) {
+                    gave_up(p.counters, 10, 2);
+                    *abort = 1;
+                }
             }
         }
-        const float *s2 = dsc + (size_t)de * 2 * ibm;
-        const uint32_t ebase = sl + (uint32_t)(x * tpi) * box + (uint32_t)g * 128u;
-        for (int i0 = 0; i0 < ntile; i0 += 2) {
-            const bool two = i0 + 1 < ntile;
-            const int row0 = (tile0 + tfirst + i0) * 8, row1 = row0 + 8;
-            float acc[2][4];
-            if (nblk == 1)
-                down_windows<1>(sbase, base, ebase + (uint32_t)i0 * box, box, two, ibu, baddr, bslot, dslot, c0, c1,
-                                qd, s2 + (row0 / 128 - rb0) * ibm, s2 + (row1 / 128 - rb0) * ibm, hfac, ib, acc);
-            else
-                down_windows<2>(sbase, base, ebase + (uint32_t)i0 * box, box, two, ibu, baddr, bslot, dslot, c0, c1,
-                                qd, s2 + (row0 / 128 - rb0) * ibm, s2 + (row1 / 128 - rb0) * ibm, hfac, ib, acc);
-            // y[t][n] = (term 0 + term 1) + term 2 of row t, into the down buffer
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                if (nb >= nblk) continue;
-                scr[g * 16 + nb * 8 + 2 * qd] = acc[nb][0];
-                scr[g * 16 + nb * 8 + 2 * qd + 1] = acc[nb][1];
-                scr[(g + 8) * 16 + nb * 8 + 2 * qd] = acc[nb][2];
-                scr[(g + 8) * 16 + nb * 8 + 2 * qd + 1] = acc[nb][3];
+        for (;;) {
+            // the next unclaimed item (warps arrive as they finish gate/up)
+            int b = 0;
+            if (lane == 0) b = atomicAdd(&sm.dn_next, 1);
+            b = __shfl_sync(0xFFFFFFFFu, b, 0);
+            if (b >= seq.n_dn || *abort) break;
+            const int q = seq.n_router + seq.n_gu + b;
+            const Item it = item_at(p, seq, q);
+            const int s = q % p.ns;
+            int sl[kStepMaxRows];
+            uint32_t routed = 0;
+            if (!wait_expert(p, sm, it, sl, &routed)) {
+                if (lane == 0) {
+                    gave_up(p.counters, 11, q);
+                    *abort = 1;
+                }
+                break;
             }
-            __syncwarp();
-            for (int u = lane; u < rows * 16; u += kWarp) {
-                const int t = u >> 4, r = u & 15;
-                if (r >= 8 && !two) continue;
-                const float y = (scr[r * 16 + 3 * t] + scr[r * 16 + 3 * t + 1]) + scr[r * 16 + 3 * t + 2];
-                if (go) ybuf[((size_t)de * rows + t) * yrow + (tfirst + i0 + (r >> 3)) * 8 + (r & 7)] = y;
+            ITEM_T(q, 3);
+            if (!wait_item(sm.tag, full, s, q, p.ns)) {
+                if (lane == 0) {
+                    gave_up(p.counters, 3, q);
+                    *abort = 1;
+                }
+                break;
             }
+            ITEM_T(q, 0);
+            const bool shared = it.a == 0;
+            const int de = shared ? 0 : 1 + (it.a - 1) * p.dn_epi;
+            const int tpi = shared ? p.dn_tpi_s : p.dn_tpi;
+            const int ibu = (shared ? p.Is : p.I) / 128;
+            const uint32_t su = base + (uint32_t)s * kSlot;
+            const float *s2e = dsc + (size_t)de * 2 * ibm;
+            float *yb = ybuf + (size_t)de * rows * yrow;
+            const int tl0 = it.p * tpi;
+            bool ok;
+            switch (rows) {
+            case 1: ok = down_item_mma<1>(p, su, tpi, ibu, tl0, nt, tile0, rb0, s2e, ibm, yb, yrow, sl, routed, bbuf, bbar, &bphase); break;
+            case 2: ok = down_item_mma<2>(p, su, tpi, ibu, tl0, nt, tile0, rb0, s2e, ibm, yb, yrow, sl, routed, bbuf, bbar, &bphase); break;
+            case 3: ok = down_item_mma<3>(p, su, tpi, ibu, tl0, nt, tile0, rb0, s2e, ibm, yb, yrow, sl, routed, bbuf, bbar, &bphase); break;
+            case 4: ok = down_item_mma<4>(p, su, tpi, ibu, tl0, nt, tile0, rb0, s2e, ibm, yb, yrow, sl, routed, bbuf, bbar, &bphase); break;
+            default: ok = down_item_mma<kStepMaxRows>(p, su, tpi, ibu, tl0, nt, tile0, rb0, s2e, ibm, yb, yrow, sl, routed, bbuf, bbar, &bphase); break;
+            }
+            if (!ok) {
+                if (lane == 0) {
+                    gave_up(p.counters, 12, q);
+                    *abort = 1;
+                }
+                break;
+            }
+            ITEM_T(q, 1);
             __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
 }
@@ -819,7 +791,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     uint64_t *empty = full + p.ns;
     uint64_t *tfull = empty + p.ns;  // [2] a unit's gate/up MMAs done (tcgen05.commit)
     uint64_t *tfree = tfull + 2;     // [2] its accumulators read (the 4 epilogue warps)
-    uint64_t *tdone = tfree + 2;     // every MMA of this CTA done
+    uint64_t *tdone = tfree + 2;     // every gate/up MMA of this CTA done
+    uint64_t *bbars = tdone + 1;     // [kStepWarps] each consumer warp's bulk copies of h terms
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
     const int rows = p.rows, H = p.H, E = p.E, K = p.K;
@@ -843,7 +816,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             mbar_init(&tfree[b], 4);
         }
         mbar_init(tdone, kIssuers);
+        for (int w = 0; w < kStepWarps; ++w) mbar_init(&bbars[w], 1);
         sm.abort = 0;
+        sm.dn_next = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1023,11 +998,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 }
             }
         }
-        // the block maxima of h and the per-expert unit counts start at zero
-        // (P2 raises them after the grid barrier)
+        // the per-expert unit counts start at zero (P2 raises them after the
+        // grid barrier)
         if (c == 0) {
-            for (int i = threadIdx.x; i < rows * (K + 1) * (p.imax / 128); i += kStepWarps * kWarp) p.hmax[i] = 0u;
-            for (int i = threadIdx.x; i <= rows * K; i += kStepWarps * kWarp) p.counters[kCtrStepReady + i] = 0;
+            for (int i = threadIdx.x; i <= rows * K; i += kStepWarps * kWarp) p.counters[kCtrStepReady + i * p.rdy] = 0;
         }
         // the logits and the zeros are ordered before thread 0's release
         // through the CTA barrier (its fence is cumulative)
@@ -1250,7 +1224,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     }
 
     // ---------------------------------------------------------------- consumers
-    uint16_t *xs = reinterpret_cast<uint16_t *>(sbase + p.o_uni);
     const float *xfac = reinterpret_cast<const float *>(sbase + p.o_xfac);
 
     // Block scales of this CTA's work into shared memory, one round trip for
@@ -1393,27 +1366,47 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 named_barrier(3, 4 * kWarp);
                 if (gate) {
                     // h = silu(gate) * up for the rows routed to this expert
-                    // (lanes 0-15), and the largest |h| of the warp's 16 into
-                    // the block maximum (one atomic a warp and row)
+                    // (lanes 0-15 of both warps: the unit's 32 values, one K
+                    // chunk of the down MMAs), as eight e5m2 terms: a power of
+                    // two puts the chunk's largest |h| in [2^14, 2^15), and
+                    // t_k = e5m2(h' - t_1 - ... - t_(k-1)) (differences exact in
+                    // fp32) sum to h' exactly for every value within 2^7 of that
+                    // maximum and to within 2^-31 of it below.  Term k of value
+                    // m goes where the down MMA's B registers want it: byte
+                    // (m % 4) + 4 (m / 16) of lane 4k + (m % 16) / 4's eight.
+                    int slots[kStepMaxRows];
+                    float hv[kStepMaxRows];
 #pragma unroll
                     for (int t = 0; t < kStepMaxRows; ++t) {
+                        slots[t] = -1;
+                        hv[t] = 0.f;
                         if (t >= rows) continue;
-                        int slot = -1;
                         if (shared) {
-                            slot = rows * K + t;
+                            slots[t] = rows * K + t;
                         } else {
                             for (int r = 0; r < K; ++r)
-                                if (sm.idx[t * K + r] == e) slot = t * K + r;
+                                if (sm.idx[t * K + r] == e) slots[t] = t * K + r;
                         }
-                        if (slot < 0) continue;  // the same in every lane
-                        float hv = 0.f;
-                        if (lane < 16) {
-                            hv = siluf_(acc[t]) * sm.xch[m * kStepMaxRows + t];
-                            p.h[(size_t)slot * p.imax + j + m] = hv;
+                        if (slots[t] >= 0 && lane < 16) hv[t] = siluf_(acc[t]) * sm.xch[m * kStepMaxRows + t];
+                        const float mx = warp_max(fabsf(hv[t]));
+                        if (lane == 0) sm.hmx[warp * kStepMaxRows + t] = mx;
+                    }
+                    named_barrier(2, 2 * kWarp);  // both gate warps' maxima
+                    const int ntc = p.imax / 32;
+#pragma unroll
+                    for (int t = 0; t < kStepMaxRows; ++t) {
+                        if (t >= rows || slots[t] < 0) continue;  // the same in every lane
+                        const int sh = block_shift(fmaxf(sm.hmx[t], sm.hmx[kStepMaxRows + t]));
+                        float x = hv[t] * pow2f(sh);
+                        unsigned char *dst = p.hterm + ((size_t)slots[t] * ntc + j / 32) * 256 + (lane >> 2) * 8 +
+                                             warp * 4 + (lane & 3);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t c = f32x2_to_e5m2x2(x, 0.f);
+                            x -= e5m2x2_to_f32x2(c).x;
+                            if (lane < 16) dst[k * 32] = (unsigned char)(c & 0xFFu);
                         }
-                        const float mx = warp_max(fabsf(hv));
-                        if (lane == 0)
-                            atomicMax(p.hmax + (size_t)slot * (p.imax / 128) + j / 128, __float_as_uint(mx));
+                        if (warp == 0 && lane == 0) p.hsc[(size_t)slots[t] * ntc + j / 32] = pow2f(-sh);
                     }
                 }
                 named_barrier(3, 4 * kWarp);  // the exchange slots are free again
@@ -1425,73 +1418,34 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                     const int u = c + l * G, us = p.Is / kGuRows;
                     const int de = u < us ? 0 : 1 + (u - us) / (p.I / kGuRows);
                     __threadfence();
-                    red_release_gpu(p.counters + kCtrStepReady + de, 1);
+                    red_release_gpu(p.counters + kCtrStepReady + de * p.rdy, 1);
+                    STEP_TL(15);  // (trace) this CTA's last unit counted
                 }
             }
         }
-        // every MMA done and every accumulator read: the tensor memory goes
-        // back before anything below can leave early
-        tc_fence_before();
-        if (warp < 4 || (warp >= kIssuer0 && warp < kIssuer0 + kIssuers)) named_barrier(4, (4 + kIssuers) * kWarp);
+        // every gate/up MMA done (before P3 reuses the x-term region and the
+        // accumulator columns)
         if (warp == 0) {
-            tc_fence_after();
             if (lane == 0 && !mbar_wait(tdone, 0, kWaitLimitNs)) {
                 gave_up(p.counters, 10, 0);
                 *abort = 1;
             }
             __syncwarp();
+            tc_fence_after();
             tmem_dealloc(tmem, (uint32_t)p.tcols);
         }
     }
-    // P3's buffers
-    const int ib = p.imax / 128;
-    uint16_t *terms = xs;  // the x region, once the gate/up MMAs are done
-    float *hfac = reinterpret_cast<float *>(sbase + p.o_hfac);
-    float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);   // [U + 1][rows][nt_max * 8]
-    float *scr = reinterpret_cast<float *>(sbase + p.o_scr) + warp * 256;  // [16 rows][16 columns]
+    float *ybuf = reinterpret_cast<float *>(sbase + p.o_y);  // [U + 1][rows][nt_max * 8]
     STEP_MARK(6, 0);
     STEP_T(7);  // warp 0's gate/up items done
-    ITEM_T(55 + warp, 3);
     pdl_trigger();  // this CTA's weight reads are all issued: the next kernel may start
-    if (*abort || nt == 0) return;
 
     // ---------------------------------------------------------------- P3
-    // no grid barrier: each down item waits until its expert's gate/up units
-    // (in whichever CTAs) are all counted, stages that expert's slots of h as
-    // terms, then runs
-    // down items, round robin over the warps (item b to warp b % 8): per
-    // expert of the item, per pair of output tiles, the full K.  A = the 16
-    // weight rows of the two tiles (rows g of the first tile in MMA rows 0-7,
-    // of the second in 8-15), B = the h terms, column 3t + j = term j of row t
-    // (two MMAs per step above 8 columns); each lane's four accumulator
-    // chains take every fourth MMA step of a window.
-    for (int b = warp; b < seq.n_dn && !*abort; b += kStepWarps) {
-        const int q = seq.n_router + seq.n_gu + b;
-        const Item it = item_at(p, seq, q);
-        const int s = q % p.ns;
-        if (!stage_expert_h(p, sm, it, U, terms, hfac, ib)) {
-            if (lane == 0) {
-                gave_up(p.counters, 11, q);
-                *abort = 1;
-            }
-            break;
-        }
-        if (warp == 0 && b == 0) STEP_T(9);  // warp 0's first expert staged
-        if (!wait_item(sm.tag, full, s, q, p.ns)) {
-            if (lane == 0) {
-                gave_up(p.counters, 3, q);
-                *abort = 1;
-            }
-            break;
-        }
-        ITEM_T(q, 0);
-        down_item(p, sm, it, base + (uint32_t)s * kSlot, sbase, base, U, rows, K, nt, tile0, rb0, ibm, ib, terms, hfac,
-                  dsc, ybuf, scr, true);
-        ITEM_T(q, 1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    named_barrier(1, kStepWarps * kWarp);
+    // No grid barrier: down items claimed by the warps as they come free
+    // (down_phase).
+    STEP_T(8);  // P3 starts
+    down_phase(p, sm, sbase, base, full, empty, tdone, bbars, seq, nt, tile0, rb0, ibm, dsc, ybuf, abort);
+    named_barrier(1, kStepWarps * kWarp);  // every down item of the CTA done
     if (*abort) return;
 
     STEP_T(10);  // down items done
@@ -1555,11 +1509,11 @@ bool make_map_gate_up(CUtensorMap *m, const void *base, uint64_t inter, uint64_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A byte tensor [outer][rows][windows of 128 bytes] as a 4-D TMA map over
-// (128 bytes, rows, windows, outer) with 128-byte-swizzled boxes
-// {128, box_rows, box_windows, 1}: a box lands as [window][box_rows][128 bytes].
-bool make_map_rows_windows(CUtensorMap *m, const void *base, uint64_t rows, uint64_t kbytes, uint64_t outer,
-                           uint64_t outer_stride, uint32_t box_windows, uint32_t box_rows = 8)
+// W2 of the expert slabs [H rows][inter bytes] as a 5-D TMA map over (128
+// bytes, 8 rows, H/8 tiles, windows, experts) with 128-byte-swizzled boxes
+// {128, 8, tiles, inter/128, 1}: a box lands as [window][tile][8 rows][128 B].
+bool make_map_down(CUtensorMap *m, const void *base, uint64_t hidden, uint64_t inter, uint64_t experts,
+                   uint64_t expert_stride, uint32_t tiles)
 {
     using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -1573,11 +1527,11 @@ bool make_map_rows_windows(CUtensorMap *m, const void *base, uint64_t rows, uint
         return reinterpret_cast<EncodeFn>(f);
     }();
     if (!fn) return false;
-    const cuuint64_t dims[4] = {128, rows, kbytes / 128, outer};
-    const cuuint64_t strides[3] = {kbytes, 128, outer_stride ? outer_stride : rows * kbytes};
-    const cuuint32_t box[4] = {128, box_rows, box_windows, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
+    const cuuint64_t dims[5] = {128, 8, hidden / 8, inter / 128, experts};
+    const cuuint64_t strides[4] = {inter, 8 * inter, 128, expert_stride ? expert_stride : 3 * inter * hidden};
+    const cuuint32_t box[5] = {128, 8, tiles, (cuuint32_t)(inter / 128), 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1600,33 +1554,31 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     s.nb = 3 * rows <= 8 ? 8 : 16;
     s.tbuf = (H / 128) * s.nb;
     s.nbuf = 2 * s.tbuf <= 512 ? 2 : 1;
-    {
-        const int need = (s.nbuf - 1) * s.tbuf + (s.tbuf + 31) / 32 * 32;  // loads take 32 columns at a time
-        s.tcols = 32;
-        while (s.tcols < need) s.tcols *= 2;
-    }
+    s.tcols = 32;
+    while (s.tcols < s.nbuf * s.tbuf) s.tcols *= 2;
     const int n8 = H / 8;
     s.nt_max = (n8 + G - 1) / G;
-    // down items: the full K of one or two output tiles per expert
+    // down items: the full K of one or two output tiles of one expert (one
+    // 5-D box, [window][tile][8 rows][128 B])
     s.dn_tpi = 2 * 8 * I <= kSlot ? 2 : 1;
     s.dn_tpi_s = 2 * 8 * Is <= kSlot ? 2 : 1;
-    s.dn_epi = 1;  // one expert per down item: more items for the warps
+    s.dn_epi = 1;
     s.rr_per_item = std::max(1, kSlot / (2 * H));
     // shared memory, after the ring
-    const int nslots = rows * (K + 1);
     s.x_stride = H + 8;
-    s.t_stride = imax + 8;
     const size_t xbytes = (size_t)rows * s.x_stride * 2;
-    const size_t tbytes = (size_t)nslots * 3 * s.t_stride * 2;
+    const int umax = std::min(d.n_experts, rows * K);
+    // the down experts' unit counters, one 128-byte line each where they fit
+    s.rdy = 32;
+    while (s.rdy > 1 && kCtrStepReady + (rows * K + 1) * s.rdy > kCtrStepDiag) s.rdy /= 2;
     size_t o = 0;
     auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 16); return (uint32_t)at; };
     const size_t xBbytes = (size_t)(H / 128) * s.nb * 128;
-    const uint32_t uni = take(std::max(xBbytes + xbytes, tbytes));  // [x terms | bf16 x] in P1-P2, h terms in P3
+    // x terms, then bf16 x; in P3 the consumer warps' buffers of h terms (16
+    // chunks of 256 bytes each)
+    const uint32_t uni = take(std::max(xBbytes + xbytes, (size_t)kStepWarps * 16 * 256));
     const uint32_t xfac = take((size_t)rows * (H / 128) * 4);
-    const uint32_t hfac = take((size_t)nslots * (imax / 128) * 4);
-    const int umax = std::min(d.n_experts, rows * K);
     const uint32_t y = take((size_t)(umax + 1) * rows * s.nt_max * 8 * 4);
-    const uint32_t scr = take((size_t)kStepWarps * 256 * 4);
     const int64_t units_max = Is / kGuRows + (int64_t)umax * (I / kGuRows);
     s.max_units = (int)((units_max + G - 1) / G);
     const uint32_t gsc = take((size_t)s.max_units * 2 * (H / 128) * 4);
@@ -1639,28 +1591,26 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     const uint32_t smo = take(sizeof(StepSmall));
     const size_t tail = o;
     // ring slots: whatever is left, up to 16
-    const size_t avail = (size_t)kSmemCap - 1024 - tail - (16 * 2 + 5) * 8;
+    const size_t avail = (size_t)kSmemCap - 1024 - tail - (16 * 2 + 16) * 8;
     s.ns = (int)std::min<size_t>(16, avail / kSlot);
     const uint32_t ring = (uint32_t)s.ns * kSlot;
     s.o_uni = ring + uni;  // 1024-aligned: the ring is a multiple of 16 KB and uni comes first
     s.o_xB = ring + uni;
     s.o_xb = ring + uni + (uint32_t)xBbytes;
     s.o_xfac = ring + xfac;
-    s.o_hfac = ring + hfac;
     s.o_y = ring + y;
-    s.o_scr = ring + scr;
     s.o_gsc = ring + gsc;
     s.o_dsc = ring + dsc;
     s.o_cand = ring + cand;
     s.o_sm = ring + smo;
     s.o_bar = (uint32_t)align_up(ring + tail, 8);
-    s.smem = s.o_bar + (2 * s.ns + 5) * 8 + 1024;
+    s.smem = s.o_bar + (2 * s.ns + 16) * 8 + 1024;
     // the router items all sit in the ring before the first slot is reused
     const int rr_max = (d.n_experts + 1 + G - 1) / G;
     const int router_items = (rr_max + s.rr_per_item - 1) / s.rr_per_item;
     s.ok = s.ns >= 2 && s.ns > router_items && s.nt_max <= kMaxNt && s.smem <= kSmemCap && 2 * H <= kSlot &&
            8 * I <= kSlot && 8 * Is <= kSlot && 3 * rows <= 16 && s.tbuf <= 512 && I % kGuRows == 0 &&
-           Is % kGuRows == 0;
+           Is % kGuRows == 0 && kCtrStepReady + (rows * K + 1) * s.rdy <= kCtrStepDiag;
     return s;
 }
 
@@ -1687,10 +1637,10 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     if (!make_map_gate_up(&p.w13, a.expert_w8, (uint64_t)I, (uint64_t)H, (uint64_t)E, 3 * (uint64_t)I * H,
                           (uint32_t)sh.gu_wp) ||
         !make_map_gate_up(&p.w13s, a.shared_w8, (uint64_t)Is, (uint64_t)H, 1, 0, (uint32_t)sh.gu_wp) ||
-        !make_map_rows_windows(&p.w2, a.expert_w8 + (size_t)2 * I * H, (uint64_t)H, (uint64_t)I, (uint64_t)E,
-                               3 * (uint64_t)I * H, (uint32_t)(I / 128)) ||
-        !make_map_rows_windows(&p.w2s, a.shared_w8 + (size_t)2 * Is * H, (uint64_t)H, (uint64_t)Is, 1, 0,
-                               (uint32_t)(Is / 128)))
+        !make_map_down(&p.w2, a.expert_w8 + (size_t)2 * I * H, (uint64_t)H, (uint64_t)I, (uint64_t)E,
+                       3 * (uint64_t)I * H, (uint32_t)sh.dn_tpi) ||
+        !make_map_down(&p.w2s, a.shared_w8 + (size_t)2 * Is * H, (uint64_t)H, (uint64_t)Is, 1, 0,
+                       (uint32_t)sh.dn_tpi_s))
         return cudaErrorInvalidValue;
     p.x = a.x;
     p.router_w = a.router_w;
@@ -1706,8 +1656,8 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.topk_w = a.topk_w;
     p.gsig = a.gsig;
     p.logits = a.logits;
-    p.h = a.h;
-    p.hmax = a.hmax;
+    p.hterm = a.hterm;
+    p.hsc = a.hsc;
     p.counters = a.counters;
     p.rows = a.rows;
     p.H = H;
@@ -1728,9 +1678,8 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.o_uni = sh.o_uni;
     p.o_xb = sh.o_xb;
     p.o_xfac = sh.o_xfac;
-    p.o_hfac = sh.o_hfac;
     p.o_y = sh.o_y;
-    p.o_scr = sh.o_scr;
+    p.rdy = sh.rdy;
     p.o_gsc = sh.o_gsc;
     p.o_dsc = sh.o_dsc;
     p.o_xB = sh.o_xB;
@@ -1744,7 +1693,6 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.o_sm = sh.o_sm;
     p.o_bar = sh.o_bar;
     p.x_stride = sh.x_stride;
-    p.t_stride = sh.t_stride;
     return launch_kernel(decode_step_kernel, dim3(sh.grid), dim3(kStepThreads), sh.smem, st, p);
 }
 

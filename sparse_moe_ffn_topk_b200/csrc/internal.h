@@ -18,7 +18,8 @@ constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per toke
 constexpr int kMaxRouterGroups = 1024;
 constexpr int kCtrStepBar = 8;          // decode step kernel: grid-barrier arrivals
 constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs past the grid barrier
-constexpr int kCtrStepReady = 16;       // decode step kernel: per down expert (shared, then the routed list), units done
+constexpr int kCtrStepReady = 16;       // decode step kernel: per down expert (shared, then the routed list), units done,
+                                        // a stride of StepShape::rdy ints apart
 constexpr int kCtrStepDiag = 2048;      // decode step kernel: per CTA, where a wait ran out (0: none)
 constexpr int kMaxBlendBlocks = 2048;   // H / 8 limit
 constexpr int kSmallRouterRows = 64;    // the grouped-GEMM path routes up to this many rows with the router kernel
@@ -34,7 +35,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Decode-path workspace, carved from the caller's buffer: the router's
 // logits and routing for all rows; h for one decode-step launch.
 struct DecodeLayout {
-    size_t counters, logits, topk_idx, topk_w, gsig, h, hmax, total;
+    size_t counters, logits, topk_idx, topk_w, gsig, hterm, hsc, total;
     int ld;
 };
 
@@ -52,8 +53,8 @@ inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
     L.topk_idx = take(sizeof(int32_t) * rows * K);
     L.topk_w = take(sizeof(float) * rows * K);
     L.gsig = take(sizeof(float) * rows);
-    L.h = take(sizeof(float) * hrows * (K + 1) * imax);
-    L.hmax = take(sizeof(uint32_t) * hrows * (K + 1) * (imax / 128));
+    L.hterm = take((size_t)8 * hrows * (K + 1) * imax);
+    L.hsc = take(sizeof(float) * hrows * (K + 1) * (imax / 32));
     L.total = o;
     return L;
 }
@@ -107,9 +108,9 @@ cudaError_t launch_router_topk(const RouterLaunch &a, cudaStream_t s);
 struct StepShape {
     bool ok;
     int grid, ns, gu_wp, gu_pieces, dn_tpi, dn_tpi_s, dn_epi, nt_max, rr_per_item;
-    int x_stride, t_stride;
-    uint32_t o_uni, o_xb, o_xfac, o_hfac, o_y, o_scr, o_sm, o_bar, o_gsc, o_dsc, o_cand, o_xB;
-    int nb, nbuf, tbuf, tcols;
+    int x_stride;
+    uint32_t o_uni, o_xb, o_xfac, o_y, o_sm, o_bar, o_gsc, o_dsc, o_cand, o_xB;
+    int nb, nbuf, tbuf, tcols, rdy;
     bool cand2;
     int max_units;
     size_t smem;
@@ -138,8 +139,8 @@ struct StepLaunch {
     float *gsig;
     float *logits;
     int logits_ld;
-    float *h;
-    uint32_t *hmax;  // per (slot, 128 block) the largest |h| as fp32 bits
+    unsigned char *hterm;  // [rows * (K + 1)][inter / 32][256]: h as e5m2 terms (the down MMAs' B layout)
+    float *hsc;            // [rows * (K + 1)][inter / 32]: each chunk's power of two
     int32_t *counters;
 };
 cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t s);

@@ -195,8 +195,8 @@ int run_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16
         a.gsig = gs + r0;
         a.logits = reinterpret_cast<float *>(base + L.logits);
         a.logits_ld = L.ld;
-        a.h = reinterpret_cast<float *>(base + L.h);
-        a.hmax = reinterpret_cast<uint32_t *>(base + L.hmax);
+        a.hterm = reinterpret_cast<unsigned char *>(base + L.hterm);
+        a.hsc = reinterpret_cast<float *>(base + L.hsc);
         a.counters = reinterpret_cast<int32_t *>(base + L.counters);
         const cudaError_t e = launch_decode_step(a, s);
         if (e != cudaSuccess) return finish(e);

@@ -99,7 +99,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 // 32 lanes x 32 columns of 32-bit words from tensor memory: thread i of the
 // warp gets lane (base lane + i), columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, float (&v)[32])

@@ -93,3 +93,29 @@ def test_bf16_splits_exactly_into_three_e5m2_terms():
     assert np.all(err[big] == 0.0)
     assert np.all(err[~big] <= 2.0 ** -17)
     assert np.any(err[~big] > 0.0)  # the bound is reached: the floor is real
+
+
+def test_fp32_splits_into_eight_e5m2_terms():
+    """The decode step feeds h (fp32) to the tensor cores as eight e5m2 terms
+    per value after a power-of-two scale that puts the block's largest
+    magnitude in [2^14, 2^15): t_k = e5m2(h' - t_1 - ... - t_(k-1)), each
+    difference taken in fp32 as the kernel does.  The terms sum exactly to h'
+    for every fp32 value with h' >= 2^7 (within 2^8 of the block maximum),
+    and to within 2^-17 of h' below that, i.e. under 2^-31 of the block
+    maximum.  Checked on random fp32 mantissas at every exponent of the scaled
+    range and below it."""
+    rng = np.random.default_rng(5)
+    mant = rng.integers(0, 1 << 23, size=4000, dtype=np.uint32)
+    exps = np.arange(127 - 30, 127 + 15, dtype=np.uint32)  # 2^-30 .. 2^14
+    bits = (exps[:, None] << 23) | mant[None, :]
+    hs = bits.ravel().view(np.float32).astype(np.float64)
+    r = hs.astype(np.float32)
+    total = np.zeros_like(hs)
+    for _ in range(8):
+        t = _e5m2(r)
+        total += t
+        r = (r - t.astype(np.float32)).astype(np.float32)
+    err = np.abs(total - hs)
+    big = hs >= 2.0 ** 7
+    assert np.all(err[big] == 0.0)
+    assert np.all(err[~big] <= 2.0 ** -17)
