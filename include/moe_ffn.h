@@ -254,6 +254,24 @@ MOE_API int moe_debug_wait_timeout_static(int32_t limit_us, void *stream);
 /* Size in bytes of the scratch array moe_ffn_forward_static uses. */
 MOE_API size_t moe_static_scratch_bytes(void);
 
+/* moe_ffn_forward with x and out in host memory: the step a serving loop
+ * makes when its tokens live on the host.  x [rows, H] and out [rows, H]
+ * (bf16, 16-byte aligned) must be pinned host memory that the device can
+ * address (cudaHostAlloc / cudaHostRegister; a pinned torch tensor): a first
+ * kernel reads x into the workspace over the host link, the forward's
+ * kernels then run as in moe_ffn_forward (path MOE_PATH_AUTO, no residual)
+ * and store out straight into the host buffer.  The caller keeps ownership
+ * of x and out; out is complete once the stream has passed the call (as for
+ * any kernel output: synchronise or wait on an event before reading it).
+ * The operation is moe_ffn_forward's (the blueprint page's Kernels table).
+ * Errors: as moe_ffn_forward, plus MOE_EINVAL when x or out is not pinned,
+ * device-addressable host memory. */
+MOE_API int moe_ffn_forward_host(const moe_dims *d, const uint16_t *x_host, int32_t rows,
+                         const uint16_t *router_w, const uint8_t *expert_w8,
+                         const float *expert_scales, const moe_fp8_expert *shared_w,
+                         const uint16_t *shared_gate, uint16_t *out_host,
+                         const float *router_bias, void *ws, size_t ws_bytes, void *stream);
+
 /* Sticky status: MOE_OK, or MOE_ECUDA after a CUDA error. */
 MOE_API int moe_status(void);
 /* Clear the sticky status (also clears a pending CUDA error of this thread). */

@@ -47,7 +47,7 @@ EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe
             "moe_debug_inject_fault", "moe_kernel_launches", "moe_auto_path", "moe_ffn_forward_timed",
             "moe_device_status", "moe_debug_wait_timeout", "moe_ffn_forward_static",
             "moe_static_scratch_bytes", "moe_static_device_status", "moe_debug_wait_timeout_static",
-            "moe_ffn_forward_norm")
+            "moe_ffn_forward_norm", "moe_ffn_forward_host")
 
 
 class MoeDims(ctypes.Structure):
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
                                            P, ctypes.c_size_t, P, I32, P, P, P]
         L.moe_ffn_forward_norm.argtypes = [DP, P, I32, P, ctypes.c_float, P, P, P, ctypes.POINTER(MoeFp8Expert), P,
                                            P, P, P, ctypes.c_size_t, P, I32]
+        L.moe_ffn_forward_host.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P,
+                                           ctypes.c_size_t, P]
         L.moe_kernel_launches.argtypes = [DP, I32, I32]
         L.moe_kernel_launches.restype = I32
         L.moe_auto_path.argtypes = [DP, I32]
@@ -201,6 +203,20 @@ def ffn_forward_path(dims, x, router_w, expert_w8, expert_scales, shared_w8, sha
                                       ws.numel() * ws.element_size(), _stream(stream), int(path),
                                       _ptr(topk_idx), _ptr(topk_w), _ptr(shared_gate_sig)),
            "moe_ffn_forward_path")
+
+
+def ffn_forward_host(dims, x_host, router_w, expert_w8, expert_scales, shared_w8, shared_scales, shared_gate,
+                     out_host, ws, router_bias=None, stream=None):
+    """ffn_forward with x_host and out_host pinned CPU tensors (bf16 [rows, H]):
+    the GPU reads x and writes out over the host link; out_host is complete
+    once the stream has passed the call."""
+    d = _dims(dims)
+    sh = MoeFp8Expert(_ptr(shared_w8), _ptr(shared_scales))
+    _check(lib().moe_ffn_forward_host(ctypes.byref(d), _ptr(x_host), _rows(x_host), _ptr(router_w),
+                                      _ptr(expert_w8), _ptr(expert_scales), ctypes.byref(sh), _ptr(shared_gate),
+                                      _ptr(out_host), _ptr(router_bias), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_ffn_forward_host")
 
 
 def ffn_forward_norm(dims, resid, norm_w, eps, router_w, expert_w8, expert_scales, shared_w8, shared_scales,

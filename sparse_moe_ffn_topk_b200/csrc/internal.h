@@ -144,6 +144,9 @@ struct StepLaunch {
     int32_t *counters;
 };
 cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t s);
+// host_io.cu: bytes (a multiple of 16) from pinned host memory (its device
+// address) to dst, by a kernel.
+cudaError_t launch_host_rows_in(const void *src_dev, void *dst, size_t bytes, cudaStream_t s);
 
 // x = bf16(rmsnorm(resid) * norm_w) for `rows` rows (one CTA per row).
 cudaError_t launch_rmsnorm(const uint16_t *resid, const uint16_t *norm_w, double eps, int H, int rows, uint16_t *x,

@@ -305,6 +305,43 @@ int moe_ffn_forward(const moe_dims *d, const uint16_t *x, int32_t rows, const ui
                                 nullptr, nullptr);
 }
 
+// The device address of pinned, device-addressable host memory, else null.
+static void *host_device_address(const void *p)
+{
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // a plain host pointer: not an error to keep
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
+int moe_ffn_forward_host(const moe_dims *d, const uint16_t *x_host, int32_t rows, const uint16_t *router_w,
+                         const uint8_t *expert_w8, const float *expert_scales, const moe_fp8_expert *shared_w,
+                         const uint16_t *shared_gate, uint16_t *out_host, const float *router_bias, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    int st = check_forward_args(d, x_host, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate,
+                                out_host, nullptr, router_bias, MOE_PATH_AUTO, nullptr, nullptr, nullptr, false);
+    if (st) return st;
+    if (rows == 0) return enter();  // a no-op: no pointer is read
+    if (!ws || !aligned16(ws)) return MOE_EINVAL;
+    if (ws_bytes < workspace_bytes(*d, rows)) return MOE_EWORKSPACE;
+    const void *xd = host_device_address(x_host);
+    void *od = host_device_address(out_host);
+    if (!xd || !od || !aligned16(xd) || !aligned16(od)) return MOE_EINVAL;
+    st = enter();
+    if (st) return st;
+    // x into the workspace's row buffer (the one the normalised entry uses)
+    uint16_t *xs = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + norm_buffer_offset(*d, rows));
+    const cudaError_t e =
+        launch_host_rows_in(xd, xs, (size_t)rows * d->hidden * 2, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return finish(e);
+    return run_forward(d, xs, rows, router_w, expert_w8, expert_scales, shared_w, shared_gate,
+                       static_cast<uint16_t *>(od), nullptr, router_bias, ws, stream, MOE_PATH_AUTO, nullptr,
+                       nullptr, nullptr, nullptr, 0.0);
+}
+
 int32_t moe_auto_path(const moe_dims *d, int32_t rows)
 {
     if (check_dims(d) != MOE_OK || rows < 0) return MOE_EINVAL;

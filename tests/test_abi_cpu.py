@@ -189,3 +189,29 @@ def test_static_entry_respects_sticky_status_and_fault_knob(L):
     assert L.moe_static_device_status(None) == moe.MOE_ECUDA
     moe.reset_status()
     assert moe.status() == moe.MOE_OK
+
+
+def host_fwd(L, d, rows=1, x=FAKE, out=FAKE + 4096, ws=FAKE, ws_bytes=None):
+    sh = moe.MoeFp8Expert(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE))
+    if ws_bytes is None:
+        ws_bytes = moe.workspace_bytes(d, max(rows, 1))
+    P = lambda a: ctypes.c_void_p(a) if a else None
+    return L.moe_ffn_forward_host(ctypes.byref(d), P(x), rows, P(FAKE), P(FAKE), P(FAKE), ctypes.byref(sh),
+                                  P(FAKE), P(out), None, P(ws), ws_bytes, None)
+
+
+def test_host_entry_rejects_memory_the_device_cannot_address(L):
+    """moe_ffn_forward_host takes pinned host buffers only: ordinary host
+    memory (here a ctypes array) is refused on the host, before anything is
+    enqueued, as are the forward's own argument errors."""
+    moe.reset_status()
+    d = D()
+    buf = (ctypes.c_uint8 * (2 * 4096 + 16))()
+    a = (ctypes.addressof(buf) + 15) // 16 * 16
+    assert host_fwd(L, d, x=a, out=a + 4096) == moe.MOE_EINVAL     # not pinned
+    assert host_fwd(L, d, x=0) == moe.MOE_EINVAL
+    assert host_fwd(L, d, x=FAKE + 2) == moe.MOE_EINVAL            # misaligned
+    assert host_fwd(L, d, out=FAKE) == moe.MOE_EINVAL              # out aliases x
+    assert host_fwd(L, d, ws_bytes=16) == moe.MOE_EWORKSPACE
+    assert host_fwd(L, d, rows=0) == moe.MOE_OK                    # a no-op
+    assert moe.status() == moe.MOE_OK
