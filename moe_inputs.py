@@ -25,6 +25,15 @@ torch's own e4m3 conversion (a library cast, round-to-nearest-even) of
 w / s with s = amax/448 per block; the oracle has its own, independent
 quantiser, and a test checks that the two agree bit for bit.
 
+NVFP4 experts (make_layer_nvfp4; the 397B-A17B checkpoint's expert format):
+the same fp32 weights stored as e2m1 codes packed two to a byte (element 2j
+in the low nibble of byte j), one e4m3 scale per 16 consecutive elements of
+a row and one fp32 scale per matrix, through library casts (torch's e4m3,
+ml_dtypes' e2m1, both round-to-nearest-even); the oracle has its own
+quantiser, checked against these bytes.  Slab per expert: codes ``[W13 (2I x
+H/2) | W2 (H x I/2)]``, scales ``[W13 (2I x H/16) | W2 (H x I/16)]``, tensor
+scales ``[gs13, gs2]``.
+
 Every tensor has its own generator, seeded from (seed, tensor name, index),
 so any single expert can be regenerated alone; tests that only need the
 experts a routing touches generate just those and leave the others zero.
@@ -110,6 +119,28 @@ def encode_e4m3_blocks(w: torch.Tensor):
     return q.reshape(R, C).view(torch.uint8).numpy().copy(), s.numpy().copy()
 
 
+def encode_nvfp4(w: torch.Tensor):
+    """Store an fp32 [R, C] matrix (C a multiple of 16) as NVFP4: gs =
+    amax/(448*6) (1 for an all-zero matrix); per 16 elements of a row, the
+    scale code = torch's e4m3 cast of amax16/(6*gs); element codes =
+    ml_dtypes' e2m1 cast of w/(e4m3(scale)*gs) (divisor and quotient in fp32;
+    0 under a zero scale).  -> (packed codes uint8 [R, C/2], scale codes uint8
+    [R, C/16], gs float)."""
+    import ml_dtypes
+
+    R, C = w.shape
+    amax = float(w.abs().max())
+    gs = np.float32(1.0) if amax == 0.0 else np.float32(amax) / np.float32(448.0 * 6.0)
+    b = w.reshape(R, C // 16, 16)
+    bmax = b.abs().amax(dim=2)
+    sf = (bmax / torch.tensor(np.float32(6.0) * gs, dtype=torch.float32)).to(torch.float8_e4m3fn)
+    div = sf.to(torch.float32) * torch.tensor(gs, dtype=torch.float32)
+    q = torch.where(div[:, :, None] == 0, torch.zeros_like(b), b / div[:, :, None])
+    codes = q.numpy().astype(ml_dtypes.float4_e2m1fn).view(np.uint8).reshape(R, C) & 0x0F
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed.copy(), sf.view(torch.uint8).numpy().copy(), float(gs)
+
+
 def expert_slab(dims: LayerDims, seed: int, e: int, inter: int | None = None, name: str = "expert"):
     """(codes uint8 [3*I*H], scales fp32 [n]) for one expert (e = -1: shared)."""
     H = dims.hidden
@@ -164,6 +195,59 @@ def make_layer(dims: LayerDims, seed: int = 0, router_bias: bool = False, expert
             list(ex.map(one, ids))
     sq, ss = expert_slab(dims, seed, -1, inter=dims.shared_inter, name="shared")
     return Layer(dims, seed, rw, g, w8, sc, sq, ss, b, frozenset(ids))
+
+
+def expert_slab_nvfp4(dims: LayerDims, seed: int, e: int, inter: int | None = None, name: str = "expert"):
+    """(packed codes uint8 [3*I*H/2], scale codes uint8 [3*I*H/16], tensor
+    scales fp32 [2]) for one expert (e = -1: shared): the same fp32 weights as
+    expert_slab, stored as NVFP4."""
+    H = dims.hidden
+    I = inter if inter is not None else dims.inter
+    w13 = _normal((2 * I, H), 0.02, seed, name + ".w13", e)
+    w2 = _normal((H, I), 0.02, seed, name + ".w2", e)
+    q13, f13, g13 = encode_nvfp4(w13)
+    q2, f2, g2 = encode_nvfp4(w2)
+    return (np.concatenate([q13.reshape(-1), q2.reshape(-1)]), np.concatenate([f13.reshape(-1), f2.reshape(-1)]),
+            np.array([g13, g2], dtype=np.float32))
+
+
+@dataclass
+class LayerNvfp4:
+    dims: LayerDims
+    seed: int
+    router_w: np.ndarray       # uint16 [E, H]
+    shared_gate: np.ndarray    # uint16 [H]
+    expert_w4: np.ndarray      # uint8  [E, 3*I*H/2]  packed e2m1 codes
+    expert_sf: np.ndarray      # uint8  [E, 3*I*H/16] e4m3 scale codes
+    expert_gs: np.ndarray      # fp32   [E, 2]
+    shared_w4: np.ndarray      # uint8  [3*Is*H/2]
+    shared_sf: np.ndarray      # uint8  [3*Is*H/16]
+    shared_gs: np.ndarray      # fp32   [2]
+    router_bias: np.ndarray | None = None
+    generated: frozenset = field(default_factory=frozenset)
+
+
+def make_layer_nvfp4(dims: LayerDims, seed: int = 0, router_bias: bool = False, experts=None,
+                     threads: int | None = None) -> LayerNvfp4:
+    """make_layer's weights stored as NVFP4 experts (the router, gate and
+    bias are the same).  Experts not drawn are zero codes and scales with unit
+    tensor scales."""
+    rw, g, b = make_router(dims, seed, router_bias)
+    E, H, I = dims.n_experts, dims.hidden, dims.inter
+    ids = list(range(E)) if experts is None else sorted(set(int(e) for e in experts))
+    w4 = np.zeros((E, 3 * I * H // 2), dtype=np.uint8)
+    sf = np.zeros((E, 3 * I * H // 16), dtype=np.uint8)
+    gs = np.ones((E, 2), dtype=np.float32)
+
+    def one(e):
+        w4[e], sf[e], gs[e] = expert_slab_nvfp4(dims, seed, e)
+
+    nthr = threads or min(32, os.cpu_count() or 1)
+    if ids:
+        with ThreadPoolExecutor(nthr) as ex:
+            list(ex.map(one, ids))
+    sw, ssf, sgs = expert_slab_nvfp4(dims, seed, -1, inter=dims.shared_inter, name="shared")
+    return LayerNvfp4(dims, seed, rw, g, w4, sf, gs, sw, ssf, sgs, b, frozenset(ids))
 
 
 def make_x(dims: LayerDims, rows: int, seed: int = 0, stream: int = 0) -> np.ndarray:

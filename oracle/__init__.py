@@ -64,6 +64,14 @@ def _load():
         lib.oracle_rmsnorm.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
         lib.oracle_moe_forward_dense.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, P, P,
                                                  P, P, P, P, P, P, P, P, P, P, ctypes.c_int32]
+        lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_encode.argtypes = [ctypes.c_double]
+        lib.oracle_e2m1_encode.restype = ctypes.c_uint8
+        lib.oracle_quantize_nvfp4.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, P, P]
+        lib.oracle_expert_ffn_nvfp4.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, P, P]
+        lib.oracle_moe_forward_nvfp4.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, P, P, P, P, P, P, P,
+                                                 P, P, P, P, ctypes.c_int32, P, P, P, P, P, ctypes.c_int32]
         _lib = lib
     return _lib
 
@@ -98,6 +106,14 @@ def e4m3_encode(v: float) -> int:
     return int(_load().oracle_e4m3_encode(float(v)))
 
 
+def e2m1_decode(code: int) -> float:
+    return _load().oracle_e2m1_decode(int(code))
+
+
+def e2m1_encode(v: float) -> int:
+    return int(_load().oracle_e2m1_encode(float(v)))
+
+
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Element-wise nearest bf16 (ties to even) of a float64 array, as uint16 bits."""
     f = np.vectorize(lambda v: _load().oracle_f64_to_bf16(float(v)), otypes=[np.uint16])
@@ -119,6 +135,60 @@ def quantize_blocks(w: np.ndarray):
     s = np.empty((R // 128, C // 128), dtype=np.float32)
     _check(_load().oracle_quantize_blocks(_ptr(w), R, C, _ptr(q), _ptr(s)), "oracle_quantize_blocks")
     return q, s
+
+
+def quantize_nvfp4(w: np.ndarray):
+    """Oracle NVFP4 quantiser: fp32 [R, C] (C a multiple of 16) -> (packed e2m1
+    codes uint8 [R, C/2] (element 2j in the low nibble of byte j), e4m3 block
+    scale codes uint8 [R, C/16], fp32 tensor scale)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    R, C = w.shape
+    q = np.zeros((R, C // 2), dtype=np.uint8)
+    sf = np.empty((R, C // 16), dtype=np.uint8)
+    gs = np.empty(1, dtype=np.float32)
+    _check(_load().oracle_quantize_nvfp4(_ptr(w), R, C, _ptr(q), _ptr(sf), _ptr(gs)), "oracle_quantize_nvfp4")
+    return q, sf, float(gs[0])
+
+
+def expert_ffn_nvfp4(w4, sf, gs, H: int, I: int, x: np.ndarray) -> np.ndarray:
+    """One SwiGLU expert with NVFP4 weights (slab layout of moe_inputs), x float64 [H] -> y [H]."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty(H, dtype=np.float64)
+    _check(_load().oracle_expert_ffn_nvfp4(_ptr(np.ascontiguousarray(w4, dtype=np.uint8)),
+                                           _ptr(np.ascontiguousarray(sf, dtype=np.uint8)),
+                                           _ptr(np.ascontiguousarray(gs, dtype=np.float32)), H, I, _ptr(x),
+                                           _ptr(y)), "oracle_expert_ffn_nvfp4")
+    return y
+
+
+def moe_forward_nvfp4(d, x, router_w, expert_w4, expert_sf, expert_gs, shared_w4, shared_sf, shared_gs,
+                      shared_gate, residual=None, router_bias=None, forced_idx=None, dense=False,
+                      want_logits=True, nthreads: int | None = None) -> ForwardResult:
+    """The layer with NVFP4 experts in double (routed; or, dense=True, every
+    expert under the top-k mask)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    rows = x.shape[0]
+    out = np.empty((rows, d.hidden), dtype=np.float64)
+    idx = np.empty((rows, d.top_k), dtype=np.int32)
+    w = np.empty((rows, d.top_k), dtype=np.float64)
+    gs = np.empty(rows, dtype=np.float64)
+    logits = np.empty((rows, d.n_experts), dtype=np.float64) if (want_logits and not dense) else None
+    if forced_idx is not None:
+        forced_idx = np.ascontiguousarray(forced_idx, dtype=np.int32)
+    dims = _dims(d)
+    rc = _load().oracle_moe_forward_nvfp4(
+        ctypes.byref(dims), _ptr(x), rows, _ptr(np.ascontiguousarray(router_w, dtype=np.uint16)),
+        _ptr(np.ascontiguousarray(expert_w4, dtype=np.uint8)), _ptr(np.ascontiguousarray(expert_sf, dtype=np.uint8)),
+        _ptr(np.ascontiguousarray(expert_gs, dtype=np.float32)),
+        _ptr(np.ascontiguousarray(shared_w4, dtype=np.uint8)), _ptr(np.ascontiguousarray(shared_sf, dtype=np.uint8)),
+        _ptr(np.ascontiguousarray(shared_gs, dtype=np.float32)),
+        _ptr(np.ascontiguousarray(shared_gate, dtype=np.uint16)),
+        _ptr(None if residual is None else np.ascontiguousarray(residual, dtype=np.uint16)),
+        _ptr(None if router_bias is None else np.ascontiguousarray(router_bias, dtype=np.float32)),
+        _ptr(forced_idx), 1 if dense else 0, _ptr(out), _ptr(idx), _ptr(w), _ptr(gs), _ptr(logits),
+        nthreads or os.cpu_count() or 1)
+    _check(rc, "oracle_moe_forward_nvfp4")
+    return ForwardResult(out, idx, w, gs, logits)
 
 
 def topk(logits: np.ndarray, k: int):

@@ -23,6 +23,13 @@
  *    up_proj are [I,H], down_proj is [H,I] (LLaMA-style SwiGLU).
  *  - OCP 8-bit Floating Point specification, E4M3: exponent bias 7, three
  *    mantissa bits, subnormals, no infinities, S.1111.111 is NaN, max 448.
+ *  - "The Config That Launched a Thousand GPUs: Inspecting
+ *    Qwen3.5-397B-A17B-NVFP4" page: the 397B checkpoint's experts are stored
+ *    in NVFP4 (modelopt).  The format (not on the pages; its public
+ *    definition): OCP MX E2M1 codes (one sign bit, two exponent bits with
+ *    bias 1, one mantissa bit, no infinities or NaN: 0, 0.5, 1, 1.5, 2, 3,
+ *    4, 6), one E4M3 scale per 16 consecutive elements along the reduction
+ *    dimension, one fp32 scale per tensor.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - top-k ties go to the lower expert index; output order is by descending
@@ -172,6 +179,100 @@ static double dq(const uint8_t *q, const float *s, int64_t cols, int64_t r, int6
     return oracle_e4m3_decode(q[r * cols + c]) * (double)s[(r / 128) * (cols / 128) + (c / 128)];
 }
 
+/* ------------------------------------------------------------- NVFP4 */
+
+/* OCP MX E2M1: code = s.ee.m, exponent bias 1; e = 0 is subnormal (m * 0.5). */
+double oracle_e2m1_decode(uint8_t code)
+{
+    int s = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double v = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, e - 1);
+    return s ? -v : v;
+}
+
+/* Nearest e2m1 value, ties to the even code (even mantissa), saturating to
+ * +-6; codes 0..7 have strictly increasing values (binary search, as for
+ * e4m3).  NaN maps to 0. */
+uint8_t oracle_e2m1_encode(double v)
+{
+    if (isnan(v)) return 0;
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    double a = fabs(v);
+    if (a >= 6.0) return (uint8_t)(sign | 0x7);
+    int lo = 0, hi = 7; /* invariant: decode(lo) <= a < decode(hi) */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (oracle_e2m1_decode((uint8_t)mid) <= a)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    double dl = a - oracle_e2m1_decode((uint8_t)lo);
+    double dh = oracle_e2m1_decode((uint8_t)hi) - a;
+    int c;
+    if (dl < dh)
+        c = lo;
+    else if (dh < dl)
+        c = hi;
+    else
+        c = (lo % 2 == 0) ? lo : hi;
+    return (uint8_t)(sign | c);
+}
+
+/* NVFP4 quantiser for a row-major fp32 matrix [rows, cols], cols a multiple
+ * of 16 (reading of the format: the tensor scale maps the largest magnitude
+ * to the largest e4m3 scale times the largest e2m1 value):
+ *   gs = amax / (448 * 6) in fp32 (1 for an all-zero matrix);
+ *   per 16 consecutive elements of a row: sf = e4m3(amax16 / (6 * gs)),
+ *     quotient in fp32;
+ *   code = e2m1(w / (e4m3(sf) * gs)), divisor and quotient in fp32 (a zero
+ *     block scale gives code 0);
+ * codes packed two to a byte, element 2j in the low nibble of byte j:
+ * q4 [rows, cols/2], sf [rows, cols/16] e4m3 codes, *gs. */
+int oracle_quantize_nvfp4(const float *w, int64_t rows, int64_t cols, uint8_t *q4, uint8_t *sf, float *gs)
+{
+    if (cols % 16) return -2;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < rows * cols; ++i)
+        if (fabsf(w[i]) > amax) amax = fabsf(w[i]);
+    const float g = (amax == 0.0f) ? 1.0f : amax / (448.0f * 6.0f);
+    *gs = g;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < cols / 16; ++b) {
+            float bmax = 0.0f;
+            for (int64_t c = b * 16; c < b * 16 + 16; ++c)
+                if (fabsf(w[r * cols + c]) > bmax) bmax = fabsf(w[r * cols + c]);
+            const float sq = bmax / (6.0f * g);
+            const uint8_t sc = oracle_e4m3_encode((double)sq);
+            sf[r * (cols / 16) + b] = sc;
+            const float div = (float)oracle_e4m3_decode(sc) * g;
+            for (int64_t c = b * 16; c < b * 16 + 16; ++c) {
+                uint8_t code = 0;
+                if (div != 0.0f) {
+                    const float qv = w[r * cols + c] / div;
+                    code = oracle_e2m1_encode((double)qv);
+                }
+                uint8_t *byte = &q4[r * (cols / 2) + c / 2];
+                if (c % 2 == 0)
+                    *byte = (uint8_t)((*byte & 0xF0) | code);
+                else
+                    *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* Dequantised weight of a [rows, cols] NVFP4 matrix: e2m1(code) * e4m3(sf)
+ * * gs. */
+static double dq4(const uint8_t *q4, const uint8_t *sf, double gs, int64_t cols, int64_t r, int64_t c)
+{
+    const uint8_t byte = q4[r * (cols / 2) + c / 2];
+    const uint8_t code = (c % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+    return oracle_e2m1_decode(code) * oracle_e4m3_decode(sf[r * (cols / 16) + c / 16]) * gs;
+}
+
 /* ------------------------------------------------------------- RMSNorm */
 
 /* The norm in front of the MoE block ("Qwen3.6-35B-A3B-FP8 on NVIDIA GB10"
@@ -302,6 +403,39 @@ int oracle_expert_ffn(const uint8_t *w8, const float *scales, int32_t H, int32_t
     return 0;
 }
 
+/* The SwiGLU expert with NVFP4 weights: the same formulas as
+ * oracle_expert_ffn with each weight e2m1(code) * e4m3(sf) * gs.  Slab
+ * layout: w4 = [W13 (2I x H/2) | W2 (H x I/2)] packed codes, sf = [W13
+ * (2I x H/16) | W2 (H x I/16)] e4m3 codes, gs = [gs13, gs2]. */
+int oracle_expert_ffn_nvfp4(const uint8_t *w4, const uint8_t *sf, const float *gs, int32_t H, int32_t I,
+                            const double *x, double *y)
+{
+    const uint8_t *w13 = w4;
+    const uint8_t *w2 = w4 + (int64_t)2 * I * H / 2;
+    const uint8_t *f13 = sf;
+    const uint8_t *f2 = sf + (int64_t)2 * I * H / 16;
+    double *gu = (double *)malloc(sizeof(double) * 2 * (size_t)I);
+    double *hv = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!gu || !hv) { free(gu); free(hv); return -1; }
+    for (int j = 0; j < 2 * I; ++j) {
+        double acc = 0.0;
+        for (int k = 0; k < H; ++k) acc += dq4(w13, f13, (double)gs[0], H, j, k) * x[k];
+        gu[j] = acc;
+    }
+    for (int j = 0; j < I; ++j) {
+        double g = gu[j];
+        hv[j] = g * sigmoid(g) * gu[I + j];
+    }
+    for (int n = 0; n < H; ++n) {
+        double acc = 0.0;
+        for (int j = 0; j < I; ++j) acc += dq4(w2, f2, (double)gs[1], I, n, j) * hv[j];
+        y[n] = acc;
+    }
+    free(gu);
+    free(hv);
+    return 0;
+}
+
 typedef struct {
     const oracle_dims *d;
     const uint16_t *x;
@@ -316,6 +450,11 @@ typedef struct {
     const float *router_bias;
     const int32_t *forced_idx;
     int dense;
+    int nvfp4;                  /* expert_w8/shared_w8 hold packed e2m1 codes */
+    const uint8_t *expert_sf;   /* NVFP4: e4m3 block scales, per expert */
+    const float *expert_gs;     /* NVFP4: [E][2] tensor scales */
+    const uint8_t *shared_sf;
+    const float *shared_gs;
     double *out;
     int32_t *idx;
     double *w;
@@ -329,6 +468,23 @@ static int64_t expert_bytes(const oracle_dims *d, int32_t I) { return (int64_t)3
 static int64_t expert_nscales(const oracle_dims *d, int32_t I)
 {
     return (int64_t)(2 * I / 128) * (d->hidden / 128) + (int64_t)(d->hidden / 128) * (I / 128);
+}
+
+/* Expert e (-1: shared) of a job applied to xr. */
+static int job_expert(const fwd_job *j, int e, const double *xr, double *y)
+{
+    const oracle_dims *d = j->d;
+    const int H = d->hidden;
+    if (j->nvfp4) {
+        const int32_t I = e < 0 ? d->shared_inter : d->inter;
+        if (e < 0) return oracle_expert_ffn_nvfp4(j->shared_w8, j->shared_sf, j->shared_gs, H, I, xr, y);
+        return oracle_expert_ffn_nvfp4(j->expert_w8 + (int64_t)e * 3 * I * H / 2,
+                                       j->expert_sf + (int64_t)e * 3 * I * H / 16, j->expert_gs + 2 * (int64_t)e,
+                                       H, I, xr, y);
+    }
+    if (e < 0) return oracle_expert_ffn(j->shared_w8, j->shared_scales, H, d->shared_inter, xr, y);
+    return oracle_expert_ffn(j->expert_w8 + (int64_t)e * expert_bytes(d, d->inter),
+                             j->expert_scales + (int64_t)e * expert_nscales(d, d->inter), H, d->inter, xr, y);
 }
 
 static void *fwd_worker(void *arg)
@@ -375,10 +531,7 @@ static void *fwd_worker(void *arg)
         if (!j->dense) {
             /* routed: the k selected experts, in rank order */
             for (int r = 0; r < K; ++r) {
-                int e = ix[r];
-                if (oracle_expert_ffn(j->expert_w8 + (int64_t)e * expert_bytes(d, d->inter),
-                                      j->expert_scales + (int64_t)e * expert_nscales(d, d->inter),
-                                      H, d->inter, xr, y)) { j->status = -1; goto done; }
+                if (job_expert(j, ix[r], xr, y)) { j->status = -1; goto done; }
                 for (int h = 0; h < H; ++h) acc[h] += wv[r] * y[h];
             }
         } else {
@@ -387,14 +540,12 @@ static void *fwd_worker(void *arg)
             for (int e = 0; e < E; ++e) mask[e] = 0.0;
             for (int r = 0; r < K; ++r) mask[ix[r]] = wv[r];
             for (int e = 0; e < E; ++e) {
-                if (oracle_expert_ffn(j->expert_w8 + (int64_t)e * expert_bytes(d, d->inter),
-                                      j->expert_scales + (int64_t)e * expert_nscales(d, d->inter),
-                                      H, d->inter, xr, y)) { j->status = -1; goto done; }
+                if (job_expert(j, e, xr, y)) { j->status = -1; goto done; }
                 for (int h = 0; h < H; ++h) acc[h] += mask[e] * y[h];
             }
         }
         /* shared expert, scaled by its sigmoid gate */
-        if (oracle_expert_ffn(j->shared_w8, j->shared_scales, H, d->shared_inter, xr, y)) {
+        if (job_expert(j, -1, xr, y)) {
             j->status = -1;
             goto done;
         }
@@ -417,19 +568,29 @@ static int check_dims(const oracle_dims *d)
     return 0;
 }
 
+typedef struct {
+    const uint8_t *expert_sf;
+    const float *expert_gs;
+    const uint8_t *shared_sf;
+    const float *shared_gs;
+} nvfp4_scales;
+
 static int run_forward(const oracle_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
                        const uint8_t *expert_w8, const float *expert_scales,
                        const uint8_t *shared_w8, const float *shared_scales,
                        const uint16_t *shared_gate, const uint16_t *residual,
                        const float *router_bias, const int32_t *forced_idx, int dense,
                        double *out, int32_t *idx, double *w, double *gate_sig, double *logits,
-                       int32_t nthreads)
+                       int32_t nthreads, const nvfp4_scales *f4)
 {
     int st = check_dims(d);
     if (st) return st;
-    if (!x || !router_w || !expert_w8 || !expert_scales || !shared_w8 || !shared_scales ||
-        !shared_gate || !out || !idx || !w || !gate_sig || rows < 0)
+    if (!x || !router_w || !expert_w8 || !shared_w8 || !shared_gate || !out || !idx || !w || !gate_sig || rows < 0)
         return -1;
+    if (f4 ? (!f4->expert_sf || !f4->expert_gs || !f4->shared_sf || !f4->shared_gs)
+           : (!expert_scales || !shared_scales))
+        return -1;
+    if (f4 && (d->hidden % 16 || d->inter % 16 || d->shared_inter % 16)) return -2;
     if (rows == 0) return 0;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = rows;
@@ -443,6 +604,11 @@ static int run_forward(const oracle_dims *d, const uint16_t *x, int32_t rows, co
         j->shared_w8 = shared_w8; j->shared_scales = shared_scales;
         j->shared_gate = shared_gate; j->residual = residual; j->router_bias = router_bias;
         j->forced_idx = forced_idx; j->dense = dense;
+        if (f4) {
+            j->nvfp4 = 1;
+            j->expert_sf = f4->expert_sf; j->expert_gs = f4->expert_gs;
+            j->shared_sf = f4->shared_sf; j->shared_gs = f4->shared_gs;
+        }
         j->out = out; j->idx = idx; j->w = w; j->gate_sig = gate_sig; j->logits = logits;
         j->row_begin = (int32_t)((int64_t)rows * i / nthreads);
         j->row_end = (int32_t)((int64_t)rows * (i + 1) / nthreads);
@@ -482,7 +648,7 @@ int oracle_moe_forward(const oracle_dims *d, const uint16_t *x, int32_t rows, co
 {
     return run_forward(d, x, rows, router_w, expert_w8, expert_scales, shared_w8, shared_scales,
                        shared_gate, residual, router_bias, forced_idx, 0, out, idx, w, gate_sig,
-                       logits, nthreads);
+                       logits, nthreads, NULL);
 }
 
 /* The same layer by brute force: all E experts evaluated for every row and
@@ -497,5 +663,24 @@ int oracle_moe_forward_dense(const oracle_dims *d, const uint16_t *x, int32_t ro
 {
     return run_forward(d, x, rows, router_w, expert_w8, expert_scales, shared_w8, shared_scales,
                        shared_gate, residual, router_bias, NULL, 1, out, idx, w, gate_sig, NULL,
-                       nthreads);
+                       nthreads, NULL);
+}
+
+/* The layer with NVFP4 experts (routed, or dense brute force when dense is
+ * non-zero): oracle_moe_forward's formulas with each weight e2m1(code) *
+ * e4m3(sf) * gs.  expert_w4 [E][3*I*H/2] packed codes, expert_sf
+ * [E][3*I*H/16] e4m3 scale codes, expert_gs [E][2] (W13, W2); the shared
+ * expert likewise with Is. */
+int oracle_moe_forward_nvfp4(const oracle_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                             const uint8_t *expert_w4, const uint8_t *expert_sf, const float *expert_gs,
+                             const uint8_t *shared_w4, const uint8_t *shared_sf, const float *shared_gs,
+                             const uint16_t *shared_gate, const uint16_t *residual,
+                             const float *router_bias, const int32_t *forced_idx, int32_t dense,
+                             double *out, int32_t *idx, double *w, double *gate_sig, double *logits,
+                             int32_t nthreads)
+{
+    nvfp4_scales f4 = {expert_sf, expert_gs, shared_sf, shared_gs};
+    return run_forward(d, x, rows, router_w, expert_w4, NULL, shared_w4, NULL, shared_gate, residual,
+                       router_bias, dense ? NULL : forced_idx, dense ? 1 : 0, out, idx, w, gate_sig,
+                       dense ? NULL : logits, nthreads, &f4);
 }
