@@ -105,6 +105,16 @@ typedef struct moe_fp8_expert {
     const float *scales;  /* (2Is/128)(H/128) + (H/128)(Is/128) fp32 scales */
 } moe_fp8_expert;
 
+/* One NVFP4 expert (the shared one): packed e2m1 codes [W13 (2Is x H/2) |
+ * W2 (H x Is/2)] (element 2j of a row in the low nibble of byte j), e4m3
+ * block scale codes [W13 (2Is x H/16) | W2 (H x Is/16)] (one per 16
+ * consecutive elements of a row), fp32 tensor scales [2] (W13, W2). */
+typedef struct moe_nvfp4_expert {
+    const uint8_t *w4;
+    const uint8_t *sf;
+    const float *gs;
+} moe_nvfp4_expert;
+
 /* Bytes of workspace needed by any call with rows <= max_rows on either path.
  * Returns 0 for invalid or unsupported dims or max_rows < 0. */
 MOE_API size_t moe_workspace_bytes(const moe_dims *d, int32_t max_rows);
@@ -271,6 +281,29 @@ MOE_API int moe_ffn_forward_host(const moe_dims *d, const uint16_t *x_host, int3
                          const float *expert_scales, const moe_fp8_expert *shared_w,
                          const uint16_t *shared_gate, uint16_t *out_host,
                          const float *router_bias, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_ffn_forward with NVFP4 experts: the 397B-A17B checkpoint's expert
+ * format ("The Config That Launched a Thousand GPUs: Inspecting
+ * Qwen3.5-397B-A17B-NVFP4" page, modelopt NVFP4; the format is its public
+ * definition): weight = e2m1(code) * e4m3(block scale) * tensor scale.  The
+ * operation is the blueprint page's Kernels chain (router GEMV, top-k
+ * softmax, gate/up with the shared expert, SiLU and down, weighted blend)
+ * at its Precision table's arithmetic (bf16 x for gate/up, f32 h for down,
+ * fp32 sums).  Layout: E contiguous expert slabs; expert_w4 [E][3*I*H/2]
+ * packed codes ([W13 (2I x H/2) | W2 (H x I/2)], element 2j of a row in the
+ * low nibble of byte j), expert_sf [E][3*I*H/16] e4m3 scale codes ([W13 (2I x
+ * H/16) | W2 (H x I/16)]), expert_gs [E][2] fp32 (W13, W2); the shared expert
+ * likewise (moe_nvfp4_expert).  The router, gate, bias, residual and out are
+ * those of moe_ffn_forward; workspace as moe_workspace_bytes(d, rows).  A
+ * decode-sized path: the weights stream once per row and routed pair, rows
+ * in chunks of up to 4.  Errors: as moe_ffn_forward (pointers 16-byte
+ * aligned, expert_gs and shared->gs 4-byte aligned). */
+MOE_API int moe_ffn_forward_nvfp4(const moe_dims *d, const uint16_t *x, int32_t rows,
+                          const uint16_t *router_w, const uint8_t *expert_w4,
+                          const uint8_t *expert_sf, const float *expert_gs,
+                          const moe_nvfp4_expert *shared, const uint16_t *shared_gate,
+                          uint16_t *out, const uint16_t *residual, const float *router_bias,
+                          void *ws, size_t ws_bytes, void *stream);
 
 /* Sticky status: MOE_OK, or MOE_ECUDA after a CUDA error. */
 MOE_API int moe_status(void);

@@ -47,7 +47,11 @@ EXPORTED = ("moe_workspace_bytes", "moe_workspace_init", "moe_router_topk", "moe
             "moe_debug_inject_fault", "moe_kernel_launches", "moe_auto_path", "moe_ffn_forward_timed",
             "moe_device_status", "moe_debug_wait_timeout", "moe_ffn_forward_static",
             "moe_static_scratch_bytes", "moe_static_device_status", "moe_debug_wait_timeout_static",
-            "moe_ffn_forward_norm", "moe_ffn_forward_host")
+            "moe_ffn_forward_norm", "moe_ffn_forward_host", "moe_ffn_forward_nvfp4")
+
+
+class MoeNvfp4Expert(ctypes.Structure):
+    _fields_ = [("w4", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("gs", ctypes.c_void_p)]
 
 
 class MoeDims(ctypes.Structure):
@@ -94,6 +98,8 @@ def lib() -> ctypes.CDLL:
                                            P, P, P, ctypes.c_size_t, P, I32]
         L.moe_ffn_forward_host.argtypes = [DP, P, I32, P, P, P, ctypes.POINTER(MoeFp8Expert), P, P, P, P,
                                            ctypes.c_size_t, P]
+        L.moe_ffn_forward_nvfp4.argtypes = [DP, P, I32, P, P, P, P, ctypes.POINTER(MoeNvfp4Expert), P, P, P, P, P,
+                                            ctypes.c_size_t, P]
         L.moe_kernel_launches.argtypes = [DP, I32, I32]
         L.moe_kernel_launches.restype = I32
         L.moe_auto_path.argtypes = [DP, I32]
@@ -217,6 +223,20 @@ def ffn_forward_host(dims, x_host, router_w, expert_w8, expert_scales, shared_w8
                                       _ptr(out_host), _ptr(router_bias), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)),
            "moe_ffn_forward_host")
+
+
+def ffn_forward_nvfp4(dims, x, router_w, expert_w4, expert_sf, expert_gs, shared_w4, shared_sf, shared_gs,
+                      shared_gate, out, ws, residual=None, router_bias=None, stream=None):
+    """The layer with NVFP4 experts (packed e2m1 codes, e4m3 block scales per 16
+    elements, fp32 tensor scales [E, 2]); device tensors in moe_inputs' slab
+    layout."""
+    d = _dims(dims)
+    sh = MoeNvfp4Expert(_ptr(shared_w4), _ptr(shared_sf), _ptr(shared_gs))
+    _check(lib().moe_ffn_forward_nvfp4(ctypes.byref(d), _ptr(x), _rows(x), _ptr(router_w), _ptr(expert_w4),
+                                       _ptr(expert_sf), _ptr(expert_gs), ctypes.byref(sh), _ptr(shared_gate),
+                                       _ptr(out), _ptr(residual), _ptr(router_bias), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_ffn_forward_nvfp4")
 
 
 def ffn_forward_norm(dims, resid, norm_w, eps, router_w, expert_w8, expert_scales, shared_w8, shared_scales,

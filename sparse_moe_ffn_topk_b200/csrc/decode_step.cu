@@ -650,7 +650,6 @@ __device__ __forceinline__ bool down_item_mma(const StepParams &p, uint32_t slot
             int ok = 1;
             if (lane == 0) ok = mbar_wait_spin(bbar, *bphase, kWaitLimitNs) ? 1 : 0;
             *bphase ^= 1u;
-            ITEM_T(40 + (threadIdx.x >> 5), 4);  // trace: the warp's last copy of h terms landed
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) return false;
             // a window (four chunks) at a time: n is a multiple of 4
             for (int i0 = 0; i0 < n; i0 += 4) {
@@ -739,7 +738,7 @@ __device__ __forceinline__ void down_phase(const StepParams &p, StepSmall &sm, u
                 }
                 break;
             }
-            ITEM_T(q, 3);
+            ITEM_T(48 + b, 0);  // (trace rows 48-63: down items in claim order) expert seen counted
             if (!wait_item(sm.tag, full, s, q, p.ns)) {
                 if (lane == 0) {
                     gave_up(p.counters, 3, q);
@@ -747,7 +746,7 @@ __device__ __forceinline__ void down_phase(const StepParams &p, StepSmall &sm, u
                 }
                 break;
             }
-            ITEM_T(q, 0);
+            ITEM_T(48 + b, 1);  // weight rows seen
             const bool shared = it.a == 0;
             const int de = shared ? 0 : 1 + (it.a - 1) * p.dn_epi;
             const int tpi = shared ? p.dn_tpi_s : p.dn_tpi;
@@ -771,7 +770,7 @@ __device__ __forceinline__ void down_phase(const StepParams &p, StepSmall &sm, u
                 }
                 break;
             }
-            ITEM_T(q, 1);
+            ITEM_T(48 + b, 2);  // done
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }

@@ -144,6 +144,28 @@ struct StepLaunch {
     int32_t *counters;
 };
 cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t s);
+// nvfp4.cu: the layer with NVFP4 experts (router, then per chunk of rows
+// gate/up and down + blend).
+struct Nvfp4Launch {
+    const moe_dims *d;
+    const uint16_t *x;
+    int32_t rows;
+    const uint16_t *router_w;
+    const float *router_bias;
+    const uint16_t *shared_gate;
+    const uint8_t *w4, *sf;   // experts: packed e2m1 codes, e4m3 block scales
+    const float *gs;          // [E][2]
+    const uint8_t *sw4, *ssf; // the shared expert
+    const float *sgs;
+    const uint16_t *residual;
+    uint16_t *out;
+    int32_t *topk_idx;        // workspace
+    float *topk_w, *gsig, *logits, *h;
+    int32_t *counters;
+};
+cudaError_t launch_nvfp4_forward(const Nvfp4Launch &a, cudaStream_t s);
+int nvfp4_rows_per_chunk(const moe_dims &d);
+int nvfp4_kernel_launches(const moe_dims &d, int32_t rows);
 // host_io.cu: bytes (a multiple of 16) from pinned host memory (its device
 // address) to dst, by a kernel.
 cudaError_t launch_host_rows_in(const void *src_dev, void *dst, size_t bytes, cudaStream_t s);

@@ -342,6 +342,55 @@ int moe_ffn_forward_host(const moe_dims *d, const uint16_t *x_host, int32_t rows
                        nullptr, nullptr, nullptr, 0.0);
 }
 
+int moe_ffn_forward_nvfp4(const moe_dims *d, const uint16_t *x, int32_t rows, const uint16_t *router_w,
+                          const uint8_t *expert_w4, const uint8_t *expert_sf, const float *expert_gs,
+                          const moe_nvfp4_expert *shared, const uint16_t *shared_gate, uint16_t *out,
+                          const uint16_t *residual, const float *router_bias, void *ws, size_t ws_bytes,
+                          void *stream)
+{
+    int st = check_dims(d);
+    if (st) return st;
+    if (rows < 0) return MOE_EINVAL;
+    if (rows == 0) return enter();  // a no-op: no pointer is read
+    const auto a4 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0; };
+    if (!x || !router_w || !expert_w4 || !expert_sf || !expert_gs || !shared || !shared->w4 || !shared->sf ||
+        !shared->gs || !shared_gate || !out || !ws)
+        return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(expert_w4) || !aligned16(expert_sf) ||
+        !a4(expert_gs) || !aligned16(shared->w4) || !aligned16(shared->sf) || !a4(shared->gs) ||
+        !aligned16(shared_gate) || !aligned16(out) || (residual && !aligned16(residual)) ||
+        (router_bias && !aligned16(router_bias)) || !aligned16(ws))
+        return MOE_EINVAL;
+    if (static_cast<const void *>(out) == static_cast<const void *>(x)) return MOE_EINVAL;
+    if (ws_bytes < workspace_bytes(*d, rows)) return MOE_EWORKSPACE;
+    st = enter();
+    if (st) return st;
+    const DecodeLayout L = decode_layout(*d, rows);
+    char *base = static_cast<char *>(ws);
+    Nvfp4Launch a;
+    a.d = d;
+    a.x = x;
+    a.rows = rows;
+    a.router_w = router_w;
+    a.router_bias = router_bias;
+    a.shared_gate = shared_gate;
+    a.w4 = expert_w4;
+    a.sf = expert_sf;
+    a.gs = expert_gs;
+    a.sw4 = shared->w4;
+    a.ssf = shared->sf;
+    a.sgs = shared->gs;
+    a.residual = residual;
+    a.out = out;
+    a.topk_idx = reinterpret_cast<int32_t *>(base + L.topk_idx);
+    a.topk_w = reinterpret_cast<float *>(base + L.topk_w);
+    a.gsig = reinterpret_cast<float *>(base + L.gsig);
+    a.logits = reinterpret_cast<float *>(base + L.logits);
+    a.h = reinterpret_cast<float *>(base + L.hterm);  // h of a chunk of rows fits the step's term region
+    a.counters = reinterpret_cast<int32_t *>(base + L.counters);
+    return finish(launch_nvfp4_forward(a, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t moe_auto_path(const moe_dims *d, int32_t rows)
 {
     if (check_dims(d) != MOE_OK || rows < 0) return MOE_EINVAL;

@@ -215,3 +215,26 @@ def test_host_entry_rejects_memory_the_device_cannot_address(L):
     assert host_fwd(L, d, ws_bytes=16) == moe.MOE_EWORKSPACE
     assert host_fwd(L, d, rows=0) == moe.MOE_OK                    # a no-op
     assert moe.status() == moe.MOE_OK
+
+
+def test_nvfp4_entry_rejects_on_host(L):
+    """moe_ffn_forward_nvfp4's argument checks answer on the host."""
+    moe.reset_status()
+    d = D()
+    sh = moe.MoeNvfp4Expert(FAKE, FAKE, FAKE)
+    P = lambda a: ctypes.c_void_p(a) if a else None
+
+    def call(x=FAKE, out=FAKE + 4096, gs=FAKE, rows=1, ws_bytes=None, shared=sh):
+        wb = moe.workspace_bytes(d, max(rows, 1)) if ws_bytes is None else ws_bytes
+        return L.moe_ffn_forward_nvfp4(ctypes.byref(d), P(x), rows, P(FAKE), P(FAKE), P(FAKE), P(gs),
+                                       ctypes.byref(shared) if shared else None, P(FAKE), P(out), None, None,
+                                       P(FAKE), wb, None)
+    assert call(x=0) == moe.MOE_EINVAL
+    assert call(x=FAKE + 8) == moe.MOE_EINVAL                    # misaligned
+    assert call(gs=FAKE + 2) == moe.MOE_EINVAL                   # tensor scales not 4-byte aligned
+    assert call(shared=None) == moe.MOE_EINVAL
+    assert call(out=FAKE) == moe.MOE_EINVAL                      # out aliases x
+    assert call(rows=-1) == moe.MOE_EINVAL
+    assert call(ws_bytes=16) == moe.MOE_EWORKSPACE
+    assert call(rows=0) == moe.MOE_OK
+    assert moe.status() == moe.MOE_OK
