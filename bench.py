@@ -431,6 +431,56 @@ class ChainBench(DecodeBench):
                                   w["shared_gate"], self.r, self.ws, stream=self.stream)
 
 
+class Nvfp4Bench(DecodeBench):
+    """Decode steps of a layer with NVFP4 experts (moe_ffn_forward_nvfp4):
+    the router, gate/up and down + blend kernels; insts hold each weight
+    copy's NVFP4 codes, block scales and tensor scales."""
+
+    def step(self, i, events=None):
+        w = self.insts[i % len(self.insts)]
+        self.moe.ffn_forward_nvfp4(self.d, self.xs[i % len(self.xs)], w["router_w"], w["w4"], w["sf"], w["gs"],
+                                   w["sw4"], w["ssf"], w["sgs"], w["shared_gate"], self.outs[i % len(self.outs)],
+                                   self.ws, stream=self.stream)
+
+
+def nvfp4_instances(d, n: int, seed: int):
+    """n copies of a layer's weights with NVFP4 experts, drawn on the GPU (the
+    timing does not depend on the values): codes uniform, block scales e4m3
+    codes of values around the N(0, 0.02) weights' block maxima, tensor scale
+    amax/(448*6); router and gate N(0, 0.02) bf16."""
+    import torch
+
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    E, H, I, Is = d.n_experts, d.hidden, d.inter, d.shared_inter
+    gs = 0.1 / (448 * 6)  # a matrix maximum near 5 sigma
+
+    def scales(n_):
+        # a 16-element block maximum near 2.5 sigma: amax16 / (6 gs) ~ 224, spread x [0.5, 1.5]
+        return (torch.rand(n_, generator=g, device="cuda") + 0.5).mul(224.0).to(torch.float8_e4m3fn).view(torch.uint8)
+
+    insts = []
+    for _ in range(n):
+        insts.append({
+            "router_w": (0.02 * torch.randn(E, H, generator=g, device="cuda")).to(torch.bfloat16),
+            "shared_gate": (0.02 * torch.randn(H, generator=g, device="cuda")).to(torch.bfloat16),
+            "w4": torch.randint(0, 256, (E, 3 * I * H // 2), generator=g, device="cuda", dtype=torch.uint8),
+            "sf": scales(E * 3 * I * H // 16).view(E, -1),
+            "gs": torch.full((E, 2), gs, device="cuda", dtype=torch.float32),
+            "sw4": torch.randint(0, 256, (3 * Is * H // 2,), generator=g, device="cuda", dtype=torch.uint8),
+            "ssf": scales(3 * Is * H // 16),
+            "sgs": torch.full((2,), gs, device="cuda", dtype=torch.float32),
+        })
+    return insts
+
+
+def nvfp4_bytes(d, rows: int, n_active: float) -> float:
+    """Algorithmic bytes of an NVFP4 step: the active experts' codes, block
+    scales and tensor scales, the shared expert, router, gate, x and out."""
+    H, I, Is, E = d.hidden, d.inter, d.shared_inter, d.n_experts
+    per = lambda i: 3 * i * H / 2 + 3 * i * H / 16 + 8
+    return n_active * per(I) + per(Is) + 2 * E * H + 2 * H + 2 * rows * H * 2
+
+
 class PrefillBench(DecodeBench):
     """Prefill steps of the same layer: `rows` tokens, a per-expert router
     bias, the prefill path (permute -> tcgen05 grouped GEMMs -> blend)."""
@@ -716,6 +766,39 @@ def run_ours(args, dist: Dist):
                            "what": "each step: r <- r + layer_l(bf16(rmsnorm(r) * w_l)) in place, l = step mod "
                                    f"{N_INSTANCES}; the norm runs inside the decode-step kernel"}
         del cb
+
+    # ---- NVFP4 experts (the 397B-A17B checkpoint's format), decode rows = 1
+    if not args.no_extras:
+        d4 = mi.QWEN35_397B_A17B
+        ninst = 4  # 4 x 3.7 GB of expert weights: larger than L2
+        i4 = nvfp4_instances(d4, ninst, args.seed + 11)
+        x4 = [torch.from_numpy(mi.make_x(d4, 1, seed=args.seed + 1, stream=4000 + i).view("int16"))
+              .view(torch.bfloat16).cuda() for i in range(64)]
+        nb = Nvfp4Bench(d4, i4, x4, 1)
+        with torch.cuda.stream(nb.stream):
+            u4 = []
+            for i in range(16):  # distinct experts a step reads (routing via the same router kernel)
+                idx = torch.empty(1, d4.top_k, dtype=torch.int32, device="cuda")
+                tw = torch.empty(1, d4.top_k, dtype=torch.float32, device="cuda")
+                tg = torch.empty(1, dtype=torch.float32, device="cuda")
+                w = i4[i % ninst]
+                moe.router_topk(d4, x4[i], w["router_w"], w["shared_gate"], idx, tw, tg, nb.ws, stream=nb.stream)
+                u4.append(int(torch.unique(idx).numel()))
+        k4 = args.steps
+        ms4, _ = nb.time_steps(k4, args.warmup, dist)
+        s4 = dist.max(ms4 / 1000.0)
+        b4 = nvfp4_bytes(d4, 1, statistics.mean(u4))
+        g4 = aggregate(k4 * b4, dist.world, s4) / 1e9
+        result["nvfp4"] = {"workload": "Qwen3.5-397B-A17B-shaped MoE FFN layer with NVFP4 experts, decode rows=1",
+                           "us_per_layer": round(s4 * 1e6 / k4, 3), "gb_s": round(g4, 1),
+                           "hbm_frac_of_measured": round(g4 / dist.world / hbm_peak, 4),
+                           "bytes_per_step": int(b4), "distinct_experts_per_step": round(statistics.mean(u4), 2),
+                           "steps": k4, "kernels": ["router_topk", "nvfp4_gate_up", "nvfp4_down_blend"],
+                           "dtype": "e2m1 weights (e4m3 scale per 16, fp32 per matrix) x bf16 x for gate/up and x "
+                                    "fp32 h for down, exact products, fp32 accumulate (CUDA cores)",
+                           "l2": f"{ninst} weight copies ({ninst * 3.7:.1f} GB of expert codes)"}
+        print(f"[bench] nvfp4 397B rows=1: {s4 * 1e6 / k4:.2f} us/layer, {g4:.1f} GB/s", file=sys.stderr, flush=True)
+        del nb, i4
 
     # ---- prefill, 4096 tokens
     result["prefill"] = prefill_leg(args, d, insts[0], dist, bus, hbm_peak, bf16_peak, peak_kind)

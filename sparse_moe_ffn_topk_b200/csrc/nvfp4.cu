@@ -30,7 +30,8 @@
 namespace moe {
 namespace {
 
-constexpr int kNvWarps = 8;  // warps per CTA of both kernels
+constexpr int kNvWarps = 8;   // warps per CTA of the gate/up kernel
+constexpr int kNvDnWarps = 16; // of the down kernel (one CTA an SM: h is staged once per SM)
 
 struct NvGuParams {
     const uint16_t *x;        // [rows, H] bf16 (the chunk's first row)
@@ -86,8 +87,9 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two)
 }
 
 // Sum over a 16-byte chunk (32 codes, two scale blocks) of code * act, each
-// block's sum times its scale.
-__device__ __forceinline__ float chunk_dot(uint4 w, uint32_t sf2, const float *act)
+// block's sum times its scale; act[k * stride] is the chunk's k-th
+// activation (a transposed layout: consecutive lanes read consecutive words).
+__device__ __forceinline__ float chunk_dot(uint4 w, uint32_t sf2, const float *act, int stride)
 {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     float blk[2] = {0.f, 0.f};
@@ -95,17 +97,9 @@ __device__ __forceinline__ float chunk_dot(uint4 w, uint32_t sf2, const float *a
     for (int i = 0; i < 4; ++i) {
         float f[8];
         e2m1x8_to_f32(ws[i], f);
-        const float4 a0 = *reinterpret_cast<const float4 *>(act + 8 * i);
-        const float4 a1 = *reinterpret_cast<const float4 *>(act + 8 * i + 4);
         float s = blk[i >> 1];
-        s = fmaf(f[0], a0.x, s);
-        s = fmaf(f[1], a0.y, s);
-        s = fmaf(f[2], a0.z, s);
-        s = fmaf(f[3], a0.w, s);
-        s = fmaf(f[4], a1.x, s);
-        s = fmaf(f[5], a1.y, s);
-        s = fmaf(f[6], a1.z, s);
-        s = fmaf(f[7], a1.w, s);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s = fmaf(f[k], act[(8 * i + k) * stride], s);
         blk[i >> 1] = s;
     }
     const float2 sc = e4m3x2_to_f32(sf2);
@@ -116,7 +110,7 @@ __device__ __forceinline__ float chunk_dot(uint4 w, uint32_t sf2, const float *a
 // warps j = 8 jb + w: h[p][j] = silu(gate_j . x_t) * (up_j . x_t).
 __global__ void __launch_bounds__(kNvWarps * 32) nvfp4_gate_up_kernel(const NvGuParams p)
 {
-    extern __shared__ float xs[];  // [H]
+    extern __shared__ float xs[];  // [32][H/32 + 1]: x[32 c + k] at xs[k * xst + c]
     pdl_wait();                    // the routing, and x when a predecessor wrote it
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -124,7 +118,18 @@ __global__ void __launch_bounds__(kNvWarps * 32) nvfp4_gate_up_kernel(const NvGu
     const bool shared = r == p.K;
     const int Iu = shared ? p.Is : p.I;
     const int j = blockIdx.x * kNvWarps + warp;
-    for (int i = threadIdx.x; i < p.H; i += blockDim.x) xs[i] = bf16_bits_to_f32(p.x[(size_t)t * p.H + i]);
+    const int xst = p.H / 32 + 1;
+#pragma unroll 2
+    for (int i = threadIdx.x; i < p.H / 8; i += blockDim.x) {  // 8 values a thread and step
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.H) + i);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        const int c = i >> 2, k0 = (i & 3) * 8;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            xs[(k0 + 2 * m) * xst + c] = bf16_bits_to_f32(vw[m] & 0xFFFFu);
+            xs[(k0 + 2 * m + 1) * xst + c] = bf16_bits_to_f32(vw[m] >> 16);
+        }
+    }
     __syncthreads();
     if (j >= Iu) return;
     const int e = shared ? 0 : __ldg(p.topk_idx + (size_t)t * p.K + r);
@@ -135,62 +140,141 @@ __global__ void __launch_bounds__(kNvWarps * 32) nvfp4_gate_up_kernel(const NvGu
     const uint8_t *wg = w4 + (size_t)j * (p.H / 2), *wu = w4 + (size_t)(Iu + j) * (p.H / 2);
     const uint8_t *fg = sf + (size_t)j * (p.H / 16), *fu = sf + (size_t)(Iu + j) * (p.H / 16);
     float g = 0.f, u = 0.f;
-    for (int c = lane; c < p.H / 32; c += 32) {  // 16-byte chunks of 32 codes
-        const uint4 qg = __ldg(reinterpret_cast<const uint4 *>(wg) + c);
-        const uint4 qu = __ldg(reinterpret_cast<const uint4 *>(wu) + c);
-        const uint32_t sg = *reinterpret_cast<const uint16_t *>(fg + 2 * c);
-        const uint32_t su = *reinterpret_cast<const uint16_t *>(fu + 2 * c);
-        g += chunk_dot(qg, sg, xs + 32 * c);
-        u += chunk_dot(qu, su, xs + 32 * c);
+    constexpr int kC = 4;  // 16-byte chunks (32 codes) a lane loads before using any
+    for (int c0 = 0; c0 < p.H / 32; c0 += 32 * kC) {
+        uint4 qg[kC], qu[kC];
+        uint32_t sg[kC], su[kC];
+#pragma unroll
+        for (int i = 0; i < kC; ++i) {
+            const int c = c0 + lane + 32 * i;
+            if (c < p.H / 32) {
+                qg[i] = __ldg(reinterpret_cast<const uint4 *>(wg) + c);
+                qu[i] = __ldg(reinterpret_cast<const uint4 *>(wu) + c);
+                sg[i] = __ldg(reinterpret_cast<const uint16_t *>(fg) + c);
+                su[i] = __ldg(reinterpret_cast<const uint16_t *>(fu) + c);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kC; ++i) {
+            const int c = c0 + lane + 32 * i;
+            if (c < p.H / 32) {
+                g += chunk_dot(qg[i], sg[i], xs + c, xst);
+                u += chunk_dot(qu[i], su[i], xs + c, xst);
+            }
+        }
     }
     g = warp_sum(g) * gs13;
     u = warp_sum(u) * gs13;
     if (lane == 0) p.h[(size_t)pair * p.imax + j] = siluf_(g) * u;
 }
 
-// Down + blend: warp w of CTA b takes output rows n = 8 b + w + 8 G k; per
-// row t of the chunk, y_p[n] = (W2_e[n] . h[p]) * gs2 for its k pairs and the
-// shared expert, out[t][n] = bf16(sum_r w_r y_r + gsig y_s (+ residual)).
-__global__ void __launch_bounds__(kNvWarps * 32) nvfp4_down_blend_kernel(const NvDownParams p)
+// Down + blend: warp w of CTA b takes output rows n = 16 b + w + 16 G k; per
+// row t of the chunk, out[t][n] = bf16(sum_r w_r gs2_r (W2_r[n] . h_r) +
+// gsig gs2_s (W2_s[n] . h_s) (+ residual)).
+__global__ void __launch_bounds__(kNvDnWarps * 32) nvfp4_down_blend_kernel(const NvDownParams p)
 {
-    extern __shared__ float hs[];  // [pairs][imax]
+    // h of every pair, transposed by 16-value blocks: h[p][16 b + i] at
+    // hs[p * hpst + i * hst + b], so that the lanes (b = lane, lane + 32, ...)
+    // read consecutive words
+    extern __shared__ float hs[];
     pdl_wait();                    // h from the gate/up kernel
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int np = p.rows * (p.K + 1);
-    for (int i = threadIdx.x; i < np * p.imax / 4; i += blockDim.x)
-        reinterpret_cast<float4 *>(hs)[i] = __ldcg(reinterpret_cast<const float4 *>(p.h) + i);
+    const int hst = p.imax / 16 + 1, hpst = 16 * hst;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < np * p.imax / 4; i += blockDim.x) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.h) + i);
+        const int pr = (4 * i) / p.imax, o = 4 * i - pr * p.imax, b = o >> 4, k = o & 15;
+        float *d = hs + (size_t)pr * hpst + b;
+        d[k * hst] = v.x;
+        d[(k + 1) * hst] = v.y;
+        d[(k + 2) * hst] = v.z;
+        d[(k + 3) * hst] = v.w;
+    }
     __syncthreads();
-    for (int n = blockIdx.x * kNvWarps + warp; n < p.H; n += gridDim.x * kNvWarps) {
+    // Per output row and row of x: each lane's share of every pair's dot
+    // product (16-code blocks b = lane, lane + 32, ...), times the pair's
+    // blend weight and tensor scale, summed over the pairs in rank order
+    // (the shared expert last); then one warp sum.  The loads of a group of
+    // pairs are all issued before any is used.
+    constexpr int kG = 4;  // pairs a group
+    for (int n = blockIdx.x * kNvDnWarps + warp; n < p.H; n += gridDim.x * kNvDnWarps) {
         for (int t = 0; t < p.rows; ++t) {
             float acc = 0.f;
-            for (int r = 0; r <= p.K; ++r) {
-                const bool shared = r == p.K;
-                const int Iu = shared ? p.Is : p.I;
-                const int e = shared ? 0 : __ldg(p.topk_idx + (size_t)t * p.K + r);
-                const size_t slab4 = (size_t)3 * Iu * p.H / 2, slabf = (size_t)3 * Iu * p.H / 16;
-                const uint8_t *w2 = (shared ? p.sw4 : p.w4 + (size_t)e * slab4) + (size_t)Iu * p.H +
-                                    (size_t)n * (Iu / 2);
-                const uint8_t *f2 = (shared ? p.ssf : p.sf + (size_t)e * slabf) + (size_t)Iu * p.H / 8 +
-                                    (size_t)n * (Iu / 16);
-                const float gs2 = shared ? __ldg(p.sgs + 1) : __ldg(p.gs + 2 * (size_t)e + 1);
-                const float *hp = hs + (size_t)(t * (p.K + 1) + r) * p.imax;
-                float s = 0.f;
-                for (int b = lane; b < Iu / 16; b += 32) {  // 8-byte blocks of 16 codes, one scale each
-                    const uint2 q = __ldg(reinterpret_cast<const uint2 *>(w2) + b);
-                    float f[8];
-                    float blk = 0.f;
-                    e2m1x8_to_f32(q.x, f);
+            for (int r0 = 0; r0 <= p.K; r0 += kG) {
+                uint2 q[kG][2];
+                uint32_t f[kG][2];
+                float wgt[kG];
+                int nb[kG];
+                const float *hp[kG];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) blk = fmaf(f[i], hp[16 * b + i], blk);
-                    e2m1x8_to_f32(q.y, f);
+                for (int g = 0; g < kG; ++g) {
+                    const int r = r0 + g;
+                    nb[g] = 0;
+                    if (r > p.K) continue;
+                    const bool shared = r == p.K;
+                    const int Iu = shared ? p.Is : p.I;
+                    const int e = shared ? 0 : __ldg(p.topk_idx + (size_t)t * p.K + r);
+                    const size_t slab4 = (size_t)3 * Iu * p.H / 2, slabf = (size_t)3 * Iu * p.H / 16;
+                    const uint8_t *w2 = (shared ? p.sw4 : p.w4 + (size_t)e * slab4) + (size_t)Iu * p.H +
+                                        (size_t)n * (Iu / 2);
+                    const uint8_t *f2 = (shared ? p.ssf : p.sf + (size_t)e * slabf) + (size_t)Iu * p.H / 8 +
+                                        (size_t)n * (Iu / 16);
+                    const float gs2 = shared ? __ldg(p.sgs + 1) : __ldg(p.gs + 2 * (size_t)e + 1);
+                    wgt[g] = (shared ? __ldg(p.gsig + t) : __ldg(p.topk_w + (size_t)t * p.K + r)) * gs2;
+                    hp[g] = hs + (size_t)(t * (p.K + 1) + r) * hpst;
+                    nb[g] = Iu / 16;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) blk = fmaf(f[i], hp[16 * b + 8 + i], blk);
-                    s = fmaf(blk, e4m3x2_to_f32(f2[b]).x, s);
+                    for (int k = 0; k < 2; ++k) {
+                        const int b = lane + 32 * k;
+                        if (b < nb[g]) {
+                            q[g][k] = __ldg(reinterpret_cast<const uint2 *>(w2) + b);
+                            f[g][k] = __ldg(f2 + b);
+                        }
+                    }
                 }
-                const float y = warp_sum(s) * gs2;
-                acc = fmaf(shared ? __ldg(p.gsig + t) : __ldg(p.topk_w + (size_t)t * p.K + r), y, acc);
+#pragma unroll
+                for (int g = 0; g < kG; ++g) {
+                    if (!nb[g]) continue;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int b = lane + 32 * k;
+                        if (b >= nb[g]) continue;
+                        float v[8], blk = 0.f;
+                        e2m1x8_to_f32(q[g][k].x, v);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) blk = fmaf(v[i], hp[g][i * hst + b], blk);
+                        e2m1x8_to_f32(q[g][k].y, v);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) blk = fmaf(v[i], hp[g][(8 + i) * hst + b], blk);
+                        sum = fmaf(blk, e4m3x2_to_f32(f[g][k]).x, sum);
+                    }
+                    // blocks beyond 64 a row (inter above 1024): the same, one at a time
+                    for (int b = lane + 64; b < nb[g]; b += 32) {
+                        const int r = r0 + g;
+                        const bool shared = r == p.K;
+                        const int Iu = shared ? p.Is : p.I;
+                        const int e = shared ? 0 : __ldg(p.topk_idx + (size_t)t * p.K + r);
+                        const uint8_t *w2 = (shared ? p.sw4 : p.w4 + (size_t)e * ((size_t)3 * Iu * p.H / 2)) +
+                                            (size_t)Iu * p.H + (size_t)n * (Iu / 2);
+                        const uint8_t *f2 = (shared ? p.ssf : p.sf + (size_t)e * ((size_t)3 * Iu * p.H / 16)) +
+                                            (size_t)Iu * p.H / 8 + (size_t)n * (Iu / 16);
+                        const uint2 qq = __ldg(reinterpret_cast<const uint2 *>(w2) + b);
+                        float v[8], blk = 0.f;
+                        e2m1x8_to_f32(qq.x, v);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) blk = fmaf(v[i], hp[g][i * hst + b], blk);
+                        e2m1x8_to_f32(qq.y, v);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) blk = fmaf(v[i], hp[g][(8 + i) * hst + b], blk);
+                        sum = fmaf(blk, e4m3x2_to_f32(__ldg(f2 + b)).x, sum);
+                    }
+                    acc = fmaf(wgt[g], sum, acc);
+                }
             }
+            acc = warp_sum(acc);
             if (lane == 0) {
                 const size_t o = (size_t)t * p.H + n;
                 if (p.residual) acc += bf16_bits_to_f32(p.residual[o]);
@@ -205,7 +289,7 @@ __global__ void __launch_bounds__(kNvWarps * 32) nvfp4_down_blend_kernel(const N
 int nvfp4_rows_per_chunk(const moe_dims &d)
 {
     // h of a chunk's pairs in one CTA's shared memory (up to 160 KB), at most 4 rows
-    const size_t per_row = (size_t)(d.top_k + 1) * std::max(d.inter, d.shared_inter) * 4;
+    const size_t per_row = (size_t)(d.top_k + 1) * 16 * (std::max(d.inter, d.shared_inter) / 16 + 1) * 4;
     return (int)std::max<size_t>(1, std::min<size_t>(4, (size_t)160 * 1024 / per_row));
 }
 
@@ -257,7 +341,7 @@ cudaError_t launch_nvfp4_forward(const Nvfp4Launch &a, cudaStream_t s)
         g.Is = Is;
         g.imax = imax;
         e = launch_kernel(nvfp4_gate_up_kernel, dim3((imax + kNvWarps - 1) / kNvWarps, n * (K + 1)),
-                          dim3(kNvWarps * 32), (size_t)H * 4, s, g);
+                          dim3(kNvWarps * 32), (size_t)32 * (H / 32 + 1) * 4, s, g);
         if (e != cudaSuccess) return e;
         NvDownParams dp;
         dp.topk_idx = a.topk_idx + (size_t)t0 * K;
@@ -278,9 +362,9 @@ cudaError_t launch_nvfp4_forward(const Nvfp4Launch &a, cudaStream_t s)
         dp.I = I;
         dp.Is = Is;
         dp.imax = imax;
-        const int grid = std::min(4 * device_info().sm_count, (H + kNvWarps - 1) / kNvWarps);
-        e = launch_kernel(nvfp4_down_blend_kernel, dim3(grid), dim3(kNvWarps * 32),
-                          (size_t)n * (K + 1) * imax * 4, s, dp);
+        const int grid = std::min(device_info().sm_count, (H + kNvDnWarps - 1) / kNvDnWarps);
+        e = launch_kernel(nvfp4_down_blend_kernel, dim3(grid), dim3(kNvDnWarps * 32),
+                          (size_t)n * (K + 1) * 16 * (imax / 16 + 1) * 4, s, dp);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
