@@ -124,6 +124,12 @@ __device__ __forceinline__ int atomic_add_release_gpu(int32_t *p, int v)
     asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
+__device__ __forceinline__ int atomic_add_relaxed_gpu(int32_t *p, int v)
+{
+    int old;
+    asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 __device__ __forceinline__ void red_release_gpu(int32_t *p, int v)
 {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -802,6 +808,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const int tile0 = first_tile(n8, G, c);
     const int nt = first_tile(n8, G, c + 1) - tile0;
     const bool producer = warp == kStepWarps;
+    int exit_old = -1;  // (thread 0) the grid barrier's exit count before this CTA's
     volatile int32_t *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -1011,7 +1018,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             for (int ri = 0; ri < s0.n_router; ++ri) mbar_arrive(&empty[ri]);
             bool ok = !*abort;
             if (ok) {
-                __threadfence();
+                // a releasing arrival: cumulative over the CTA's logits and
+                // zeros, which the CTA barrier above ordered before it
                 atomic_add_release_gpu(p.counters + kCtrStepBar, 1);
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_gpu(p.counters + kCtrStepBar) < G) {
@@ -1023,14 +1031,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                     }
                 }
             }
-            if (ok) {
-                // every CTA has passed the barrier once the exit count is
-                // full: the last one resets both for the next call
-                if (atomic_add_acq_rel_gpu(p.counters + kCtrStepExit, 1) == G - 1) {
-                    p.counters[kCtrStepBar] = 0;
-                    p.counters[kCtrStepExit] = 0;
-                }
-            }
+            // every CTA has passed the barrier once the exit count is full;
+            // the count's answer is needed only after P3 (the last CTA to
+            // pass resets both for the next call then), so its round trip
+            // stays off the critical path
+            if (ok) exit_old = atomic_add_relaxed_gpu(p.counters + kCtrStepExit, 1);
         }
         named_barrier(1, kStepWarps * kWarp);
         STEP_T(4);  // grid barrier 1 passed
@@ -1445,6 +1450,13 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     STEP_T(8);  // P3 starts
     down_phase(p, sm, sbase, base, full, empty, tdone, bbars, seq, nt, tile0, rb0, ibm, dsc, ybuf, abort);
     named_barrier(1, kStepWarps * kWarp);  // every down item of the CTA done
+    // (thread 0) the last CTA past grid barrier 1 resets its counters for the
+    // next call; the next launch reaches the barrier only after its PDL wait,
+    // that is after this grid has finished
+    if (threadIdx.x == 0 && exit_old == G - 1) {
+        p.counters[kCtrStepBar] = 0;
+        p.counters[kCtrStepExit] = 0;
+    }
     if (*abort) return;
 
     STEP_T(10);  // down items done
