@@ -1416,12 +1416,13 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 named_barrier(3, 4 * kWarp);  // the exchange slots are free again
                 if (lane == 0) mbar_arrive(&tfree[b]);
                 if (threadIdx.x == kEpiWaiter) {
-                    // this unit's h (both warps' writes, ordered by the CTA
-                    // barrier above) before its count for the expert: the down
-                    // items of every CTA wait for their expert's full count
+                    // this unit's h before its count for the expert: the
+                    // releasing add is cumulative over both warps' h writes,
+                    // which the named barrier above ordered before it; the
+                    // down items of every CTA wait for their expert's full
+                    // count with acquiring loads
                     const int u = c + l * G, us = p.Is / kGuRows;
                     const int de = u < us ? 0 : 1 + (u - us) / (p.I / kGuRows);
-                    __threadfence();
                     red_release_gpu(p.counters + kCtrStepReady + de * p.rdy, 1);
                     STEP_TL(15);  // (trace) this CTA's last unit counted
                 }
