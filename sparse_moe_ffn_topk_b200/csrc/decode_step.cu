@@ -405,6 +405,39 @@ struct Seq {
 // Down items: per group of experts (the shared expert alone, then groups of
 // dn_epi routed experts of the list), per chunk of dn_tpi output tiles of
 // this CTA, the full K of the down rows (one TMA box per expert and tile).
+// The parts of make_seq that do not depend on the routing (computed before
+// the plan): router items, down tile chunks, units of the shared expert and
+// of one routed expert.
+struct SeqConst {
+    int n_router, n_tc_s, n_tc_r, us, per;
+};
+__device__ __forceinline__ SeqConst seq_const(const StepParams &p, int nt, int nr)
+{
+    SeqConst k;
+    k.n_router = (nr + p.rr_per_item - 1) / p.rr_per_item;
+    k.n_tc_s = nt > 0 ? (nt + p.dn_tpi_s - 1) / p.dn_tpi_s : 0;
+    k.n_tc_r = nt > 0 ? (nt + p.dn_tpi - 1) / p.dn_tpi : 0;
+    k.us = p.Is / kGuRows;
+    k.per = p.I / kGuRows;
+    return k;
+}
+// make_seq from those (the same sequence): one division after the plan.
+__device__ __forceinline__ Seq make_seq_k(const StepParams &p, const SeqConst &k, int U)
+{
+    const int G = gridDim.x, c = blockIdx.x;
+    Seq s;
+    s.n_router = k.n_router;
+    const int units = k.us + U * k.per;
+    s.n_units_local = units > c ? (units - 1 - c) / G + 1 : 0;
+    s.n_gu = s.n_units_local * p.gu_pieces;
+    s.n_tc_s = k.n_tc_s;
+    s.n_tc_r = k.n_tc_r;
+    s.n_groups_r = p.dn_epi == 1 ? U : (U + p.dn_epi - 1) / p.dn_epi;
+    s.n_dn = s.n_tc_s + s.n_groups_r * s.n_tc_r;
+    s.total = s.n_router + s.n_gu + s.n_dn;
+    return s;
+}
+
 __device__ __forceinline__ Seq make_seq(const StepParams &p, int U, int nt, int nr)
 {
     const int G = gridDim.x, c = blockIdx.x;
@@ -842,6 +875,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     // rows, then the shared expert's gate/up units (the first local units).
     const uint64_t pol = policy_evict_first();
     const Seq s0 = make_seq(p, 0, 0, nr_total);  // U = 0: router and shared-expert items only (a prefix of the full sequence)
+    const SeqConst sk = seq_const(p, nt, nr_total);
     const int p0_count = min(s0.total, p.ns);
     if (producer) {
         if (lane == 0) {
@@ -1163,7 +1197,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     __syncthreads();  // the plan is ready (all 288 threads)
     STEP_T(5);
     const int U = *abort ? 0 : sm.n_list;
-    const Seq seq = make_seq(p, U, nt, nr_total);
+    const Seq seq = make_seq_k(p, sk, U);
 
     if (producer) {
         // ---------------------------------------------------------- producer
