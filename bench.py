@@ -62,7 +62,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true", help="skip the rows=64 and per-kernel legs")
-    ap.add_argument("--profile", choices=["decode", "prefill", "narrow"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "narrow", "nvfp4"], default=None,
                     help="a small case for a profiler: a few eager layer calls on one weight copy, then exit "
                          "(decode: rows=1; prefill: 4096 biased rows; narrow: the narrow grouped GEMMs at --rows)")
     ap.add_argument("--rows", type=int, default=64, help="rows of --profile narrow")
@@ -936,12 +936,27 @@ def run_sweep(args, dist: Dist):
 def run_profile_case(args):
     """A few eager calls of one workload (35B-shaped layer, one weight copy):
     decode at rows = 1 on fresh x each call, the 4096-token biased prefill, or
-    the narrow grouped GEMMs at --rows rows.  Small enough for a profiler to
-    replay every kernel."""
+    the narrow grouped GEMMs at --rows rows; or the 397B-shaped layer with
+    NVFP4 experts at rows = 1.  Small enough for a profiler to replay every
+    kernel."""
     import torch
 
     import moe_inputs as mi
     import sparse_moe_ffn_topk_b200 as moe
+    if args.profile == "nvfp4":
+        # the 397B-A17B-shaped layer with NVFP4 experts, one weight copy (3.7 GB) drawn on the GPU
+        d4 = mi.QWEN35_397B_A17B
+        w = nvfp4_instances(d4, 1, args.seed + 11)[0]
+        ws = moe.alloc_workspace(d4, 1)
+        out = torch.empty(1, d4.hidden, dtype=torch.bfloat16, device="cuda")
+        for i in range(args.calls):
+            x = torch.from_numpy(mi.make_x(d4, 1, seed=args.seed + 5, stream=i).view("int16")).view(torch.bfloat16).cuda()
+            moe.ffn_forward_nvfp4(d4, x, w["router_w"], w["w4"], w["sf"], w["gs"], w["sw4"], w["ssf"], w["sgs"],
+                                  w["shared_gate"], out, ws)
+        torch.cuda.synchronize()
+        st = moe.device_status(ws)
+        print(json.dumps({"profile": args.profile, "calls": args.calls, "rows": 1, "device_status": st}), flush=True)
+        return 0 if st == moe.MOE_OK else 1
     d = mi.QWEN36_35B_A3B
     inst = make_instances(mi.make_layer(d, seed=args.seed), 1)[0]
     if args.profile == "decode":
