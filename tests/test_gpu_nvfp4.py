@@ -105,3 +105,29 @@ def test_nvfp4_residual_and_batch_invariance():
     for t in (0, 4):
         one, _ = _run(d, x[t:t + 1], layer, residual=res[t:t + 1])
         assert np.array_equal(one[0], got[t])
+
+
+@pytest.mark.parametrize("dims,rows", [
+    # I > 1024: 72 scale blocks a down row (the lanes' blocks past 64); H/32 = 12 chunks, fewer than
+    # the lanes; Is != I; two chunks of rows
+    (mi.LayerDims(hidden=384, n_experts=12, top_k=3, inter=1152, shared_inter=640), 5),
+    (mi.LayerDims(hidden=256, n_experts=16, top_k=16, inter=128, shared_inter=128), 2),   # k = E
+    (mi.LayerDims(hidden=128, n_experts=1, top_k=1, inter=128, shared_inter=128), 1),     # one expert
+    (mi.LayerDims(hidden=8192, n_experts=4, top_k=2, inter=128, shared_inter=256), 3),    # 256 chunks: two load rounds
+])
+def test_nvfp4_odd_shapes(dims, rows):
+    x, layer, logits = _case(dims, rows, seed=25, all_experts=True)
+    got, idx = _run(dims, x, layer)
+    _check(dims, x, layer, logits, got, idx)
+
+
+def test_nvfp4_rows_zero_is_noop():
+    d = mi.TINY
+    layer = mi.make_layer_nvfp4(d, seed=26)
+    dev = _dev(layer)
+    ws = moe.alloc_workspace(d, 1)
+    x = torch.empty(0, d.hidden, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(0, d.hidden, dtype=torch.bfloat16, device="cuda")
+    moe.ffn_forward_nvfp4(d, x, dev["router_w"], dev["w4"], dev["sf"], dev["gs"], dev["sw4"], dev["ssf"],
+                          dev["sgs"], dev["shared_gate"], out, ws)
+    torch.cuda.synchronize()
