@@ -1376,6 +1376,22 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             // (the loop holds named barriers)
             for (int l = 0; l < seq.n_units_local; ++l) {
                 const int b = l % p.nbuf, kk = l / p.nbuf;
+                // the unit and its rows' slots of h while its MMAs run
+                bool shared;
+                int e, j;
+                unit_of(p, sm, c + l * G, shared, e, j);
+                int slots[kStepMaxRows];
+#pragma unroll
+                for (int t = 0; t < kStepMaxRows; ++t) {
+                    slots[t] = -1;
+                    if (t >= rows) continue;
+                    if (shared) {
+                        slots[t] = rows * K + t;
+                    } else {
+                        for (int r = 0; r < K; ++r)
+                            if (sm.idx[t * K + r] == e) slots[t] = t * K + r;
+                    }
+                }
                 if (threadIdx.x == kEpiWaiter) {
                     const bool ok = !*abort && mbar_wait_spin(&tfull[b], (uint32_t)(kk & 1), kWaitLimitNs);
                     if (!ok) {
@@ -1387,9 +1403,6 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 named_barrier(3, 4 * kWarp);
                 if (sm.gu_stop) break;
                 tc_fence_after();
-                bool shared;
-                int e, j;
-                unit_of(p, sm, c + l * G, shared, e, j);
                 const float *srow = gsc + (size_t)l * 2 * hb + (gate ? 0 : hb);
                 float acc[kStepMaxRows];
                 const uint32_t tb = tmem + (uint32_t)(b * p.tbuf) + ((uint32_t)(32 * warp) << 16);
@@ -1412,19 +1425,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                     // maximum and to within 2^-31 of it below.  Term k of value
                     // m goes where the down MMA's B registers want it: byte
                     // (m % 4) + 4 (m / 16) of lane 4k + (m % 16) / 4's eight.
-                    int slots[kStepMaxRows];
                     float hv[kStepMaxRows];
 #pragma unroll
                     for (int t = 0; t < kStepMaxRows; ++t) {
-                        slots[t] = -1;
                         hv[t] = 0.f;
                         if (t >= rows) continue;
-                        if (shared) {
-                            slots[t] = rows * K + t;
-                        } else {
-                            for (int r = 0; r < K; ++r)
-                                if (sm.idx[t * K + r] == e) slots[t] = t * K + r;
-                        }
                         if (slots[t] >= 0 && lane < 16) hv[t] = siluf_(acc[t]) * sm.xch[m * kStepMaxRows + t];
                         const float mx = warp_max(fabsf(hv[t]));
                         if (lane == 0) sm.hmx[warp * kStepMaxRows + t] = mx;
