@@ -134,6 +134,16 @@ __device__ __forceinline__ void red_release_gpu(int32_t *p, int v)
 {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ int ld_acquire_cta_shared(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta_shared(int32_t *p, int v)
+{
+    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
 __device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
 {
     int v;
@@ -370,6 +380,7 @@ struct StepSmall {
     uint32_t tmem;                          // tensor-memory base of this CTA's accumulators
     int32_t gu_stop;                        // gate/up epilogue: leave the unit loop (written by its waiter)
     int32_t dn_next;                        // down phase: the next item to claim
+    int32_t dsc_ready;                      // the down block scales are staged (warps 0-3 -> 4-7)
     double red[kStepWarps * kStepMaxRows];  // RMSNorm: per-warp sums of squares
     double inv[kStepMaxRows];               // RMSNorm: 1 / sqrt(mean square + eps) per row
     int32_t n_list;
@@ -752,6 +763,15 @@ __device__ __forceinline__ void down_phase(const StepParams &p, StepSmall &sm, u
         {
             int okd = 1;
             if (lane == 0) okd = mbar_wait(tdone, 0, kWaitLimitNs) ? 1 : 0;
+            // the down block scales staged by warps 0-3 (long done by now)
+            if (lane == 0 && okd && ld_acquire_cta_shared(&sm.dsc_ready) == 0) {
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_cta_shared(&sm.dsc_ready) == 0)
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        okd = 0;
+                        break;
+                    }
+            }
             if (!__shfl_sync(0xFFFFFFFFu, okd, 0)) {
                 if (lane == 0) {
                     gave_up(p.counters, 10, 2);
@@ -858,6 +878,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         for (int w = 0; w < kStepWarps; ++w) mbar_init(&bbars[w], 1);
         sm.abort = 0;
         sm.dn_next = 0;
+        sm.dsc_ready = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1265,18 +1286,20 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const float *xfac = reinterpret_cast<const float *>(sbase + p.o_xfac);
 
     // Block scales of this CTA's work into shared memory, one round trip for
-    // all of them (the weight copies are in flight meanwhile): per local
-    // gate/up unit its gate and up row blocks [2][H/128]; per down expert
-    // (shared first, then the routed list) the row blocks of this CTA's
-    // output rows [2][Iu/128].
+    // all of them (the weight copies are in flight meanwhile), by the
+    // epilogue warps 0-3 (the issuing warps need none and start their MMAs
+    // at once): per local gate/up unit its gate and up row blocks [2][H/128];
+    // per down expert (shared first, then the routed list) the row blocks of
+    // this CTA's output rows [2][Iu/128].  The down items of warps 4-7 read
+    // the latter after thread 0's release below.
     float *gsc = reinterpret_cast<float *>(sbase + p.o_gsc);
     float *dsc = reinterpret_cast<float *>(sbase + p.o_dsc);
     const int ibm = p.imax / 128;
     const int rb0 = (tile0 * 8) / 128;
-    {
+    if (warp < 4) {
         const int ng = seq.n_units_local * 2 * hb;
         const int nd = nt > 0 ? (U + 1) * 2 * ibm : 0;
-        for (int i = threadIdx.x; i < ng + nd; i += kStepWarps * kWarp) {
+        for (int i = threadIdx.x; i < ng + nd; i += 4 * kWarp) {
             if (i < ng) {
                 const int l = i / (2 * hb), rem = i - l * 2 * hb, half = rem / hb, W = rem - half * hb;
                 bool shared;
@@ -1303,7 +1326,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 dsc[k] = v;
             }
         }
-        named_barrier(1, kStepWarps * kWarp);
+        named_barrier(5, 4 * kWarp);
+        if (threadIdx.x == 0) st_release_cta_shared(&sm.dsc_ready, 1);  // (the barrier ordered warps 0-3's writes)
     }
 
     // gate/up on the tensor cores.  Four issuing threads take, per local unit, the MMAs
