@@ -898,6 +898,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const Seq s0 = make_seq(p, 0, 0, nr_total);  // U = 0: router and shared-expert items only (a prefix of the full sequence)
     const SeqConst sk = seq_const(p, nt, nr_total);
     const int p0_count = min(s0.total, p.ns);
+    // This CTA's first gate/up unit is the shared expert's and all of its
+    // copies are issued in P0: its MMAs go out while the CTA waits at the
+    // grid barrier (they need only x's terms), not after the plan.
+    const bool gu_early = s0.n_units_local > 0 && s0.n_router + p.gu_pieces <= p0_count;
     if (producer) {
         if (lane == 0) {
             tma_prefetch_desc(&p.w13);
@@ -1091,6 +1095,40 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             // pass resets both for the next call then), so its round trip
             // stays off the critical path
             if (ok) exit_old = atomic_add_relaxed_gpu(p.counters + kCtrStepExit, 1);
+        }
+        if (gu_early && warp >= kIssuer0 && warp < kIssuer0 + kIssuers && lane == 0) {
+            // the shared unit's MMAs (buffer 0), as the issuing loop below
+            // would issue them; x's terms were fenced for the async proxy and
+            // ordered by the CTA barrier above
+            const int me = warp - kIssuer0;
+            const uint32_t idesc = idesc_e4m3_e5m2_f32(2 * kGuRows, p.nb);
+            const uint32_t xb_u32 = base + p.o_xB;
+            bool ok = true;
+            for (int pc = me; pc < p.gu_pieces && ok; pc += kIssuers) {
+                const int q = s0.n_router + pc;
+                const int s = q % p.ns;
+                if (!wait_item_lane(sm.tag, full, s, q, p.ns)) {
+                    gave_up(p.counters, 2, q);
+                    *abort = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sl = base + (uint32_t)s * kSlot;
+                for (int wl = 0; wl < p.gu_wp; ++wl) {
+                    const int W = pc * p.gu_wp + wl;
+                    if (W >= hb) break;
+                    const uint32_t a0 = sl + (uint32_t)wl * kGuWindow;
+                    const uint32_t b0 = xb_u32 + (uint32_t)(W * p.nb * 128);
+                    const uint32_t d = tmem + (uint32_t)(W * p.nb);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        umma_f8f6f4(d, umma_desc_sw128(a0 + 32 * k4), umma_desc_sw128(b0 + 32 * k4), idesc,
+                                    k4 > 0 ? 1u : 0u);
+                }
+                umma_commit(&empty[s]);
+            }
+            if (ok) umma_commit(&tfull[0]);
         }
         named_barrier(1, kStepWarps * kWarp);
         STEP_T(4);  // grid barrier 1 passed
@@ -1347,7 +1385,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             if (lane == 0) {
                 const int me = warp - kIssuer0;
                 const uint32_t idesc = idesc_e4m3_e5m2_f32(2 * kGuRows, p.nb);
-                for (int l = 0; l < seq.n_units_local && !*abort; ++l) {
+                for (int l = gu_early ? 1 : 0; l < seq.n_units_local && !*abort; ++l) {  // (unit 0 went out early)
                     const int b = l % p.nbuf, kk = l / p.nbuf;
                     if (kk >= 1 && !mbar_wait_spin(&tfree[b], (uint32_t)((kk - 1) & 1), kWaitLimitNs)) {
                         gave_up(p.counters, 8, l);
