@@ -101,6 +101,37 @@ def test_odd_shapes(dims, rows):
     check(case)
 
 
+@pytest.mark.parametrize("dims,rows", [
+    (mi.LayerDims(hidden=1024, n_experts=256, top_k=8, inter=256, shared_inter=256), 1),   # chunk ranks, ranked merge
+    (mi.LayerDims(hidden=1024, n_experts=256, top_k=8, inter=256, shared_inter=256), 3),   # experts shared by rows
+    (mi.LayerDims(hidden=1024, n_experts=512, top_k=10, inter=256, shared_inter=256), 2),  # merge by rounds
+    (mi.LayerDims(hidden=512, n_experts=64, top_k=32, inter=128, shared_inter=128), 1),    # k = 32: a whole chunk
+])
+def test_exact_logit_ties_take_the_lower_expert_first(dims, rows):
+    """Experts 2i and 2i+1 share one router row, so their logits are equal
+    bit for bit in any summation order.  Equal logits keep ascending expert
+    order: where 2i+1 is chosen, 2i is chosen just before it with the same
+    weight; where only one of the pair is chosen, it is 2i."""
+    seed = 31
+    rw, g, _ = mi.make_router(dims, seed)
+    rw[1::2] = rw[0::2]
+    x = mi.make_x(dims, rows, seed=seed, stream=rows)
+    logits, _, _, _ = oracle.router_topk(dims, x, rw, g)
+    layer = mi.make_layer(dims, seed=seed, experts=P.needed_experts(logits, dims.top_k))
+    layer.router_w[1::2] = layer.router_w[0::2]
+    case = P.build_case(dims, rows, seed=seed, layer=layer)
+    out, idx, w, gs = run_forward(case)
+    _, _, ow, ogs = oracle.router_topk(dims, case.x, layer.router_w, layer.shared_gate)
+    P.check_routing(case, idx, w, gs, ow, ogs)
+    P.compare_output(case, out, idx)
+    for t in range(rows):
+        pos = {int(e): i for i, e in enumerate(idx[t])}
+        for e, i in pos.items():
+            if e % 2 == 1:
+                assert pos.get(e - 1) == i - 1, f"row {t}: expert {e} at {i} without {e - 1} just before it"
+                assert w[t, i] == w[t, i - 1]
+
+
 def test_residual_and_router_bias():
     d = mi.LayerDims(hidden=512, n_experts=32, top_k=4, inter=256, shared_inter=256)
     case = P.build_case(d, 6, router_bias=True, all_experts=True, residual=True)
