@@ -34,7 +34,6 @@ POINTS = [
     (13, "top-k done"),
     (14, "distinct-expert list done"),
     (5, "plan done"),
-    (6, "first gate/up item landed (warp 0's view)"),
     (15, "this CTA's last gate/up unit counted (epilogue thread)"),
     (7, "gate/up done (warp 0)"),
     (8, "P3 entered (warp 0)"),
