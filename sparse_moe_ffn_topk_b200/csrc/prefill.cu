@@ -321,20 +321,30 @@ struct RouterTcParams {
     int32_t *counters;
 };
 
+// Insert (k, e) into a row's running top-k (keys descending).  The new key
+// goes in front of the first key it strictly exceeds, so equal keys keep the
+// lower expert first.  Every place of the new list is taken from the old list
+// at once (kept, shifted down one, or the new key): KM independent selects
+// instead of a chain of compare-and-swaps through k, which one thread per row
+// would otherwise run at the latency of each step.
 template <int KM>
 __device__ __forceinline__ void topk_insert(uint32_t (&keys)[KM], int (&ids)[KM], uint32_t k, int e)
 {
-    if (k <= keys[KM - 1]) return;  // equal keys keep the lower expert first
+    bool gt[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) gt[j] = k > keys[j];  // false then true: the list is sorted
+    uint32_t nk[KM];
+    int ni[KM];
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
-        if (k > keys[j]) {
-            const uint32_t tk = keys[j];
-            const int ti = ids[j];
-            keys[j] = k;
-            ids[j] = e;
-            k = tk;
-            e = ti;
-        }
+        const bool shift = gt[j] && j > 0 && gt[j > 0 ? j - 1 : 0];
+        nk[j] = !gt[j] ? keys[j] : (shift ? keys[j > 0 ? j - 1 : 0] : k);
+        ni[j] = !gt[j] ? ids[j] : (shift ? ids[j > 0 ? j - 1 : 0] : e);
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        keys[j] = nk[j];
+        ids[j] = ni[j];
     }
 }
 

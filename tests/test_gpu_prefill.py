@@ -54,6 +54,38 @@ def test_prefill_small_shapes(dims, rows, bias):
     P.compare_output(case, out, idx)
 
 
+@pytest.mark.parametrize("dims,rows", [
+    (mi.LayerDims(hidden=1024, n_experts=256, top_k=8, inter=256, shared_inter=256), 130),   # top-8 kept per row
+    (mi.LayerDims(hidden=512, n_experts=128, top_k=10, inter=128, shared_inter=128), 200),   # top-16 kept
+    (mi.LayerDims(hidden=512, n_experts=64, top_k=32, inter=128, shared_inter=128), 129),    # top-32 kept
+])
+def test_exact_logit_ties_take_the_lower_expert_first(dims, rows):
+    """The tensor-core router of the token-tile paths: experts 2i and 2i+1
+    share one router row, so their logits are equal bit for bit.  Equal
+    logits keep ascending expert order even when a larger logit is inserted
+    above them later: where 2i+1 is chosen, 2i is chosen just before it with
+    the same weight."""
+    seed = 32
+    rw, g, _ = mi.make_router(dims, seed)
+    rw[1::2] = rw[0::2]
+    x = mi.make_x(dims, rows, seed=seed, stream=rows)
+    logits, _, _, _ = oracle.router_topk(dims, x, rw, g)
+    layer = mi.make_layer(dims, seed=seed, experts=P.needed_experts(logits, dims.top_k))
+    layer.router_w[1::2] = layer.router_w[0::2]
+    case = P.build_case(dims, rows, seed=seed, layer=layer)
+    for path in (moe.MOE_PATH_PREFILL, moe.MOE_PATH_PREFILL_NARROW):
+        out, idx, w, gs = run(case, path)
+        _, _, ow, ogs = oracle.router_topk(dims, case.x, layer.router_w, layer.shared_gate)
+        P.check_routing(case, idx, w, gs, ow, ogs)
+        P.compare_output(case, out, idx)
+        for t in range(rows):
+            pos = {int(e): i for i, e in enumerate(idx[t])}
+            for e, i in pos.items():
+                if e % 2 == 1:
+                    assert pos.get(e - 1) == i - 1, f"row {t}: expert {e} at {i} without {e - 1} just before it"
+                    assert w[t, i] == w[t, i - 1]
+
+
 def test_auto_path_switch():
     d = mi.TINY
     assert moe.auto_path(d, moe.MOE_AUTO_DECODE_MAX_ROWS) == moe.MOE_PATH_DECODE
