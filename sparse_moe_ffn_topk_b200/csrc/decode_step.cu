@@ -11,7 +11,8 @@
 //
 // Here one CTA per SM (eight consumer warps and a producer warp that keeps a
 // ring of 16 KB shared-memory slots filled by TMA) runs the whole step with
-// one grid-wide barrier:
+// no grid-wide barrier: CTAs wait only for the data they read (tagged
+// logits, per-expert unit counts):
 //
 //   P0  (before the programmatic-dependent-launch wait: weights only)
 //       the producer starts the copies of this CTA's router rows and of its
@@ -19,16 +20,18 @@
 //   P1  x -> shared memory (bf16, and as three e5m2 terms per value with one
 //       power-of-two scale per (row, 128 block): the gate/up MMAs' B
 //       operand); the CTA's router rows (and the gate vector) against bf16 x
-//       in fp32 -> logits in the workspace;                  grid barrier 1
-//   P2  every CTA takes the top-k of every row from the logits (two stages
-//       over all warps; no CTA waits for a designated one), builds the same
+//       in fp32 -> logits in the workspace, each with the call's tag in the
+//       same 8-byte word;
+//   P2  every CTA takes the top-k of every row from the logits as their
+//       tagged words arrive (two stages over all warps; no CTA waits for a
+//       designated one, nor for the others beyond their logits), builds the same
 //       list of distinct experts, and runs its share of gate/up units (32
 //       gate + 32 up rows of one expert) on tcgen05: A = the e4m3 weight rows
 //       from the ring, B = the x terms, fp32 accumulators in tensor memory;
 //       the epilogue writes h = silu(gate) * up to the workspace as eight
 //       e5m2 terms per value (one power of two per 32 values, laid out as
 //       the down MMAs' B registers) and counts the unit for its expert;
-//   P3  no second grid barrier: each down item (one expert, this CTA's one
+//   P3  no grid barrier: each down item (one expert, this CTA's one
 //       or two 8-row output tiles, the full K) waits until its expert's
 //       units are all counted, bulk-copies the expert's h terms, and runs
 //       mma.sync m16n8k32 (A = the weight rows through ldmatrix, B = the h
@@ -150,6 +153,62 @@ __device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const int32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Router logits travel between CTAs as 8-byte words: the fp32 value in the
+// low half and the call's tag in the high half, stored and loaded whole (an
+// aligned 8-byte access is single-copy atomic), so a reader that sees the
+// tag sees the value, with no barrier between writer and reader.  The tag is
+// the call's epoch + 1; words of earlier calls carry smaller tags and a
+// fresh workspace holds zeros.
+__device__ __forceinline__ void st_logit(uint64_t *w, float v, uint32_t tag)
+{
+    const uint64_t x = ((uint64_t)tag << 32) | (uint64_t)__float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(w), "l"(x) : "memory");
+}
+// The value of a logit word once it carries `tag`; false when the wait runs
+// out (t0: the caller's start of waiting).
+__device__ __forceinline__ bool ld_logit(const uint64_t *w, uint32_t tag, uint64_t t0, float &v)
+{
+    uint64_t x;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(x) : "l"(w) : "memory");
+    while ((uint32_t)(x >> 32) != tag) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(x) : "l"(w) : "memory");
+    }
+    v = __uint_as_float((uint32_t)x);
+    return true;
+}
+
+// Top-k of one row of tagged logits (one warp; the layout of topk_select);
+// false in every lane when a wait ran out.
+template <int EPL>
+__device__ bool topk_select_tagged(const uint64_t *lrow, int E, int K, uint32_t tag, uint64_t t0, int32_t *out_idx,
+                                   float *out_w, float *out_gsig)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t v[EPL];
+    int id[EPL];
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane * EPL + i;
+        float l = 0.f;
+        if (e < E && ok) ok = ld_logit(lrow + e, tag, t0, l);
+        v[i] = (e < E) ? topk_key(l) : 0u;
+        id[i] = e;
+    }
+    float z = 0.f;
+    if (ok) ok = ld_logit(lrow + E, tag, t0, z);
+    if (!__all_sync(0xFFFFFFFFu, ok)) return false;
+    topk_select_keys<EPL>(v, id, z, K, out_idx, out_w, out_gsig);
+    return true;
+}
 
 // A bounded wait, taken by lane 0 for the whole warp, for item q in ring
 // slot s: the result is the same in every lane and the warp is converged
@@ -206,8 +265,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
 // A wait that ran out: MOE_ETIMEOUT in the status word, and where this CTA
 // gave up (the first time) in its diagnostic word: kind << 24 | item.
 //   kind 1 router rows, 2 gate/up item (consumer), 3 down item (consumer),
-//   4 producer before grid barrier 2, 5 producer after it, 6 grid barrier 1,
-//   7 grid barrier 2.
+//   4 producer, 6 a router logit (top-k), 8-10 gate/up MMAs and epilogue.
 __device__ __forceinline__ void gave_up(int32_t *counters, int kind, int item)
 {
     set_status(counters, MOE_ETIMEOUT);
@@ -344,10 +402,10 @@ struct StepParams {
     int32_t *topk_idx;  // routing outputs [rows][K], [rows][K], [rows] (written by CTA 0)
     float *topk_w;
     float *gsig;
-    float *logits;      // workspace [rows][ld]
+    uint64_t *lw;       // counters + kCtrStepLogits, [rows][ld]: the router logits as tagged words (column E: the gate)
     unsigned char *hterm;  // workspace [rows * (K + 1)][imax / 32][256]: h as e5m2 terms in the down MMAs' B layout
     float *hsc;            // workspace [rows * (K + 1)][imax / 32]: the power of two of each chunk of terms
-    int32_t *counters;  // workspace counters (grid barrier, exit, status)
+    int32_t *counters;  // workspace counters (epoch, exit count, status, unit counts)
     int rows, H, E, K, I, Is, ld, imax;
     int ns;              // ring slots
     int gu_wp, gu_pieces;               // gate/up: K windows per piece, pieces
@@ -385,7 +443,8 @@ struct StepSmall {
     double inv[kStepMaxRows];               // RMSNorm: 1 / sqrt(mean square + eps) per row
     int32_t n_list;
     int32_t abort;
-    int32_t pad[2];
+    uint32_t epoch;                         // this call's epoch (the logits' tag is epoch + 1)
+    int32_t pad;
 };
 
 __host__ __device__ inline int n_router_rows(int E, int G, int c)
@@ -606,7 +665,7 @@ __device__ __forceinline__ bool wait_expert(const StepParams &p, const StepSmall
     const int e = shared ? 0 : sm.list[li];
     const int de = shared ? 0 : 1 + li;
     const int need = (shared ? p.Is : p.I) / kGuRows;
-    const int32_t *ready = p.counters + kCtrStepReady + de * p.rdy;
+    const int32_t *ready = p.counters + kCtrStepReady + (int)(sm.epoch & 1u) * kStepReadyHalf + de * p.rdy;
     int ok = 1;
     if (lane == 0 && ld_acquire_gpu(ready) < need) {
         const uint64_t t0 = globaltimer_ns();
@@ -861,7 +920,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const int tile0 = first_tile(n8, G, c);
     const int nt = first_tile(n8, G, c + 1) - tile0;
     const bool producer = warp == kStepWarps;
-    int exit_old = -1;  // (thread 0) the grid barrier's exit count before this CTA's
+    int exit_old = -1;  // (thread 0) the count of CTAs that had read the epoch before this one
     volatile int32_t *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -900,7 +959,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     const int p0_count = min(s0.total, p.ns);
     // This CTA's first gate/up unit is the shared expert's and all of its
     // copies are issued in P0: its MMAs go out while the CTA waits at the
-    // grid barrier (they need only x's terms), not after the plan.
+    // other CTAs' logits (they need only x's terms), not after the plan.
     const bool gu_early = s0.n_units_local > 0 && s0.n_router + p.gu_pieces <= p0_count;
     if (producer) {
         if (lane == 0) {
@@ -937,6 +996,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     }
     pdl_wait();  // x and the workspace may be written by the previous kernel
     STEP_T(1);
+    // this call's epoch, written by the previous call's last CTA (its grid has
+    // finished: the PDL wait); the load is not waited on before x's loads
+    const uint32_t ep = threadIdx.x == 0 ? ld_relaxed_gpu_u32(p.counters + kCtrStepEpoch) : 0u;
 
     // ---------------------------------------------------------------- P1
     if (!producer) {
@@ -976,7 +1038,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                     __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)t * H) + ch);
             }
         }
+        if (ct == 0) sm.epoch = ep;
         named_barrier(1, kStepWarps * kWarp);
+        // (thread 0) this CTA has read the epoch: the count's answer is needed
+        // only after P3 (the last CTA to be counted advances the epoch then)
+        if (ct == 0) exit_old = atomic_add_relaxed_gpu(p.counters + kCtrStepExit, 1);
         // x -> three e5m2 terms per value, the B operand of the gate/up
         // products: per (row, 128 block) a power of two puts the block's
         // largest magnitude in [2^14, 2^15), and t1 = e5m2(x'),
@@ -1019,7 +1085,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         }
         fence_proxy_async_smem();  // the tensor cores read the terms through the async proxy
         STEP_T(2);  // x staged
-        // router rows (router items 0 .. n_router-1 in slots 0 ..)
+        // router rows (router items 0 .. n_router-1 in slots 0 ..), each
+        // logit published with this call's tag
+        const uint32_t tag = sm.epoch + 1;
         for (int ri = 0; ri < s0.n_router; ++ri) {
             if (!warp_wait(&full[ri], 0)) {
                 if (lane == 0) {
@@ -1058,44 +1126,24 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                 for (int t = 0; t < kStepMaxRows; ++t) {
                     if (t < rows) {
                         const float v = warp_sum(acc[t]);
-                        if (lane == 0) p.logits[(size_t)t * p.ld + e] = v + ((e < E && p.router_bias) ? p.router_bias[e] : 0.f);
+                        if (lane == 0)
+                            st_logit(p.lw + (size_t)t * p.ld + e, v + ((e < E && p.router_bias) ? p.router_bias[e] : 0.f),
+                                     tag);
                     }
                 }
             }
         }
-        // the per-expert unit counts start at zero (P2 raises them after the
-        // grid barrier)
+        // the unit counts of the next call start at zero: calls alternate
+        // between two sets by epoch, and the call before this one (the
+        // other set's last user) has finished
         if (c == 0) {
-            for (int i = threadIdx.x; i <= rows * K; i += kStepWarps * kWarp) p.counters[kCtrStepReady + i * p.rdy] = 0;
+            int32_t *nxt = p.counters + kCtrStepReady + (int)((sm.epoch + 1u) & 1u) * kStepReadyHalf;
+            for (int i = threadIdx.x; i < kStepReadyHalf; i += kStepWarps * kWarp) nxt[i] = 0;
         }
-        // the logits and the zeros are ordered before thread 0's release
-        // through the CTA barrier (its fence is cumulative)
-        named_barrier(1, kStepWarps * kWarp);
+        named_barrier(1, kStepWarps * kWarp);  // every warp is done with the router rows
         STEP_T(3);  // router rows done
-        if (threadIdx.x == 0) {
-            // the router slots are free again
-            for (int ri = 0; ri < s0.n_router; ++ri) mbar_arrive(&empty[ri]);
-            bool ok = !*abort;
-            if (ok) {
-                // a releasing arrival: cumulative over the CTA's logits and
-                // zeros, which the CTA barrier above ordered before it
-                atomic_add_release_gpu(p.counters + kCtrStepBar, 1);
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_gpu(p.counters + kCtrStepBar) < G) {
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                        gave_up(p.counters, 6, 0);
-                        *abort = 1;
-                        ok = false;
-                        break;
-                    }
-                }
-            }
-            // every CTA has passed the barrier once the exit count is full;
-            // the count's answer is needed only after P3 (the last CTA to
-            // pass resets both for the next call then), so its round trip
-            // stays off the critical path
-            if (ok) exit_old = atomic_add_relaxed_gpu(p.counters + kCtrStepExit, 1);
-        }
+        if (threadIdx.x == 0)
+            for (int ri = 0; ri < s0.n_router; ++ri) mbar_arrive(&empty[ri]);  // the router slots are free again
         if (gu_early && warp >= kIssuer0 && warp < kIssuer0 + kIssuers && lane == 0) {
             // the shared unit's MMAs (buffer 0), as the issuing loop below
             // would issue them; x's terms were fenced for the async proxy and
@@ -1130,48 +1178,74 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             }
             if (ok) umma_commit(&tfull[0]);
         }
-        named_barrier(1, kStepWarps * kWarp);
-        STEP_T(4);  // grid barrier 1 passed
         // ------------------------------------------------------------ P2
         // top-k of every row, in every CTA: in two stages over all warps
         // (the k best of each chunk of 32 experts, then of the chunks'
         // candidates), or one warp per row
         if (warp == 0) STEP_T(12);
         const int nch = (E + kWarp - 1) / kWarp;
+        // Each logit is read once its word carries this call's tag: no CTA
+        // waits for the others beyond the logits it reads.
+        const uint64_t t0 = globaltimer_ns();
         if (!*abort && p.cand2) {
             uint32_t *ckey = reinterpret_cast<uint32_t *>(sbase + p.o_cand);
             int32_t *cid = reinterpret_cast<int32_t *>(ckey + rows * nch * K);
             for (int task = warp; task < rows * nch; task += kStepWarps) {
                 const int t = task / nch, ch = task - t * nch;
-                topk_chunk(p.logits + (size_t)t * p.ld, E, K, ch, ckey + task * K, cid + task * K);
+                const int e = ch * kWarp + lane;
+                float l = 0.f;
+                const bool ok = e >= E || ld_logit(p.lw + (size_t)t * p.ld + e, tag, t0, l);
+                if (!__all_sync(0xFFFFFFFFu, ok)) {
+                    if (lane == 0) {
+                        gave_up(p.counters, 6, task);
+                        *abort = 1;
+                    }
+                    break;
+                }
+                topk_chunk(e < E ? topk_key(l) : 0u, e, K, ckey + task * K, cid + task * K);
             }
             named_barrier(1, kStepWarps * kWarp);
-            if (warp < rows) {
+            if (!*abort && warp < rows) {
+                // the shared-gate logit (column E), by lane 0 for the warp
+                float z = 0.f;
+                int okz = 1;
+                if (lane == 0) okz = ld_logit(p.lw + (size_t)warp * p.ld + E, tag, t0, z) ? 1 : 0;
+                okz = __shfl_sync(0xFFFFFFFFu, okz, 0);
+                z = __shfl_sync(0xFFFFFFFFu, z, 0);
                 const int n = nch * K;
                 const uint32_t *rk = ckey + warp * n;
                 const int32_t *ri = cid + warp * n;
-                const float *lrow = p.logits + (size_t)warp * p.ld;
                 int32_t *oi = sm.idx + warp * K;
                 float *ow = sm.w + warp * K;
                 float *og = sm.gs + warp;
-                if (n <= kWarp) topk_merge<1>(rk, ri, n, lrow, E, K, oi, ow, og);
-                else if (n <= 2 * kWarp) topk_merge<2>(rk, ri, n, lrow, E, K, oi, ow, og);
-                else if (n <= 4 * kWarp) topk_merge<4>(rk, ri, n, lrow, E, K, oi, ow, og);
-                else if (n <= 8 * kWarp) topk_merge<8>(rk, ri, n, lrow, E, K, oi, ow, og);
-                else topk_merge<16>(rk, ri, n, lrow, E, K, oi, ow, og);
+                if (!okz) {
+                    if (lane == 0) {
+                        gave_up(p.counters, 6, rows * nch + warp);
+                        *abort = 1;
+                    }
+                } else if (n <= kWarp) topk_merge<1>(rk, ri, n, z, K, oi, ow, og);
+                else if (n <= 2 * kWarp) topk_merge<2>(rk, ri, n, z, K, oi, ow, og);
+                else if (n <= 4 * kWarp) topk_merge<4>(rk, ri, n, z, K, oi, ow, og);
+                else if (n <= 8 * kWarp) topk_merge<8>(rk, ri, n, z, K, oi, ow, og);
+                else topk_merge<16>(rk, ri, n, z, K, oi, ow, og);
             }
             if (warp == 0) STEP_T(13);
         } else if (!*abort && warp < rows) {
-            const float *lrow = p.logits + (size_t)warp * p.ld;
+            const uint64_t *lrow = p.lw + (size_t)warp * p.ld;
             int32_t *oi = sm.idx + warp * K;
             float *ow = sm.w + warp * K;
             float *og = sm.gs + warp;
-            if (E <= 32) topk_select<1>(lrow, E, K, oi, ow, og);
-            else if (E <= 64) topk_select<2>(lrow, E, K, oi, ow, og);
-            else if (E <= 128) topk_select<4>(lrow, E, K, oi, ow, og);
-            else if (E <= 256) topk_select<8>(lrow, E, K, oi, ow, og);
-            else if (E <= 512) topk_select<16>(lrow, E, K, oi, ow, og);
-            else topk_select<32>(lrow, E, K, oi, ow, og);
+            bool ok;
+            if (E <= 32) ok = topk_select_tagged<1>(lrow, E, K, tag, t0, oi, ow, og);
+            else if (E <= 64) ok = topk_select_tagged<2>(lrow, E, K, tag, t0, oi, ow, og);
+            else if (E <= 128) ok = topk_select_tagged<4>(lrow, E, K, tag, t0, oi, ow, og);
+            else if (E <= 256) ok = topk_select_tagged<8>(lrow, E, K, tag, t0, oi, ow, og);
+            else if (E <= 512) ok = topk_select_tagged<16>(lrow, E, K, tag, t0, oi, ow, og);
+            else ok = topk_select_tagged<32>(lrow, E, K, tag, t0, oi, ow, og);
+            if (!ok && lane == 0) {
+                gave_up(p.counters, 6, warp);
+                *abort = 1;
+            }
             if (warp == 0) STEP_T(13);
         }
         named_barrier(1, kStepWarps * kWarp);
@@ -1524,7 +1598,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
                     // count with acquiring loads
                     const int u = c + l * G, us = p.Is / kGuRows;
                     const int de = u < us ? 0 : 1 + (u - us) / (p.I / kGuRows);
-                    red_release_gpu(p.counters + kCtrStepReady + de * p.rdy, 1);
+                    red_release_gpu(p.counters + kCtrStepReady + (int)(sm.epoch & 1u) * kStepReadyHalf + de * p.rdy, 1);
                     STEP_TL(15);  // (trace) this CTA's last unit counted
                 }
             }
@@ -1552,12 +1626,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     STEP_T(8);  // P3 starts
     down_phase(p, sm, sbase, base, full, empty, tdone, bbars, seq, nt, tile0, rb0, ibm, dsc, ybuf, abort);
     named_barrier(1, kStepWarps * kWarp);  // every down item of the CTA done
-    // (thread 0) the last CTA past grid barrier 1 resets its counters for the
-    // next call; the next launch reaches the barrier only after its PDL wait,
+    // (thread 0) the last CTA to have read the epoch advances it and resets
+    // the count for the next call, which reads both only after its PDL wait,
     // that is after this grid has finished
     if (threadIdx.x == 0 && exit_old == G - 1) {
-        p.counters[kCtrStepBar] = 0;
         p.counters[kCtrStepExit] = 0;
+        p.counters[kCtrStepEpoch] = (int32_t)(sm.epoch + 1u);
     }
     if (*abort) return;
 
@@ -1683,7 +1757,7 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     const int umax = std::min(d.n_experts, rows * K);
     // the down experts' unit counters, one 128-byte line each where they fit
     s.rdy = 32;
-    while (s.rdy > 1 && kCtrStepReady + (rows * K + 1) * s.rdy > kCtrStepDiag) s.rdy /= 2;
+    while (s.rdy > 1 && (rows * K + 1) * s.rdy > kStepReadyHalf) s.rdy /= 2;
     size_t o = 0;
     auto take = [&](size_t b) { size_t at = o; o = align_up(o + b, 16); return (uint32_t)at; };
     const size_t xBbytes = (size_t)(H / 128) * s.nb * 128;
@@ -1723,7 +1797,7 @@ StepShape step_shape(const moe_dims &d, int rows, int sms)
     const int router_items = (rr_max + s.rr_per_item - 1) / s.rr_per_item;
     s.ok = s.ns >= 2 && s.ns > router_items && s.nt_max <= kMaxNt && s.smem <= kSmemCap && 2 * H <= kSlot &&
            8 * I <= kSlot && 8 * Is <= kSlot && 3 * rows <= 16 && s.tbuf <= 512 && I % kGuRows == 0 &&
-           Is % kGuRows == 0 && kCtrStepReady + (rows * K + 1) * s.rdy <= kCtrStepDiag;
+           Is % kGuRows == 0 && (rows * K + 1) * s.rdy <= kStepReadyHalf;
     return s;
 }
 
@@ -1768,7 +1842,7 @@ cudaError_t launch_decode_step(const StepLaunch &a, cudaStream_t st)
     p.topk_idx = a.topk_idx;
     p.topk_w = a.topk_w;
     p.gsig = a.gsig;
-    p.logits = a.logits;
+    p.lw = reinterpret_cast<uint64_t *>(a.counters + kCtrStepLogits);
     p.hterm = a.hterm;
     p.hsc = a.hsc;
     p.counters = a.counters;

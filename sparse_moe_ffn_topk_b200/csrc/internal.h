@@ -11,21 +11,27 @@ namespace moe {
 
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
-constexpr int kCounters = 4096;         // int32 counters at the head of the workspace
+constexpr int kStepMaxRows = 4;           // decode step kernel: rows per launch; more rows run as several launches
+constexpr int kStepMaxLd = (kMaxExperts + 1 + 3) / 4 * 4;  // router logits a row (E + 1, in fours), at most
 constexpr int kCtrRouter = 0;           // last-arriver counter over the router's token groups
 constexpr int kCtrStatus = 1;           // device status word: 0, or a MOE_* error a kernel recorded
 constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per token-group counters
 constexpr int kMaxRouterGroups = 1024;
-constexpr int kCtrStepBar = 8;          // decode step kernel: grid-barrier arrivals
-constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs past the grid barrier
-constexpr int kCtrStepReady = 16;       // decode step kernel: per down expert (shared, then the routed list), units done,
-                                        // a stride of StepShape::rdy ints apart
-constexpr int kCtrStepDiag = 2048;      // decode step kernel: per CTA, where a wait ran out (0: none)
+constexpr int kCtrStepEpoch = 8;        // decode step kernel: calls so far (the logits' tag is epoch + 1)
+constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs of the running call that have read the epoch
+constexpr int kCtrStepReady = 16;       // decode step kernel: two sets (by epoch parity) of kStepReadyHalf ints: per
+                                        // down expert (shared, then the routed list), units done, StepShape::rdy apart
+constexpr int kCtrStepDiag = 2048;      // decode step kernel: per CTA, where a wait ran out (0: none); the trace
+                                        // build's marks reach 2048 + 256 + 16 * CTAs
+constexpr int kStepReadyHalf = (kCtrStepDiag - kCtrStepReady) / 2;
+constexpr int kCtrStepLogits = 6144;    // decode step kernel: the router logits as tagged 8-byte words [rows][ld]: a
+                                        // fixed place that only these words and zeros ever occupy
+constexpr int kCounters = kCtrStepLogits + 2 * kStepMaxRows * kStepMaxLd;  // int32 words at the head of the workspace
+static_assert(kCtrStepLogits % 2 == 0, "the tagged logits are 8-byte words");
 constexpr int kMaxBlendBlocks = 2048;   // H / 8 limit
 constexpr int kSmallRouterRows = 64;    // the grouped-GEMM path routes up to this many rows with the router kernel
 
 // The decode step kernel (decode_step.cu).
-constexpr int kStepMaxRows = 4;           // rows per launch; more rows run as several launches
 constexpr int kStepWarps = 8;             // consumer warps; plus one producer warp
 constexpr int kStepThreads = (kStepWarps + 1) * 32;
 constexpr int kStepMaxExpertsPerItem = 2; // down experts per ring item
@@ -49,7 +55,7 @@ inline DecodeLayout decode_layout(const moe_dims &d, int64_t rows)
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
     L.ld = (int)((E + 1 + 3) / 4 * 4);
     L.counters = take(sizeof(int32_t) * kCounters);
-    L.logits = take(sizeof(float) * rows * L.ld);
+    L.logits = take(sizeof(float) * rows * L.ld);  // the router kernel's (the decode step's are in the counters)
     L.topk_idx = take(sizeof(int32_t) * rows * K);
     L.topk_w = take(sizeof(float) * rows * K);
     L.gsig = take(sizeof(float) * rows);

@@ -71,6 +71,19 @@ __device__ __forceinline__ void topk_finish(int K, int my_e, uint32_t my_k, floa
     if (lane == 0) *out_gsig = sigmoidf_(z);
 }
 
+// Top-k of one row from its keys (one warp): lane L holds the keys of the
+// experts L*EPL .. L*EPL+EPL-1 in v (0 for absent ones) and their ids, z is
+// the shared-gate logit.
+template <int EPL>
+__device__ __forceinline__ void topk_select_keys(uint32_t (&v)[EPL], int (&id)[EPL], float z, int K,
+                                                 int32_t *out_idx, float *out_w, float *out_gsig)
+{
+    int my_e;
+    uint32_t my_k;
+    topk_rounds<EPL>(v, id, K, my_e, my_k);
+    topk_finish(K, my_e, my_k, z, out_idx, out_w, out_gsig);
+}
+
 // Top-k of one row of logits (one warp): lane L holds the experts
 // L*EPL .. L*EPL+EPL-1.  A NaN logit gets key 1, so the selection always
 // returns valid experts.
@@ -88,10 +101,7 @@ __device__ void topk_select(const float *lrow, int E, int K, int32_t *out_idx, f
         id[i] = e;
     }
     const float z = __ldcg(lrow + E);
-    int my_e;
-    uint32_t my_k;
-    topk_rounds<EPL>(v, id, K, my_e, my_k);
-    topk_finish(K, my_e, my_k, z, out_idx, out_w, out_gsig);
+    topk_select_keys<EPL>(v, id, z, K, out_idx, out_w, out_gsig);
 }
 
 // Two-stage top-k for a CTA's warps.  Stage 1 (one warp per chunk of 32
@@ -101,11 +111,12 @@ __device__ void topk_select(const float *lrow, int E, int K, int32_t *out_idx, f
 // through both stages (a chunk's candidates of equal key come out by lane,
 // and lower chunks hold lower experts), so the result is the one-warp
 // selection's.
-__device__ __forceinline__ void topk_chunk(const float *lrow, int E, int K, int ch, uint32_t *ckey, int32_t *cid)
+//
+// Stage 1 for one chunk: lane L holds the key of expert e = chunk * 32 + L
+// (0 when absent).
+__device__ __forceinline__ void topk_chunk(uint32_t key, int e, int K, uint32_t *ckey, int32_t *cid)
 {
     const int lane = threadIdx.x & 31;
-    const int e = ch * kWarp + lane;
-    uint32_t key = (e < E) ? topk_key(__ldcg(lrow + e)) : 0u;
     for (int r = 0; r < K; ++r) {
         const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, key);
         const int wl = __ffs(__ballot_sync(0xFFFFFFFFu, key == kmax)) - 1;
@@ -118,10 +129,10 @@ __device__ __forceinline__ void topk_chunk(const float *lrow, int E, int K, int 
 }
 
 // Stage 2 over n = chunks * k candidates: lane L takes candidates
-// L*CPL .. L*CPL+CPL-1 (n <= 32 * CPL).
+// L*CPL .. L*CPL+CPL-1 (n <= 32 * CPL); z is the shared-gate logit.
 template <int CPL>
-__device__ void topk_merge(const uint32_t *ckey, const int32_t *cid, int n, const float *lrow, int E, int K,
-                           int32_t *out_idx, float *out_w, float *out_gsig)
+__device__ void topk_merge(const uint32_t *ckey, const int32_t *cid, int n, float z, int K, int32_t *out_idx,
+                           float *out_w, float *out_gsig)
 {
     const int lane = threadIdx.x & 31;
     uint32_t v[CPL];
@@ -132,11 +143,7 @@ __device__ void topk_merge(const uint32_t *ckey, const int32_t *cid, int n, cons
         v[i] = c < n ? ckey[c] : 0u;
         id[i] = c < n ? cid[c] : 0;
     }
-    const float z = __ldcg(lrow + E);
-    int my_e;
-    uint32_t my_k;
-    topk_rounds<CPL>(v, id, K, my_e, my_k);
-    topk_finish(K, my_e, my_k, z, out_idx, out_w, out_gsig);
+    topk_select_keys<CPL>(v, id, z, K, out_idx, out_w, out_gsig);
 }
 
 }  // namespace moe

@@ -29,7 +29,6 @@ POINTS = [
     (1, "PDL wait passed"),
     (2, "x staged"),
     (3, "router rows done"),
-    (4, "grid barrier 1 passed"),
     (12, "top-k started"),
     (13, "top-k done"),
     (14, "distinct-expert list done"),
