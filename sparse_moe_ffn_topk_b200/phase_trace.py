@@ -28,7 +28,7 @@ POINTS = [
     (0, "kernel start"),
     (1, "PDL wait passed"),
     (2, "x staged"),
-    (3, "router rows done"),
+    (3, "router rows done (this CTA's logits published)"),
     (12, "top-k started"),
     (13, "top-k done"),
     (14, "distinct-expert list done"),
