@@ -15,7 +15,6 @@ constexpr int kStepMaxRows = 4;           // decode step kernel: rows per launch
 constexpr int kStepMaxLd = (kMaxExperts + 1 + 3) / 4 * 4;  // router logits a row (E + 1, in fours), at most
 constexpr int kCtrRouter = 0;           // last-arriver counter over the router's token groups
 constexpr int kCtrStatus = 1;           // device status word: 0, or a MOE_* error a kernel recorded
-constexpr int kCtrRouterGroup = 16;     // [16, 16 + kMaxRouterGroups): per token-group counters
 constexpr int kMaxRouterGroups = 1024;
 constexpr int kCtrStepEpoch = 8;        // decode step kernel: calls so far (the logits' tag is epoch + 1)
 constexpr int kCtrStepExit = 9;         // decode step kernel: CTAs of the running call that have read the epoch
@@ -26,8 +25,11 @@ constexpr int kCtrStepDiag = 2048;      // decode step kernel: per CTA, where a 
 constexpr int kStepReadyHalf = (kCtrStepDiag - kCtrStepReady) / 2;
 constexpr int kCtrStepLogits = 6144;    // decode step kernel: the router logits as tagged 8-byte words [rows][ld]: a
                                         // fixed place that only these words and zeros ever occupy
-constexpr int kCounters = kCtrStepLogits + 2 * kStepMaxRows * kStepMaxLd;  // int32 words at the head of the workspace
+constexpr int kCtrRouterGroup = kCtrStepLogits + 2 * kStepMaxRows * kStepMaxLd;  // router kernel: per token group, the
+                                        // CTAs done (a range of its own: the decode step leaves its unit counts set)
+constexpr int kCounters = kCtrRouterGroup + kMaxRouterGroups;  // int32 words at the head of the workspace
 static_assert(kCtrStepLogits % 2 == 0, "the tagged logits are 8-byte words");
+static_assert(kCtrStepDiag + 256 + 16 * 236 <= kCtrStepLogits, "the trace build's marks stay below the tagged logits");
 constexpr int kMaxBlendBlocks = 2048;   // H / 8 limit
 constexpr int kSmallRouterRows = 64;    // the grouped-GEMM path routes up to this many rows with the router kernel
 

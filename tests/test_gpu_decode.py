@@ -202,3 +202,49 @@ def test_router_topk_entry_point(dims, rows):
     torch.cuda.synchronize()
     case = P.Case(dims, None, x, logits)
     P.check_routing(case, idx.cpu().numpy(), w.cpu().numpy(), gs.cpu().numpy(), ow, ogs)
+
+
+def test_paths_in_turn_on_one_workspace(layer35, dev35):
+    """Decode steps, the router-only entry and the grouped path (its router
+    kernel below 64 rows) called in turn on one workspace give, bit for bit,
+    what each gives on a fresh workspace: the decode step leaves its
+    per-expert unit counts set between calls, and the router kernel's
+    token-group counts must not start from them."""
+    d = mi.QWEN36_35B_A3B
+    c1 = P.build_case(d, 1, layer=layer35)
+    c8 = P.build_case(d, 8, layer=layer35)
+    x1, x8 = P.bf16_tensor(c1.x), P.bf16_tensor(c8.x)
+
+    def decode(ws):
+        out = torch.empty(1, d.hidden, dtype=torch.bfloat16, device="cuda")
+        moe.ffn_forward_path(d, x1, dev35["router_w"], dev35["expert_w8"], dev35["expert_scales"],
+                             dev35["shared_w8"], dev35["shared_scales"], dev35["shared_gate"], out, ws,
+                             path=moe.MOE_PATH_DECODE)
+        return out
+
+    def route(ws):
+        idx = torch.empty(8, d.top_k, dtype=torch.int32, device="cuda")
+        w = torch.empty(8, d.top_k, dtype=torch.float32, device="cuda")
+        gs = torch.empty(8, dtype=torch.float32, device="cuda")
+        moe.router_topk(d, x8, dev35["router_w"], dev35["shared_gate"], idx, w, gs, ws)
+        return idx, w
+
+    def narrow(ws):
+        out = torch.empty(8, d.hidden, dtype=torch.bfloat16, device="cuda")
+        moe.ffn_forward_path(d, x8, dev35["router_w"], dev35["expert_w8"], dev35["expert_scales"],
+                             dev35["shared_w8"], dev35["shared_scales"], dev35["shared_gate"], out, ws,
+                             path=moe.MOE_PATH_PREFILL_NARROW)
+        return out
+
+    ref_d, ref_r, ref_n = decode(moe.alloc_workspace(d, 8)), route(moe.alloc_workspace(d, 8)), \
+        narrow(moe.alloc_workspace(d, 8))
+    ws = moe.alloc_workspace(d, 8)
+    for _ in range(3):  # both parities of the decode step's counter sets
+        got_d = decode(ws)
+        got_r = route(ws)
+        got_n = narrow(ws)
+        torch.cuda.synchronize()
+        assert moe.device_status(ws) == moe.MOE_OK
+        assert torch.equal(got_d, ref_d)
+        assert torch.equal(got_r[0], ref_r[0]) and torch.equal(got_r[1], ref_r[1])
+        assert torch.equal(got_n, ref_n)
