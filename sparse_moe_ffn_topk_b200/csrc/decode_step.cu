@@ -121,12 +121,6 @@ __device__ __forceinline__ int block_shift(float amax)
 }
 __device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }
 
-__device__ __forceinline__ int atomic_add_release_gpu(int32_t *p, int v)
-{
-    int old;
-    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
 __device__ __forceinline__ int atomic_add_relaxed_gpu(int32_t *p, int v)
 {
     int old;
