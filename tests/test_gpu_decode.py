@@ -101,6 +101,16 @@ def test_odd_shapes(dims, rows):
     check(case)
 
 
+@pytest.mark.parametrize("rows", [1, 2])
+def test_max_experts_and_top_k(rows):
+    """E = 1024 and k = 32, the most the library takes: the one-warp top-k
+    over tagged logits (the chunk candidates would not fit), and at 2 rows
+    more routed pairs than lanes (the bitmask list of distinct experts)."""
+    d = mi.LayerDims(hidden=256, n_experts=1024, top_k=32, inter=128, shared_inter=128)
+    case = P.build_case(d, rows)
+    check(case)
+
+
 @pytest.mark.parametrize("dims,rows", [
     (mi.LayerDims(hidden=1024, n_experts=256, top_k=8, inter=256, shared_inter=256), 1),   # chunk ranks, ranked merge
     (mi.LayerDims(hidden=1024, n_experts=256, top_k=8, inter=256, shared_inter=256), 3),   # experts shared by rows
